@@ -1,0 +1,224 @@
+/*
+ * ss2d_oracle.c -- float64 CPU oracle for the SS2D forward path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library under selective_scan_ss2d_b200/) never links, loads or
+ * calls it, and it shares no code, header or table with that path.
+ *
+ * What it computes, written out plainly and sequentially in float64:
+ *
+ *   cross_scan   -- "Vision Mamba" (dileepadev tutorial), section "The 2D
+ *                   Challenge: Adapting SSMs to Images", CrossScanModule:
+ *                   four scan orders of an H x W map -- row-major, its
+ *                   reverse, column-major, its reverse.  The same four, in
+ *                   the same stacking order [h, h_inv, v, v_inv], appear in
+ *                   the cross_scan snippet of "VMamba架构解析", section 1.
+ *   selective scan -- "Vision Mamba" (dileepadev), section "Background:
+ *                   State Space Models and Mamba", SelectiveSSM: A is
+ *                   -exp(A_log); dt = softplus(projection + bias);
+ *                   dA = exp(dt*A); dB = dt*B (first-order hold);
+ *                   h_t = dA*h_{t-1} + dB*u_t from h = 0;
+ *                   y_t = sum_n C_t[n] h_t[n] + D*u_t.
+ *                   The recurrence itself is the discrete system of
+ *                   "Vision Mamba: Efficient Visual Representation Learning
+ *                   with Bidirectional State Space Model" (aipaper.cc
+ *                   summary), section 4.1.
+ *   cross_merge  -- same CrossScanModule: each direction's output is mapped
+ *                   back to pixel order; the tutorial's prose says the four
+ *                   are summed.  Summation is in the fixed order k=0,1,2,3.
+ *   1D variant   -- Vim block ("Vision Mamba ..." summary, section 4.3):
+ *                   a forward scan and a scan of the reversed sequence, the
+ *                   reversed output flipped back, the two added.
+ *
+ * Readings taken where the pages are open (each is listed in the design
+ * notes of the repository):
+ *   - B-bar is the first-order dt*B of the tutorial's listing; the ZOH form
+ *     of section 4.1 is available here only as a check (bbar = 1).
+ *   - softplus(z) = log(1 + exp(z)), evaluated as z + log1p(exp(-z)) for
+ *     z > 0 so that it never overflows; this is the same number.
+ *   - Parameters A_log, Dskip and delta_bias are per direction: row k*D+d.
+ *   - delta, Bs and Cs are given in each direction's own scan order.
+ *   - The column-major order of an H x W map visits l = w*H + h.
+ *
+ * Layouts (all contiguous, row-major):
+ *   x          (B, D, H, W)      or u (B, D, L) for the 1D variant
+ *   delta      (B, K, D, L)      scan order of direction k
+ *   Bs, Cs     (B, K, N, L)      scan order of direction k
+ *   A_log      (K*D, N)
+ *   Dskip      (K*D)
+ *   delta_bias (K*D)
+ *   y          (B, D, H, W)  / (B, D, L), overwritten
+ *   y_dir      optional (B, K, D, L): direction k's output in PIXEL order
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* softplus(z) = log(1 + e^z).  For z > 0 the identity
+ * log(1 + e^z) = z + log(1 + e^-z) keeps exp() from overflowing. */
+double oracle_softplus(double z)
+{
+    if (z > 0.0)
+        return z + log1p(exp(-z));
+    return log1p(exp(z));
+}
+
+/* Scan order of direction k over an H x W map: the pixel p = h*W + w that
+ * is visited at step l.
+ *   k = 0  row-major              p = l
+ *   k = 1  reversed row-major     p = L-1-l
+ *   k = 2  column-major           l = w*H + h  ->  p = (l % H)*W + l / H
+ *   k = 3  reversed column-major  the k = 2 pixel of step L-1-l
+ * For the 1D variant (mode 1) only k = 0 (p = l) and k = 1 (p = L-1-l). */
+int64_t oracle_scan_pixel(int mode, int k, int64_t l, int H, int W)
+{
+    const int64_t L = (int64_t)H * W;
+    if (mode == 1 || k < 2)
+        return (k % 2 == 0) ? l : (L - 1 - l);
+    if (k == 3)
+        l = L - 1 - l;
+    const int64_t h = l % H;
+    const int64_t w = l / H;
+    return h * W + w;
+}
+
+/* One channel of one direction: the recurrence over l in scan order.
+ *   u_pix      the channel's input in pixel order (length L)
+ *   delta_seq  (L) raw delta in scan order
+ *   B_dir,C_dir  (N, L) for this (b, k), scan order
+ *   y_pix      output in pixel order (length L), overwritten
+ * bbar = 0: dB = dt*B (the path).  bbar = 1: zero-order hold
+ * dB = (exp(dt*A) - 1)/A * B (check only; A = 0 gives dt*B). */
+static void scan_channel(int mode, int k, int H, int W, int N,
+                         const double *u_pix, const double *delta_seq,
+                         const double *A_log_row, const double *B_dir,
+                         const double *C_dir, double Dskip, double dbias,
+                         int bbar, double *h, double *y_pix)
+{
+    const int64_t L = (int64_t)H * W;
+    for (int n = 0; n < N; ++n)
+        h[n] = 0.0;
+    for (int64_t l = 0; l < L; ++l) {
+        const int64_t p = oracle_scan_pixel(mode, k, l, H, W);
+        const double u = u_pix[p];
+        const double dt = oracle_softplus(delta_seq[l] + dbias);
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) {
+            const double A = -exp(A_log_row[n]);
+            const double dA = exp(dt * A);
+            const double Bv = B_dir[(int64_t)n * L + l];
+            double dB;
+            if (bbar == 0 || A == 0.0)
+                dB = dt * Bv;
+            else
+                dB = expm1(dt * A) / A * Bv;
+            h[n] = dA * h[n] + dB * u;
+            acc += C_dir[(int64_t)n * L + l] * h[n];
+        }
+        y_pix[p] = acc + Dskip * u;
+    }
+}
+
+/* Shared driver for the 2D (mode 0, map H x W) and 1D (mode 1, H = 1,
+ * W = L) forward passes.  Channels (b, d) are independent; each one runs
+ * its K directions in order k = 0..K-1 and adds them into y in that fixed
+ * order, so y = ((Y0 + Y1) + Y2) + Y3 exactly as written. */
+static int forward_impl(int mode, const double *x, const double *delta,
+                        const double *A_log, const double *Bs,
+                        const double *Cs, const double *Dskip,
+                        const double *delta_bias, double *y, double *y_dir,
+                        int B, int D, int H, int W, int N, int K, int bbar,
+                        int nthreads)
+{
+    if (!x || !delta || !A_log || !Bs || !Cs || !Dskip || !delta_bias || !y)
+        return -1;
+    if (B < 0 || D < 0 || H < 0 || W < 0 || N < 1 || K < 1)
+        return -2;
+    if (mode == 0 && !(K == 1 || K == 2 || K == 4))
+        return -4;
+    if (mode == 1 && !(K == 1 || K == 2))
+        return -4;
+    const int64_t L = (int64_t)H * W;
+    const int64_t BD = (int64_t)B * D;
+    if (nthreads < 1)
+        nthreads = 1;
+    int status = 0;
+
+#pragma omp parallel num_threads(nthreads)
+    {
+        double *h = (double *)malloc(sizeof(double) * (size_t)N);
+        double *yk = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        if (!h || !yk) {
+#pragma omp atomic write
+            status = -7;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bd = 0; bd < BD; ++bd) {
+                const int64_t b = bd / D, d = bd % D;
+                const double *u_pix = x + bd * L;
+                double *y_pix = y + bd * L;
+                for (int64_t p = 0; p < L; ++p)
+                    y_pix[p] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    const int64_t kd = (int64_t)k * D + d;
+                    const double *dseq = delta + ((b * K + k) * D + d) * L;
+                    const double *Bd = Bs + (b * K + k) * (int64_t)N * L;
+                    const double *Cd = Cs + (b * K + k) * (int64_t)N * L;
+                    scan_channel(mode, k, H, W, N, u_pix, dseq,
+                                 A_log + kd * N, Bd, Cd, Dskip[kd],
+                                 delta_bias[kd], bbar, h, yk);
+                    for (int64_t p = 0; p < L; ++p)
+                        y_pix[p] += yk[p];
+                    if (y_dir) {
+                        double *dst = y_dir + ((b * K + k) * D + d) * L;
+                        memcpy(dst, yk, sizeof(double) * (size_t)L);
+                    }
+                }
+            }
+        }
+        free(h);
+        free(yk);
+    }
+    return status;
+}
+
+/* SS2D forward: cross_scan -> selective scan per direction -> cross_merge.
+ * K in {1, 2, 4}: the first K of the four orders.  Returns 0 on success,
+ * -1 null pointer, -2 bad size, -4 bad K, -7 out of host memory. */
+int oracle_ss2d_forward(const double *x, const double *delta,
+                        const double *A_log, const double *Bs,
+                        const double *Cs, const double *Dskip,
+                        const double *delta_bias, double *y, double *y_dir,
+                        int B, int D, int H, int W, int N, int K, int bbar,
+                        int nthreads)
+{
+    return forward_impl(0, x, delta, A_log, Bs, Cs, Dskip, delta_bias, y,
+                        y_dir, B, D, H, W, N, K, bbar, nthreads);
+}
+
+/* 1D selective scan: K = 1 (forward) or K = 2 (forward + reversed, the
+ * reversed output flipped back and added).  u is (B, D, L). */
+int oracle_selective_scan_fwd(const double *u, const double *delta,
+                              const double *A_log, const double *Bs,
+                              const double *Cs, const double *Dskip,
+                              const double *delta_bias, double *y,
+                              double *y_dir, int B, int D, int L, int N,
+                              int K, int bbar, int nthreads)
+{
+    return forward_impl(1, u, delta, A_log, Bs, Cs, Dskip, delta_bias, y,
+                        y_dir, B, D, 1, L, N, K, bbar, nthreads);
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

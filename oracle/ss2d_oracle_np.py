@@ -1,0 +1,96 @@
+"""NumPy float64 write-up of the SS2D forward path -- TEST INFRASTRUCTURE ONLY.
+
+A second, independent statement of the same definition as ``ss2d_oracle.c``
+(see that file's header for the page passages each step follows).  Here the
+four scan orders are built the way the pages build them -- reshape, flip and
+transpose of the H x W map ("VMamba架构解析", section 1, cross_scan; "Vision
+Mamba" tutorial, CrossScanModule) -- instead of by index arithmetic, and the
+recurrence runs over the scan index with all channels of a direction as one
+array ("Vision Mamba" tutorial, SelectiveSSM._selective_scan).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def softplus(z):
+    """log(1 + e^z), written so that e^z never overflows."""
+    z = np.asarray(z, dtype=np.float64)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
+def scan_orders_2d(H: int, W: int) -> list[np.ndarray]:
+    """Pixel index visited at each scan step for the four SS2D directions,
+    in the stacking order [row-major, its flip, column-major, its flip]."""
+    pix = np.arange(H * W).reshape(H, W)
+    row_major = pix.reshape(-1)
+    col_major = pix.T.reshape(-1)
+    return [row_major, row_major[::-1].copy(), col_major, col_major[::-1].copy()]
+
+
+def scan_orders_1d(L: int) -> list[np.ndarray]:
+    seq = np.arange(L)
+    return [seq, seq[::-1].copy()]
+
+
+def _scan_direction(u_scan, dt, A, Bk, Ck, Dk, bbar):
+    """u_scan, dt: (B, D, L) in scan order; A: (D, N); Bk, Ck: (B, N, L);
+    Dk: (D,).  Returns y in scan order, (B, D, L)."""
+    Bb, D, L = u_scan.shape
+    N = A.shape[1]
+    h = np.zeros((Bb, D, N))
+    y = np.empty((Bb, D, L))
+    for t in range(L):
+        dA = np.exp(dt[:, :, t, None] * A[None, :, :])
+        if bbar == "euler":
+            dB = dt[:, :, t, None] * Bk[:, None, :, t]
+        else:
+            safeA = np.where(A == 0.0, 1.0, A)
+            zoh = np.expm1(dt[:, :, t, None] * A[None]) / safeA[None]
+            zoh = np.where(A[None] == 0.0, dt[:, :, t, None], zoh)
+            dB = zoh * Bk[:, None, :, t]
+        h = dA * h + dB * u_scan[:, :, t, None]
+        y[:, :, t] = (h * Ck[:, None, :, t]).sum(-1) + Dk[None, :] * u_scan[:, :, t]
+    return y
+
+
+def _forward(u_pix, orders, delta, A_log, Bs, Cs, Dskip, delta_bias, K, bbar):
+    Bb, D, L = u_pix.shape
+    y = np.zeros((Bb, D, L))
+    ydirs = np.empty((Bb, K, D, L))
+    for k in range(K):
+        perm = orders[k]
+        rows = slice(k * D, (k + 1) * D)
+        A = -np.exp(A_log[rows])
+        dt = softplus(delta[:, k] + delta_bias[rows][None, :, None])
+        yk_scan = _scan_direction(u_pix[:, :, perm], dt, A, Bs[:, k], Cs[:, k],
+                                  Dskip[rows], bbar)
+        yk_pix = np.empty_like(yk_scan)
+        yk_pix[:, :, perm] = yk_scan
+        ydirs[:, k] = yk_pix
+        y = y + yk_pix
+    return y, ydirs
+
+
+def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, K=4,
+                 bbar="euler", return_dirs=False):
+    x = np.asarray(x, dtype=np.float64)
+    Bb, D, H, W = x.shape
+    y, yd = _forward(x.reshape(Bb, D, H * W), scan_orders_2d(H, W),
+                     np.asarray(delta, np.float64), np.asarray(A_log, np.float64),
+                     np.asarray(Bs, np.float64), np.asarray(Cs, np.float64),
+                     np.asarray(Dskip, np.float64),
+                     np.asarray(delta_bias, np.float64), K, bbar)
+    y = y.reshape(Bb, D, H, W)
+    return (y, yd) if return_dirs else y
+
+
+def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, K=2,
+                       bbar="euler", return_dirs=False):
+    u = np.asarray(u, dtype=np.float64)
+    Bb, D, L = u.shape
+    y, yd = _forward(u, scan_orders_1d(L), np.asarray(delta, np.float64),
+                     np.asarray(A_log, np.float64), np.asarray(Bs, np.float64),
+                     np.asarray(Cs, np.float64), np.asarray(Dskip, np.float64),
+                     np.asarray(delta_bias, np.float64), K, bbar)
+    return (y, yd) if return_dirs else y
