@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Throughput of the SS2D forward path on B200: state updates per second
+(B*K*D*L*N / s) for one workload, plus its fraction of the HBM and exp-unit
+rooflines.
+
+A step is one full forward pass (cross_scan -> selective scan -> cross_merge)
+over one batch of the workload, through the library's C ABI.  Inputs are
+seeded synthetic arrays already resident in HBM; the L2 cache is flushed
+(a write larger than L2) before every timed step, outside the step's events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+  python bench.py --impl reference ...   # the float64 CPU oracle, rank 0
+  python bench.py --report               # one line per workload (not the
+                                         # contract line; for the notes)
+
+Multi-GPU (torchrun): the path has no exchange step, so every rank runs an
+independent replica of the workload (weak scaling, no collective on the data
+path); the barrier and the max-over-ranks time use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("SS2D state updates/s (B·K·D·L·N) and % of HBM roofline, "
+          "VMamba-T stage 1")
+DEFAULT_CONFIG = "vmamba_t_stage1"
+MUFU_EX2_PER_CLK_PER_SM = 16       # exp2 results per clock per SM (MUFU)
+NUM_SMS = 148
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_SM_MAX_MHZ = 1965.0
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from ncu
+# captures recorded under profiles/, keyed by workload; each entry carries
+# the hash of the kernel sources it was taken from, and is reported only
+# while the sources are unchanged.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_scan_ss2d_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", FALLBACK_SM_MAX_MHZ)),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MAX_MHZ, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def _query_once(self):
+        try:
+            r = subprocess.run(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                "--format=csv,noheader,nounits"], capture_output=True,
+                               text=True, timeout=10)
+            return [ln for ln in r.stdout.splitlines() if ln.strip()]
+        except Exception:
+            return []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+        if not self.lines:
+            self.lines = self._query_once()
+        return self.summary()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def build_arrays(cfg, seed, device, pin=False):
+    import numpy as np
+    import torch
+    from selective_scan_ss2d_b200 import workloads as wl
+    inp = wl.make_inputs(cfg, seed=seed)
+    out = {}
+    for name in wl.Inputs.STREAMED + wl.Inputs.PARAMS:
+        a = getattr(inp, name)
+        t = (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+             if a.dtype == np.uint16 else torch.from_numpy(np.ascontiguousarray(a)))
+        if device is None:
+            out[name] = t.pin_memory() if pin else t
+        else:
+            out[name] = t.to(device)
+    return inp, out
+
+
+def cpu_baseline_parallel(cfg, target_s: float, threads: int):
+    """Time the float64 oracle, as it stands, on a bounded sample of the
+    workload: whole output channels (all K directions over the full L), first
+    the channels of batch element 0, then whole batch elements, grown until
+    one call takes about target_s seconds.  The oracle's OpenMP loop spreads
+    the channels over `threads` host cores.  Returns (updates/s, description,
+    seconds)."""
+    import oracle
+    from selective_scan_ss2d_b200 import workloads as wl
+    inp = wl.make_inputs(cfg, seed=0)
+    fn = oracle.ss2d_forward if cfg.kind == "2d" else oracle.selective_scan_fwd
+
+    def run(nb, nd):
+        sub = slice_sample(inp, nb, nd)
+        ff = sub.as_f64()
+        t0 = time.perf_counter()
+        fn(ff["x"], ff["delta"], ff["A_log"], ff["Bs"], ff["Cs"], ff["Dskip"], ff["delta_bias"],
+           K=cfg.K, threads=threads)
+        return time.perf_counter() - t0, sub.cfg.updates
+
+    nb, nd = 1, min(cfg.D, max(threads, 1))
+    dt, upd = run(nb, nd)
+    while dt < target_s and (nd < cfg.D or nb < cfg.B):
+        grow = max(2.0, target_s / max(dt, 1e-3))
+        if nd < cfg.D:
+            nd = min(cfg.D, int(nd * grow))
+        else:
+            nb = min(cfg.B, max(nb + 1, int(nb * grow)))
+        dt, upd = run(nb, nd)
+    desc = (f"batch elements 0..{nb - 1}, channels 0..{nd - 1} of {cfg.D}, all {cfg.K} "
+            f"directions over the full L={cfg.L}: {upd} updates in {dt:.1f} s")
+    return upd / dt, desc, dt
+
+
+def slice_sample(inp, nb, nd):
+    """Batch elements 0..nb-1, channels 0..nd-1 of a workload (pure slicing)."""
+    import numpy as np
+    from selective_scan_ss2d_b200 import workloads as wl
+    cfg = inp.cfg
+    K, D = cfg.K, cfg.D
+    rows = [k * D + d for k in range(K) for d in range(nd)]
+    sub = cfg.with_(name=f"{cfg.name}[b<{nb},d<{nd}]", B=nb, D=nd)
+    return wl.Inputs(sub, np.ascontiguousarray(inp.x[:nb, :nd]),
+                     np.ascontiguousarray(inp.delta[:nb, :, :nd]),
+                     np.ascontiguousarray(inp.Bs[:nb]), np.ascontiguousarray(inp.Cs[:nb]),
+                     np.ascontiguousarray(inp.A_log[rows]),
+                     np.ascontiguousarray(inp.Dskip[rows]),
+                     np.ascontiguousarray(inp.delta_bias[rows]))
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from selective_scan_ss2d_b200 import binding
+    from selective_scan_ss2d_b200 import workloads as wl
+
+    cfg = wl.CONFIGS[args.config]
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    binding.lib()
+    inp, t = build_arrays(cfg, seed=rank, device=dev)
+    fn = binding.ss2d_forward if cfg.kind == "2d" else binding.selective_scan_fwd
+    y = torch.empty(inp.x.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
+    flush = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"], y,
+           variant=args.variant)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+
+    gpu_id = str(getattr(props, "uuid", local_rank))
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.2)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    value = cfg.updates * args.steps * world / (total_ms / 1e3)
+
+    # dominant kernel alone (the per-direction scan; for K = 1 it is the
+    # whole step), same inputs, same flushes, CUDA events on this stream
+    ydir = torch.empty((cfg.B, cfg.K, cfg.D, cfg.L), dtype=torch.float32, device=dev)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    two_d = cfg.kind == "2d"
+    xx = t["x"]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        kev[i][0].record(stream)
+        binding.ss2d_scan_directions(xx, t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"],
+                                     t["delta_bias"], ydir.view((cfg.B, cfg.K, cfg.D, cfg.H,
+                                                                 cfg.W) if two_d else
+                                                                (cfg.B, cfg.K, cfg.D, cfg.L)),
+                                     two_d=two_d, variant=args.variant)
+        kev[i][1].record(stream)
+    torch.cuda.synchronize()
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+
+    result = {"rank_value": value}
+    if rank == 0:
+        peaks = measured_peaks()
+        alg_bytes = cfg.algorithmic_bytes
+        achieved_gbs = alg_bytes / (scan_ms / 1e3) / 1e9
+        exps = cfg.updates + cfg.B * cfg.K * cfg.D * cfg.L
+        mufu_peak = NUM_SMS * MUFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e9
+        achieved_gexp = exps / (scan_ms / 1e3) / 1e9
+        src_hash = kernel_source_hash()
+        tr = NCU_TRAFFIC.get(cfg.name)
+        traffic = tr["bytes"] if tr and tr.get("src") == src_hash else None
+        variant = args.variant if args.variant >= 0 else binding.ss2d_pick_variant(
+            two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K)
+        step_bytes = alg_bytes
+        result["line"] = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "updates/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded N(0,1) inputs, bf16-rounded where the workload is bf16)",
+            "config": {"workload": cfg.name, "B": cfg.B, "D": cfg.D, "H": cfg.H, "W": cfg.W,
+                       "L": cfg.L, "K": cfg.K, "N": cfg.N, "input_dtype": cfg.dtype,
+                       "state_dtype": "f32", "updates_per_step": cfg.updates,
+                       "algorithmic_bytes_per_step": step_bytes,
+                       "kernel_variant": binding.ss2d_variant_name(variant),
+                       "l2": "flushed before every timed step (2x L2 write, outside events)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                         "traffic": traffic,
+                         "kernel": "scan_fwd_kernel",
+                         "kernel_ms": scan_ms,
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"},
+            "roofline_alu": {"bound": "alu", "achieved": achieved_gexp, "peak": mufu_peak,
+                             "unit": "Gexp2/s", "frac": achieved_gexp / mufu_peak,
+                             "note": "MUFU exp2 unit: 16/clk/SM x 148 SMs x max SM clock; "
+                                     "1 exp per state update + 1 per (b,k,d,l) for softplus"},
+            "gpu_launches": args.steps * (1 if cfg.K == 1 else 2),
+        }
+        result["clocks"] = clocks
+    return result
+
+
+def run_e2e(args, cfg_name, local_rank):
+    """Same metric through the C ABI with host (pinned) buffers: every step
+    copies the inputs in, computes, and copies y out, inside the call."""
+    import torch
+    from selective_scan_ss2d_b200 import binding
+    from selective_scan_ss2d_b200 import workloads as wl
+    cfg = wl.CONFIGS[cfg_name]
+    dev = torch.device(f"cuda:{local_rank}")
+    inp, t = build_arrays(cfg, seed=0, device=None, pin=True)
+    y = torch.empty(inp.x.shape, dtype=torch.float32).pin_memory()
+    fn = binding.ss2d_forward if cfg.kind == "2d" else binding.selective_scan_fwd
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(1, min(args.warmup, 3))):
+        fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"], y,
+           stream=stream.cuda_stream, variant=args.variant)
+    n = max(3, min(args.steps, 20))
+    evs = []
+    for _ in range(n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"], y,
+           stream=stream.cuda_stream, variant=args.variant)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    h2d = sum(getattr(inp, nm).nbytes for nm in wl.Inputs.STREAMED + wl.Inputs.PARAMS)
+    d2h = y.numel() * 4
+    return {"value": cfg.updates / (ms / 1e3), "unit": "updates/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
+
+
+def run_reference(args):
+    """The float64 oracle on the host cores: each step is a bounded sample
+    (whole channels of batch element 0) of the workload."""
+    import oracle
+    from selective_scan_ss2d_b200 import workloads as wl
+    cfg = wl.CONFIGS[args.config]
+    threads = oracle.max_threads()
+    # size one step to ~ (budget / (steps + warmup)) seconds of host work
+    budget_s = float(os.environ.get("SS2D_REFERENCE_BUDGET_S", "150"))
+    per_step_s = max(0.5, min(10.0, budget_s / max(1, args.steps + args.warmup)))
+    _, desc, _ = cpu_baseline_parallel(cfg, per_step_s, threads)
+    nb = int(desc.split("batch elements 0..")[1].split(",")[0]) + 1
+    nd = int(desc.split("channels 0..")[1].split(" ")[0]) + 1
+    inp = wl.make_inputs(cfg, seed=0)
+    sub = slice_sample(inp, nb, nd)
+    ff = sub.as_f64()
+    fn = oracle.ss2d_forward if cfg.kind == "2d" else oracle.selective_scan_fwd
+
+    def step():
+        fn(ff["x"], ff["delta"], ff["A_log"], ff["Bs"], ff["Cs"], ff["Dskip"], ff["delta_bias"],
+           K=cfg.K, threads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    upd = sub.cfg.updates
+    value = upd * args.steps / dt
+    sample = (f"per step: batch elements 0..{nb - 1}, channels 0..{nd - 1} of {cfg.D}, all "
+              f"{cfg.K} directions over the full L={cfg.L} ({upd} updates)")
+    return {
+        "metric": METRIC, "value": value, "unit": "updates/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": cfg.name, "B": cfg.B, "D": cfg.D, "H": cfg.H, "W": cfg.W,
+                   "K": cfg.K, "N": cfg.N, "input_dtype": cfg.dtype},
+        "cpu_baseline": {"value": value, "unit": "updates/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "updates/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--variant", type=int, default=-1)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="host seconds for the oracle sample of cpu_baseline")
+    ap.add_argument("--report", action="store_true",
+                    help="one JSON line per workload (device-resident only)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    if args.report:
+        from selective_scan_ss2d_b200 import workloads as wl
+        for name in wl.CONFIG_ORDER:
+            a = argparse.Namespace(**vars(args))
+            a.config = name
+            r = run_ours(a, rank, world, local_rank)
+            if rank == 0:
+                line = r["line"]
+                line["clocks"] = r.get("clocks")
+                print(json.dumps(line), flush=True)
+        return 0
+
+    r = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        line = r["line"]
+        line["clocks"] = r.get("clocks")
+        if not args.no_e2e:
+            line["e2e"] = run_e2e(args, args.config, local_rank)
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            from selective_scan_ss2d_b200 import workloads as wl
+            cfg = wl.CONFIGS[args.config]
+            threads = oracle.max_threads()
+            v, desc, _ = cpu_baseline_parallel(cfg, args.cpu_seconds, threads)
+            line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": threads,
+                                    "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

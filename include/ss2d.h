@@ -1,0 +1,165 @@
+/*
+ * ss2d.h -- C ABI of the B200 (sm_100a) SS2D forward library.
+ *
+ * The library computes the forward pass of the 2D selective scan (SS2D) used
+ * by VMamba, and the 1D selective scan with one or two directions used by
+ * Vision Mamba (Vim):
+ *
+ *   cross_scan   "Vision Mamba" (dileepadev tutorial), section "The 2D
+ *                Challenge: Adapting SSMs to Images", CrossScanModule; and
+ *                "VMamba架构解析" (mhpn.cn), section 1, cross_scan: an H x W
+ *                map is read in four orders, stacked as
+ *                  k = 0  row-major                     p = l
+ *                  k = 1  row-major reversed            p = L-1-l
+ *                  k = 2  column-major (l = w*H + h)    p = h*W + w
+ *                  k = 3  column-major reversed
+ *                where p = h*W + w is the pixel visited at scan step l.
+ *   selective scan  "Vision Mamba" (dileepadev), section "Background: State
+ *                Space Models and Mamba", SelectiveSSM; the recurrence is the
+ *                discrete system of "Vision Mamba: Efficient Visual
+ *                Representation Learning with Bidirectional State Space
+ *                Model" (aipaper.cc), section 4.1.  Per direction k and
+ *                channel d (row kd = k*D + d of the parameters):
+ *                  A[n]  = -exp(A_log[kd, n])
+ *                  dt_l  = softplus(delta[b,k,d,l] + delta_bias[kd])
+ *                  h_l[n] = exp(dt_l*A[n]) * h_{l-1}[n] + dt_l*Bs[b,k,n,l]*u_l,
+ *                           h_{-1} = 0, state held in float32
+ *                  Y_k[l] = sum_n Cs[b,k,n,l]*h_l[n] + Dskip[kd]*u_l
+ *                with u_l = x[b, d, p(l)].
+ *   cross_merge  same CrossScanModule: each Y_k is put back in pixel order
+ *                and the directions are summed, always in the order
+ *                ((Y_0 + Y_1) + Y_2) + Y_3, so results are deterministic.
+ *   1D variant   Vim block ("Vision Mamba ..." summary, section 4.3): a
+ *                forward scan (k = 0) and a scan of the reversed sequence
+ *                (k = 1, whose output is flipped back), added.
+ *
+ * Memory: every pointer is either a DEVICE pointer (memory of the current
+ * CUDA device, or managed memory) or a HOST pointer; all pointers of one call
+ * must be of the same kind.
+ *   - device pointers: the call is asynchronous on `stream` and returns after
+ *     enqueueing.  Scratch for the per-direction partial outputs (K > 1,
+ *     4*B*K*D*L bytes) is taken from a stream-ordered pool on `stream` and
+ *     returned on `stream`.  Nothing is synchronised.
+ *   - host pointers (pageable or pinned): the call copies the inputs to the
+ *     current device, runs the device path, copies y back and synchronises
+ *     `stream` before returning.  Device buffers come from the same pool.
+ * The caller owns every buffer; the library keeps no pointer after a call.
+ * Inputs are never written.  y must not overlap any input.
+ *
+ * Layouts (contiguous, C order):
+ *   x          (B, D, H, W)   dtype   (u of the 1D call: (B, D, L))
+ *   delta      (B, K, D, L)   dtype   raw delta, in direction k's SCAN order
+ *   Bs, Cs     (B, K, N, L)   dtype   in direction k's SCAN order
+ *   A_log      (K*D, N)       float32
+ *   Dskip      (K*D)          float32
+ *   delta_bias (K*D)          float32
+ *   y          (B, D, H, W) / (B, D, L)  float32, pixel order, overwritten
+ * where L = H*W.  Every pointer must be 16-byte aligned.
+ *
+ * Precision: dtype is the storage type of x, delta, Bs and Cs; all
+ * arithmetic and the state are float32.
+ *
+ * Errors: every entry point returns an ss2d_status; nothing else crosses
+ * the ABI.  A status below zero means nothing was enqueued, except
+ * SS2D_ERR_CUDA, which reports a CUDA error seen while enqueueing or (host
+ * path) while running; ss2d_last_error() then gives CUDA's message for the
+ * calling thread.  Sizes of zero (B, D, H or W) are valid and do nothing.
+ * The functions hold no global mutable state besides the per-thread error
+ * text and are safe to call from several threads.
+ */
+#ifndef SS2D_B200_H
+#define SS2D_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SS2D_OK = 0,
+    SS2D_ERR_NULL = -1,   /* a required pointer is NULL                      */
+    SS2D_ERR_SHAPE = -2,  /* a size is negative, or a product overflows     */
+    SS2D_ERR_DTYPE = -3,  /* dtype is not one of ss2d_dtype                  */
+    SS2D_ERR_K = -4,      /* K not in {1,2,4} (2D) or {1,2} (1D)             */
+    SS2D_ERR_N = -5,      /* N not in 1..16                                  */
+    SS2D_ERR_ALIGN = -6,  /* a pointer is not 16-byte aligned                */
+    SS2D_ERR_ALLOC = -7,  /* device memory for scratch or staging ran out    */
+    SS2D_ERR_CUDA = -8,   /* a CUDA call failed; see ss2d_last_error()       */
+    SS2D_ERR_PTR = -9,    /* host and device pointers mixed in one call      */
+    SS2D_ERR_VARIANT = -10 /* unknown kernel variant (ss2d_forward_ex)       */
+} ss2d_status;
+
+typedef enum {
+    SS2D_F32 = 0,   /* x, delta, Bs, Cs stored as float32  */
+    SS2D_BF16 = 1   /* x, delta, Bs, Cs stored as bfloat16 */
+} ss2d_dtype;
+
+/* SS2D forward: cross_scan -> selective scan of each direction -> cross_merge.
+ * K = 4 is the SS2D of the pages; K = 2 (directions 0 and 1 only) and K = 1
+ * (row-major only) are also accepted.  N in 1..16.  `stream` is a
+ * cudaStream_t (NULL = the legacy default stream). */
+int ss2d_forward(const void *x, const void *delta, const float *A_log,
+                 const void *Bs, const void *Cs, const float *Dskip,
+                 const float *delta_bias, float *y,
+                 int B, int D, int H, int W, int N, int K, int dtype,
+                 void *stream);
+
+/* 1D selective scan, Vim's bidirectional case: u (B, D, L); K = 1 (forward
+ * only) or K = 2 (forward plus the reversed sequence, flipped back, added).
+ * Direction 1 reads u from the end (u[L-1-l] at step l); its delta, Bs and
+ * Cs rows are in that reversed scan order.  Other arguments as ss2d_forward. */
+int selective_scan_fwd(const void *u, const void *delta, const float *A_log,
+                       const void *Bs, const void *Cs, const float *Dskip,
+                       const float *delta_bias, float *y,
+                       int B, int D, int L, int N, int K, int dtype,
+                       void *stream);
+
+/* cross_scan + selective scan WITHOUT cross_merge: writes each direction's
+ * output, in PIXEL order, to y_dir (B, K, D, H, W) float32 (for the 1D call
+ * with two_d = 0: (B, K, D, L), direction 1 flipped back to sequence order).
+ * This is what the tutorial's CrossScanModule concatenates before its output
+ * projection.  Device pointers only (SS2D_ERR_PTR otherwise); asynchronous
+ * on `stream`; no scratch memory.  variant as in ss2d_forward_ex. */
+int ss2d_scan_directions(const void *x, const void *delta, const float *A_log,
+                         const void *Bs, const void *Cs, const float *Dskip,
+                         const float *delta_bias, float *y_dir,
+                         int B, int D, int H, int W, int N, int K, int dtype,
+                         int two_d, void *stream, int variant);
+
+/* As ss2d_forward, with an explicit kernel variant (index into the table
+ * that ss2d_variant_name() describes; -1 = the library's own choice for the
+ * shape).  Every variant computes the same result up to float32 rounding
+ * order; the choice only changes how the work is laid out on the GPU. */
+int ss2d_forward_ex(const void *x, const void *delta, const float *A_log,
+                    const void *Bs, const void *Cs, const float *Dskip,
+                    const float *delta_bias, float *y,
+                    int B, int D, int H, int W, int N, int K, int dtype,
+                    void *stream, int variant);
+
+/* As selective_scan_fwd, with an explicit kernel variant (see above). */
+int selective_scan_fwd_ex(const void *u, const void *delta, const float *A_log,
+                          const void *Bs, const void *Cs, const float *Dskip,
+                          const float *delta_bias, float *y,
+                          int B, int D, int L, int N, int K, int dtype,
+                          void *stream, int variant);
+
+/* Number of kernel variants, and a static description of variant i
+ * ("" for an index out of range). */
+int ss2d_num_variants(void);
+const char *ss2d_variant_name(int i);
+
+/* The variant ss2d_forward / selective_scan_fwd would pick for this shape
+ * (two_d = 1 for ss2d_forward, 0 for the 1D call; H = 1, W = L for 1D). */
+int ss2d_pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
+
+/* Static text for a status code. */
+const char *ss2d_status_string(int status);
+
+/* CUDA's message for the last SS2D_ERR_CUDA / SS2D_ERR_ALLOC seen on the
+ * calling thread ("" if none). */
+const char *ss2d_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS2D_B200_H */

@@ -1,0 +1,207 @@
+"""Thin ctypes binding of the C ABI in include/ss2d.h.
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+library.  Tensors are torch tensors, either all on the current CUDA device
+(asynchronous on the current stream) or all in host memory (the library
+copies in, computes on the current device, copies out and synchronises).
+There is no CPU fallback: if the library is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+
+SS2D_F32 = 0
+SS2D_BF16 = 1
+_DTYPES = {torch.float32: SS2D_F32, torch.bfloat16: SS2D_BF16}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SS2DError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"ss2d status {status}: {message}")
+        self.status = status
+
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib",
+                         "libss2d_b200.so")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _LIB_PATH
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"CUDA library {path} is missing: build it with "
+                    "`python -m selective_scan_ss2d_b200.build`")
+            L = ctypes.CDLL(path)
+            vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+            fwd = [vp, vp, fp, vp, vp, fp, fp, fp]
+            L.ss2d_forward.argtypes = fwd + [i] * 7 + [vp]
+            L.ss2d_forward.restype = i
+            L.ss2d_forward_ex.argtypes = fwd + [i] * 7 + [vp, i]
+            L.ss2d_forward_ex.restype = i
+            L.selective_scan_fwd.argtypes = fwd + [i] * 6 + [vp]
+            L.selective_scan_fwd.restype = i
+            L.selective_scan_fwd_ex.argtypes = fwd + [i] * 6 + [vp, i]
+            L.selective_scan_fwd_ex.restype = i
+            L.ss2d_scan_directions.argtypes = fwd + [i] * 8 + [vp, i]
+            L.ss2d_scan_directions.restype = i
+            L.ss2d_num_variants.argtypes = []
+            L.ss2d_num_variants.restype = i
+            L.ss2d_variant_name.argtypes = [i]
+            L.ss2d_variant_name.restype = ctypes.c_char_p
+            L.ss2d_pick_variant.argtypes = [i] * 7
+            L.ss2d_pick_variant.restype = i
+            L.ss2d_status_string.argtypes = [i]
+            L.ss2d_status_string.restype = ctypes.c_char_p
+            L.ss2d_last_error.argtypes = []
+            L.ss2d_last_error.restype = ctypes.c_char_p
+            _lib = L
+        return _lib
+
+
+def ss2d_status_string(status: int) -> str:
+    return lib().ss2d_status_string(int(status)).decode()
+
+
+def ss2d_num_variants() -> int:
+    return lib().ss2d_num_variants()
+
+
+def ss2d_variant_name(i: int) -> str:
+    return lib().ss2d_variant_name(int(i)).decode()
+
+
+def ss2d_pick_variant(two_d: bool, B: int, D: int, H: int, W: int, N: int, K: int) -> int:
+    return lib().ss2d_pick_variant(int(bool(two_d)), B, D, H, W, N, K)
+
+
+def _check(status: int):
+    if status != 0:
+        L = lib()
+        msg = L.ss2d_status_string(status).decode()
+        detail = L.ss2d_last_error().decode()
+        raise SS2DError(status, msg + (f" -- {detail}" if detail and status in (-7, -8) else ""))
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else ctypes.c_void_p(0)
+
+
+def _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, xdims):
+    streamed = (x, delta, Bs, Cs)
+    dt = x.dtype
+    if dt not in _DTYPES:
+        raise TypeError(f"x must be float32 or bfloat16, got {dt}")
+    for t in streamed:
+        if t.dtype != dt:
+            raise TypeError("x, delta, Bs and Cs must share one dtype")
+    for t in (A_log, Dskip, delta_bias):
+        if t.dtype != torch.float32:
+            raise TypeError("A_log, Dskip and delta_bias must be float32")
+    tensors = list(streamed) + [A_log, Dskip, delta_bias]
+    on_gpu = x.is_cuda
+    for t in tensors:
+        if t.is_cuda != on_gpu or (on_gpu and t.device != x.device):
+            raise ValueError("all tensors must be on the same device (or all on the host)")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+    if y is None:
+        y = torch.empty(xdims, dtype=torch.float32, device=x.device,
+                        pin_memory=(not on_gpu and x.is_pinned()))
+    if y.dtype != torch.float32 or tuple(y.shape) != tuple(xdims) or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous float32 tensor of shape {tuple(xdims)}")
+    if y.is_cuda != on_gpu:
+        raise ValueError("y must live where the inputs live")
+    return y, _DTYPES[dt], on_gpu
+
+
+def _stream(on_gpu, device, stream):
+    if stream is not None:
+        return ctypes.c_void_p(stream if isinstance(stream, int) else stream.cuda_stream)
+    if on_gpu:
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    return ctypes.c_void_p(0)
+
+
+def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y=None, *, stream=None,
+                 variant: int = -1):
+    """SS2D forward (cross_scan -> selective scan -> cross_merge).
+
+    x (B,D,H,W); delta (B,K,D,L) and Bs, Cs (B,K,N,L) in each direction's
+    scan order; A_log (K*D,N), Dskip and delta_bias (K*D,) float32.
+    Returns y (B,D,H,W) float32."""
+    B, D, H, W = x.shape
+    K, N = delta.shape[1], Bs.shape[2]
+    L = H * W
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for ss2d_forward")
+    y, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, (B, D, H, W))
+    st = _stream(on_gpu, x.device, stream)
+    rc = lib().ss2d_forward_ex(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                               _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, H, W, N, K,
+                               dt, st, int(variant))
+    _check(rc)
+    return y
+
+
+def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, y=None, *, stream=None,
+                       variant: int = -1):
+    """1D selective scan, K = 1 (forward) or 2 (forward + reversed, added).
+
+    u (B,D,L); delta (B,K,D,L); Bs, Cs (B,K,N,L) in each direction's scan
+    order.  Returns y (B,D,L) float32."""
+    B, D, L = u.shape
+    K, N = delta.shape[1], Bs.shape[2]
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for selective_scan_fwd")
+    y, dt, on_gpu = _prepare(u, delta, A_log, Bs, Cs, Dskip, delta_bias, y, (B, D, L))
+    st = _stream(on_gpu, u.device, stream)
+    rc = lib().selective_scan_fwd_ex(_ptr(u), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                                     _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, L, N, K,
+                                     dt, st, int(variant))
+    _check(rc)
+    return y
+
+
+def ss2d_scan_directions(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y_dir=None, *,
+                         two_d: bool = True, stream=None, variant: int = -1):
+    """cross_scan + selective scan without the merge: each direction's output
+    in pixel order, (B,K,D,H,W) (2D) or (B,K,D,L) (1D).  CUDA tensors only."""
+    if two_d:
+        B, D, H, W = x.shape
+    else:
+        B, D, L1 = x.shape
+        H, W = 1, L1
+    K, N = delta.shape[1], Bs.shape[2]
+    L = H * W
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for ss2d_scan_directions")
+    odims = (B, K, D, H, W) if two_d else (B, K, D, L)
+    y_dir, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y_dir, odims)
+    st = _stream(on_gpu, x.device, stream)
+    rc = lib().ss2d_scan_directions(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                                    _ptr(Dskip), _ptr(delta_bias), _ptr(y_dir), B, D, H, W,
+                                    N, K, dt, int(bool(two_d)), st, int(variant))
+    _check(rc)
+    return y_dir

@@ -1,0 +1,190 @@
+"""GPU parity: the CUDA library against the float64 oracle on the same seeded
+inputs, through the C ABI (ctypes binding).
+
+Bars: index maps bit-exact (integer-valued inputs); fp32 inputs per element
+|y - y_ref| <= 1e-4 * max(1, |y_ref|); bf16 inputs (fp32 state) relative L2
+<= 1e-3, the oracle reading the same bf16-rounded values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import _gpu
+from selective_scan_ss2d_b200 import binding
+from selective_scan_ss2d_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+NV = None
+
+
+def nvariants():
+    global NV
+    if NV is None:
+        NV = binding.ss2d_num_variants()
+    return NV
+
+
+def small(kind="2d", B=2, D=12, H=7, W=9, K=4, N=16, dtype=wl.F32):
+    if kind == "1d":
+        return wl.Config(f"small1d_{B}_{D}_{W}_{K}_{N}_{dtype}", "1d", B, D, 1, W, K, N, dtype)
+    return wl.Config(f"small2d_{B}_{D}_{H}x{W}_{K}_{N}_{dtype}", "2d", B, D, H, W, K, N, dtype)
+
+
+# ---------------------------------------------------------------------------
+# small shapes: several tiles, ragged tails, every variant
+# ---------------------------------------------------------------------------
+SMALL_2D = [
+    small(),                                        # non-square, L = 63 (ragged)
+    small(B=1, D=8, H=8, W=8, K=4, N=4),            # the tiny config's shape
+    small(B=3, D=37, H=5, W=13, K=4, N=16),         # D not a multiple of any tile
+    small(B=2, D=16, H=16, W=20, K=4, N=8),         # L = 320 (> one chunk)
+    small(B=1, D=8, H=33, W=31, K=4, N=16),         # L = 1023, long ragged chunks
+    small(B=2, D=9, H=6, W=5, K=2, N=5),            # K = 2, odd N
+    small(B=2, D=9, H=6, W=5, K=1, N=1),            # K = 1, N = 1
+]
+SMALL_1D = [
+    small("1d", B=3, D=20, W=197, K=2, N=16),
+    small("1d", B=2, D=7, W=50, K=1, N=3),
+    small("1d", B=1, D=33, W=1000, K=2, N=16),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL_2D + SMALL_1D, ids=lambda c: c.name)
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+def test_small_shapes_all_variants(cfg, dtype):
+    cfg = cfg.with_(dtype=dtype)
+    inp = wl.make_inputs(cfg, seed=1)
+    ref = _gpu.run_oracle(inp)
+    t = _gpu.tensors(inp)
+    for v in [-1] + list(range(nvariants())):
+        y = _gpu.run_gpu(inp, variant=v, t=t)
+        _gpu.assert_close(y, ref, dtype, f"{cfg.name} variant {v}")
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_config(seed):
+    inp = wl.make_inputs("tiny_fp32", seed=seed)
+    y = _gpu.run_gpu(inp)
+    _gpu.assert_close(y, _gpu.run_oracle(inp), wl.F32, "tiny_fp32")
+
+
+# ---------------------------------------------------------------------------
+# index maps: bit-exact with integer-valued inputs
+# ---------------------------------------------------------------------------
+def _running_sum_inputs(cfg, rng):
+    """dt = 32 exactly (softplus(z) = z above 20), A = 0 (A_log = -inf), N = 1,
+    B = 1, C = 1/32: every direction's output is the running sum of the
+    integer inputs along its scan order, exact in float32."""
+    K, D, L = cfg.K, cfg.D, cfg.L
+    xshape = (cfg.B, D, cfg.H, cfg.W) if cfg.kind == "2d" else (cfg.B, D, L)
+    x = rng.integers(-4, 5, size=xshape).astype(np.float32)
+    return wl.Inputs(cfg, x,
+                     np.zeros((cfg.B, K, D, L), np.float32),
+                     np.ones((cfg.B, K, 1, L), np.float32),
+                     np.full((cfg.B, K, 1, L), 1.0 / 32.0, np.float32),
+                     np.full((K * D, 1), -np.inf, np.float32),
+                     np.zeros(K * D, np.float32),
+                     np.full(K * D, 32.0, np.float32))
+
+
+@pytest.mark.parametrize("cfg", [small(B=2, D=5, H=5, W=7, N=1), small(B=1, D=3, H=56, W=56, N=1),
+                                 small(B=1, D=2, H=24, W=40, N=1), small(B=1, D=4, H=7, W=9, K=2, N=1),
+                                 small("1d", B=2, D=5, W=197, K=2, N=1)],
+                         ids=lambda c: c.name)
+def test_index_maps_bit_exact(cfg):
+    rng = np.random.default_rng(5)
+    inp = _running_sum_inputs(cfg, rng)
+    ref = _gpu.run_oracle(inp).astype(np.float32)
+    t = _gpu.tensors(inp)
+    for v in [-1] + list(range(nvariants())):
+        y = _gpu.run_gpu(inp, variant=v, t=t).astype(np.float32)
+        assert np.array_equal(y, ref), f"variant {v}: index maps not bit-exact"
+
+
+def test_identity_scan_is_4x_bit_exact():
+    cfg = small(B=2, D=10, H=9, W=11, N=16)
+    rng = np.random.default_rng(6)
+    inp = wl.make_inputs(cfg, seed=2)
+    inp.x = rng.integers(-100, 101, size=inp.x.shape).astype(np.float32)
+    inp.Bs = np.zeros_like(inp.Bs)
+    y = _gpu.run_gpu(inp).astype(np.float32)
+    assert np.array_equal(y, 4.0 * inp.x)
+
+
+# ---------------------------------------------------------------------------
+# determinism, host-buffer path, errors
+# ---------------------------------------------------------------------------
+def test_deterministic():
+    inp = wl.make_inputs(small(B=2, D=24, H=14, W=14, dtype=wl.BF16), seed=3)
+    t = _gpu.tensors(inp)
+    for v in [-1] + list(range(nvariants())):
+        a = _gpu.run_gpu(inp, variant=v, t=t)
+        b = _gpu.run_gpu(inp, variant=v, t=t)
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("pin", [False, True])
+def test_host_buffers_match_device(pin):
+    inp = wl.make_inputs(small(B=2, D=16, H=10, W=12, dtype=wl.BF16), seed=4)
+    yd = _gpu.run_gpu(inp)
+    th = _gpu.tensors(inp, device=None, pin=pin)
+    yh = binding.ss2d_forward(th["x"], th["delta"], th["A_log"], th["Bs"], th["Cs"],
+                              th["Dskip"], th["delta_bias"])
+    assert not yh.is_cuda
+    assert np.array_equal(yh.numpy().astype(np.float64), yd)
+
+
+def test_mixed_pointers_rejected():
+    inp = wl.make_inputs(small(B=1, D=4, H=4, W=4), seed=0)
+    t = _gpu.tensors(inp)
+    xc = t["x"].cpu()
+    lib = binding.lib()
+    args = [binding._ptr(a) for a in (xc, t["delta"], t["A_log"], t["Bs"], t["Cs"],
+                                      t["Dskip"], t["delta_bias"])]
+    y = torch.empty_like(t["x"], dtype=torch.float32)
+    rc = lib.ss2d_forward(*args, binding._ptr(y), 1, 4, 4, 4, 16, 4, 0, None)
+    assert rc == -9
+
+
+def test_empty_shapes():
+    x = torch.zeros(0, 4, 3, 3, device="cuda")
+    delta = torch.zeros(0, 4, 4, 9, device="cuda")
+    Bs = torch.zeros(0, 4, 16, 9, device="cuda")
+    A_log = torch.zeros(16, 16, device="cuda")
+    Dk = torch.zeros(16, device="cuda")
+    y = binding.ss2d_forward(x, delta, A_log, Bs, Bs, Dk, Dk)
+    assert y.shape == (0, 4, 3, 3)
+
+
+def test_extreme_delta():
+    """softplus saturation and underflow: dt far above 20 and far below."""
+    cfg = small(B=1, D=6, H=5, W=6, N=16)
+    inp = wl.make_inputs(cfg, seed=7)
+    inp.delta = (inp.delta * 30.0).astype(np.float32)
+    _gpu.assert_close(_gpu.run_gpu(inp), _gpu.run_oracle(inp), wl.F32, "extreme delta")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the benchmark times:
+# sampled output channels against the oracle run channel by channel
+# ---------------------------------------------------------------------------
+FULL = ["tiny_fp32", "vmamba_t_stage1", "vmamba_b_stage3", "highres_256", "vim_s_bidir"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_channels(name):
+    cfg = wl.CONFIGS[name]
+    inp = wl.make_inputs(cfg, seed=0)
+    y = _gpu.run_gpu(inp)
+    rng = np.random.default_rng(123)
+    pairs = {(0, 0), (cfg.B - 1, cfg.D - 1)}
+    while len(pairs) < min(8, cfg.B * cfg.D):
+        pairs.add((int(rng.integers(cfg.B)), int(rng.integers(cfg.D))))
+    got, want = [], []
+    for (b, d) in sorted(pairs):
+        sub = wl.channel_subproblem(inp, b, d)
+        want.append(_gpu.run_oracle(sub)[0, 0].reshape(-1))
+        got.append(y[b, d].reshape(-1))
+    _gpu.assert_close(np.concatenate(got), np.concatenate(want), cfg.dtype, name)
