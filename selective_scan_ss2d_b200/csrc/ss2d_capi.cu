@@ -1,6 +1,7 @@
 // ss2d_capi.cu -- the C ABI declared in include/ss2d.h: argument checks,
-// scratch memory, the host-buffer path, and the launch sequence
-// scan (per direction, pixel-order partials) -> merge (fixed-order sum).
+// scratch memory, the host-buffer path, and the launch of the scan kernel
+// (per-direction pixel-order partials, merged in fixed order by the last CTA
+// of each channel tile).
 #include <cuda_runtime.h>
 #include <limits.h>
 #include <stdint.h>
@@ -141,11 +142,9 @@ int check_pointers(const Problem &pr)
     return SS2D_OK;
 }
 
-// Device path: every pointer is device memory of the current device.
-int run_device(const Problem &pr, cudaStream_t st, int variant)
+ss2d::ScanParams make_params(const Problem &pr)
 {
-    const long long L = (long long)pr.H * pr.W;
-    ss2d::ScanParams p;
+    ss2d::ScanParams p{};
     p.x = pr.x;
     p.delta = pr.delta;
     p.A_log = pr.A_log;
@@ -157,17 +156,27 @@ int run_device(const Problem &pr, cudaStream_t st, int variant)
     p.D = pr.D;
     p.H = pr.H;
     p.W = pr.W;
-    p.L = (int)L;
+    p.L = pr.H * pr.W;
     p.N = pr.N;
     p.K = pr.K;
     p.two_d = pr.two_d;
-    const bool bf16 = pr.dtype == SS2D_BF16;
-    const long long DL = (long long)pr.D * L;
+    return p;
+}
 
+// Device path: every pointer is device memory of the current device.
+// K = 1: the scan writes y directly.  K > 1: the scan writes per-direction
+// partials to pool scratch, and the last CTA of each channel tile adds them
+// into y (tickets zeroed here, on the stream, before the launch).
+int run_device(const Problem &pr, cudaStream_t st, int variant)
+{
+    ss2d::ScanParams p = make_params(pr);
+    const bool bf16 = pr.dtype == SS2D_BF16;
+    const long long DL = (long long)pr.D * p.L;
     if (pr.K == 1) {
         p.out = pr.y;
         p.out_b_stride = DL;
         p.out_k_stride = 0;
+        p.merge = 0;
         cudaError_t e = ss2d::launch_scan_variant(variant, bf16, p, st);
         if (e != cudaSuccess) {
             set_error("scan kernel launch", e);
@@ -175,20 +184,27 @@ int run_device(const Problem &pr, cudaStream_t st, int variant)
         }
         return SS2D_OK;
     }
+    const ss2d::VariantInfo *vi = ss2d::variant(variant);
+    const long long tiles = (pr.D + vi->channels_per_cta - 1) / vi->channels_per_cta;
+    const size_t part_bytes = sizeof(float) * (size_t)pr.B * pr.K * DL;
+    const size_t part_up = (part_bytes + 255) & ~(size_t)255;
+    const size_t ticket_bytes = sizeof(unsigned int) * (size_t)pr.B * tiles;
     void *scratch = nullptr;
-    const size_t bytes = sizeof(float) * (size_t)pr.B * pr.K * DL;
-    int rc = pool_alloc(&scratch, bytes, st);
+    int rc = pool_alloc(&scratch, part_up + ticket_bytes, st);
     if (rc != SS2D_OK)
         return rc;
     p.out = static_cast<float *>(scratch);
     p.out_b_stride = (long long)pr.K * DL;
     p.out_k_stride = DL;
-    cudaError_t e = ss2d::launch_scan_variant(variant, bf16, p, st);
+    p.y = pr.y;
+    p.tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(scratch) + part_up);
+    p.merge = 1;
+    cudaError_t e = cudaMemsetAsync(p.tickets, 0, ticket_bytes, st);
     if (e == cudaSuccess)
-        e = ss2d::launch_merge(pr.K, p.out, pr.y, DL, (long long)pr.B * DL, st);
+        e = ss2d::launch_scan_variant(variant, bf16, p, st);
     cudaError_t ef = cudaFreeAsync(scratch, st);
     if (e != cudaSuccess) {
-        set_error("scan/merge kernel launch", e);
+        set_error("scan kernel launch", e);
         return SS2D_ERR_CUDA;
     }
     if (ef != cudaSuccess) {
@@ -201,27 +217,12 @@ int run_device(const Problem &pr, cudaStream_t st, int variant)
 // Per-direction outputs only: the scan kernel writes straight into y_dir.
 int run_directions(const Problem &pr, cudaStream_t st, int variant)
 {
-    const long long L = (long long)pr.H * pr.W;
-    ss2d::ScanParams p;
-    p.x = pr.x;
-    p.delta = pr.delta;
-    p.A_log = pr.A_log;
-    p.Bs = pr.Bs;
-    p.Cs = pr.Cs;
-    p.Dskip = pr.Dskip;
-    p.delta_bias = pr.delta_bias;
-    p.B = pr.B;
-    p.D = pr.D;
-    p.H = pr.H;
-    p.W = pr.W;
-    p.L = (int)L;
-    p.N = pr.N;
-    p.K = pr.K;
-    p.two_d = pr.two_d;
-    const long long DL = (long long)pr.D * L;
+    ss2d::ScanParams p = make_params(pr);
+    const long long DL = (long long)pr.D * p.L;
     p.out = pr.y;
     p.out_b_stride = (long long)pr.K * DL;
     p.out_k_stride = DL;
+    p.merge = 0;
     cudaError_t e = ss2d::launch_scan_variant(variant, pr.dtype == SS2D_BF16, p, st);
     if (e != cudaSuccess) {
         set_error("scan kernel launch", e);

@@ -1,38 +1,49 @@
 // ss2d_kernels.cuh -- sm_100a kernels of the SS2D forward path.
 //
-// One launch of scan_fwd_kernel runs the selective scan of a tile of DC
-// channels of one (batch b, direction k) over the whole sequence, with the
-// cross_scan folded into its address generation and its output written in
-// pixel order.  merge_kernel then adds the K per-direction outputs in the
-// fixed order k = 0, 1, 2, 3 (cross_merge).
+// Recurrence ("Vision Mamba" tutorial, section "Background: State Space
+// Models and Mamba", SelectiveSSM; "Vision Mamba ..." summary, section 4.1),
+// per direction k, channel d and state n:
+//     dt_l = softplus(delta_l + bias)
+//     h_l  = exp(dt_l * A_n) * h_{l-1} + dt_l * B_{n,l} * u_l        (h_{-1} = 0)
+//     y_l  = sum_n C_{n,l} h_l + Dskip * u_l
+// with u_l = x[pixel(k, l)] (cross_scan folded into address generation) and
+// the K outputs put back in pixel order and summed in the fixed order
+// k = 0, 1, 2, 3 (cross_merge).
 //
-// Recurrence ("Vision Mamba" tutorial, SelectiveSSM; "Vision Mamba ..."
-// summary, section 4.1), per channel and state n:
-//     dt_l  = softplus(delta_l + bias)
-//     h_l   = exp(dt_l * A_n) * h_{l-1} + dt_l * B_{n,l} * u_l
-//     y_l   = sum_n C_{n,l} h_l + Dskip * u_l
-// exp(dt*A) is evaluated as 2^(dt * A*log2(e)) on the MUFU unit.
+// Two kernel families share the staging and epilogue code:
 //
-// Work layout.  A CTA owns DC channels of one (b, k) and walks the sequence
-// in chunks of LC = NS * I steps.  Per chunk it stages in shared memory:
-//   * the B and C columns of the chunk, shared by all DC channels, as float32
-//     rows of 16 states (zero padded past N);
-//   * per channel: dt (softplus applied once per (channel, step)), dt*u and
-//     u, gathered through the direction's scan->pixel map.
-// Inside a warp, lanes are (channel cw, time segment jw, state group g):
-// each lane owns S = 16/G states of one channel.  The C.h reduction over the
-// G lanes of a channel is done for four steps at a time with a transposing
-// butterfly (G-1 shuffles per four steps).
+//  * scan_direct_kernel -- one lane per (b, k, d) channel, all 16 states in
+//    registers.  For workloads with many channels (VMamba-B stage 3, Vim).
+//    Each lane loads its own delta and x (prefetched one batch of four steps
+//    ahead) and computes softplus once per step; B and C of a chunk of steps,
+//    shared by every channel of the CTA, are staged in shared memory with a
+//    register prefetch one chunk ahead (double buffer).
 //
-// Long sequences with few channels are split in time: a chunk is cut into
-// NS = J*JW segments of I steps (JW inside a warp, J across warps).  Each
-// lane first runs its segment from a zero state, keeping every exp(dt*A) in
-// registers and accumulating the segment's transfer pair (P, Q) with
-// h_out = P*h_in + Q.  The pairs are combined with the associative operator
-// (P1,Q1) then (P2,Q2) = (P2*P1, P2*Q1 + Q2) -- shuffles inside a warp,
-// shared memory across warps, plus the carry from the previous chunk -- and
-// each lane replays its segment from its true entry state using the kept
-// exponentials, so no exponential is evaluated twice.
+//  * scan_split_kernel -- four lanes per channel (4 states each) and the
+//    sequence split in time, for long sequences with few channels (VMamba-T
+//    stage 1, 256x256 maps).  A chunk of LC steps is cut into NS segments of
+//    I steps (JW segments inside a warp, J warps).  Each lane runs its segment
+//    from a zero state keeping every exp(dt*A) in registers, and accumulates
+//    the segment's transfer pair (P, Q), h_out = P*h_in + Q.  The pairs are
+//    combined with the associative operator (P1,Q1) then (P2,Q2) =
+//    (P2*P1, P2*Q1 + Q2) -- shuffles inside the warp, shared memory across
+//    warps, together with the carry of the previous chunk -- and each lane
+//    replays its segment from its true entry state with the kept
+//    exponentials, so no exponential is evaluated twice.  The raw B, C and
+//    delta rows of the next chunk are copied to shared memory with 16-byte
+//    asynchronous copies (cp.async) while the current chunk computes; a
+//    conversion pass then builds float32 tiles of B|C and of dt (one softplus
+//    per (channel, step)), dt*u and u.
+//
+// Both write each direction's output in pixel order.  With K > 1 they write
+// it to a scratch buffer and the last of the K CTAs that cover the same
+// channels (an atomic ticket per tile, no waiting) adds the K outputs in the
+// fixed order and writes y; so the merge costs no extra launch and reads
+// partials that are still in L2.
+//
+// exp(dt*A) runs on the MUFU unit as 2^(dt * A*log2(e)).  The float32 pair
+// arithmetic uses the sm_100 packed f32x2 instructions (__ffma2_rn,
+// __fmul2_rn), which round each lane exactly as fmaf / a float multiply do.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -53,10 +64,13 @@ struct ScanParams {
     const float *Dskip;      // (K*D)
     const float *delta_bias; // (K*D)
     float *out;              // partials (B,K,D,L) or y (B,D,L), pixel order
+    float *y;                // final y (B,D,L) when the kernel merges (K > 1)
+    unsigned int *tickets;   // one zeroed counter per (b, channel tile) when merging
     int B, D, H, W, L, N, K;
-    int two_d;               // 1: SS2D scan orders; 0: 1D (k=1 reversed)
+    int two_d;               // 1: SS2D scan orders; 0: 1D (k = 1 reversed)
     long long out_b_stride;  // elements between batches in `out`
     long long out_k_stride;  // elements between directions in `out`
+    int merge;               // 1: the last CTA of a tile sums the K partials into y
 };
 
 __device__ __forceinline__ float load_in(const float *p) { return __ldg(p); }
@@ -64,20 +78,9 @@ __device__ __forceinline__ float load_in(const __nv_bfloat16 *p)
 {
     return __bfloat162float(__ldg(p));
 }
-
-// Pixel visited at scan step l of direction k (see include/ss2d.h).
-__device__ __forceinline__ int scan_pixel(int two_d, int k, int l, int H, int W,
-                                          int L)
-{
-    if (k & 1)
-        l = L - 1 - l;
-    if (two_d && k >= 2) {
-        const int h = l % H;
-        const int w = l / H;
-        return h * W + w;
-    }
-    return l;
-}
+// element of a staged (shared-memory) row
+__device__ __forceinline__ float load_in_smem(const float *p) { return *p; }
+__device__ __forceinline__ float load_in_smem(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
 // 2^x on the multi-function unit (PTX ex2.approx.ftz.f32).
 __device__ __forceinline__ float mufu_ex2(float x)
@@ -87,11 +90,23 @@ __device__ __forceinline__ float mufu_ex2(float x)
     return y;
 }
 
-// softplus(z) = log(1 + e^z); above 20 the correction e^-z is below float32
-// resolution of z and z itself is returned.
+// softplus(z) = log(1 + e^z) = max(z, 0) + log1p(e), e = exp(-|z|) in (0, 1].
+// log1p(e) = e * q(e) with q a degree-7 polynomial fitted (Chebyshev nodes,
+// least squares) to log1p(e)/e on [0, 1]; evaluated in float32 its relative
+// error stays below 4e-7 over the whole interval.  Never overflows: for large
+// |z| the correction e underflows to 0.
 __device__ __forceinline__ float softplus_f(float z)
 {
-    return z > 20.f ? z : log1pf(__expf(z));
+    const float e = mufu_ex2(-fabsf(z) * kLog2e);
+    float q = -8.574676205e-03f;
+    q = fmaf(q, e, 4.421419234e-02f);
+    q = fmaf(q, e, -1.078536792e-01f);
+    q = fmaf(q, e, 1.775702399e-01f);
+    q = fmaf(q, e, -2.449961172e-01f);
+    q = fmaf(q, e, 3.327617657e-01f);
+    q = fmaf(q, e, -4.999744938e-01f);
+    q = fmaf(q, e, 9.999998102e-01f);
+    return fmaf(e, q, fmaxf(z, 0.f));
 }
 
 __device__ __forceinline__ float f4(const float4 &v, int i)
@@ -99,118 +114,369 @@ __device__ __forceinline__ float f4(const float4 &v, int i)
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
-// Reduce yp[0..3] (partial sums of four consecutive steps) over the G lanes
-// of a channel and write y = sum + Dskip*u for those steps.  After the
-// butterfly, lane g of the group holds whole sums for 4/G of the steps.
-template <int G>
-__device__ __forceinline__ void reduce_store(float (&yp)[4], float *ydst,
-                                             const float *usrc, float dsk,
-                                             int g)
+// Walks direction k's scan -> pixel map (see include/ss2d.h) one step, or a
+// fixed stride of steps, at a time, without divisions.
+struct PixWalk {
+    int p;      // pixel of the current step (only meaningful while l < L)
+    int h, w;   // row and column, for the column-major directions
+    int mode;   // 0: p = l; 1: p = L-1-l; 2: column-major; 3: reversed column-major
+
+    __device__ __forceinline__ void init(int two_d, int k, int l, int H, int W, int L)
+    {
+        if (!two_d || k < 2) {
+            mode = k & 1;
+            p = (k & 1) ? L - 1 - l : l;
+            h = w = 0;
+        } else {
+            mode = k;
+            const int m = (k == 3) ? L - 1 - l : l;
+            h = m % H;
+            w = m / H;
+            p = h * W + w;
+        }
+    }
+    __device__ __forceinline__ void next(int H, int W)
+    {
+        if (mode == 0) {
+            ++p;
+        } else if (mode == 1) {
+            --p;
+        } else if (mode == 2) {
+            if (++h == H) {
+                h = 0;
+                ++w;
+                p = w;
+            } else {
+                p += W;
+            }
+        } else {
+            if (--h < 0) {
+                h = H - 1;
+                --w;
+                p = h * W + w;
+            } else {
+                p -= W;
+            }
+        }
+    }
+    // advance by n = nq*H + nr steps (nq = n / H, nr = n % H precomputed)
+    __device__ __forceinline__ void advance(int n, int nq, int nr, int H, int W)
+    {
+        if (mode == 0) {
+            p += n;
+        } else if (mode == 1) {
+            p -= n;
+        } else if (mode == 2) {
+            h += nr;
+            w += nq;
+            if (h >= H) {
+                h -= H;
+                ++w;
+            }
+            p = h * W + w;
+        } else {
+            h -= nr;
+            w -= nq;
+            if (h < 0) {
+                h += H;
+                --w;
+            }
+            p = h * W + w;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// cross_merge epilogue: the last of the K CTAs covering channels
+// [d0, d0 + nc) of batch b adds the K pixel-order partials, k = 0..K-1 in
+// order, and writes y.  Called by every thread of the CTA after its partial
+// outputs are written.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void merge_epilogue(const ScanParams &p, int b, int tile, int d0,
+                                               int nc, int nthreads)
 {
-    if constexpr (G == 1) {
-        const float4 u4 = *reinterpret_cast<const float4 *>(usrc);
-        float4 o;
-        o.x = fmaf(dsk, u4.x, yp[0]);
-        o.y = fmaf(dsk, u4.y, yp[1]);
-        o.z = fmaf(dsk, u4.z, yp[2]);
-        o.w = fmaf(dsk, u4.w, yp[3]);
-        *reinterpret_cast<float4 *>(ydst) = o;
-    } else if constexpr (G == 2) {
-        const bool hi = g & 1;
-        const float s0 = hi ? yp[0] : yp[2];
-        const float s1 = hi ? yp[1] : yp[3];
-        float k0 = hi ? yp[2] : yp[0];
-        float k1 = hi ? yp[3] : yp[1];
-        k0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-        k1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-        const int t = 2 * (g & 1);
-        ydst[t] = fmaf(dsk, usrc[t], k0);
-        ydst[t + 1] = fmaf(dsk, usrc[t + 1], k1);
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned int t = atomicAdd(p.tickets + (size_t)b * gridDim.y + tile, 1u);
+        s_last = (t == (unsigned int)(p.K - 1));
+    }
+    __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence();
+    const long long L = p.L;
+    const long long cnt = (long long)nc * L;
+    const float *src = p.out + (size_t)b * p.out_b_stride + (size_t)d0 * L;
+    float *dst = p.y + ((size_t)b * p.D + d0) * L;
+    const long long ks = p.out_k_stride;
+    const bool vec = ((((uintptr_t)src) | ((uintptr_t)dst)) & 15) == 0 && (ks % 4) == 0 &&
+                     (cnt % 4) == 0;
+    if (vec) {
+        for (long long i = (long long)threadIdx.x * 4; i < cnt; i += (long long)nthreads * 4) {
+            float4 acc = __ldcg(reinterpret_cast<const float4 *>(src + i));
+            for (int k = 1; k < p.K; ++k) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + k * ks + i));
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            *reinterpret_cast<float4 *>(dst + i) = acc;
+        }
     } else {
-        static_assert(G == 4, "state groups of 1, 2 or 4 lanes");
-        const bool b1 = (g >> 1) & 1;
-        const float s0 = b1 ? yp[0] : yp[2];
-        const float s1 = b1 ? yp[1] : yp[3];
-        float k0 = b1 ? yp[2] : yp[0];
-        float k1 = b1 ? yp[3] : yp[1];
-        k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-        k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-        const bool b0 = g & 1;
-        const float s = b0 ? k0 : k1;
-        float v = b0 ? k1 : k0;
-        v += __shfl_xor_sync(0xffffffffu, s, 1);
-        ydst[g] = fmaf(dsk, usrc[g], v);
+        for (long long i = threadIdx.x; i < cnt; i += nthreads) {
+            float acc = __ldcg(src + i);
+            for (int k = 1; k < p.K; ++k)
+                acc += __ldcg(src + k * ks + i);
+            dst[i] = acc;
+        }
     }
 }
 
-template <int G, int JW, int J, int WC, int I>
-struct ScanShape {
-    static constexpr int S = kNP / G;          // states per lane
-    static constexpr int CW = 32 / (G * JW);   // channels per warp
-    static constexpr int DC = WC * CW;         // channels per CTA
-    static constexpr int NT = 32 * WC * J;     // threads per CTA
-    static constexpr int NS = J * JW;          // time segments per chunk
-    static constexpr int LC = NS * I;          // steps per chunk
-    static constexpr int SEG = I + 4;          // padded segment, channel rows
-    static constexpr int RS0 = NS * SEG;
-    // channel row stride: an odd number of 16-byte units, so float4 reads of
-    // consecutive channels fall in distinct bank groups
-    static constexpr int RS = RS0 + (((RS0 / 4) % 2 == 0) ? 4 : 8);
-    static constexpr int BSEG = I * kNP + 4;   // padded segment, B/C tiles
-    static constexpr bool SPLIT = NS > 1;
-    static constexpr int TILE_FLOATS = NS * BSEG;       // one of sB, sC
-    static constexpr int ROW_FLOATS = DC * RS;          // one of sDt..sY
-    static constexpr int TOT_FLOATS = (SPLIT && J > 1) ? J * DC * kNP * 2 : 0;
-    static constexpr int CAR_FLOATS = (SPLIT && J > 1) ? 2 * DC * kNP : 0;
-    static constexpr int SMEM_FLOATS =
-        2 * TILE_FLOATS + 4 * ROW_FLOATS + TOT_FLOATS + CAR_FLOATS;
-    static constexpr size_t SMEM_BYTES = sizeof(float) * SMEM_FLOATS;
-    static_assert(I % 4 == 0, "segments hold whole groups of four steps");
-    static_assert(G == 1 || G == 2 || G == 4, "state groups of 1, 2 or 4 lanes");
-    static_assert(32 % (G * JW) == 0 && CW >= 1, "lanes split evenly");
+// ===========================================================================
+// scan_direct_kernel: lane = channel, 16 states per lane
+// ===========================================================================
+template <int WC, int LC>
+struct DirectShape {
+    static constexpr int NT = 32 * WC;       // threads = channels per CTA
+    static constexpr int NE = LC * 8;        // float4 entries of a B|C chunk tile
+    static constexpr int EPT = NE / NT;      // entries staged per thread per chunk
+    static_assert(NE % NT == 0, "whole entries per thread");
+    static_assert(LC % 4 == 0, "steps come in groups of four");
 };
 
-template <typename Tin, int G, int JW, int J, int WC, int I, int MINB>
-__global__ void __launch_bounds__(32 * WC * J, MINB)
-    scan_fwd_kernel(const ScanParams p)
+template <typename Tin, int WC, int LC, int MINB>
+__global__ void __launch_bounds__(32 * WC, MINB) scan_direct_kernel(const ScanParams p)
 {
-    using Sh = ScanShape<G, JW, J, WC, I>;
-    constexpr int S = Sh::S, CW = Sh::CW, DC = Sh::DC, NT = Sh::NT;
-    constexpr int LC = Sh::LC, SEG = Sh::SEG, RS = Sh::RS, BSEG = Sh::BSEG;
-    constexpr bool SPLIT = Sh::SPLIT;
-
-    extern __shared__ float4 smem_f4[];
-    float *sB = reinterpret_cast<float *>(smem_f4);
-    float *sC = sB + Sh::TILE_FLOATS;
-    float *sDt = sC + Sh::TILE_FLOATS;
-    float *sDu = sDt + Sh::ROW_FLOATS;
-    float *sU = sDu + Sh::ROW_FLOATS;
-    float *sY = sU + Sh::ROW_FLOATS;
-    float *sTot = sY + Sh::ROW_FLOATS;   // [J][DC][kNP][2]
-    float *sCar = sTot + Sh::TOT_FLOATS; // [2][DC][kNP]
+    using Sh = DirectShape<WC, LC>;
+    constexpr int NT = Sh::NT, EPT = Sh::EPT;
+    // [buffer][step][B n0-3 | B n4-7 | B n8-11 | B n12-15 | C ... ]
+    __shared__ __align__(16) float4 sBC[2][LC * 8];
 
     const int tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    const int wc = warp % WC, j = warp / WC;
+    const int k = blockIdx.x, tile = blockIdx.y, b = blockIdx.z;
+    const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W;
+    const int d0 = tile * NT;
+    const int d = d0 + tid;
+    const bool cvalid = d < D;
+    const int kd = k * D + (cvalid ? d : 0);
+
+    float2 A2[8];   // A[n] * log2(e) for states (2j, 2j+1)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int n0 = 2 * j, n1 = 2 * j + 1;
+        A2[j].x = (cvalid && n0 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0)) * kLog2e : 0.f;
+        A2[j].y = (cvalid && n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
+    }
+    const float dsk = cvalid ? __ldg(p.Dskip + kd) : 0.f;
+    const float bias = cvalid ? __ldg(p.delta_bias + kd) : 0.f;
+
+    const Tin *xg = static_cast<const Tin *>(p.x) + ((size_t)b * D + (cvalid ? d : 0)) * L;
+    const Tin *dg = static_cast<const Tin *>(p.delta) +
+                    (((size_t)b * p.K + k) * D + (cvalid ? d : 0)) * L;
+    const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * p.K + k) * N * L;
+    const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * p.K + k) * N * L;
+    float *og = p.out + (size_t)b * p.out_b_stride + (size_t)k * p.out_k_stride +
+                (size_t)(cvalid ? d : 0) * L;
+
+    // ---- B/C staging: entry e = (step t = e >> 3, block q = e & 7) ----
+    float raw[EPT][4];
+    auto load_bc = [&](int l0) {
+#pragma unroll
+        for (int r = 0; r < EPT; ++r) {
+            const int e = tid + r * NT;
+            const int q = e & 7, t = e >> 3;
+            const int l = l0 + t;
+            const Tin *src = (q < 4) ? Bg : Cg;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int n = (q & 3) * 4 + i;
+                raw[r][i] = (l < L && n < N) ? load_in(src + (size_t)n * L + l) : 0.f;
+            }
+        }
+    };
+    auto store_bc = [&](int buf) {
+#pragma unroll
+        for (int r = 0; r < EPT; ++r)
+            sBC[buf][tid + r * NT] = make_float4(raw[r][0], raw[r][1], raw[r][2], raw[r][3]);
+    };
+
+    // ---- per-lane delta / x, prefetched one batch of four steps ahead ----
+    PixWalk pw;
+    pw.init(p.two_d, k, 0, H, W, L);
+    float qd[4], qx[4];
+    int qp[4];
+    auto load_batch = [&](int l) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool ok = cvalid && (l + i) < L;
+            qp[i] = pw.p;
+            qd[i] = ok ? load_in(dg + l + i) : 0.f;
+            qx[i] = ok ? load_in(xg + pw.p) : 0.f;
+            pw.next(H, W);
+        }
+    };
+
+    float2 h2[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        h2[j] = make_float2(0.f, 0.f);
+
+    load_bc(0);
+    store_bc(0);
+    load_batch(0);
+    __syncthreads();
+
+    int buf = 0;
+    for (int l0 = 0; l0 < L; l0 += LC, buf ^= 1) {
+        const bool more = l0 + LC < L;
+        if (more)
+            load_bc(l0 + LC);
+        const float4 *sb = sBC[buf];
+#pragma unroll 1
+        for (int t0 = 0; t0 < LC; t0 += 4) {
+            float cd[4], cx[4];
+            int cp[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                cd[i] = qd[i];
+                cx[i] = qx[i];
+                cp[i] = qp[i];
+            }
+            load_batch(l0 + t0 + 4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float dt = softplus_f(cd[i] + bias);
+                const float u = cx[i];
+                const float2 dt2 = make_float2(dt, dt);
+                const float du = dt * u;
+                const float2 du2 = make_float2(du, du);
+                const float4 *row = sb + (t0 + i) * 8;
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 bv = row[q];
+                    const float4 cv = row[4 + q];
+                    const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
+                    const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
+                    const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
+                    const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
+                    h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
+                    h2[2 * q + 1] =
+                        __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
+                    acc = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc);
+                    acc = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc);
+                }
+                const float yv = fmaf(dsk, u, acc.x + acc.y);
+                if (cvalid && l0 + t0 + i < L)
+                    og[cp[i]] = yv;
+            }
+        }
+        if (more)
+            store_bc(buf ^ 1);
+        __syncthreads();
+    }
+    if (p.merge) {
+        const int nc = min(NT, D - d0);
+        merge_epilogue(p, b, tile, d0, nc, NT);
+    }
+}
+
+// ===========================================================================
+// scan_split_kernel: four lanes per channel, sequence split in time
+// ===========================================================================
+// 16-byte asynchronous copy global -> shared (cp.async.cg); with src_bytes = 0
+// nothing is read and the 16 destination bytes are zero-filled.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
+{
+    const unsigned int s = (unsigned int)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+template <typename Tin, int JW, int J, int I>
+struct SplitShape {
+    static constexpr int G = 4;                  // lanes per channel
+    static constexpr int S = kNP / G;            // states per lane (4)
+    static constexpr int CW = 32 / (G * JW);     // channels per warp = per CTA
+    static constexpr int DC = CW;
+    static constexpr int NT = 32 * J;            // threads
+    static constexpr int NS = J * JW;            // time segments per chunk
+    static constexpr int LC = NS * I;            // steps per chunk
+    static constexpr int ESZ = sizeof(Tin);
+    static constexpr int EPP = 16 / ESZ;         // elements per 16-byte piece
+    static constexpr int PPR = LC / EPP;         // pieces per raw row
+    static constexpr int RAWROW = LC + EPP;      // raw row stride in elements (16 B pad)
+    static constexpr int RAW_ROWS = 2 * kNP + DC;        // B rows, C rows, delta rows
+    static constexpr int RAW_ELEMS = RAW_ROWS * RAWROW;  // per raw buffer
+    static constexpr int SEG = I + 4;            // padded segment in channel rows
+    static constexpr int RS0 = NS * SEG;
+    static constexpr int RS = RS0 + (((RS0 / 4) % 2 == 0) ? 4 : 8);   // channel row stride
+    static constexpr int BSEG4 = I * 8 + 4;      // padded segment of the B|C tile (float4)
+    static constexpr int TILE4 = NS * BSEG4;     // float4 in the B|C tile
+    static constexpr int ROWF = DC * RS;         // floats per dt / dt*u / u tile
+    static constexpr int NE = LC * 8;            // B|C float4 entries per chunk
+    static constexpr int NR = DC * LC;           // (channel, step) elements per chunk
+    static constexpr int RPT = (NR + NT - 1) / NT;
+    static constexpr int NPIECE = RAW_ROWS * PPR;        // 16-byte copies per chunk
+    static constexpr size_t RAW_BYTES = (size_t)ESZ * 2 * RAW_ELEMS;
+    static constexpr size_t SMEM_BYTES =
+        RAW_BYTES + sizeof(float4) * TILE4 + sizeof(float) * 3 * ROWF + sizeof(int) * LC +
+        sizeof(float) * (J > 1 ? (J * DC * kNP * 2 + 2 * DC * kNP) : 0);
+    static_assert(I % 4 == 0, "segments hold whole groups of four steps");
+    static_assert(LC % EPP == 0, "chunks are whole 16-byte pieces");
+    static_assert(32 % (G * JW) == 0 && CW >= 1, "lanes split evenly");
+    static_assert((RAW_BYTES % 16) == 0, "raw buffers keep 16-byte alignment");
+};
+
+template <typename Tin, int JW, int J, int I, int MINB>
+__global__ void __launch_bounds__(32 * J, MINB) scan_split_kernel(const ScanParams p)
+{
+    using Sh = SplitShape<Tin, JW, J, I>;
+    constexpr int G = Sh::G, DC = Sh::DC, NT = Sh::NT, LC = Sh::LC;
+    constexpr int SEG = Sh::SEG, RS = Sh::RS, BSEG4 = Sh::BSEG4;
+    constexpr int RPT = Sh::RPT, NE = Sh::NE, NR = Sh::NR;
+    constexpr int EPP = Sh::EPP, PPR = Sh::PPR, RAWROW = Sh::RAWROW;
+
+    extern __shared__ float4 smem_f4[];
+    Tin *sRaw = reinterpret_cast<Tin *>(smem_f4);                   // [2][RAW_ROWS][RAWROW]
+    float4 *sBC = reinterpret_cast<float4 *>(reinterpret_cast<char *>(smem_f4) + Sh::RAW_BYTES);
+    float *sDt = reinterpret_cast<float *>(sBC + Sh::TILE4);        // [DC][RS]
+    float *sDu = sDt + Sh::ROWF;
+    float *sU = sDu + Sh::ROWF;
+    int *sPix = reinterpret_cast<int *>(sU + Sh::ROWF);             // [LC]
+    float *sTot = reinterpret_cast<float *>(sPix + LC);             // [J][DC][kNP][2]
+    float *sCar = sTot + J * DC * kNP * 2;                          // [2][DC][kNP]
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, j = tid >> 5;
     const int g = lane % G;
     const int jw = (lane / G) % JW;
-    const int cw = lane / (G * JW);
-    const int c = wc * CW + cw;
+    const int c = lane / (G * JW);
     const int js = j * JW + jw;
 
     const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W;
-    const int d0 = blockIdx.x * DC;
-    const int k = blockIdx.y, b = blockIdx.z;
+    const int k = blockIdx.x, tile = blockIdx.y, b = blockIdx.z;
+    const int d0 = tile * DC;
     const int d = d0 + c;
     const bool cvalid = d < D;
     const int kd = k * D + (cvalid ? d : 0);
 
-    float A2[S];
+    float2 A2[2];
+    {
+        const int n0 = g * 4;
+        float a[4];
 #pragma unroll
-    for (int s = 0; s < S; ++s) {
-        const int n = g * S + s;
-        A2[s] = (cvalid && n < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n)) * kLog2e
-                                  : 0.f;
+        for (int s = 0; s < 4; ++s)
+            a[s] = (cvalid && n0 + s < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0 + s)) * kLog2e
+                                          : 0.f;
+        A2[0] = make_float2(a[0], a[1]);
+        A2[1] = make_float2(a[2], a[3]);
     }
     const float dsk = cvalid ? __ldg(p.Dskip + kd) : 0.f;
 
@@ -219,261 +485,262 @@ __global__ void __launch_bounds__(32 * WC * J, MINB)
     const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * p.K + k) * N * L;
     const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * p.K + k) * N * L;
     const float *biasg = p.delta_bias + (size_t)k * D;
-    float *og = p.out + (size_t)b * p.out_b_stride + (size_t)k * p.out_k_stride;
+    float *og = p.out + (size_t)b * p.out_b_stride + (size_t)k * p.out_k_stride +
+                (size_t)(cvalid ? d : 0) * L;
+    // rows start on 16-byte boundaries: copy 16-byte pieces asynchronously;
+    // otherwise fall back to element loads
+    const bool async_ok = ((L * (int)sizeof(Tin)) % 16) == 0 &&
+                          (((uintptr_t)p.delta | (uintptr_t)p.Bs | (uintptr_t)p.Cs) & 15) == 0;
 
-    float h[S];      // state entering the current step (direct path)
-    float hcar[S];   // state entering the current chunk (split path, J == 1)
+    // raw row r of a chunk: B rows 0..15, C rows 16..31, delta rows 32..32+DC-1
+    auto row_src = [&](int r) -> const Tin * {
+        if (r < kNP)
+            return r < N ? Bg + (size_t)r * L : nullptr;
+        if (r < 2 * kNP)
+            return (r - kNP) < N ? Cg + (size_t)(r - kNP) * L : nullptr;
+        const int dd = d0 + (r - 2 * kNP);
+        return dd < D ? dg + (size_t)dd * L : nullptr;
+    };
+    auto stage_raw = [&](int rb, int l0) {
+        Tin *dst0 = sRaw + rb * Sh::RAW_ELEMS;
+        if (async_ok) {
+            for (int e = tid; e < Sh::NPIECE; e += NT) {
+                const int r = e / PPR, q = e % PPR;
+                const int l = l0 + q * EPP;
+                const Tin *src = row_src(r);
+                const bool ok = src != nullptr && l < L;
+                cp_async16(dst0 + r * RAWROW + q * EPP, ok ? src + l : p.Bs, ok ? 16 : 0);
+            }
+            cp_async_commit();
+        } else {
+            for (int e = tid; e < Sh::RAW_ROWS * LC; e += NT) {
+                const int r = e / LC, t = e % LC;
+                const int l = l0 + t;
+                const Tin *src = row_src(r);
+                dst0[r * RAWROW + t] = (src != nullptr && l < L) ? src[l] : Tin(0.f);
+            }
+        }
+    };
+
+    // x of a chunk: register prefetch through per-thread pixel walkers;
+    // (channel, step) element e = tid + r*NT: step e % LC, channel e / LC
+    PixWalk rw[RPT];
+    const int nq = LC / H, nr = LC % H;
 #pragma unroll
-    for (int s = 0; s < S; ++s) {
-        h[s] = 0.f;
-        hcar[s] = 0.f;
+    for (int r = 0; r < RPT; ++r)
+        rw[r].init(p.two_d, k, (tid + r * NT) % LC, H, W, L);
+    float rx[RPT];
+    auto load_x = [&](int l0) {
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int e = tid + r * NT;
+            const int t = e % LC, cc = e / LC;
+            const int l = l0 + t, dd = d0 + cc;
+            const bool ok = (e < NR) && l < L && dd < D;
+            rx[r] = ok ? load_in(xg + (size_t)dd * L + rw[r].p) : 0.f;
+        }
+    };
+    // raw chunk -> float32 tiles: B|C as [segment][step][8 float4], dt, dt*u, u
+    // as [channel][segment][step], and the chunk's pixel table
+    auto convert = [&](int rb, int l0) {
+        const Tin *raw = sRaw + rb * Sh::RAW_ELEMS;
+        for (int e = tid; e < NE; e += NT) {
+            const int q = e & 7, t = e >> 3;
+            const Tin *src = raw + ((q < 4 ? 0 : kNP) + (q & 3) * 4) * RAWROW + t;
+            sBC[(t / I) * BSEG4 + (t % I) * 8 + q] =
+                make_float4(load_in_smem(src), load_in_smem(src + RAWROW),
+                            load_in_smem(src + 2 * RAWROW), load_in_smem(src + 3 * RAWROW));
+        }
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int e = tid + r * NT;
+            if (e < NR) {
+                const int t = e % LC, cc = e / LC;
+                const int l = l0 + t, dd = d0 + cc;
+                const bool ok = l < L && dd < D;
+                const float z = load_in_smem(raw + (2 * kNP + cc) * RAWROW + t);
+                const float dt = ok ? softplus_f(z + __ldg(biasg + dd)) : 0.f;
+                const int si = cc * RS + (t / I) * SEG + (t % I);
+                sDt[si] = dt;
+                sDu[si] = dt * rx[r];
+                sU[si] = rx[r];
+                if (cc == 0)
+                    sPix[t] = rw[r].p;
+            }
+            rw[r].advance(LC, nq, nr, H, W);
+        }
+    };
+
+    // zero both raw buffers once, so steps past the end of the sequence read
+    // finite zeros
+    {
+        float4 *z = smem_f4;
+        for (int e = tid; e < (int)(Sh::RAW_BYTES / 16); e += NT)
+            z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if constexpr (SPLIT && J > 1) {
-        for (int e = tid; e < Sh::CAR_FLOATS; e += NT)
+    float2 hcar[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    if constexpr (J > 1) {
+        for (int e = tid; e < 2 * DC * kNP; e += NT)
             sCar[e] = 0.f;
     }
+    __syncthreads();
+    stage_raw(0, 0);
+    load_x(0);
 
-    int chunk = 0;
-    for (int l0 = 0; l0 < L; l0 += LC, ++chunk) {
-        // ---------------- stage the chunk ----------------
-        for (int e = tid; e < LC * (kNP / 4); e += NT) {
-            const int nb = e & 3;
-            const int t = e >> 2;
-            const int l = l0 + t;
-            float vb[4], vc[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int n = nb * 4 + q;
-                const bool ok = (l < L) && (n < N);
-                vb[q] = ok ? load_in(Bg + (size_t)n * L + l) : 0.f;
-                vc[q] = ok ? load_in(Cg + (size_t)n * L + l) : 0.f;
-            }
-            const int off = (t / I) * BSEG + (t % I) * kNP + nb * 4;
-            *reinterpret_cast<float4 *>(sB + off) = make_float4(vb[0], vb[1], vb[2], vb[3]);
-            *reinterpret_cast<float4 *>(sC + off) = make_float4(vc[0], vc[1], vc[2], vc[3]);
-        }
-        for (int e = tid; e < DC * LC; e += NT) {
-            const int t = e % LC;
-            const int cc = e / LC;
-            const int l = l0 + t;
-            const int dd = d0 + cc;
-            float dt = 0.f, du = 0.f, u = 0.f;
-            if (l < L && dd < D) {
-                const int pix = scan_pixel(p.two_d, k, l, H, W, L);
-                u = load_in(xg + (size_t)dd * L + pix);
-                const float z = load_in(dg + (size_t)dd * L + l) + __ldg(biasg + dd);
-                dt = softplus_f(z);
-                du = dt * u;
-            }
-            const int si = cc * RS + (t / I) * SEG + (t % I);
-            sDt[si] = dt;
-            sDu[si] = du;
-            sU[si] = u;
-        }
+    int rb = 0, chunk = 0;
+    for (int l0 = 0; l0 < L; l0 += LC, rb ^= 1, ++chunk) {
+        const bool more = l0 + LC < L;
+        if (async_ok)
+            cp_async_wait_all();
         __syncthreads();
+        convert(rb, l0);
+        __syncthreads();
+        if (more) {
+            stage_raw(rb ^ 1, l0 + LC);
+            load_x(l0 + LC);
+        }
+        const float4 *tb = sBC + js * BSEG4 + g;
+        const float *dtb = sDt + c * RS + js * SEG;
+        const float *dub = sDu + c * RS + js * SEG;
+        const float *ub = sU + c * RS + js * SEG;
 
-        // ---------------- scan the chunk ----------------
-        const int rb0 = c * RS + js * SEG;   // this lane's segment, channel rows
-        const int bb0 = js * BSEG + g * S;   // this lane's segment, B/C tiles
-        if constexpr (!SPLIT) {
-#pragma unroll 1
-            for (int i0 = 0; i0 < I; i0 += 4) {
-                const float4 dt4 = *reinterpret_cast<const float4 *>(sDt + rb0 + i0);
-                const float4 du4 = *reinterpret_cast<const float4 *>(sDu + rb0 + i0);
-                float yp[4];
+        // pass 1: the segment from a zero state; keep exp(dt*A)
+        float2 av[I][2];
+        float2 P[2] = {make_float2(1.f, 1.f), make_float2(1.f, 1.f)};
+        float2 Q[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int tt = 0; tt < 4; ++tt) {
-                    const float dt = f4(dt4, tt), du = f4(du4, tt);
-                    const float *rowB = sB + bb0 + (i0 + tt) * kNP;
-                    const float *rowC = sC + bb0 + (i0 + tt) * kNP;
-                    float acc = 0.f;
+        for (int i0 = 0; i0 < I; i0 += 4) {
+            const float4 dt4 = *reinterpret_cast<const float4 *>(dtb + i0);
+            const float4 du4 = *reinterpret_cast<const float4 *>(dub + i0);
 #pragma unroll
-                    for (int s4 = 0; s4 < S; s4 += 4) {
-                        const float4 bv = *reinterpret_cast<const float4 *>(rowB + s4);
-                        const float4 cv = *reinterpret_cast<const float4 *>(rowC + s4);
+            for (int ii = 0; ii < 4; ++ii) {
+                const int i = i0 + ii;
+                const float dt = f4(dt4, ii), du = f4(du4, ii);
+                const float2 dt2 = make_float2(dt, dt), du2 = make_float2(du, du);
+                const float4 bv = tb[i * 8];
+                const float2 arg0 = __fmul2_rn(dt2, A2[0]);
+                const float2 arg1 = __fmul2_rn(dt2, A2[1]);
+                av[i][0] = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
+                av[i][1] = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
+                Q[0] = __ffma2_rn(av[i][0], Q[0], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
+                Q[1] = __ffma2_rn(av[i][1], Q[1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
+                P[0] = __fmul2_rn(P[0], av[i][0]);
+                P[1] = __fmul2_rn(P[1], av[i][1]);
+            }
+        }
+        // inclusive scan of the transfer pairs over the warp's segments
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int s = s4 + q;
-                            const float a = mufu_ex2(dt * A2[s]);
-                            h[s] = fmaf(a, h[s], du * f4(bv, q));
-                            acc = fmaf(f4(cv, q), h[s], acc);
-                        }
-                    }
-                    yp[tt] = acc;
+        for (int rr = 1; rr < JW; rr <<= 1) {
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                float2 Pp, Qp;
+                Pp.x = __shfl_up_sync(0xffffffffu, P[s].x, rr * G);
+                Pp.y = __shfl_up_sync(0xffffffffu, P[s].y, rr * G);
+                Qp.x = __shfl_up_sync(0xffffffffu, Q[s].x, rr * G);
+                Qp.y = __shfl_up_sync(0xffffffffu, Q[s].y, rr * G);
+                if (jw >= rr) {
+                    Q[s] = __ffma2_rn(P[s], Qp, Q[s]);
+                    P[s] = __fmul2_rn(P[s], Pp);
                 }
-                reduce_store<G>(yp, sY + rb0 + i0, sU + rb0 + i0, dsk, g);
+            }
+        }
+        float2 Pex[2], Qex[2];   // segments of this warp before mine
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            float2 Pp, Qp;
+            Pp.x = __shfl_up_sync(0xffffffffu, P[s].x, G);
+            Pp.y = __shfl_up_sync(0xffffffffu, P[s].y, G);
+            Qp.x = __shfl_up_sync(0xffffffffu, Q[s].x, G);
+            Qp.y = __shfl_up_sync(0xffffffffu, Q[s].y, G);
+            Pex[s] = (jw == 0) ? make_float2(1.f, 1.f) : Pp;
+            Qex[s] = (jw == 0) ? make_float2(0.f, 0.f) : Qp;
+        }
+        float2 hw[2];   // state entering this warp's first segment
+        if constexpr (J == 1) {
+            const int last = (c * JW + JW - 1) * G + g;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                hw[s] = hcar[s];
+                float2 Pt, Qt;
+                Pt.x = __shfl_sync(0xffffffffu, P[s].x, last);
+                Pt.y = __shfl_sync(0xffffffffu, P[s].y, last);
+                Qt.x = __shfl_sync(0xffffffffu, Q[s].x, last);
+                Qt.y = __shfl_sync(0xffffffffu, Q[s].y, last);
+                hcar[s] = __ffma2_rn(Pt, hcar[s], Qt);
             }
         } else {
-            // pass 1: run the segment from a zero state, keep exp(dt*A)
-            float av[I][S];
-            float P[S], Q[S];
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                P[s] = 1.f;
-                Q[s] = 0.f;
+            if (jw == JW - 1) {
+                float4 *dst = reinterpret_cast<float4 *>(sTot + ((j * DC + c) * kNP + g * 4) * 2);
+                dst[0] = make_float4(P[0].x, Q[0].x, P[0].y, Q[0].y);
+                dst[1] = make_float4(P[1].x, Q[1].x, P[1].y, Q[1].y);
             }
-#pragma unroll
-            for (int i0 = 0; i0 < I; i0 += 4) {
-                const float4 dt4 = *reinterpret_cast<const float4 *>(sDt + rb0 + i0);
-                const float4 du4 = *reinterpret_cast<const float4 *>(sDu + rb0 + i0);
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt) {
-                    const float dt = f4(dt4, tt), du = f4(du4, tt);
-                    const float *rowB = sB + bb0 + (i0 + tt) * kNP;
-#pragma unroll
-                    for (int s4 = 0; s4 < S; s4 += 4) {
-                        const float4 bv = *reinterpret_cast<const float4 *>(rowB + s4);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int s = s4 + q;
-                            const float a = mufu_ex2(dt * A2[s]);
-                            av[i0 + tt][s] = a;
-                            Q[s] = fmaf(a, Q[s], du * f4(bv, q));
-                            P[s] *= a;
-                        }
-                    }
-                }
+            __syncthreads();
+            const float *car = sCar + (chunk & 1) * DC * kNP + c * kNP + g * 4;
+            float hc[4] = {car[0], car[1], car[2], car[3]};
+            for (int jj = 0; jj < j; ++jj) {
+                const float4 *tot =
+                    reinterpret_cast<const float4 *>(sTot + ((jj * DC + c) * kNP + g * 4) * 2);
+                const float4 t0 = tot[0], t1 = tot[1];
+                hc[0] = fmaf(t0.x, hc[0], t0.y);
+                hc[1] = fmaf(t0.z, hc[1], t0.w);
+                hc[2] = fmaf(t1.x, hc[2], t1.y);
+                hc[3] = fmaf(t1.z, hc[3], t1.w);
             }
-            // combine the segments' transfer pairs inside the warp
-#pragma unroll
-            for (int r = 1; r < JW; r <<= 1) {
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    const float Pp = __shfl_up_sync(0xffffffffu, P[s], r * G);
-                    const float Qp = __shfl_up_sync(0xffffffffu, Q[s], r * G);
-                    if (jw >= r) {
-                        Q[s] = fmaf(P[s], Qp, Q[s]);
-                        P[s] *= Pp;
-                    }
-                }
-            }
-            float Pex[S], Qex[S];   // segments before mine, inside the warp
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                const float Pp = __shfl_up_sync(0xffffffffu, P[s], G);
-                const float Qp = __shfl_up_sync(0xffffffffu, Q[s], G);
-                Pex[s] = (jw == 0) ? 1.f : Pp;
-                Qex[s] = (jw == 0) ? 0.f : Qp;
-            }
-            float hw[S];   // state entering this warp's first segment
-            if constexpr (J == 1) {
-                const int last = (cw * JW + JW - 1) * G + g;
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    hw[s] = hcar[s];
-                    const float Pt = __shfl_sync(0xffffffffu, P[s], last);
-                    const float Qt = __shfl_sync(0xffffffffu, Q[s], last);
-                    hcar[s] = fmaf(Pt, hcar[s], Qt);
-                }
-            } else {
-                if (jw == JW - 1) {
-#pragma unroll
-                    for (int s = 0; s < S; ++s) {
-                        float *dst = sTot + ((j * DC + c) * kNP + g * S + s) * 2;
-                        dst[0] = P[s];
-                        dst[1] = Q[s];
-                    }
-                }
-                __syncthreads();
-                const float *car = sCar + (chunk & 1) * DC * kNP + c * kNP + g * S;
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    float hc = car[s];
-                    for (int jj = 0; jj < j; ++jj) {
-                        const float *tot = sTot + ((jj * DC + c) * kNP + g * S + s) * 2;
-                        hc = fmaf(tot[0], hc, tot[1]);
-                    }
-                    hw[s] = hc;
-                }
-                if (j == J - 1 && jw == JW - 1) {
-                    float *ncar = sCar + ((chunk + 1) & 1) * DC * kNP + c * kNP + g * S;
-#pragma unroll
-                    for (int s = 0; s < S; ++s)
-                        ncar[s] = fmaf(P[s], hw[s], Q[s]);
-                }
-            }
-            // pass 2: replay the segment from its entry state
-#pragma unroll
-            for (int s = 0; s < S; ++s)
-                h[s] = fmaf(Pex[s], hw[s], Qex[s]);
-#pragma unroll
-            for (int i0 = 0; i0 < I; i0 += 4) {
-                const float4 du4 = *reinterpret_cast<const float4 *>(sDu + rb0 + i0);
-                float yp[4];
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt) {
-                    const float du = f4(du4, tt);
-                    const float *rowB = sB + bb0 + (i0 + tt) * kNP;
-                    const float *rowC = sC + bb0 + (i0 + tt) * kNP;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int s4 = 0; s4 < S; s4 += 4) {
-                        const float4 bv = *reinterpret_cast<const float4 *>(rowB + s4);
-                        const float4 cv = *reinterpret_cast<const float4 *>(rowC + s4);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int s = s4 + q;
-                            h[s] = fmaf(av[i0 + tt][s], h[s], du * f4(bv, q));
-                            acc = fmaf(f4(cv, q), h[s], acc);
-                        }
-                    }
-                    yp[tt] = acc;
-                }
-                reduce_store<G>(yp, sY + rb0 + i0, sU + rb0 + i0, dsk, g);
+            hw[0] = make_float2(hc[0], hc[1]);
+            hw[1] = make_float2(hc[2], hc[3]);
+            if (j == J - 1 && jw == JW - 1) {
+                float *ncar = sCar + ((chunk + 1) & 1) * DC * kNP + c * kNP + g * 4;
+                const float2 n0 = __ffma2_rn(P[0], hw[0], Q[0]);
+                const float2 n1 = __ffma2_rn(P[1], hw[1], Q[1]);
+                ncar[0] = n0.x;
+                ncar[1] = n0.y;
+                ncar[2] = n1.x;
+                ncar[3] = n1.y;
             }
         }
-        __syncthreads();
-
-        // ---------------- write the chunk's outputs in pixel order -------
-        for (int e = tid; e < DC * LC; e += NT) {
-            const int t = e % LC;
-            const int cc = e / LC;
-            const int l = l0 + t;
-            const int dd = d0 + cc;
-            if (l < L && dd < D) {
-                const int pix = scan_pixel(p.two_d, k, l, H, W, L);
-                og[(size_t)dd * L + pix] = sY[cc * RS + (t / I) * SEG + (t % I)];
+        // pass 2: replay the segment from its entry state
+        float2 h[2];
+        h[0] = __ffma2_rn(Pex[0], hw[0], Qex[0]);
+        h[1] = __ffma2_rn(Pex[1], hw[1], Qex[1]);
+        const int *pix = sPix + js * I;
+#pragma unroll
+        for (int i0 = 0; i0 < I; i0 += 4) {
+            const float4 du4 = *reinterpret_cast<const float4 *>(dub + i0);
+            float yp[4];
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const int i = i0 + ii;
+                const float du = f4(du4, ii);
+                const float2 du2 = make_float2(du, du);
+                const float4 bv = tb[i * 8];
+                const float4 cv = tb[i * 8 + 4];
+                h[0] = __ffma2_rn(av[i][0], h[0], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
+                h[1] = __ffma2_rn(av[i][1], h[1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
+                float2 acc = __fmul2_rn(make_float2(cv.x, cv.y), h[0]);
+                acc = __ffma2_rn(make_float2(cv.z, cv.w), h[1], acc);
+                yp[ii] = acc.x + acc.y;
             }
+            // sum the four lanes of the channel; lane g keeps step i0 + g
+            const bool b1 = (g >> 1) & 1;
+            const float s0 = b1 ? yp[0] : yp[2];
+            const float s1 = b1 ? yp[1] : yp[3];
+            float k0 = b1 ? yp[2] : yp[0];
+            float k1 = b1 ? yp[3] : yp[1];
+            k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+            k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+            const bool b0 = g & 1;
+            const float sx = b0 ? k0 : k1;
+            float v = b0 ? k1 : k0;
+            v += __shfl_xor_sync(0xffffffffu, sx, 1);
+            const int t = js * I + i0 + g;
+            if (cvalid && l0 + t < L)
+                og[pix[i0 + g]] = fmaf(dsk, ub[i0 + g], v);
         }
     }
-}
-
-// y[b, r] = ((part[b,0,r] + part[b,1,r]) + part[b,2,r]) + part[b,3,r]
-// for r over the D*L outputs of batch b; K = 2 stops after the first add.
-template <int K>
-__global__ void merge_kernel(const float *__restrict__ part, float *__restrict__ y,
-                             long long DL, long long total)
-{
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    if ((DL & 3) == 0) {
-        const long long total4 = total >> 2;
-        for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total4;
-             i += stride) {
-            const long long e = i << 2;
-            const long long bb = e / DL, r = e - bb * DL;
-            const float *src = part + bb * K * DL + r;
-            float4 acc = __ldg(reinterpret_cast<const float4 *>(src));
-#pragma unroll
-            for (int kk = 1; kk < K; ++kk) {
-                const float4 v = __ldg(reinterpret_cast<const float4 *>(src + kk * DL));
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-            }
-            *reinterpret_cast<float4 *>(y + e) = acc;
-        }
-    } else {
-        for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-             e += stride) {
-            const long long bb = e / DL, r = e - bb * DL;
-            const float *src = part + bb * K * DL + r;
-            float acc = __ldg(src);
-#pragma unroll
-            for (int kk = 1; kk < K; ++kk)
-                acc += __ldg(src + kk * DL);
-            y[e] = acc;
-        }
+    if (p.merge) {
+        __syncthreads();
+        const int nc = min(DC, D - d0);
+        merge_epilogue(p, b, tile, d0, nc, NT);
     }
 }
 

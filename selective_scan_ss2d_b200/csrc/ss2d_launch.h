@@ -10,10 +10,11 @@ struct ScanParams;
 
 struct VariantInfo {
     const char *name;
-    int G, JW, J, WC, I;
-    int channels_per_cta;
+    int split;             // 0: one lane per channel; 1: time-split, 4 lanes per channel
+    int channels_per_cta;  // channel tile; one ticket per (batch, tile) when merging
     int threads;
-    int chunk;
+    int chunk;             // steps staged per chunk
+    int segments;          // time segments per chunk
     size_t smem_bytes;
     cudaError_t (*launch_f32)(const ScanParams &, cudaStream_t);
     cudaError_t (*launch_bf16)(const ScanParams &, cudaStream_t);
@@ -23,7 +24,5 @@ int num_variants();
 const VariantInfo *variant(int i);
 int pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
 cudaError_t launch_scan_variant(int v, bool bf16, const ScanParams &p, cudaStream_t st);
-cudaError_t launch_merge(int K, const float *part, float *y, long long DL, long long total,
-                         cudaStream_t st);
 
 }  // namespace ss2d
