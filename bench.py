@@ -266,24 +266,22 @@ def run_ours(args, rank, world, local_rank):
         total_ms = float(tt.item())
     value = cfg.updates * args.steps * world / (total_ms / 1e3)
 
-    # dominant kernel alone (the per-direction scan; for K = 1 it is the
-    # whole step), same inputs, same flushes, CUDA events on this stream
-    ydir = torch.empty((cfg.B, cfg.K, cfg.D, cfg.L), dtype=torch.float32, device=dev)
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    # per-launch device times of the same calls (same inputs, same flushes),
+    # CUDA events recorded by the library on this stream around each launch
     two_d = cfg.kind == "2d"
-    xx = t["x"]
+    per = []
     for i in range(args.steps):
         flush.fill_(float(i))
-        kev[i][0].record(stream)
-        binding.ss2d_scan_directions(xx, t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"],
-                                     t["delta_bias"], ydir.view((cfg.B, cfg.K, cfg.D, cfg.H,
-                                                                 cfg.W) if two_d else
-                                                                (cfg.B, cfg.K, cfg.D, cfg.L)),
-                                     two_d=two_d, variant=args.variant)
-        kev[i][1].record(stream)
-    torch.cuda.synchronize()
-    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+        per.append(binding.ss2d_forward_timed(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"],
+                                              t["Dskip"], t["delta_bias"], y, two_d=two_d,
+                                              stream=stream.cuda_stream, variant=args.variant))
+    names = ["chunk_state_pass", "carry", "scan_pass", "cross_merge"]
+    launch_ms = {}
+    for j, nm in enumerate(names):
+        vals = [r[j] for r in per if r[j] >= 0]
+        if vals:
+            launch_ms[nm] = statistics.mean(vals)
+    scan_ms = launch_ms["scan_pass"]
 
     result = {"rank_value": value}
     if rank == 0:
@@ -298,7 +296,9 @@ def run_ours(args, rank, world, local_rank):
         traffic = tr["bytes"] if tr and tr.get("src") == src_hash else None
         variant = args.variant if args.variant >= 0 else binding.ss2d_pick_variant(
             two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K)
+        plan = binding.ss2d_plan(two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K, variant)
         step_bytes = alg_bytes
+        step_s = total_ms / args.steps / 1e3
         result["line"] = {
             "metric": METRIC,
             "value": value,
@@ -322,14 +322,21 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
                          "traffic": traffic,
-                         "kernel": "scan_fwd_kernel",
+                         "kernel": "chunk_scan_kernel (scan pass: every update, every "
+                                   "algorithmic byte)",
                          "kernel_ms": scan_ms,
-                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"},
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)",
+                         "step": {"achieved": alg_bytes / step_s / 1e9,
+                                  "frac": alg_bytes / step_s / 1e9 / peaks["hbm_gbs"]}},
             "roofline_alu": {"bound": "alu", "achieved": achieved_gexp, "peak": mufu_peak,
                              "unit": "Gexp2/s", "frac": achieved_gexp / mufu_peak,
                              "note": "MUFU exp2 unit: 16/clk/SM x 148 SMs x max SM clock; "
-                                     "1 exp per state update + 1 per (b,k,d,l) for softplus"},
-            "gpu_launches": args.steps * (1 if cfg.K == 1 else 2),
+                                     "1 exp per state update + 1 per (b,k,d,l) for softplus",
+                             "step": {"achieved": exps / step_s / 1e9,
+                                      "frac": exps / step_s / 1e9 / mufu_peak}},
+            "launch_ms": launch_ms,
+            "plan": plan,
+            "gpu_launches": args.steps * plan["launches"],
         }
         result["clocks"] = clocks
     return result

@@ -142,6 +142,25 @@ int selective_scan_fwd_ex(const void *u, const void *delta, const float *A_log,
                           int B, int D, int L, int N, int K, int dtype,
                           void *stream, int variant);
 
+/* How a call with this shape and variant (-1 = the library's choice) is
+ * executed: steps per chunk, chunks per sequence, and kernel launches per
+ * call (1 scan pass, or state pass + carry + scan pass when the sequence is
+ * chunked; plus one cross_merge launch when K > 1).  Host only. */
+int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
+              int *chunk_len, int *num_chunks, int *launches);
+
+/* Measurement helper: runs one ss2d_forward (two_d = 1) or
+ * selective_scan_fwd (two_d = 0) call on device pointers, recording CUDA
+ * events on `stream` around each of its kernel launches, synchronises the
+ * stream and writes the device time of each launch in milliseconds to
+ * launch_ms[0..3] in the order [chunk state pass, carry, scan pass,
+ * cross_merge]; a launch the call does not make gets -1.  Blocking. */
+int ss2d_forward_timed(const void *x, const void *delta, const float *A_log,
+                       const void *Bs, const void *Cs, const float *Dskip,
+                       const float *delta_bias, float *y,
+                       int B, int D, int H, int W, int N, int K, int dtype,
+                       int two_d, void *stream, int variant, float *launch_ms);
+
 /* Number of kernel variants, and a static description of variant i
  * ("" for an index out of range). */
 int ss2d_num_variants(void);

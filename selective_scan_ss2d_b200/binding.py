@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
             L.selective_scan_fwd_ex.restype = i
             L.ss2d_scan_directions.argtypes = fwd + [i] * 8 + [vp, i]
             L.ss2d_scan_directions.restype = i
+            L.ss2d_plan.argtypes = [i] * 8 + [ctypes.POINTER(ctypes.c_int)] * 3
+            L.ss2d_plan.restype = i
+            L.ss2d_forward_timed.argtypes = fwd + [i] * 8 + [vp, i, ctypes.POINTER(ctypes.c_float)]
+            L.ss2d_forward_timed.restype = i
             L.ss2d_num_variants.argtypes = []
             L.ss2d_num_variants.restype = i
             L.ss2d_variant_name.argtypes = [i]
@@ -205,3 +209,32 @@ def ss2d_scan_directions(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y_dir=None,
                                     N, K, dt, int(bool(two_d)), st, int(variant))
     _check(rc)
     return y_dir
+
+
+def ss2d_plan(two_d: bool, B: int, D: int, H: int, W: int, N: int, K: int,
+              variant: int = -1) -> dict:
+    """Execution plan of a call: steps per chunk, chunks, kernel launches."""
+    lc, nc, nl = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().ss2d_plan(int(bool(two_d)), B, D, H, W, N, K, int(variant), ctypes.byref(lc),
+                           ctypes.byref(nc), ctypes.byref(nl)))
+    return {"chunk_len": lc.value, "num_chunks": nc.value, "launches": nl.value}
+
+
+def ss2d_forward_timed(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, *, two_d: bool = True,
+                       stream=None, variant: int = -1) -> list:
+    """One forward call on CUDA tensors with per-launch device times in ms:
+    [chunk state pass, carry, scan pass, cross_merge] (-1 = not launched).
+    Blocking (measurement helper)."""
+    if two_d:
+        B, D, H, W = x.shape
+    else:
+        B, D, W = x.shape
+        H = 1
+    K, N = delta.shape[1], Bs.shape[2]
+    y, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, tuple(x.shape))
+    st = _stream(on_gpu, x.device, stream)
+    ms = (ctypes.c_float * 4)()
+    _check(lib().ss2d_forward_timed(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                                    _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, H, W, N, K,
+                                    dt, int(bool(two_d)), st, int(variant), ms))
+    return [float(v) for v in ms]

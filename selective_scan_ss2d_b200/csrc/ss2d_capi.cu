@@ -1,7 +1,6 @@
 // ss2d_capi.cu -- the C ABI declared in include/ss2d.h: argument checks,
-// scratch memory, the host-buffer path, and the launch of the scan kernel
-// (per-direction pixel-order partials, merged in fixed order by the last CTA
-// of each channel tile).
+// scratch memory, the host-buffer path, and the launch sequence of a call
+// (chunk state pass, carry, output pass, cross_merge).
 #include <cuda_runtime.h>
 #include <limits.h>
 #include <stdint.h>
@@ -11,7 +10,7 @@
 #include <mutex>
 
 #include "ss2d.h"
-#include "ss2d_kernels.cuh"
+#include "ss2d_params.h"
 #include "ss2d_launch.h"
 
 namespace {
@@ -163,69 +162,58 @@ ss2d::ScanParams make_params(const Problem &pr)
     return p;
 }
 
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
 // Device path: every pointer is device memory of the current device.
-// K = 1: the scan writes y directly.  K > 1: the scan writes per-direction
-// partials to pool scratch, and the last CTA of each channel tile adds them
-// into y (tickets zeroed here, on the stream, before the launch).
-int run_device(const Problem &pr, cudaStream_t st, int variant)
+//   chunked (plan.NC > 1): state pass, carry, output pass;
+//   K = 1: the output pass writes y (scan order of direction 0 = pixel order);
+//   K > 1: the output pass writes per-direction scan-order rows to scratch
+//   and the merge kernel sums them into y in fixed order (directions = true:
+//   copies them to y as per-direction pixel-order outputs instead).
+// Scratch comes from the pool on the stream and goes back to it on the stream.
+int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
+               cudaEvent_t *ev = nullptr)
 {
     ss2d::ScanParams p = make_params(pr);
     const bool bf16 = pr.dtype == SS2D_BF16;
-    const long long DL = (long long)pr.D * p.L;
-    if (pr.K == 1) {
-        p.out = pr.y;
-        p.out_b_stride = DL;
-        p.out_k_stride = 0;
-        p.merge = 0;
-        cudaError_t e = ss2d::launch_scan_variant(variant, bf16, p, st);
-        if (e != cudaSuccess) {
-            set_error("scan kernel launch", e);
-            return SS2D_ERR_CUDA;
-        }
-        return SS2D_OK;
-    }
-    const ss2d::VariantInfo *vi = ss2d::variant(variant);
-    const long long tiles = (pr.D + vi->channels_per_cta - 1) / vi->channels_per_cta;
-    const size_t part_bytes = sizeof(float) * (size_t)pr.B * pr.K * DL;
-    const size_t part_up = (part_bytes + 255) & ~(size_t)255;
-    const size_t ticket_bytes = sizeof(unsigned int) * (size_t)pr.B * tiles;
+    const long long L = p.L;
+    const ss2d::Plan pl = ss2d::make_plan(variant, pr.B, pr.D, (int)L, pr.K);
+    if ((long long)pr.B * pl.NC > 65535)
+        return SS2D_ERR_SHAPE;
+    if (ss2d::merge_smem_bytes(pr.W, pr.K, pr.two_d) > 200 * 1024)
+        return SS2D_ERR_SHAPE;
+    const bool need_part = pr.K > 1;
+    const size_t rows = (size_t)pr.B * pr.K * pr.D;
+    const size_t part_bytes = need_part ? align256(sizeof(float) * rows * L) : 0;
+    const size_t hs_bytes = pl.NC > 1 ? align256(sizeof(float) * rows * (pl.NC - 1) * ss2d::kNP) : 0;
+    const size_t ds_bytes = pl.NC > 1 ? align256(sizeof(float) * rows * (pl.NC - 1)) : 0;
+    const size_t total = part_bytes + hs_bytes + ds_bytes;
     void *scratch = nullptr;
-    int rc = pool_alloc(&scratch, part_up + ticket_bytes, st);
-    if (rc != SS2D_OK)
-        return rc;
-    p.out = static_cast<float *>(scratch);
-    p.out_b_stride = (long long)pr.K * DL;
-    p.out_k_stride = DL;
-    p.y = pr.y;
-    p.tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(scratch) + part_up);
-    p.merge = 1;
-    cudaError_t e = cudaMemsetAsync(p.tickets, 0, ticket_bytes, st);
-    if (e == cudaSuccess)
-        e = ss2d::launch_scan_variant(variant, bf16, p, st);
-    cudaError_t ef = cudaFreeAsync(scratch, st);
+    if (total > 0) {
+        int rc = pool_alloc(&scratch, total, st);
+        if (rc != SS2D_OK)
+            return rc;
+    }
+    char *base = static_cast<char *>(scratch);
+    p.out = need_part ? reinterpret_cast<float *>(base) : pr.y;
+    p.hstate = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes) : nullptr;
+    p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes + hs_bytes) : nullptr;
+    cudaError_t e = ss2d::launch_scan(pl, bf16, p, st, ev);
+    if (e == cudaSuccess && need_part) {
+        e = ss2d::launch_merge(p.out, pr.y, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d,
+                               directions ? 0 : 1, st);
+        if (ev)
+            cudaEventRecord(ev[4], st);
+    }
+    cudaError_t ef = cudaSuccess;
+    if (scratch)
+        ef = cudaFreeAsync(scratch, st);
     if (e != cudaSuccess) {
-        set_error("scan kernel launch", e);
+        set_error("kernel launch", e);
         return SS2D_ERR_CUDA;
     }
     if (ef != cudaSuccess) {
         set_error("cudaFreeAsync", ef);
-        return SS2D_ERR_CUDA;
-    }
-    return SS2D_OK;
-}
-
-// Per-direction outputs only: the scan kernel writes straight into y_dir.
-int run_directions(const Problem &pr, cudaStream_t st, int variant)
-{
-    ss2d::ScanParams p = make_params(pr);
-    const long long DL = (long long)pr.D * p.L;
-    p.out = pr.y;
-    p.out_b_stride = (long long)pr.K * DL;
-    p.out_k_stride = DL;
-    p.merge = 0;
-    cudaError_t e = ss2d::launch_scan_variant(variant, pr.dtype == SS2D_BF16, p, st);
-    if (e != cudaSuccess) {
-        set_error("scan kernel launch", e);
         return SS2D_ERR_CUDA;
     }
     return SS2D_OK;
@@ -272,7 +260,7 @@ int run_host(const Problem &pr, cudaStream_t st, int variant)
     dp.Dskip = reinterpret_cast<const float *>(base + off[5]);
     dp.delta_bias = reinterpret_cast<const float *>(base + off[6]);
     dp.y = reinterpret_cast<float *>(base + off[7]);
-    rc = run_device(dp, st, variant);
+    rc = run_device(dp, st, variant, false);
     if (rc == SS2D_OK) {
         e = cudaMemcpyAsync(pr.y, dp.y, sz[7], cudaMemcpyDeviceToHost, st);
         if (e != cudaSuccess) {
@@ -318,8 +306,8 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
             return SS2D_ERR_PTR;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (directions_only)
-        return kind == kDevicePtr ? run_directions(pr, st, variant) : SS2D_ERR_PTR;
-    return kind == kDevicePtr ? run_device(pr, st, variant) : run_host(pr, st, variant);
+        return kind == kDevicePtr ? run_device(pr, st, variant, true) : SS2D_ERR_PTR;
+    return kind == kDevicePtr ? run_device(pr, st, variant, false) : run_host(pr, st, variant);
 }
 
 }  // namespace
@@ -368,6 +356,95 @@ int ss2d_scan_directions(const void *x, const void *delta, const float *A_log,
     Problem pr{x, delta, Bs, Cs, A_log, Dskip, delta_bias, y_dir, B, D, H, W, N, K, dtype,
                two_d ? 1 : 0};
     return forward(pr, stream, variant, true);
+}
+
+int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
+              int *chunk_len, int *num_chunks, int *launches)
+{
+    Problem pr{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+               B, D, H, W, N, K, SS2D_F32, two_d ? 1 : 0};
+    int rc = validate(pr);
+    if (rc != SS2D_OK)
+        return rc;
+    if (variant < -1 || variant >= ss2d::num_variants())
+        return SS2D_ERR_VARIANT;
+    if (variant < 0)
+        variant = ss2d::pick_variant(pr.two_d, B, D, H, W, N, K);
+    const ss2d::Plan pl = ss2d::make_plan(variant, B, D, H * W, K);
+    if (chunk_len)
+        *chunk_len = pl.LC;
+    if (num_chunks)
+        *num_chunks = pl.NC;
+    if (launches)
+        *launches = pl.launches;
+    return SS2D_OK;
+}
+
+int ss2d_forward_timed(const void *x, const void *delta, const float *A_log, const void *Bs,
+                       const void *Cs, const float *Dskip, const float *delta_bias, float *y,
+                       int B, int D, int H, int W, int N, int K, int dtype, int two_d,
+                       void *stream, int variant, float *launch_ms)
+{
+    if (!launch_ms)
+        return SS2D_ERR_NULL;
+    Problem pr{x, delta, Bs, Cs, A_log, Dskip, delta_bias, y, B, D, H, W, N, K, dtype,
+               two_d ? 1 : 0};
+    int rc = validate(pr);
+    if (rc != SS2D_OK)
+        return rc;
+    if (variant < -1 || variant >= ss2d::num_variants())
+        return SS2D_ERR_VARIANT;
+    if (is_empty(pr))
+        return SS2D_OK;
+    rc = check_pointers(pr);
+    if (rc != SS2D_OK)
+        return rc;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_error("cudaGetDevice", e);
+        return SS2D_ERR_CUDA;
+    }
+    const void *ptrs[] = {x, delta, Bs, Cs, A_log, Dskip, delta_bias, y};
+    for (const void *q : ptrs)
+        if (pointer_kind(q, dev) != kDevicePtr)
+            return SS2D_ERR_PTR;
+    if (variant < 0)
+        variant = ss2d::pick_variant(pr.two_d, B, D, H, W, N, K);
+    cudaEvent_t ev[5];
+    for (int i = 0; i < 5; ++i) {
+        e = cudaEventCreate(&ev[i]);
+        if (e != cudaSuccess) {
+            for (int j = 0; j < i; ++j)
+                cudaEventDestroy(ev[j]);
+            set_error("cudaEventCreate", e);
+            return SS2D_ERR_CUDA;
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ss2d::Plan pl = ss2d::make_plan(variant, B, D, H * W, K);
+    rc = run_device(pr, st, variant, false, ev);
+    if (rc == SS2D_OK) {
+        e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) {
+            set_error("cudaStreamSynchronize", e);
+            rc = SS2D_ERR_CUDA;
+        }
+    }
+    for (int i = 0; i < 4; ++i)
+        launch_ms[i] = -1.f;
+    if (rc == SS2D_OK) {
+        if (pl.NC > 1) {
+            cudaEventElapsedTime(&launch_ms[0], ev[0], ev[1]);
+            cudaEventElapsedTime(&launch_ms[1], ev[1], ev[2]);
+        }
+        cudaEventElapsedTime(&launch_ms[2], ev[2], ev[3]);
+        if (K > 1)
+            cudaEventElapsedTime(&launch_ms[3], ev[3], ev[4]);
+    }
+    for (int i = 0; i < 5; ++i)
+        cudaEventDestroy(ev[i]);
+    return rc;
 }
 
 int ss2d_num_variants(void) { return ss2d::num_variants(); }

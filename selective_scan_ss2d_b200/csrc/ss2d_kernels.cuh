@@ -6,40 +6,33 @@
 //     dt_l = softplus(delta_l + bias)
 //     h_l  = exp(dt_l * A_n) * h_{l-1} + dt_l * B_{n,l} * u_l        (h_{-1} = 0)
 //     y_l  = sum_n C_{n,l} h_l + Dskip * u_l
-// with u_l = x[pixel(k, l)] (cross_scan folded into address generation) and
-// the K outputs put back in pixel order and summed in the fixed order
-// k = 0, 1, 2, 3 (cross_merge).
+// with u_l = x[pixel(k, l)]: the cross_scan is folded into the address
+// generation; no unfolded copy of x exists.
 //
-// Two kernel families share the staging and epilogue code:
+// Work decomposition.  One lane owns one (b, k, d) channel with all 16
+// states in registers; a CTA holds 32*WC channels of one (b, k).  Long
+// sequences with few channels are cut into NC chunks of LC steps so that
+// enough lanes exist; the chunks are independent given their entry state:
+//   1. chunk_scan_kernel<..., kModeState>: every chunk but the last runs
+//      from a zero state and stores its end state and its sum of dt;
+//   2. carry_kernel: per (b,k,d,n), sequentially over the chunks,
+//      h_in[c+1] = exp(A_n * sum_c(dt)) * h_in[c] + h_end[c];
+//   3. chunk_scan_kernel<..., kModeOutput>: every chunk from its true entry
+//      state, writing y_k in scan order (per-direction scratch, or y when
+//      K = 1);
+//   4. merge_kernel (K > 1): y[p] = ((Y_0[s_0(p)] + Y_1[s_1(p)]) +
+//      Y_2[s_2(p)]) + Y_3[s_3(p)], s_k the pixel -> scan-step map of
+//      direction k (cross_merge), always in that order.
+// Chunking costs one extra exp per update on the chunked workloads only,
+// and keeps every pass a uniform mix of MUFU and FMA work.
 //
-//  * scan_direct_kernel -- one lane per (b, k, d) channel, all 16 states in
-//    registers.  For workloads with many channels (VMamba-B stage 3, Vim).
-//    Each lane loads its own delta and x (prefetched one batch of four steps
-//    ahead) and computes softplus once per step; B and C of a chunk of steps,
-//    shared by every channel of the CTA, are staged in shared memory with a
-//    register prefetch one chunk ahead (double buffer).
-//
-//  * scan_split_kernel -- four lanes per channel (4 states each) and the
-//    sequence split in time, for long sequences with few channels (VMamba-T
-//    stage 1, 256x256 maps).  A chunk of LC steps is cut into NS segments of
-//    I steps (JW segments inside a warp, J warps).  Each lane runs its segment
-//    from a zero state keeping every exp(dt*A) in registers, and accumulates
-//    the segment's transfer pair (P, Q), h_out = P*h_in + Q.  The pairs are
-//    combined with the associative operator (P1,Q1) then (P2,Q2) =
-//    (P2*P1, P2*Q1 + Q2) -- shuffles inside the warp, shared memory across
-//    warps, together with the carry of the previous chunk -- and each lane
-//    replays its segment from its true entry state with the kept
-//    exponentials, so no exponential is evaluated twice.  The raw B, C and
-//    delta rows of the next chunk are copied to shared memory with 16-byte
-//    asynchronous copies (cp.async) while the current chunk computes; a
-//    conversion pass then builds float32 tiles of B|C and of dt (one softplus
-//    per (channel, step)), dt*u and u.
-//
-// Both write each direction's output in pixel order.  With K > 1 they write
-// it to a scratch buffer and the last of the K CTAs that cover the same
-// channels (an atomic ticket per tile, no waiting) adds the K outputs in the
-// fixed order and writes y; so the merge costs no extra launch and reads
-// partials that are still in L2.
+// Memory traffic is coalesced: per 32-step sub-chunk, each warp loads delta
+// and x for its 32 channels one channel per instruction (lanes = steps) and
+// transposes them through a warp-private shared-memory tile; outputs go back
+// the same way.  B and C of a sub-chunk (shared by every channel of the CTA)
+// are staged once per CTA as a float32 [step][32] tile, read with broadcast
+// float4 loads.  The next sub-chunk's loads are spread over the current
+// sub-chunk's compute (software pipelining; nothing waits on a flag).
 //
 // exp(dt*A) runs on the MUFU unit as 2^(dt * A*log2(e)).  The float32 pair
 // arithmetic uses the sm_100 packed f32x2 instructions (__ffma2_rn,
@@ -50,37 +43,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ss2d_params.h"
+
 namespace ss2d {
 
-constexpr int kNP = 16;  // states per channel held by the kernels (N <= 16)
-constexpr float kLog2e = 1.4426950408889634f;
-
-struct ScanParams {
-    const void *x;           // (B,D,H,W) / (B,D,L)
-    const void *delta;       // (B,K,D,L) scan order
-    const float *A_log;      // (K*D,N)
-    const void *Bs;          // (B,K,N,L) scan order
-    const void *Cs;          // (B,K,N,L) scan order
-    const float *Dskip;      // (K*D)
-    const float *delta_bias; // (K*D)
-    float *out;              // partials (B,K,D,L) or y (B,D,L), pixel order
-    float *y;                // final y (B,D,L) when the kernel merges (K > 1)
-    unsigned int *tickets;   // one zeroed counter per (b, channel tile) when merging
-    int B, D, H, W, L, N, K;
-    int two_d;               // 1: SS2D scan orders; 0: 1D (k = 1 reversed)
-    long long out_b_stride;  // elements between batches in `out`
-    long long out_k_stride;  // elements between directions in `out`
-    int merge;               // 1: the last CTA of a tile sums the K partials into y
-};
-
-__device__ __forceinline__ float load_in(const float *p) { return __ldg(p); }
-__device__ __forceinline__ float load_in(const __nv_bfloat16 *p)
-{
-    return __bfloat162float(__ldg(p));
-}
-// element of a staged (shared-memory) row
-__device__ __forceinline__ float load_in_smem(const float *p) { return *p; }
-__device__ __forceinline__ float load_in_smem(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // 2^x on the multi-function unit (PTX ex2.approx.ftz.f32).
 __device__ __forceinline__ float mufu_ex2(float x)
@@ -109,15 +77,10 @@ __device__ __forceinline__ float softplus_f(float z)
     return fmaf(e, q, fmaxf(z, 0.f));
 }
 
-__device__ __forceinline__ float f4(const float4 &v, int i)
-{
-    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
-
-// Walks direction k's scan -> pixel map (see include/ss2d.h) one step, or a
-// fixed stride of steps, at a time, without divisions.
+// Walks direction k's scan -> pixel map (see include/ss2d.h) a fixed stride
+// of steps at a time, without divisions.
 struct PixWalk {
-    int p;      // pixel of the current step (only meaningful while l < L)
+    int p;      // pixel of the current step (meaningful while the step is < L)
     int h, w;   // row and column, for the column-major directions
     int mode;   // 0: p = l; 1: p = L-1-l; 2: column-major; 3: reversed column-major
 
@@ -133,30 +96,6 @@ struct PixWalk {
             h = m % H;
             w = m / H;
             p = h * W + w;
-        }
-    }
-    __device__ __forceinline__ void next(int H, int W)
-    {
-        if (mode == 0) {
-            ++p;
-        } else if (mode == 1) {
-            --p;
-        } else if (mode == 2) {
-            if (++h == H) {
-                h = 0;
-                ++w;
-                p = w;
-            } else {
-                p += W;
-            }
-        } else {
-            if (--h < 0) {
-                h = H - 1;
-                --w;
-                p = h * W + w;
-            } else {
-                p -= W;
-            }
         }
     }
     // advance by n = nq*H + nr steps (nq = n / H, nr = n % H precomputed)
@@ -186,179 +125,190 @@ struct PixWalk {
     }
 };
 
-// ---------------------------------------------------------------------------
-// cross_merge epilogue: the last of the K CTAs covering channels
-// [d0, d0 + nc) of batch b adds the K pixel-order partials, k = 0..K-1 in
-// order, and writes y.  Called by every thread of the CTA after its partial
-// outputs are written.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void merge_epilogue(const ScanParams &p, int b, int tile, int d0,
-                                               int nc, int nthreads)
-{
-    __shared__ int s_last;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned int t = atomicAdd(p.tickets + (size_t)b * gridDim.y + tile, 1u);
-        s_last = (t == (unsigned int)(p.K - 1));
-    }
-    __syncthreads();
-    if (!s_last)
-        return;
-    __threadfence();
-    const long long L = p.L;
-    const long long cnt = (long long)nc * L;
-    const float *src = p.out + (size_t)b * p.out_b_stride + (size_t)d0 * L;
-    float *dst = p.y + ((size_t)b * p.D + d0) * L;
-    const long long ks = p.out_k_stride;
-    const bool vec = ((((uintptr_t)src) | ((uintptr_t)dst)) & 15) == 0 && (ks % 4) == 0 &&
-                     (cnt % 4) == 0;
-    if (vec) {
-        for (long long i = (long long)threadIdx.x * 4; i < cnt; i += (long long)nthreads * 4) {
-            float4 acc = __ldcg(reinterpret_cast<const float4 *>(src + i));
-            for (int k = 1; k < p.K; ++k) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + k * ks + i));
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-            }
-            *reinterpret_cast<float4 *>(dst + i) = acc;
-        }
-    } else {
-        for (long long i = threadIdx.x; i < cnt; i += nthreads) {
-            float acc = __ldcg(src + i);
-            for (int k = 1; k < p.K; ++k)
-                acc += __ldcg(src + k * ks + i);
-            dst[i] = acc;
-        }
-    }
-}
+enum ScanMode { kModeState = 0, kModeOutput = 1 };
 
-// ===========================================================================
-// scan_direct_kernel: lane = channel, 16 states per lane
-// ===========================================================================
-template <int WC, int LC>
-struct DirectShape {
-    static constexpr int NT = 32 * WC;       // threads = channels per CTA
-    static constexpr int NE = LC * 8;        // float4 entries of a B|C chunk tile
-    static constexpr int EPT = NE / NT;      // entries staged per thread per chunk
-    static_assert(NE % NT == 0, "whole entries per thread");
-    static_assert(LC % 4 == 0, "steps come in groups of four");
+template <int WC>
+struct ChunkShape {
+    static constexpr int NT = 32 * WC;                     // threads = channels per CTA
+    static constexpr int TROW = 33;                        // padded row of a warp tile
+    static constexpr int WTILE = kT * TROW;                // floats per warp tile
+    static constexpr int BC_ENTRIES = kT * 8;              // float4 per B|C sub-chunk tile
+    static constexpr int BC_PER_THREAD = BC_ENTRIES / NT;  // float4 staged per thread
+    static_assert(BC_ENTRIES % NT == 0, "whole B|C entries per thread");
+    static_assert(BC_PER_THREAD <= 8, "B|C staging spread over the 8 batches");
+    // shared memory: B|C double buffer, then per warp: delta and x double
+    // buffers and one output tile
+    static constexpr size_t SMEM_BYTES =
+        sizeof(float4) * 2 * BC_ENTRIES + sizeof(float) * WC * 5 * WTILE;
 };
 
-template <typename Tin, int WC, int LC, int MINB>
-__global__ void __launch_bounds__(32 * WC, MINB) scan_direct_kernel(const ScanParams p)
+// One chunk of LC steps of 32*WC channels of one (b, k); see the header.
+// grid: x = k, y = channel tile, z = b * NCg + chunk, NCg = chunks launched
+// (NC - 1 in kModeState, NC in kModeOutput).
+template <typename Tin, int WC, int MODE, int MINB>
+__global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
 {
-    using Sh = DirectShape<WC, LC>;
-    constexpr int NT = Sh::NT, EPT = Sh::EPT;
-    // [buffer][step][B n0-3 | B n4-7 | B n8-11 | B n12-15 | C ... ]
-    __shared__ __align__(16) float4 sBC[2][LC * 8];
+    using Sh = ChunkShape<WC>;
+    constexpr int NT = Sh::NT, TROW = Sh::TROW, WTILE = Sh::WTILE;
+    constexpr int BCPT = Sh::BC_PER_THREAD;
+
+    extern __shared__ float4 smem_f4[];
+    float4 *sBC = smem_f4;   // [2][kT][8], slot q of step t stored at t*8 + (q ^ (t & 7))
+    float *wtiles = reinterpret_cast<float *>(sBC + 2 * Sh::BC_ENTRIES);
 
     const int tid = threadIdx.x;
-    const int k = blockIdx.x, tile = blockIdx.y, b = blockIdx.z;
-    const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W;
+    const int lane = tid & 31, warp = tid >> 5;
+    float *sD = wtiles + warp * 5 * WTILE;   // [2][kT][33] raw delta
+    float *sX = sD + 2 * WTILE;              // [2][kT][33] u
+    float *sY = sX + 2 * WTILE;              // [kT][33] outputs
+
+    const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W, K = p.K;
+    const int k = blockIdx.x, tile = blockIdx.y;
+    const int ncg = (MODE == kModeState) ? p.NC - 1 : p.NC;
+    const int b = blockIdx.z / ncg, chunk = blockIdx.z % ncg;
     const int d0 = tile * NT;
+    const int wd0 = d0 + warp * 32;          // first channel of this warp
     const int d = d0 + tid;
     const bool cvalid = d < D;
-    const int kd = k * D + (cvalid ? d : 0);
+    const int dc = cvalid ? d : D - 1;       // clamped channel for parameter reads
+    const int kd = k * D + dc;
+    const int l_begin = chunk * p.LC;
+    const int l_end = min(l_begin + p.LC, L);
 
     float2 A2[8];   // A[n] * log2(e) for states (2j, 2j+1)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int n0 = 2 * j, n1 = 2 * j + 1;
-        A2[j].x = (cvalid && n0 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0)) * kLog2e : 0.f;
-        A2[j].y = (cvalid && n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
+        A2[j].x = (n0 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0)) * kLog2e : 0.f;
+        A2[j].y = (n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
     }
-    const float dsk = cvalid ? __ldg(p.Dskip + kd) : 0.f;
-    const float bias = cvalid ? __ldg(p.delta_bias + kd) : 0.f;
+    const float dsk = __ldg(p.Dskip + kd);
+    const float bias = __ldg(p.delta_bias + kd);
 
-    const Tin *xg = static_cast<const Tin *>(p.x) + ((size_t)b * D + (cvalid ? d : 0)) * L;
-    const Tin *dg = static_cast<const Tin *>(p.delta) +
-                    (((size_t)b * p.K + k) * D + (cvalid ? d : 0)) * L;
-    const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * p.K + k) * N * L;
-    const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * p.K + k) * N * L;
-    float *og = p.out + (size_t)b * p.out_b_stride + (size_t)k * p.out_k_stride +
-                (size_t)(cvalid ? d : 0) * L;
+    const size_t row_bk = ((size_t)b * K + k) * D;   // row index of (b, k, d = 0)
+    const Tin *xg = static_cast<const Tin *>(p.x) + (size_t)b * D * L;
+    const Tin *dg = static_cast<const Tin *>(p.delta) + row_bk * L;
+    const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * K + k) * N * L;
+    const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * K + k) * N * L;
 
-    // ---- B/C staging: entry e = (step t = e >> 3, block q = e & 7) ----
-    float raw[EPT][4];
-    auto load_bc = [&](int l0) {
+    // entry state
+    float2 h2[8];
+    if (MODE == kModeOutput && chunk > 0) {
+        const float4 *hs = reinterpret_cast<const float4 *>(
+            p.hstate + ((row_bk + dc) * (p.NC - 1) + (chunk - 1)) * kNP);
 #pragma unroll
-        for (int r = 0; r < EPT; ++r) {
-            const int e = tid + r * NT;
-            const int q = e & 7, t = e >> 3;
-            const int l = l0 + t;
-            const Tin *src = (q < 4) ? Bg : Cg;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = (q & 3) * 4 + i;
-                raw[r][i] = (l < L && n < N) ? load_in(src + (size_t)n * L + l) : 0.f;
-            }
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = hs[q];
+            h2[2 * q] = make_float2(v.x, v.y);
+            h2[2 * q + 1] = make_float2(v.z, v.w);
         }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            h2[j] = make_float2(0.f, 0.f);
+    }
+    float dtsum = 0.f;
+
+    // ---- staging of the sub-chunk that starts at ld_l0 ------------------
+    // delta / x: batch j (0..7) loads channels 4j .. 4j+3 of this warp, lane
+    // = step, into registers; the next batch stores them transposed into the
+    // warp tile [step][channel].
+    PixWalk xw;   // pixel of step ld_l0 + lane
+    xw.init(p.two_d, k, l_begin + lane, H, W, L);
+    const int sq = kT / H, sr = kT % H;
+    float rd[4], rx[4];
+    int ld_l0 = l_begin;
+    auto load_dx = [&](int j) {
+        const int l = ld_l0 + lane;
+        const bool lok = l < l_end;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int cc = wd0 + j * 4 + i;
+            const bool ok = lok && cc < D;
+            rd[i] = ok ? to_f32(dg[(size_t)cc * L + l]) : 0.f;
+            rx[i] = ok ? to_f32(xg[(size_t)cc * L + xw.p]) : 0.f;
+        }
+    };
+    auto store_dx = [&](int buf, int j) {
+        float *td = sD + buf * WTILE + lane * TROW + j * 4;
+        float *tx = sX + buf * WTILE + lane * TROW + j * 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            td[i] = rd[i];
+            tx[i] = rx[i];
+        }
+    };
+    // B|C: float4 entry e = (slot q = e / kT, step t = e % kT) holds rows
+    // 4q..4q+3 of B (q < 4) or C (q >= 4) at step t
+    float4 rbc[BCPT];
+    auto load_bc_one = [&](int r) {
+        const int e = tid + r * NT;
+        const int q = e / kT, t = e % kT;
+        const int l = ld_l0 + t;
+        const Tin *src = (q < 4) ? Bg : Cg;
+        float v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int n = (q & 3) * 4 + i;
+            v[i] = (l < l_end && n < N) ? to_f32(src[(size_t)n * L + l]) : 0.f;
+        }
+        rbc[r] = make_float4(v[0], v[1], v[2], v[3]);
     };
     auto store_bc = [&](int buf) {
 #pragma unroll
-        for (int r = 0; r < EPT; ++r)
-            sBC[buf][tid + r * NT] = make_float4(raw[r][0], raw[r][1], raw[r][2], raw[r][3]);
-    };
-
-    // ---- per-lane delta / x, prefetched one batch of four steps ahead ----
-    PixWalk pw;
-    pw.init(p.two_d, k, 0, H, W, L);
-    float qd[4], qx[4];
-    int qp[4];
-    auto load_batch = [&](int l) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool ok = cvalid && (l + i) < L;
-            qp[i] = pw.p;
-            qd[i] = ok ? load_in(dg + l + i) : 0.f;
-            qx[i] = ok ? load_in(xg + pw.p) : 0.f;
-            pw.next(H, W);
+        for (int r = 0; r < BCPT; ++r) {
+            const int e = tid + r * NT;
+            const int q = e / kT, t = e % kT;
+            sBC[buf * Sh::BC_ENTRIES + t * 8 + (q ^ (t & 7))] = rbc[r];
         }
     };
 
-    float2 h2[8];
+    // prologue: stage the first sub-chunk
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        h2[j] = make_float2(0.f, 0.f);
-
-    load_bc(0);
+    for (int r = 0; r < BCPT; ++r)
+        load_bc_one(r);
     store_bc(0);
-    load_batch(0);
+#pragma unroll 1
+    for (int j = 0; j < 8; ++j) {
+        load_dx(j);
+        store_dx(0, j);
+    }
     __syncthreads();
 
     int buf = 0;
-    for (int l0 = 0; l0 < L; l0 += LC, buf ^= 1) {
-        const bool more = l0 + LC < L;
-        if (more)
-            load_bc(l0 + LC);
-        const float4 *sb = sBC[buf];
-#pragma unroll 1
-        for (int t0 = 0; t0 < LC; t0 += 4) {
-            float cd[4], cx[4];
-            int cp[4];
+    for (int l0 = l_begin; l0 < l_end; l0 += kT, buf ^= 1) {
+        const bool more = l0 + kT < l_end;
+        ld_l0 = l0 + kT;
+        xw.advance(kT, sq, sr, H, W);
+        const float4 *sb = sBC + buf * Sh::BC_ENTRIES;
+        const float *td = sD + buf * WTILE;
+        const float *tx = sX + buf * WTILE;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                cd[i] = qd[i];
-                cx[i] = qx[i];
-                cp[i] = qp[i];
+        for (int j = 0; j < 8; ++j) {
+            // software-pipelined staging of the next sub-chunk
+            if (more) {
+                if (j > 0)
+                    store_dx(buf ^ 1, j - 1);
+                load_dx(j);
+                if (j < BCPT)
+                    load_bc_one(j);
             }
-            load_batch(l0 + t0 + 4);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float dt = softplus_f(cd[i] + bias);
-                const float u = cx[i];
-                const float2 dt2 = make_float2(dt, dt);
+                const int t = j * 4 + i;
+                const float raw = td[t * TROW + lane];
+                const float u = tx[t * TROW + lane];
+                const float dt = (l0 + t < l_end) ? softplus_f(raw + bias) : 0.f;
+                dtsum += dt;
                 const float du = dt * u;
+                const float2 dt2 = make_float2(dt, dt);
                 const float2 du2 = make_float2(du, du);
-                const float4 *row = sb + (t0 + i) * 8;
+                const float4 *row = sb + t * 8;
+                const int sw = t & 7;
                 float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float4 bv = row[q];
-                    const float4 cv = row[4 + q];
+                    const float4 bv = row[q ^ sw];
                     const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
                     const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
                     const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
@@ -366,381 +316,129 @@ __global__ void __launch_bounds__(32 * WC, MINB) scan_direct_kernel(const ScanPa
                     h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
                     h2[2 * q + 1] =
                         __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                    acc = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc);
-                    acc = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc);
+                    if (MODE == kModeOutput) {
+                        const float4 cv = row[(4 + q) ^ sw];
+                        acc = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc);
+                        acc = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc);
+                    }
                 }
-                const float yv = fmaf(dsk, u, acc.x + acc.y);
-                if (cvalid && l0 + t0 + i < L)
-                    og[cp[i]] = yv;
+                if (MODE == kModeOutput)
+                    sY[t * TROW + lane] = fmaf(dsk, u, acc.x + acc.y);
             }
         }
-        if (more)
-            store_bc(buf ^ 1);
-        __syncthreads();
-    }
-    if (p.merge) {
-        const int nc = min(NT, D - d0);
-        merge_epilogue(p, b, tile, d0, nc, NT);
-    }
-}
-
-// ===========================================================================
-// scan_split_kernel: four lanes per channel, sequence split in time
-// ===========================================================================
-// 16-byte asynchronous copy global -> shared (cp.async.cg); with src_bytes = 0
-// nothing is read and the 16 destination bytes are zero-filled.
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
-{
-    const unsigned int s = (unsigned int)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
-
-template <typename Tin, int JW, int J, int I>
-struct SplitShape {
-    static constexpr int G = 4;                  // lanes per channel
-    static constexpr int S = kNP / G;            // states per lane (4)
-    static constexpr int CW = 32 / (G * JW);     // channels per warp = per CTA
-    static constexpr int DC = CW;
-    static constexpr int NT = 32 * J;            // threads
-    static constexpr int NS = J * JW;            // time segments per chunk
-    static constexpr int LC = NS * I;            // steps per chunk
-    static constexpr int ESZ = sizeof(Tin);
-    static constexpr int EPP = 16 / ESZ;         // elements per 16-byte piece
-    static constexpr int PPR = LC / EPP;         // pieces per raw row
-    static constexpr int RAWROW = LC + EPP;      // raw row stride in elements (16 B pad)
-    static constexpr int RAW_ROWS = 2 * kNP + DC;        // B rows, C rows, delta rows
-    static constexpr int RAW_ELEMS = RAW_ROWS * RAWROW;  // per raw buffer
-    static constexpr int SEG = I + 4;            // padded segment in channel rows
-    static constexpr int RS0 = NS * SEG;
-    static constexpr int RS = RS0 + (((RS0 / 4) % 2 == 0) ? 4 : 8);   // channel row stride
-    static constexpr int BSEG4 = I * 8 + 4;      // padded segment of the B|C tile (float4)
-    static constexpr int TILE4 = NS * BSEG4;     // float4 in the B|C tile
-    static constexpr int ROWF = DC * RS;         // floats per dt / dt*u / u tile
-    static constexpr int NE = LC * 8;            // B|C float4 entries per chunk
-    static constexpr int NR = DC * LC;           // (channel, step) elements per chunk
-    static constexpr int RPT = (NR + NT - 1) / NT;
-    static constexpr int NPIECE = RAW_ROWS * PPR;        // 16-byte copies per chunk
-    static constexpr size_t RAW_BYTES = (size_t)ESZ * 2 * RAW_ELEMS;
-    static constexpr size_t SMEM_BYTES =
-        RAW_BYTES + sizeof(float4) * TILE4 + sizeof(float) * 3 * ROWF + sizeof(int) * LC +
-        sizeof(float) * (J > 1 ? (J * DC * kNP * 2 + 2 * DC * kNP) : 0);
-    static_assert(I % 4 == 0, "segments hold whole groups of four steps");
-    static_assert(LC % EPP == 0, "chunks are whole 16-byte pieces");
-    static_assert(32 % (G * JW) == 0 && CW >= 1, "lanes split evenly");
-    static_assert((RAW_BYTES % 16) == 0, "raw buffers keep 16-byte alignment");
-};
-
-template <typename Tin, int JW, int J, int I, int MINB>
-__global__ void __launch_bounds__(32 * J, MINB) scan_split_kernel(const ScanParams p)
-{
-    using Sh = SplitShape<Tin, JW, J, I>;
-    constexpr int G = Sh::G, DC = Sh::DC, NT = Sh::NT, LC = Sh::LC;
-    constexpr int SEG = Sh::SEG, RS = Sh::RS, BSEG4 = Sh::BSEG4;
-    constexpr int RPT = Sh::RPT, NE = Sh::NE, NR = Sh::NR;
-    constexpr int EPP = Sh::EPP, PPR = Sh::PPR, RAWROW = Sh::RAWROW;
-
-    extern __shared__ float4 smem_f4[];
-    Tin *sRaw = reinterpret_cast<Tin *>(smem_f4);                   // [2][RAW_ROWS][RAWROW]
-    float4 *sBC = reinterpret_cast<float4 *>(reinterpret_cast<char *>(smem_f4) + Sh::RAW_BYTES);
-    float *sDt = reinterpret_cast<float *>(sBC + Sh::TILE4);        // [DC][RS]
-    float *sDu = sDt + Sh::ROWF;
-    float *sU = sDu + Sh::ROWF;
-    int *sPix = reinterpret_cast<int *>(sU + Sh::ROWF);             // [LC]
-    float *sTot = reinterpret_cast<float *>(sPix + LC);             // [J][DC][kNP][2]
-    float *sCar = sTot + J * DC * kNP * 2;                          // [2][DC][kNP]
-
-    const int tid = threadIdx.x;
-    const int lane = tid & 31, j = tid >> 5;
-    const int g = lane % G;
-    const int jw = (lane / G) % JW;
-    const int c = lane / (G * JW);
-    const int js = j * JW + jw;
-
-    const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W;
-    const int k = blockIdx.x, tile = blockIdx.y, b = blockIdx.z;
-    const int d0 = tile * DC;
-    const int d = d0 + c;
-    const bool cvalid = d < D;
-    const int kd = k * D + (cvalid ? d : 0);
-
-    float2 A2[2];
-    {
-        const int n0 = g * 4;
-        float a[4];
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            a[s] = (cvalid && n0 + s < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0 + s)) * kLog2e
-                                          : 0.f;
-        A2[0] = make_float2(a[0], a[1]);
-        A2[1] = make_float2(a[2], a[3]);
-    }
-    const float dsk = cvalid ? __ldg(p.Dskip + kd) : 0.f;
-
-    const Tin *xg = static_cast<const Tin *>(p.x) + (size_t)b * D * L;
-    const Tin *dg = static_cast<const Tin *>(p.delta) + ((size_t)b * p.K + k) * D * L;
-    const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * p.K + k) * N * L;
-    const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * p.K + k) * N * L;
-    const float *biasg = p.delta_bias + (size_t)k * D;
-    float *og = p.out + (size_t)b * p.out_b_stride + (size_t)k * p.out_k_stride +
-                (size_t)(cvalid ? d : 0) * L;
-    // rows start on 16-byte boundaries: copy 16-byte pieces asynchronously;
-    // otherwise fall back to element loads
-    const bool async_ok = ((L * (int)sizeof(Tin)) % 16) == 0 &&
-                          (((uintptr_t)p.delta | (uintptr_t)p.Bs | (uintptr_t)p.Cs) & 15) == 0;
-
-    // raw row r of a chunk: B rows 0..15, C rows 16..31, delta rows 32..32+DC-1
-    auto row_src = [&](int r) -> const Tin * {
-        if (r < kNP)
-            return r < N ? Bg + (size_t)r * L : nullptr;
-        if (r < 2 * kNP)
-            return (r - kNP) < N ? Cg + (size_t)(r - kNP) * L : nullptr;
-        const int dd = d0 + (r - 2 * kNP);
-        return dd < D ? dg + (size_t)dd * L : nullptr;
-    };
-    auto stage_raw = [&](int rb, int l0) {
-        Tin *dst0 = sRaw + rb * Sh::RAW_ELEMS;
-        if (async_ok) {
-            for (int e = tid; e < Sh::NPIECE; e += NT) {
-                const int r = e / PPR, q = e % PPR;
-                const int l = l0 + q * EPP;
-                const Tin *src = row_src(r);
-                const bool ok = src != nullptr && l < L;
-                cp_async16(dst0 + r * RAWROW + q * EPP, ok ? src + l : p.Bs, ok ? 16 : 0);
-            }
-            cp_async_commit();
-        } else {
-            for (int e = tid; e < Sh::RAW_ROWS * LC; e += NT) {
-                const int r = e / LC, t = e % LC;
-                const int l = l0 + t;
-                const Tin *src = row_src(r);
-                dst0[r * RAWROW + t] = (src != nullptr && l < L) ? src[l] : Tin(0.f);
-            }
-        }
-    };
-
-    // x of a chunk: register prefetch through per-thread pixel walkers;
-    // (channel, step) element e = tid + r*NT: step e % LC, channel e / LC
-    PixWalk rw[RPT];
-    const int nq = LC / H, nr = LC % H;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r)
-        rw[r].init(p.two_d, k, (tid + r * NT) % LC, H, W, L);
-    float rx[RPT];
-    auto load_x = [&](int l0) {
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) {
-            const int e = tid + r * NT;
-            const int t = e % LC, cc = e / LC;
-            const int l = l0 + t, dd = d0 + cc;
-            const bool ok = (e < NR) && l < L && dd < D;
-            rx[r] = ok ? load_in(xg + (size_t)dd * L + rw[r].p) : 0.f;
-        }
-    };
-    // raw chunk -> float32 tiles: B|C as [segment][step][8 float4], dt, dt*u, u
-    // as [channel][segment][step], and the chunk's pixel table
-    auto convert = [&](int rb, int l0) {
-        const Tin *raw = sRaw + rb * Sh::RAW_ELEMS;
-        for (int e = tid; e < NE; e += NT) {
-            const int q = e & 7, t = e >> 3;
-            const Tin *src = raw + ((q < 4 ? 0 : kNP) + (q & 3) * 4) * RAWROW + t;
-            sBC[(t / I) * BSEG4 + (t % I) * 8 + q] =
-                make_float4(load_in_smem(src), load_in_smem(src + RAWROW),
-                            load_in_smem(src + 2 * RAWROW), load_in_smem(src + 3 * RAWROW));
-        }
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) {
-            const int e = tid + r * NT;
-            if (e < NR) {
-                const int t = e % LC, cc = e / LC;
-                const int l = l0 + t, dd = d0 + cc;
-                const bool ok = l < L && dd < D;
-                const float z = load_in_smem(raw + (2 * kNP + cc) * RAWROW + t);
-                const float dt = ok ? softplus_f(z + __ldg(biasg + dd)) : 0.f;
-                const int si = cc * RS + (t / I) * SEG + (t % I);
-                sDt[si] = dt;
-                sDu[si] = dt * rx[r];
-                sU[si] = rx[r];
-                if (cc == 0)
-                    sPix[t] = rw[r].p;
-            }
-            rw[r].advance(LC, nq, nr, H, W);
-        }
-    };
-
-    // zero both raw buffers once, so steps past the end of the sequence read
-    // finite zeros
-    {
-        float4 *z = smem_f4;
-        for (int e = tid; e < (int)(Sh::RAW_BYTES / 16); e += NT)
-            z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float2 hcar[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    if constexpr (J > 1) {
-        for (int e = tid; e < 2 * DC * kNP; e += NT)
-            sCar[e] = 0.f;
-    }
-    __syncthreads();
-    stage_raw(0, 0);
-    load_x(0);
-
-    int rb = 0, chunk = 0;
-    for (int l0 = 0; l0 < L; l0 += LC, rb ^= 1, ++chunk) {
-        const bool more = l0 + LC < L;
-        if (async_ok)
-            cp_async_wait_all();
-        __syncthreads();
-        convert(rb, l0);
-        __syncthreads();
         if (more) {
-            stage_raw(rb ^ 1, l0 + LC);
-            load_x(l0 + LC);
+            store_dx(buf ^ 1, 7);
+            store_bc(buf ^ 1);
         }
-        const float4 *tb = sBC + js * BSEG4 + g;
-        const float *dtb = sDt + c * RS + js * SEG;
-        const float *dub = sDu + c * RS + js * SEG;
-        const float *ub = sU + c * RS + js * SEG;
-
-        // pass 1: the segment from a zero state; keep exp(dt*A)
-        float2 av[I][2];
-        float2 P[2] = {make_float2(1.f, 1.f), make_float2(1.f, 1.f)};
-        float2 Q[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int i0 = 0; i0 < I; i0 += 4) {
-            const float4 dt4 = *reinterpret_cast<const float4 *>(dtb + i0);
-            const float4 du4 = *reinterpret_cast<const float4 *>(dub + i0);
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int i = i0 + ii;
-                const float dt = f4(dt4, ii), du = f4(du4, ii);
-                const float2 dt2 = make_float2(dt, dt), du2 = make_float2(du, du);
-                const float4 bv = tb[i * 8];
-                const float2 arg0 = __fmul2_rn(dt2, A2[0]);
-                const float2 arg1 = __fmul2_rn(dt2, A2[1]);
-                av[i][0] = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
-                av[i][1] = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
-                Q[0] = __ffma2_rn(av[i][0], Q[0], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
-                Q[1] = __ffma2_rn(av[i][1], Q[1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                P[0] = __fmul2_rn(P[0], av[i][0]);
-                P[1] = __fmul2_rn(P[1], av[i][1]);
-            }
-        }
-        // inclusive scan of the transfer pairs over the warp's segments
-#pragma unroll
-        for (int rr = 1; rr < JW; rr <<= 1) {
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                float2 Pp, Qp;
-                Pp.x = __shfl_up_sync(0xffffffffu, P[s].x, rr * G);
-                Pp.y = __shfl_up_sync(0xffffffffu, P[s].y, rr * G);
-                Qp.x = __shfl_up_sync(0xffffffffu, Q[s].x, rr * G);
-                Qp.y = __shfl_up_sync(0xffffffffu, Q[s].y, rr * G);
-                if (jw >= rr) {
-                    Q[s] = __ffma2_rn(P[s], Qp, Q[s]);
-                    P[s] = __fmul2_rn(P[s], Pp);
+        if (MODE == kModeOutput) {
+            // the sub-chunk's outputs, one channel (32 consecutive steps) per store
+            __syncwarp();
+            const int l = l0 + lane;
+            if (l < l_end) {
+                float *orow = p.out + (row_bk + wd0) * L + l;
+#pragma unroll 4
+                for (int cc = 0; cc < 32; ++cc) {
+                    if (wd0 + cc < D)
+                        orow[(size_t)cc * L] = sY[lane * TROW + cc];
                 }
             }
+            __syncwarp();
         }
-        float2 Pex[2], Qex[2];   // segments of this warp before mine
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            float2 Pp, Qp;
-            Pp.x = __shfl_up_sync(0xffffffffu, P[s].x, G);
-            Pp.y = __shfl_up_sync(0xffffffffu, P[s].y, G);
-            Qp.x = __shfl_up_sync(0xffffffffu, Q[s].x, G);
-            Qp.y = __shfl_up_sync(0xffffffffu, Q[s].y, G);
-            Pex[s] = (jw == 0) ? make_float2(1.f, 1.f) : Pp;
-            Qex[s] = (jw == 0) ? make_float2(0.f, 0.f) : Qp;
-        }
-        float2 hw[2];   // state entering this warp's first segment
-        if constexpr (J == 1) {
-            const int last = (c * JW + JW - 1) * G + g;
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                hw[s] = hcar[s];
-                float2 Pt, Qt;
-                Pt.x = __shfl_sync(0xffffffffu, P[s].x, last);
-                Pt.y = __shfl_sync(0xffffffffu, P[s].y, last);
-                Qt.x = __shfl_sync(0xffffffffu, Q[s].x, last);
-                Qt.y = __shfl_sync(0xffffffffu, Q[s].y, last);
-                hcar[s] = __ffma2_rn(Pt, hcar[s], Qt);
-            }
-        } else {
-            if (jw == JW - 1) {
-                float4 *dst = reinterpret_cast<float4 *>(sTot + ((j * DC + c) * kNP + g * 4) * 2);
-                dst[0] = make_float4(P[0].x, Q[0].x, P[0].y, Q[0].y);
-                dst[1] = make_float4(P[1].x, Q[1].x, P[1].y, Q[1].y);
-            }
-            __syncthreads();
-            const float *car = sCar + (chunk & 1) * DC * kNP + c * kNP + g * 4;
-            float hc[4] = {car[0], car[1], car[2], car[3]};
-            for (int jj = 0; jj < j; ++jj) {
-                const float4 *tot =
-                    reinterpret_cast<const float4 *>(sTot + ((jj * DC + c) * kNP + g * 4) * 2);
-                const float4 t0 = tot[0], t1 = tot[1];
-                hc[0] = fmaf(t0.x, hc[0], t0.y);
-                hc[1] = fmaf(t0.z, hc[1], t0.w);
-                hc[2] = fmaf(t1.x, hc[2], t1.y);
-                hc[3] = fmaf(t1.z, hc[3], t1.w);
-            }
-            hw[0] = make_float2(hc[0], hc[1]);
-            hw[1] = make_float2(hc[2], hc[3]);
-            if (j == J - 1 && jw == JW - 1) {
-                float *ncar = sCar + ((chunk + 1) & 1) * DC * kNP + c * kNP + g * 4;
-                const float2 n0 = __ffma2_rn(P[0], hw[0], Q[0]);
-                const float2 n1 = __ffma2_rn(P[1], hw[1], Q[1]);
-                ncar[0] = n0.x;
-                ncar[1] = n0.y;
-                ncar[2] = n1.x;
-                ncar[3] = n1.y;
-            }
-        }
-        // pass 2: replay the segment from its entry state
-        float2 h[2];
-        h[0] = __ffma2_rn(Pex[0], hw[0], Qex[0]);
-        h[1] = __ffma2_rn(Pex[1], hw[1], Qex[1]);
-        const int *pix = sPix + js * I;
-#pragma unroll
-        for (int i0 = 0; i0 < I; i0 += 4) {
-            const float4 du4 = *reinterpret_cast<const float4 *>(dub + i0);
-            float yp[4];
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int i = i0 + ii;
-                const float du = f4(du4, ii);
-                const float2 du2 = make_float2(du, du);
-                const float4 bv = tb[i * 8];
-                const float4 cv = tb[i * 8 + 4];
-                h[0] = __ffma2_rn(av[i][0], h[0], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
-                h[1] = __ffma2_rn(av[i][1], h[1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                float2 acc = __fmul2_rn(make_float2(cv.x, cv.y), h[0]);
-                acc = __ffma2_rn(make_float2(cv.z, cv.w), h[1], acc);
-                yp[ii] = acc.x + acc.y;
-            }
-            // sum the four lanes of the channel; lane g keeps step i0 + g
-            const bool b1 = (g >> 1) & 1;
-            const float s0 = b1 ? yp[0] : yp[2];
-            const float s1 = b1 ? yp[1] : yp[3];
-            float k0 = b1 ? yp[2] : yp[0];
-            float k1 = b1 ? yp[3] : yp[1];
-            k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-            k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-            const bool b0 = g & 1;
-            const float sx = b0 ? k0 : k1;
-            float v = b0 ? k1 : k0;
-            v += __shfl_xor_sync(0xffffffffu, sx, 1);
-            const int t = js * I + i0 + g;
-            if (cvalid && l0 + t < L)
-                og[pix[i0 + g]] = fmaf(dsk, ub[i0 + g], v);
-        }
-    }
-    if (p.merge) {
         __syncthreads();
-        const int nc = min(DC, D - d0);
-        merge_epilogue(p, b, tile, d0, nc, NT);
+    }
+
+    if (MODE == kModeState && cvalid) {
+        float4 *hs = reinterpret_cast<float4 *>(
+            p.hstate + ((row_bk + d) * (p.NC - 1) + chunk) * kNP);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            hs[q] = make_float4(h2[2 * q].x, h2[2 * q].y, h2[2 * q + 1].x, h2[2 * q + 1].y);
+        p.dtsum[(row_bk + d) * (p.NC - 1) + chunk] = dtsum;
+    }
+}
+
+// Entry states of every chunk after the first, in place over the chunk end
+// states: slot c of (b,k,d) holds h_end of chunk c on entry and h_in of chunk
+// c+1 on exit.  One thread per (b, k, d, n).
+__global__ void carry_kernel(const ScanParams p)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)p.B * p.K * p.D * kNP;
+    if (idx >= total)
+        return;
+    const int n = (int)(idx % kNP);
+    const long long bkd = idx / kNP;
+    const int d = (int)(bkd % p.D);
+    const int k = (int)((bkd / p.D) % p.K);
+    const float a2 =
+        n < p.N ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.N + n)) * kLog2e : 0.f;
+    float *hs = p.hstate + (size_t)bkd * (p.NC - 1) * kNP + n;
+    const float *ds = p.dtsum + (size_t)bkd * (p.NC - 1);
+    float h = 0.f;
+    for (int c = 0; c < p.NC - 1; ++c) {
+        h = fmaf(mufu_ex2(a2 * ds[c]), h, hs[(size_t)c * kNP]);
+        hs[(size_t)c * kNP] = h;
+    }
+}
+
+// cross_merge: scan-order rows part[(b,k,d)][l] -> pixel order.  One CTA per
+// (b, d, band of kMergeRows image rows).  The column-major directions are
+// gathered through a shared-memory tile so that global reads stay coalesced
+// (each image column's band is a run of consecutive scan steps).
+//   sum = 1: y[b,d,p] = ((Y_0 + Y_1) + Y_2) + Y_3       (first K terms)
+//   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
+// A 1D sequence is a single image row (H = 1, W = L).
+__global__ void merge_kernel(const float *__restrict__ part, float *__restrict__ y, int B,
+                             int D, int H, int W, int K, int two_d, int sum)
+{
+    constexpr int R = kMergeRows;
+    extern __shared__ float smem_m[];   // [2][W][R + 1] for k = 2, 3
+    const int L = H * W;
+    const int nblk = (H + R - 1) / R;
+    const int blk = blockIdx.x % nblk;
+    const int bd = blockIdx.x / nblk;
+    const int b = bd / D, d = bd % D;
+    const int h0 = blk * R;
+    const int hr = min(R, H - h0);
+    const int np = hr * W;
+    const int p0 = h0 * W;
+    const float *rows = part + ((size_t)b * K * D + d) * L;   // row of (b, k = 0, d)
+    const size_t kstride = (size_t)D * L;
+    const bool cols = two_d && K == 4;
+    if (cols) {
+        for (int e = threadIdx.x; e < W * hr; e += blockDim.x) {
+            const int w = e / hr, hh = e % hr;
+            const int s2 = w * H + h0 + hh;
+            smem_m[w * (R + 1) + hh] = __ldg(rows + 2 * kstride + s2);
+            smem_m[(W + w) * (R + 1) + hh] = __ldg(rows + 3 * kstride + (L - 1 - s2));
+        }
+        __syncthreads();
+    }
+    for (int e = threadIdx.x; e < np; e += blockDim.x) {
+        const int pix = p0 + e;
+        float v[4];
+        v[0] = __ldg(rows + pix);
+        v[1] = (K >= 2) ? __ldg(rows + kstride + (L - 1 - pix)) : 0.f;
+        if (cols) {
+            const int hh = e / W, w = e % W;
+            v[2] = smem_m[w * (R + 1) + hh];
+            v[3] = smem_m[(W + w) * (R + 1) + hh];
+        } else {
+            v[2] = v[3] = 0.f;
+        }
+        if (sum) {
+            float acc = v[0];
+            if (K >= 2)
+                acc += v[1];
+            if (K == 4) {
+                acc += v[2];
+                acc += v[3];
+            }
+            y[((size_t)b * D + d) * L + pix] = acc;
+        } else {
+            for (int kk = 0; kk < K; ++kk)
+                y[(((size_t)b * K + kk) * D + d) * L + pix] = v[kk];
+        }
     }
 }
 

@@ -1,4 +1,4 @@
-// ss2d_launch.cu -- the table of kernel variants and their launchers.
+// ss2d_launch.cu -- kernel variants, the execution plan of a call, launchers.
 #include "ss2d_launch.h"
 
 #include <cuda_bf16.h>
@@ -9,20 +9,26 @@ namespace ss2d {
 
 namespace {
 
-template <typename Tin, int WC, int LC, int MINB>
-cudaError_t launch_direct(const ScanParams &p, cudaStream_t st)
-{
-    using Sh = DirectShape<WC, LC>;
-    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT), (unsigned)p.B);
-    scan_direct_kernel<Tin, WC, LC, MINB><<<grid, Sh::NT, 0, st>>>(p);
-    return cudaGetLastError();
-}
+// name: wc<W>_<chunking>; wc = 32-channel warps per CTA.
+const VariantInfo kVariants[] = {
+    {"wc2_auto", 2, 0},    {"wc4_auto", 4, 0},    {"wc1_auto", 1, 0},
+    {"wc2_lc32", 2, 32},   {"wc4_lc64", 4, 64},   {"wc2_nochunk", 2, -1},
+    {"wc2_lc256", 2, 256}, {"wc4_lc512", 4, 512}, {"wc1_lc128", 1, 128},
+};
+constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
-template <typename Tin, int JW, int J, int I, int MINB>
-cudaError_t launch_split(const ScanParams &p, cudaStream_t st)
+// Minimum resident CTAs per SM the kernels are compiled for: a register cap
+// of 65536 / (32 * WC * MINB) = 128 per thread.
+template <int WC>
+struct MinBlocks {
+    static constexpr int value = 16 / WC;
+};
+
+template <typename Tin, int WC, int MODE>
+cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
 {
-    using Sh = SplitShape<Tin, JW, J, I>;
-    auto kern = scan_split_kernel<Tin, JW, J, I, MINB>;
+    using Sh = ChunkShape<WC>;
+    auto kern = chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC>::value>;
     const size_t smem = Sh::SMEM_BYTES;
     if (smem > 48 * 1024) {
         cudaError_t e =
@@ -30,64 +36,37 @@ cudaError_t launch_split(const ScanParams &p, cudaStream_t st)
         if (e != cudaSuccess)
             return e;
     }
-    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::DC - 1) / Sh::DC), (unsigned)p.B);
+    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT), (unsigned)(p.B * ncg));
     kern<<<grid, Sh::NT, smem, st>>>(p);
     return cudaGetLastError();
 }
 
-template <int WC, int LC, int MINB>
-VariantInfo direct_variant(const char *name)
+template <typename Tin, int WC>
+cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
 {
-    using Sh = DirectShape<WC, LC>;
-    VariantInfo v{};
-    v.name = name;
-    v.split = 0;
-    v.channels_per_cta = Sh::NT;
-    v.threads = Sh::NT;
-    v.chunk = LC;
-    v.segments = 1;
-    v.smem_bytes = sizeof(float4) * 2 * LC * 8;
-    v.launch_f32 = &launch_direct<float, WC, LC, MINB>;
-    v.launch_bf16 = &launch_direct<__nv_bfloat16, WC, LC, MINB>;
-    return v;
+    cudaError_t e;
+    if (plan.NC > 1) {
+        if (ev)
+            cudaEventRecord(ev[0], st);
+        e = launch_chunk<Tin, WC, kModeState>(p, plan.NC - 1, st);
+        if (e != cudaSuccess)
+            return e;
+        if (ev)
+            cudaEventRecord(ev[1], st);
+        const long long total = (long long)p.B * p.K * p.D * kNP;
+        const int threads = 256;
+        carry_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, st>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    if (ev)
+        cudaEventRecord(ev[2], st);
+    e = launch_chunk<Tin, WC, kModeOutput>(p, plan.NC, st);
+    if (ev)
+        cudaEventRecord(ev[3], st);
+    return e;
 }
-
-template <int JW, int J, int I, int MINB>
-VariantInfo split_variant(const char *name)
-{
-    using Sh = SplitShape<__nv_bfloat16, JW, J, I>;
-    VariantInfo v{};
-    v.name = name;
-    v.split = 1;
-    v.channels_per_cta = Sh::DC;
-    v.threads = Sh::NT;
-    v.chunk = Sh::LC;
-    v.segments = Sh::NS;
-    v.smem_bytes = Sh::SMEM_BYTES;
-    v.launch_f32 = &launch_split<float, JW, J, I, MINB>;
-    v.launch_bf16 = &launch_split<__nv_bfloat16, JW, J, I, MINB>;
-    return v;
-}
-
-// direct_wc<W>_lc<LC>: 32*W threads, one channel per thread, chunks of LC steps.
-// split_jw<JW>_j<J>_i<I>: 4 lanes per channel, JW segments per warp, J warps,
-// I steps per segment.
-const VariantInfo kVariants[] = {
-    direct_variant<4, 64, 4>("direct_wc4_lc64"),
-    direct_variant<2, 64, 6>("direct_wc2_lc64"),
-    direct_variant<4, 32, 4>("direct_wc4_lc32"),
-    split_variant<2, 4, 16, 4>("split_jw2_j4_i16"),
-    split_variant<2, 2, 16, 8>("split_jw2_j2_i16"),
-    split_variant<1, 4, 16, 4>("split_jw1_j4_i16"),
-    split_variant<4, 2, 16, 8>("split_jw4_j2_i16"),
-    split_variant<4, 4, 16, 4>("split_jw4_j4_i16"),
-    split_variant<8, 2, 16, 8>("split_jw8_j2_i16"),
-    split_variant<8, 4, 16, 4>("split_jw8_j4_i16"),
-    split_variant<8, 1, 16, 8>("split_jw8_j1_i16"),
-    split_variant<1, 8, 16, 2>("split_jw1_j8_i16"),
-    split_variant<2, 1, 16, 8>("split_jw2_j1_i16"),
-};
-constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
 }  // namespace
 
@@ -103,29 +82,85 @@ const VariantInfo *variant(int i)
 int pick_variant(int two_d, int B, int D, int H, int W, int N, int K)
 {
     (void)two_d;
+    (void)B;
+    (void)H;
+    (void)W;
     (void)N;
-    const long long L = (long long)H * W;
-    const long long seqs = (long long)B * K * D;
-    // Lanes wanted resident at once: about four warps per SM sub-partition.
-    const long long want = 148LL * 4 * 4 * 32;
-    if (seqs * 2 >= want || L <= 256)
-        return 0;                                 // direct_wc4_lc64
-    const long long lanes4 = seqs * 4;            // split: 4 lanes per channel
-    if (lanes4 * 4 >= want)
-        return 4;                                 // split_jw2_j2 (4 segments)
-    if (lanes4 * 8 >= want)
-        return 6;                                 // split_jw4_j2 (8 segments)
-    if (lanes4 * 16 >= want)
-        return 8;                                 // split_jw8_j2 (16 segments)
-    return 9;                                     // split_jw8_j4 (32 segments)
+    (void)K;
+    if (D <= 32)
+        return 2;   // wc1_auto
+    return 0;       // wc2_auto
 }
 
-cudaError_t launch_scan_variant(int v, bool bf16, const ScanParams &p, cudaStream_t st)
+Plan make_plan(int v, int B, int D, int L, int K)
 {
     const VariantInfo *vi = variant(v);
-    if (!vi)
+    Plan pl;
+    pl.variant = v;
+    pl.wc = vi->wc;
+    int lc;
+    if (vi->chunk > 0) {
+        lc = vi->chunk;
+    } else if (vi->chunk < 0) {
+        lc = L;
+    } else {
+        // enough lanes for about four resident warps per SM sub-partition on
+        // 148 SMs; short sequences are never split
+        const long long want = 148LL * 16 * 32;
+        const long long seqs = (long long)B * K * D;
+        long long nc = (seqs >= want / 2 || L <= 512) ? 1 : (want + seqs - 1) / seqs;
+        if (nc < 1)
+            nc = 1;
+        lc = (int)((L + nc - 1) / nc);
+    }
+    lc = ((lc + kT - 1) / kT) * kT;
+    if (lc < kT)
+        lc = kT;
+    pl.LC = lc;
+    pl.NC = (L + lc - 1) / lc;
+    pl.launches = (pl.NC > 1 ? 3 : 1) + (K > 1 ? 1 : 0);
+    return pl;
+}
+
+cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t st,
+                        cudaEvent_t *ev)
+{
+    p.LC = plan.LC;
+    p.NC = plan.NC;
+    switch (plan.wc) {
+    case 1:
+        return bf16 ? launch_passes<__nv_bfloat16, 1>(plan, p, st, ev)
+                    : launch_passes<float, 1>(plan, p, st, ev);
+    case 2:
+        return bf16 ? launch_passes<__nv_bfloat16, 2>(plan, p, st, ev)
+                    : launch_passes<float, 2>(plan, p, st, ev);
+    case 4:
+        return bf16 ? launch_passes<__nv_bfloat16, 4>(plan, p, st, ev)
+                    : launch_passes<float, 4>(plan, p, st, ev);
+    default:
         return cudaErrorInvalidValue;
-    return bf16 ? vi->launch_bf16(p, st) : vi->launch_f32(p, st);
+    }
+}
+
+size_t merge_smem_bytes(int W, int K, int two_d)
+{
+    return (two_d && K == 4) ? sizeof(float) * 2 * (size_t)W * (kMergeRows + 1) : 0;
+}
+
+cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
+                         int two_d, int sum, cudaStream_t st)
+{
+    const size_t smem = merge_smem_bytes(W, K, two_d);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(merge_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    const int nblk = (H + kMergeRows - 1) / kMergeRows;
+    const long long grid = (long long)B * D * nblk;
+    merge_kernel<<<(unsigned)grid, 256, smem, st>>>(part, y, B, D, H, W, K, two_d, sum);
+    return cudaGetLastError();
 }
 
 }  // namespace ss2d

@@ -8,21 +8,39 @@ namespace ss2d {
 
 struct ScanParams;
 
+// A kernel variant: CTA width (32*wc channels) and chunking policy
+// (chunk = 0: chosen from the shape; chunk > 0: that many steps per chunk;
+// chunk < 0: never chunk).
 struct VariantInfo {
     const char *name;
-    int split;             // 0: one lane per channel; 1: time-split, 4 lanes per channel
-    int channels_per_cta;  // channel tile; one ticket per (batch, tile) when merging
-    int threads;
-    int chunk;             // steps staged per chunk
-    int segments;          // time segments per chunk
-    size_t smem_bytes;
-    cudaError_t (*launch_f32)(const ScanParams &, cudaStream_t);
-    cudaError_t (*launch_bf16)(const ScanParams &, cudaStream_t);
+    int wc;
+    int chunk;
+};
+
+// How one call is executed.
+struct Plan {
+    int variant;
+    int wc;
+    int LC;        // steps per chunk (multiple of 32)
+    int NC;        // chunks per sequence
+    int launches;  // kernel launches of a forward call
 };
 
 int num_variants();
 const VariantInfo *variant(int i);
 int pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
-cudaError_t launch_scan_variant(int v, bool bf16, const ScanParams &p, cudaStream_t st);
+Plan make_plan(int variant, int B, int D, int L, int K);
+
+// Launch the scan passes (state, carry, output) for a plan; the caller has
+// set p.out (and p.hstate / p.dtsum when plan.NC > 1).  If ev is not null,
+// ev[0..3] are recorded on the stream before the state pass, the carry, the
+// output pass and after it (the first two only when the plan is chunked).
+cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t st,
+                        cudaEvent_t *ev = nullptr);
+// cross_merge of the scan-order rows in `part` into y (sum = 1) or into the
+// per-direction pixel-order copy (sum = 0).
+cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
+                         int two_d, int sum, cudaStream_t st);
+size_t merge_smem_bytes(int W, int K, int two_d);
 
 }  // namespace ss2d

@@ -1,0 +1,30 @@
+// ss2d_params.h -- launch parameters and constants shared by the C ABI and
+// the kernels.
+#pragma once
+
+namespace ss2d {
+
+constexpr int kNP = 16;     // states per channel held by the kernels (N <= 16)
+constexpr int kT = 32;      // steps per sub-chunk
+constexpr int kMergeRows = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct ScanParams {
+    const void *x;            // (B,D,H,W) / (B,D,L)
+    const void *delta;        // (B,K,D,L) scan order
+    const float *A_log;       // (K*D,N)
+    const void *Bs;           // (B,K,N,L) scan order
+    const void *Cs;           // (B,K,N,L) scan order
+    const float *Dskip;       // (K*D)
+    const float *delta_bias;  // (K*D)
+    float *out;               // y_k in scan order, row (b,k,d) at out + ((b*K+k)*D+d)*L
+                              // (K = 1: y itself)
+    float *hstate;            // (B,K,D,NC-1,16): chunk end states, then entry states
+    float *dtsum;             // (B,K,D,NC-1): sum of dt over every chunk but the last
+    int B, D, H, W, L, N, K;
+    int two_d;                // 1: SS2D scan orders; 0: 1D (k = 1 reversed)
+    int LC;                   // steps per chunk (multiple of kT)
+    int NC;                   // chunks per sequence
+};
+
+}  // namespace ss2d

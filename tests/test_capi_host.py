@@ -114,3 +114,18 @@ def test_binding_validates_tensors(lib):
     with pytest.raises(ValueError):
         binding.ss2d_forward(x, delta, A_log, Bs.transpose(2, 3).contiguous().transpose(2, 3),
                              Bs, Dk, Dk)
+
+
+def test_plans_for_the_workloads(lib):
+    from selective_scan_ss2d_b200 import workloads as wl
+    for name, cfg in wl.CONFIGS.items():
+        pl = binding.ss2d_plan(cfg.kind == "2d", cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K)
+        assert pl["chunk_len"] % 32 == 0
+        assert pl["num_chunks"] == -(-cfg.L // pl["chunk_len"])
+        want = (3 if pl["num_chunks"] > 1 else 1) + (1 if cfg.K > 1 else 0)
+        assert pl["launches"] == want
+    # long sequences with few channels are chunked, short ones are not
+    t = wl.CONFIGS["vmamba_t_stage1"]
+    assert binding.ss2d_plan(True, t.B, t.D, t.H, t.W, t.N, t.K)["num_chunks"] > 1
+    b = wl.CONFIGS["vmamba_b_stage3"]
+    assert binding.ss2d_plan(True, b.B, b.D, b.H, b.W, b.N, b.K)["num_chunks"] == 1

@@ -194,3 +194,40 @@ def test_full_size_sampled_channels(name):
         want.append(_gpu.run_oracle(sub)[0, 0].reshape(-1))
         got.append(y[b, d].reshape(-1))
     _gpu.assert_close(np.concatenate(got), np.concatenate(want), cfg.dtype, name)
+
+
+# ---------------------------------------------------------------------------
+# per-direction outputs and the timed call
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("cfg", [small(B=2, D=40, H=7, W=9, K=4), small(B=1, D=33, H=20, W=12, K=2),
+                                 small("1d", B=2, D=33, W=100, K=2)],
+                         ids=lambda c: c.name)
+def test_scan_directions_match_oracle(cfg):
+    inp = wl.make_inputs(cfg, seed=8)
+    f = inp.as_f64()
+    fn = oracle.ss2d_forward if cfg.kind == "2d" else oracle.selective_scan_fwd
+    _, yd_ref = fn(f["x"], f["delta"], f["A_log"], f["Bs"], f["Cs"], f["Dskip"],
+                   f["delta_bias"], K=cfg.K, return_dirs=True)
+    t = _gpu.tensors(inp)
+    for v in [-1, 3, 5]:
+        yd = binding.ss2d_scan_directions(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"],
+                                          t["Dskip"], t["delta_bias"], two_d=cfg.kind == "2d",
+                                          variant=v)
+        torch.cuda.synchronize()
+        got = yd.double().cpu().numpy().reshape(cfg.B, cfg.K, cfg.D, cfg.L)
+        _gpu.assert_close(got, yd_ref, wl.F32, f"directions variant {v}")
+
+
+def test_timed_call_matches_forward():
+    cfg = small(B=2, D=70, H=24, W=40, K=4, dtype=wl.BF16)
+    inp = wl.make_inputs(cfg, seed=9)
+    t = _gpu.tensors(inp)
+    for v in [-1, 3]:
+        y1 = _gpu.run_gpu(inp, variant=v, t=t)
+        y2 = torch.empty(inp.x.shape, dtype=torch.float32, device="cuda")
+        ms = binding.ss2d_forward_timed(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"],
+                                        t["Dskip"], t["delta_bias"], y2, variant=v)
+        assert np.array_equal(y2.double().cpu().numpy(), y1)
+        plan = binding.ss2d_plan(True, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K, v)
+        assert ms[2] > 0 and ms[3] > 0
+        assert (ms[0] > 0) == (plan["num_chunks"] > 1)
