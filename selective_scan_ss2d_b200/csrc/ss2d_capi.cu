@@ -180,7 +180,7 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     const ss2d::Plan pl = ss2d::make_plan(variant, pr.B, pr.D, (int)L, pr.K);
     if ((long long)pr.B * pl.NC > 65535)
         return SS2D_ERR_SHAPE;
-    if (ss2d::merge_smem_bytes(pr.W, pr.K, pr.two_d) > 200 * 1024)
+    if (ss2d::merge_smem_bytes(pr.H, pr.W, pr.K, pr.two_d) > 200 * 1024)
         return SS2D_ERR_SHAPE;
     const bool need_part = pr.K > 1;
     const size_t rows = (size_t)pr.B * pr.K * pr.D;

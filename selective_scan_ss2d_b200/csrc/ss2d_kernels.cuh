@@ -130,16 +130,16 @@ enum ScanMode { kModeState = 0, kModeOutput = 1 };
 template <int WC>
 struct ChunkShape {
     static constexpr int NT = 32 * WC;                     // threads = channels per CTA
-    static constexpr int TROW = 33;                        // padded row of a warp tile
+    static constexpr int TROW = 34;                        // padded row of a warp tile
     static constexpr int WTILE = kT * TROW;                // floats per warp tile
     static constexpr int BC_ENTRIES = kT * 8;              // float4 per B|C sub-chunk tile
-    static constexpr int BC_PER_THREAD = BC_ENTRIES / NT;  // float4 staged per thread
-    static_assert(BC_ENTRIES % NT == 0, "whole B|C entries per thread");
-    static_assert(BC_PER_THREAD <= 8, "B|C staging spread over the 8 batches");
-    // shared memory: B|C double buffer, then per warp: delta and x double
-    // buffers and one output tile
+    static constexpr int BC_PER_THREAD = (BC_ENTRIES + NT - 1) / NT;
+    static_assert(kT == 16, "a warp stages two channels x 16 steps per load");
+    static_assert(BC_PER_THREAD <= 4, "B|C staging spread over the 4 batches");
+    // shared memory: B|C double buffer, then per warp the delta and x double
+    // buffers (the delta tile is reused for the outputs)
     static constexpr size_t SMEM_BYTES =
-        sizeof(float4) * 2 * BC_ENTRIES + sizeof(float) * WC * 5 * WTILE;
+        sizeof(float4) * 2 * BC_ENTRIES + sizeof(float) * WC * 4 * WTILE;
 };
 
 // One chunk of LC steps of 32*WC channels of one (b, k); see the header.
@@ -158,9 +158,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
-    float *sD = wtiles + warp * 5 * WTILE;   // [2][kT][33] raw delta
-    float *sX = sD + 2 * WTILE;              // [2][kT][33] u
-    float *sY = sX + 2 * WTILE;              // [kT][33] outputs
+    float *sD = wtiles + warp * 4 * WTILE;   // [2][kT][TROW] raw delta, then outputs
+    float *sX = sD + 2 * WTILE;              // [2][kT][TROW] u
 
     const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W, K = p.K;
     const int k = blockIdx.x, tile = blockIdx.y;
@@ -210,32 +209,33 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     float dtsum = 0.f;
 
     // ---- staging of the sub-chunk that starts at ld_l0 ------------------
-    // delta / x: batch j (0..7) loads channels 4j .. 4j+3 of this warp, lane
-    // = step, into registers; the next batch stores them transposed into the
-    // warp tile [step][channel].
-    PixWalk xw;   // pixel of step ld_l0 + lane
-    xw.init(p.two_d, k, l_begin + lane, H, W, L);
+    // delta / x: lane = (step t = lane & 15, channel parity lane >> 4); batch j
+    // (0..3) loads channels 8j .. 8j+7 of this warp into registers, the next
+    // batch stores them transposed into the warp tile [step][channel].
+    const int st = lane & 15, sh = lane >> 4;
+    PixWalk xw;   // pixel of step ld_l0 + st
+    xw.init(p.two_d, k, l_begin + st, H, W, L);
     const int sq = kT / H, sr = kT % H;
     float rd[4], rx[4];
     int ld_l0 = l_begin;
     auto load_dx = [&](int j) {
-        const int l = ld_l0 + lane;
+        const int l = ld_l0 + st;
         const bool lok = l < l_end;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int cc = wd0 + j * 4 + i;
+            const int cc = wd0 + 8 * j + 2 * i + sh;
             const bool ok = lok && cc < D;
             rd[i] = ok ? to_f32(dg[(size_t)cc * L + l]) : 0.f;
             rx[i] = ok ? to_f32(xg[(size_t)cc * L + xw.p]) : 0.f;
         }
     };
     auto store_dx = [&](int buf, int j) {
-        float *td = sD + buf * WTILE + lane * TROW + j * 4;
-        float *tx = sX + buf * WTILE + lane * TROW + j * 4;
+        float *td = sD + buf * WTILE + st * TROW + 8 * j + sh;
+        float *tx = sX + buf * WTILE + st * TROW + 8 * j + sh;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            td[i] = rd[i];
-            tx[i] = rx[i];
+            td[2 * i] = rd[i];
+            tx[2 * i] = rx[i];
         }
     };
     // B|C: float4 entry e = (slot q = e / kT, step t = e % kT) holds rows
@@ -250,7 +250,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int n = (q & 3) * 4 + i;
-            v[i] = (l < l_end && n < N) ? to_f32(src[(size_t)n * L + l]) : 0.f;
+            v[i] = (e < Sh::BC_ENTRIES && l < l_end && n < N) ? to_f32(src[(size_t)n * L + l])
+                                                              : 0.f;
         }
         rbc[r] = make_float4(v[0], v[1], v[2], v[3]);
     };
@@ -258,8 +259,10 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
         for (int r = 0; r < BCPT; ++r) {
             const int e = tid + r * NT;
-            const int q = e / kT, t = e % kT;
-            sBC[buf * Sh::BC_ENTRIES + t * 8 + (q ^ (t & 7))] = rbc[r];
+            if (e < Sh::BC_ENTRIES) {
+                const int q = e / kT, t = e % kT;
+                sBC[buf * Sh::BC_ENTRIES + t * 8 + (q ^ (t & 7))] = rbc[r];
+            }
         }
     };
 
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         load_bc_one(r);
     store_bc(0);
 #pragma unroll 1
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
         load_dx(j);
         store_dx(0, j);
     }
@@ -281,10 +284,10 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         ld_l0 = l0 + kT;
         xw.advance(kT, sq, sr, H, W);
         const float4 *sb = sBC + buf * Sh::BC_ENTRIES;
-        const float *td = sD + buf * WTILE;
+        float *td = sD + buf * WTILE;
         const float *tx = sX + buf * WTILE;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
             // software-pipelined staging of the next sub-chunk
             if (more) {
                 if (j > 0)
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
                 const float2 du2 = make_float2(du, du);
                 const float4 *row = sb + t * 8;
                 const int sw = t & 7;
-                float2 acc = make_float2(0.f, 0.f);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float4 bv = row[q ^ sw];
@@ -318,31 +321,30 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
                         __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
                     if (MODE == kModeOutput) {
                         const float4 cv = row[(4 + q) ^ sw];
-                        acc = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc);
-                        acc = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc);
+                        acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
+                        acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
                     }
                 }
-                if (MODE == kModeOutput)
-                    sY[t * TROW + lane] = fmaf(dsk, u, acc.x + acc.y);
+                if (MODE == kModeOutput)   // the output takes the consumed delta slot
+                    td[t * TROW + lane] = fmaf(dsk, u, (acc0.x + acc0.y) + (acc1.x + acc1.y));
+            }
+        }
+        if (MODE == kModeOutput) {
+            // the sub-chunk's outputs: two channels x 16 consecutive steps per store
+            __syncwarp();
+            const int l = l0 + st;
+            if (l < l_end) {
+                float *orow = p.out + (row_bk + wd0 + sh) * L + l;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    if (wd0 + 2 * i + sh < D)
+                        orow[(size_t)(2 * i) * L] = td[st * TROW + 2 * i + sh];
+                }
             }
         }
         if (more) {
-            store_dx(buf ^ 1, 7);
+            store_dx(buf ^ 1, 3);
             store_bc(buf ^ 1);
-        }
-        if (MODE == kModeOutput) {
-            // the sub-chunk's outputs, one channel (32 consecutive steps) per store
-            __syncwarp();
-            const int l = l0 + lane;
-            if (l < l_end) {
-                float *orow = p.out + (row_bk + wd0) * L + l;
-#pragma unroll 4
-                for (int cc = 0; cc < 32; ++cc) {
-                    if (wd0 + cc < D)
-                        orow[(size_t)cc * L] = sY[lane * TROW + cc];
-                }
-            }
-            __syncwarp();
         }
         __syncthreads();
     }
@@ -374,58 +376,83 @@ __global__ void carry_kernel(const ScanParams p)
         n < p.N ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.N + n)) * kLog2e : 0.f;
     float *hs = p.hstate + (size_t)bkd * (p.NC - 1) * kNP + n;
     const float *ds = p.dtsum + (size_t)bkd * (p.NC - 1);
+    const int nc1 = p.NC - 1;
     float h = 0.f;
-    for (int c = 0; c < p.NC - 1; ++c) {
-        h = fmaf(mufu_ex2(a2 * ds[c]), h, hs[(size_t)c * kNP]);
-        hs[(size_t)c * kNP] = h;
+    for (int c0 = 0; c0 < nc1; c0 += 8) {
+        float he[8], dc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {   // the loads do not depend on h: issue them first
+            const bool ok = c0 + i < nc1;
+            he[i] = ok ? hs[(size_t)(c0 + i) * kNP] : 0.f;
+            dc[i] = ok ? ds[c0 + i] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (c0 + i < nc1) {
+                h = fmaf(mufu_ex2(a2 * dc[i]), h, he[i]);
+                hs[(size_t)(c0 + i) * kNP] = h;
+            }
+        }
     }
 }
 
-// cross_merge: scan-order rows part[(b,k,d)][l] -> pixel order.  One CTA per
-// (b, d, band of kMergeRows image rows).  The column-major directions are
-// gathered through a shared-memory tile so that global reads stay coalesced
-// (each image column's band is a run of consecutive scan steps).
+// cross_merge: scan-order rows part[(b,k,d)][l] -> pixel order.  A CTA
+// takes cpb consecutive (b,d) channels x a band of R image rows (R = H for
+// small maps: whole images).  The column-major directions are gathered
+// through a shared-memory tile, so global reads stay coalesced (the band of
+// each image column is a run of consecutive scan steps).
 //   sum = 1: y[b,d,p] = ((Y_0 + Y_1) + Y_2) + Y_3       (first K terms)
 //   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
 // A 1D sequence is a single image row (H = 1, W = L).
 __global__ void merge_kernel(const float *__restrict__ part, float *__restrict__ y, int B,
-                             int D, int H, int W, int K, int two_d, int sum)
+                             int D, int H, int W, int K, int two_d, int sum, int R, int cpb)
 {
-    constexpr int R = kMergeRows;
-    extern __shared__ float smem_m[];   // [2][W][R + 1] for k = 2, 3
+    extern __shared__ float smem_m[];   // [cpb][2][W][R + 1] for k = 2, 3
     const int L = H * W;
     const int nblk = (H + R - 1) / R;
     const int blk = blockIdx.x % nblk;
-    const int bd = blockIdx.x / nblk;
-    const int b = bd / D, d = bd % D;
+    const int bd0 = (blockIdx.x / nblk) * cpb;
+    const int nch = min(cpb, B * D - bd0);
     const int h0 = blk * R;
     const int hr = min(R, H - h0);
     const int np = hr * W;
     const int p0 = h0 * W;
-    const float *rows = part + ((size_t)b * K * D + d) * L;   // row of (b, k = 0, d)
     const size_t kstride = (size_t)D * L;
     const bool cols = two_d && K == 4;
+    auto row0 = [&](int bd) {   // row of (b, k = 0, d)
+        const int b = bd / D, d = bd % D;
+        return part + ((size_t)b * K * D + d) * L;
+    };
     if (cols) {
-        for (int e = threadIdx.x; e < W * hr; e += blockDim.x) {
-            const int w = e / hr, hh = e % hr;
+        const int per = W * hr;
+        for (int e = threadIdx.x; e < nch * per; e += blockDim.x) {
+            const int c = e / per, r = e % per;
+            const int w = r / hr, hh = r % hr;
+            const float *rows = row0(bd0 + c);
             const int s2 = w * H + h0 + hh;
-            smem_m[w * (R + 1) + hh] = __ldg(rows + 2 * kstride + s2);
-            smem_m[(W + w) * (R + 1) + hh] = __ldg(rows + 3 * kstride + (L - 1 - s2));
+            float *sm = smem_m + (size_t)c * 2 * W * (R + 1);
+            sm[w * (R + 1) + hh] = __ldg(rows + 2 * kstride + s2);
+            sm[(W + w) * (R + 1) + hh] = __ldg(rows + 3 * kstride + (L - 1 - s2));
         }
         __syncthreads();
     }
-    for (int e = threadIdx.x; e < np; e += blockDim.x) {
-        const int pix = p0 + e;
+    for (int e = threadIdx.x; e < nch * np; e += blockDim.x) {
+        const int c = e / np, r = e % np;
+        const int bd = bd0 + c;
+        const float *rows = row0(bd);
+        const int pix = p0 + r;
         float v[4];
         v[0] = __ldg(rows + pix);
         v[1] = (K >= 2) ? __ldg(rows + kstride + (L - 1 - pix)) : 0.f;
         if (cols) {
-            const int hh = e / W, w = e % W;
-            v[2] = smem_m[w * (R + 1) + hh];
-            v[3] = smem_m[(W + w) * (R + 1) + hh];
+            const int hh = r / W, w = r % W;
+            const float *sm = smem_m + (size_t)c * 2 * W * (R + 1);
+            v[2] = sm[w * (R + 1) + hh];
+            v[3] = sm[(W + w) * (R + 1) + hh];
         } else {
             v[2] = v[3] = 0.f;
         }
+        const int b = bd / D, d = bd % D;
         if (sum) {
             float acc = v[0];
             if (K >= 2)

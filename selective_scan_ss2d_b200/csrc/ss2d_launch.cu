@@ -12,16 +12,16 @@ namespace {
 // name: wc<W>_<chunking>; wc = 32-channel warps per CTA.
 const VariantInfo kVariants[] = {
     {"wc2_auto", 2, 0},    {"wc4_auto", 4, 0},    {"wc1_auto", 1, 0},
-    {"wc2_lc32", 2, 32},   {"wc4_lc64", 4, 64},   {"wc2_nochunk", 2, -1},
+    {"wc2_lc16", 2, 16},   {"wc4_lc64", 4, 64},   {"wc2_nochunk", 2, -1},
     {"wc2_lc256", 2, 256}, {"wc4_lc512", 4, 512}, {"wc1_lc128", 1, 128},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
-// Minimum resident CTAs per SM the kernels are compiled for: a register cap
-// of 65536 / (32 * WC * MINB) = 128 per thread.
+// Minimum resident CTAs per SM the kernels are compiled for: 20 warps per
+// SM, a register cap of 65536 / 640 = 102 per thread.
 template <int WC>
 struct MinBlocks {
-    static constexpr int value = 16 / WC;
+    static constexpr int value = 20 / WC;
 };
 
 template <typename Tin, int WC, int MODE>
@@ -142,24 +142,50 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
     }
 }
 
-size_t merge_smem_bytes(int W, int K, int two_d)
+namespace {
+// merge work unit: cpb channels x R image rows, about 2048 pixels
+void merge_shape(int H, int W, int K, int two_d, int *R, int *cpb)
 {
-    return (two_d && K == 4) ? sizeof(float) * 2 * (size_t)W * (kMergeRows + 1) : 0;
+    const bool cols = two_d && K == 4;
+    int r = cols ? 2048 / (W > 0 ? W : 1) : H;
+    if (r < 8)
+        r = 8;
+    if (r > H)
+        r = H;
+    *R = r;
+    const long long px = (long long)r * W;
+    long long c = px >= 2048 ? 1 : 2048 / (px > 0 ? px : 1);
+    if (c < 1)
+        c = 1;
+    *cpb = (int)c;
+}
+}  // namespace
+
+size_t merge_smem_bytes(int H, int W, int K, int two_d)
+{
+    if (!(two_d && K == 4))
+        return 0;
+    int R, cpb;
+    merge_shape(H, W, K, two_d, &R, &cpb);
+    return sizeof(float) * (size_t)cpb * 2 * W * (R + 1);
 }
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st)
 {
-    const size_t smem = merge_smem_bytes(W, K, two_d);
+    int R, cpb;
+    merge_shape(H, W, K, two_d, &R, &cpb);
+    const size_t smem = merge_smem_bytes(H, W, K, two_d);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(merge_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
     }
-    const int nblk = (H + kMergeRows - 1) / kMergeRows;
-    const long long grid = (long long)B * D * nblk;
-    merge_kernel<<<(unsigned)grid, 256, smem, st>>>(part, y, B, D, H, W, K, two_d, sum);
+    const int nblk = (H + R - 1) / R;
+    const long long groups = ((long long)B * D + cpb - 1) / cpb;
+    merge_kernel<<<(unsigned)(groups * nblk), 256, smem, st>>>(part, y, B, D, H, W, K, two_d,
+                                                               sum, R, cpb);
     return cudaGetLastError();
 }
 

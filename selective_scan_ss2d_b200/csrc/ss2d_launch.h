@@ -41,6 +41,6 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 // per-direction pixel-order copy (sum = 0).
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st);
-size_t merge_smem_bytes(int W, int K, int two_d);
+size_t merge_smem_bytes(int H, int W, int K, int two_d);
 
 }  // namespace ss2d

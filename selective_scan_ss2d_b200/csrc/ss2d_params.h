@@ -5,7 +5,7 @@
 namespace ss2d {
 
 constexpr int kNP = 16;     // states per channel held by the kernels (N <= 16)
-constexpr int kT = 32;      // steps per sub-chunk
+constexpr int kT = 16;      // steps per sub-chunk
 constexpr int kMergeRows = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 

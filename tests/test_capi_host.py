@@ -120,7 +120,7 @@ def test_plans_for_the_workloads(lib):
     from selective_scan_ss2d_b200 import workloads as wl
     for name, cfg in wl.CONFIGS.items():
         pl = binding.ss2d_plan(cfg.kind == "2d", cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K)
-        assert pl["chunk_len"] % 32 == 0
+        assert pl["chunk_len"] % 16 == 0
         assert pl["num_chunks"] == -(-cfg.L // pl["chunk_len"])
         want = (3 if pl["num_chunks"] > 1 else 1) + (1 if cfg.K > 1 else 0)
         assert pl["launches"] == want
