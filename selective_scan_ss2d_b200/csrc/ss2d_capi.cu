@@ -121,6 +121,8 @@ int validate(const Problem &pr)
     const long long L = (long long)pr.H * pr.W;
     if (L > INT_MAX || pr.B > 65535 || (long long)pr.K * pr.D > INT_MAX)
         return SS2D_ERR_SHAPE;
+    if (pr.two_d && pr.K == 4 && pr.W > 512)
+        return SS2D_ERR_SHAPE;
     return SS2D_OK;
 }
 

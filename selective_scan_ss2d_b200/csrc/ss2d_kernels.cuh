@@ -27,9 +27,9 @@
 // and keeps every pass a uniform mix of MUFU and FMA work.
 //
 // Memory traffic is coalesced: per 32-step sub-chunk, each warp loads delta
-// and x for its 32 channels one channel per instruction (lanes = steps) and
-// transposes them through a warp-private shared-memory tile; outputs go back
-// the same way.  B and C of a sub-chunk (shared by every channel of the CTA)
+// and x for its 32 channels two channels per instruction (lanes = 16 steps x
+// 2 channels), applies softplus to delta as it stores them transposed into a
+// warp-private shared-memory tile, and the outputs go back the same way.  B and C of a sub-chunk (shared by every channel of the CTA)
 // are staged once per CTA as a float32 [step][32] tile, read with broadcast
 // float4 loads.  The next sub-chunk's loads are spread over the current
 // sub-chunk's compute (software pipelining; nothing waits on a flag).
@@ -145,7 +145,7 @@ struct ChunkShape {
 // One chunk of LC steps of 32*WC channels of one (b, k); see the header.
 // grid: x = k, y = channel tile, z = b * NCg + chunk, NCg = chunks launched
 // (NC - 1 in kModeState, NC in kModeOutput).
-template <typename Tin, int WC, int MODE, int MINB>
+template <typename Tin, int WC, int MODE, int MINB, bool PACK>
 __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
 {
     using Sh = ChunkShape<WC>;
@@ -182,7 +182,6 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         A2[j].y = (n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
     }
     const float dsk = __ldg(p.Dskip + kd);
-    const float bias = __ldg(p.delta_bias + kd);
 
     const size_t row_bk = ((size_t)b * K + k) * D;   // row index of (b, k, d = 0)
     const Tin *xg = static_cast<const Tin *>(p.x) + (size_t)b * D * L;
@@ -229,12 +228,17 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
             rx[i] = ok ? to_f32(xg[(size_t)cc * L + xw.p]) : 0.f;
         }
     };
+    // the staging lanes apply softplus once per (channel, step) and store dt
+    // (and u), so each step of the scan loop starts from shared memory
+    const float *bias_w = p.delta_bias + (size_t)k * D;
     auto store_dx = [&](int buf, int j) {
         float *td = sD + buf * WTILE + st * TROW + 8 * j + sh;
         float *tx = sX + buf * WTILE + st * TROW + 8 * j + sh;
+        const bool lok = ld_l0 + st < l_end;   // the step these registers were loaded for
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            td[2 * i] = rd[i];
+            const int cc = wd0 + 8 * j + 2 * i + sh;
+            td[2 * i] = (lok && cc < D) ? softplus_f(rd[i] + __ldg(bias_w + cc)) : 0.f;
             tx[2 * i] = rx[i];
         }
     };
@@ -299,9 +303,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = j * 4 + i;
-                const float raw = td[t * TROW + lane];
+                const float dt = td[t * TROW + lane];
                 const float u = tx[t * TROW + lane];
-                const float dt = (l0 + t < l_end) ? softplus_f(raw + bias) : 0.f;
                 dtsum += dt;
                 const float du = dt * u;
                 const float2 dt2 = make_float2(dt, dt);
@@ -312,17 +315,36 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float4 bv = row[q ^ sw];
-                    const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
-                    const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
-                    const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
-                    const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
-                    h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
-                    h2[2 * q + 1] =
-                        __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                    if (MODE == kModeOutput) {
-                        const float4 cv = row[(4 + q) ^ sw];
-                        acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
-                        acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
+                    if constexpr (PACK) {
+                        const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
+                        const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
+                        const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
+                        const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
+                        h2[2 * q] =
+                            __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
+                        h2[2 * q + 1] =
+                            __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
+                        if (MODE == kModeOutput) {
+                            const float4 cv = row[(4 + q) ^ sw];
+                            acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
+                            acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
+                        }
+                    } else {
+                        const float a0 = mufu_ex2(dt * A2[2 * q].x);
+                        const float a1 = mufu_ex2(dt * A2[2 * q].y);
+                        const float a2 = mufu_ex2(dt * A2[2 * q + 1].x);
+                        const float a3 = mufu_ex2(dt * A2[2 * q + 1].y);
+                        h2[2 * q].x = fmaf(a0, h2[2 * q].x, du * bv.x);
+                        h2[2 * q].y = fmaf(a1, h2[2 * q].y, du * bv.y);
+                        h2[2 * q + 1].x = fmaf(a2, h2[2 * q + 1].x, du * bv.z);
+                        h2[2 * q + 1].y = fmaf(a3, h2[2 * q + 1].y, du * bv.w);
+                        if (MODE == kModeOutput) {
+                            const float4 cv = row[(4 + q) ^ sw];
+                            acc0.x = fmaf(cv.x, h2[2 * q].x, acc0.x);
+                            acc0.y = fmaf(cv.y, h2[2 * q].y, acc0.y);
+                            acc1.x = fmaf(cv.z, h2[2 * q + 1].x, acc1.x);
+                            acc1.y = fmaf(cv.w, h2[2 * q + 1].y, acc1.y);
+                        }
                     }
                 }
                 if (MODE == kModeOutput)   // the output takes the consumed delta slot
@@ -396,75 +418,121 @@ __global__ void carry_kernel(const ScanParams p)
     }
 }
 
-// cross_merge: scan-order rows part[(b,k,d)][l] -> pixel order.  A CTA
-// takes cpb consecutive (b,d) channels x a band of R image rows (R = H for
-// small maps: whole images).  The column-major directions are gathered
-// through a shared-memory tile, so global reads stay coalesced (the band of
-// each image column is a run of consecutive scan steps).
+// cross_merge: scan-order rows part[(b,k,d)][l] -> pixel order.  A CTA of
+// kMergeThreads threads covers kMergePix "slots": 2^cpb_log2 consecutive
+// (b,d) channels, each with one band of its pixels.  Two band shapes:
+//  * cols = 1 (SS2D, K = 4): R image rows padded to 2^rp_log2 x 2^wp_log2
+//    slots; the column-major directions are gathered through a shared-memory
+//    tile, so global reads stay coalesced (the band of each image column is a
+//    run of consecutive scan steps);
+//  * cols = 0 (K <= 2, SS2D or 1D): 2^wp_log2 consecutive pixels.
+// Slots map to (row, column) with shifts and masks, and every thread issues
+// all of its loads before it uses any (memory-level parallelism).
 //   sum = 1: y[b,d,p] = ((Y_0 + Y_1) + Y_2) + Y_3       (first K terms)
 //   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
-// A 1D sequence is a single image row (H = 1, W = L).
-__global__ void merge_kernel(const float *__restrict__ part, float *__restrict__ y, int B,
-                             int D, int H, int W, int K, int two_d, int sum, int R, int cpb)
+constexpr int kMergeThreads = 128;
+constexpr int kMergePix = 512;
+constexpr int kMergeIt = 4;   // kMergePix / kMergeThreads
+
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
+                 int W, int K, int cols, int sum, int R, int rp_log2, int wp_log2,
+                 int cpb_log2, int nblk)
 {
-    extern __shared__ float smem_m[];   // [cpb][2][W][R + 1] for k = 2, 3
-    const int L = H * W;
-    const int nblk = (H + R - 1) / R;
-    const int blk = blockIdx.x % nblk;
-    const int bd0 = (blockIdx.x / nblk) * cpb;
-    const int nch = min(cpb, B * D - bd0);
-    const int h0 = blk * R;
-    const int hr = min(R, H - h0);
-    const int np = hr * W;
-    const int p0 = h0 * W;
+    extern __shared__ float smem_m[];   // [cpb][2][W][R + 1] when cols
+    const long long L = (long long)H * W;
     const size_t kstride = (size_t)D * L;
-    const bool cols = two_d && K == 4;
-    auto row0 = [&](int bd) {   // row of (b, k = 0, d)
-        const int b = bd / D, d = bd % D;
-        return part + ((size_t)b * K * D + d) * L;
-    };
+    const int RP = 1 << rp_log2, WP = 1 << wp_log2;
+    const int S_log2 = rp_log2 + wp_log2;          // slots per channel band
+    const long long ch_total = (long long)B * D;
+    const int blk = blockIdx.x % nblk;
+    const long long bd0 = (long long)(blockIdx.x / nblk) << cpb_log2;
+    const int h0 = blk * R;
+    const int hr = cols ? min(R, H - h0) : 0;
+    const long long p0 = cols ? (long long)h0 * W : (long long)blk * WP;
+    const size_t tile = 2 * (size_t)W * (R + 1);
     if (cols) {
-        const int per = W * hr;
-        for (int e = threadIdx.x; e < nch * per; e += blockDim.x) {
-            const int c = e / per, r = e % per;
-            const int w = r / hr, hh = r % hr;
-            const float *rows = row0(bd0 + c);
-            const int s2 = w * H + h0 + hh;
-            float *sm = smem_m + (size_t)c * 2 * W * (R + 1);
-            sm[w * (R + 1) + hh] = __ldg(rows + 2 * kstride + s2);
-            sm[(W + w) * (R + 1) + hh] = __ldg(rows + 3 * kstride + (L - 1 - s2));
+        float g2[kMergeIt], g3[kMergeIt];
+        int gi[kMergeIt];
+#pragma unroll
+        for (int i = 0; i < kMergeIt; ++i) {   // slot -> (channel, column, band row)
+            const int e = threadIdx.x + i * kMergeThreads;
+            const int c = e >> S_log2, sl = e & ((1 << S_log2) - 1);
+            const int w = sl >> rp_log2, hh = sl & (RP - 1);
+            const long long bd = bd0 + c;
+            const bool ok = bd < ch_total && w < W && hh < hr;
+            gi[i] = ok ? (int)(c * tile) + w * (R + 1) + hh : -1;
+            g2[i] = g3[i] = 0.f;
+            if (ok) {
+                const float *rows = part + ((size_t)(bd / D) * K * D + (size_t)(bd % D)) * L;
+                const long long s2 = (long long)w * H + h0 + hh;
+                g2[i] = __ldg(rows + 2 * kstride + s2);
+                g3[i] = __ldg(rows + 3 * kstride + (L - 1 - s2));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kMergeIt; ++i) {
+            if (gi[i] >= 0) {
+                smem_m[gi[i]] = g2[i];
+                smem_m[gi[i] + W * (R + 1)] = g3[i];
+            }
         }
         __syncthreads();
     }
-    for (int e = threadIdx.x; e < nch * np; e += blockDim.x) {
-        const int c = e / np, r = e % np;
-        const int bd = bd0 + c;
-        const float *rows = row0(bd);
-        const int pix = p0 + r;
-        float v[4];
-        v[0] = __ldg(rows + pix);
-        v[1] = (K >= 2) ? __ldg(rows + kstride + (L - 1 - pix)) : 0.f;
-        if (cols) {
-            const int hh = r / W, w = r % W;
-            const float *sm = smem_m + (size_t)c * 2 * W * (R + 1);
-            v[2] = sm[w * (R + 1) + hh];
-            v[3] = sm[(W + w) * (R + 1) + hh];
-        } else {
-            v[2] = v[3] = 0.f;
+    float v0[kMergeIt], v1[kMergeIt];
+    long long pixv[kMergeIt];   // pixel, -1 if the slot is empty
+    size_t rowk[kMergeIt], rowy[kMergeIt];
+    int si[kMergeIt];
+#pragma unroll
+    for (int i = 0; i < kMergeIt; ++i) {
+        const int e = threadIdx.x + i * kMergeThreads;
+        const int c = e >> S_log2, sl = e & ((1 << S_log2) - 1);
+        const long long bd = bd0 + c;
+        long long pix;
+        bool ok;
+        if (cols) {   // slot -> (channel, band row, column)
+            const int hh = sl >> wp_log2, w = sl & (WP - 1);
+            ok = bd < ch_total && hh < hr && w < W;
+            pix = p0 + (long long)hh * W + w;
+            si[i] = (int)(c * tile) + w * (R + 1) + hh;
+        } else {      // slot -> (channel, pixel of the band)
+            pix = p0 + sl;
+            ok = bd < ch_total && pix < L;
+            si[i] = 0;
         }
-        const int b = bd / D, d = bd % D;
+        const size_t b = ok ? (size_t)(bd / D) : 0, d = ok ? (size_t)(bd % D) : 0;
+        rowk[i] = (b * K * D + d) * (size_t)L;
+        rowy[i] = (b * D + d) * (size_t)L;
+        pixv[i] = ok ? pix : -1;
+        const float *rows = part + rowk[i];
+        v0[i] = ok ? __ldg(rows + pix) : 0.f;
+        v1[i] = (ok && K >= 2) ? __ldg(rows + kstride + (L - 1 - pix)) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kMergeIt; ++i) {
+        const long long pix = pixv[i];
+        if (pix < 0)
+            continue;
+        const float v2 = cols ? smem_m[si[i]] : 0.f;
+        const float v3 = cols ? smem_m[si[i] + W * (R + 1)] : 0.f;
         if (sum) {
-            float acc = v[0];
+            float acc = v0[i];
             if (K >= 2)
-                acc += v[1];
+                acc += v1[i];
             if (K == 4) {
-                acc += v[2];
-                acc += v[3];
+                acc += v2;
+                acc += v3;
             }
-            y[((size_t)b * D + d) * L + pix] = acc;
+            y[rowy[i] + pix] = acc;
         } else {
-            for (int kk = 0; kk < K; ++kk)
-                y[(((size_t)b * K + kk) * D + d) * L + pix] = v[kk];
+            // per-direction layout (B, K, D, L): row (b, k, d) = rowk + k*D*L
+            y[rowk[i] + pix] = v0[i];
+            if (K >= 2)
+                y[rowk[i] + kstride + pix] = v1[i];
+            if (K == 4) {
+                y[rowk[i] + 2 * kstride + pix] = v2;
+                y[rowk[i] + 3 * kstride + pix] = v3;
+            }
         }
     }
 }

@@ -11,9 +11,10 @@ namespace {
 
 // name: wc<W>_<chunking>; wc = 32-channel warps per CTA.
 const VariantInfo kVariants[] = {
-    {"wc2_auto", 2, 0},    {"wc4_auto", 4, 0},    {"wc1_auto", 1, 0},
-    {"wc2_lc16", 2, 16},   {"wc4_lc64", 4, 64},   {"wc2_nochunk", 2, -1},
-    {"wc2_lc256", 2, 256}, {"wc4_lc512", 4, 512}, {"wc1_lc128", 1, 128},
+    {"wc2_auto", 2, 0, 1},     {"wc4_auto", 4, 0, 1},     {"wc1_auto", 1, 0, 1},
+    {"wc2_lc16", 2, 16, 1},    {"wc4_lc64", 4, 64, 1},    {"wc2_nochunk", 2, -1, 1},
+    {"wc2_lc256", 2, 256, 1},  {"wc4_lc512", 4, 512, 1},  {"wc1_lc128", 1, 128, 1},
+    {"wc2_auto_f32", 2, 0, 0}, {"wc4_auto_f32", 4, 0, 0}, {"wc4_lc64_f32", 4, 64, 0},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
@@ -24,11 +25,11 @@ struct MinBlocks {
     static constexpr int value = 20 / WC;
 };
 
-template <typename Tin, int WC, int MODE>
+template <typename Tin, int WC, int MODE, bool PACK>
 cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
 {
     using Sh = ChunkShape<WC>;
-    auto kern = chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC>::value>;
+    auto kern = chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC>::value, PACK>;
     const size_t smem = Sh::SMEM_BYTES;
     if (smem > 48 * 1024) {
         cudaError_t e =
@@ -41,14 +42,14 @@ cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <typename Tin, int WC>
+template <typename Tin, int WC, bool PACK>
 cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
 {
     cudaError_t e;
     if (plan.NC > 1) {
         if (ev)
             cudaEventRecord(ev[0], st);
-        e = launch_chunk<Tin, WC, kModeState>(p, plan.NC - 1, st);
+        e = launch_chunk<Tin, WC, kModeState, PACK>(p, plan.NC - 1, st);
         if (e != cudaSuccess)
             return e;
         if (ev)
@@ -62,7 +63,7 @@ cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
     }
     if (ev)
         cudaEventRecord(ev[2], st);
-    e = launch_chunk<Tin, WC, kModeOutput>(p, plan.NC, st);
+    e = launch_chunk<Tin, WC, kModeOutput, PACK>(p, plan.NC, st);
     if (ev)
         cudaEventRecord(ev[3], st);
     return e;
@@ -98,6 +99,7 @@ Plan make_plan(int v, int B, int D, int L, int K)
     Plan pl;
     pl.variant = v;
     pl.wc = vi->wc;
+    pl.pack = vi->pack;
     int lc;
     if (vi->chunk > 0) {
         lc = vi->chunk;
@@ -127,54 +129,90 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 {
     p.LC = plan.LC;
     p.NC = plan.NC;
+    if (!plan.pack) {
+        switch (plan.wc) {
+        case 2:
+            return bf16 ? launch_passes<__nv_bfloat16, 2, false>(plan, p, st, ev)
+                        : launch_passes<float, 2, false>(plan, p, st, ev);
+        case 4:
+            return bf16 ? launch_passes<__nv_bfloat16, 4, false>(plan, p, st, ev)
+                        : launch_passes<float, 4, false>(plan, p, st, ev);
+        default:
+            return cudaErrorInvalidValue;
+        }
+    }
     switch (plan.wc) {
     case 1:
-        return bf16 ? launch_passes<__nv_bfloat16, 1>(plan, p, st, ev)
-                    : launch_passes<float, 1>(plan, p, st, ev);
+        return bf16 ? launch_passes<__nv_bfloat16, 1, true>(plan, p, st, ev)
+                    : launch_passes<float, 1, true>(plan, p, st, ev);
     case 2:
-        return bf16 ? launch_passes<__nv_bfloat16, 2>(plan, p, st, ev)
-                    : launch_passes<float, 2>(plan, p, st, ev);
+        return bf16 ? launch_passes<__nv_bfloat16, 2, true>(plan, p, st, ev)
+                    : launch_passes<float, 2, true>(plan, p, st, ev);
     case 4:
-        return bf16 ? launch_passes<__nv_bfloat16, 4>(plan, p, st, ev)
-                    : launch_passes<float, 4>(plan, p, st, ev);
+        return bf16 ? launch_passes<__nv_bfloat16, 4, true>(plan, p, st, ev)
+                    : launch_passes<float, 4, true>(plan, p, st, ev);
     default:
         return cudaErrorInvalidValue;
     }
 }
 
 namespace {
-// merge work unit: cpb channels x R image rows, about 2048 pixels
-void merge_shape(int H, int W, int K, int two_d, int *R, int *cpb)
+// merge work unit (see merge_kernel): a channel band of at most kMergePix
+// slots, and as many channels per CTA as the kMergePix slots hold
+struct MergeShape {
+    int cols, R, rp, wp, cpb_log2, nblk;
+    bool ok;
+};
+MergeShape merge_shape(int H, int W, int K, int two_d)
 {
-    const bool cols = two_d && K == 4;
-    int r = cols ? 2048 / (W > 0 ? W : 1) : H;
-    if (r < 8)
-        r = 8;
-    if (r > H)
-        r = H;
-    *R = r;
-    const long long px = (long long)r * W;
-    long long c = px >= 2048 ? 1 : 2048 / (px > 0 ? px : 1);
-    if (c < 1)
-        c = 1;
-    *cpb = (int)c;
+    MergeShape m{};
+    m.cols = (two_d && K == 4) ? 1 : 0;
+    const long long L = (long long)H * W;
+    int wp = 0, rp = 0;
+    if (m.cols) {
+        while ((1 << wp) < W)
+            ++wp;
+        if ((1 << wp) > kMergePix) {
+            m.ok = false;
+            return m;
+        }
+        while ((1 << (rp + 1)) <= (kMergePix >> wp) && (1 << rp) < H)
+            ++rp;
+        m.R = (1 << rp) < H ? (1 << rp) : H;
+        m.nblk = (H + m.R - 1) / m.R;
+    } else {
+        while ((1LL << wp) < L && (1 << wp) < kMergePix)
+            ++wp;
+        m.R = 1;
+        m.nblk = (int)((L + (1LL << wp) - 1) >> wp);
+    }
+    m.rp = rp;
+    m.wp = wp;
+    int cl = 0;   // channels per CTA: the slots left over
+    while ((1 << (cl + 1 + rp + wp)) <= kMergePix)
+        ++cl;
+    m.cpb_log2 = cl;
+    m.ok = true;
+    return m;
 }
 }  // namespace
 
 size_t merge_smem_bytes(int H, int W, int K, int two_d)
 {
-    if (!(two_d && K == 4))
+    const MergeShape m = merge_shape(H, W, K, two_d);
+    if (!m.ok)
+        return (size_t)1 << 40;
+    if (!m.cols)
         return 0;
-    int R, cpb;
-    merge_shape(H, W, K, two_d, &R, &cpb);
-    return sizeof(float) * (size_t)cpb * 2 * W * (R + 1);
+    return sizeof(float) * ((size_t)1 << m.cpb_log2) * 2 * (size_t)W * (m.R + 1);
 }
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st)
 {
-    int R, cpb;
-    merge_shape(H, W, K, two_d, &R, &cpb);
+    const MergeShape m = merge_shape(H, W, K, two_d);
+    if (!m.ok)
+        return cudaErrorInvalidValue;
     const size_t smem = merge_smem_bytes(H, W, K, two_d);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(merge_kernel,
@@ -182,10 +220,9 @@ cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W
         if (e != cudaSuccess)
             return e;
     }
-    const int nblk = (H + R - 1) / R;
-    const long long groups = ((long long)B * D + cpb - 1) / cpb;
-    merge_kernel<<<(unsigned)(groups * nblk), 256, smem, st>>>(part, y, B, D, H, W, K, two_d,
-                                                               sum, R, cpb);
+    const long long groups = (((long long)B * D) + (1LL << m.cpb_log2) - 1) >> m.cpb_log2;
+    merge_kernel<<<(unsigned)(groups * m.nblk), kMergeThreads, smem, st>>>(
+        part, y, B, D, H, W, K, m.cols, sum, m.R, m.rp, m.wp, m.cpb_log2, m.nblk);
     return cudaGetLastError();
 }
 

@@ -15,12 +15,14 @@ struct VariantInfo {
     const char *name;
     int wc;
     int chunk;
+    int pack;   // 1: packed f32x2 arithmetic; 0: scalar float32
 };
 
 // How one call is executed.
 struct Plan {
     int variant;
     int wc;
+    int pack;
     int LC;        // steps per chunk (multiple of 32)
     int NC;        // chunks per sequence
     int launches;  // kernel launches of a forward call
