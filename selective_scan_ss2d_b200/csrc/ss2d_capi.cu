@@ -198,6 +198,15 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     }
     char *base = static_cast<char *>(scratch);
     p.out = need_part ? reinterpret_cast<float *>(base) : pr.y;
+    {
+        // vector access to the rows of delta and x (dtype) and of out (float32)
+        // needs every row start on a boundary of the vector width
+        const size_t esz = bf16 ? 2 : 4;
+        const bool ptr_ok = (((uintptr_t)pr.x | (uintptr_t)pr.delta | (uintptr_t)p.out) & 15) == 0;
+        const size_t rb = (size_t)L * esz;
+        p.vec = !ptr_ok ? 0 : (rb % 16 == 0 ? 16 : (rb % 8 == 0 ? 8 : 0));
+        p.ovec = (ptr_ok && ((size_t)L * 4) % 16 == 0) ? 1 : 0;
+    }
     p.hstate = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes) : nullptr;
     p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes + hs_bytes) : nullptr;
     cudaError_t e = ss2d::launch_scan(pl, bf16, p, st, ev);

@@ -26,13 +26,14 @@
 // Chunking costs one extra exp per update on the chunked workloads only,
 // and keeps every pass a uniform mix of MUFU and FMA work.
 //
-// Memory traffic is coalesced: per 32-step sub-chunk, each warp loads delta
-// and x for its 32 channels two channels per instruction (lanes = 16 steps x
-// 2 channels), applies softplus to delta as it stores them transposed into a
-// warp-private shared-memory tile, and the outputs go back the same way.  B and C of a sub-chunk (shared by every channel of the CTA)
-// are staged once per CTA as a float32 [step][32] tile, read with broadcast
-// float4 loads.  The next sub-chunk's loads are spread over the current
-// sub-chunk's compute (software pipelining; nothing waits on a flag).
+// Staging: each lane loads 16 steps of its own channel's delta and x with
+// 16-byte vector loads (x of the column-major directions through the pixel
+// walker), one 16-step sub-chunk ahead; it applies softplus once per
+// (channel, step) and parks (dt, u) in a warp-private shared-memory tile, and
+// its outputs go back as 16-byte vectors of its scan-order row.  B and C of a
+// sub-chunk (shared by every channel of the CTA) are staged once per CTA as a
+// float32 [step][32] tile read with broadcast float4 loads, also one
+// sub-chunk ahead.  Nothing waits on a flag.
 //
 // exp(dt*A) runs on the MUFU unit as 2^(dt * A*log2(e)).  The float32 pair
 // arithmetic uses the sm_100 packed f32x2 instructions (__ffma2_rn,
@@ -98,6 +99,31 @@ struct PixWalk {
             p = h * W + w;
         }
     }
+    // one step forward
+    __device__ __forceinline__ void next(int H, int W)
+    {
+        if (mode == 0) {
+            ++p;
+        } else if (mode == 1) {
+            --p;
+        } else if (mode == 2) {
+            if (++h == H) {
+                h = 0;
+                ++w;
+                p = w;
+            } else {
+                p += W;
+            }
+        } else {
+            if (--h < 0) {
+                h = H - 1;
+                --w;
+                p = h * W + w;
+            } else {
+                p -= W;
+            }
+        }
+    }
     // advance by n = nq*H + nr steps (nq = n / H, nr = n % H precomputed)
     __device__ __forceinline__ void advance(int n, int nq, int nr, int H, int W)
     {
@@ -130,17 +156,73 @@ enum ScanMode { kModeState = 0, kModeOutput = 1 };
 template <int WC>
 struct ChunkShape {
     static constexpr int NT = 32 * WC;                     // threads = channels per CTA
-    static constexpr int TROW = 34;                        // padded row of a warp tile
-    static constexpr int WTILE = kT * TROW;                // floats per warp tile
     static constexpr int BC_ENTRIES = kT * 8;              // float4 per B|C sub-chunk tile
     static constexpr int BC_PER_THREAD = (BC_ENTRIES + NT - 1) / NT;
-    static_assert(kT == 16, "a warp stages two channels x 16 steps per load");
-    static_assert(BC_PER_THREAD <= 4, "B|C staging spread over the 4 batches");
-    // shared memory: B|C double buffer, then per warp the delta and x double
-    // buffers (the delta tile is reused for the outputs)
+    static constexpr int DU_WARP = 2 * kT * 32;            // float2 per warp: [2][kT][32] (dt, u)
+    static constexpr int Y_WARP = kT * 33;                 // floats per warp: [kT][33] outputs
+    static_assert(kT == 16, "sub-chunks of 16 steps: two 16-byte bf16 vectors per lane");
     static constexpr size_t SMEM_BYTES =
-        sizeof(float4) * 2 * BC_ENTRIES + sizeof(float) * WC * 4 * WTILE;
+        sizeof(float4) * 2 * BC_ENTRIES +
+        (size_t)WC * (sizeof(float2) * DU_WARP + sizeof(float) * Y_WARP);
 };
+
+// 16 consecutive values of one row, held as raw 32-bit words (bf16: 8 words,
+// two values each; float: 16 words)
+template <typename Tin>
+struct Row16 {
+    static constexpr int RW = kT * (int)sizeof(Tin) / 4;
+    uint32_t w[RW];
+    __device__ __forceinline__ float get(int i) const
+    {
+        if constexpr (sizeof(Tin) == 2) {
+            const uint32_t v = w[i >> 1];
+            return __uint_as_float((i & 1) ? (v & 0xffff0000u) : (v << 16));
+        } else {
+            return __uint_as_float(w[i]);
+        }
+    }
+    // 16-byte vector loads; src 16-byte aligned
+    __device__ __forceinline__ void load_vec(const Tin *src)
+    {
+        const uint4 *v = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+        for (int q = 0; q < RW / 4; ++q) {
+            const uint4 x = __ldg(v + q);
+            w[4 * q] = x.x;
+            w[4 * q + 1] = x.y;
+            w[4 * q + 2] = x.z;
+            w[4 * q + 3] = x.w;
+        }
+    }
+    // 8-byte vector loads; src 8-byte aligned
+    __device__ __forceinline__ void load_vec8(const Tin *src)
+    {
+        const uint2 *v = reinterpret_cast<const uint2 *>(src);
+#pragma unroll
+        for (int q = 0; q < RW / 2; ++q) {
+            const uint2 x = __ldg(v + q);
+            w[2 * q] = x.x;
+            w[2 * q + 1] = x.y;
+        }
+    }
+    __device__ __forceinline__ void set_raw(int i, uint32_t bits)   // bits of one value
+    {
+        if constexpr (sizeof(Tin) == 2) {
+            if (i & 1)
+                w[i >> 1] = (w[i >> 1] & 0xffffu) | (bits << 16);
+            else
+                w[i >> 1] = (w[i >> 1] & 0xffff0000u) | (bits & 0xffffu);
+        } else {
+            w[i] = bits;
+        }
+    }
+};
+
+__device__ __forceinline__ uint32_t raw_bits(const float *p) { return __float_as_uint(__ldg(p)); }
+__device__ __forceinline__ uint32_t raw_bits(const __nv_bfloat16 *p)
+{
+    return (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p));
+}
 
 // One chunk of LC steps of 32*WC channels of one (b, k); see the header.
 // grid: x = k, y = channel tile, z = b * NCg + chunk, NCg = chunks launched
@@ -149,27 +231,24 @@ template <typename Tin, int WC, int MODE, int MINB, bool PACK>
 __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
 {
     using Sh = ChunkShape<WC>;
-    constexpr int NT = Sh::NT, TROW = Sh::TROW, WTILE = Sh::WTILE;
-    constexpr int BCPT = Sh::BC_PER_THREAD;
+    constexpr int NT = Sh::NT, BCPT = Sh::BC_PER_THREAD;
 
     extern __shared__ float4 smem_f4[];
     float4 *sBC = smem_f4;   // [2][kT][8], slot q of step t stored at t*8 + (q ^ (t & 7))
-    float *wtiles = reinterpret_cast<float *>(sBC + 2 * Sh::BC_ENTRIES);
-
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
-    float *sD = wtiles + warp * 4 * WTILE;   // [2][kT][TROW] raw delta, then outputs
-    float *sX = sD + 2 * WTILE;              // [2][kT][TROW] u
+    float2 *sDU = reinterpret_cast<float2 *>(sBC + 2 * Sh::BC_ENTRIES) + warp * Sh::DU_WARP;
+    float *sY = reinterpret_cast<float *>(reinterpret_cast<float2 *>(sBC + 2 * Sh::BC_ENTRIES) +
+                                          WC * Sh::DU_WARP) + warp * Sh::Y_WARP;
 
     const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W, K = p.K;
     const int k = blockIdx.x, tile = blockIdx.y;
     const int ncg = (MODE == kModeState) ? p.NC - 1 : p.NC;
     const int b = blockIdx.z / ncg, chunk = blockIdx.z % ncg;
     const int d0 = tile * NT;
-    const int wd0 = d0 + warp * 32;          // first channel of this warp
     const int d = d0 + tid;
     const bool cvalid = d < D;
-    const int dc = cvalid ? d : D - 1;       // clamped channel for parameter reads
+    const int dc = cvalid ? d : D - 1;       // clamped channel for addressing
     const int kd = k * D + dc;
     const int l_begin = chunk * p.LC;
     const int l_end = min(l_begin + p.LC, L);
@@ -182,12 +261,18 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         A2[j].y = (n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
     }
     const float dsk = __ldg(p.Dskip + kd);
+    const float bias = __ldg(p.delta_bias + kd);
 
     const size_t row_bk = ((size_t)b * K + k) * D;   // row index of (b, k, d = 0)
-    const Tin *xg = static_cast<const Tin *>(p.x) + (size_t)b * D * L;
-    const Tin *dg = static_cast<const Tin *>(p.delta) + row_bk * L;
+    const Tin *drow = static_cast<const Tin *>(p.delta) + (row_bk + dc) * L;   // my delta row
+    const Tin *xrow = static_cast<const Tin *>(p.x) + ((size_t)b * D + dc) * L;  // my x map
     const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * K + k) * N * L;
     const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * K + k) * N * L;
+    // x order of this direction: 0 forward, 1 reversed (both contiguous),
+    // 2 through the pixel walker (column-major directions)
+    const int xmode = (p.two_d && k >= 2) ? 2 : (k & 1);
+    const int vbytes = p.vec;   // 16 or 8: vector width of delta/x row loads; 0: scalar
+    const bool ovec = p.ovec != 0;
 
     // entry state
     float2 h2[8];
@@ -207,57 +292,81 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     }
     float dtsum = 0.f;
 
-    // ---- staging of the sub-chunk that starts at ld_l0 ------------------
-    // delta / x: lane = (step t = lane & 15, channel parity lane >> 4); batch j
-    // (0..3) loads channels 8j .. 8j+7 of this warp into registers, the next
-    // batch stores them transposed into the warp tile [step][channel].
-    const int st = lane & 15, sh = lane >> 4;
-    PixWalk xw;   // pixel of step ld_l0 + st
-    xw.init(p.two_d, k, l_begin + st, H, W, L);
-    const int sq = kT / H, sr = kT % H;
-    float rd[4], rx[4];
-    int ld_l0 = l_begin;
-    auto load_dx = [&](int j) {
-        const int l = ld_l0 + st;
-        const bool lok = l < l_end;
+    // ---- per-lane prefetch of 16 steps of this lane's delta and x ------
+    PixWalk xw;   // column-major directions: pixel of the next step to prefetch
+    xw.init(p.two_d, k, l_begin, H, W, L);
+    Row16<Tin> pd, px;
+    auto prefetch = [&](int ls) {   // steps ls .. ls + 15
+        const bool whole = vbytes > 0 && ls + kT <= L;
+        auto load_row = [&](Row16<Tin> &r, const Tin *src) {
+            if (vbytes == 16)
+                r.load_vec(src);
+            else
+                r.load_vec8(src);
+        };
+        if (whole) {
+            load_row(pd, drow + ls);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int cc = wd0 + 8 * j + 2 * i + sh;
-            const bool ok = lok && cc < D;
-            rd[i] = ok ? to_f32(dg[(size_t)cc * L + l]) : 0.f;
-            rx[i] = ok ? to_f32(xg[(size_t)cc * L + xw.p]) : 0.f;
+            for (int i = 0; i < kT; ++i)
+                pd.set_raw(i, ls + i < L ? raw_bits(drow + ls + i) : 0u);
+        }
+        if (xmode == 0) {
+            if (whole) {
+                load_row(px, xrow + ls);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kT; ++i)
+                    px.set_raw(i, ls + i < L ? raw_bits(xrow + ls + i) : 0u);
+            }
+        } else if (xmode == 1) {   // pixels L-1-ls-i: load ascending, read reversed
+            if (whole) {
+                load_row(px, xrow + (L - kT - ls));
+            } else {
+#pragma unroll
+                for (int i = 0; i < kT; ++i) {   // value of step ls + 15 - i
+                    const int l = ls + kT - 1 - i;
+                    px.set_raw(i, l < L ? raw_bits(xrow + (L - 1 - l)) : 0u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kT; ++i) {
+                px.set_raw(i, ls + i < L ? raw_bits(xrow + xw.p) : 0u);
+                xw.next(H, W);
+            }
         }
     };
-    // the staging lanes apply softplus once per (channel, step) and store dt
-    // (and u), so each step of the scan loop starts from shared memory
-    const float *bias_w = p.delta_bias + (size_t)k * D;
-    auto store_dx = [&](int buf, int j) {
-        float *td = sD + buf * WTILE + st * TROW + 8 * j + sh;
-        float *tx = sX + buf * WTILE + st * TROW + 8 * j + sh;
-        const bool lok = ld_l0 + st < l_end;   // the step these registers were loaded for
+    // softplus once per (channel, step); dt and u to the warp tile [t][lane]
+    auto unpack_store = [&](int buf, int ls) {
+        float2 *du = sDU + buf * (kT * 32) + lane;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int cc = wd0 + 8 * j + 2 * i + sh;
-            td[2 * i] = (lok && cc < D) ? softplus_f(rd[i] + __ldg(bias_w + cc)) : 0.f;
-            tx[2 * i] = rx[i];
+        for (int i = 0; i < kT; ++i) {
+            const bool ok = ls + i < l_end;
+            const float dt = ok ? softplus_f(pd.get(i) + bias) : 0.f;
+            const float u = (xmode == 1) ? px.get(kT - 1 - i) : px.get(i);
+            du[i * 32] = make_float2(dt, u);
         }
     };
     // B|C: float4 entry e = (slot q = e / kT, step t = e % kT) holds rows
     // 4q..4q+3 of B (q < 4) or C (q >= 4) at step t
     float4 rbc[BCPT];
-    auto load_bc_one = [&](int r) {
-        const int e = tid + r * NT;
-        const int q = e / kT, t = e % kT;
-        const int l = ld_l0 + t;
-        const Tin *src = (q < 4) ? Bg : Cg;
-        float v[4];
+    auto load_bc = [&](int ls) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int n = (q & 3) * 4 + i;
-            v[i] = (e < Sh::BC_ENTRIES && l < l_end && n < N) ? to_f32(src[(size_t)n * L + l])
-                                                              : 0.f;
+        for (int r = 0; r < BCPT; ++r) {
+            const int e = tid + r * NT;
+            const int q = e / kT, t = e % kT;
+            const int l = ls + t;
+            const Tin *src = (q < 4) ? Bg : Cg;
+            float v[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int n = (q & 3) * 4 + i;
+                v[i] = (e < Sh::BC_ENTRIES && l < l_end && n < N) ? to_f32(src[(size_t)n * L + l])
+                                                                  : 0.f;
+            }
+            rbc[r] = make_float4(v[0], v[1], v[2], v[3]);
         }
-        rbc[r] = make_float4(v[0], v[1], v[2], v[3]);
     };
     auto store_bc = [&](int buf) {
 #pragma unroll
@@ -270,103 +379,95 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         }
     };
 
-    // prologue: stage the first sub-chunk
-#pragma unroll
-    for (int r = 0; r < BCPT; ++r)
-        load_bc_one(r);
+    // prologue: sub-chunk 0 staged, sub-chunk 1 in flight
+    prefetch(l_begin);
+    load_bc(l_begin);
+    unpack_store(0, l_begin);
     store_bc(0);
-#pragma unroll 1
-    for (int j = 0; j < 4; ++j) {
-        load_dx(j);
-        store_dx(0, j);
+    if (l_begin + kT < l_end) {
+        prefetch(l_begin + kT);
+        load_bc(l_begin + kT);
     }
     __syncthreads();
 
     int buf = 0;
     for (int l0 = l_begin; l0 < l_end; l0 += kT, buf ^= 1) {
         const bool more = l0 + kT < l_end;
-        ld_l0 = l0 + kT;
-        xw.advance(kT, sq, sr, H, W);
         const float4 *sb = sBC + buf * Sh::BC_ENTRIES;
-        float *td = sD + buf * WTILE;
-        const float *tx = sX + buf * WTILE;
+        const float2 *du_t = sDU + buf * (kT * 32) + lane;
+#pragma unroll 4
+        for (int t = 0; t < kT; ++t) {
+            const float2 dtu = du_t[t * 32];
+            const float dt = dtu.x, u = dtu.y;
+            dtsum += dt;
+            const float du = dt * u;
+            const float2 dt2 = make_float2(dt, dt);
+            const float2 du2 = make_float2(du, du);
+            const float4 *row = sb + t * 8;
+            const int sw = t & 7;
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            // software-pipelined staging of the next sub-chunk
-            if (more) {
-                if (j > 0)
-                    store_dx(buf ^ 1, j - 1);
-                load_dx(j);
-                if (j < BCPT)
-                    load_bc_one(j);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t = j * 4 + i;
-                const float dt = td[t * TROW + lane];
-                const float u = tx[t * TROW + lane];
-                dtsum += dt;
-                const float du = dt * u;
-                const float2 dt2 = make_float2(dt, dt);
-                const float2 du2 = make_float2(du, du);
-                const float4 *row = sb + t * 8;
-                const int sw = t & 7;
-                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 bv = row[q ^ sw];
-                    if constexpr (PACK) {
-                        const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
-                        const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
-                        const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
-                        const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
-                        h2[2 * q] =
-                            __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
-                        h2[2 * q + 1] =
-                            __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                        if (MODE == kModeOutput) {
-                            const float4 cv = row[(4 + q) ^ sw];
-                            acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
-                            acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
-                        }
-                    } else {
-                        const float a0 = mufu_ex2(dt * A2[2 * q].x);
-                        const float a1 = mufu_ex2(dt * A2[2 * q].y);
-                        const float a2 = mufu_ex2(dt * A2[2 * q + 1].x);
-                        const float a3 = mufu_ex2(dt * A2[2 * q + 1].y);
-                        h2[2 * q].x = fmaf(a0, h2[2 * q].x, du * bv.x);
-                        h2[2 * q].y = fmaf(a1, h2[2 * q].y, du * bv.y);
-                        h2[2 * q + 1].x = fmaf(a2, h2[2 * q + 1].x, du * bv.z);
-                        h2[2 * q + 1].y = fmaf(a3, h2[2 * q + 1].y, du * bv.w);
-                        if (MODE == kModeOutput) {
-                            const float4 cv = row[(4 + q) ^ sw];
-                            acc0.x = fmaf(cv.x, h2[2 * q].x, acc0.x);
-                            acc0.y = fmaf(cv.y, h2[2 * q].y, acc0.y);
-                            acc1.x = fmaf(cv.z, h2[2 * q + 1].x, acc1.x);
-                            acc1.y = fmaf(cv.w, h2[2 * q + 1].y, acc1.y);
-                        }
+            for (int q = 0; q < 4; ++q) {
+                const float4 bv = row[q ^ sw];
+                if constexpr (PACK) {
+                    const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
+                    const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
+                    const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
+                    const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
+                    h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
+                    h2[2 * q + 1] =
+                        __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
+                    if (MODE == kModeOutput) {
+                        const float4 cv = row[(4 + q) ^ sw];
+                        acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
+                        acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
+                    }
+                } else {
+                    const float a0 = mufu_ex2(dt * A2[2 * q].x);
+                    const float a1 = mufu_ex2(dt * A2[2 * q].y);
+                    const float a2 = mufu_ex2(dt * A2[2 * q + 1].x);
+                    const float a3 = mufu_ex2(dt * A2[2 * q + 1].y);
+                    h2[2 * q].x = fmaf(a0, h2[2 * q].x, du * bv.x);
+                    h2[2 * q].y = fmaf(a1, h2[2 * q].y, du * bv.y);
+                    h2[2 * q + 1].x = fmaf(a2, h2[2 * q + 1].x, du * bv.z);
+                    h2[2 * q + 1].y = fmaf(a3, h2[2 * q + 1].y, du * bv.w);
+                    if (MODE == kModeOutput) {
+                        const float4 cv = row[(4 + q) ^ sw];
+                        acc0.x = fmaf(cv.x, h2[2 * q].x, acc0.x);
+                        acc0.y = fmaf(cv.y, h2[2 * q].y, acc0.y);
+                        acc1.x = fmaf(cv.z, h2[2 * q + 1].x, acc1.x);
+                        acc1.y = fmaf(cv.w, h2[2 * q + 1].y, acc1.y);
                     }
                 }
-                if (MODE == kModeOutput)   // the output takes the consumed delta slot
-                    td[t * TROW + lane] = fmaf(dsk, u, (acc0.x + acc0.y) + (acc1.x + acc1.y));
             }
+            if (MODE == kModeOutput)
+                sY[t * 33 + lane] = fmaf(dsk, u, (acc0.x + acc0.y) + (acc1.x + acc1.y));
         }
-        if (MODE == kModeOutput) {
-            // the sub-chunk's outputs: two channels x 16 consecutive steps per store
-            __syncwarp();
-            const int l = l0 + st;
-            if (l < l_end) {
-                float *orow = p.out + (row_bk + wd0 + sh) * L + l;
-#pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    if (wd0 + 2 * i + sh < D)
-                        orow[(size_t)(2 * i) * L] = td[st * TROW + 2 * i + sh];
-                }
+        if (MODE == kModeOutput && cvalid) {
+            // this lane's 16 outputs, one row segment of the scan-order output
+            float *orow = p.out + (row_bk + d) * L + l0;
+            if (ovec && l0 + kT <= l_end) {
+#pragma unroll
+                for (int q = 0; q < kT / 4; ++q)
+                    reinterpret_cast<float4 *>(orow)[q] =
+                        make_float4(sY[(4 * q) * 33 + lane], sY[(4 * q + 1) * 33 + lane],
+                                    sY[(4 * q + 2) * 33 + lane], sY[(4 * q + 3) * 33 + lane]);
+            } else {
+#pragma unroll
+                for (int t = 0; t < kT; ++t)
+                    if (l0 + t < l_end)
+                        orow[t] = sY[t * 33 + lane];
             }
         }
         if (more) {
-            store_dx(buf ^ 1, 3);
+            // stage the next sub-chunk (its loads were issued one sub-chunk
+            // ago) and issue the loads of the one after it
+            unpack_store(buf ^ 1, l0 + kT);
             store_bc(buf ^ 1);
+            if (l0 + 2 * kT < l_end) {
+                prefetch(l0 + 2 * kT);
+                load_bc(l0 + 2 * kT);
+            }
         }
         __syncthreads();
     }

@@ -18,11 +18,11 @@ const VariantInfo kVariants[] = {
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
-// Minimum resident CTAs per SM the kernels are compiled for: 20 warps per
-// SM, a register cap of 65536 / 640 = 102 per thread.
+// Minimum resident CTAs per SM the kernels are compiled for: 16 warps per
+// SM, a register cap of 65536 / 512 = 128 per thread.
 template <int WC>
 struct MinBlocks {
-    static constexpr int value = 20 / WC;
+    static constexpr int value = 16 / WC;
 };
 
 template <typename Tin, int WC, int MODE, bool PACK>

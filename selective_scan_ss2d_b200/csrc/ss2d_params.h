@@ -25,6 +25,8 @@ struct ScanParams {
     int two_d;                // 1: SS2D scan orders; 0: 1D (k = 1 reversed)
     int LC;                   // steps per chunk (multiple of kT)
     int NC;                   // chunks per sequence
+    int vec;                  // 16 / 8: byte width of vector loads of delta and x rows; 0: none
+    int ovec;                 // 1: rows of out allow 16-byte vector stores
 };
 
 }  // namespace ss2d
