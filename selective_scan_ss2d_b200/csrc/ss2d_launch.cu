@@ -11,25 +11,28 @@ namespace {
 
 // name: wc<W>_<chunking>; wc = 32-channel warps per CTA.
 const VariantInfo kVariants[] = {
-    {"wc2_auto", 2, 0, 1},     {"wc4_auto", 4, 0, 1},     {"wc1_auto", 1, 0, 1},
-    {"wc2_lc16", 2, 16, 1},    {"wc4_lc64", 4, 64, 1},    {"wc2_nochunk", 2, -1, 1},
-    {"wc2_lc256", 2, 256, 1},  {"wc4_lc512", 4, 512, 1},  {"wc1_lc128", 1, 128, 1},
-    {"wc2_auto_f32", 2, 0, 0}, {"wc4_auto_f32", 4, 0, 0}, {"wc4_lc64_f32", 4, 64, 0},
+    {"wc2_auto", 2, 0, 128},       {"wc4_auto", 4, 0, 128},       {"wc1_auto", 1, 0, 128},
+    {"wc2_lc16", 2, 16, 128},      {"wc4_lc64", 4, 64, 128},      {"wc2_nochunk", 2, -1, 128},
+    {"wc2_lc256", 2, 256, 128},    {"wc4_lc512", 4, 512, 128},    {"wc1_lc128", 1, 128, 128},
+    {"wc2_auto_r168", 2, 0, 168},  {"wc4_auto_r168", 4, 0, 168},  {"wc4_lc64_r168", 4, 64, 168},
+    {"wc2_lc128_r168", 2, 128, 168},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
-// Minimum resident CTAs per SM the kernels are compiled for: 16 warps per
-// SM, a register cap of 65536 / 512 = 128 per thread.
-template <int WC>
+// Minimum resident CTAs per SM the kernels are compiled for: R = 128 gives
+// 16 warps per SM and a register cap of 65536 / 512 = 128 per thread;
+// R = 168 gives 12 warps per SM and a cap of 168 (more room for the compiler
+// to keep loads in flight and interleave steps).
+template <int WC, int R>
 struct MinBlocks {
-    static constexpr int value = 16 / WC;
+    static constexpr int value = (R == 128 ? 16 : 12) / WC;
 };
 
-template <typename Tin, int WC, int MODE, bool PACK>
+template <typename Tin, int WC, int MODE, int R>
 cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
 {
     using Sh = ChunkShape<WC>;
-    auto kern = chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC>::value, PACK>;
+    auto kern = chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, true>;
     const size_t smem = Sh::SMEM_BYTES;
     if (smem > 48 * 1024) {
         cudaError_t e =
@@ -42,14 +45,14 @@ cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <typename Tin, int WC, bool PACK>
+template <typename Tin, int WC, int R>
 cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
 {
     cudaError_t e;
     if (plan.NC > 1) {
         if (ev)
             cudaEventRecord(ev[0], st);
-        e = launch_chunk<Tin, WC, kModeState, PACK>(p, plan.NC - 1, st);
+        e = launch_chunk<Tin, WC, kModeState, R>(p, plan.NC - 1, st);
         if (e != cudaSuccess)
             return e;
         if (ev)
@@ -63,7 +66,7 @@ cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
     }
     if (ev)
         cudaEventRecord(ev[2], st);
-    e = launch_chunk<Tin, WC, kModeOutput, PACK>(p, plan.NC, st);
+    e = launch_chunk<Tin, WC, kModeOutput, R>(p, plan.NC, st);
     if (ev)
         cudaEventRecord(ev[3], st);
     return e;
@@ -80,17 +83,31 @@ const VariantInfo *variant(int i)
     return &kVariants[i];
 }
 
+namespace {
+// Sequences of a call are split into chunks when there are too few of them
+// to give every SM sub-partition about four resident warps.
+constexpr long long kWantLanes = 148LL * 16 * 32;
+
+bool wants_chunks(long long seqs, long long L)
+{
+    return seqs < kWantLanes / 2 && L > 512;
+}
+}  // namespace
+
 int pick_variant(int two_d, int B, int D, int H, int W, int N, int K)
 {
-    (void)two_d;
-    (void)B;
-    (void)H;
-    (void)W;
     (void)N;
-    (void)K;
-    if (D <= 32)
-        return 2;   // wc1_auto
-    return 0;       // wc2_auto
+    const long long L = two_d ? (long long)H * W : (long long)W;
+    // chunked shapes: 128-step chunks with the 168-register kernels (fewer,
+    // fuller warps hide the longer per-chunk dependency chains better)
+    if (wants_chunks((long long)B * K * D, L))
+        return 12;  // wc2_lc128_r168
+    // otherwise the widest CTA that leaves no channel tile mostly empty
+    if (D % 128 == 0)
+        return 1;   // wc4_auto
+    if (D % 64 == 0 || D > 64)
+        return 0;   // wc2_auto
+    return 2;       // wc1_auto
 }
 
 Plan make_plan(int v, int B, int D, int L, int K)
@@ -99,7 +116,7 @@ Plan make_plan(int v, int B, int D, int L, int K)
     Plan pl;
     pl.variant = v;
     pl.wc = vi->wc;
-    pl.pack = vi->pack;
+    pl.regs = vi->regs;
     int lc;
     if (vi->chunk > 0) {
         lc = vi->chunk;
@@ -108,9 +125,8 @@ Plan make_plan(int v, int B, int D, int L, int K)
     } else {
         // enough lanes for about four resident warps per SM sub-partition on
         // 148 SMs; short sequences are never split
-        const long long want = 148LL * 16 * 32;
         const long long seqs = (long long)B * K * D;
-        long long nc = (seqs >= want / 2 || L <= 512) ? 1 : (want + seqs - 1) / seqs;
+        long long nc = wants_chunks(seqs, L) ? (kWantLanes + seqs - 1) / seqs : 1;
         if (nc < 1)
             nc = 1;
         lc = (int)((L + nc - 1) / nc);
@@ -129,31 +145,17 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 {
     p.LC = plan.LC;
     p.NC = plan.NC;
-    if (!plan.pack) {
-        switch (plan.wc) {
-        case 2:
-            return bf16 ? launch_passes<__nv_bfloat16, 2, false>(plan, p, st, ev)
-                        : launch_passes<float, 2, false>(plan, p, st, ev);
-        case 4:
-            return bf16 ? launch_passes<__nv_bfloat16, 4, false>(plan, p, st, ev)
-                        : launch_passes<float, 4, false>(plan, p, st, ev);
-        default:
-            return cudaErrorInvalidValue;
-        }
-    }
-    switch (plan.wc) {
-    case 1:
-        return bf16 ? launch_passes<__nv_bfloat16, 1, true>(plan, p, st, ev)
-                    : launch_passes<float, 1, true>(plan, p, st, ev);
-    case 2:
-        return bf16 ? launch_passes<__nv_bfloat16, 2, true>(plan, p, st, ev)
-                    : launch_passes<float, 2, true>(plan, p, st, ev);
-    case 4:
-        return bf16 ? launch_passes<__nv_bfloat16, 4, true>(plan, p, st, ev)
-                    : launch_passes<float, 4, true>(plan, p, st, ev);
-    default:
-        return cudaErrorInvalidValue;
-    }
+#define SS2D_DISPATCH(WCV, RV)                                                   \
+    if (plan.wc == WCV && plan.regs == RV)                                       \
+        return bf16 ? launch_passes<__nv_bfloat16, WCV, RV>(plan, p, st, ev)     \
+                    : launch_passes<float, WCV, RV>(plan, p, st, ev);
+    SS2D_DISPATCH(1, 128)
+    SS2D_DISPATCH(2, 128)
+    SS2D_DISPATCH(4, 128)
+    SS2D_DISPATCH(2, 168)
+    SS2D_DISPATCH(4, 168)
+#undef SS2D_DISPATCH
+    return cudaErrorInvalidValue;
 }
 
 namespace {

@@ -15,14 +15,14 @@ struct VariantInfo {
     const char *name;
     int wc;
     int chunk;
-    int pack;   // 1: packed f32x2 arithmetic; 0: scalar float32
+    int regs;   // register cap per thread the kernels are compiled for (128 or 168)
 };
 
 // How one call is executed.
 struct Plan {
     int variant;
     int wc;
-    int pack;
+    int regs;
     int LC;        // steps per chunk (multiple of 32)
     int NC;        // chunks per sequence
     int launches;  // kernel launches of a forward call
