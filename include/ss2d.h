@@ -38,8 +38,9 @@
  * must be of the same kind.
  *   - device pointers: the call is asynchronous on `stream` and returns after
  *     enqueueing.  Scratch for the per-direction partial outputs (K > 1,
- *     4*B*K*D*L bytes) is taken from a stream-ordered pool on `stream` and
- *     returned on `stream`.  Nothing is synchronised.
+ *     4*B*K*D*L bytes) and, when sequences are split into chunks, for the
+ *     chunk states (68*B*K*D*(chunks-1) bytes) is taken from a stream-ordered
+ *     pool on `stream` and returned on `stream`.  Nothing is synchronised.
  *   - host pointers (pageable or pinned): the call copies the inputs to the
  *     current device, runs the device path, copies y back and synchronises
  *     `stream` before returning.  Device buffers come from the same pool.
@@ -119,7 +120,9 @@ int selective_scan_fwd(const void *u, const void *delta, const float *A_log,
  * with two_d = 0: (B, K, D, L), direction 1 flipped back to sequence order).
  * This is what the tutorial's CrossScanModule concatenates before its output
  * projection.  Device pointers only (SS2D_ERR_PTR otherwise); asynchronous
- * on `stream`; no scratch memory.  variant as in ss2d_forward_ex. */
+ * on `stream`; scratch from the same stream-ordered pool as ss2d_forward
+ * (the scan-order rows, then a copy kernel puts each direction in pixel
+ * order).  variant as in ss2d_forward_ex. */
 int ss2d_scan_directions(const void *x, const void *delta, const float *A_log,
                          const void *Bs, const void *Cs, const float *Dskip,
                          const float *delta_bias, float *y_dir,
