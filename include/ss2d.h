@@ -87,7 +87,9 @@ typedef enum {
     SS2D_ERR_ALLOC = -7,  /* device memory for scratch or staging ran out    */
     SS2D_ERR_CUDA = -8,   /* a CUDA call failed; see ss2d_last_error()       */
     SS2D_ERR_PTR = -9,    /* host and device pointers mixed in one call      */
-    SS2D_ERR_VARIANT = -10 /* unknown kernel variant (ss2d_forward_ex)       */
+    SS2D_ERR_VARIANT = -10, /* unknown kernel variant (ss2d_forward_ex)      */
+    SS2D_ERR_SCRATCH = -11  /* needs more scratch than ss2d_forward_noalloc's
+                               fixed buffer holds                             */
 } ss2d_status;
 
 typedef enum {
@@ -174,11 +176,46 @@ const char *ss2d_variant_name(int i);
  * (two_d = 1 for ss2d_forward, 0 for the 1D call; H = 1, W = L for 1D). */
 int ss2d_pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
 
+/* Size in bytes of the fixed device scratch buffer of ss2d_forward_noalloc
+ * (96 MiB): enough for the VMamba-T stage-1 SS2D layer, B = 8, D = 192,
+ * 56 x 56, K = 4. */
+#define SS2D_NOALLOC_SCRATCH_BYTES (96u * 1024u * 1024u)
+
+/* ss2d_forward that allocates no memory.  There is no counterpart in the
+ * papers: the entry point exists for callers that cannot let a library
+ * allocate device memory once they run -- programs whose own caching
+ * allocator has reserved (nearly) all device memory, latency-bound loops in
+ * which a growing pool would call into the driver, processes held to a fixed
+ * device footprint.  Its scratch (the per-direction rows and chunk states
+ * ss2d_forward takes from its pool: 4*B*K*D*H*W bytes when K > 1, plus
+ * 68*B*K*D*(chunks-1) bytes when ss2d_plan reports chunks > 1, each rounded
+ * up to 256) lives in one statically sized device buffer of
+ * SS2D_NOALLOC_SCRATCH_BYTES per device, part of the library's device image.
+ *   - Same arguments, layouts, results and limits as ss2d_forward, DEVICE
+ *     pointers only (SS2D_ERR_PTR otherwise); asynchronous on `stream`.
+ *   - A problem whose scratch would not fit returns SS2D_ERR_SCRATCH before
+ *     anything is enqueued; ss2d_last_error() then gives the bytes needed.
+ *   - First call on a device: the buffer's address on that device is looked
+ *     up (with that device current) and kept.  The lookup loads the module
+ *     that holds the buffer, which is when its memory is reserved; make this
+ *     first call on each device before any stream capture begins.
+ *   - Nothing in the buffer has to start at zero: every word a call reads is
+ *     written earlier in the same call.
+ *   - One buffer per device: calls on one device whose work can overlap in
+ *     time (other streams, other host threads) race on it and give wrong
+ *     results.  Serialise them: one stream, or streams ordered by events. */
+int ss2d_forward_noalloc(const void *x, const void *delta, const float *A_log,
+                         const void *Bs, const void *Cs, const float *Dskip,
+                         const float *delta_bias, float *y,
+                         int B, int D, int H, int W, int N, int K, int dtype,
+                         void *stream);
+
 /* Static text for a status code. */
 const char *ss2d_status_string(int status);
 
 /* CUDA's message for the last SS2D_ERR_CUDA / SS2D_ERR_ALLOC seen on the
- * calling thread ("" if none). */
+ * calling thread, or the scratch bytes of the last SS2D_ERR_SCRATCH ("" if
+ * none). */
 const char *ss2d_last_error(void);
 
 #ifdef __cplusplus

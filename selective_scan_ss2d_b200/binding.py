@@ -17,6 +17,7 @@ import torch
 
 SS2D_F32 = 0
 SS2D_BF16 = 1
+NOALLOC_SCRATCH_BYTES = 96 * 1024 * 1024   # SS2D_NOALLOC_SCRATCH_BYTES of the C header
 _DTYPES = {torch.float32: SS2D_F32, torch.bfloat16: SS2D_BF16}
 
 _lock = threading.Lock()
@@ -62,6 +63,8 @@ def lib() -> ctypes.CDLL:
             L.ss2d_scan_directions.restype = i
             L.ss2d_plan.argtypes = [i] * 8 + [ctypes.POINTER(ctypes.c_int)] * 3
             L.ss2d_plan.restype = i
+            L.ss2d_forward_noalloc.argtypes = fwd + [i] * 7 + [vp]
+            L.ss2d_forward_noalloc.restype = i
             L.ss2d_forward_timed.argtypes = fwd + [i] * 8 + [vp, i, ctypes.POINTER(ctypes.c_float)]
             L.ss2d_forward_timed.restype = i
             L.ss2d_num_variants.argtypes = []
@@ -99,7 +102,7 @@ def _check(status: int):
         L = lib()
         msg = L.ss2d_status_string(status).decode()
         detail = L.ss2d_last_error().decode()
-        raise SS2DError(status, msg + (f" -- {detail}" if detail and status in (-7, -8) else ""))
+        raise SS2DError(status, msg + (f" -- {detail}" if detail and status in (-7, -8, -11) else ""))
 
 
 def _ptr(t: torch.Tensor):
@@ -161,6 +164,29 @@ def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y=None, *, stream=N
     rc = lib().ss2d_forward_ex(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
                                _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, H, W, N, K,
                                dt, st, int(variant))
+    _check(rc)
+    return y
+
+
+def ss2d_forward_noalloc(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, *, stream=None):
+    """ss2d_forward without any allocation by the library: scratch lives in a
+    fixed device buffer of NOALLOC_SCRATCH_BYTES per device (SS2DError with
+    status -11 when the problem needs more).  Device tensors only, y given by
+    the caller; calls on one device must not overlap in time."""
+    B, D, H, W = x.shape
+    K, N = delta.shape[1], Bs.shape[2]
+    L = H * W
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for ss2d_forward_noalloc")
+    if y is None:
+        raise ValueError("ss2d_forward_noalloc needs a caller-provided y")
+    y, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, (B, D, H, W))
+    st = _stream(on_gpu, x.device, stream)
+    rc = lib().ss2d_forward_noalloc(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                                    _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, H, W, N, K,
+                                    dt, st)
     _check(rc)
     return y
 

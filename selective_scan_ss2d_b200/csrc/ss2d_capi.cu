@@ -323,6 +323,11 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
 
 }  // namespace
 
+namespace ss2d {
+void record_error(const char *what, cudaError_t e) { set_error(what, e); }
+void record_message(const char *text) { snprintf(g_last_error, sizeof(g_last_error), "%s", text); }
+}  // namespace ss2d
+
 extern "C" {
 
 int ss2d_forward_ex(const void *x, const void *delta, const float *A_log, const void *Bs,
@@ -496,6 +501,9 @@ const char *ss2d_status_string(int status)
         return "pointers mix host and device memory, or name another device";
     case SS2D_ERR_VARIANT:
         return "unknown kernel variant";
+    case SS2D_ERR_SCRATCH:
+        return "problem needs more scratch than the fixed buffer of ss2d_forward_noalloc "
+               "(SS2D_NOALLOC_SCRATCH_BYTES) holds";
     default:
         return "unknown status";
     }

@@ -45,4 +45,8 @@ cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W
                          int two_d, int sum, cudaStream_t st);
 size_t merge_smem_bytes(int H, int W, int K, int two_d);
 
+// Text that ss2d_last_error() returns on the calling thread.
+void record_error(const char *what, cudaError_t e);
+void record_message(const char *text);
+
 }  // namespace ss2d

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for st in range(0, -11, -1):
+    for st in range(0, -12, -1):
         s = binding.ss2d_status_string(st)
         assert s and s != "unknown status"
     assert binding.ss2d_status_string(-99) == "unknown status"
