@@ -32,7 +32,7 @@
 // (channel, step) and parks (dt, u) in a warp-private shared-memory tile, and
 // its outputs go back as 16-byte vectors of its scan-order row.  B and C of a
 // sub-chunk (shared by every channel of the CTA) are staged once per CTA as a
-// float32 [step][32] tile read with broadcast float4 loads, also one
+// float32 [slot][step] tile read with broadcast float4 loads, also one
 // sub-chunk ahead.  Nothing waits on a flag.
 //
 // exp(dt*A) runs on the MUFU unit as 2^(dt * A*log2(e)).  The float32 pair
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     constexpr int NT = Sh::NT, BCPT = Sh::BC_PER_THREAD;
 
     extern __shared__ float4 smem_f4[];
-    float4 *sBC = smem_f4;   // [2][kT][8], slot q of step t stored at t*8 + (q ^ (t & 7))
+    float4 *sBC = smem_f4;   // [2][8][kT]: slot q of step t at q*kT + t
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     float2 *sDU = reinterpret_cast<float2 *>(sBC + 2 * Sh::BC_ENTRIES) + warp * Sh::DU_WARP;
@@ -340,30 +340,44 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     // softplus once per (channel, step); dt and u to the warp tile [t][lane]
     auto unpack_store = [&](int buf, int ls) {
         float2 *du = sDU + buf * (kT * 32) + lane;
+        if (ls + kT <= l_end) {   // whole sub-chunk inside the chunk
+            if (xmode == 1) {
 #pragma unroll
-        for (int i = 0; i < kT; ++i) {
-            const bool ok = ls + i < l_end;
-            const float dt = ok ? softplus_f(pd.get(i) + bias) : 0.f;
-            const float u = (xmode == 1) ? px.get(kT - 1 - i) : px.get(i);
-            du[i * 32] = make_float2(dt, u);
+                for (int i = 0; i < kT; ++i)
+                    du[i * 32] = make_float2(softplus_f(pd.get(i) + bias), px.get(kT - 1 - i));
+            } else {
+#pragma unroll
+                for (int i = 0; i < kT; ++i)
+                    du[i * 32] = make_float2(softplus_f(pd.get(i) + bias), px.get(i));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kT; ++i) {
+                const bool ok = ls + i < l_end;
+                const float dt = ok ? softplus_f(pd.get(i) + bias) : 0.f;
+                const float u = (xmode == 1) ? px.get(kT - 1 - i) : px.get(i);
+                du[i * 32] = make_float2(dt, u);
+            }
         }
     };
     // B|C: float4 entry e = (slot q = e / kT, step t = e % kT) holds rows
     // 4q..4q+3 of B (q < 4) or C (q >= 4) at step t
     float4 rbc[BCPT];
     auto load_bc = [&](int ls) {
+        const bool whole = N == kNP && ls + kT <= l_end;
 #pragma unroll
         for (int r = 0; r < BCPT; ++r) {
             const int e = tid + r * NT;
             const int q = e / kT, t = e % kT;
             const int l = ls + t;
             const Tin *src = (q < 4) ? Bg : Cg;
+            const bool ok = (Sh::BC_ENTRIES % NT == 0 || e < Sh::BC_ENTRIES) &&
+                            (whole || l < l_end);
             float v[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int n = (q & 3) * 4 + i;
-                v[i] = (e < Sh::BC_ENTRIES && l < l_end && n < N) ? to_f32(src[(size_t)n * L + l])
-                                                                  : 0.f;
+                v[i] = (ok && (whole || n < N)) ? to_f32(src[(size_t)n * L + l]) : 0.f;
             }
             rbc[r] = make_float4(v[0], v[1], v[2], v[3]);
         }
@@ -372,10 +386,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
         for (int r = 0; r < BCPT; ++r) {
             const int e = tid + r * NT;
-            if (e < Sh::BC_ENTRIES) {
-                const int q = e / kT, t = e % kT;
-                sBC[buf * Sh::BC_ENTRIES + t * 8 + (q ^ (t & 7))] = rbc[r];
-            }
+            if (Sh::BC_ENTRIES % NT == 0 || e < Sh::BC_ENTRIES)
+                sBC[buf * Sh::BC_ENTRIES + e] = rbc[r];
         }
     };
 
@@ -403,12 +415,11 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
             const float du = dt * u;
             const float2 dt2 = make_float2(dt, dt);
             const float2 du2 = make_float2(du, du);
-            const float4 *row = sb + t * 8;
-            const int sw = t & 7;
+            const float4 *col = sb + t;   // slot q at col[q * kT]
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float4 bv = row[q ^ sw];
+                const float4 bv = col[q * kT];
                 if constexpr (PACK) {
                     const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
                     const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
                     h2[2 * q + 1] =
                         __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
                     if (MODE == kModeOutput) {
-                        const float4 cv = row[(4 + q) ^ sw];
+                        const float4 cv = col[(4 + q) * kT];
                         acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
                         acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
                     }
@@ -432,7 +443,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
                     h2[2 * q + 1].x = fmaf(a2, h2[2 * q + 1].x, du * bv.z);
                     h2[2 * q + 1].y = fmaf(a3, h2[2 * q + 1].y, du * bv.w);
                     if (MODE == kModeOutput) {
-                        const float4 cv = row[(4 + q) ^ sw];
+                        const float4 cv = col[(4 + q) * kT];
                         acc0.x = fmaf(cv.x, h2[2 * q].x, acc0.x);
                         acc0.y = fmaf(cv.y, h2[2 * q].y, acc0.y);
                         acc1.x = fmaf(cv.z, h2[2 * q + 1].x, acc1.x);

@@ -4,18 +4,22 @@
 #include <cuda_bf16.h>
 
 #include "ss2d_kernels.cuh"
+#include "ss2d_quad.cuh"
 
 namespace ss2d {
 
 namespace {
 
-// name: wc<W>_<chunking>; wc = 32-channel warps per CTA.
+// name: wc<W>_<chunking>: one lane per channel, wc = 32-channel warps per CTA;
+// quad<W>_<chunking>: four lanes per channel, W warps of 8 channels per CTA.
 const VariantInfo kVariants[] = {
     {"wc2_auto", 2, 0, 128},       {"wc4_auto", 4, 0, 128},       {"wc1_auto", 1, 0, 128},
     {"wc2_lc16", 2, 16, 128},      {"wc4_lc64", 4, 64, 128},      {"wc2_nochunk", 2, -1, 128},
     {"wc2_lc256", 2, 256, 128},    {"wc4_lc512", 4, 512, 128},    {"wc1_lc128", 1, 128, 128},
     {"wc2_auto_r168", 2, 0, 168},  {"wc4_auto_r168", 4, 0, 168},  {"wc4_lc64_r168", 4, 64, 168},
     {"wc2_lc128_r168", 2, 128, 168},
+    {"quad4_auto", 4, 0, 128, 1},  {"quad4_nochunk", 4, -1, 128, 1},
+    {"quad4_lc512", 4, 512, 128, 1},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
@@ -45,14 +49,33 @@ cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <typename Tin, int WC, int R>
+template <typename Tin, int MODE, int NW, int R>
+cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st)
+{
+    constexpr int MINB = 65536 / (32 * NW * R);
+    constexpr int CH = kQCh * NW;
+    dim3 grid((unsigned)p.K, (unsigned)((p.D + CH - 1) / CH), (unsigned)(p.B * ncg));
+    quad_scan_kernel<Tin, MODE, NW, MINB><<<grid, 32 * NW, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tin, int LAYOUT, int WC, int R, int MODE>
+cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st)
+{
+    if constexpr (LAYOUT == 0)
+        return launch_chunk<Tin, WC, MODE, R>(p, ncg, st);
+    else
+        return launch_quad<Tin, MODE, WC, R>(p, ncg, st);
+}
+
+template <typename Tin, int LAYOUT, int WC, int R>
 cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
 {
     cudaError_t e;
     if (plan.NC > 1) {
         if (ev)
             cudaEventRecord(ev[0], st);
-        e = launch_chunk<Tin, WC, kModeState, R>(p, plan.NC - 1, st);
+        e = launch_pass<Tin, LAYOUT, WC, R, kModeState>(p, plan.NC - 1, st);
         if (e != cudaSuccess)
             return e;
         if (ev)
@@ -66,7 +89,7 @@ cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
     }
     if (ev)
         cudaEventRecord(ev[2], st);
-    e = launch_chunk<Tin, WC, kModeOutput, R>(p, plan.NC, st);
+    e = launch_pass<Tin, LAYOUT, WC, R, kModeOutput>(p, plan.NC, st);
     if (ev)
         cudaEventRecord(ev[3], st);
     return e;
@@ -117,6 +140,7 @@ Plan make_plan(int v, int B, int D, int L, int K)
     pl.variant = v;
     pl.wc = vi->wc;
     pl.regs = vi->regs;
+    pl.layout = vi->layout;
     int lc;
     if (vi->chunk > 0) {
         lc = vi->chunk;
@@ -126,7 +150,14 @@ Plan make_plan(int v, int B, int D, int L, int K)
         // enough lanes for about four resident warps per SM sub-partition on
         // 148 SMs; short sequences are never split
         const long long seqs = (long long)B * K * D;
-        long long nc = wants_chunks(seqs, L) ? (kWantLanes + seqs - 1) / seqs : 1;
+        long long nc;
+        if (vi->layout == 1) {
+            // quad: about eight resident warps per SM are enough
+            const long long lanes = seqs * kQLanes, want = kWantLanes / 2;
+            nc = (lanes < want && L > 512) ? (want + lanes - 1) / lanes : 1;
+        } else {
+            nc = wants_chunks(seqs, L) ? (kWantLanes + seqs - 1) / seqs : 1;
+        }
         if (nc < 1)
             nc = 1;
         lc = (int)((L + nc - 1) / nc);
@@ -145,15 +176,16 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 {
     p.LC = plan.LC;
     p.NC = plan.NC;
-#define SS2D_DISPATCH(WCV, RV)                                                   \
-    if (plan.wc == WCV && plan.regs == RV)                                       \
-        return bf16 ? launch_passes<__nv_bfloat16, WCV, RV>(plan, p, st, ev)     \
-                    : launch_passes<float, WCV, RV>(plan, p, st, ev);
-    SS2D_DISPATCH(1, 128)
-    SS2D_DISPATCH(2, 128)
-    SS2D_DISPATCH(4, 128)
-    SS2D_DISPATCH(2, 168)
-    SS2D_DISPATCH(4, 168)
+#define SS2D_DISPATCH(LY, WCV, RV)                                                  \
+    if (plan.layout == LY && plan.wc == WCV && plan.regs == RV)                     \
+        return bf16 ? launch_passes<__nv_bfloat16, LY, WCV, RV>(plan, p, st, ev)    \
+                    : launch_passes<float, LY, WCV, RV>(plan, p, st, ev);
+    SS2D_DISPATCH(0, 1, 128)
+    SS2D_DISPATCH(0, 2, 128)
+    SS2D_DISPATCH(0, 4, 128)
+    SS2D_DISPATCH(0, 2, 168)
+    SS2D_DISPATCH(0, 4, 168)
+    SS2D_DISPATCH(1, 4, 128)
 #undef SS2D_DISPATCH
     return cudaErrorInvalidValue;
 }

@@ -8,14 +8,15 @@ namespace ss2d {
 
 struct ScanParams;
 
-// A kernel variant: CTA width (32*wc channels) and chunking policy
+// A kernel variant: layout, CTA width (wc warps) and chunking policy
 // (chunk = 0: chosen from the shape; chunk > 0: that many steps per chunk;
 // chunk < 0: never chunk).
 struct VariantInfo {
     const char *name;
     int wc;
     int chunk;
-    int regs;   // register cap per thread the kernels are compiled for (128 or 168)
+    int regs;   // register cap per thread the kernels are compiled for
+    int layout; // 0: one lane per channel (chunk_scan_kernel); 1: four (quad_scan_kernel)
 };
 
 // How one call is executed.
@@ -23,6 +24,7 @@ struct Plan {
     int variant;
     int wc;
     int regs;
+    int layout;
     int LC;        // steps per chunk (multiple of 32)
     int NC;        // chunks per sequence
     int launches;  // kernel launches of a forward call
