@@ -20,7 +20,7 @@
 //   3. chunk_scan_kernel<..., kModeOutput>: every chunk from its true entry
 //      state, writing y_k in scan order (per-direction scratch, or y when
 //      K = 1);
-//   4. merge_kernel (K > 1): y[p] = ((Y_0[s_0(p)] + Y_1[s_1(p)]) +
+//   4. merge2_kernel (K > 1): y[p] = ((Y_0[s_0(p)] + Y_1[s_1(p)]) +
 //      Y_2[s_2(p)]) + Y_3[s_3(p)], s_k the pixel -> scan-step map of
 //      direction k (cross_merge), always in that order.
 // Chunking costs one extra exp per update on the chunked workloads only,
@@ -530,121 +530,153 @@ __global__ void carry_kernel(const ScanParams p)
     }
 }
 
-// cross_merge: scan-order rows part[(b,k,d)][l] -> pixel order.  A CTA of
-// kMergeThreads threads covers kMergePix "slots": 2^cpb_log2 consecutive
-// (b,d) channels, each with one band of its pixels.  Two band shapes:
-//  * cols = 1 (SS2D, K = 4): R image rows padded to 2^rp_log2 x 2^wp_log2
-//    slots; the column-major directions are gathered through a shared-memory
-//    tile, so global reads stay coalesced (the band of each image column is a
-//    run of consecutive scan steps);
-//  * cols = 0 (K <= 2, SS2D or 1D): 2^wp_log2 consecutive pixels.
-// Slots map to (row, column) with shifts and masks, and every thread issues
-// all of its loads before it uses any (memory-level parallelism).
+// cross_merge, band form: a CTA covers `rows` full image rows (the band
+// starting at row h0 = blockIdx.y * R) of CG consecutive (b, d) channels.
+//  * cols (SS2D, K = 4): for each channel, the column-major directions'
+//    values of the band are read as runs (column w of the band is scan steps
+//    w*H + h0 .. w*H + h0 + rows - 1 of direction 2, the mirror run of
+//    direction 3) and transposed through shared memory [rows][W + 1];
+//  * the row-major directions (and every direction of K <= 2 or 1D) are
+//    contiguous: direction 0 at p, direction 1 at L-1-p.
+// VEC = 4: float4 accesses (needs W % 4 == 0, and H % 4 == 0 and R % 4 == 0
+// when cols); VEC = 1: scalar.
 //   sum = 1: y[b,d,p] = ((Y_0 + Y_1) + Y_2) + Y_3       (first K terms)
 //   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
-constexpr int kMergeThreads = 128;
-constexpr int kMergePix = 512;
-constexpr int kMergeIt = 4;   // kMergePix / kMergeThreads
+constexpr int kMerge2Threads = 256;
 
-__global__ void __launch_bounds__(kMergeThreads)
-    merge_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
-                 int W, int K, int cols, int sum, int R, int rp_log2, int wp_log2,
-                 int cpb_log2, int nblk)
+template <int VEC, int CG>
+__global__ void __launch_bounds__(kMerge2Threads)
+    merge2_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
+                  int W, int K, int cols, int sum, int R)
 {
-    extern __shared__ float smem_m[];   // [cpb][2][W][R + 1] when cols
-    const long long L = (long long)H * W;
+    extern __shared__ float smem_m2[];   // [CG][2][R][W + 1] when cols
+    const int L = H * W;
     const size_t kstride = (size_t)D * L;
-    const int RP = 1 << rp_log2, WP = 1 << wp_log2;
-    const int S_log2 = rp_log2 + wp_log2;          // slots per channel band
-    const long long ch_total = (long long)B * D;
-    const int blk = blockIdx.x % nblk;
-    const long long bd0 = (long long)(blockIdx.x / nblk) << cpb_log2;
-    const int h0 = blk * R;
-    const int hr = cols ? min(R, H - h0) : 0;
-    const long long p0 = cols ? (long long)h0 * W : (long long)blk * WP;
-    const size_t tile = 2 * (size_t)W * (R + 1);
+    const long long nch = (long long)B * D;
+    const long long bd0 = (long long)blockIdx.x * CG;
+    const int h0 = blockIdx.y * R;
+    const int rows = min(R, H - h0);
+    const int p0 = h0 * W, n = rows * W;
+    const int WS = W + 1;
+    long long b = bd0 / D;
+    int d = (int)(bd0 - b * D);
+    int nc = 0;   // channels of this CTA that exist
     if (cols) {
-        float g2[kMergeIt], g3[kMergeIt];
-        int gi[kMergeIt];
-#pragma unroll
-        for (int i = 0; i < kMergeIt; ++i) {   // slot -> (channel, column, band row)
-            const int e = threadIdx.x + i * kMergeThreads;
-            const int c = e >> S_log2, sl = e & ((1 << S_log2) - 1);
-            const int w = sl >> rp_log2, hh = sl & (RP - 1);
-            const long long bd = bd0 + c;
-            const bool ok = bd < ch_total && w < W && hh < hr;
-            gi[i] = ok ? (int)(c * tile) + w * (R + 1) + hh : -1;
-            g2[i] = g3[i] = 0.f;
-            if (ok) {
-                const float *rows = part + ((size_t)(bd / D) * K * D + (size_t)(bd % D)) * L;
-                const long long s2 = (long long)w * H + h0 + hh;
-                g2[i] = __ldg(rows + 2 * kstride + s2);
-                g3[i] = __ldg(rows + 3 * kstride + (L - 1 - s2));
+        long long bb = b;
+        int dd = d;
+        for (int c = 0; c < CG && bd0 + c < nch; ++c, ++nc) {
+            const float *r2 = part + ((size_t)(bb * K + 2) * D + dd) * L;
+            const float *r3 = r2 + kstride;
+            float *s2 = smem_m2 + (size_t)c * 2 * R * WS;
+            float *s3 = s2 + (size_t)R * WS;
+            if (VEC == 4) {
+                const int rq = R / 4;              // float4 runs per column
+                const int per = kMerge2Threads / rq;
+                const int q = threadIdx.x % rq;
+                for (int w = threadIdx.x / rq; w < W; w += per) {
+                    const int r = 4 * q;
+                    if (threadIdx.x < per * rq && r < rows) {
+                        const int s = w * H + h0 + r;
+                        const float4 a = __ldg(reinterpret_cast<const float4 *>(r2 + s));
+                        const float4 m = __ldg(reinterpret_cast<const float4 *>(r3 + (L - 4 - s)));
+                        s2[(r + 0) * WS + w] = a.x;
+                        s2[(r + 1) * WS + w] = a.y;
+                        s2[(r + 2) * WS + w] = a.z;
+                        s2[(r + 3) * WS + w] = a.w;
+                        s3[(r + 0) * WS + w] = m.w;
+                        s3[(r + 1) * WS + w] = m.z;
+                        s3[(r + 2) * WS + w] = m.y;
+                        s3[(r + 3) * WS + w] = m.x;
+                    }
+                }
+            } else {
+                // element e of the band in column-major order: w = e / rows
+                for (int e = threadIdx.x; e < n; e += kMerge2Threads) {
+                    const int w = e / rows, r = e - w * rows;
+                    const int s = w * H + h0 + r;
+                    s2[r * WS + w] = __ldg(r2 + s);
+                    s3[r * WS + w] = __ldg(r3 + (L - 1 - s));
+                }
             }
-        }
-#pragma unroll
-        for (int i = 0; i < kMergeIt; ++i) {
-            if (gi[i] >= 0) {
-                smem_m[gi[i]] = g2[i];
-                smem_m[gi[i] + W * (R + 1)] = g3[i];
+            if (++dd == D) {
+                dd = 0;
+                ++bb;
             }
         }
         __syncthreads();
+    } else {
+        nc = (int)min((long long)CG, nch - bd0);
     }
-    float v0[kMergeIt], v1[kMergeIt];
-    long long pixv[kMergeIt];   // pixel, -1 if the slot is empty
-    size_t rowk[kMergeIt], rowy[kMergeIt];
-    int si[kMergeIt];
-#pragma unroll
-    for (int i = 0; i < kMergeIt; ++i) {
-        const int e = threadIdx.x + i * kMergeThreads;
-        const int c = e >> S_log2, sl = e & ((1 << S_log2) - 1);
-        const long long bd = bd0 + c;
-        long long pix;
-        bool ok;
-        if (cols) {   // slot -> (channel, band row, column)
-            const int hh = sl >> wp_log2, w = sl & (WP - 1);
-            ok = bd < ch_total && hh < hr && w < W;
-            pix = p0 + (long long)hh * W + w;
-            si[i] = (int)(c * tile) + w * (R + 1) + hh;
-        } else {      // slot -> (channel, pixel of the band)
-            pix = p0 + sl;
-            ok = bd < ch_total && pix < L;
-            si[i] = 0;
-        }
-        const size_t b = ok ? (size_t)(bd / D) : 0, d = ok ? (size_t)(bd % D) : 0;
-        rowk[i] = (b * K * D + d) * (size_t)L;
-        rowy[i] = (b * D + d) * (size_t)L;
-        pixv[i] = ok ? pix : -1;
-        const float *rows = part + rowk[i];
-        v0[i] = ok ? __ldg(rows + pix) : 0.f;
-        v1[i] = (ok && K >= 2) ? __ldg(rows + kstride + (L - 1 - pix)) : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < kMergeIt; ++i) {
-        const long long pix = pixv[i];
-        if (pix < 0)
-            continue;
-        const float v2 = cols ? smem_m[si[i]] : 0.f;
-        const float v3 = cols ? smem_m[si[i] + W * (R + 1)] : 0.f;
-        if (sum) {
-            float acc = v0[i];
-            if (K >= 2)
-                acc += v1[i];
-            if (K == 4) {
-                acc += v2;
-                acc += v3;
+    for (int c = 0; c < nc; ++c) {
+        const size_t rk = ((size_t)b * K * D + d) * L;   // row (b, 0, d) of part
+        const float *r0 = part + rk;
+        const float *r1 = r0 + kstride;
+        const float *s2 = smem_m2 + (size_t)c * 2 * R * WS;
+        const float *s3 = s2 + (size_t)R * WS;
+        float *yo = sum ? y + ((size_t)b * D + d) * L : y + rk;
+        if (VEC == 4) {
+            for (int i = 4 * threadIdx.x; i < n; i += 4 * kMerge2Threads) {
+                const int p = p0 + i;
+                float4 v = __ldg(reinterpret_cast<const float4 *>(r0 + p));
+                float4 v1 = make_float4(0.f, 0.f, 0.f, 0.f), v2 = v1, v3 = v1;
+                if (K >= 2) {
+                    const float4 m = __ldg(reinterpret_cast<const float4 *>(r1 + (L - 4 - p)));
+                    v1 = make_float4(m.w, m.z, m.y, m.x);
+                }
+                if (cols) {
+                    const int r = i / W, w = i - r * W;
+                    const float *a2 = s2 + r * WS + w, *a3 = s3 + r * WS + w;
+                    v2 = make_float4(a2[0], a2[1], a2[2], a2[3]);
+                    v3 = make_float4(a3[0], a3[1], a3[2], a3[3]);
+                }
+                if (sum) {
+                    if (K >= 2)
+                        v = make_float4(v.x + v1.x, v.y + v1.y, v.z + v1.z, v.w + v1.w);
+                    if (cols)
+                        v = make_float4((v.x + v2.x) + v3.x, (v.y + v2.y) + v3.y,
+                                        (v.z + v2.z) + v3.z, (v.w + v2.w) + v3.w);
+                    *reinterpret_cast<float4 *>(yo + p) = v;
+                } else {
+                    *reinterpret_cast<float4 *>(yo + p) = v;
+                    if (K >= 2)
+                        *reinterpret_cast<float4 *>(yo + kstride + p) = v1;
+                    if (cols) {
+                        *reinterpret_cast<float4 *>(yo + 2 * kstride + p) = v2;
+                        *reinterpret_cast<float4 *>(yo + 3 * kstride + p) = v3;
+                    }
+                }
             }
-            y[rowy[i] + pix] = acc;
         } else {
-            // per-direction layout (B, K, D, L): row (b, k, d) = rowk + k*D*L
-            y[rowk[i] + pix] = v0[i];
-            if (K >= 2)
-                y[rowk[i] + kstride + pix] = v1[i];
-            if (K == 4) {
-                y[rowk[i] + 2 * kstride + pix] = v2;
-                y[rowk[i] + 3 * kstride + pix] = v3;
+            for (int i = threadIdx.x; i < n; i += kMerge2Threads) {
+                const int p = p0 + i;
+                float v = __ldg(r0 + p);
+                const float v1 = K >= 2 ? __ldg(r1 + (L - 1 - p)) : 0.f;
+                float v2 = 0.f, v3 = 0.f;
+                if (cols) {
+                    const int r = i / W, w = i - r * W;
+                    v2 = s2[r * WS + w];
+                    v3 = s3[r * WS + w];
+                }
+                if (sum) {
+                    if (K >= 2)
+                        v += v1;
+                    if (cols)
+                        v = (v + v2) + v3;
+                    yo[p] = v;
+                } else {
+                    yo[p] = v;
+                    if (K >= 2)
+                        yo[kstride + p] = v1;
+                    if (cols) {
+                        yo[2 * kstride + p] = v2;
+                        yo[3 * kstride + p] = v3;
+                    }
+                }
             }
+        }
+        if (++d == D) {
+            d = 0;
+            ++b;
         }
     }
 }

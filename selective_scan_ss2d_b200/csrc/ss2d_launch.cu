@@ -191,73 +191,77 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 }
 
 namespace {
-// merge work unit (see merge_kernel): a channel band of at most kMergePix
-// slots, and as many channels per CTA as the kMergePix slots hold
+// merge work unit (see merge2_kernel): bands of R full image rows holding
+// about kMergeTarget pixels, and CG channels per CTA so that a CTA moves
+// about kMergeTarget pixels of every direction; the column-major tiles of a
+// CTA stay within 48 KB of shared memory
+constexpr int kMergeTarget = 4096;
+constexpr size_t kMergeSmemMax = 48 * 1024;
+
 struct MergeShape {
-    int cols, R, rp, wp, cpb_log2, nblk;
-    bool ok;
+    int cols, vec, R, CG, nbands;
+    size_t smem;
 };
+
 MergeShape merge_shape(int H, int W, int K, int two_d)
 {
     MergeShape m{};
     m.cols = (two_d && K == 4) ? 1 : 0;
-    const long long L = (long long)H * W;
-    int wp = 0, rp = 0;
-    if (m.cols) {
-        while ((1 << wp) < W)
-            ++wp;
-        if ((1 << wp) > kMergePix) {
-            m.ok = false;
-            return m;
-        }
-        while ((1 << (rp + 1)) <= (kMergePix >> wp) && (1 << rp) < H)
-            ++rp;
-        m.R = (1 << rp) < H ? (1 << rp) : H;
-        m.nblk = (H + m.R - 1) / m.R;
-    } else {
-        while ((1LL << wp) < L && (1 << wp) < kMergePix)
-            ++wp;
-        m.R = 1;
-        m.nblk = (int)((L + (1LL << wp) - 1) >> wp);
-    }
-    m.rp = rp;
-    m.wp = wp;
-    int cl = 0;   // channels per CTA: the slots left over
-    while ((1 << (cl + 1 + rp + wp)) <= kMergePix)
-        ++cl;
-    m.cpb_log2 = cl;
-    m.ok = true;
+    m.vec = (W % 4 == 0 && (!m.cols || H % 4 == 0)) ? 4 : 1;
+    int R = W >= kMergeTarget ? 1 : kMergeTarget / W;
+    if (R > H)
+        R = H;
+    if (m.vec == 4 && m.cols)
+        R = R < 4 ? 4 : (R & ~3);   // H % 4 == 0, so R <= H stays true
+    m.R = R;
+    m.nbands = (H + R - 1) / R;
+    const long long band = (long long)R * W;
+    int cg = (int)(kMergeTarget / band);
+    if (cg < 1)
+        cg = 1;
+    const size_t per_ch = m.cols ? sizeof(float) * 2 * (size_t)R * (W + 1) : 0;
+    while (cg > 1 && per_ch * cg > kMergeSmemMax)
+        --cg;
+    int cgp = 1;   // compiled channel-group sizes: 1, 2, 4, 8, 16
+    while (cgp * 2 <= cg && cgp < 16)
+        cgp *= 2;
+    m.CG = cgp;
+    m.smem = per_ch * cgp;
     return m;
+}
+
+template <int VEC, int CG>
+cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int B, int D,
+                          int H, int W, int K, int sum, cudaStream_t st)
+{
+    const long long groups = ((long long)B * D + CG - 1) / CG;
+    dim3 grid((unsigned)groups, (unsigned)m.nbands);
+    merge2_kernel<VEC, CG><<<grid, kMerge2Threads, m.smem, st>>>(part, y, B, D, H, W, K, m.cols,
+                                                               sum, m.R);
+    return cudaGetLastError();
 }
 }  // namespace
 
 size_t merge_smem_bytes(int H, int W, int K, int two_d)
 {
-    const MergeShape m = merge_shape(H, W, K, two_d);
-    if (!m.ok)
-        return (size_t)1 << 40;
-    if (!m.cols)
-        return 0;
-    return sizeof(float) * ((size_t)1 << m.cpb_log2) * 2 * (size_t)W * (m.R + 1);
+    return merge_shape(H, W, K, two_d).smem;
 }
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st)
 {
     const MergeShape m = merge_shape(H, W, K, two_d);
-    if (!m.ok)
+    if (m.smem > kMergeSmemMax)
         return cudaErrorInvalidValue;
-    const size_t smem = merge_smem_bytes(H, W, K, two_d);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(merge_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-    }
-    const long long groups = (((long long)B * D) + (1LL << m.cpb_log2) - 1) >> m.cpb_log2;
-    merge_kernel<<<(unsigned)(groups * m.nblk), kMergeThreads, smem, st>>>(
-        part, y, B, D, H, W, K, m.cols, sum, m.R, m.rp, m.wp, m.cpb_log2, m.nblk);
-    return cudaGetLastError();
+    if ((long long)B * D > 0x7fffffffLL * m.CG || m.nbands > 65535)
+        return cudaErrorInvalidConfiguration;
+#define SS2D_MERGE(V, C)                                                             \
+    if (m.vec == V && m.CG == C)                                                     \
+        return launch_merge2<V, C>(m, part, y, B, D, H, W, K, sum, st);
+    SS2D_MERGE(4, 1) SS2D_MERGE(4, 2) SS2D_MERGE(4, 4) SS2D_MERGE(4, 8) SS2D_MERGE(4, 16)
+    SS2D_MERGE(1, 1) SS2D_MERGE(1, 2) SS2D_MERGE(1, 4) SS2D_MERGE(1, 8) SS2D_MERGE(1, 16)
+#undef SS2D_MERGE
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace ss2d

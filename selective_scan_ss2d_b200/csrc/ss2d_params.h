@@ -6,7 +6,6 @@ namespace ss2d {
 
 constexpr int kNP = 16;     // states per channel held by the kernels (N <= 16)
 constexpr int kT = 16;      // steps per sub-chunk
-constexpr int kMergeRows = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ScanParams {
