@@ -17,8 +17,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libss2d_b200.so")
-SOURCES = ["ss2d_capi.cu", "ss2d_launch.cu", "ss2d_noalloc.cu"]
-HEADERS = ["ss2d_kernels.cuh", "ss2d_quad.cuh", "ss2d_launch.h", "ss2d_params.h"]
+SOURCES = ["ss2d_capi.cu", "ss2d_launch.cu", "ss2d_noalloc.cu", "ss2d_scan_bf16.cu",
+           "ss2d_scan_f32.cu"]
+HEADERS = ["ss2d_kernels.cuh", "ss2d_quad.cuh", "ss2d_scan_launch.cuh", "ss2d_launch.h",
+           "ss2d_params.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -47,19 +49,28 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     os.makedirs(LIBDIR, exist_ok=True)
-    objs = []
-    log_lines = []
+    # every translation unit compiles in its own nvcc process, all at once
+    objs, procs = [], []
     for src in SOURCES:
-        obj = os.path.join(LIBDIR, os.path.splitext(src)[0] + ".o")
+        obj = os.path.join(LIBDIR, os.path.splitext(src)[0] + f".{os.getpid()}.o")
         cmd = [nvcc(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
                "-Xptxas", "-v", "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src),
                "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        log_lines.append(r.stdout + r.stderr)
-        if r.returncode != 0:
-            sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError(f"nvcc failed on {src}")
+        procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
+                                            text=True)))
         objs.append(obj)
+    log_lines, failed = [], []
+    for src, pr in procs:
+        out, _ = pr.communicate()
+        log_lines.append(out)
+        if pr.returncode != 0:
+            failed.append(src)
+            sys.stderr.write(out)
+    if failed:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
+        raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)

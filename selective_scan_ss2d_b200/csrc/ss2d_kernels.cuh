@@ -205,6 +205,37 @@ struct Row16 {
             w[2 * q + 1] = x.y;
         }
     }
+    // bf16 rows whose start is only 2-byte aligned: nine 4-byte word loads
+    // from the aligned word at or before src, realigned with funnel shifts.
+    // Reads up to two values past the sixteen; the caller guarantees they
+    // exist.
+    __device__ __forceinline__ void load_words(const Tin *src)
+    {
+        static_assert(sizeof(Tin) == 2, "4-byte words hold two bf16 values");
+        const uintptr_t a = reinterpret_cast<uintptr_t>(src);
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(a & ~(uintptr_t)3);
+        const unsigned sh = (unsigned)(a & 2) * 8;   // 0 or 16
+        uint32_t v[RW + 1];
+#pragma unroll
+        for (int j = 0; j <= RW; ++j)
+            v[j] = __ldg(wp + j);
+#pragma unroll
+        for (int j = 0; j < RW; ++j)
+            w[j] = __funnelshift_r(v[j], v[j + 1], sh);
+    }
+    // sixteen values loaded one by one (each in the low bits of e[i])
+    __device__ __forceinline__ void pack(const uint32_t (&e)[kT])
+    {
+        if constexpr (sizeof(Tin) == 2) {
+#pragma unroll
+            for (int j = 0; j < RW; ++j)
+                w[j] = __byte_perm(e[2 * j], e[2 * j + 1], 0x5410);
+        } else {
+#pragma unroll
+            for (int i = 0; i < kT; ++i)
+                w[i] = e[i];
+        }
+    }
     __device__ __forceinline__ void set_raw(int i, uint32_t bits)   // bits of one value
     {
         if constexpr (sizeof(Tin) == 2) {
@@ -227,7 +258,8 @@ __device__ __forceinline__ uint32_t raw_bits(const __nv_bfloat16 *p)
 // One chunk of LC steps of 32*WC channels of one (b, k); see the header.
 // grid: x = k, y = channel tile, z = b * NCg + chunk, NCg = chunks launched
 // (NC - 1 in kModeState, NC in kModeOutput).
-template <typename Tin, int WC, int MODE, int MINB, bool PACK>
+// COLS: the column-major directions (SS2D with K = 4) are compiled in.
+template <typename Tin, int WC, int MODE, int MINB, bool COLS>
 __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
 {
     using Sh = ChunkShape<WC>;
@@ -270,7 +302,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * K + k) * N * L;
     // x order of this direction: 0 forward, 1 reversed (both contiguous),
     // 2 through the pixel walker (column-major directions)
-    const int xmode = (p.two_d && k >= 2) ? 2 : (k & 1);
+    const int xmode = (COLS && k >= 2) ? 2 : (k & 1);
     const int vbytes = p.vec;   // 16 or 8: vector width of delta/x row loads; 0: scalar
     const bool ovec = p.ovec != 0;
 
@@ -296,16 +328,36 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     PixWalk xw;   // column-major directions: pixel of the next step to prefetch
     xw.init(p.two_d, k, l_begin, H, W, L);
     Row16<Tin> pd, px;
+    const int adv_q = kT / H, adv_r = kT % H;   // the walker's 16-step advance
     auto prefetch = [&](int ls) {   // steps ls .. ls + 15
-        const bool whole = vbytes > 0 && ls + kT <= L;
-        auto load_row = [&](Row16<Tin> &r, const Tin *src) {
+        const bool whole = ls + kT <= L;
+        // a row segment of 16 values starting at src (ascending), or the
+        // values of steps ls.. one by one where it is cut by the row end
+        auto load_row = [&](Row16<Tin> &r, const Tin *src, bool words_ok) {
             if (vbytes == 16)
                 r.load_vec(src);
-            else
+            else if (vbytes == 8)
                 r.load_vec8(src);
+            else if constexpr (sizeof(Tin) == 2) {
+                if (words_ok) {
+                    r.load_words(src);
+                } else {
+                    uint32_t e[kT];
+#pragma unroll
+                    for (int i = 0; i < kT; ++i)
+                        e[i] = raw_bits(src + i);
+                    r.pack(e);
+                }
+            } else {
+                uint32_t e[kT];
+#pragma unroll
+                for (int i = 0; i < kT; ++i)
+                    e[i] = raw_bits(src + i);
+                r.pack(e);
+            }
         };
         if (whole) {
-            load_row(pd, drow + ls);
+            load_row(pd, drow + ls, ls + kT + 2 <= L);
         } else {
 #pragma unroll
             for (int i = 0; i < kT; ++i)
@@ -313,7 +365,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         }
         if (xmode == 0) {
             if (whole) {
-                load_row(px, xrow + ls);
+                load_row(px, xrow + ls, ls + kT + 2 <= L);
             } else {
 #pragma unroll
                 for (int i = 0; i < kT; ++i)
@@ -321,7 +373,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
             }
         } else if (xmode == 1) {   // pixels L-1-ls-i: load ascending, read reversed
             if (whole) {
-                load_row(px, xrow + (L - kT - ls));
+                load_row(px, xrow + (L - kT - ls), ls > 0);
             } else {
 #pragma unroll
                 for (int i = 0; i < kT; ++i) {   // value of step ls + 15 - i
@@ -329,6 +381,32 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
                     px.set_raw(i, l < L ? raw_bits(xrow + (L - 1 - l)) : 0u);
                 }
             }
+        } else if constexpr (!COLS) {
+            // no column-major direction in this instantiation
+        } else if (whole && H >= 8) {
+            // column-major directions: pixel of step ls + i without walking.
+            // Each column wrap moves the pixel by L - 1 against the row
+            // stride; with H >= 8 there are at most two wraps in 16 steps
+            // (one when H >= 16).
+            uint32_t e[kT];
+            const int p0 = xw.p, h0 = xw.h, Lm1 = L - 1;
+            if (k == 2) {
+#pragma unroll
+                for (int i = 0; i < kT; ++i) {
+                    const int hh = h0 + i;
+                    const int c = (hh >= H) + (H < kT && hh >= 2 * H);
+                    e[i] = raw_bits(xrow + (p0 + i * W - c * Lm1));
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < kT; ++i) {
+                    const int hh = h0 - i;
+                    const int c = (hh < 0) + (H < kT && hh < -H);
+                    e[i] = raw_bits(xrow + (p0 - i * W + c * Lm1));
+                }
+            }
+            px.pack(e);
+            xw.advance(kT, adv_q, adv_r, H, W);
         } else {
 #pragma unroll
             for (int i = 0; i < kT; ++i) {
@@ -420,35 +498,17 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 bv = col[q * kT];
-                if constexpr (PACK) {
-                    const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
-                    const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
-                    const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
-                    const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
-                    h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
-                    h2[2 * q + 1] =
-                        __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                    if (MODE == kModeOutput) {
-                        const float4 cv = col[(4 + q) * kT];
-                        acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
-                        acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
-                    }
-                } else {
-                    const float a0 = mufu_ex2(dt * A2[2 * q].x);
-                    const float a1 = mufu_ex2(dt * A2[2 * q].y);
-                    const float a2 = mufu_ex2(dt * A2[2 * q + 1].x);
-                    const float a3 = mufu_ex2(dt * A2[2 * q + 1].y);
-                    h2[2 * q].x = fmaf(a0, h2[2 * q].x, du * bv.x);
-                    h2[2 * q].y = fmaf(a1, h2[2 * q].y, du * bv.y);
-                    h2[2 * q + 1].x = fmaf(a2, h2[2 * q + 1].x, du * bv.z);
-                    h2[2 * q + 1].y = fmaf(a3, h2[2 * q + 1].y, du * bv.w);
-                    if (MODE == kModeOutput) {
-                        const float4 cv = col[(4 + q) * kT];
-                        acc0.x = fmaf(cv.x, h2[2 * q].x, acc0.x);
-                        acc0.y = fmaf(cv.y, h2[2 * q].y, acc0.y);
-                        acc1.x = fmaf(cv.z, h2[2 * q + 1].x, acc1.x);
-                        acc1.y = fmaf(cv.w, h2[2 * q + 1].y, acc1.y);
-                    }
+                const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
+                const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
+                const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
+                const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
+                h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
+                h2[2 * q + 1] =
+                    __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
+                if (MODE == kModeOutput) {
+                    const float4 cv = col[(4 + q) * kT];
+                    acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
+                    acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
                 }
             }
             if (MODE == kModeOutput)
@@ -496,7 +556,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 // Entry states of every chunk after the first, in place over the chunk end
 // states: slot c of (b,k,d) holds h_end of chunk c on entry and h_in of chunk
 // c+1 on exit.  One thread per (b, k, d, n).
-__global__ void carry_kernel(const ScanParams p)
+static __global__ void carry_kernel(const ScanParams p)
 {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long total = (long long)p.B * p.K * p.D * kNP;
@@ -532,14 +592,19 @@ __global__ void carry_kernel(const ScanParams p)
 
 // cross_merge, band form: a CTA covers `rows` full image rows (the band
 // starting at row h0 = blockIdx.y * R) of CG consecutive (b, d) channels.
-//  * cols (SS2D, K = 4): for each channel, the column-major directions'
-//    values of the band are read as runs (column w of the band is scan steps
-//    w*H + h0 .. w*H + h0 + rows - 1 of direction 2, the mirror run of
-//    direction 3) and transposed through shared memory [rows][W + 1];
+//  * cols (SS2D, K = 4): the column-major directions' values of the band are
+//    staged in shared memory first:
+//      - whole (the band is the whole image, L % 4 == 0): their rows are
+//        copied as they are (float4, scan order) and read at the scan index
+//        of each pixel;
+//      - otherwise column w of the band is the run of scan steps
+//        w*H + h0 .. w*H + h0 + rows - 1 of direction 2 (the mirror run of
+//        direction 3), read as runs and transposed to [rows][W + 1];
 //  * the row-major directions (and every direction of K <= 2 or 1D) are
 //    contiguous: direction 0 at p, direction 1 at L-1-p.
-// VEC = 4: float4 accesses (needs W % 4 == 0, and H % 4 == 0 and R % 4 == 0
-// when cols); VEC = 1: scalar.
+// Work units (float4 groups of pixels when VEC = 4 or whole, pixels when
+// VEC = 1) of all CG channels are spread over the whole CTA.  VEC = 4 needs
+// W % 4 == 0, and H % 4 == 0 and R % 4 == 0 when cols.
 //   sum = 1: y[b,d,p] = ((Y_0 + Y_1) + Y_2) + Y_3       (first K terms)
 //   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
 constexpr int kMerge2Threads = 256;
@@ -547,9 +612,9 @@ constexpr int kMerge2Threads = 256;
 template <int VEC, int CG>
 __global__ void __launch_bounds__(kMerge2Threads)
     merge2_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
-                  int W, int K, int cols, int sum, int R)
+                  int W, int K, int cols, int sum, int R, int whole)
 {
-    extern __shared__ float smem_m2[];   // [CG][2][R][W + 1] when cols
+    extern __shared__ float smem_m2[];   // cols: [CG][2][R][W + 1], whole: [CG][2][L]
     const int L = H * W;
     const size_t kstride = (size_t)D * L;
     const long long nch = (long long)B * D;
@@ -558,125 +623,165 @@ __global__ void __launch_bounds__(kMerge2Threads)
     const int rows = min(R, H - h0);
     const int p0 = h0 * W, n = rows * W;
     const int WS = W + 1;
-    long long b = bd0 / D;
-    int d = (int)(bd0 - b * D);
-    int nc = 0;   // channels of this CTA that exist
+    const long long b0 = bd0 / D;
+    const int d0 = (int)(bd0 - b0 * D);
+    const int nc = (int)min((long long)CG, nch - bd0);   // channels of this CTA
+    const size_t tile = whole ? 2 * (size_t)L : 2 * (size_t)R * WS;   // smem floats per channel
+    // row (b, 0, d) of part for the c-th channel of the CTA
+    auto part_row = [&](int c) {
+        long long bb = b0;
+        int dd = d0 + c;
+        while (dd >= D) {
+            dd -= D;
+            ++bb;
+        }
+        return ((size_t)bb * K * D + dd) * (size_t)L;
+    };
+    auto y_row = [&](int c) {
+        long long bb = b0;
+        int dd = d0 + c;
+        while (dd >= D) {
+            dd -= D;
+            ++bb;
+        }
+        return ((size_t)bb * D + dd) * (size_t)L;
+    };
+
+    // thread slice of each channel: TPC consecutive threads per channel
+    constexpr int TPC = kMerge2Threads / CG;
+    const int c = threadIdx.x / TPC, t0 = threadIdx.x % TPC;
+    const bool active = c < nc;
+    const size_t rk = active ? part_row(c) : 0;   // row (b, 0, d) of part
+
     if (cols) {
-        long long bb = b;
-        int dd = d;
-        for (int c = 0; c < CG && bd0 + c < nch; ++c, ++nc) {
-            const float *r2 = part + ((size_t)(bb * K + 2) * D + dd) * L;
+        if (active) {
+            const float *r2 = part + rk + 2 * kstride;
             const float *r3 = r2 + kstride;
-            float *s2 = smem_m2 + (size_t)c * 2 * R * WS;
-            float *s3 = s2 + (size_t)R * WS;
-            if (VEC == 4) {
-                const int rq = R / 4;              // float4 runs per column
-                const int per = kMerge2Threads / rq;
-                const int q = threadIdx.x % rq;
-                for (int w = threadIdx.x / rq; w < W; w += per) {
-                    const int r = 4 * q;
-                    if (threadIdx.x < per * rq && r < rows) {
-                        const int s = w * H + h0 + r;
-                        const float4 a = __ldg(reinterpret_cast<const float4 *>(r2 + s));
-                        const float4 m = __ldg(reinterpret_cast<const float4 *>(r3 + (L - 4 - s)));
-                        s2[(r + 0) * WS + w] = a.x;
-                        s2[(r + 1) * WS + w] = a.y;
-                        s2[(r + 2) * WS + w] = a.z;
-                        s2[(r + 3) * WS + w] = a.w;
-                        s3[(r + 0) * WS + w] = m.w;
-                        s3[(r + 1) * WS + w] = m.z;
-                        s3[(r + 2) * WS + w] = m.y;
-                        s3[(r + 3) * WS + w] = m.x;
-                    }
+            float *s2 = smem_m2 + c * tile;
+            if (whole) {
+                const int q4 = L / 4;   // float4 per row
+                float4 *t2 = reinterpret_cast<float4 *>(s2), *t3 = t2 + q4;
+                for (int j = t0; j < q4; j += TPC) {
+                    t2[j] = __ldg(reinterpret_cast<const float4 *>(r2) + j);
+                    t3[j] = __ldg(reinterpret_cast<const float4 *>(r3) + j);
+                }
+            } else if (VEC == 4) {
+                float *s3 = s2 + (size_t)R * WS;
+                const int rq = rows / 4;   // float4 runs per column
+                for (int e = t0; e < W * rq; e += TPC) {
+                    const int w = e / rq, r = 4 * (e - w * rq);
+                    const int sc = w * H + h0 + r;
+                    const float4 a = __ldg(reinterpret_cast<const float4 *>(r2 + sc));
+                    const float4 m = __ldg(reinterpret_cast<const float4 *>(r3 + (L - 4 - sc)));
+                    s2[(r + 0) * WS + w] = a.x;
+                    s2[(r + 1) * WS + w] = a.y;
+                    s2[(r + 2) * WS + w] = a.z;
+                    s2[(r + 3) * WS + w] = a.w;
+                    s3[(r + 0) * WS + w] = m.w;
+                    s3[(r + 1) * WS + w] = m.z;
+                    s3[(r + 2) * WS + w] = m.y;
+                    s3[(r + 3) * WS + w] = m.x;
                 }
             } else {
+                float *s3 = s2 + (size_t)R * WS;
                 // element e of the band in column-major order: w = e / rows
-                for (int e = threadIdx.x; e < n; e += kMerge2Threads) {
+                for (int e = t0; e < n; e += TPC) {
                     const int w = e / rows, r = e - w * rows;
-                    const int s = w * H + h0 + r;
-                    s2[r * WS + w] = __ldg(r2 + s);
-                    s3[r * WS + w] = __ldg(r3 + (L - 1 - s));
+                    const int sc = w * H + h0 + r;
+                    s2[r * WS + w] = __ldg(r2 + sc);
+                    s3[r * WS + w] = __ldg(r3 + (L - 1 - sc));
                 }
-            }
-            if (++dd == D) {
-                dd = 0;
-                ++bb;
             }
         }
         __syncthreads();
-    } else {
-        nc = (int)min((long long)CG, nch - bd0);
     }
-    for (int c = 0; c < nc; ++c) {
-        const size_t rk = ((size_t)b * K * D + d) * L;   // row (b, 0, d) of part
-        const float *r0 = part + rk;
-        const float *r1 = r0 + kstride;
-        const float *s2 = smem_m2 + (size_t)c * 2 * R * WS;
-        const float *s3 = s2 + (size_t)R * WS;
-        float *yo = sum ? y + ((size_t)b * D + d) * L : y + rk;
-        if (VEC == 4) {
-            for (int i = 4 * threadIdx.x; i < n; i += 4 * kMerge2Threads) {
-                const int p = p0 + i;
-                float4 v = __ldg(reinterpret_cast<const float4 *>(r0 + p));
-                float4 v1 = make_float4(0.f, 0.f, 0.f, 0.f), v2 = v1, v3 = v1;
-                if (K >= 2) {
-                    const float4 m = __ldg(reinterpret_cast<const float4 *>(r1 + (L - 4 - p)));
-                    v1 = make_float4(m.w, m.z, m.y, m.x);
-                }
-                if (cols) {
-                    const int r = i / W, w = i - r * W;
-                    const float *a2 = s2 + r * WS + w, *a3 = s3 + r * WS + w;
-                    v2 = make_float4(a2[0], a2[1], a2[2], a2[3]);
-                    v3 = make_float4(a3[0], a3[1], a3[2], a3[3]);
-                }
-                if (sum) {
-                    if (K >= 2)
-                        v = make_float4(v.x + v1.x, v.y + v1.y, v.z + v1.z, v.w + v1.w);
-                    if (cols)
-                        v = make_float4((v.x + v2.x) + v3.x, (v.y + v2.y) + v3.y,
-                                        (v.z + v2.z) + v3.z, (v.w + v2.w) + v3.w);
-                    *reinterpret_cast<float4 *>(yo + p) = v;
-                } else {
-                    *reinterpret_cast<float4 *>(yo + p) = v;
-                    if (K >= 2)
-                        *reinterpret_cast<float4 *>(yo + kstride + p) = v1;
-                    if (cols) {
-                        *reinterpret_cast<float4 *>(yo + 2 * kstride + p) = v2;
-                        *reinterpret_cast<float4 *>(yo + 3 * kstride + p) = v3;
+    if (!active)
+        return;
+
+    const int vw = (whole || VEC == 4) ? 4 : 1;
+    const int upc = n / vw;   // units per channel
+    const float *r0 = part + rk, *r1 = r0 + kstride;
+    float *yo = sum ? y + y_row(c) : y + rk;
+    for (int iu = t0; iu < upc; iu += TPC) {
+        const int i = iu * vw;   // band pixel index
+        const int p = p0 + i;
+        if (vw == 4) {
+            const float4 v0 = __ldg(reinterpret_cast<const float4 *>(r0 + p));
+            float4 v1 = make_float4(0.f, 0.f, 0.f, 0.f), v2 = v1, v3 = v1;
+            if (K >= 2) {
+                const float4 m = __ldg(reinterpret_cast<const float4 *>(r1 + (L - 4 - p)));
+                v1 = make_float4(m.w, m.z, m.y, m.x);
+            }
+            if (cols) {
+                float a2[4], a3[4];
+                if (whole) {
+                    const float *t2 = smem_m2 + c * tile, *t3 = t2 + L;
+                    int h = p / W, w = p - h * W;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int sc = w * H + h;   // column-major scan index of pixel p + j
+                        a2[j] = t2[sc];
+                        a3[j] = t3[L - 1 - sc];
+                        if (++w == W) {
+                            w = 0;
+                            ++h;
+                        }
                     }
+                } else {
+                    const int r = i / W, w = i - r * W;
+                    const float *s2 = smem_m2 + c * tile + r * WS + w;
+                    const float *s3 = s2 + (size_t)R * WS;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        a2[j] = s2[j];
+                        a3[j] = s3[j];
+                    }
+                }
+                v2 = make_float4(a2[0], a2[1], a2[2], a2[3]);
+                v3 = make_float4(a3[0], a3[1], a3[2], a3[3]);
+            }
+            if (sum) {
+                float4 v = v0;
+                if (K >= 2)
+                    v = make_float4(v.x + v1.x, v.y + v1.y, v.z + v1.z, v.w + v1.w);
+                if (cols)
+                    v = make_float4((v.x + v2.x) + v3.x, (v.y + v2.y) + v3.y,
+                                    (v.z + v2.z) + v3.z, (v.w + v2.w) + v3.w);
+                *reinterpret_cast<float4 *>(yo + p) = v;
+            } else {
+                *reinterpret_cast<float4 *>(yo + p) = v0;
+                if (K >= 2)
+                    *reinterpret_cast<float4 *>(yo + kstride + p) = v1;
+                if (cols) {
+                    *reinterpret_cast<float4 *>(yo + 2 * kstride + p) = v2;
+                    *reinterpret_cast<float4 *>(yo + 3 * kstride + p) = v3;
                 }
             }
         } else {
-            for (int i = threadIdx.x; i < n; i += kMerge2Threads) {
-                const int p = p0 + i;
-                float v = __ldg(r0 + p);
-                const float v1 = K >= 2 ? __ldg(r1 + (L - 1 - p)) : 0.f;
-                float v2 = 0.f, v3 = 0.f;
+            float v = __ldg(r0 + p);
+            const float v1 = K >= 2 ? __ldg(r1 + (L - 1 - p)) : 0.f;
+            float v2 = 0.f, v3 = 0.f;
+            if (cols) {
+                const int r = i / W, w = i - r * W;
+                const float *s2 = smem_m2 + c * tile;
+                v2 = s2[r * WS + w];
+                v3 = s2[(size_t)R * WS + r * WS + w];
+            }
+            if (sum) {
+                if (K >= 2)
+                    v += v1;
+                if (cols)
+                    v = (v + v2) + v3;
+                yo[p] = v;
+            } else {
+                yo[p] = v;
+                if (K >= 2)
+                    yo[kstride + p] = v1;
                 if (cols) {
-                    const int r = i / W, w = i - r * W;
-                    v2 = s2[r * WS + w];
-                    v3 = s3[r * WS + w];
-                }
-                if (sum) {
-                    if (K >= 2)
-                        v += v1;
-                    if (cols)
-                        v = (v + v2) + v3;
-                    yo[p] = v;
-                } else {
-                    yo[p] = v;
-                    if (K >= 2)
-                        yo[kstride + p] = v1;
-                    if (cols) {
-                        yo[2 * kstride + p] = v2;
-                        yo[3 * kstride + p] = v3;
-                    }
+                    yo[2 * kstride + p] = v2;
+                    yo[3 * kstride + p] = v3;
                 }
             }
-        }
-        if (++d == D) {
-            d = 0;
-            ++b;
         }
     }
 }

@@ -1,8 +1,6 @@
 // ss2d_launch.cu -- kernel variants, the execution plan of a call, launchers.
 #include "ss2d_launch.h"
 
-#include <cuda_bf16.h>
-
 #include "ss2d_kernels.cuh"
 #include "ss2d_quad.cuh"
 
@@ -22,78 +20,6 @@ const VariantInfo kVariants[] = {
     {"quad4_lc512", 4, 512, 128, 1},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
-
-// Minimum resident CTAs per SM the kernels are compiled for: R = 128 gives
-// 16 warps per SM and a register cap of 65536 / 512 = 128 per thread;
-// R = 168 gives 12 warps per SM and a cap of 168 (more room for the compiler
-// to keep loads in flight and interleave steps).
-template <int WC, int R>
-struct MinBlocks {
-    static constexpr int value = (R == 128 ? 16 : 12) / WC;
-};
-
-template <typename Tin, int WC, int MODE, int R>
-cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
-{
-    using Sh = ChunkShape<WC>;
-    auto kern = chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, true>;
-    const size_t smem = Sh::SMEM_BYTES;
-    if (smem > 48 * 1024) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-    }
-    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT), (unsigned)(p.B * ncg));
-    kern<<<grid, Sh::NT, smem, st>>>(p);
-    return cudaGetLastError();
-}
-
-template <typename Tin, int MODE, int NW, int R>
-cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st)
-{
-    constexpr int MINB = 65536 / (32 * NW * R);
-    constexpr int CH = kQCh * NW;
-    dim3 grid((unsigned)p.K, (unsigned)((p.D + CH - 1) / CH), (unsigned)(p.B * ncg));
-    quad_scan_kernel<Tin, MODE, NW, MINB><<<grid, 32 * NW, 0, st>>>(p);
-    return cudaGetLastError();
-}
-
-template <typename Tin, int LAYOUT, int WC, int R, int MODE>
-cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st)
-{
-    if constexpr (LAYOUT == 0)
-        return launch_chunk<Tin, WC, MODE, R>(p, ncg, st);
-    else
-        return launch_quad<Tin, MODE, WC, R>(p, ncg, st);
-}
-
-template <typename Tin, int LAYOUT, int WC, int R>
-cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
-{
-    cudaError_t e;
-    if (plan.NC > 1) {
-        if (ev)
-            cudaEventRecord(ev[0], st);
-        e = launch_pass<Tin, LAYOUT, WC, R, kModeState>(p, plan.NC - 1, st);
-        if (e != cudaSuccess)
-            return e;
-        if (ev)
-            cudaEventRecord(ev[1], st);
-        const long long total = (long long)p.B * p.K * p.D * kNP;
-        const int threads = 256;
-        carry_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, st>>>(p);
-        e = cudaGetLastError();
-        if (e != cudaSuccess)
-            return e;
-    }
-    if (ev)
-        cudaEventRecord(ev[2], st);
-    e = launch_pass<Tin, LAYOUT, WC, R, kModeOutput>(p, plan.NC, st);
-    if (ev)
-        cudaEventRecord(ev[3], st);
-    return e;
-}
 
 }  // namespace
 
@@ -176,18 +102,7 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 {
     p.LC = plan.LC;
     p.NC = plan.NC;
-#define SS2D_DISPATCH(LY, WCV, RV)                                                  \
-    if (plan.layout == LY && plan.wc == WCV && plan.regs == RV)                     \
-        return bf16 ? launch_passes<__nv_bfloat16, LY, WCV, RV>(plan, p, st, ev)    \
-                    : launch_passes<float, LY, WCV, RV>(plan, p, st, ev);
-    SS2D_DISPATCH(0, 1, 128)
-    SS2D_DISPATCH(0, 2, 128)
-    SS2D_DISPATCH(0, 4, 128)
-    SS2D_DISPATCH(0, 2, 168)
-    SS2D_DISPATCH(0, 4, 168)
-    SS2D_DISPATCH(1, 4, 128)
-#undef SS2D_DISPATCH
-    return cudaErrorInvalidValue;
+    return bf16 ? launch_scan_bf16(plan, p, st, ev) : launch_scan_f32(plan, p, st, ev);
 }
 
 namespace {
@@ -199,7 +114,7 @@ constexpr int kMergeTarget = 4096;
 constexpr size_t kMergeSmemMax = 48 * 1024;
 
 struct MergeShape {
-    int cols, vec, R, CG, nbands;
+    int cols, vec, R, CG, nbands, whole;
     size_t smem;
 };
 
@@ -219,7 +134,14 @@ MergeShape merge_shape(int H, int W, int K, int two_d)
     int cg = (int)(kMergeTarget / band);
     if (cg < 1)
         cg = 1;
-    const size_t per_ch = m.cols ? sizeof(float) * 2 * (size_t)R * (W + 1) : 0;
+    // a band that is the whole image whose column-major rows cannot use the
+    // float4 transpose: copy those rows as they are
+    const long long L = (long long)H * W;
+    m.whole = (m.cols && m.vec == 1 && R == H && L % 4 == 0 &&
+               sizeof(float) * 2 * L <= kMergeSmemMax) ? 1 : 0;
+    const size_t per_ch = !m.cols ? 0
+                          : m.whole ? sizeof(float) * 2 * (size_t)L
+                                    : sizeof(float) * 2 * (size_t)R * (W + 1);
     while (cg > 1 && per_ch * cg > kMergeSmemMax)
         --cg;
     int cgp = 1;   // compiled channel-group sizes: 1, 2, 4, 8, 16
@@ -237,7 +159,7 @@ cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int 
     const long long groups = ((long long)B * D + CG - 1) / CG;
     dim3 grid((unsigned)groups, (unsigned)m.nbands);
     merge2_kernel<VEC, CG><<<grid, kMerge2Threads, m.smem, st>>>(part, y, B, D, H, W, K, m.cols,
-                                                               sum, m.R);
+                                                               sum, m.R, m.whole);
     return cudaGetLastError();
 }
 }  // namespace

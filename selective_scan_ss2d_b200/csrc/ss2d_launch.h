@@ -41,6 +41,9 @@ Plan make_plan(int variant, int B, int D, int L, int K);
 // output pass and after it (the first two only when the plan is chunked).
 cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t st,
                         cudaEvent_t *ev = nullptr);
+// the same for one input dtype (ss2d_scan_bf16.cu, ss2d_scan_f32.cu)
+cudaError_t launch_scan_bf16(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
+cudaError_t launch_scan_f32(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
 // cross_merge of the scan-order rows in `part` into y (sum = 1) or into the
 // per-direction pixel-order copy (sum = 0).
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,

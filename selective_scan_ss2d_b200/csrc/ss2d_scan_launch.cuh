@@ -1,0 +1,107 @@
+// ss2d_scan_launch.cuh -- launchers of the scan passes (state pass, carry,
+// output pass) for one input dtype; included by ss2d_scan_bf16.cu and
+// ss2d_scan_f32.cu so that the two dtypes compile as separate units.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ss2d_kernels.cuh"
+#include "ss2d_launch.h"
+#include "ss2d_quad.cuh"
+
+namespace ss2d {
+namespace {
+
+// Minimum resident CTAs per SM the kernels are compiled for: R = 128 gives
+// 16 warps per SM and a register cap of 65536 / 512 = 128 per thread;
+// R = 168 gives 12 warps per SM and a cap of 168 (more room for the compiler
+// to keep loads in flight and interleave steps).
+template <int WC, int R>
+struct MinBlocks {
+    static constexpr int value = (R == 128 ? 16 : 12) / WC;
+};
+
+template <typename Tin, int WC, int MODE, int R>
+cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
+{
+    using Sh = ChunkShape<WC>;
+    auto kern = (p.two_d && p.K == 4) ? chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, true>
+                                      : chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, false>;
+    const size_t smem = Sh::SMEM_BYTES;
+    if (smem > 48 * 1024) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT), (unsigned)(p.B * ncg));
+    kern<<<grid, Sh::NT, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tin, int MODE, int NW, int R>
+cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st)
+{
+    constexpr int MINB = 65536 / (32 * NW * R);
+    constexpr int CH = kQCh * NW;
+    dim3 grid((unsigned)p.K, (unsigned)((p.D + CH - 1) / CH), (unsigned)(p.B * ncg));
+    quad_scan_kernel<Tin, MODE, NW, MINB><<<grid, 32 * NW, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tin, int LAYOUT, int WC, int R, int MODE>
+cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st)
+{
+    if constexpr (LAYOUT == 0)
+        return launch_chunk<Tin, WC, MODE, R>(p, ncg, st);
+    else
+        return launch_quad<Tin, MODE, WC, R>(p, ncg, st);
+}
+
+template <typename Tin, int LAYOUT, int WC, int R>
+cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
+{
+    cudaError_t e;
+    if (plan.NC > 1) {
+        if (ev)
+            cudaEventRecord(ev[0], st);
+        e = launch_pass<Tin, LAYOUT, WC, R, kModeState>(p, plan.NC - 1, st);
+        if (e != cudaSuccess)
+            return e;
+        if (ev)
+            cudaEventRecord(ev[1], st);
+        const long long total = (long long)p.B * p.K * p.D * kNP;
+        const int threads = 256;
+        carry_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, st>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    if (ev)
+        cudaEventRecord(ev[2], st);
+    e = launch_pass<Tin, LAYOUT, WC, R, kModeOutput>(p, plan.NC, st);
+    if (ev)
+        cudaEventRecord(ev[3], st);
+    return e;
+}
+
+}  // namespace
+
+// The scan passes of a plan for input dtype Tin (see launch_scan).
+template <typename Tin>
+cudaError_t launch_scan_t(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev)
+{
+#define SS2D_DISPATCH(LY, WCV, RV)                                       \
+    if (plan.layout == LY && plan.wc == WCV && plan.regs == RV)          \
+        return launch_passes<Tin, LY, WCV, RV>(plan, p, st, ev);
+    SS2D_DISPATCH(0, 1, 128)
+    SS2D_DISPATCH(0, 2, 128)
+    SS2D_DISPATCH(0, 4, 128)
+    SS2D_DISPATCH(0, 2, 168)
+    SS2D_DISPATCH(0, 4, 168)
+    SS2D_DISPATCH(1, 4, 128)
+#undef SS2D_DISPATCH
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ss2d
