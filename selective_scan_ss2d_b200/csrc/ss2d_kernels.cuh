@@ -515,19 +515,31 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
                 sY[t * 33 + lane] = fmaf(dsk, u, (acc0.x + acc0.y) + (acc1.x + acc1.y));
         }
         if (MODE == kModeOutput && cvalid) {
-            // this lane's 16 outputs, one row segment of the scan-order output
-            float *orow = p.out + (row_bk + d) * L + l0;
+            // this lane's 16 outputs, one segment of its output row: in scan
+            // order, except direction 1 of a multi-direction call (the reversed
+            // row-major order), which is stored flipped, in pixel order
+            const bool flip = k == 1 && K > 1;
+            float *rowp = p.out + (row_bk + d) * L;
             if (ovec && l0 + kT <= l_end) {
+                float *orow = rowp + (flip ? L - kT - l0 : l0);
+                if (flip) {
 #pragma unroll
-                for (int q = 0; q < kT / 4; ++q)
-                    reinterpret_cast<float4 *>(orow)[q] =
-                        make_float4(sY[(4 * q) * 33 + lane], sY[(4 * q + 1) * 33 + lane],
-                                    sY[(4 * q + 2) * 33 + lane], sY[(4 * q + 3) * 33 + lane]);
+                    for (int q = 0; q < kT / 4; ++q)
+                        reinterpret_cast<float4 *>(orow)[q] = make_float4(
+                            sY[(15 - 4 * q) * 33 + lane], sY[(14 - 4 * q) * 33 + lane],
+                            sY[(13 - 4 * q) * 33 + lane], sY[(12 - 4 * q) * 33 + lane]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < kT / 4; ++q)
+                        reinterpret_cast<float4 *>(orow)[q] =
+                            make_float4(sY[(4 * q) * 33 + lane], sY[(4 * q + 1) * 33 + lane],
+                                        sY[(4 * q + 2) * 33 + lane], sY[(4 * q + 3) * 33 + lane]);
+                }
             } else {
 #pragma unroll
                 for (int t = 0; t < kT; ++t)
                     if (l0 + t < l_end)
-                        orow[t] = sY[t * 33 + lane];
+                        rowp[flip ? L - 1 - l0 - t : l0 + t] = sY[t * 33 + lane];
             }
         }
         if (more) {
@@ -601,9 +613,12 @@ static __global__ void carry_kernel(const ScanParams p)
 //        w*H + h0 .. w*H + h0 + rows - 1 of direction 2 (the mirror run of
 //        direction 3), read as runs and transposed to [rows][W + 1];
 //  * the row-major directions (and every direction of K <= 2 or 1D) are
-//    contiguous: direction 0 at p, direction 1 at L-1-p.
+//    read at p: direction 0's row is in scan order = pixel order, and the
+//    output pass stores direction 1's row flipped, in pixel order.
 // Work units (float4 groups of pixels when VEC = 4 or whole, pixels when
-// VEC = 1) of all CG channels are spread over the whole CTA.  VEC = 4 needs
+// VEC = 1) of all CG channels are spread over the whole CTA.  flat (no
+// column-major direction, one band per image, CG | D, 4 | CG): the CTA's
+// channels form one contiguous block of each row set, streamed as float4.  VEC = 4 needs
 // W % 4 == 0, and H % 4 == 0 and R % 4 == 0 when cols.
 //   sum = 1: y[b,d,p] = ((Y_0 + Y_1) + Y_2) + Y_3       (first K terms)
 //   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
@@ -612,7 +627,7 @@ constexpr int kMerge2Threads = 256;
 template <int VEC, int CG>
 __global__ void __launch_bounds__(kMerge2Threads)
     merge2_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
-                  int W, int K, int cols, int sum, int R, int whole)
+                  int W, int K, int cols, int sum, int R, int whole, int flat)
 {
     extern __shared__ float smem_m2[];   // cols: [CG][2][R][W + 1], whole: [CG][2][L]
     const int L = H * W;
@@ -647,6 +662,30 @@ __global__ void __launch_bounds__(kMerge2Threads)
         return ((size_t)bb * D + dd) * (size_t)L;
     };
 
+    if (flat) {
+        // no column-major direction, whole rows, CG | D and 4 | CG: the CTA's
+        // channels are one contiguous, 16-byte aligned block of every row set
+        const size_t nb = (size_t)CG * L / 4;
+        const size_t rk0 = part_row(0);
+        const float4 *a = reinterpret_cast<const float4 *>(part + rk0);
+        const float4 *m = reinterpret_cast<const float4 *>(part + rk0 + kstride);
+        float4 *yo = reinterpret_cast<float4 *>(sum ? y + y_row(0) : y + rk0);
+        float4 *yo1 = reinterpret_cast<float4 *>(y + rk0 + kstride);
+#pragma unroll 4
+        for (size_t f = threadIdx.x; f < nb; f += kMerge2Threads) {
+            const float4 v0 = __ldg(a + f);
+            const float4 v1 = K >= 2 ? __ldg(m + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (sum) {
+                yo[f] = make_float4(v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w);
+            } else {
+                yo[f] = v0;
+                if (K >= 2)
+                    yo1[f] = v1;
+            }
+        }
+        return;
+    }
+
     // thread slice of each channel: TPC consecutive threads per channel
     constexpr int TPC = kMerge2Threads / CG;
     const int c = threadIdx.x / TPC, t0 = threadIdx.x % TPC;
@@ -661,6 +700,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
             if (whole) {
                 const int q4 = L / 4;   // float4 per row
                 float4 *t2 = reinterpret_cast<float4 *>(s2), *t3 = t2 + q4;
+#pragma unroll 4
                 for (int j = t0; j < q4; j += TPC) {
                     t2[j] = __ldg(reinterpret_cast<const float4 *>(r2) + j);
                     t3[j] = __ldg(reinterpret_cast<const float4 *>(r3) + j);
@@ -702,16 +742,15 @@ __global__ void __launch_bounds__(kMerge2Threads)
     const int upc = n / vw;   // units per channel
     const float *r0 = part + rk, *r1 = r0 + kstride;
     float *yo = sum ? y + y_row(c) : y + rk;
+#pragma unroll 4
     for (int iu = t0; iu < upc; iu += TPC) {
         const int i = iu * vw;   // band pixel index
         const int p = p0 + i;
         if (vw == 4) {
             const float4 v0 = __ldg(reinterpret_cast<const float4 *>(r0 + p));
             float4 v1 = make_float4(0.f, 0.f, 0.f, 0.f), v2 = v1, v3 = v1;
-            if (K >= 2) {
-                const float4 m = __ldg(reinterpret_cast<const float4 *>(r1 + (L - 4 - p)));
-                v1 = make_float4(m.w, m.z, m.y, m.x);
-            }
+            if (K >= 2)
+                v1 = __ldg(reinterpret_cast<const float4 *>(r1 + p));
             if (cols) {
                 float a2[4], a3[4];
                 if (whole) {
@@ -759,7 +798,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
             }
         } else {
             float v = __ldg(r0 + p);
-            const float v1 = K >= 2 ? __ldg(r1 + (L - 1 - p)) : 0.f;
+            const float v1 = K >= 2 ? __ldg(r1 + p) : 0.f;
             float v2 = 0.f, v3 = 0.f;
             if (cols) {
                 const int r = i / W, w = i - r * W;

@@ -51,6 +51,10 @@ int pick_variant(int two_d, int B, int D, int H, int W, int N, int K)
     // fuller warps hide the longer per-chunk dependency chains better)
     if (wants_chunks((long long)B * K * D, L))
         return 12;  // wc2_lc128_r168
+    // SS2D (four directions, two column-major) unchunked: 64-channel CTAs at
+    // 168 registers
+    if (two_d && K == 4 && D % 64 == 0)
+        return 9;   // wc2_auto_r168
     // otherwise the widest CTA that leaves no channel tile mostly empty
     if (D % 128 == 0)
         return 1;   // wc4_auto
@@ -114,11 +118,11 @@ constexpr int kMergeTarget = 4096;
 constexpr size_t kMergeSmemMax = 48 * 1024;
 
 struct MergeShape {
-    int cols, vec, R, CG, nbands, whole;
+    int cols, vec, R, CG, nbands, whole, flat;
     size_t smem;
 };
 
-MergeShape merge_shape(int H, int W, int K, int two_d)
+MergeShape merge_shape(int D, int H, int W, int K, int two_d)
 {
     MergeShape m{};
     m.cols = (two_d && K == 4) ? 1 : 0;
@@ -149,6 +153,7 @@ MergeShape merge_shape(int H, int W, int K, int two_d)
         cgp *= 2;
     m.CG = cgp;
     m.smem = per_ch * cgp;
+    m.flat = (!m.cols && m.nbands == 1 && D % cgp == 0 && cgp % 4 == 0) ? 1 : 0;
     return m;
 }
 
@@ -159,20 +164,20 @@ cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int 
     const long long groups = ((long long)B * D + CG - 1) / CG;
     dim3 grid((unsigned)groups, (unsigned)m.nbands);
     merge2_kernel<VEC, CG><<<grid, kMerge2Threads, m.smem, st>>>(part, y, B, D, H, W, K, m.cols,
-                                                               sum, m.R, m.whole);
+                                                               sum, m.R, m.whole, m.flat);
     return cudaGetLastError();
 }
 }  // namespace
 
 size_t merge_smem_bytes(int H, int W, int K, int two_d)
 {
-    return merge_shape(H, W, K, two_d).smem;
+    return merge_shape(1, H, W, K, two_d).smem;
 }
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st)
 {
-    const MergeShape m = merge_shape(H, W, K, two_d);
+    const MergeShape m = merge_shape(D, H, W, K, two_d);
     if (m.smem > kMergeSmemMax)
         return cudaErrorInvalidValue;
     if ((long long)B * D > 0x7fffffffLL * m.CG || m.nbands > 65535)

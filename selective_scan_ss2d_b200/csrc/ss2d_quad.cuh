@@ -279,7 +279,18 @@ __global__ void __launch_bounds__(32 * NW, MINB) quad_scan_kernel(const ScanPara
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     o[i] = fmaf(dsk, u_cur[i], r4[i]);
-                if (v4 && l + 3 < l_end) {
+                if (k == 1 && K > 1) {
+                    // direction 1 of a multi-direction call: pixel order
+                    if (v4 && l + 3 < l_end) {
+                        *reinterpret_cast<float4 *>(orow + (L - 4 - l)) =
+                            make_float4(o[3], o[2], o[1], o[0]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (l + i < l_end)
+                                orow[L - 1 - l - i] = o[i];
+                    }
+                } else if (v4 && l + 3 < l_end) {
                     *reinterpret_cast<float4 *>(orow + l) = make_float4(o[0], o[1], o[2], o[3]);
                 } else {
 #pragma unroll

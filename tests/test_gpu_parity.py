@@ -37,6 +37,8 @@ def small(kind="2d", B=2, D=12, H=7, W=9, K=4, N=16, dtype=wl.F32):
 # ---------------------------------------------------------------------------
 SMALL_2D = [
     small(),                                        # non-square, L = 63 (ragged)
+    small(B=2, D=40, H=14, W=14, K=4, N=16),        # VMamba-B stage-3 image, two column wraps
+    small(B=1, D=24, H=11, W=23, K=4, N=16),        # odd height between 8 and 16
     small(B=1, D=8, H=8, W=8, K=4, N=4),            # the tiny config's shape
     small(B=3, D=37, H=5, W=13, K=4, N=16),         # D not a multiple of any tile
     small(B=2, D=16, H=16, W=20, K=4, N=8),         # L = 320 (> one chunk)
@@ -89,13 +91,29 @@ def _running_sum_inputs(cfg, rng):
                      np.full(K * D, 32.0, np.float32))
 
 
-@pytest.mark.parametrize("cfg", [small(B=2, D=5, H=5, W=7, N=1), small(B=1, D=3, H=56, W=56, N=1),
-                                 small(B=1, D=2, H=24, W=40, N=1), small(B=1, D=4, H=7, W=9, K=2, N=1),
-                                 small("1d", B=2, D=5, W=197, K=2, N=1)],
-                         ids=lambda c: c.name)
-def test_index_maps_bit_exact(cfg):
+# heights below 8 use the pixel walker; 8..15 can wrap a column twice within
+# one 16-step sub-chunk, 16 and more at most once; odd 1D lengths take the
+# realigned 4-byte loads of bf16 rows
+INDEX_SHAPES = [small(B=2, D=5, H=5, W=7, N=1), small(B=1, D=3, H=56, W=56, N=1),
+                small(B=1, D=2, H=24, W=40, N=1), small(B=1, D=4, H=7, W=9, K=2, N=1),
+                small(B=1, D=3, H=14, W=14, N=1), small(B=1, D=2, H=9, W=17, N=1),
+                small(B=1, D=2, H=11, W=6, N=1), small(B=1, D=2, H=16, W=3, N=1),
+                small(B=1, D=2, H=15, W=33, N=1),
+                small("1d", B=2, D=5, W=197, K=2, N=1), small("1d", B=2, D=3, W=201, K=2, N=1),
+                small("1d", B=3, D=2, W=34, K=2, N=1)]
+
+
+@pytest.mark.parametrize("cfg", INDEX_SHAPES, ids=lambda c: c.name)
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+def test_index_maps_bit_exact(cfg, dtype):
     rng = np.random.default_rng(5)
     inp = _running_sum_inputs(cfg, rng)
+    if dtype == wl.BF16:
+        # every value involved (small integers, 0, 1, 1/32) is exact in bf16
+        b = inp.cfg.with_(dtype=wl.BF16)
+        inp = wl.Inputs(b, wl.f32_to_bf16_bits(inp.x), wl.f32_to_bf16_bits(inp.delta),
+                        wl.f32_to_bf16_bits(inp.Bs), wl.f32_to_bf16_bits(inp.Cs), inp.A_log,
+                        inp.Dskip, inp.delta_bias)
     # The exact result is an integer running sum.  The oracle's float64
     # softplus(32) is 32 * (1 + 4e-16), so its sums carry residues below
     # 1e-12; rounding to the nearest integer recovers the exact values.
