@@ -73,6 +73,38 @@ def measured_peaks() -> dict:
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU, no collective on the data path
+# ---------------------------------------------------------------------------
+def init_distributed(world: int, local_rank: int, backend: str = "nccl") -> None:
+    """Join the job's process group (torchrun's env://) when world > 1."""
+    if world <= 1:
+        return
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of x over all ranks (x itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the
+    slowest rank's time."""
+    return units_per_rank_step * steps * world / (max_total_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -264,12 +296,8 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    value = cfg.updates * args.steps * world / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(step_ms), dev)
+    value = whole_job_rate(cfg.updates, args.steps, world, total_ms)
 
     # per-launch device times of the same calls (same inputs, same flushes),
     # CUDA events recorded by the library on this stream around each launch
@@ -349,9 +377,10 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-def run_e2e(args, cfg_name, local_rank):
+def run_e2e(args, cfg_name, local_rank, world=1):
     """Same metric through the C ABI with host (pinned) buffers: every step
-    copies the inputs in, computes, and copies y out, inside the call."""
+    copies the inputs in, computes, and copies y out, inside the call.  Every
+    rank runs it; the slowest rank's time counts."""
     import torch
     from selective_scan_ss2d_b200 import binding
     from selective_scan_ss2d_b200 import workloads as wl
@@ -374,11 +403,12 @@ def run_e2e(args, cfg_name, local_rank):
         b.record(stream)
         evs.append((a, b))
     torch.cuda.synchronize()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dev)
     h2d = sum(getattr(inp, nm).nbytes for nm in wl.Inputs.STREAMED + wl.Inputs.PARAMS)
     d2h = y.numel() * 4
-    return {"value": cfg.updates / (ms / 1e3), "unit": "updates/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
+    return {"value": whole_job_rate(cfg.updates, n, world, total), "unit": "updates/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": total / n,
+            "steps": n}
 
 
 def run_reference(args):
@@ -455,12 +485,7 @@ def main():
         print(json.dumps(run_reference(args)), flush=True)
         return 0
 
-    if world > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    init_distributed(world, local_rank)
 
     if args.report:
         from selective_scan_ss2d_b200 import workloads as wl
@@ -475,11 +500,12 @@ def main():
         return 0
 
     r = run_ours(args, rank, world, local_rank)
+    e2e = None if args.no_e2e else run_e2e(args, args.config, local_rank, world)
     if rank == 0:
         line = r["line"]
         line["clocks"] = r.get("clocks")
-        if not args.no_e2e:
-            line["e2e"] = run_e2e(args, args.config, local_rank)
+        if e2e is not None:
+            line["e2e"] = e2e
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             from selective_scan_ss2d_b200 import workloads as wl
