@@ -583,22 +583,38 @@ static __global__ void carry_kernel(const ScanParams p)
     float *hs = p.hstate + (size_t)bkd * (p.NC - 1) * kNP + n;
     const float *ds = p.dtsum + (size_t)bkd * (p.NC - 1);
     const int nc1 = p.NC - 1;
-    float h = 0.f;
-    for (int c0 = 0; c0 < nc1; c0 += 8) {
-        float he[8], dc[8];
+    // the loads do not depend on h: groups of G chunks, the next group in
+    // flight while the current one is applied
+    constexpr int G = 16;
+    float heA[G], dcA[G], heB[G], dcB[G];
+    auto load = [&](float *he, float *dc, int c0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {   // the loads do not depend on h: issue them first
+        for (int i = 0; i < G; ++i) {
             const bool ok = c0 + i < nc1;
             he[i] = ok ? hs[(size_t)(c0 + i) * kNP] : 0.f;
             dc[i] = ok ? ds[c0 + i] : 0.f;
         }
+    };
+    float h = 0.f;
+    auto apply = [&](const float *he, const float *dc, int c0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < G; ++i) {
             if (c0 + i < nc1) {
                 h = fmaf(mufu_ex2(a2 * dc[i]), h, he[i]);
                 hs[(size_t)(c0 + i) * kNP] = h;
             }
         }
+    };
+    load(heA, dcA, 0);
+    for (int c0 = 0; c0 < nc1; c0 += 2 * G) {
+        if (c0 + G < nc1)
+            load(heB, dcB, c0 + G);
+        apply(heA, dcA, c0);
+        if (c0 + G >= nc1)
+            break;
+        if (c0 + 2 * G < nc1)
+            load(heA, dcA, c0 + 2 * G);
+        apply(heB, dcB, c0 + G);
     }
 }
 

@@ -18,6 +18,7 @@ const VariantInfo kVariants[] = {
     {"wc2_lc128_r168", 2, 128, 168},
     {"quad4_auto", 4, 0, 128, 1},  {"quad4_nochunk", 4, -1, 128, 1},
     {"quad4_lc512", 4, 512, 128, 1},
+    {"wc2_lc256_r168", 2, 256, 168}, {"wc2_lc512_r168", 2, 512, 168},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
