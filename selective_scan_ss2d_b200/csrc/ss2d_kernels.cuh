@@ -758,7 +758,6 @@ __global__ void __launch_bounds__(kMerge2Threads)
     const int upc = n / vw;   // units per channel
     const float *r0 = part + rk, *r1 = r0 + kstride;
     float *yo = sum ? y + y_row(c) : y + rk;
-#pragma unroll 4
     for (int iu = t0; iu < upc; iu += TPC) {
         const int i = iu * vw;   // band pixel index
         const int p = p0 + i;
