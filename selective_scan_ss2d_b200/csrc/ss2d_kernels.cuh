@@ -51,6 +51,14 @@ namespace ss2d {
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
+// Programmatic dependent launch (sm_90+): a kernel launched as a dependent
+// of the previous one on the stream may start before that one has finished;
+// grid_dependency_wait() blocks until it has completed and its writes are
+// visible (a no-op for a kernel launched without the dependency), and
+// allow_dependents() lets the next kernel start launching early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // 2^x on the multi-function unit (PTX ex2.approx.ftz.f32).
 __device__ __forceinline__ float mufu_ex2(float x)
 {
@@ -306,22 +314,12 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     const int vbytes = p.vec;   // 16 or 8: vector width of delta/x row loads; 0: scalar
     const bool ovec = p.ovec != 0;
 
-    // entry state
+    // entry state (chunks after the first of the output pass: loaded once the
+    // carry kernel has finished, after the staging prologue below)
     float2 h2[8];
-    if (MODE == kModeOutput && chunk > 0) {
-        const float4 *hs = reinterpret_cast<const float4 *>(
-            p.hstate + ((row_bk + dc) * (p.NC - 1) + (chunk - 1)) * kNP);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = hs[q];
-            h2[2 * q] = make_float2(v.x, v.y);
-            h2[2 * q + 1] = make_float2(v.z, v.w);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            h2[j] = make_float2(0.f, 0.f);
-    }
+    for (int j = 0; j < 8; ++j)
+        h2[j] = make_float2(0.f, 0.f);
     float dtsum = 0.f;
 
     // ---- per-lane prefetch of 16 steps of this lane's delta and x ------
@@ -469,7 +467,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         }
     };
 
-    // prologue: sub-chunk 0 staged, sub-chunk 1 in flight
+    // prologue: sub-chunk 0 staged, sub-chunk 1 in flight (inputs only)
     prefetch(l_begin);
     load_bc(l_begin);
     unpack_store(0, l_begin);
@@ -477,6 +475,19 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     if (l_begin + kT < l_end) {
         prefetch(l_begin + kT);
         load_bc(l_begin + kT);
+    }
+    // everything below may read or overwrite what the previous kernel on the
+    // stream wrote (entry states, the output rows)
+    grid_dependency_wait();
+    if (MODE == kModeOutput && chunk > 0) {
+        const float4 *hs = reinterpret_cast<const float4 *>(
+            p.hstate + ((row_bk + dc) * (p.NC - 1) + (chunk - 1)) * kNP);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = hs[q];
+            h2[2 * q] = make_float2(v.x, v.y);
+            h2[2 * q + 1] = make_float2(v.z, v.w);
+        }
     }
     __syncthreads();
 
@@ -554,6 +565,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
         }
         __syncthreads();
     }
+    allow_dependents();
 
     if (MODE == kModeState && cvalid) {
         float4 *hs = reinterpret_cast<float4 *>(
@@ -570,6 +582,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 // c+1 on exit.  One thread per (b, k, d, n).
 static __global__ void carry_kernel(const ScanParams p)
 {
+    grid_dependency_wait();   // the chunk end states of the state pass
+    allow_dependents();
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long total = (long long)p.B * p.K * p.D * kNP;
     if (idx >= total)
@@ -646,6 +660,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
                   int W, int K, int cols, int sum, int R, int whole, int flat)
 {
     extern __shared__ float smem_m2[];   // cols: [CG][2][R][W + 1], whole: [CG][2][L]
+    grid_dependency_wait();   // the output pass's rows
     const int L = H * W;
     const size_t kstride = (size_t)D * L;
     const long long nch = (long long)B * D;

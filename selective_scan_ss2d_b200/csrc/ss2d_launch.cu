@@ -9,6 +9,8 @@ namespace ss2d {
 namespace {
 
 // name: wc<W>_<chunking>: one lane per channel, wc = 32-channel warps per CTA;
+// chunking: auto (from the shape), lc<N> (N steps), nochunk, lcfit (the
+// multiple of 16 in 96..160 that pads the sequence least, ties toward 128);
 // quad<W>_<chunking>: four lanes per channel, W warps of 8 channels per CTA.
 const VariantInfo kVariants[] = {
     {"wc2_auto", 2, 0, 128},       {"wc4_auto", 4, 0, 128},       {"wc1_auto", 1, 0, 128},
@@ -19,6 +21,7 @@ const VariantInfo kVariants[] = {
     {"quad4_auto", 4, 0, 128, 1},  {"quad4_nochunk", 4, -1, 128, 1},
     {"quad4_lc512", 4, 512, 128, 1},
     {"wc2_lc256_r168", 2, 256, 168}, {"wc2_lc512_r168", 2, 512, 168},
+    {"wc2_lcfit_r168", 2, -2, 168},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
@@ -51,7 +54,7 @@ int pick_variant(int two_d, int B, int D, int H, int W, int N, int K)
     // chunked shapes: 128-step chunks with the 168-register kernels (fewer,
     // fuller warps hide the longer per-chunk dependency chains better)
     if (wants_chunks((long long)B * K * D, L))
-        return 12;  // wc2_lc128_r168
+        return 18;  // wc2_lcfit_r168
     // SS2D (four directions, two column-major) unchunked: 64-channel CTAs at
     // 168 registers
     if (two_d && K == 4 && D % 64 == 0)
@@ -75,6 +78,20 @@ Plan make_plan(int v, int B, int D, int L, int K)
     int lc;
     if (vi->chunk > 0) {
         lc = vi->chunk;
+    } else if (vi->chunk == -2) {
+        // chunks of about 128 steps that leave the last one as full as possible
+        lc = 128;
+        long long best = -1;
+        for (int c = 96; c <= 160; c += kT) {
+            const long long pad = ((L + c - 1) / c) * (long long)c - L;
+            const long long key = pad * 1024 + (c > 128 ? c - 128 : 128 - c);
+            if (best < 0 || key < best) {
+                best = key;
+                lc = c;
+            }
+        }
+        if (lc > L)
+            lc = L;
     } else if (vi->chunk < 0) {
         lc = L;
     } else {
@@ -164,9 +181,8 @@ cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int 
 {
     const long long groups = ((long long)B * D + CG - 1) / CG;
     dim3 grid((unsigned)groups, (unsigned)m.nbands);
-    merge2_kernel<VEC, CG><<<grid, kMerge2Threads, m.smem, st>>>(part, y, B, D, H, W, K, m.cols,
-                                                               sum, m.R, m.whole, m.flat);
-    return cudaGetLastError();
+    return launch_kernel(merge2_kernel<VEC, CG>, grid, dim3(kMerge2Threads), m.smem, st, true,
+                         part, y, B, D, H, W, K, m.cols, sum, m.R, m.whole, m.flat);
 }
 }  // namespace
 

@@ -8,9 +8,33 @@ namespace ss2d {
 
 struct ScanParams;
 
+// Launch kern on st; dependent = true launches it as a programmatic
+// dependent of the previous kernel on the stream (it may start before that
+// one finishes and waits in-kernel, with grid_dependency_wait, before it
+// reads that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, bool dependent, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (dependent) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // A kernel variant: layout, CTA width (wc warps) and chunking policy
 // (chunk = 0: chosen from the shape; chunk > 0: that many steps per chunk;
-// chunk < 0: never chunk).
+// chunk = -2: about 128 steps, fitted to the sequence length; chunk = -1:
+// never chunk).
 struct VariantInfo {
     const char *name;
     int wc;

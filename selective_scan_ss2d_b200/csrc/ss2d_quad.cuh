@@ -130,7 +130,9 @@ __global__ void __launch_bounds__(32 * NW, MINB) quad_scan_kernel(const ScanPara
     walk.init(p.two_d, k, min(l_begin + 4 * q, L - 1), H, W, L);
     const int adv_q = kT / H, adv_r = kT % H;
 
-    // entry state
+    // entry state (written by the carry kernel, which may still be running
+    // when this kernel starts as its dependent)
+    grid_dependency_wait();
     float2 h2[2];
     if (MODE == kModeOutput && chunk > 0) {
         const float4 v = *reinterpret_cast<const float4 *>(

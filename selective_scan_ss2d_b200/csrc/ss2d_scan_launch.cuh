@@ -22,7 +22,7 @@ struct MinBlocks {
 };
 
 template <typename Tin, int WC, int MODE, int R>
-cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
+cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
     using Sh = ChunkShape<WC>;
     auto kern = (p.two_d && p.K == 4) ? chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, true>
@@ -35,27 +35,26 @@ cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st)
             return e;
     }
     dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT), (unsigned)(p.B * ncg));
-    kern<<<grid, Sh::NT, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, dim3(Sh::NT), smem, st, dependent, p);
 }
 
 template <typename Tin, int MODE, int NW, int R>
-cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st)
+cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
     constexpr int MINB = 65536 / (32 * NW * R);
     constexpr int CH = kQCh * NW;
     dim3 grid((unsigned)p.K, (unsigned)((p.D + CH - 1) / CH), (unsigned)(p.B * ncg));
-    quad_scan_kernel<Tin, MODE, NW, MINB><<<grid, 32 * NW, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(quad_scan_kernel<Tin, MODE, NW, MINB>, grid, dim3(32 * NW), 0, st,
+                         dependent, p);
 }
 
 template <typename Tin, int LAYOUT, int WC, int R, int MODE>
-cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st)
+cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
     if constexpr (LAYOUT == 0)
-        return launch_chunk<Tin, WC, MODE, R>(p, ncg, st);
+        return launch_chunk<Tin, WC, MODE, R>(p, ncg, st, dependent);
     else
-        return launch_quad<Tin, MODE, WC, R>(p, ncg, st);
+        return launch_quad<Tin, MODE, WC, R>(p, ncg, st, dependent);
 }
 
 template <typename Tin, int LAYOUT, int WC, int R>
@@ -65,21 +64,21 @@ cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
     if (plan.NC > 1) {
         if (ev)
             cudaEventRecord(ev[0], st);
-        e = launch_pass<Tin, LAYOUT, WC, R, kModeState>(p, plan.NC - 1, st);
+        e = launch_pass<Tin, LAYOUT, WC, R, kModeState>(p, plan.NC - 1, st, false);
         if (e != cudaSuccess)
             return e;
         if (ev)
             cudaEventRecord(ev[1], st);
         const long long total = (long long)p.B * p.K * p.D * kNP;
         const int threads = 256;
-        carry_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, st>>>(p);
-        e = cudaGetLastError();
+        e = launch_kernel(carry_kernel, dim3((unsigned)((total + threads - 1) / threads)),
+                          dim3(threads), 0, st, ev == nullptr, p);
         if (e != cudaSuccess)
             return e;
     }
     if (ev)
         cudaEventRecord(ev[2], st);
-    e = launch_pass<Tin, LAYOUT, WC, R, kModeOutput>(p, plan.NC, st);
+    e = launch_pass<Tin, LAYOUT, WC, R, kModeOutput>(p, plan.NC, st, plan.NC > 1 && ev == nullptr);
     if (ev)
         cudaEventRecord(ev[3], st);
     return e;
