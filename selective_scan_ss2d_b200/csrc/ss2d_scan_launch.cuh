@@ -12,13 +12,12 @@
 namespace ss2d {
 namespace {
 
-// Minimum resident CTAs per SM the kernels are compiled for: R = 128 gives
-// 16 warps per SM and a register cap of 65536 / 512 = 128 per thread;
-// R = 168 gives 12 warps per SM and a cap of 168 (more room for the compiler
-// to keep loads in flight and interleave steps).
+// Minimum resident CTAs per SM the kernels are compiled for, from a register
+// cap R per thread: R = 128 gives 16 warps per SM, R = 168 gives 12 (more room
+// for the compiler to keep loads in flight and interleave steps).
 template <int WC, int R>
 struct MinBlocks {
-    static constexpr int value = (R == 128 ? 16 : 12) / WC;
+    static constexpr int value = 65536 / (32 * WC * R);
 };
 
 template <typename Tin, int WC, int MODE, int R>
