@@ -85,6 +85,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_softplus.restype = ctypes.c_double
     lib.oracle_scan_pixel.argtypes = [i, i, ctypes.c_int64, i, i]
     lib.oracle_scan_pixel.restype = ctypes.c_int64
+    lib.oracle_silu.argtypes = [ctypes.c_double]
+    lib.oracle_silu.restype = ctypes.c_double
+    lib.oracle_gate.argtypes = [_dp, _dp, ctypes.c_int64]
+    lib.oracle_gate.restype = i
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i
     return lib
@@ -109,11 +113,22 @@ def _ptr(a: np.ndarray):
 _BBAR = {"euler": 0, "zoh": 1}
 
 
+def _gate(y: np.ndarray, z, lb) -> np.ndarray:
+    z = _f64(z)
+    assert z.shape == y.shape
+    st = lb.oracle_gate(_ptr(y), _ptr(z), y.size)
+    if st != 0:
+        raise RuntimeError(f"oracle_gate failed with status {st}")
+    return y
+
+
 def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, *, K=4,
-                 bbar="euler", threads=1, return_dirs=False, _lib=None):
+                 bbar="euler", threads=1, return_dirs=False, z=None, _lib=None):
     """SS2D forward in float64.  x (B,D,H,W); delta (B,K,D,L); Bs, Cs
     (B,K,N,L); A_log (K*D,N); Dskip, delta_bias (K*D,).  Returns y (B,D,H,W)
-    and, if asked, the per-direction outputs (B,K,D,L) in pixel order."""
+    and, if asked, the per-direction outputs (B,K,D,L) in pixel order.  With
+    z (the layout of x): the merged output times SiLU(z) (the per-direction
+    outputs stay ungated)."""
     x = _f64(x)
     Bb, D, H, W = x.shape
     L = H * W
@@ -132,13 +147,16 @@ def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, *, K=4,
                                 Bb, D, H, W, N, K, _BBAR[bbar], int(threads))
     if st != 0:
         raise RuntimeError(f"oracle_ss2d_forward failed with status {st}")
+    if z is not None:
+        _gate(y, z, lb)
     return (y, yd) if return_dirs else y
 
 
 def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, *, K=2,
-                       bbar="euler", threads=1, return_dirs=False, _lib=None):
+                       bbar="euler", threads=1, return_dirs=False, z=None, _lib=None):
     """1D selective scan in float64: u (B,D,L); K=1 forward, K=2 forward plus
-    reversed (flipped back, then added)."""
+    reversed (flipped back, then added).  With z (B,D,L): the summed output
+    times SiLU(z)."""
     u = _f64(u)
     Bb, D, L = u.shape
     delta, Bs, Cs = _f64(delta), _f64(Bs), _f64(Cs)
@@ -157,11 +175,17 @@ def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, *, K=2,
                                       int(threads))
     if st != 0:
         raise RuntimeError(f"oracle_selective_scan_fwd failed with status {st}")
+    if z is not None:
+        _gate(y, z, lb)
     return (y, yd) if return_dirs else y
 
 
 def softplus(z: float) -> float:
     return lib().oracle_softplus(float(z))
+
+
+def silu(z: float) -> float:
+    return lib().oracle_silu(float(z))
 
 
 def scan_pixel(mode: int, k: int, l: int, H: int, W: int) -> int:

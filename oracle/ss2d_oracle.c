@@ -30,6 +30,9 @@
  *   1D variant   -- Vim block ("Vision Mamba ..." summary, section 4.3):
  *                   a forward scan and a scan of the reversed sequence, the
  *                   reversed output flipped back, the two added.
+ *   gate         -- the same Vim block (and the tutorial's SelectiveSSM):
+ *                   the output times SiLU(z), z = z*sigmoid(z), pointwise
+ *                   (oracle_silu, oracle_gate).
  *
  * Readings taken where the pages are open (each is listed in the design
  * notes of the repository):
@@ -212,6 +215,33 @@ int oracle_selective_scan_fwd(const double *u, const double *delta,
 {
     return forward_impl(1, u, delta, A_log, Bs, Cs, Dskip, delta_bias, y,
                         y_dir, B, D, 1, L, N, K, bbar, nthreads);
+}
+
+/* SiLU(z) = z * sigmoid(z) = z / (1 + e^-z): the gate of the Vim block
+ * ("Vision Mamba ..." summary, section 4.3: both directions' outputs are
+ * multiplied by SiLU(z) before they are added) and of the tutorial's
+ * SelectiveSSM ("Vision Mamba" (dileepadev), section "Background: State Space
+ * Models and Mamba": the scan output times SiLU(z)).  For z < 0 the form
+ * z e^z / (1 + e^z) keeps exp() from overflowing; it is the same number. */
+double oracle_silu(double z)
+{
+    if (z >= 0.0)
+        return z / (1.0 + exp(-z));
+    const double e = exp(z);
+    return z * e / (1.0 + e);
+}
+
+/* Gated output: y[i] *= SiLU(z[i]) for i < n, z in the layout of x.  The
+ * gate multiplies the merged sum of the directions (the Vim block gates each
+ * direction with the same z before the sum; by distributivity that is the
+ * same number up to rounding). */
+int oracle_gate(double *y, const double *z, int64_t n)
+{
+    if (!y || !z || n < 0)
+        return -1;
+    for (int64_t i = 0; i < n; ++i)
+        y[i] *= oracle_silu(z[i]);
+    return 0;
 }
 
 int oracle_max_threads(void)

@@ -19,6 +19,15 @@ def softplus(z):
     return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
 
 
+def silu(z):
+    """z * sigmoid(z), written with the logistic function of |z| so that e^x
+    never overflows (the Vim block's gate; see ss2d_oracle.c)."""
+    z = np.asarray(z, dtype=np.float64)
+    e = np.exp(-np.abs(z))
+    sig = np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return z * sig
+
+
 def scan_orders_2d(H: int, W: int) -> list[np.ndarray]:
     """Pixel index visited at each scan step for the four SS2D directions,
     in the stacking order [row-major, its flip, column-major, its flip]."""
@@ -73,7 +82,7 @@ def _forward(u_pix, orders, delta, A_log, Bs, Cs, Dskip, delta_bias, K, bbar):
 
 
 def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, K=4,
-                 bbar="euler", return_dirs=False):
+                 bbar="euler", return_dirs=False, z=None):
     x = np.asarray(x, dtype=np.float64)
     Bb, D, H, W = x.shape
     y, yd = _forward(x.reshape(Bb, D, H * W), scan_orders_2d(H, W),
@@ -82,15 +91,19 @@ def ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, K=4,
                      np.asarray(Dskip, np.float64),
                      np.asarray(delta_bias, np.float64), K, bbar)
     y = y.reshape(Bb, D, H, W)
+    if z is not None:
+        y = y * silu(z)
     return (y, yd) if return_dirs else y
 
 
 def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, K=2,
-                       bbar="euler", return_dirs=False):
+                       bbar="euler", return_dirs=False, z=None):
     u = np.asarray(u, dtype=np.float64)
     Bb, D, L = u.shape
     y, yd = _forward(u, scan_orders_1d(L), np.asarray(delta, np.float64),
                      np.asarray(A_log, np.float64), np.asarray(Bs, np.float64),
                      np.asarray(Cs, np.float64), np.asarray(Dskip, np.float64),
                      np.asarray(delta_bias, np.float64), K, bbar)
+    if z is not None:
+        y = y * silu(z)
     return (y, yd) if return_dirs else y

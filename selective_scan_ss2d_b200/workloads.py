@@ -157,6 +157,22 @@ def make_inputs(cfg: Config | str, seed: int = 0) -> Inputs:
     return Inputs(cfg, x, delta, Bs, Cs, A_log, Dskip, delta_bias)
 
 
+def make_gate(cfg: Config | str, seed: int = 0) -> np.ndarray:
+    """The gate input z of a gated call: N(0, 1) in the layout of x, in the
+    workload's storage dtype (a stream of its own, so the other inputs of the
+    same seed are unchanged)."""
+    if isinstance(cfg, str):
+        cfg = CONFIGS[cfg]
+    rng = np.random.default_rng([seed, 0x6a7e])
+    xshape = (cfg.B, cfg.D, cfg.H, cfg.W) if cfg.kind == "2d" else (cfg.B, cfg.D, cfg.L)
+    return _normal(rng, xshape, cfg.dtype)
+
+
+def gate_as_f64(z: np.ndarray, cfg: Config) -> np.ndarray:
+    """The exact values a gated call sees, widened to float64."""
+    return (bf16_bits_to_f32(z) if cfg.dtype == BF16 else z).astype(np.float64)
+
+
 def channel_subproblem(inp: Inputs, b: int, d: int) -> Inputs:
     """The inputs that one output channel (b, d) depends on, as a B=1, D=1
     workload of its own (pure slicing; used to check sampled channels of a

@@ -399,7 +399,41 @@ def pin_extreme_softplus(impl):
         np.testing.assert_allclose(y.reshape(-1), [dt], rtol=1e-14, atol=0)
 
 
+def pin_gate(impl):
+    """The gate multiplies the merged output by SiLU(z) = z * sigmoid(z)
+    pointwise.  With the identity scan (Bs = 0, Dskip = 1) the ungated output
+    is 4x (2x for the 1D K = 2 case), so the gated output is a closed form:
+    sigmoid(ln 3) = 3/4 gives SiLU(ln 3) = (3/4) ln 3 and SiLU(-ln 3) =
+    -(1/4) ln 3; SiLU(0) = 0; SiLU(40) is 40 to 1e-15 relative; SiLU(-40)
+    is -40 e^-40 to 1e-15 relative (no overflow, the small value kept).
+    Without z the output is the ungated one."""
+    rng = np.random.default_rng(20)
+    ln3 = math.log(3.0)
+    table = {ln3: 0.75 * ln3, -ln3: -0.25 * ln3, 0.0: 0.0, 40.0: 40.0,
+             -40.0: -40.0 * math.exp(-40.0)}
+    keys = np.array(sorted(table))
+    H, W, B, D, K, N = 3, 4, 2, 3, 4, 2
+    p = rand_problem(rng, B, D, H, W, K, N)
+    p["x"] = rng.integers(-8, 9, size=(B, D, H, W)).astype(np.float64)
+    p["Bs"] = np.zeros((B, K, N, H * W))
+    p["Dskip"] = np.ones(K * D)
+    z = keys[rng.integers(0, len(keys), size=p["x"].shape)]
+    want = 4.0 * p["x"] * np.vectorize(table.get)(z)
+    y = call2d(impl, p, K=4, z=z)
+    np.testing.assert_allclose(y, want, rtol=1e-15, atol=0)
+    assert np.array_equal(call2d(impl, p, K=4), 4.0 * p["x"]), "ungated output changed"
+    # 1D, K = 2
+    L = 10
+    p = rand_problem(rng, B, D, 1, L, 2, N, one_d=True)
+    p["x"] = rng.integers(-8, 9, size=(B, D, L)).astype(np.float64)
+    p["Cs"] = np.zeros((B, 2, N, L))
+    p["Dskip"] = np.ones(2 * D)
+    z = keys[rng.integers(0, len(keys), size=p["x"].shape)]
+    y = call1d(impl, p, K=2, z=z)
+    np.testing.assert_allclose(y, 2.0 * p["x"] * np.vectorize(table.get)(z), rtol=1e-15, atol=0)
+
+
 ALL_PINS = [pin_hand_worked, pin_integrator_scan_orders, pin_single_step_closed_form,
             pin_geometric_series, pin_matrix_exponential_discretisation,
             pin_convolution_form, pin_identity_scan, pin_reversal_invariant,
-            pin_linearity, pin_decomposition, pin_extreme_softplus]
+            pin_linearity, pin_decomposition, pin_extreme_softplus, pin_gate]

@@ -119,6 +119,10 @@ MUTATIONS = {
     "state_not_reset": ("    for (int n = 0; n < N; ++n)\n        h[n] = 0.0;\n", ""),
     "params_of_direction_0": ("const int64_t kd = (int64_t)k * D + d;",
                               "const int64_t kd = d;"),
+    "gate_is_sigmoid": ("        return z / (1.0 + exp(-z));",
+                        "        return 1.0 / (1.0 + exp(-z));"),
+    "gate_sign_flipped": ("    return z * e / (1.0 + e);", "    return -z * e / (1.0 + e);"),
+    "gate_skipped": ("        y[i] *= oracle_silu(z[i]);", "        y[i] *= 1.0;"),
 }
 
 
