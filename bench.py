@@ -266,9 +266,23 @@ def run_ours(args, rank, world, local_rank):
     l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
     flush = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev)
 
+    gate = getattr(args, "gate", False)
+    if gate:
+        # the SiLU output gate: a seeded z in x's layout, the gated entry point
+        # (the library's own variant choice)
+        import numpy as np
+        zr = wl.make_gate(cfg, seed=rank)
+        zt = (torch.from_numpy(zr.view(np.int16)).view(torch.bfloat16) if zr.dtype == np.uint16
+              else torch.from_numpy(zr)).to(dev)
+        fn_g = binding.ss2d_forward_gated if cfg.kind == "2d" else binding.selective_scan_fwd_gated
+
     def step():
-        fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"], y,
-           variant=args.variant)
+        if gate:
+            fn_g(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"],
+                 zt, y)
+        else:
+            fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"], y,
+               variant=args.variant)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -350,6 +364,7 @@ def run_ours(args, rank, world, local_rank):
                        "state_dtype": "f32", "updates_per_step": cfg.updates,
                        "algorithmic_bytes_per_step": step_bytes,
                        "kernel_variant": binding.ss2d_variant_name(variant),
+                       "output_gate": "SiLU(z), gated entry point" if gate else None,
                        "l2": "flushed before every timed step (2x L2 write, outside events)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "alu", "achieved": achieved_gexp, "peak": mufu_peak,
@@ -469,6 +484,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="host seconds for the oracle sample of cpu_baseline")
+    ap.add_argument("--gate", action="store_true",
+                    help="time the gated entry point (y * SiLU(z)); device buffers only, "
+                         "so no e2e leg")
     ap.add_argument("--report", action="store_true",
                     help="one JSON line per workload (device-resident only)")
     args = ap.parse_args()
@@ -500,7 +518,7 @@ def main():
         return 0
 
     r = run_ours(args, rank, world, local_rank)
-    e2e = None if args.no_e2e else run_e2e(args, args.config, local_rank, world)
+    e2e = None if (args.no_e2e or args.gate) else run_e2e(args, args.config, local_rank, world)
     if rank == 0:
         line = r["line"]
         line["clocks"] = r.get("clocks")

@@ -131,6 +131,27 @@ int ss2d_scan_directions(const void *x, const void *delta, const float *A_log,
                          int B, int D, int H, int W, int N, int K, int dtype,
                          int two_d, void *stream, int variant);
 
+/* Gated forward: as ss2d_forward / selective_scan_fwd, then y = SiLU(z) * y
+ * pointwise, SiLU(z) = z / (1 + e^-z) -- the output gate of the Vim block
+ * ("Vision Mamba ..." summary, section 4.3: each direction's output is
+ * multiplied by SiLU(z) before the directions are added; the same z for all
+ * directions, so the gate is applied once to the fixed-order sum) and of the
+ * tutorial's SelectiveSSM ("Vision Mamba" (dileepadev), section "Background:
+ * State Space Models and Mamba").  z has the layout and dtype of x (u).
+ * Device pointers only (SS2D_ERR_PTR otherwise); asynchronous on `stream`;
+ * the gate runs inside the cross_merge kernel, which every gated call
+ * launches (also for K = 1). */
+int ss2d_forward_gated(const void *x, const void *delta, const float *A_log,
+                       const void *Bs, const void *Cs, const float *Dskip,
+                       const float *delta_bias, const void *z, float *y,
+                       int B, int D, int H, int W, int N, int K, int dtype,
+                       void *stream);
+int selective_scan_fwd_gated(const void *u, const void *delta, const float *A_log,
+                             const void *Bs, const void *Cs, const float *Dskip,
+                             const float *delta_bias, const void *z, float *y,
+                             int B, int D, int L, int N, int K, int dtype,
+                             void *stream);
+
 /* As ss2d_forward, with an explicit kernel variant (index into the table
  * that ss2d_variant_name() describes; -1 = the library's own choice for the
  * shape).  Every variant computes the same result up to float32 rounding

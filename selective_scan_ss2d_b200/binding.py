@@ -60,6 +60,11 @@ def lib() -> ctypes.CDLL:
             L.selective_scan_fwd_ex.argtypes = fwd + [i] * 6 + [vp, i]
             L.selective_scan_fwd_ex.restype = i
             L.ss2d_scan_directions.argtypes = fwd + [i] * 8 + [vp, i]
+            gfwd = fwd[:7] + [vp] + fwd[7:]   # the gate z before y
+            L.ss2d_forward_gated.argtypes = gfwd + [i] * 7 + [vp]
+            L.ss2d_forward_gated.restype = i
+            L.selective_scan_fwd_gated.argtypes = gfwd + [i] * 6 + [vp]
+            L.selective_scan_fwd_gated.restype = i
             L.ss2d_scan_directions.restype = i
             L.ss2d_plan.argtypes = [i] * 8 + [ctypes.POINTER(ctypes.c_int)] * 3
             L.ss2d_plan.restype = i
@@ -208,6 +213,52 @@ def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, y=None, *, st
     rc = lib().selective_scan_fwd_ex(_ptr(u), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
                                      _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, L, N, K,
                                      dt, st, int(variant))
+    _check(rc)
+    return y
+
+
+def _check_gate(z, x):
+    if z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape) or not z.is_contiguous() \
+            or z.device != x.device:
+        raise ValueError("z must be a contiguous tensor of x's dtype, shape and device")
+
+
+def ss2d_forward_gated(x, delta, A_log, Bs, Cs, Dskip, delta_bias, z, y=None, *, stream=None):
+    """ss2d_forward, then y * SiLU(z) (z in x's layout and dtype).  Device
+    tensors only."""
+    B, D, H, W = x.shape
+    K, N = delta.shape[1], Bs.shape[2]
+    L = H * W
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for ss2d_forward_gated")
+    _check_gate(z, x)
+    y, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, (B, D, H, W))
+    st = _stream(on_gpu, x.device, stream)
+    rc = lib().ss2d_forward_gated(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                                  _ptr(Dskip), _ptr(delta_bias), _ptr(z), _ptr(y), B, D, H, W,
+                                  N, K, dt, st)
+    _check(rc)
+    return y
+
+
+def selective_scan_fwd_gated(u, delta, A_log, Bs, Cs, Dskip, delta_bias, z, y=None, *,
+                             stream=None):
+    """selective_scan_fwd, then y * SiLU(z) (z in u's layout and dtype).
+    Device tensors only."""
+    B, D, L = u.shape
+    K, N = delta.shape[1], Bs.shape[2]
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for selective_scan_fwd_gated")
+    _check_gate(z, u)
+    y, dt, on_gpu = _prepare(u, delta, A_log, Bs, Cs, Dskip, delta_bias, y, (B, D, L))
+    st = _stream(on_gpu, u.device, stream)
+    rc = lib().selective_scan_fwd_gated(_ptr(u), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs),
+                                        _ptr(Dskip), _ptr(delta_bias), _ptr(z), _ptr(y), B, D,
+                                        L, N, K, dt, st)
     _check(rc)
     return y
 

@@ -106,6 +106,7 @@ struct Problem {
     const float *A_log, *Dskip, *delta_bias;
     float *y;
     int B, D, H, W, N, K, dtype, two_d;
+    const void *z = nullptr;   // output gate (gated calls)
 };
 
 int validate(const Problem &pr)
@@ -133,7 +134,8 @@ bool is_empty(const Problem &pr)
 
 int check_pointers(const Problem &pr)
 {
-    const void *ptrs[] = {pr.x, pr.delta, pr.Bs, pr.Cs, pr.A_log, pr.Dskip, pr.delta_bias, pr.y};
+    const void *ptrs[] = {pr.x, pr.delta, pr.Bs, pr.Cs, pr.A_log, pr.Dskip, pr.delta_bias, pr.y,
+                          pr.z ? pr.z : pr.x};
     for (const void *q : ptrs)
         if (!q)
             return SS2D_ERR_NULL;
@@ -184,7 +186,7 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
         return SS2D_ERR_SHAPE;
     if (ss2d::merge_smem_bytes(pr.H, pr.W, pr.K, pr.two_d) > 200 * 1024)
         return SS2D_ERR_SHAPE;
-    const bool need_part = pr.K > 1;
+    const bool need_part = pr.K > 1 || pr.z;   // gated calls always merge (the gate runs there)
     const size_t rows = (size_t)pr.B * pr.K * pr.D;
     const size_t part_bytes = need_part ? align256(sizeof(float) * rows * L) : 0;
     const size_t hs_bytes = pl.NC > 1 ? align256(sizeof(float) * rows * (pl.NC - 1) * ss2d::kNP) : 0;
@@ -212,7 +214,7 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     cudaError_t e = ss2d::launch_scan(pl, bf16, p, st, ev);
     if (e == cudaSuccess && need_part) {
         e = ss2d::launch_merge(p.out, pr.y, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d,
-                               directions ? 0 : 1, st);
+                               directions ? 0 : 1, st, pr.z, pr.dtype == SS2D_BF16);
         if (ev)
             cudaEventRecord(ev[4], st);
     }
@@ -288,8 +290,11 @@ int run_host(const Problem &pr, cudaStream_t st, int variant)
     return rc;
 }
 
-int forward(const Problem &pr, void *stream, int variant, bool directions_only = false)
+int forward(const Problem &pr, void *stream, int variant, bool directions_only = false,
+            bool gated = false)
 {
+    if (gated && !pr.z)
+        return SS2D_ERR_NULL;
     int rc = validate(pr);
     if (rc != SS2D_OK)
         return rc;
@@ -308,7 +313,8 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
         set_error("cudaGetDevice", e);
         return SS2D_ERR_CUDA;
     }
-    const void *ptrs[] = {pr.x, pr.delta, pr.Bs, pr.Cs, pr.A_log, pr.Dskip, pr.delta_bias, pr.y};
+    const void *ptrs[] = {pr.x, pr.delta, pr.Bs, pr.Cs, pr.A_log, pr.Dskip, pr.delta_bias, pr.y,
+                          pr.z ? pr.z : pr.x};
     const PtrKind kind = pointer_kind(ptrs[0], dev);
     if (kind == kBadPtr)
         return SS2D_ERR_PTR;
@@ -316,8 +322,8 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
         if (pointer_kind(q, dev) != kind)
             return SS2D_ERR_PTR;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (directions_only)
-        return kind == kDevicePtr ? run_device(pr, st, variant, true) : SS2D_ERR_PTR;
+    if (directions_only || gated)
+        return kind == kDevicePtr ? run_device(pr, st, variant, directions_only) : SS2D_ERR_PTR;
     return kind == kDevicePtr ? run_device(pr, st, variant, false) : run_host(pr, st, variant);
 }
 
@@ -362,6 +368,24 @@ int selective_scan_fwd(const void *u, const void *delta, const float *A_log, con
 {
     return selective_scan_fwd_ex(u, delta, A_log, Bs, Cs, Dskip, delta_bias, y, B, D, L, N,
                                  K, dtype, stream, -1);
+}
+
+int ss2d_forward_gated(const void *x, const void *delta, const float *A_log, const void *Bs,
+                       const void *Cs, const float *Dskip, const float *delta_bias,
+                       const void *z, float *y, int B, int D, int H, int W, int N, int K,
+                       int dtype, void *stream)
+{
+    Problem pr{x, delta, Bs, Cs, A_log, Dskip, delta_bias, y, B, D, H, W, N, K, dtype, 1, z};
+    return forward(pr, stream, -1, false, true);
+}
+
+int selective_scan_fwd_gated(const void *u, const void *delta, const float *A_log,
+                             const void *Bs, const void *Cs, const float *Dskip,
+                             const float *delta_bias, const void *z, float *y, int B, int D,
+                             int L, int N, int K, int dtype, void *stream)
+{
+    Problem pr{u, delta, Bs, Cs, A_log, Dskip, delta_bias, y, B, D, 1, L, N, K, dtype, 0, z};
+    return forward(pr, stream, -1, false, true);
 }
 
 int ss2d_scan_directions(const void *x, const void *delta, const float *A_log,

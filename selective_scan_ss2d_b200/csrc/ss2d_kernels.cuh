@@ -654,10 +654,39 @@ static __global__ void carry_kernel(const ScanParams p)
 //   sum = 0: y[b,k,d,p] = Y_k                          (per-direction copy)
 constexpr int kMerge2Threads = 256;
 
+// SiLU(z) = z / (1 + e^-z), the optional output gate of cross_merge (fast
+// exp and division intrinsics; for z below about -88 the denominator is
+// infinite and the result is -0)
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+// gate factors of four consecutive y elements starting at index i of z
+__device__ __forceinline__ float4 gate4(const void *z, int bf16, size_t i)
+{
+    float4 g;
+    if (bf16) {
+        const uint2 r = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(z) + i));
+        g = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                        __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+    } else {
+        g = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(z) + i));
+    }
+    return make_float4(silu_f(g.x), silu_f(g.y), silu_f(g.z), silu_f(g.w));
+}
+__device__ __forceinline__ float gate1(const void *z, int bf16, size_t i)
+{
+    const float v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(z)[i])
+                         : __ldg(static_cast<const float *>(z) + i);
+    return silu_f(v);
+}
+__device__ __forceinline__ float4 mul4(float4 a, float4 b)
+{
+    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+
 template <int VEC, int CG>
 __global__ void __launch_bounds__(kMerge2Threads)
     merge2_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
-                  int W, int K, int cols, int sum, int R, int whole, int flat)
+                  int W, int K, int cols, int sum, int R, int whole, int flat,
+                  const void *__restrict__ z, int z_bf16)
 {
     extern __shared__ float smem_m2[];   // cols: [CG][2][R][W + 1], whole: [CG][2][L]
     grid_dependency_wait();   // the output pass's rows
@@ -700,14 +729,18 @@ __global__ void __launch_bounds__(kMerge2Threads)
         const size_t rk0 = part_row(0);
         const float4 *a = reinterpret_cast<const float4 *>(part + rk0);
         const float4 *m = reinterpret_cast<const float4 *>(part + rk0 + kstride);
-        float4 *yo = reinterpret_cast<float4 *>(sum ? y + y_row(0) : y + rk0);
+        const size_t yr0 = y_row(0);
+        float4 *yo = reinterpret_cast<float4 *>(sum ? y + yr0 : y + rk0);
         float4 *yo1 = reinterpret_cast<float4 *>(y + rk0 + kstride);
 #pragma unroll 4
         for (size_t f = threadIdx.x; f < nb; f += kMerge2Threads) {
             const float4 v0 = __ldg(a + f);
             const float4 v1 = K >= 2 ? __ldg(m + f) : make_float4(0.f, 0.f, 0.f, 0.f);
             if (sum) {
-                yo[f] = make_float4(v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w);
+                float4 v = make_float4(v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w);
+                if (z)
+                    v = mul4(v, gate4(z, z_bf16, yr0 + 4 * f));
+                yo[f] = v;
             } else {
                 yo[f] = v0;
                 if (K >= 2)
@@ -772,7 +805,8 @@ __global__ void __launch_bounds__(kMerge2Threads)
     const int vw = (whole || VEC == 4) ? 4 : 1;
     const int upc = n / vw;   // units per channel
     const float *r0 = part + rk, *r1 = r0 + kstride;
-    float *yo = sum ? y + y_row(c) : y + rk;
+    const size_t yr = y_row(c);
+    float *yo = sum ? y + yr : y + rk;
     for (int iu = t0; iu < upc; iu += TPC) {
         const int i = iu * vw;   // band pixel index
         const int p = p0 + i;
@@ -816,6 +850,8 @@ __global__ void __launch_bounds__(kMerge2Threads)
                 if (cols)
                     v = make_float4((v.x + v2.x) + v3.x, (v.y + v2.y) + v3.y,
                                     (v.z + v2.z) + v3.z, (v.w + v2.w) + v3.w);
+                if (z)
+                    v = mul4(v, gate4(z, z_bf16, yr + p));
                 *reinterpret_cast<float4 *>(yo + p) = v;
             } else {
                 *reinterpret_cast<float4 *>(yo + p) = v0;
@@ -841,6 +877,8 @@ __global__ void __launch_bounds__(kMerge2Threads)
                     v += v1;
                 if (cols)
                     v = (v + v2) + v3;
+                if (z)
+                    v *= gate1(z, z_bf16, yr + p);
                 yo[p] = v;
             } else {
                 yo[p] = v;

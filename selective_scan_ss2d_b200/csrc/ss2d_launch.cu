@@ -177,12 +177,13 @@ MergeShape merge_shape(int D, int H, int W, int K, int two_d)
 
 template <int VEC, int CG>
 cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int B, int D,
-                          int H, int W, int K, int sum, cudaStream_t st)
+                          int H, int W, int K, int sum, cudaStream_t st, const void *z,
+                          int z_bf16)
 {
     const long long groups = ((long long)B * D + CG - 1) / CG;
     dim3 grid((unsigned)groups, (unsigned)m.nbands);
     return launch_kernel(merge2_kernel<VEC, CG>, grid, dim3(kMerge2Threads), m.smem, st, true,
-                         part, y, B, D, H, W, K, m.cols, sum, m.R, m.whole, m.flat);
+                         part, y, B, D, H, W, K, m.cols, sum, m.R, m.whole, m.flat, z, z_bf16);
 }
 }  // namespace
 
@@ -192,7 +193,7 @@ size_t merge_smem_bytes(int H, int W, int K, int two_d)
 }
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
-                         int two_d, int sum, cudaStream_t st)
+                         int two_d, int sum, cudaStream_t st, const void *z, int z_bf16)
 {
     const MergeShape m = merge_shape(D, H, W, K, two_d);
     if (m.smem > kMergeSmemMax)
@@ -201,7 +202,7 @@ cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W
         return cudaErrorInvalidConfiguration;
 #define SS2D_MERGE(V, C)                                                             \
     if (m.vec == V && m.CG == C)                                                     \
-        return launch_merge2<V, C>(m, part, y, B, D, H, W, K, sum, st);
+        return launch_merge2<V, C>(m, part, y, B, D, H, W, K, sum, st, z, z_bf16);
     SS2D_MERGE(4, 1) SS2D_MERGE(4, 2) SS2D_MERGE(4, 4) SS2D_MERGE(4, 8) SS2D_MERGE(4, 16)
     SS2D_MERGE(1, 1) SS2D_MERGE(1, 2) SS2D_MERGE(1, 4) SS2D_MERGE(1, 8) SS2D_MERGE(1, 16)
 #undef SS2D_MERGE

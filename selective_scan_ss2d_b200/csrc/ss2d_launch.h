@@ -69,9 +69,11 @@ cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t
 cudaError_t launch_scan_bf16(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
 cudaError_t launch_scan_f32(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
 // cross_merge of the scan-order rows in `part` into y (sum = 1) or into the
-// per-direction pixel-order copy (sum = 0).
+// per-direction pixel-order copy (sum = 0); with z (sum = 1 only), y is
+// multiplied by SiLU(z) (z in the layout of y, bf16 when z_bf16).
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
-                         int two_d, int sum, cudaStream_t st);
+                         int two_d, int sum, cudaStream_t st, const void *z = nullptr,
+                         int z_bf16 = 0);
 size_t merge_smem_bytes(int H, int W, int K, int two_d);
 
 // Text that ss2d_last_error() returns on the calling thread.

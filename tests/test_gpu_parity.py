@@ -249,3 +249,53 @@ def test_timed_call_matches_forward():
         plan = binding.ss2d_plan(True, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K, v)
         assert ms[2] > 0 and ms[3] > 0
         assert (ms[0] > 0) == (plan["num_chunks"] > 1)
+
+
+# ---------------------------------------------------------------------------
+# the SiLU output gate (gated entry points)
+# ---------------------------------------------------------------------------
+GATED = [small(B=2, D=12, H=7, W=9, K=4, N=16), small(B=1, D=40, H=14, W=14, K=4, N=16),
+         small(B=1, D=16, H=20, W=24, K=2, N=16), small(B=2, D=9, H=6, W=5, K=1, N=5),
+         small(B=1, D=8, H=40, W=40, K=4, N=16),
+         small("1d", B=3, D=20, W=197, K=2, N=16), small("1d", B=2, D=16, W=64, K=2, N=16),
+         small("1d", B=2, D=7, W=50, K=1, N=3)]
+
+
+@pytest.mark.parametrize("cfg", GATED, ids=lambda c: c.name)
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+def test_gated_matches_oracle(cfg, dtype):
+    cfg = cfg.with_(dtype=dtype)
+    inp = wl.make_inputs(cfg, seed=4)
+    zraw = wl.make_gate(cfg, seed=4)
+    f = inp.as_f64()
+    z64 = wl.gate_as_f64(zraw, cfg)
+    th = oracle.max_threads()
+    if cfg.kind == "2d":
+        ref = oracle.ss2d_forward(f["x"], f["delta"], f["A_log"], f["Bs"], f["Cs"], f["Dskip"],
+                                  f["delta_bias"], K=cfg.K, threads=th, z=z64)
+    else:
+        ref = oracle.selective_scan_fwd(f["x"], f["delta"], f["A_log"], f["Bs"], f["Cs"],
+                                        f["Dskip"], f["delta_bias"], K=cfg.K, threads=th, z=z64)
+    t = _gpu.tensors(inp)
+    z = _gpu.to_torch(zraw, cfg.dtype, "cuda")
+    fn = binding.ss2d_forward_gated if cfg.kind == "2d" else binding.selective_scan_fwd_gated
+    y = fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"], z)
+    torch.cuda.synchronize()
+    _gpu.assert_close(y.cpu().numpy().astype(np.float64), ref, dtype, cfg.name + " gated")
+
+
+def test_gated_rejects_host_pointers_and_missing_gate():
+    inp = wl.make_inputs(small(B=1, D=4, H=4, W=4, K=4, N=4), seed=0)
+    t = _gpu.tensors(inp, device=None)
+    z = torch.zeros_like(t["x"])
+    with pytest.raises(binding.SS2DError) as ei:
+        binding.ss2d_forward_gated(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"],
+                                   t["delta_bias"], z)
+    assert ei.value.status == -9
+    lib = binding.lib()
+    td = _gpu.tensors(inp)
+    y = torch.empty_like(td["x"])
+    rc = lib.ss2d_forward_gated(*[binding._ptr(td[n]) for n in ("x", "delta", "A_log", "Bs", "Cs",
+                                                               "Dskip", "delta_bias")],
+                                None, binding._ptr(y), 1, 4, 4, 4, 4, 4, 0, None)
+    assert rc == -1
