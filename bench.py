@@ -42,13 +42,13 @@ FALLBACK_SM_MAX_MHZ = 1965.0
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from ncu
 # captures recorded under profiles/, keyed by workload; each entry carries
-# the hash of the kernel sources it was taken from, and is reported only
-# while the sources are unchanged.
+# the input dtype and the hash of the kernel sources it was taken from, and
+# is reported only for that dtype while the sources are unchanged.
 NCU_TRAFFIC = {
     # profiles/chunk_scan_vmamba_t_stage1.md: output pass, dram read 64192000 + write 28228096
-    "vmamba_t_stage1": {"bytes": 92420096, "src": "bd0ae525ebcfaa3b"},
+    "vmamba_t_stage1": {"bytes": 92420096, "dtype": "bf16", "src": "bd0ae525ebcfaa3b"},
     # profiles/chunk_scan_vmamba_b_stage3.md: output pass, dram read 141739264 + write 164204800
-    "vmamba_b_stage3": {"bytes": 305944064, "src": "bd0ae525ebcfaa3b"},
+    "vmamba_b_stage3": {"bytes": 305944064, "dtype": "bf16", "src": "bd0ae525ebcfaa3b"},
 }
 
 
@@ -248,13 +248,21 @@ def slice_sample(inp, nb, nd):
                      np.ascontiguousarray(inp.delta_bias[rows]))
 
 
+def workload_config(name, dtype=None):
+    """The named workload, with its streamed inputs' storage dtype replaced
+    when ``dtype`` is given (f32, bf16 or f16)."""
+    from selective_scan_ss2d_b200 import workloads as wl
+    cfg = wl.CONFIGS[name]
+    return cfg.with_(dtype=dtype) if dtype else cfg
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from selective_scan_ss2d_b200 import binding
     from selective_scan_ss2d_b200 import workloads as wl
 
-    cfg = wl.CONFIGS[args.config]
+    cfg = workload_config(args.config, args.dtype)
     dev = torch.device(f"cuda:{local_rank}")
     torch.cuda.set_device(dev)
     binding.lib()
@@ -340,7 +348,8 @@ def run_ours(args, rank, world, local_rank):
         achieved_gexp = exps / (scan_ms / 1e3) / 1e9
         src_hash = kernel_source_hash()
         tr = NCU_TRAFFIC.get(cfg.name)
-        traffic = tr["bytes"] if tr and tr.get("src") == src_hash else None
+        traffic = (tr["bytes"] if tr and tr.get("src") == src_hash and tr["dtype"] == cfg.dtype
+                   else None)
         variant = args.variant if args.variant >= 0 else binding.ss2d_pick_variant(
             two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K)
         plan = binding.ss2d_plan(two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K, variant)
@@ -358,7 +367,7 @@ def run_ours(args, rank, world, local_rank):
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "f32",
-            "data": "synthetic (seeded N(0,1) inputs, bf16-rounded where the workload is bf16)",
+            "data": "synthetic (seeded N(0,1) inputs, rounded to the workload's bf16 or f16 storage)",
             "config": {"workload": cfg.name, "B": cfg.B, "D": cfg.D, "H": cfg.H, "W": cfg.W,
                        "L": cfg.L, "K": cfg.K, "N": cfg.N, "input_dtype": cfg.dtype,
                        "state_dtype": "f32", "updates_per_step": cfg.updates,
@@ -399,7 +408,7 @@ def run_e2e(args, cfg_name, local_rank, world=1):
     import torch
     from selective_scan_ss2d_b200 import binding
     from selective_scan_ss2d_b200 import workloads as wl
-    cfg = wl.CONFIGS[cfg_name]
+    cfg = workload_config(cfg_name, args.dtype)
     dev = torch.device(f"cuda:{local_rank}")
     inp, t = build_arrays(cfg, seed=0, device=None, pin=True)
     y = torch.empty(inp.x.shape, dtype=torch.float32).pin_memory()
@@ -431,7 +440,7 @@ def run_reference(args):
     (whole channels of batch element 0) of the workload."""
     import oracle
     from selective_scan_ss2d_b200 import workloads as wl
-    cfg = wl.CONFIGS[args.config]
+    cfg = workload_config(args.config, args.dtype)
     threads = oracle.max_threads()
     # size one step to ~ (budget / (steps + warmup)) seconds of host work
     budget_s = float(os.environ.get("SS2D_REFERENCE_BUDGET_S", "150"))
@@ -480,6 +489,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--variant", type=int, default=-1)
+    ap.add_argument("--dtype", choices=["f32", "bf16", "f16"], default=None,
+                    help="storage dtype of x, delta, Bs, Cs (default: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -527,7 +538,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             from selective_scan_ss2d_b200 import workloads as wl
-            cfg = wl.CONFIGS[args.config]
+            cfg = workload_config(args.config, args.dtype)
             threads = oracle.max_threads()
             v, desc, _ = cpu_baseline_parallel(cfg, args.cpu_seconds, threads)
             line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": threads,

@@ -94,7 +94,9 @@ typedef enum {
 
 typedef enum {
     SS2D_F32 = 0,   /* x, delta, Bs, Cs stored as float32  */
-    SS2D_BF16 = 1   /* x, delta, Bs, Cs stored as bfloat16 */
+    SS2D_BF16 = 1,  /* x, delta, Bs, Cs stored as bfloat16 */
+    SS2D_F16 = 2    /* x, delta, Bs, Cs stored as IEEE float16 (the FP16 path of
+                       "VMamba架构解析", section 2; the state stays float32) */
 } ss2d_dtype;
 
 /* SS2D forward: cross_scan -> selective scan of each direction -> cross_merge.

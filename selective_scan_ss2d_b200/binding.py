@@ -18,7 +18,8 @@ import torch
 SS2D_F32 = 0
 SS2D_BF16 = 1
 NOALLOC_SCRATCH_BYTES = 96 * 1024 * 1024   # SS2D_NOALLOC_SCRATCH_BYTES of the C header
-_DTYPES = {torch.float32: SS2D_F32, torch.bfloat16: SS2D_BF16}
+SS2D_F16 = 2
+_DTYPES = {torch.float32: SS2D_F32, torch.bfloat16: SS2D_BF16, torch.float16: SS2D_F16}
 
 _lock = threading.Lock()
 _lib = None
@@ -118,7 +119,7 @@ def _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, xdims):
     streamed = (x, delta, Bs, Cs)
     dt = x.dtype
     if dt not in _DTYPES:
-        raise TypeError(f"x must be float32 or bfloat16, got {dt}")
+        raise TypeError(f"x must be float32, bfloat16 or float16, got {dt}")
     for t in streamed:
         if t.dtype != dt:
             raise TypeError("x, delta, Bs and Cs must share one dtype")

@@ -113,7 +113,7 @@ int validate(const Problem &pr)
 {
     if (pr.B < 0 || pr.D < 0 || pr.H < 0 || pr.W < 0)
         return SS2D_ERR_SHAPE;
-    if (pr.dtype != SS2D_F32 && pr.dtype != SS2D_BF16)
+    if (pr.dtype != SS2D_F32 && pr.dtype != SS2D_BF16 && pr.dtype != SS2D_F16)
         return SS2D_ERR_DTYPE;
     if (pr.two_d ? !(pr.K == 1 || pr.K == 2 || pr.K == 4) : !(pr.K == 1 || pr.K == 2))
         return SS2D_ERR_K;
@@ -179,7 +179,7 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
                cudaEvent_t *ev = nullptr)
 {
     ss2d::ScanParams p = make_params(pr);
-    const bool bf16 = pr.dtype == SS2D_BF16;
+    const size_t in_esz = pr.dtype == SS2D_F32 ? 4 : 2;   // bytes per stored input value
     const long long L = p.L;
     const ss2d::Plan pl = ss2d::make_plan(variant, pr.B, pr.D, (int)L, pr.K);
     if ((long long)pr.B * pl.NC > 65535)
@@ -203,7 +203,7 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     {
         // vector access to the rows of delta and x (dtype) and of out (float32)
         // needs every row start on a boundary of the vector width
-        const size_t esz = bf16 ? 2 : 4;
+        const size_t esz = in_esz;
         const bool ptr_ok = (((uintptr_t)pr.x | (uintptr_t)pr.delta | (uintptr_t)p.out) & 15) == 0;
         const size_t rb = (size_t)L * esz;
         p.vec = !ptr_ok ? 0 : (rb % 16 == 0 ? 16 : (rb % 8 == 0 ? 8 : 0));
@@ -211,10 +211,10 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     }
     p.hstate = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes) : nullptr;
     p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes + hs_bytes) : nullptr;
-    cudaError_t e = ss2d::launch_scan(pl, bf16, p, st, ev);
+    cudaError_t e = ss2d::launch_scan(pl, pr.dtype, p, st, ev);
     if (e == cudaSuccess && need_part) {
         e = ss2d::launch_merge(p.out, pr.y, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d,
-                               directions ? 0 : 1, st, pr.z, pr.dtype == SS2D_BF16);
+                               directions ? 0 : 1, st, pr.z, pr.dtype);
         if (ev)
             cudaEventRecord(ev[4], st);
     }
@@ -236,7 +236,7 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
 int run_host(const Problem &pr, cudaStream_t st, int variant)
 {
     const size_t L = (size_t)pr.H * pr.W;
-    const size_t esz = pr.dtype == SS2D_BF16 ? 2 : 4;
+    const size_t esz = pr.dtype == SS2D_F32 ? 4 : 2;
     const size_t n_x = (size_t)pr.B * pr.D * L;
     const size_t n_dl = (size_t)pr.B * pr.K * pr.D * L;
     const size_t n_bc = (size_t)pr.B * pr.K * pr.N * L;

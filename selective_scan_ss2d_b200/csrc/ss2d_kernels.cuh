@@ -41,7 +41,10 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 #include <stdint.h>
 
 #include "ss2d_params.h"
@@ -50,6 +53,17 @@ namespace ss2d {
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
+
+// float value of the 16 stored bits of a 2-byte input type
+template <typename Tin>
+__device__ __forceinline__ float half_bits_to_f32(uint32_t bits16)
+{
+    if constexpr (std::is_same_v<Tin, __half>)
+        return __half2float(__ushort_as_half((unsigned short)bits16));
+    else
+        return __uint_as_float(bits16 << 16);
+}
 
 // Programmatic dependent launch (sm_90+): a kernel launched as a dependent
 // of the previous one on the stream may start before that one has finished;
@@ -182,9 +196,11 @@ struct Row16 {
     uint32_t w[RW];
     __device__ __forceinline__ float get(int i) const
     {
-        if constexpr (sizeof(Tin) == 2) {
+        if constexpr (std::is_same_v<Tin, __nv_bfloat16>) {
             const uint32_t v = w[i >> 1];
             return __uint_as_float((i & 1) ? (v & 0xffff0000u) : (v << 16));
+        } else if constexpr (std::is_same_v<Tin, __half>) {
+            return half_bits_to_f32<Tin>((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xffffu));
         } else {
             return __uint_as_float(w[i]);
         }
@@ -213,13 +229,13 @@ struct Row16 {
             w[2 * q + 1] = x.y;
         }
     }
-    // bf16 rows whose start is only 2-byte aligned: nine 4-byte word loads
+    // 2-byte rows whose start is only 2-byte aligned: nine 4-byte word loads
     // from the aligned word at or before src, realigned with funnel shifts.
     // Reads up to two values past the sixteen; the caller guarantees they
     // exist.
     __device__ __forceinline__ void load_words(const Tin *src)
     {
-        static_assert(sizeof(Tin) == 2, "4-byte words hold two bf16 values");
+        static_assert(sizeof(Tin) == 2, "4-byte words hold two 2-byte values");
         const uintptr_t a = reinterpret_cast<uintptr_t>(src);
         const uint32_t *wp = reinterpret_cast<const uint32_t *>(a & ~(uintptr_t)3);
         const unsigned sh = (unsigned)(a & 2) * 8;   // 0 or 16
@@ -259,6 +275,10 @@ struct Row16 {
 
 __device__ __forceinline__ uint32_t raw_bits(const float *p) { return __float_as_uint(__ldg(p)); }
 __device__ __forceinline__ uint32_t raw_bits(const __nv_bfloat16 *p)
+{
+    return (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p));
+}
+__device__ __forceinline__ uint32_t raw_bits(const __half *p)
 {
     return (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p));
 }
@@ -659,22 +679,37 @@ constexpr int kMerge2Threads = 256;
 // infinite and the result is -0)
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
 // gate factors of four consecutive y elements starting at index i of z
-__device__ __forceinline__ float4 gate4(const void *z, int bf16, size_t i)
+// (zt: 0 float32, 1 bfloat16, 2 float16 storage of z)
+__device__ __forceinline__ float4 gate4(const void *z, int zt, size_t i)
 {
     float4 g;
-    if (bf16) {
-        const uint2 r = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(z) + i));
-        g = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
-                        __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
-    } else {
+    if (zt == 0) {
         g = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(z) + i));
+    } else {
+        const uint2 r =
+            __ldg(reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(z) + i));
+        if (zt == 1)
+            g = make_float4(half_bits_to_f32<__nv_bfloat16>(r.x & 0xffffu),
+                            half_bits_to_f32<__nv_bfloat16>(r.x >> 16),
+                            half_bits_to_f32<__nv_bfloat16>(r.y & 0xffffu),
+                            half_bits_to_f32<__nv_bfloat16>(r.y >> 16));
+        else
+            g = make_float4(half_bits_to_f32<__half>(r.x & 0xffffu),
+                            half_bits_to_f32<__half>(r.x >> 16),
+                            half_bits_to_f32<__half>(r.y & 0xffffu),
+                            half_bits_to_f32<__half>(r.y >> 16));
     }
     return make_float4(silu_f(g.x), silu_f(g.y), silu_f(g.z), silu_f(g.w));
 }
-__device__ __forceinline__ float gate1(const void *z, int bf16, size_t i)
+__device__ __forceinline__ float gate1(const void *z, int zt, size_t i)
 {
-    const float v = bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(z)[i])
-                         : __ldg(static_cast<const float *>(z) + i);
+    float v;
+    if (zt == 0) {
+        v = __ldg(static_cast<const float *>(z) + i);
+    } else {
+        const uint32_t b = __ldg(static_cast<const unsigned short *>(z) + i);
+        v = zt == 1 ? half_bits_to_f32<__nv_bfloat16>(b) : half_bits_to_f32<__half>(b);
+    }
     return silu_f(v);
 }
 __device__ __forceinline__ float4 mul4(float4 a, float4 b)
@@ -686,7 +721,7 @@ template <int VEC, int CG>
 __global__ void __launch_bounds__(kMerge2Threads)
     merge2_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
                   int W, int K, int cols, int sum, int R, int whole, int flat,
-                  const void *__restrict__ z, int z_bf16)
+                  const void *__restrict__ z, int zt)
 {
     extern __shared__ float smem_m2[];   // cols: [CG][2][R][W + 1], whole: [CG][2][L]
     grid_dependency_wait();   // the output pass's rows
@@ -739,7 +774,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
             if (sum) {
                 float4 v = make_float4(v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w);
                 if (z)
-                    v = mul4(v, gate4(z, z_bf16, yr0 + 4 * f));
+                    v = mul4(v, gate4(z, zt, yr0 + 4 * f));
                 yo[f] = v;
             } else {
                 yo[f] = v0;
@@ -851,7 +886,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
                     v = make_float4((v.x + v2.x) + v3.x, (v.y + v2.y) + v3.y,
                                     (v.z + v2.z) + v3.z, (v.w + v2.w) + v3.w);
                 if (z)
-                    v = mul4(v, gate4(z, z_bf16, yr + p));
+                    v = mul4(v, gate4(z, zt, yr + p));
                 *reinterpret_cast<float4 *>(yo + p) = v;
             } else {
                 *reinterpret_cast<float4 *>(yo + p) = v0;
@@ -878,7 +913,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
                 if (cols)
                     v = (v + v2) + v3;
                 if (z)
-                    v *= gate1(z, z_bf16, yr + p);
+                    v *= gate1(z, zt, yr + p);
                 yo[p] = v;
             } else {
                 yo[p] = v;

@@ -119,12 +119,19 @@ Plan make_plan(int v, int B, int D, int L, int K)
     return pl;
 }
 
-cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t st,
+cudaError_t launch_scan(const Plan &plan, int dtype, ScanParams &p, cudaStream_t st,
                         cudaEvent_t *ev)
 {
     p.LC = plan.LC;
     p.NC = plan.NC;
-    return bf16 ? launch_scan_bf16(plan, p, st, ev) : launch_scan_f32(plan, p, st, ev);
+    switch (dtype) {
+    case 1:
+        return launch_scan_bf16(plan, p, st, ev);
+    case 2:
+        return launch_scan_f16(plan, p, st, ev);
+    default:
+        return launch_scan_f32(plan, p, st, ev);
+    }
 }
 
 namespace {
@@ -178,12 +185,12 @@ MergeShape merge_shape(int D, int H, int W, int K, int two_d)
 template <int VEC, int CG>
 cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int B, int D,
                           int H, int W, int K, int sum, cudaStream_t st, const void *z,
-                          int z_bf16)
+                          int zt)
 {
     const long long groups = ((long long)B * D + CG - 1) / CG;
     dim3 grid((unsigned)groups, (unsigned)m.nbands);
     return launch_kernel(merge2_kernel<VEC, CG>, grid, dim3(kMerge2Threads), m.smem, st, true,
-                         part, y, B, D, H, W, K, m.cols, sum, m.R, m.whole, m.flat, z, z_bf16);
+                         part, y, B, D, H, W, K, m.cols, sum, m.R, m.whole, m.flat, z, zt);
 }
 }  // namespace
 
@@ -193,7 +200,7 @@ size_t merge_smem_bytes(int H, int W, int K, int two_d)
 }
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
-                         int two_d, int sum, cudaStream_t st, const void *z, int z_bf16)
+                         int two_d, int sum, cudaStream_t st, const void *z, int zt)
 {
     const MergeShape m = merge_shape(D, H, W, K, two_d);
     if (m.smem > kMergeSmemMax)
@@ -202,7 +209,7 @@ cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W
         return cudaErrorInvalidConfiguration;
 #define SS2D_MERGE(V, C)                                                             \
     if (m.vec == V && m.CG == C)                                                     \
-        return launch_merge2<V, C>(m, part, y, B, D, H, W, K, sum, st, z, z_bf16);
+        return launch_merge2<V, C>(m, part, y, B, D, H, W, K, sum, st, z, zt);
     SS2D_MERGE(4, 1) SS2D_MERGE(4, 2) SS2D_MERGE(4, 4) SS2D_MERGE(4, 8) SS2D_MERGE(4, 16)
     SS2D_MERGE(1, 1) SS2D_MERGE(1, 2) SS2D_MERGE(1, 4) SS2D_MERGE(1, 8) SS2D_MERGE(1, 16)
 #undef SS2D_MERGE

@@ -63,17 +63,18 @@ Plan make_plan(int variant, int B, int D, int L, int K);
 // set p.out (and p.hstate / p.dtsum when plan.NC > 1).  If ev is not null,
 // ev[0..3] are recorded on the stream before the state pass, the carry, the
 // output pass and after it (the first two only when the plan is chunked).
-cudaError_t launch_scan(const Plan &plan, bool bf16, ScanParams &p, cudaStream_t st,
+cudaError_t launch_scan(const Plan &plan, int dtype, ScanParams &p, cudaStream_t st,
                         cudaEvent_t *ev = nullptr);
-// the same for one input dtype (ss2d_scan_bf16.cu, ss2d_scan_f32.cu)
+// the same for one input dtype (ss2d_scan_bf16.cu, ss2d_scan_f32.cu, ss2d_scan_f16.cu)
 cudaError_t launch_scan_bf16(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
 cudaError_t launch_scan_f32(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
+cudaError_t launch_scan_f16(const Plan &plan, ScanParams &p, cudaStream_t st, cudaEvent_t *ev);
 // cross_merge of the scan-order rows in `part` into y (sum = 1) or into the
 // per-direction pixel-order copy (sum = 0); with z (sum = 1 only), y is
-// multiplied by SiLU(z) (z in the layout of y, bf16 when z_bf16).
+// multiplied by SiLU(z) (z in the layout of y; zt = the ss2d_dtype of z).
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st, const void *z = nullptr,
-                         int z_bf16 = 0);
+                         int zt = 0);
 size_t merge_smem_bytes(int H, int W, int K, int two_d);
 
 // Text that ss2d_last_error() returns on the calling thread.

@@ -86,7 +86,7 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     int rc = ss2d_plan(1, B, D, H, W, N, K, -1, &LC, &NC, &launches);
     if (rc != SS2D_OK)
         return rc;
-    if (dtype != SS2D_F32 && dtype != SS2D_BF16)
+    if (dtype != SS2D_F32 && dtype != SS2D_BF16 && dtype != SS2D_F16)
         return SS2D_ERR_DTYPE;
     if (B == 0 || D == 0 || H == 0 || W == 0)
         return SS2D_OK;
@@ -154,14 +154,14 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes + hs_bytes) : nullptr;
     {
         // row vector width of delta/x (dtype) and of out (float32), as ss2d_forward
-        const size_t esz = dtype == SS2D_BF16 ? 2 : 4;
+        const size_t esz = dtype == SS2D_F32 ? 4 : 2;
         const bool ptr_ok = (((uintptr_t)x | (uintptr_t)delta | (uintptr_t)p.out) & 15) == 0;
         const size_t rb = (size_t)L * esz;
         p.vec = !ptr_ok ? 0 : (rb % 16 == 0 ? 16 : (rb % 8 == 0 ? 8 : 0));
         p.ovec = (ptr_ok && ((size_t)L * 4) % 16 == 0) ? 1 : 0;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    e = ss2d::launch_scan(pl, dtype == SS2D_BF16, p, st, nullptr);
+    e = ss2d::launch_scan(pl, dtype, p, st, nullptr);
     if (e == cudaSuccess && K > 1)
         e = ss2d::launch_merge(p.out, y, B, D, H, W, K, 1, 1, st);
     if (e != cudaSuccess) {

@@ -33,13 +33,15 @@ static_assert(kQStates == 4 && kT == 16, "quad layout: 4 states per lane, 16-ste
 // four consecutive values of one row as raw 32-bit words
 template <typename Tin>
 struct Quad4 {
-    static constexpr int RW = (int)sizeof(Tin);   // words: bf16 2, float 4
+    static constexpr int RW = (int)sizeof(Tin);   // words: 2-byte types 2, float 4
     uint32_t w[RW];
     __device__ __forceinline__ float get(int i) const
     {
-        if constexpr (sizeof(Tin) == 2) {
+        if constexpr (std::is_same_v<Tin, __nv_bfloat16>) {
             const uint32_t v = w[i >> 1];
             return __uint_as_float((i & 1) ? (v & 0xffff0000u) : (v << 16));
+        } else if constexpr (std::is_same_v<Tin, __half>) {
+            return half_bits_to_f32<Tin>((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xffffu));
         } else {
             return __uint_as_float(w[i]);
         }

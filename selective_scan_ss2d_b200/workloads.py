@@ -2,8 +2,8 @@
 
 This module draws inputs and nothing else: it holds none of the method's
 arithmetic.  The same arrays feed the CUDA library and the float64 oracle, so
-both see identical values (bf16 inputs are rounded here once, and the oracle
-reads those rounded values back as float64).
+both see identical values (bf16 and fp16 inputs are rounded here once, and
+the oracle reads those rounded values back as float64).
 
 Shapes follow the models the pages describe: the VMamba hierarchy ("Vision
 Mamba" tutorial, section "VMamba Hierarchical Architecture": 4x4 patches,
@@ -16,8 +16,8 @@ Recipe (seeded NumPy PCG64, one generator per workload, draws in this order):
 x (or u), delta, Bs, Cs ~ N(0, 1) in float32; then dt = exp(U[ln 1e-3, ln 1e-1])
 per row k*D+d; delta_bias = softplus^-1(dt) = ln(expm1(dt)); A_log[kd, n] =
 ln(n + 1) (the tutorial's initialisation of A); Dskip = 1.  For bf16
-workloads x, delta, Bs and Cs are rounded to bfloat16 (round to nearest,
-ties to even).  Parameters stay float32.
+workloads x, delta, Bs and Cs are rounded to bfloat16, for f16 workloads to
+IEEE float16 (both round to nearest, ties to even).  Parameters stay float32.
 """
 from __future__ import annotations
 
@@ -28,6 +28,7 @@ import numpy as np
 
 F32 = "f32"
 BF16 = "bf16"
+F16 = "f16"   # IEEE binary16 storage (float16 arrays)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -103,8 +104,9 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 @dataclasses.dataclass
 class Inputs:
-    """One workload's arrays in storage form: float32, or uint16 bfloat16
-    patterns for the four streamed inputs of bf16 workloads."""
+    """One workload's arrays in storage form: float32, uint16 bfloat16
+    patterns (bf16 workloads) or float16 (f16 workloads) for the four streamed
+    inputs."""
     cfg: Config
     x: np.ndarray          # (B,D,H,W) or (B,D,L)
     delta: np.ndarray      # (B,K,D,L)
@@ -135,7 +137,11 @@ class Inputs:
 
 def _normal(rng, shape, dtype):
     a = rng.standard_normal(size=shape, dtype=np.float32)
-    return f32_to_bf16_bits(a).reshape(shape) if dtype == BF16 else a
+    if dtype == BF16:
+        return f32_to_bf16_bits(a).reshape(shape)
+    if dtype == F16:
+        return a.astype(np.float16)   # IEEE round to nearest, ties to even
+    return a
 
 
 def make_inputs(cfg: Config | str, seed: int = 0) -> Inputs:

@@ -12,7 +12,7 @@ from selective_scan_ss2d_b200 import workloads as wl
 
 # fp32 inputs: per element |y - y_ref| <= FP32_TOL * max(1, |y_ref|)
 FP32_TOL = 1e-4
-# bf16 inputs (fp32 state): ||y - y_ref||_2 <= BF16_REL_L2 * ||y_ref||_2
+# bf16 or fp16 inputs (fp32 state): ||y - y_ref||_2 <= BF16_REL_L2 * ||y_ref||_2
 BF16_REL_L2 = 1e-3
 
 

@@ -2,8 +2,8 @@
 inputs, through the C ABI (ctypes binding).
 
 Bars: index maps bit-exact (integer-valued inputs); fp32 inputs per element
-|y - y_ref| <= 1e-4 * max(1, |y_ref|); bf16 inputs (fp32 state) relative L2
-<= 1e-3, the oracle reading the same bf16-rounded values.
+|y - y_ref| <= 1e-4 * max(1, |y_ref|); bf16 or fp16 inputs (fp32 state)
+relative L2 <= 1e-3, the oracle reading the same rounded values.
 """
 import numpy as np
 import pytest
@@ -54,7 +54,7 @@ SMALL_1D = [
 
 
 @pytest.mark.parametrize("cfg", SMALL_2D + SMALL_1D, ids=lambda c: c.name)
-@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16, wl.F16])
 def test_small_shapes_all_variants(cfg, dtype):
     cfg = cfg.with_(dtype=dtype)
     inp = wl.make_inputs(cfg, seed=1)
@@ -104,16 +104,15 @@ INDEX_SHAPES = [small(B=2, D=5, H=5, W=7, N=1), small(B=1, D=3, H=56, W=56, N=1)
 
 
 @pytest.mark.parametrize("cfg", INDEX_SHAPES, ids=lambda c: c.name)
-@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16, wl.F16])
 def test_index_maps_bit_exact(cfg, dtype):
     rng = np.random.default_rng(5)
     inp = _running_sum_inputs(cfg, rng)
-    if dtype == wl.BF16:
-        # every value involved (small integers, 0, 1, 1/32) is exact in bf16
-        b = inp.cfg.with_(dtype=wl.BF16)
-        inp = wl.Inputs(b, wl.f32_to_bf16_bits(inp.x), wl.f32_to_bf16_bits(inp.delta),
-                        wl.f32_to_bf16_bits(inp.Bs), wl.f32_to_bf16_bits(inp.Cs), inp.A_log,
-                        inp.Dskip, inp.delta_bias)
+    if dtype != wl.F32:
+        # every value involved (small integers, 0, 1, 1/32) is exact in bf16 and f16
+        cast = wl.f32_to_bf16_bits if dtype == wl.BF16 else (lambda a: a.astype(np.float16))
+        inp = wl.Inputs(inp.cfg.with_(dtype=dtype), cast(inp.x), cast(inp.delta), cast(inp.Bs),
+                        cast(inp.Cs), inp.A_log, inp.Dskip, inp.delta_bias)
     # The exact result is an integer running sum.  The oracle's float64
     # softplus(32) is 32 * (1 + 4e-16), so its sums carry residues below
     # 1e-12; rounding to the nearest integer recovers the exact values.
@@ -262,7 +261,7 @@ GATED = [small(B=2, D=12, H=7, W=9, K=4, N=16), small(B=1, D=40, H=14, W=14, K=4
 
 
 @pytest.mark.parametrize("cfg", GATED, ids=lambda c: c.name)
-@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16, wl.F16])
 def test_gated_matches_oracle(cfg, dtype):
     cfg = cfg.with_(dtype=dtype)
     inp = wl.make_inputs(cfg, seed=4)

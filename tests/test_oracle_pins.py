@@ -187,6 +187,27 @@ def test_workload_recipe():
     assert cfg.updates == 8192
 
 
+def test_half_workloads_round_the_float32_draws():
+    """bf16 and f16 workloads are the float32 draws rounded to nearest-even
+    (same seed, same order), and as_f64 gives back exactly those values."""
+    base = wl.make_inputs("tiny_fp32", seed=2)
+    f16 = wl.make_inputs(base.cfg.with_(dtype=wl.F16), seed=2)
+    bf = wl.make_inputs(base.cfg.with_(dtype=wl.BF16), seed=2)
+    assert f16.x.dtype == np.float16 and bf.x.dtype == np.uint16
+    for name in wl.Inputs.STREAMED:
+        a = getattr(base, name)
+        assert np.array_equal(getattr(f16, name), a.astype(np.float16))
+        assert np.array_equal(f16.as_f64()[name], a.astype(np.float16).astype(np.float64))
+        assert np.array_equal(bf.as_f64()[name],
+                              wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(a)).astype(np.float64))
+        # both roundings stay within half a unit in the last place of their format
+        assert np.all(np.abs(f16.as_f64()[name] - a) <= np.abs(a) * 2.0 ** -11 + 2.0 ** -25)
+    assert f16.cfg.in_bytes_per_elem == 2 and base.cfg.in_bytes_per_elem == 4
+    z = wl.make_gate(f16.cfg, seed=2)
+    assert z.dtype == np.float16
+    assert np.array_equal(wl.gate_as_f64(z, f16.cfg), z.astype(np.float64))
+
+
 def test_config_table_matches_the_workloads():
     c = wl.CONFIGS
     assert (c["vmamba_t_stage1"].B, c["vmamba_t_stage1"].D, c["vmamba_t_stage1"].L) == (8, 192, 3136)
