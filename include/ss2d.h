@@ -154,6 +154,35 @@ int selective_scan_fwd_gated(const void *u, const void *delta, const float *A_lo
                              int B, int D, int L, int N, int K, int dtype,
                              void *stream);
 
+/* Backward of ss2d_forward / selective_scan_fwd: the gradients of
+ * sum(dy * y) with respect to every input ("Vision Mamba ..." summary,
+ * section 4.4: the backward recomputes the scan from the inputs instead of
+ * reading stored states; here from chunk entry states every 16 steps).
+ *   dy          float32, the layout of y (and of x / u)
+ *   dx / du     float32, the layout of x / u
+ *   ddelta      float32 (B,K,D,L), scan order, like delta
+ *   dA_log      float32 (K*D,N)      dBs, dCs  float32 (B,K,N,L)
+ *   dDskip      float32 (K*D)        ddelta_bias float32 (K*D)
+ * Every output is overwritten.  The inputs are those of the forward call
+ * (same dtype, layouts, K and N rules); all pointers are device pointers of
+ * the current device, 16-byte aligned (host pointers: SS2D_ERR_PTR).
+ * Asynchronous on `stream`; scratch comes from the library's stream-ordered
+ * pool.  The parameter gradients are summed over the batch and the
+ * sequence in a fixed order, so repeated calls give identical results.
+ * With B, H*W or L zero the parameter gradients are set to zero. */
+int ss2d_backward(const void *x, const void *delta, const float *A_log,
+                  const void *Bs, const void *Cs, const float *Dskip,
+                  const float *delta_bias, const float *dy,
+                  float *dx, float *ddelta, float *dA_log, float *dBs, float *dCs,
+                  float *dDskip, float *ddelta_bias,
+                  int B, int D, int H, int W, int N, int K, int dtype, void *stream);
+int selective_scan_bwd(const void *u, const void *delta, const float *A_log,
+                       const void *Bs, const void *Cs, const float *Dskip,
+                       const float *delta_bias, const float *dy,
+                       float *du, float *ddelta, float *dA_log, float *dBs, float *dCs,
+                       float *dDskip, float *ddelta_bias,
+                       int B, int D, int L, int N, int K, int dtype, void *stream);
+
 /* As ss2d_forward, with an explicit kernel variant (index into the table
  * that ss2d_variant_name() describes; -1 = the library's own choice for the
  * shape).  Every variant computes the same result up to float32 rounding

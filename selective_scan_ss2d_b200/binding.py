@@ -67,6 +67,11 @@ def lib() -> ctypes.CDLL:
             L.selective_scan_fwd_gated.argtypes = gfwd + [i] * 6 + [vp]
             L.selective_scan_fwd_gated.restype = i
             L.ss2d_scan_directions.restype = i
+            bwd = fwd[:7] + [fp] + [fp] * 7   # dy, then the seven gradients
+            L.ss2d_backward.argtypes = bwd + [i] * 7 + [vp]
+            L.ss2d_backward.restype = i
+            L.selective_scan_bwd.argtypes = bwd + [i] * 6 + [vp]
+            L.selective_scan_bwd.restype = i
             L.ss2d_plan.argtypes = [i] * 8 + [ctypes.POINTER(ctypes.c_int)] * 3
             L.ss2d_plan.restype = i
             L.ss2d_forward_noalloc.argtypes = fwd + [i] * 7 + [vp]
@@ -316,3 +321,51 @@ def ss2d_forward_timed(x, delta, A_log, Bs, Cs, Dskip, delta_bias, y, *, two_d: 
                                     _ptr(Dskip), _ptr(delta_bias), _ptr(y), B, D, H, W, N, K,
                                     dt, int(bool(two_d)), st, int(variant), ms))
     return [float(v) for v in ms]
+
+
+GRAD_NAMES = ("dx", "ddelta", "dA_log", "dBs", "dCs", "dDskip", "ddelta_bias")
+
+
+def _backward(fn, name, x, delta, A_log, Bs, Cs, Dskip, delta_bias, dy, dims, stream):
+    K, N = delta.shape[1], Bs.shape[2]
+    B, D = x.shape[0], x.shape[1]
+    L = 1
+    for v in x.shape[2:]:
+        L *= v
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError(f"inconsistent shapes for {name}")
+    if dy.dtype != torch.float32 or tuple(dy.shape) != tuple(x.shape) or not dy.is_contiguous() \
+            or dy.device != x.device:
+        raise ValueError("dy must be a contiguous float32 tensor of x's shape and device")
+    _, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, dy, tuple(x.shape))
+    if not on_gpu:
+        raise ValueError(f"{name} takes device tensors only")
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = dict(dx=torch.empty(tuple(x.shape), **f32), ddelta=torch.empty(tuple(delta.shape), **f32),
+             dA_log=torch.empty((K * D, N), **f32), dBs=torch.empty(tuple(Bs.shape), **f32),
+             dCs=torch.empty(tuple(Cs.shape), **f32), dDskip=torch.empty((K * D,), **f32),
+             ddelta_bias=torch.empty((K * D,), **f32))
+    st = _stream(True, x.device, stream)
+    rc = fn(_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs), _ptr(Dskip),
+            _ptr(delta_bias), _ptr(dy), *[_ptr(g[n]) for n in GRAD_NAMES], B, D, *dims, N, K,
+            dt, st)
+    _check(rc)
+    return g
+
+
+def ss2d_backward(x, delta, A_log, Bs, Cs, Dskip, delta_bias, dy, *, stream=None):
+    """Gradients of sum(dy * ss2d_forward(...)) with respect to every input.
+    Device tensors only; dy float32 of x's shape.  Returns a dict of float32
+    tensors: dx, ddelta, dA_log, dBs, dCs, dDskip, ddelta_bias."""
+    H, W = x.shape[2], x.shape[3]
+    return _backward(lib().ss2d_backward, "ss2d_backward", x, delta, A_log, Bs, Cs, Dskip,
+                     delta_bias, dy, (H, W), stream)
+
+
+def selective_scan_bwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, dy, *, stream=None):
+    """Gradients of sum(dy * selective_scan_fwd(...)); the dict's "dx" is the
+    gradient with respect to u."""
+    return _backward(lib().selective_scan_bwd, "selective_scan_bwd", u, delta, A_log, Bs, Cs,
+                     Dskip, delta_bias, dy, (u.shape[2],), stream)

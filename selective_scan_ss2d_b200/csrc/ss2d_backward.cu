@@ -1,0 +1,105 @@
+// ss2d_backward.cu -- plan and launch sequence of the backward pass (kernels
+// in ss2d_backward.cuh), for the three input dtypes.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ss2d_backward.cuh"
+#include "ss2d_launch.h"
+
+namespace ss2d {
+
+namespace {
+// CTAs (one warp each) wanted in flight: about five resident per SM (the
+// final kernel's 42 KB of shared memory) times four waves
+constexpr long long kBwdWantCtas = 148LL * 5 * 4;
+
+template <typename Tin>
+cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
+{
+    const dim3 grid((unsigned)((long long)p.G * p.B * p.K), (unsigned)p.CGN);
+    if (p.NC > 1) {
+        bwd_local_kernel<Tin><<<grid, kBwdLanes, 0, st>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+        // the forward's carry over the chunk end states, then over the
+        // reversed local adjoints
+        ScanParams c{};
+        c.A_log = p.A_log;
+        c.B = p.B;
+        c.D = p.D;
+        c.K = p.K;
+        c.N = p.N;
+        c.L = p.L;
+        c.NC = p.NC;
+        const long long total = (long long)p.B * p.K * p.D * kNP;
+        const dim3 cgrid((unsigned)((total + 255) / 256));
+        c.hstate = p.hfwd;
+        c.dtsum = p.dtf;
+        carry_kernel<<<cgrid, 256, 0, st>>>(c);
+        c.hstate = p.hadj;
+        c.dtsum = p.dta;
+        carry_kernel<<<cgrid, 256, 0, st>>>(c);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    bwd_final_kernel<Tin><<<grid, kBwdLanes, kBwdFinalSmem, st>>>(p);
+    return cudaGetLastError();
+}
+}  // namespace
+
+BwdShape backward_shape(int B, int D, int L, int K)
+{
+    BwdShape s;
+    s.NC = (L + kT - 1) / kT;
+    s.G = (D + kBwdLanes - 1) / kBwdLanes;
+    const long long ctas = (long long)s.G * B * K;
+    long long cgn = ctas > 0 ? (kBwdWantCtas + ctas - 1) / ctas : 1;
+    if (cgn > s.NC)
+        cgn = s.NC;
+    if (cgn < 1)
+        cgn = 1;
+    long long cpb = (s.NC + cgn - 1) / cgn;
+    const long long min_cpb = (s.NC + 65534) / 65535;   // gridDim.y <= 65535
+    if (cpb < min_cpb)
+        cpb = min_cpb;
+    if (cpb < 1)
+        cpb = 1;
+    s.CPB = (int)cpb;
+    s.CGN = (int)((s.NC + cpb - 1) / cpb);
+    return s;
+}
+
+cudaError_t launch_backward(const BwdParams &p, int dtype, cudaStream_t st)
+{
+    switch (dtype) {
+    case 1:
+        return launch_bwd_t<__nv_bfloat16>(p, st);
+    case 2:
+        return launch_bwd_t<__half>(p, st);
+    default:
+        return launch_bwd_t<float>(p, st);
+    }
+}
+
+cudaError_t launch_backward_reduce(const BwdParams &p, float *dBs, float *dCs, float *dA_log,
+                                   float *dDskip, float *ddelta_bias, cudaStream_t st)
+{
+    const long long nbc = (long long)p.B * p.K * 2 * p.N * p.L;
+    long long blocks = (nbc + 255) / 256;
+    if (blocks > 148LL * 64)
+        blocks = 148LL * 64;
+    bwd_reduce_bc_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.bc_part, dBs, dCs, p.B * p.K, p.G,
+                                                          p.N, p.L);
+    const long long npr = (long long)p.K * p.D * (p.N + 2);
+    blocks = (npr + 127) / 128;
+    if (blocks > 148LL * 64)
+        blocks = 148LL * 64;
+    bwd_reduce_param_kernel<<<(unsigned)blocks, 128, 0, st>>>(p.prm_part, p.A_log, dA_log, dDskip,
+                                                             ddelta_bias, p.B, p.K, p.D, p.N,
+                                                             p.CGN);
+    return cudaGetLastError();
+}
+
+}  // namespace ss2d

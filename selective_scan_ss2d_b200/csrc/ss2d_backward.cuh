@@ -1,0 +1,403 @@
+// ss2d_backward.cuh -- sm_100a kernels of the SS2D backward pass (gradients
+// of sum(dy * y) with respect to every input of the forward).
+//
+// The pages ask for a backward that recomputes the scan instead of keeping
+// the states in HBM ("Vision Mamba ..." summary, section 4.4).  With
+// a_t = exp(dt_t A) and the adjoint g_t = dLoss/dh_t,
+//     g_t   = dy_t C_t + a_{t+1} g_{t+1}
+//     dC_t  = sum_d dy_t h_t            dB_t = sum_d g_t dt_t u_t
+//     du_t  = Dskip dy_t + dt_t sum_n g_n B_t,n
+//     ddt_t = sum_n g_n (A_n a_t h_{t-1} + B_t,n u_t),  a_t h_{t-1} = h_t - dt_t u_t B_t
+//     dA_n  = sum_t g_n dt_t a_t h_{t-1},n
+// then ddelta = ddt * sigmoid(delta + bias), dA_log = dA * A, dbias and
+// dDskip the sums over (b, t), and dx gathers du of every direction back to
+// its pixel (the adjoint of cross_scan is cross_merge).
+//
+// Work decomposition: chunks of kT = 16 steps; a CTA is one warp holding 32
+// channels of one (b, k) and walks a range of chunks.
+//   1. bwd_local_kernel: per chunk, from zero, the forward end state h_end[c]
+//      and the local adjoint Q[c] = a_s g_s (g from zero at the chunk end),
+//      each with the chunk's sum of dt.  Q is stored in reversed chunk
+//      order, so that
+//   2. carry_kernel (the forward's) run twice gives the entry state of every
+//      chunk and, over the reversed order, the adjoint G[c] = a_{e+1} g_{e+1}
+//      entering every chunk from its end: G[c-1] = exp(A sum_c dt) G[c] + Q[c].
+//   3. bwd_final_kernel: per chunk, h recomputed from its entry state (the
+//      16 states of 16 steps of every lane parked in shared memory), then the
+//      reverse walk from G[c] writes ddelta and du, reduces dB and dC over
+//      the warp's channels (one reduce-scatter of 32 values per step) into a
+//      per-channel-group partial, and accumulates the parameter gradients.
+//   4. merge2_kernel (K > 1) sums du of the directions into dx; two fixed-order
+//      reductions finish dBs, dCs and dA_log, dDskip, ddelta_bias.
+// Every reduction runs in a fixed order: the result is reproducible.
+#pragma once
+
+#include "ss2d_bwd_params.h"
+#include "ss2d_kernels.cuh"
+
+namespace ss2d {
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+// shared memory of both kernels (floats): B and C of the chunk [t][n], and the
+// lanes' staged dt, u, dy and sigmoid(delta + bias) [t][lane]
+constexpr int kBwdStage = 2 * kT * kNP + 4 * kT * kBwdLanes;
+// the final kernel adds the recomputed states [t][n][lane] and the reduced
+// dB | dC values [t][lane]
+constexpr int kBwdStates = kT * kNP * kBwdLanes + kT * kBwdLanes;
+constexpr size_t kBwdFinalSmem = sizeof(float) * (kBwdStage + kBwdStates);
+
+struct BwdLane {
+    int b, k, gi, d, bk;
+    bool active;
+    size_t bkd;   // row (b, k, d) (d clamped for idle lanes)
+};
+
+__device__ __forceinline__ BwdLane bwd_lane(const BwdParams &p)
+{
+    BwdLane r;
+    const int lane = threadIdx.x;
+    r.gi = (int)(blockIdx.x % (unsigned)p.G);
+    r.bk = (int)(blockIdx.x / (unsigned)p.G);
+    r.b = r.bk / p.K;
+    r.k = r.bk - r.b * p.K;
+    r.d = r.gi * kBwdLanes + lane;
+    r.active = r.d < p.D;
+    if (!r.active)
+        r.d = p.D - 1;
+    r.bkd = ((size_t)r.b * p.K + r.k) * p.D + r.d;
+    return r;
+}
+
+// B and C of steps s .. s+nt-1 into sB, sC [t][n] (zeros past N and nt)
+template <typename Tin>
+__device__ __forceinline__ void bwd_stage_bc(const BwdParams &p, const BwdLane &q, int s, int nt,
+                                             float *sB, float *sC)
+{
+    const int lane = threadIdx.x;
+    const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
+    const bool nok = n < p.N;
+    const size_t row = (((size_t)q.b * p.K + q.k) * p.N + (nok ? n : 0)) * p.L + s;
+    const Tin *Bp = static_cast<const Tin *>(p.Bs) + row;
+    const Tin *Cp = static_cast<const Tin *>(p.Cs) + row;
+#pragma unroll
+    for (int i = 0; i < kT / 2; ++i) {
+        const int t = t0 + i;
+        const bool ok = nok && t < nt;
+        sB[t * kNP + n] = ok ? to_f32(Bp[t]) : 0.f;
+        sC[t * kNP + n] = ok ? to_f32(Cp[t]) : 0.f;
+    }
+}
+
+// this lane's dt, u, dy and sigmoid(delta + bias) of steps s .. s+nt-1 (zeros
+// past nt: dt = 0 makes a padded step the identity)
+template <typename Tin>
+__device__ __forceinline__ void bwd_stage_lane(const BwdParams &p, const BwdLane &q, int s, int nt,
+                                               float bias, float *sdt, float *su, float *sgy,
+                                               float *ssg)
+{
+    const int lane = threadIdx.x;
+    const Tin *dl = static_cast<const Tin *>(p.delta) + q.bkd * p.L + s;
+    const size_t xrow = ((size_t)q.b * p.D + q.d) * p.L;
+    const Tin *xp = static_cast<const Tin *>(p.x) + xrow;
+    const float *gp = p.dy + xrow;
+    PixWalk w;
+    w.init(p.two_d, q.k, s, p.H, p.W, p.L);
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+        float dt = 0.f, u = 0.f, gy = 0.f, sg = 0.f;
+        if (t < nt && q.active) {   // idle lanes add nothing to the dB, dC sums
+            const float z = to_f32(dl[t]) + bias;
+            dt = softplus_f(z);
+            // sigmoid(z) = 1 / (1 + e^-z); e^-z = inf gives 0
+            sg = __fdividef(1.f, 1.f + mufu_ex2(-z * kLog2e));
+            u = to_f32(xp[w.p]);
+            gy = __ldg(gp + w.p);
+            if (t + 1 < nt)
+                w.next(p.H, p.W);
+        }
+        sdt[t * kBwdLanes + lane] = dt;
+        su[t * kBwdLanes + lane] = u;
+        sgy[t * kBwdLanes + lane] = gy;
+        ssg[t * kBwdLanes + lane] = sg;
+    }
+}
+
+__device__ __forceinline__ void load16(float *v, const float *src)
+{
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int i = 0; i < kNP / 4; ++i) {
+        const float4 a = s4[i];
+        v[4 * i] = a.x;
+        v[4 * i + 1] = a.y;
+        v[4 * i + 2] = a.z;
+        v[4 * i + 3] = a.w;
+    }
+}
+
+__device__ __forceinline__ void store16(float *dst, const float *v)
+{
+    float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < kNP / 4; ++i)
+        d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
+{
+    __shared__ float sm[kBwdStage];
+    float *sB = sm, *sC = sB + kT * kNP, *sdt = sC + kT * kNP;
+    float *su = sdt + kT * kBwdLanes, *sgy = su + kT * kBwdLanes, *ssg = sgy + kT * kBwdLanes;
+    const int lane = threadIdx.x;
+    const BwdLane q = bwd_lane(p);
+    const size_t kd = (size_t)q.k * p.D + q.d;
+    float A2[kNP];
+#pragma unroll
+    for (int n = 0; n < kNP; ++n)
+        A2[n] = n < p.N ? -expf(__ldg(p.A_log + kd * p.N + n)) * kLog2e : 0.f;
+    const float bias = __ldg(p.delta_bias + kd);
+    const int nc1 = p.NC - 1;
+    const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
+    for (int c = c0; c < c1; ++c) {
+        const int s = c * kT, nt = min(kT, p.L - s);
+        __syncwarp();
+        bwd_stage_bc<Tin>(p, q, s, nt, sB, sC);
+        bwd_stage_lane<Tin>(p, q, s, nt, bias, sdt, su, sgy, ssg);
+        __syncwarp();
+        float dts = 0.f;
+#pragma unroll
+        for (int t = 0; t < kT; ++t)
+            dts += sdt[t * kBwdLanes + lane];
+        if (c < nc1) {
+            float h[kNP];
+#pragma unroll
+            for (int n = 0; n < kNP; ++n)
+                h[n] = 0.f;
+#pragma unroll
+            for (int t = 0; t < kT; ++t) {
+                const float dt = sdt[t * kBwdLanes + lane];
+                const float dtu = dt * su[t * kBwdLanes + lane];
+#pragma unroll
+                for (int n = 0; n < kNP; ++n)
+                    h[n] = fmaf(mufu_ex2(dt * A2[n]), h[n], dtu * sB[t * kNP + n]);
+            }
+            if (q.active) {
+                store16(p.hfwd + (q.bkd * nc1 + c) * kNP, h);
+                p.dtf[q.bkd * nc1 + c] = dts;
+            }
+        }
+        if (c > 0) {
+            float g[kNP];
+#pragma unroll
+            for (int n = 0; n < kNP; ++n)
+                g[n] = 0.f;
+#pragma unroll
+            for (int t = kT - 1; t >= 0; --t) {
+                const float dt = sdt[t * kBwdLanes + lane];
+                const float gy = sgy[t * kBwdLanes + lane];
+#pragma unroll
+                for (int n = 0; n < kNP; ++n)
+                    g[n] = mufu_ex2(dt * A2[n]) * fmaf(gy, sC[t * kNP + n], g[n]);
+            }
+            if (q.active) {
+                const int r = nc1 - c;   // reversed chunk order
+                store16(p.hadj + (q.bkd * nc1 + r) * kNP, g);
+                p.dta[q.bkd * nc1 + r] = dts;
+            }
+        }
+    }
+}
+
+// One halving exchange: lanes with bit M set keep v[M..2M) (moved to v[0..M)),
+// the others v[0..M); each adds the half its partner sends.
+template <int M>
+__device__ __forceinline__ void halve(float *v)
+{
+    const bool hi = (threadIdx.x & M) != 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        const float lo = v[i], up = v[i + M];
+        const float send = hi ? lo : up;
+        const float keep = hi ? up : lo;
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+    }
+}
+
+// Sum over the 32 lanes of v[j] for j = lane (v[0..15]: dB of the 16 states,
+// v[16..31]: dC): five halving exchanges, 31 shuffles.
+__device__ __forceinline__ float reduce_scatter32(float *v)
+{
+    halve<16>(v);
+    halve<8>(v);
+    halve<4>(v);
+    halve<2>(v);
+    halve<1>(v);
+    return v[0];
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
+{
+    extern __shared__ float4 smem_bwd4[];
+    float *sm = reinterpret_cast<float *>(smem_bwd4);
+    float *sB = sm, *sC = sB + kT * kNP, *sdt = sC + kT * kNP;
+    float *su = sdt + kT * kBwdLanes, *sgy = su + kT * kBwdLanes, *ssg = sgy + kT * kBwdLanes;
+    float *hs = ssg + kT * kBwdLanes;   // [t][n][lane]
+    float *sout = hs + kT * kNP * kBwdLanes;   // [t][lane]
+    const int lane = threadIdx.x;
+    const BwdLane q = bwd_lane(p);
+    const size_t kd = (size_t)q.k * p.D + q.d;
+    float A2[kNP];
+#pragma unroll
+    for (int n = 0; n < kNP; ++n)
+        A2[n] = n < p.N ? -expf(__ldg(p.A_log + kd * p.N + n)) * kLog2e : 0.f;
+    const float bias = __ldg(p.delta_bias + kd);
+    const float Dk = __ldg(p.Dskip + kd);
+    const int L = p.L, nc1 = p.NC - 1;
+    const bool flip = p.flip1 && q.k == 1;
+    float *durow = p.du + q.bkd * L;
+    float *ddrow = p.ddelta + q.bkd * L;
+    float *bcrow = p.bc_part +
+                   ((((size_t)q.bk * p.G + q.gi) * 2 + (lane >> 4)) * kNP + (lane & 15)) * L;
+    const bool bc_ok = (lane & 15) < p.N;
+    float dA[kNP];
+#pragma unroll
+    for (int n = 0; n < kNP; ++n)
+        dA[n] = 0.f;
+    float dD = 0.f, db = 0.f;
+    const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
+    for (int c = c0; c < c1; ++c) {
+        const int s = c * kT, nt = min(kT, L - s);
+        __syncwarp();
+        bwd_stage_bc<Tin>(p, q, s, nt, sB, sC);
+        bwd_stage_lane<Tin>(p, q, s, nt, bias, sdt, su, sgy, ssg);
+        __syncwarp();
+        // states of the chunk, from its entry state
+        {
+            float h[kNP];
+            if (c > 0)
+                load16(h, p.hfwd + (q.bkd * nc1 + (c - 1)) * kNP);
+            else
+#pragma unroll
+                for (int n = 0; n < kNP; ++n)
+                    h[n] = 0.f;
+#pragma unroll 1
+            for (int t = 0; t < kT; ++t) {
+                const float dt = sdt[t * kBwdLanes + lane];
+                const float dtu = dt * su[t * kBwdLanes + lane];
+#pragma unroll
+                for (int n = 0; n < kNP; ++n) {
+                    h[n] = fmaf(mufu_ex2(dt * A2[n]), h[n], dtu * sB[t * kNP + n]);
+                    hs[(t * kNP + n) * kBwdLanes + lane] = h[n];
+                }
+            }
+        }
+        // reverse walk from the adjoint entering at the chunk end
+        float g[kNP];
+        if (c < nc1)
+            load16(g, p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
+        else
+#pragma unroll
+            for (int n = 0; n < kNP; ++n)
+                g[n] = 0.f;
+#pragma unroll 1
+        for (int t = kT - 1; t >= 0; --t) {
+            const float dt = sdt[t * kBwdLanes + lane];
+            const float u = su[t * kBwdLanes + lane];
+            const float gy = sgy[t * kBwdLanes + lane];
+            const float dtu = dt * u;
+            float v[2 * kNP];
+            float s1 = 0.f, s2 = 0.f;   // sum g A2 (a h_prev), sum g B
+#pragma unroll
+            for (int n = 0; n < kNP; ++n) {
+                const float Bv = sB[t * kNP + n];
+                const float hv = hs[(t * kNP + n) * kBwdLanes + lane];
+                g[n] = fmaf(gy, sC[t * kNP + n], g[n]);
+                const float hp = fmaf(-dtu, Bv, hv);   // a_t h_{t-1}
+                const float gdt = g[n] * dt;
+                v[n] = gdt * u;
+                v[kNP + n] = gy * hv;
+                s2 = fmaf(g[n], Bv, s2);
+                s1 = fmaf(g[n] * A2[n], hp, s1);
+                dA[n] = fmaf(gdt, hp, dA[n]);
+                g[n] *= mufu_ex2(dt * A2[n]);
+            }
+            sout[t * kBwdLanes + lane] = reduce_scatter32(v);
+            if (q.active && t < nt) {
+                const int l = s + t;
+                const float ddl = fmaf(kLn2, s1, u * s2) * ssg[t * kBwdLanes + lane];
+                dD = fmaf(gy, u, dD);
+                db += ddl;
+                ddrow[l] = ddl;
+                durow[flip ? L - 1 - l : l] = fmaf(Dk, gy, dt * s2);
+            }
+        }
+        if (bc_ok) {
+            for (int t = 0; t < nt; ++t)
+                bcrow[s + t] = sout[t * kBwdLanes + lane];
+        }
+    }
+    if (q.active) {
+        float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * kPrm;
+#pragma unroll
+        for (int n = 0; n < kNP; ++n)
+            pr[n] = dA[n];
+        pr[kNP] = dD;
+        pr[kNP + 1] = db;
+    }
+}
+
+// dBs, dCs (B,K,N,L) = the sum over the channel groups, in group order
+__global__ void bwd_reduce_bc_kernel(const float *__restrict__ part, float *__restrict__ dBs,
+                                     float *__restrict__ dCs, int BK, int G, int N, int L)
+{
+    const long long total = (long long)BK * 2 * N * L;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int l = (int)(i % L);
+        long long r = i / L;
+        const int n = (int)(r % N);
+        r /= N;
+        const int which = (int)(r & 1);
+        const long long bk = r >> 1;
+        const float *src = part + (((size_t)bk * G * 2 + which) * kNP + n) * L + l;
+        const size_t gstride = (size_t)2 * kNP * L;
+        float s = 0.f;
+        for (int g = 0; g < G; ++g)
+            s += __ldg(src + g * gstride);
+        (which ? dCs : dBs)[((size_t)bk * N + n) * L + l] = s;
+    }
+}
+
+// dA_log = A * sum dA, dDskip, ddelta_bias: per (k, d), the sum over b and
+// the chunk groups, in that order
+__global__ void bwd_reduce_param_kernel(const float *__restrict__ prm,
+                                        const float *__restrict__ A_log, float *__restrict__ dA_log,
+                                        float *__restrict__ dDskip, float *__restrict__ dbias,
+                                        int B, int K, int D, int N, int CGN)
+{
+    const long long total = (long long)K * D * (N + 2);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int j = (int)(i % (N + 2));
+        const long long kd = i / (N + 2);
+        const int k = (int)(kd / D), d = (int)(kd % D);
+        const int jj = j < N ? j : (j == N ? kNP : kNP + 1);
+        float s = 0.f;
+        for (int b = 0; b < B; ++b) {
+            const float *src = prm + ((((size_t)b * K + k) * D + d) * CGN) * kPrm + jj;
+            for (int cg = 0; cg < CGN; ++cg)
+                s += __ldg(src + (size_t)cg * kPrm);
+        }
+        if (j < N)
+            dA_log[kd * N + j] = s * -expf(__ldg(A_log + kd * N + j));
+        else if (j == N)
+            dDskip[kd] = s;
+        else
+            dbias[kd] = s;
+    }
+}
+
+}  // namespace ss2d

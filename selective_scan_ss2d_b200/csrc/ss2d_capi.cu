@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "ss2d.h"
+#include "ss2d_bwd_params.h"
 #include "ss2d_params.h"
 #include "ss2d_launch.h"
 
@@ -327,6 +328,132 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
     return kind == kDevicePtr ? run_device(pr, st, variant, false) : run_host(pr, st, variant);
 }
 
+// Backward: gradients of sum(dy * y).  Device pointers only.  Scratch from
+// the pool: chunk entry states and adjoints (when L > 16), the per-direction
+// du rows (K > 1) and the two reduction partials.
+struct Grads {
+    const float *dy;
+    float *dx, *ddelta, *dA_log, *dBs, *dCs, *dDskip, *ddelta_bias;
+};
+
+int backward(const Problem &pr, const Grads &gr, void *stream)
+{
+    int rc = validate(pr);
+    if (rc != SS2D_OK)
+        return rc;
+    if (pr.K * (long long)pr.D == 0)
+        return SS2D_OK;
+    // an empty batch or sequence reads nothing and writes only the parameter
+    // gradients (zero); otherwise every pointer is used
+    const bool empty = is_empty(pr);
+    const void *all[] = {gr.dA_log, gr.dDskip, gr.ddelta_bias, pr.x, pr.delta, pr.Bs, pr.Cs,
+                         pr.A_log, pr.Dskip, pr.delta_bias, gr.dy, gr.dx, gr.ddelta, gr.dBs,
+                         gr.dCs};
+    const int nptr = empty ? 3 : 15;
+    for (int i = 0; i < nptr; ++i)
+        if (!all[i])
+            return SS2D_ERR_NULL;
+    for (int i = 0; i < nptr; ++i)
+        if (((uintptr_t)all[i] & 15u) != 0)
+            return SS2D_ERR_ALIGN;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_error("cudaGetDevice", e);
+        return SS2D_ERR_CUDA;
+    }
+    for (int i = 0; i < nptr; ++i)
+        if (pointer_kind(all[i], dev) != kDevicePtr)
+            return SS2D_ERR_PTR;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long L = (long long)pr.H * pr.W;
+    if (empty) {
+        // no step anywhere: the parameter gradients are zero
+        const size_t kd = (size_t)pr.K * pr.D;
+        e = cudaMemsetAsync(gr.dA_log, 0, sizeof(float) * kd * pr.N, st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(gr.dDskip, 0, sizeof(float) * kd, st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(gr.ddelta_bias, 0, sizeof(float) * kd, st);
+        if (e != cudaSuccess) {
+            set_error("cudaMemsetAsync", e);
+            return SS2D_ERR_CUDA;
+        }
+        return SS2D_OK;
+    }
+    if (pr.K > 1 && ss2d::merge_smem_bytes(pr.H, pr.W, pr.K, pr.two_d) > 200 * 1024)
+        return SS2D_ERR_SHAPE;
+    const ss2d::BwdShape sh = ss2d::backward_shape(pr.B, pr.D, (int)L, pr.K);
+    if ((long long)sh.G * pr.B * pr.K > INT_MAX)
+        return SS2D_ERR_SHAPE;
+    const size_t rows = (size_t)pr.B * pr.K * pr.D;
+    const size_t nc1 = (size_t)sh.NC - 1;
+    const size_t hs_bytes = align256(sizeof(float) * rows * nc1 * ss2d::kNP);
+    const size_t ds_bytes = align256(sizeof(float) * rows * nc1);
+    const size_t du_bytes = pr.K > 1 ? align256(sizeof(float) * rows * L) : 0;
+    const size_t bc_bytes =
+        align256(sizeof(float) * pr.B * pr.K * (size_t)sh.G * 2 * ss2d::kNP * L);
+    const size_t pr_bytes = align256(sizeof(float) * rows * sh.CGN * ss2d::kPrm);
+    const size_t total = 2 * hs_bytes + 2 * ds_bytes + du_bytes + bc_bytes + pr_bytes;
+    void *scratch = nullptr;
+    rc = pool_alloc(&scratch, total, st);
+    if (rc != SS2D_OK)
+        return rc;
+    char *base = static_cast<char *>(scratch);
+    ss2d::BwdParams p{};
+    p.x = pr.x;
+    p.delta = pr.delta;
+    p.Bs = pr.Bs;
+    p.Cs = pr.Cs;
+    p.A_log = pr.A_log;
+    p.Dskip = pr.Dskip;
+    p.delta_bias = pr.delta_bias;
+    p.dy = gr.dy;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        float *q = bytes ? reinterpret_cast<float *>(base + off) : nullptr;
+        off += bytes;
+        return q;
+    };
+    p.hfwd = take(hs_bytes);
+    p.hadj = take(hs_bytes);
+    p.dtf = take(ds_bytes);
+    p.dta = take(ds_bytes);
+    p.du = pr.K > 1 ? take(du_bytes) : gr.dx;
+    p.bc_part = take(bc_bytes);
+    p.prm_part = take(pr_bytes);
+    p.ddelta = gr.ddelta;
+    p.B = pr.B;
+    p.D = pr.D;
+    p.H = pr.H;
+    p.W = pr.W;
+    p.L = (int)L;
+    p.N = pr.N;
+    p.K = pr.K;
+    p.two_d = pr.two_d;
+    p.NC = sh.NC;
+    p.G = sh.G;
+    p.CPB = sh.CPB;
+    p.CGN = sh.CGN;
+    p.flip1 = pr.K > 1 ? 1 : 0;
+    e = ss2d::launch_backward(p, pr.dtype, st);
+    if (e == cudaSuccess && pr.K > 1)
+        e = ss2d::launch_merge(p.du, gr.dx, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d, 1, st);
+    if (e == cudaSuccess)
+        e = ss2d::launch_backward_reduce(p, gr.dBs, gr.dCs, gr.dA_log, gr.dDskip,
+                                         gr.ddelta_bias, st);
+    const cudaError_t ef = cudaFreeAsync(scratch, st);
+    if (e != cudaSuccess) {
+        set_error("kernel launch", e);
+        return SS2D_ERR_CUDA;
+    }
+    if (ef != cudaSuccess) {
+        set_error("cudaFreeAsync", ef);
+        return SS2D_ERR_CUDA;
+    }
+    return SS2D_OK;
+}
+
 }  // namespace
 
 namespace ss2d {
@@ -386,6 +513,26 @@ int selective_scan_fwd_gated(const void *u, const void *delta, const float *A_lo
 {
     Problem pr{u, delta, Bs, Cs, A_log, Dskip, delta_bias, y, B, D, 1, L, N, K, dtype, 0, z};
     return forward(pr, stream, -1, false, true);
+}
+
+int ss2d_backward(const void *x, const void *delta, const float *A_log, const void *Bs,
+                  const void *Cs, const float *Dskip, const float *delta_bias, const float *dy,
+                  float *dx, float *ddelta, float *dA_log, float *dBs, float *dCs,
+                  float *dDskip, float *ddelta_bias, int B, int D, int H, int W, int N, int K,
+                  int dtype, void *stream)
+{
+    Problem pr{x, delta, Bs, Cs, A_log, Dskip, delta_bias, dx, B, D, H, W, N, K, dtype, 1};
+    return backward(pr, Grads{dy, dx, ddelta, dA_log, dBs, dCs, dDskip, ddelta_bias}, stream);
+}
+
+int selective_scan_bwd(const void *u, const void *delta, const float *A_log, const void *Bs,
+                       const void *Cs, const float *Dskip, const float *delta_bias,
+                       const float *dy, float *du, float *ddelta, float *dA_log, float *dBs,
+                       float *dCs, float *dDskip, float *ddelta_bias, int B, int D, int L, int N,
+                       int K, int dtype, void *stream)
+{
+    Problem pr{u, delta, Bs, Cs, A_log, Dskip, delta_bias, du, B, D, 1, L, N, K, dtype, 0};
+    return backward(pr, Grads{dy, du, ddelta, dA_log, dBs, dCs, dDskip, ddelta_bias}, stream);
 }
 
 int ss2d_scan_directions(const void *x, const void *delta, const float *A_log,

@@ -77,6 +77,21 @@ cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W
                          int zt = 0);
 size_t merge_smem_bytes(int H, int W, int K, int two_d);
 
+// Backward pass (ss2d_backward.cu): chunks of 16 steps, NC per sequence; G
+// groups of 32 channels; CPB chunks per CTA in CGN groups.
+struct BwdParams;
+struct BwdShape {
+    int NC, G, CPB, CGN;
+};
+BwdShape backward_shape(int B, int D, int L, int K);
+// local pass, both carries and the final pass (the caller has filled every
+// field of p, scratch included)
+cudaError_t launch_backward(const BwdParams &p, int dtype, cudaStream_t st);
+// dBs, dCs from the channel-group partials; dA_log, dDskip, ddelta_bias from
+// the per-chunk-group partials
+cudaError_t launch_backward_reduce(const BwdParams &p, float *dBs, float *dCs, float *dA_log,
+                                   float *dDskip, float *ddelta_bias, cudaStream_t st);
+
 // Text that ss2d_last_error() returns on the calling thread.
 void record_error(const char *what, cudaError_t e);
 void record_message(const char *text);

@@ -174,6 +174,17 @@ def make_gate(cfg: Config | str, seed: int = 0) -> np.ndarray:
     return _normal(rng, xshape, cfg.dtype)
 
 
+def make_cotangent(cfg: Config | str, seed: int = 0) -> np.ndarray:
+    """The cotangent dy of a backward call: N(0, 1) float32 in the layout of
+    y (a stream of its own, so the other inputs of the same seed are
+    unchanged)."""
+    if isinstance(cfg, str):
+        cfg = CONFIGS[cfg]
+    rng = np.random.default_rng([seed, 0xd1])
+    xshape = (cfg.B, cfg.D, cfg.H, cfg.W) if cfg.kind == "2d" else (cfg.B, cfg.D, cfg.L)
+    return rng.standard_normal(size=xshape, dtype=np.float32)
+
+
 def gate_as_f64(z: np.ndarray, cfg: Config) -> np.ndarray:
     """The exact values a gated call sees, widened to float64."""
     return (bf16_bits_to_f32(z) if cfg.dtype == BF16 else z).astype(np.float64)
@@ -195,3 +206,11 @@ def channel_subproblem(inp: Inputs, b: int, d: int) -> Inputs:
                   np.ascontiguousarray(inp.A_log[rows]),
                   np.ascontiguousarray(inp.Dskip[rows]),
                   np.ascontiguousarray(inp.delta_bias[rows]))
+
+
+def batch_subproblem(inp: Inputs, b: int) -> Inputs:
+    """Batch element b of a workload as a B=1 workload of its own (pure
+    slicing; every channel kept)."""
+    sub = inp.cfg.with_(name=f"{inp.cfg.name}[b={b}]", B=1)
+    return Inputs(sub, *[np.ascontiguousarray(getattr(inp, n)[b:b + 1]) for n in Inputs.STREAMED],
+                  inp.A_log, inp.Dskip, inp.delta_bias)

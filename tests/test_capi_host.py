@@ -129,3 +129,43 @@ def test_plans_for_the_workloads(lib):
     assert binding.ss2d_plan(True, t.B, t.D, t.H, t.W, t.N, t.K)["num_chunks"] > 1
     b = wl.CONFIGS["vmamba_b_stage3"]
     assert binding.ss2d_plan(True, b.B, b.D, b.H, b.W, b.N, b.K)["num_chunks"] == 1
+
+
+def _bwd_call(lib, ptr, B=1, D=1, H=2, W=2, N=4, K=4, dtype=0, two_d=True, nulls=()):
+    args = [ptr] * 15   # seven inputs, dy, seven gradients
+    for i in nulls:
+        args[i] = None
+    if two_d:
+        return lib.ss2d_backward(*args, B, D, H, W, N, K, dtype, None)
+    return lib.selective_scan_bwd(*args, B, D, H * W, N, K, dtype, None)
+
+
+def test_backward_argument_errors_are_reported_without_cuda(lib):
+    buf = (ctypes.c_float * 64)()
+    addr = ctypes.addressof(buf)
+    aligned = ctypes.c_void_p(addr + (-addr) % 16)
+    assert _bwd_call(lib, aligned, B=-1) == -2
+    assert _bwd_call(lib, aligned, dtype=9) == -3
+    assert _bwd_call(lib, aligned, K=3) == -4
+    assert _bwd_call(lib, aligned, K=4, two_d=False) == -4
+    assert _bwd_call(lib, aligned, N=17) == -5
+    for i in (0, 7, 8, 14):   # x, dy, dx, ddelta_bias
+        assert _bwd_call(lib, aligned, nulls=(i,)) == -1
+    assert _bwd_call(lib, ctypes.c_void_p(aligned.value + 4)) == -6
+
+
+def test_backward_binding_validates_tensors(lib):
+    import torch
+    x = torch.zeros(1, 2, 3, 3)
+    delta = torch.zeros(1, 4, 2, 9)
+    Bs = torch.zeros(1, 4, 4, 9)
+    A_log = torch.zeros(8, 4)
+    Dk = torch.zeros(8)
+    with pytest.raises(ValueError, match="dy"):
+        binding.ss2d_backward(x, delta, A_log, Bs, Bs, Dk, Dk, torch.zeros(1, 2, 3, 4))
+    with pytest.raises(ValueError, match="dy"):
+        binding.ss2d_backward(x, delta, A_log, Bs, Bs, Dk, Dk, x.double())
+    with pytest.raises(ValueError, match="device tensors only"):
+        binding.ss2d_backward(x, delta, A_log, Bs, Bs, Dk, Dk, x.clone())
+    with pytest.raises(ValueError, match="inconsistent"):
+        binding.selective_scan_bwd(x[:, :, 0], delta, A_log, Bs, Bs, Dk, Dk, x[:, :, 0].clone())
