@@ -401,6 +401,95 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def run_backward(args, rank, world, local_rank):
+    """The backward pass (ss2d_backward / selective_scan_bwd) of the workload:
+    one step = the gradients of every input for one seeded cotangent, inputs
+    resident in HBM, L2 flushed before every timed step.  Returns the JSON
+    line (rank 0) with the exp-unit roofline of the whole call."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from selective_scan_ss2d_b200 import binding
+    from selective_scan_ss2d_b200 import workloads as wl
+
+    cfg = workload_config(args.config, args.dtype)
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    binding.lib()
+    inp, t = build_arrays(cfg, seed=rank, device=dev)
+    dy = torch.from_numpy(wl.make_cotangent(cfg, seed=rank)).to(dev)
+    fn = binding.ss2d_backward if cfg.kind == "2d" else binding.selective_scan_bwd
+    stream = torch.cuda.current_stream(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
+    flush = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        return fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"],
+                  dy, stream=stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    gpu_id = str(getattr(props, "uuid", local_rank))
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.2)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
+    value = whole_job_rate(cfg.updates, args.steps, world, total_ms)
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    step_s = total_ms / args.steps / 1e3
+    mufu_peak = NUM_SMS * MUFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e9
+    bkdl = cfg.B * cfg.K * cfg.D * cfg.L
+    exps = 2 * cfg.updates + 2 * bkdl            # recompute + reverse walk; softplus + sigmoid
+    exps_done = (4 * cfg.updates + 4 * bkdl) if cfg.L > 16 else exps
+    in_b = cfg.in_bytes_per_elem
+    nbc = cfg.B * cfg.K * cfg.N * cfg.L
+    grad_bytes = (cfg.B * cfg.D * cfg.L * (in_b + 4 + 4) + bkdl * (in_b + 4) + nbc * 2 * (in_b + 4))
+    return {
+        "metric": "SS2D backward: state updates/s (B·K·D·L·N) of the gradient pass",
+        "value": value, "unit": "updates/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) inputs and cotangent)",
+        "config": {"workload": cfg.name, "B": cfg.B, "D": cfg.D, "H": cfg.H, "W": cfg.W,
+                   "L": cfg.L, "K": cfg.K, "N": cfg.N, "input_dtype": cfg.dtype,
+                   "pass": "backward (all seven gradients)",
+                   "l2": "flushed before every timed step (2x L2 write, outside events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "alu", "achieved": exps / step_s / 1e9, "peak": mufu_peak,
+                     "unit": "Gexp2/s", "frac": exps / step_s / 1e9 / mufu_peak,
+                     "work": "2 exp2 per state update (recompute, reverse walk) + 2 per "
+                             "(b,k,d,l) (softplus, sigmoid); this implementation issues "
+                             f"{exps_done / exps:.2f}x that (the chunk-local pass)",
+                     "peak_source": f"MUFU exp2 x {peaks['sm_max_mhz']:.0f} MHz ({peaks['source']})"},
+        "roofline_hbm": {"bound": "hbm", "achieved": grad_bytes / step_s / 1e9,
+                         "peak": peaks["hbm_gbs"],
+                         "frac": grad_bytes / step_s / 1e9 / peaks["hbm_gbs"],
+                         "unit": "GB/s", "bytes": "inputs and dy read once, gradients written once"},
+        "clocks": clocks,
+    }
+
+
 def run_e2e(args, cfg_name, local_rank, world=1):
     """Same metric through the C ABI with host (pinned) buffers: every step
     copies the inputs in, computes, and copies y out, inside the call.  Every
@@ -498,6 +587,9 @@ def main():
     ap.add_argument("--gate", action="store_true",
                     help="time the gated entry point (y * SiLU(z)); device buffers only, "
                          "so no e2e leg")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (gradients of every input) instead; "
+                         "device buffers only, no e2e or CPU leg")
     ap.add_argument("--report", action="store_true",
                     help="one JSON line per workload (device-resident only)")
     args = ap.parse_args()
@@ -515,6 +607,16 @@ def main():
         return 0
 
     init_distributed(world, local_rank)
+
+    if args.backward:
+        line = run_backward(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     if args.report:
         from selective_scan_ss2d_b200 import workloads as wl

@@ -23,8 +23,9 @@
 //      chunk and, over the reversed order, the adjoint G[c] = a_{e+1} g_{e+1}
 //      entering every chunk from its end: G[c-1] = exp(A sum_c dt) G[c] + Q[c].
 //   3. bwd_final_kernel: per chunk, h recomputed from its entry state (the
-//      16 states of 16 steps of every lane parked in shared memory), then the
-//      reverse walk from G[c] writes ddelta and du, reduces dB and dC over
+//      16 states of 8 steps of every lane parked in shared memory at a time:
+//      the chunk is walked back in two halves), then the reverse walk from
+//      G[c] writes ddelta and du, reduces dB and dC over
 //      the warp's channels (one reduce-scatter of 32 values per step) into a
 //      per-channel-group partial, and accumulates the parameter gradients.
 //   4. merge2_kernel (K > 1) sums du of the directions into dx; two fixed-order
@@ -40,11 +41,13 @@ namespace ss2d {
 constexpr float kLn2 = 0.6931471805599453f;
 
 // shared memory of both kernels (floats): B and C of the chunk [t][n], and the
-// lanes' staged dt, u, dy and sigmoid(delta + bias) [t][lane]
+// lanes' staged (dt, u, dy, sigmoid(delta + bias)) as float4 [t][lane]
 constexpr int kBwdStage = 2 * kT * kNP + 4 * kT * kBwdLanes;
-// the final kernel adds the recomputed states [t][n][lane] and the reduced
-// dB | dC values [t][lane]
-constexpr int kBwdStates = kT * kNP * kBwdLanes + kT * kBwdLanes;
+// the final kernel adds the recomputed states of half a chunk, float4
+// [t][lane][4] with the float4 index XOR-swizzled by (lane >> 1) & 3 (no bank
+// conflicts for the lanes' 16-byte accesses)
+constexpr int kHalf = kT / 2;
+constexpr int kBwdStates = kHalf * kNP * kBwdLanes;
 constexpr size_t kBwdFinalSmem = sizeof(float) * (kBwdStage + kBwdStates);
 
 struct BwdLane {
@@ -69,59 +72,84 @@ __device__ __forceinline__ BwdLane bwd_lane(const BwdParams &p)
     return r;
 }
 
-// B and C of steps s .. s+nt-1 into sB, sC [t][n] (zeros past N and nt)
+// The raw inputs of one chunk (steps s .. s+nt-1) that a lane stages: its
+// channel's delta, x and dy, and its share of the chunk's B and C (state
+// n = lane >> 1, 8 steps), loaded one chunk ahead into registers and turned
+// into the shared-memory tiles after the current chunk's work.
 template <typename Tin>
-__device__ __forceinline__ void bwd_stage_bc(const BwdParams &p, const BwdLane &q, int s, int nt,
-                                             float *sB, float *sC)
-{
-    const int lane = threadIdx.x;
-    const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
-    const bool nok = n < p.N;
-    const size_t row = (((size_t)q.b * p.K + q.k) * p.N + (nok ? n : 0)) * p.L + s;
-    const Tin *Bp = static_cast<const Tin *>(p.Bs) + row;
-    const Tin *Cp = static_cast<const Tin *>(p.Cs) + row;
-#pragma unroll
-    for (int i = 0; i < kT / 2; ++i) {
-        const int t = t0 + i;
-        const bool ok = nok && t < nt;
-        sB[t * kNP + n] = ok ? to_f32(Bp[t]) : 0.f;
-        sC[t * kNP + n] = ok ? to_f32(Cp[t]) : 0.f;
-    }
-}
+struct BwdRaw {
+    using RawT = std::conditional_t<sizeof(Tin) == 2, unsigned short, float>;
+    RawT dl[kT], x[kT], b[kT / 2], c[kT / 2];
+    float gy[kT];
+    int nt;
 
-// this lane's dt, u, dy and sigmoid(delta + bias) of steps s .. s+nt-1 (zeros
-// past nt: dt = 0 makes a padded step the identity)
-template <typename Tin>
-__device__ __forceinline__ void bwd_stage_lane(const BwdParams &p, const BwdLane &q, int s, int nt,
-                                               float bias, float *sdt, float *su, float *sgy,
-                                               float *ssg)
-{
-    const int lane = threadIdx.x;
-    const Tin *dl = static_cast<const Tin *>(p.delta) + q.bkd * p.L + s;
-    const size_t xrow = ((size_t)q.b * p.D + q.d) * p.L;
-    const Tin *xp = static_cast<const Tin *>(p.x) + xrow;
-    const float *gp = p.dy + xrow;
-    PixWalk w;
-    w.init(p.two_d, q.k, s, p.H, p.W, p.L);
+    __device__ __forceinline__ static float f32(RawT v)
+    {
+        if constexpr (sizeof(Tin) == 2)
+            return half_bits_to_f32<Tin>(v);
+        else
+            return v;
+    }
+
+    __device__ __forceinline__ void fetch(const BwdParams &p, const BwdLane &q, int s)
+    {
+        nt = min(kT, p.L - s);
+        const int lane = threadIdx.x;
+        const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
+        const bool nok = n < p.N;
+        const size_t row = (((size_t)q.b * p.K + q.k) * p.N + (nok ? n : 0)) * p.L + s + t0;
+        const RawT *Bp = static_cast<const RawT *>(p.Bs) + row;
+        const RawT *Cp = static_cast<const RawT *>(p.Cs) + row;
 #pragma unroll
-    for (int t = 0; t < kT; ++t) {
-        float dt = 0.f, u = 0.f, gy = 0.f, sg = 0.f;
-        if (t < nt && q.active) {   // idle lanes add nothing to the dB, dC sums
-            const float z = to_f32(dl[t]) + bias;
-            dt = softplus_f(z);
-            // sigmoid(z) = 1 / (1 + e^-z); e^-z = inf gives 0
-            sg = __fdividef(1.f, 1.f + mufu_ex2(-z * kLog2e));
-            u = to_f32(xp[w.p]);
-            gy = __ldg(gp + w.p);
+        for (int i = 0; i < kT / 2; ++i) {
+            const bool ok = nok && t0 + i < nt;
+            b[i] = ok ? __ldg(Bp + i) : RawT(0);
+            c[i] = ok ? __ldg(Cp + i) : RawT(0);
+        }
+        const RawT *dp = static_cast<const RawT *>(p.delta) + q.bkd * p.L + s;
+        const size_t xrow = ((size_t)q.b * p.D + q.d) * p.L;
+        const RawT *xp = static_cast<const RawT *>(p.x) + xrow;
+        const float *gp = p.dy + xrow;
+        PixWalk w;
+        w.init(p.two_d, q.k, s, p.H, p.W, p.L);
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+            const bool ok = t < nt && q.active;   // idle lanes add nothing to dB, dC
+            dl[t] = ok ? __ldg(dp + t) : RawT(0);
+            x[t] = ok ? __ldg(xp + w.p) : RawT(0);
+            gy[t] = ok ? __ldg(gp + w.p) : 0.f;
             if (t + 1 < nt)
                 w.next(p.H, p.W);
         }
-        sdt[t * kBwdLanes + lane] = dt;
-        su[t * kBwdLanes + lane] = u;
-        sgy[t * kBwdLanes + lane] = gy;
-        ssg[t * kBwdLanes + lane] = sg;
     }
-}
+
+    // sB, sC [t][n] and st4 [t][lane] = (dt, u, dy, sigmoid(z)), z = delta + bias;
+    // steps past nt (and idle lanes) stage zeros: dt = 0 makes a step the identity
+    __device__ __forceinline__ void commit(float *sB, float *sC, float4 *st4, float bias,
+                                           bool active) const
+    {
+        const int lane = threadIdx.x;
+        const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
+#pragma unroll
+        for (int i = 0; i < kT / 2; ++i) {
+            sB[(t0 + i) * kNP + n] = f32(b[i]);
+            sC[(t0 + i) * kNP + n] = f32(c[i]);
+        }
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < nt && active) {
+                const float z = f32(dl[t]) + bias;
+                v.x = softplus_f(z);
+                v.y = f32(x[t]);
+                v.z = gy[t];
+                // sigmoid(z) = 1 / (1 + e^-z); e^-z = inf gives 0
+                v.w = __fdividef(1.f, 1.f + mufu_ex2(-z * kLog2e));
+            }
+            st4[t * kBwdLanes + lane] = v;
+        }
+    }
+};
 
 __device__ __forceinline__ void load16(float *v, const float *src)
 {
@@ -147,9 +175,9 @@ __device__ __forceinline__ void store16(float *dst, const float *v)
 template <typename Tin>
 __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
 {
-    __shared__ float sm[kBwdStage];
-    float *sB = sm, *sC = sB + kT * kNP, *sdt = sC + kT * kNP;
-    float *su = sdt + kT * kBwdLanes, *sgy = su + kT * kBwdLanes, *ssg = sgy + kT * kBwdLanes;
+    __shared__ float4 sm4[kBwdStage / 4];
+    float *sB = reinterpret_cast<float *>(sm4), *sC = sB + kT * kNP;
+    float4 *st4 = sm4 + 2 * kT * kNP / 4;
     const int lane = threadIdx.x;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
@@ -160,16 +188,18 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
     const float bias = __ldg(p.delta_bias + kd);
     const int nc1 = p.NC - 1;
     const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
+    BwdRaw<Tin> raw;
+    raw.fetch(p, q, c0 * kT);
     for (int c = c0; c < c1; ++c) {
-        const int s = c * kT, nt = min(kT, p.L - s);
         __syncwarp();
-        bwd_stage_bc<Tin>(p, q, s, nt, sB, sC);
-        bwd_stage_lane<Tin>(p, q, s, nt, bias, sdt, su, sgy, ssg);
+        raw.commit(sB, sC, st4, bias, q.active);
         __syncwarp();
+        if (c + 1 < c1)
+            raw.fetch(p, q, (c + 1) * kT);   // in flight during this chunk's work
         float dts = 0.f;
 #pragma unroll
         for (int t = 0; t < kT; ++t)
-            dts += sdt[t * kBwdLanes + lane];
+            dts += st4[t * kBwdLanes + lane].x;
         if (c < nc1) {
             float h[kNP];
 #pragma unroll
@@ -177,11 +207,11 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
                 h[n] = 0.f;
 #pragma unroll
             for (int t = 0; t < kT; ++t) {
-                const float dt = sdt[t * kBwdLanes + lane];
-                const float dtu = dt * su[t * kBwdLanes + lane];
+                const float4 v = st4[t * kBwdLanes + lane];
+                const float dtu = v.x * v.y;
 #pragma unroll
                 for (int n = 0; n < kNP; ++n)
-                    h[n] = fmaf(mufu_ex2(dt * A2[n]), h[n], dtu * sB[t * kNP + n]);
+                    h[n] = fmaf(mufu_ex2(v.x * A2[n]), h[n], dtu * sB[t * kNP + n]);
             }
             if (q.active) {
                 store16(p.hfwd + (q.bkd * nc1 + c) * kNP, h);
@@ -195,11 +225,10 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
                 g[n] = 0.f;
 #pragma unroll
             for (int t = kT - 1; t >= 0; --t) {
-                const float dt = sdt[t * kBwdLanes + lane];
-                const float gy = sgy[t * kBwdLanes + lane];
+                const float4 v = st4[t * kBwdLanes + lane];
 #pragma unroll
                 for (int n = 0; n < kNP; ++n)
-                    g[n] = mufu_ex2(dt * A2[n]) * fmaf(gy, sC[t * kNP + n], g[n]);
+                    g[n] = mufu_ex2(v.x * A2[n]) * fmaf(v.z, sC[t * kNP + n], g[n]);
             }
             if (q.active) {
                 const int r = nc1 - c;   // reversed chunk order
@@ -241,12 +270,11 @@ template <typename Tin>
 __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
 {
     extern __shared__ float4 smem_bwd4[];
-    float *sm = reinterpret_cast<float *>(smem_bwd4);
-    float *sB = sm, *sC = sB + kT * kNP, *sdt = sC + kT * kNP;
-    float *su = sdt + kT * kBwdLanes, *sgy = su + kT * kBwdLanes, *ssg = sgy + kT * kBwdLanes;
-    float *hs = ssg + kT * kBwdLanes;   // [t][n][lane]
-    float *sout = hs + kT * kNP * kBwdLanes;   // [t][lane]
+    float *sB = reinterpret_cast<float *>(smem_bwd4), *sC = sB + kT * kNP;
+    float4 *st4 = smem_bwd4 + 2 * kT * kNP / 4;
+    float4 *hs4 = st4 + kT * kBwdLanes;   // [t][lane][4 float4], half a chunk
     const int lane = threadIdx.x;
+    const int swz = (lane >> 1) & 3;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
     float A2[kNP];
@@ -268,76 +296,106 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
         dA[n] = 0.f;
     float dD = 0.f, db = 0.f;
     const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
+    BwdRaw<Tin> raw;
+    raw.fetch(p, q, c0 * kT);
     for (int c = c0; c < c1; ++c) {
         const int s = c * kT, nt = min(kT, L - s);
         __syncwarp();
-        bwd_stage_bc<Tin>(p, q, s, nt, sB, sC);
-        bwd_stage_lane<Tin>(p, q, s, nt, bias, sdt, su, sgy, ssg);
+        raw.commit(sB, sC, st4, bias, q.active);
         __syncwarp();
-        // states of the chunk, from its entry state
-        {
-            float h[kNP];
+        if (c + 1 < c1)
+            raw.fetch(p, q, (c + 1) * kT);   // in flight during this chunk's work
+        // The chunk in two halves of 8 steps, so that only half of its states
+        // are parked at a time: the first recompute runs the whole chunk from
+        // the entry state and parks steps 8..15 for the walk back over them;
+        // the second recomputes steps 0..7 from the entry state again.
+        auto entry = [&](float *h) {
             if (c > 0)
                 load16(h, p.hfwd + (q.bkd * nc1 + (c - 1)) * kNP);
             else
 #pragma unroll
                 for (int n = 0; n < kNP; ++n)
                     h[n] = 0.f;
+        };
+        auto recompute = [&](float *h, int t1, int park0) {
 #pragma unroll 1
-            for (int t = 0; t < kT; ++t) {
-                const float dt = sdt[t * kBwdLanes + lane];
-                const float dtu = dt * su[t * kBwdLanes + lane];
+            for (int t = 0; t < t1; ++t) {
+                const float4 v = st4[t * kBwdLanes + lane];
+                const float dtu = v.x * v.y;
 #pragma unroll
-                for (int n = 0; n < kNP; ++n) {
-                    h[n] = fmaf(mufu_ex2(dt * A2[n]), h[n], dtu * sB[t * kNP + n]);
-                    hs[(t * kNP + n) * kBwdLanes + lane] = h[n];
+                for (int n = 0; n < kNP; ++n)
+                    h[n] = fmaf(mufu_ex2(v.x * A2[n]), h[n], dtu * sB[t * kNP + n]);
+                if (t >= park0) {
+                    float4 *row = hs4 + ((t - park0) * kBwdLanes + lane) * 4;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        row[j ^ swz] = make_float4(h[4 * j], h[4 * j + 1], h[4 * j + 2],
+                                                   h[4 * j + 3]);
                 }
             }
-        }
-        // reverse walk from the adjoint entering at the chunk end
+        };
         float g[kNP];
+        auto walk_back = [&](int t_hi, int base) {
+#pragma unroll 2
+            for (int t = t_hi; t >= base; --t) {
+                const float4 v4 = st4[t * kBwdLanes + lane];
+                const float dt = v4.x, u = v4.y, gy = v4.z;
+                const float dtu = dt * u;
+                const float4 *row = hs4 + ((t - base) * kBwdLanes + lane) * 4;
+                float v[2 * kNP];
+                float s1 = 0.f, s2 = 0.f;   // sum g A2 (a h_prev), sum g B
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 h4 = row[j ^ swz];
+                    const float hj[4] = {h4.x, h4.y, h4.z, h4.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = 4 * j + i;
+                        const float Bv = sB[t * kNP + n];
+                        const float hv = hj[i];
+                        g[n] = fmaf(gy, sC[t * kNP + n], g[n]);
+                        const float hp = fmaf(-dtu, Bv, hv);   // a_t h_{t-1}
+                        const float gdt = g[n] * dt;
+                        v[n] = g[n] * dtu;
+                        v[kNP + n] = gy * hv;
+                        s2 = fmaf(g[n], Bv, s2);
+                        s1 = fmaf(g[n] * A2[n], hp, s1);
+                        dA[n] = fmaf(gdt, hp, dA[n]);
+                        g[n] *= mufu_ex2(dt * A2[n]);
+                    }
+                }
+                const float red = reduce_scatter32(v);
+                if (bc_ok && t < nt)
+                    bcrow[s + t] = red;
+                if (q.active && t < nt) {
+                    const int l = s + t;
+                    const float ddl = fmaf(kLn2, s1, u * s2) * v4.w;
+                    dD = fmaf(gy, u, dD);
+                    db += ddl;
+                    ddrow[l] = ddl;
+                    durow[flip ? L - 1 - l : l] = fmaf(Dk, gy, dt * s2);
+                }
+            }
+        };
+        // the adjoint entering at the chunk end
         if (c < nc1)
             load16(g, p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
         else
 #pragma unroll
             for (int n = 0; n < kNP; ++n)
                 g[n] = 0.f;
-#pragma unroll 1
-        for (int t = kT - 1; t >= 0; --t) {
-            const float dt = sdt[t * kBwdLanes + lane];
-            const float u = su[t * kBwdLanes + lane];
-            const float gy = sgy[t * kBwdLanes + lane];
-            const float dtu = dt * u;
-            float v[2 * kNP];
-            float s1 = 0.f, s2 = 0.f;   // sum g A2 (a h_prev), sum g B
-#pragma unroll
-            for (int n = 0; n < kNP; ++n) {
-                const float Bv = sB[t * kNP + n];
-                const float hv = hs[(t * kNP + n) * kBwdLanes + lane];
-                g[n] = fmaf(gy, sC[t * kNP + n], g[n]);
-                const float hp = fmaf(-dtu, Bv, hv);   // a_t h_{t-1}
-                const float gdt = g[n] * dt;
-                v[n] = gdt * u;
-                v[kNP + n] = gy * hv;
-                s2 = fmaf(g[n], Bv, s2);
-                s1 = fmaf(g[n] * A2[n], hp, s1);
-                dA[n] = fmaf(gdt, hp, dA[n]);
-                g[n] *= mufu_ex2(dt * A2[n]);
-            }
-            sout[t * kBwdLanes + lane] = reduce_scatter32(v);
-            if (q.active && t < nt) {
-                const int l = s + t;
-                const float ddl = fmaf(kLn2, s1, u * s2) * ssg[t * kBwdLanes + lane];
-                dD = fmaf(gy, u, dD);
-                db += ddl;
-                ddrow[l] = ddl;
-                durow[flip ? L - 1 - l : l] = fmaf(Dk, gy, dt * s2);
-            }
+        {
+            float h[kNP];
+            entry(h);
+            recompute(h, kT, kHalf);
         }
-        if (bc_ok) {
-            for (int t = 0; t < nt; ++t)
-                bcrow[s + t] = sout[t * kBwdLanes + lane];
+        walk_back(kT - 1, kHalf);
+        {
+            float h[kNP];
+            entry(h);
+            recompute(h, kHalf, 0);
         }
+        walk_back(kHalf - 1, 0);
     }
     if (q.active) {
         float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * kPrm;
