@@ -82,7 +82,8 @@ typedef enum {
     SS2D_ERR_SHAPE = -2,  /* a size is negative, or a product overflows     */
     SS2D_ERR_DTYPE = -3,  /* dtype is not one of ss2d_dtype                  */
     SS2D_ERR_K = -4,      /* K not in {1,2,4} (2D) or {1,2} (1D)             */
-    SS2D_ERR_N = -5,      /* N not in 1..16                                  */
+    SS2D_ERR_N = -5,      /* N not in 1..64 (forward) or 1..16 (backward and
+                             ss2d_forward_timed)                         */
     SS2D_ERR_ALIGN = -6,  /* a pointer is not 16-byte aligned                */
     SS2D_ERR_ALLOC = -7,  /* device memory for scratch or staging ran out    */
     SS2D_ERR_CUDA = -8,   /* a CUDA call failed; see ss2d_last_error()       */
@@ -101,8 +102,11 @@ typedef enum {
 
 /* SS2D forward: cross_scan -> selective scan of each direction -> cross_merge.
  * K = 4 is the SS2D of the pages; K = 2 (directions 0 and 1 only) and K = 1
- * (row-major only) are also accepted.  N in 1..16.  `stream` is a
- * cudaStream_t (NULL = the legacy default stream). */
+ * (row-major only) are also accepted.  N in 1..64: the states of a channel
+ * never interact, so more than 16 run as groups of 16 states one after the
+ * other, each adding its C.h terms to the output (the skip term once); the
+ * pages use N = 16 and mention d_state 8 ("VMamba架构解析", section 5).
+ * `stream` is a cudaStream_t (NULL = the legacy default stream). */
 int ss2d_forward(const void *x, const void *delta, const float *A_log,
                  const void *Bs, const void *Cs, const float *Dskip,
                  const float *delta_bias, float *y,
@@ -153,6 +157,24 @@ int selective_scan_fwd_gated(const void *u, const void *delta, const float *A_lo
                              const float *delta_bias, const void *z, float *y,
                              int B, int D, int L, int N, int K, int dtype,
                              void *stream);
+
+/* As ss2d_forward_ex / selective_scan_fwd_ex, and also the final states:
+ * h_last (B,K,D,N) float32 receives, for every direction k and channel d,
+ * the state h after the last step of direction k's scan order (the state a
+ * scan continued past the end of the sequence would start from; the Vim
+ * summary's section 4.4 keeps states on chip and writes only outputs, so
+ * this is the one state a caller can get back).  Device pointers only
+ * (host pointers: SS2D_ERR_PTR); h_last null: SS2D_ERR_NULL. */
+int ss2d_forward_final_state(const void *x, const void *delta, const float *A_log,
+                             const void *Bs, const void *Cs, const float *Dskip,
+                             const float *delta_bias, float *y, float *h_last,
+                             int B, int D, int H, int W, int N, int K, int dtype,
+                             void *stream, int variant);
+int selective_scan_fwd_final_state(const void *u, const void *delta, const float *A_log,
+                                   const void *Bs, const void *Cs, const float *Dskip,
+                                   const float *delta_bias, float *y, float *h_last,
+                                   int B, int D, int L, int N, int K, int dtype,
+                                   void *stream, int variant);
 
 /* Backward of ss2d_forward / selective_scan_fwd: the gradients of
  * sum(dy * y) with respect to every input ("Vision Mamba ..." summary,

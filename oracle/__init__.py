@@ -17,7 +17,8 @@ Two independent write-ups of the same definition live here:
 What they compute and which page passage each step follows is stated in the
 header of ``ss2d_oracle.c``.  ``ss2d_backward_np.py`` (:func:`ss2d_backward`,
 :func:`selective_scan_bwd`) is the float64 reverse-mode gradient of the same
-forward definition, pinned against finite differences of the C forward.  Every part is pinned by ``tests/test_oracle_pins.py``
+forward definition, pinned against finite differences of the C forward;
+:func:`final_states` gives the state after each direction's last step.  Every part is pinned by ``tests/test_oracle_pins.py``
 against closed forms, a matrix-exponential discretisation, an O(L^2) brute
 force and exact index-map invariants; parity is pinned for every function
 (no function here is "parity unpinned").
@@ -32,6 +33,7 @@ import threading
 import numpy as np
 
 from .ss2d_backward_np import selective_scan_bwd, ss2d_backward  # noqa: F401
+from .ss2d_oracle_np import final_states  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ss2d_oracle.c")

@@ -107,3 +107,36 @@ def selective_scan_fwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, K=2,
     if z is not None:
         y = y * silu(z)
     return (y, yd) if return_dirs else y
+
+
+def final_states(x, delta, A_log, Bs, delta_bias, *, K, two_d=True):
+    """The state after the last step of every direction's scan, h_L
+    (B, K, D, N), float64: the recurrence of the forward (dt = softplus(delta
+    + bias), h = exp(dt A) h + dt B u from h = 0) run to the end of direction
+    k's scan order (the state a continued scan would start from)."""
+    x = np.asarray(x, dtype=np.float64)
+    Bb, D = x.shape[:2]
+    if two_d:
+        H, W = x.shape[2:]
+        L, orders = H * W, scan_orders_2d(H, W)
+    else:
+        L = x.shape[2]
+        orders = scan_orders_1d(L)
+    u_pix = x.reshape(Bb, D, L)
+    delta = np.asarray(delta, np.float64)
+    A_log = np.asarray(A_log, np.float64)
+    Bs = np.asarray(Bs, np.float64)
+    delta_bias = np.asarray(delta_bias, np.float64)
+    N = A_log.shape[1]
+    out = np.zeros((Bb, K, D, N))
+    for k in range(K):
+        rows = slice(k * D, (k + 1) * D)
+        A = -np.exp(A_log[rows])
+        dt = softplus(delta[:, k] + delta_bias[rows][None, :, None])
+        u = u_pix[:, :, orders[k]]
+        h = np.zeros((Bb, D, N))
+        for t in range(L):
+            h = np.exp(dt[:, :, t, None] * A[None]) * h + \
+                dt[:, :, t, None] * Bs[:, k][:, None, :, t] * u[:, :, t, None]
+        out[:, k] = h
+    return out

@@ -5,12 +5,12 @@ The computation lives in the CUDA library built from ``csrc/`` (C ABI in
 ``include/ss2d.h``); :mod:`.binding` marshals torch tensors into it.
 :mod:`.workloads` draws the seeded synthetic inputs.
 """
-from .binding import (SS2DError, selective_scan_bwd, selective_scan_fwd,
+from .binding import (SS2DError, forward_final_state, selective_scan_bwd, selective_scan_fwd,
                       selective_scan_fwd_gated, ss2d_backward, ss2d_forward, ss2d_forward_gated,
                       ss2d_forward_noalloc, ss2d_num_variants, ss2d_pick_variant,
                       ss2d_scan_directions, ss2d_status_string, ss2d_variant_name)
 
 __all__ = ["ss2d_forward", "ss2d_forward_gated", "ss2d_forward_noalloc", "selective_scan_fwd",
-           "selective_scan_fwd_gated", "ss2d_backward", "selective_scan_bwd", "ss2d_status_string",
+           "selective_scan_fwd_gated", "ss2d_backward", "forward_final_state", "selective_scan_bwd", "ss2d_status_string",
            "ss2d_num_variants", "ss2d_variant_name", "ss2d_pick_variant", "ss2d_scan_directions",
            "SS2DError"]

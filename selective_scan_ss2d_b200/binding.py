@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.selective_scan_fwd_gated.argtypes = gfwd + [i] * 6 + [vp]
             L.selective_scan_fwd_gated.restype = i
             L.ss2d_scan_directions.restype = i
+            L.ss2d_forward_final_state.argtypes = fwd + [fp] + [i] * 7 + [vp, i]
+            L.ss2d_forward_final_state.restype = i
+            L.selective_scan_fwd_final_state.argtypes = fwd + [fp] + [i] * 6 + [vp, i]
+            L.selective_scan_fwd_final_state.restype = i
             bwd = fwd[:7] + [fp] + [fp] * 7   # dy, then the seven gradients
             L.ss2d_backward.argtypes = bwd + [i] * 7 + [vp]
             L.ss2d_backward.restype = i
@@ -369,3 +373,32 @@ def selective_scan_bwd(u, delta, A_log, Bs, Cs, Dskip, delta_bias, dy, *, stream
     gradient with respect to u."""
     return _backward(lib().selective_scan_bwd, "selective_scan_bwd", u, delta, A_log, Bs, Cs,
                      Dskip, delta_bias, dy, (u.shape[2],), stream)
+
+
+def forward_final_state(x, delta, A_log, Bs, Cs, Dskip, delta_bias, *, stream=None,
+                        variant: int = -1):
+    """ss2d_forward (x 4-D) or selective_scan_fwd (x 3-D) that also returns
+    the final states: (y, h_last), h_last (B,K,D,N) float32 the state after
+    the last step of every direction's scan.  Device tensors only."""
+    two_d = x.dim() == 4
+    B, D = x.shape[0], x.shape[1]
+    K, N = delta.shape[1], Bs.shape[2]
+    L = x.shape[2] * x.shape[3] if two_d else x.shape[2]
+    if tuple(delta.shape) != (B, K, D, L) or tuple(Bs.shape) != (B, K, N, L) \
+            or tuple(Cs.shape) != (B, K, N, L) or tuple(A_log.shape) != (K * D, N) \
+            or tuple(Dskip.shape) != (K * D,) or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for forward_final_state")
+    y, dt, on_gpu = _prepare(x, delta, A_log, Bs, Cs, Dskip, delta_bias, None, tuple(x.shape))
+    if not on_gpu:
+        raise ValueError("forward_final_state takes device tensors only")
+    h_last = torch.empty((B, K, D, N), dtype=torch.float32, device=x.device)
+    st = _stream(True, x.device, stream)
+    args = [_ptr(x), _ptr(delta), _ptr(A_log), _ptr(Bs), _ptr(Cs), _ptr(Dskip), _ptr(delta_bias),
+            _ptr(y), _ptr(h_last)]
+    if two_d:
+        rc = lib().ss2d_forward_final_state(*args, B, D, x.shape[2], x.shape[3], N, K, dt, st,
+                                            int(variant))
+    else:
+        rc = lib().selective_scan_fwd_final_state(*args, B, D, L, N, K, dt, st, int(variant))
+    _check(rc)
+    return y, h_last

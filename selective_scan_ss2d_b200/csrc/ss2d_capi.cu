@@ -108,6 +108,7 @@ struct Problem {
     float *y;
     int B, D, H, W, N, K, dtype, two_d;
     const void *z = nullptr;   // output gate (gated calls)
+    float *hlast = nullptr;    // final states (final-state calls)
 };
 
 int validate(const Problem &pr)
@@ -118,7 +119,7 @@ int validate(const Problem &pr)
         return SS2D_ERR_DTYPE;
     if (pr.two_d ? !(pr.K == 1 || pr.K == 2 || pr.K == 4) : !(pr.K == 1 || pr.K == 2))
         return SS2D_ERR_K;
-    if (pr.N < 1 || pr.N > ss2d::kNP)
+    if (pr.N < 1 || pr.N > ss2d::kMaxN)
         return SS2D_ERR_N;
     const long long L = (long long)pr.H * pr.W;
     if (L > INT_MAX || pr.B > 65535 || (long long)pr.K * pr.D > INT_MAX)
@@ -164,6 +165,8 @@ ss2d::ScanParams make_params(const Problem &pr)
     p.N = pr.N;
     p.K = pr.K;
     p.two_d = pr.two_d;
+    p.hlast = pr.hlast;
+    p.NS = pr.N;
     return p;
 }
 
@@ -179,6 +182,8 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
                cudaEvent_t *ev = nullptr)
 {
+    if (ev && pr.N > ss2d::kNP)
+        return SS2D_ERR_N;   // per-launch timing covers one state group
     ss2d::ScanParams p = make_params(pr);
     const size_t in_esz = pr.dtype == SS2D_F32 ? 4 : 2;   // bytes per stored input value
     const long long L = p.L;
@@ -292,9 +297,9 @@ int run_host(const Problem &pr, cudaStream_t st, int variant)
 }
 
 int forward(const Problem &pr, void *stream, int variant, bool directions_only = false,
-            bool gated = false)
+            bool gated = false, bool final_state = false)
 {
-    if (gated && !pr.z)
+    if ((gated && !pr.z) || (final_state && !pr.hlast))
         return SS2D_ERR_NULL;
     int rc = validate(pr);
     if (rc != SS2D_OK)
@@ -315,7 +320,7 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
         return SS2D_ERR_CUDA;
     }
     const void *ptrs[] = {pr.x, pr.delta, pr.Bs, pr.Cs, pr.A_log, pr.Dskip, pr.delta_bias, pr.y,
-                          pr.z ? pr.z : pr.x};
+                          pr.z ? pr.z : pr.x, pr.hlast ? pr.hlast : pr.x};
     const PtrKind kind = pointer_kind(ptrs[0], dev);
     if (kind == kBadPtr)
         return SS2D_ERR_PTR;
@@ -323,7 +328,7 @@ int forward(const Problem &pr, void *stream, int variant, bool directions_only =
         if (pointer_kind(q, dev) != kind)
             return SS2D_ERR_PTR;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (directions_only || gated)
+    if (directions_only || gated || final_state)
         return kind == kDevicePtr ? run_device(pr, st, variant, directions_only) : SS2D_ERR_PTR;
     return kind == kDevicePtr ? run_device(pr, st, variant, false) : run_host(pr, st, variant);
 }
@@ -341,6 +346,8 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     int rc = validate(pr);
     if (rc != SS2D_OK)
         return rc;
+    if (pr.N > ss2d::kNP)
+        return SS2D_ERR_N;   // the backward keeps all states of a channel in one lane
     if (pr.K * (long long)pr.D == 0)
         return SS2D_OK;
     // an empty batch or sequence reads nothing and writes only the parameter
@@ -515,6 +522,27 @@ int selective_scan_fwd_gated(const void *u, const void *delta, const float *A_lo
     return forward(pr, stream, -1, false, true);
 }
 
+int ss2d_forward_final_state(const void *x, const void *delta, const float *A_log,
+                             const void *Bs, const void *Cs, const float *Dskip,
+                             const float *delta_bias, float *y, float *h_last, int B, int D,
+                             int H, int W, int N, int K, int dtype, void *stream, int variant)
+{
+    Problem pr{x, delta, Bs, Cs, A_log, Dskip, delta_bias, y, B, D, H, W, N, K, dtype, 1};
+    pr.hlast = h_last;
+    return forward(pr, stream, variant, false, false, true);
+}
+
+int selective_scan_fwd_final_state(const void *u, const void *delta, const float *A_log,
+                                   const void *Bs, const void *Cs, const float *Dskip,
+                                   const float *delta_bias, float *y, float *h_last, int B,
+                                   int D, int L, int N, int K, int dtype, void *stream,
+                                   int variant)
+{
+    Problem pr{u, delta, Bs, Cs, A_log, Dskip, delta_bias, y, B, D, 1, L, N, K, dtype, 0};
+    pr.hlast = h_last;
+    return forward(pr, stream, variant, false, false, true);
+}
+
 int ss2d_backward(const void *x, const void *delta, const float *A_log, const void *Bs,
                   const void *Cs, const float *Dskip, const float *delta_bias, const float *dy,
                   float *dx, float *ddelta, float *dA_log, float *dBs, float *dCs,
@@ -563,7 +591,7 @@ int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
     if (num_chunks)
         *num_chunks = pl.NC;
     if (launches)
-        *launches = pl.launches;
+        *launches = pl.launches + (pl.NC > 1 ? 3 : 1) * ((N + ss2d::kNP - 1) / ss2d::kNP - 1);
     return SS2D_OK;
 }
 

@@ -317,17 +317,19 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int n0 = 2 * j, n1 = 2 * j + 1;
-        A2[j].x = (n0 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0)) * kLog2e : 0.f;
-        A2[j].y = (n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
+        const float *al = p.A_log + (size_t)kd * p.NS + p.n0;
+        A2[j].x = (n0 < N) ? -expf(__ldg(al + n0)) * kLog2e : 0.f;
+        A2[j].y = (n1 < N) ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
     }
-    const float dsk = __ldg(p.Dskip + kd);
+    const bool accum = p.accum != 0;   // a later state group: add to out, no skip term
+    const float dsk = accum ? 0.f : __ldg(p.Dskip + kd);
     const float bias = __ldg(p.delta_bias + kd);
 
     const size_t row_bk = ((size_t)b * K + k) * D;   // row index of (b, k, d = 0)
     const Tin *drow = static_cast<const Tin *>(p.delta) + (row_bk + dc) * L;   // my delta row
     const Tin *xrow = static_cast<const Tin *>(p.x) + ((size_t)b * D + dc) * L;  // my x map
-    const Tin *Bg = static_cast<const Tin *>(p.Bs) + ((size_t)b * K + k) * N * L;
-    const Tin *Cg = static_cast<const Tin *>(p.Cs) + ((size_t)b * K + k) * N * L;
+    const Tin *Bg = static_cast<const Tin *>(p.Bs) + (((size_t)b * K + k) * p.NS + p.n0) * L;
+    const Tin *Cg = static_cast<const Tin *>(p.Cs) + (((size_t)b * K + k) * p.NS + p.n0) * L;
     // x order of this direction: 0 forward, 1 reversed (both contiguous),
     // 2 through the pixel walker (column-major directions)
     const int xmode = (COLS && k >= 2) ? 2 : (k & 1);
@@ -552,25 +554,30 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
             const bool flip = k == 1 && K > 1;
             float *rowp = p.out + (row_bk + d) * L;
             if (ovec && l0 + kT <= l_end) {
-                float *orow = rowp + (flip ? L - kT - l0 : l0);
-                if (flip) {
+                float4 *orow = reinterpret_cast<float4 *>(rowp + (flip ? L - kT - l0 : l0));
 #pragma unroll
-                    for (int q = 0; q < kT / 4; ++q)
-                        reinterpret_cast<float4 *>(orow)[q] = make_float4(
-                            sY[(15 - 4 * q) * 33 + lane], sY[(14 - 4 * q) * 33 + lane],
-                            sY[(13 - 4 * q) * 33 + lane], sY[(12 - 4 * q) * 33 + lane]);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < kT / 4; ++q)
-                        reinterpret_cast<float4 *>(orow)[q] =
-                            make_float4(sY[(4 * q) * 33 + lane], sY[(4 * q + 1) * 33 + lane],
-                                        sY[(4 * q + 2) * 33 + lane], sY[(4 * q + 3) * 33 + lane]);
+                for (int q = 0; q < kT / 4; ++q) {
+                    float4 v = flip ? make_float4(sY[(15 - 4 * q) * 33 + lane],
+                                                  sY[(14 - 4 * q) * 33 + lane],
+                                                  sY[(13 - 4 * q) * 33 + lane],
+                                                  sY[(12 - 4 * q) * 33 + lane])
+                                    : make_float4(sY[(4 * q) * 33 + lane],
+                                                  sY[(4 * q + 1) * 33 + lane],
+                                                  sY[(4 * q + 2) * 33 + lane],
+                                                  sY[(4 * q + 3) * 33 + lane]);
+                    if (accum) {
+                        const float4 o = orow[q];
+                        v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+                    }
+                    orow[q] = v;
                 }
             } else {
 #pragma unroll
                 for (int t = 0; t < kT; ++t)
-                    if (l0 + t < l_end)
-                        rowp[flip ? L - 1 - l0 - t : l0 + t] = sY[t * 33 + lane];
+                    if (l0 + t < l_end) {
+                        float *o = rowp + (flip ? L - 1 - l0 - t : l0 + t);
+                        *o = accum ? *o + sY[t * 33 + lane] : sY[t * 33 + lane];
+                    }
             }
         }
         if (more) {
@@ -595,6 +602,17 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
             hs[q] = make_float4(h2[2 * q].x, h2[2 * q].y, h2[2 * q + 1].x, h2[2 * q + 1].y);
         p.dtsum[(row_bk + d) * (p.NC - 1) + chunk] = dtsum;
     }
+    // the state after the last step (steps past L stage dt = 0: identity)
+    if (MODE == kModeOutput && p.hlast && cvalid && chunk == p.NC - 1) {
+        float *hl = p.hlast + (row_bk + d) * p.NS + p.n0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (2 * j < N)
+                hl[2 * j] = h2[j].x;
+            if (2 * j + 1 < N)
+                hl[2 * j + 1] = h2[j].y;
+        }
+    }
 }
 
 // Entry states of every chunk after the first, in place over the chunk end
@@ -613,7 +631,8 @@ static __global__ void carry_kernel(const ScanParams p)
     const int d = (int)(bkd % p.D);
     const int k = (int)((bkd / p.D) % p.K);
     const float a2 =
-        n < p.N ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.N + n)) * kLog2e : 0.f;
+        n < p.N ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0 + n)) * kLog2e
+                : 0.f;
     float *hs = p.hstate + (size_t)bkd * (p.NC - 1) * kNP + n;
     const float *ds = p.dtsum + (size_t)bkd * (p.NC - 1);
     const int nc1 = p.NC - 1;

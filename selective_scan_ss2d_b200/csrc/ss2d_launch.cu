@@ -124,14 +124,30 @@ cudaError_t launch_scan(const Plan &plan, int dtype, ScanParams &p, cudaStream_t
 {
     p.LC = plan.LC;
     p.NC = plan.NC;
-    switch (dtype) {
-    case 1:
-        return launch_scan_bf16(plan, p, st, ev);
-    case 2:
-        return launch_scan_f16(plan, p, st, ev);
-    default:
-        return launch_scan_f32(plan, p, st, ev);
+    // more than 16 states: the passes once per group of at most 16 states, in
+    // order on the stream, the later groups adding to the first group's rows
+    const int ns = p.N;
+    cudaError_t e = cudaSuccess;
+    for (int n0 = 0; n0 < ns && e == cudaSuccess; n0 += kNP) {
+        ScanParams q = p;
+        q.n0 = n0;
+        q.NS = ns;
+        q.N = ns - n0 < kNP ? ns - n0 : kNP;
+        q.accum = n0 > 0 ? 1 : 0;
+        cudaEvent_t *qev = n0 == 0 ? ev : nullptr;
+        switch (dtype) {
+        case 1:
+            e = launch_scan_bf16(plan, q, st, qev);
+            break;
+        case 2:
+            e = launch_scan_f16(plan, q, st, qev);
+            break;
+        default:
+            e = launch_scan_f32(plan, q, st, qev);
+            break;
+        }
     }
+    return e;
 }
 
 namespace {

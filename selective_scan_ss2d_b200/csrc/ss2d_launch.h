@@ -8,6 +8,8 @@ namespace ss2d {
 
 struct ScanParams;
 
+constexpr int kMaxN = 64;   // states per channel a forward call accepts
+
 // Launch kern on st; dependent = true launches it as a programmatic
 // dependent of the previous kernel on the stream (it may start before that
 // one finishes and waits in-kernel, with grid_dependency_wait, before it
@@ -60,7 +62,8 @@ int pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
 Plan make_plan(int variant, int B, int D, int L, int K);
 
 // Launch the scan passes (state, carry, output) for a plan; the caller has
-// set p.out (and p.hstate / p.dtsum when plan.NC > 1).  If ev is not null,
+// set p.out (and p.hstate / p.dtsum when plan.NC > 1) and p.N to the call's
+// state count (up to kMaxN; more than 16 states run as groups of 16).  If ev is not null,
 // ev[0..3] are recorded on the stream before the state pass, the carry, the
 // output pass and after it (the first two only when the plan is chunked).
 cudaError_t launch_scan(const Plan &plan, int dtype, ScanParams &p, cudaStream_t st,

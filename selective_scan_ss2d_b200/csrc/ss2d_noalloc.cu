@@ -147,6 +147,7 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     p.W = W;
     p.L = (int)L;
     p.N = N;
+    p.NS = N;
     p.K = K;
     p.two_d = 1;
     p.out = K > 1 ? reinterpret_cast<float *>(base) : y;

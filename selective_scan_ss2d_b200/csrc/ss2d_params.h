@@ -26,6 +26,12 @@ struct ScanParams {
     int NC;                   // chunks per sequence
     int vec;                  // 16 / 8: byte width of vector loads of delta and x rows; 0: none
     int ovec;                 // 1: rows of out allow 16-byte vector stores
+    float *hlast;             // (B,K,D,NS): state after each direction's last step, or null
+    // state groups: a call with more than 16 states runs the passes once per
+    // group of at most 16 (the states of a channel never interact)
+    int n0;                   // first state of this group
+    int NS;                   // states per row of A_log, Bs, Cs, hlast (N is this group's count)
+    int accum;                // 1: add this group's output to `out` (skip term left out)
 };
 
 }  // namespace ss2d

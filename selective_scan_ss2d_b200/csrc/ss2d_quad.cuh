@@ -105,10 +105,12 @@ __global__ void __launch_bounds__(32 * NW, MINB) quad_scan_kernel(const ScanPara
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const int n0 = 4 * q + 2 * j, n1 = n0 + 1;
-        A2[j].x = (n0 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n0)) * kLog2e : 0.f;
-        A2[j].y = (n1 < N) ? -expf(__ldg(p.A_log + (size_t)kd * N + n1)) * kLog2e : 0.f;
+        const float *al = p.A_log + (size_t)kd * p.NS + p.n0;
+        A2[j].x = (n0 < N) ? -expf(__ldg(al + n0)) * kLog2e : 0.f;
+        A2[j].y = (n1 < N) ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
     }
-    const float dsk = __ldg(p.Dskip + kd);
+    const bool accum = p.accum != 0;   // a later state group: add to out, no skip term
+    const float dsk = accum ? 0.f : __ldg(p.Dskip + kd);
     const float bias = __ldg(p.delta_bias + kd);
 
     const size_t row_bk = ((size_t)b * K + k) * D;
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(32 * NW, MINB) quad_scan_kernel(const ScanPara
     {
         const int n = r & 15;
         const Tin *base = static_cast<const Tin *>(r < 16 ? p.Bs : p.Cs);
-        bcrow = n < N ? base + (((size_t)b * K + k) * N + n) * L : nullptr;
+        bcrow = n < N ? base + (((size_t)b * K + k) * p.NS + p.n0 + n) * L : nullptr;
     }
     constexpr int BC_ITEMS = 2 * kNP * (kT / 4);   // (row, group) items per sub-chunk: 128
     constexpr int BC_PER_THREAD = (BC_ITEMS + NT - 1) / NT;
@@ -283,24 +285,32 @@ __global__ void __launch_bounds__(32 * NW, MINB) quad_scan_kernel(const ScanPara
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     o[i] = fmaf(dsk, u_cur[i], r4[i]);
+                auto put4 = [&](float *dst, float4 v) {
+                    float4 *d4 = reinterpret_cast<float4 *>(dst);
+                    if (accum) {
+                        const float4 e = *d4;
+                        v = make_float4(e.x + v.x, e.y + v.y, e.z + v.z, e.w + v.w);
+                    }
+                    *d4 = v;
+                };
+                auto put1 = [&](float *dst, float v) { *dst = accum ? *dst + v : v; };
                 if (k == 1 && K > 1) {
                     // direction 1 of a multi-direction call: pixel order
                     if (v4 && l + 3 < l_end) {
-                        *reinterpret_cast<float4 *>(orow + (L - 4 - l)) =
-                            make_float4(o[3], o[2], o[1], o[0]);
+                        put4(orow + (L - 4 - l), make_float4(o[3], o[2], o[1], o[0]));
                     } else {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             if (l + i < l_end)
-                                orow[L - 1 - l - i] = o[i];
+                                put1(orow + (L - 1 - l - i), o[i]);
                     }
                 } else if (v4 && l + 3 < l_end) {
-                    *reinterpret_cast<float4 *>(orow + l) = make_float4(o[0], o[1], o[2], o[3]);
+                    put4(orow + l, make_float4(o[0], o[1], o[2], o[3]));
                 } else {
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         if (l + i < l_end)
-                            orow[l + i] = o[i];
+                            put1(orow + l + i, o[i]);
                 }
             }
         }
@@ -320,6 +330,15 @@ __global__ void __launch_bounds__(32 * NW, MINB) quad_scan_kernel(const ScanPara
             if (q == 0)
                 p.dtsum[(row_bk + d) * (p.NC - 1) + chunk] = dts;
         }
+    }
+    // the state after the last step: states 4q .. 4q+3 of this lane
+    if (MODE == kModeOutput && p.hlast && cvalid && chunk == p.NC - 1) {
+        float *hl = p.hlast + (row_bk + d) * p.NS + p.n0 + 4 * q;
+        const float hv[4] = {h2[0].x, h2[0].y, h2[1].x, h2[1].y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (4 * q + i < p.N)
+                hl[i] = hv[i];
     }
 }
 

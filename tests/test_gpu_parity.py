@@ -298,3 +298,108 @@ def test_gated_rejects_host_pointers_and_missing_gate():
                                                                "Dskip", "delta_bias")],
                                 None, binding._ptr(y), 1, 4, 4, 4, 4, 4, 0, None)
     assert rc == -1
+
+
+# ---------------------------------------------------------------------------
+# final states (ss2d_forward_final_state / selective_scan_fwd_final_state)
+# ---------------------------------------------------------------------------
+FINAL = [small(B=2, D=12, H=7, W=9), small(B=1, D=40, H=14, W=14), small(B=1, D=8, H=33, W=31),
+         small(B=2, D=9, H=6, W=5, K=2, N=5), small(B=2, D=9, H=6, W=5, K=1, N=1),
+         small("1d", B=3, D=20, W=197, K=2), small("1d", B=1, D=33, W=1000, K=2),
+         small("1d", B=2, D=7, W=50, K=1, N=3)]
+
+
+def _final_oracle(inp):
+    f = inp.as_f64()
+    return oracle.final_states(f["x"], f["delta"], f["A_log"], f["Bs"], f["delta_bias"],
+                               K=inp.cfg.K, two_d=inp.cfg.kind == "2d")
+
+
+@pytest.mark.parametrize("cfg", FINAL, ids=lambda c: c.name)
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+def test_final_state_matches_oracle(cfg, dtype):
+    cfg = cfg.with_(dtype=dtype)
+    inp = wl.make_inputs(cfg, seed=6)
+    ref = _final_oracle(inp)
+    t = _gpu.tensors(inp)
+    args = [t[n] for n in ("x", "delta", "A_log", "Bs", "Cs", "Dskip", "delta_bias")]
+    for v in [-1] + list(range(nvariants())):
+        y, h = binding.forward_final_state(*args, variant=v)
+        torch.cuda.synchronize()
+        # the same kernels as the plain forward: y identical to the bit
+        y0 = _gpu.run_gpu(inp, variant=v, t=t)
+        assert np.array_equal(y.cpu().numpy().astype(np.float64), y0), f"variant {v}: y differs"
+        _gpu.assert_close(h.cpu().numpy().astype(np.float64), ref, dtype,
+                          f"{cfg.name} variant {v} final state")
+
+
+@pytest.mark.parametrize("name", ["vmamba_t_stage1", "highres_256"])
+def test_final_state_full_size_sampled(name):
+    inp = wl.make_inputs(name, seed=0)
+    t = _gpu.tensors(inp)
+    _, h = binding.forward_final_state(*[t[n] for n in ("x", "delta", "A_log", "Bs", "Cs", "Dskip",
+                                                        "delta_bias")])
+    h = h.cpu().numpy().astype(np.float64)
+    for (b, d) in [(0, 0), (inp.cfg.B - 1, inp.cfg.D - 1), (0, inp.cfg.D // 2)]:
+        sub = wl.channel_subproblem(inp, b, d)
+        ref = _final_oracle(sub)
+        _gpu.assert_close(h[b:b + 1, :, d:d + 1], ref, inp.cfg.dtype, f"{name} ({b},{d})")
+
+
+def test_final_state_rejects_missing_or_host_buffers():
+    inp = wl.make_inputs(small(B=1, D=4, H=4, W=4, K=4, N=4), seed=0)
+    td = _gpu.tensors(inp)
+    lib = binding.lib()
+    names = ("x", "delta", "A_log", "Bs", "Cs", "Dskip", "delta_bias")
+    y = torch.empty_like(td["x"])
+    rc = lib.ss2d_forward_final_state(*[binding._ptr(td[n]) for n in names], binding._ptr(y),
+                                      None, 1, 4, 4, 4, 4, 4, 0, None, -1)
+    assert rc == -1
+    hh = torch.empty((1, 4, 4, 4))
+    rc = lib.ss2d_forward_final_state(*[binding._ptr(td[n]) for n in names], binding._ptr(y),
+                                      binding._ptr(hh), 1, 4, 4, 4, 4, 4, 0, None, -1)
+    assert rc == -9
+
+
+# ---------------------------------------------------------------------------
+# more than 16 states: groups of 16 run one after the other
+# ---------------------------------------------------------------------------
+WIDE_N = [small(B=2, D=12, H=7, W=9, N=17), small(B=1, D=40, H=14, W=14, N=32),
+          small(B=1, D=8, H=33, W=31, N=40), small(B=2, D=9, H=6, W=5, K=2, N=64),
+          small("1d", B=3, D=20, W=197, K=2, N=24), small("1d", B=2, D=7, W=50, K=1, N=48)]
+
+
+@pytest.mark.parametrize("cfg", WIDE_N, ids=lambda c: c.name)
+@pytest.mark.parametrize("dtype", [wl.F32, wl.BF16])
+def test_more_than_16_states(cfg, dtype):
+    cfg = cfg.with_(dtype=dtype)
+    inp = wl.make_inputs(cfg, seed=8)
+    ref = _gpu.run_oracle(inp)
+    href = _final_oracle(inp)
+    t = _gpu.tensors(inp)
+    args = [t[n] for n in ("x", "delta", "A_log", "Bs", "Cs", "Dskip", "delta_bias")]
+    for v in [-1] + list(range(nvariants())):
+        _gpu.assert_close(_gpu.run_gpu(inp, variant=v, t=t), ref, dtype, f"{cfg.name} v{v}")
+        y, h = binding.forward_final_state(*args, variant=v)
+        torch.cuda.synchronize()
+        _gpu.assert_close(h.cpu().numpy().astype(np.float64), href, dtype,
+                          f"{cfg.name} v{v} final state")
+
+
+def test_more_than_16_states_full_size_sampled():
+    """VMamba-T stage 1 with N = 32: sampled channels against the oracle."""
+    cfg = wl.CONFIGS["vmamba_t_stage1"].with_(N=32)
+    inp = wl.make_inputs(cfg, seed=0)
+    y = _gpu.run_gpu(inp)
+    for (b, d) in [(0, 0), (7, 191), (3, 77)]:
+        sub = wl.channel_subproblem(inp, b, d)
+        _gpu.assert_close(y[b:b + 1, d:d + 1], _gpu.run_oracle(sub), cfg.dtype, f"N=32 ({b},{d})")
+
+
+def test_backward_rejects_more_than_16_states():
+    inp = wl.make_inputs(small(B=1, D=4, H=4, W=4, N=20), seed=0)
+    t = _gpu.tensors(inp)
+    with pytest.raises(binding.SS2DError) as ei:
+        binding.ss2d_backward(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"],
+                              t["delta_bias"], torch.zeros((1, 4, 4, 4), device="cuda"))
+    assert ei.value.status == -5

@@ -237,3 +237,27 @@ def test_softplus_definition():
         assert math.isclose(oracle.softplus(z), math.log1p(math.exp(z)), rel_tol=1e-15)
         assert math.isclose(float(onp.softplus(z)), math.log1p(math.exp(z)), rel_tol=1e-15)
     assert oracle.softplus(1000.0) == 1000.0
+
+
+def test_states_split_into_groups():
+    """The states of a channel never interact: y with N = 40 states equals the
+    sum of the outputs of states 0..15, 16..31 and 32..39 run alone, with the
+    skip term counted once (pins the oracle where N is above 16)."""
+    rng = np.random.default_rng(9)
+    B, D, H, W, K, N = 1, 3, 4, 5, 4, 40
+    L = H * W
+    x = rng.standard_normal((B, D, H, W))
+    delta = rng.standard_normal((B, K, D, L))
+    A_log = rng.uniform(-1, 1, (K * D, N))
+    Bs = rng.standard_normal((B, K, N, L))
+    Cs = rng.standard_normal((B, K, N, L))
+    Dskip = rng.standard_normal(K * D)
+    bias = rng.uniform(-1, 1, K * D)
+    y = oracle.ss2d_forward(x, delta, A_log, Bs, Cs, Dskip, bias, K=4)
+    parts = []
+    for lo, hi in [(0, 16), (16, 32), (32, 40)]:
+        parts.append(oracle.ss2d_forward(x, delta, A_log[:, lo:hi], Bs[:, :, lo:hi],
+                                         Cs[:, :, lo:hi], np.zeros(K * D), bias, K=4))
+    skip = oracle.ss2d_forward(x, delta, A_log[:, :1], Bs[:, :, :1], 0 * Cs[:, :, :1], Dskip,
+                               bias, K=4)
+    np.testing.assert_allclose(y, parts[0] + parts[1] + parts[2] + skip, rtol=1e-12, atol=1e-12)

@@ -58,7 +58,7 @@ def test_noalloc_refuses_oversize_before_cuda(lib):
 def test_noalloc_shape_rules_match_forward(lib):
     p = ctypes.c_void_p(0)
     assert lib.ss2d_forward_noalloc(p, p, p, p, p, p, p, p, 1, 1, 2, 2, 4, 3, 0, None) == -4
-    assert lib.ss2d_forward_noalloc(p, p, p, p, p, p, p, p, 1, 1, 2, 2, 17, 4, 0, None) == -5
+    assert lib.ss2d_forward_noalloc(p, p, p, p, p, p, p, p, 1, 1, 2, 2, 65, 4, 0, None) == -5
     assert lib.ss2d_forward_noalloc(p, p, p, p, p, p, p, p, 1, 1, 2, 2, 4, 4, 7, None) == -3
     assert lib.ss2d_forward_noalloc(p, p, p, p, p, p, p, p, 0, 1, 2, 2, 4, 4, 0, None) == 0
     assert lib.ss2d_forward_noalloc(p, p, p, p, p, p, p, p, 1, 1, 2, 2, 4, 4, 0, None) == -1
