@@ -736,7 +736,7 @@ __device__ __forceinline__ float4 mul4(float4 a, float4 b)
     return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
 }
 
-template <int VEC, int CG>
+template <int VEC, int CG, bool GATE>
 __global__ void __launch_bounds__(kMerge2Threads)
     merge2_kernel(const float *__restrict__ part, float *__restrict__ y, int B, int D, int H,
                   int W, int K, int cols, int sum, int R, int whole, int flat,
@@ -792,7 +792,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
             const float4 v1 = K >= 2 ? __ldg(m + f) : make_float4(0.f, 0.f, 0.f, 0.f);
             if (sum) {
                 float4 v = make_float4(v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w);
-                if (z)
+                if constexpr (GATE)
                     v = mul4(v, gate4(z, zt, yr0 + 4 * f));
                 yo[f] = v;
             } else {
@@ -904,7 +904,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
                 if (cols)
                     v = make_float4((v.x + v2.x) + v3.x, (v.y + v2.y) + v3.y,
                                     (v.z + v2.z) + v3.z, (v.w + v2.w) + v3.w);
-                if (z)
+                if constexpr (GATE)
                     v = mul4(v, gate4(z, zt, yr + p));
                 *reinterpret_cast<float4 *>(yo + p) = v;
             } else {
@@ -931,7 +931,7 @@ __global__ void __launch_bounds__(kMerge2Threads)
                     v += v1;
                 if (cols)
                     v = (v + v2) + v3;
-                if (z)
+                if constexpr (GATE)
                     v *= gate1(z, zt, yr + p);
                 yo[p] = v;
             } else {

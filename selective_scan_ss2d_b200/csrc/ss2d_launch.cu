@@ -205,8 +205,10 @@ cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int 
 {
     const long long groups = ((long long)B * D + CG - 1) / CG;
     dim3 grid((unsigned)groups, (unsigned)m.nbands);
-    return launch_kernel(merge2_kernel<VEC, CG>, grid, dim3(kMerge2Threads), m.smem, st, true,
-                         part, y, B, D, H, W, K, m.cols, sum, m.R, m.whole, m.flat, z, zt);
+    // the gate is compiled in only for gated calls
+    auto kern = z ? merge2_kernel<VEC, CG, true> : merge2_kernel<VEC, CG, false>;
+    return launch_kernel(kern, grid, dim3(kMerge2Threads), m.smem, st, true, part, y, B, D, H,
+                         W, K, m.cols, sum, m.R, m.whole, m.flat, z, zt);
 }
 }  // namespace
 
