@@ -42,13 +42,14 @@ FALLBACK_SM_MAX_MHZ = 1965.0
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from ncu
 # captures recorded under profiles/, keyed by workload; each entry carries
-# the input dtype and the hash of the kernel sources it was taken from, and
-# is reported only for that dtype while the sources are unchanged.
+# the input dtype, the state count and the hash of the kernel sources it was
+# taken from, and is reported only for that configuration while the sources
+# are unchanged.
 NCU_TRAFFIC = {
-    # profiles/chunk_scan_vmamba_t_stage1.md: output pass, dram read 65369344 + write 26022912
-    "vmamba_t_stage1": {"bytes": 91392256, "dtype": "bf16", "src": "1e7e65e446868e14"},
-    # profiles/chunk_scan_vmamba_b_stage3.md: output pass, dram read 141666816 + write 161465856
-    "vmamba_b_stage3": {"bytes": 303132672, "dtype": "bf16", "src": "1e7e65e446868e14"},
+    # profiles/chunk_scan_vmamba_t_stage1.md: output pass, dram read 65492224 + write 25570560
+    "vmamba_t_stage1": {"bytes": 91062784, "dtype": "bf16", "N": 16, "src": "4f946ebf7ed334c0"},
+    # profiles/chunk_scan_vmamba_b_stage3.md: output pass, dram read 141669632 + write 161776128
+    "vmamba_b_stage3": {"bytes": 303445760, "dtype": "bf16", "N": 16, "src": "4f946ebf7ed334c0"},
 }
 
 
@@ -255,12 +256,16 @@ def slice_sample(inp, nb, nd):
                      np.ascontiguousarray(inp.delta_bias[rows]))
 
 
-def workload_config(name, dtype=None):
-    """The named workload, with its streamed inputs' storage dtype replaced
-    when ``dtype`` is given (f32, bf16 or f16)."""
+def workload_config(name, dtype=None, n_states=None):
+    """The named workload, with its streamed inputs' storage dtype (f32, bf16
+    or f16) and its state count N replaced when given."""
     from selective_scan_ss2d_b200 import workloads as wl
     cfg = wl.CONFIGS[name]
-    return cfg.with_(dtype=dtype) if dtype else cfg
+    if dtype:
+        cfg = cfg.with_(dtype=dtype)
+    if n_states:
+        cfg = cfg.with_(N=int(n_states))
+    return cfg
 
 
 def run_ours(args, rank, world, local_rank):
@@ -269,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
     from selective_scan_ss2d_b200 import binding
     from selective_scan_ss2d_b200 import workloads as wl
 
-    cfg = workload_config(args.config, args.dtype)
+    cfg = workload_config(args.config, args.dtype, args.n_states)
     dev = torch.device(f"cuda:{local_rank}")
     torch.cuda.set_device(dev)
     binding.lib()
@@ -356,7 +361,7 @@ def run_ours(args, rank, world, local_rank):
         src_hash = kernel_source_hash()
         tr = NCU_TRAFFIC.get(cfg.name)
         traffic = (tr["bytes"] if tr and tr.get("src") == src_hash and tr["dtype"] == cfg.dtype
-                   else None)
+                   and tr["N"] == cfg.N else None)
         variant = args.variant if args.variant >= 0 else binding.ss2d_pick_variant(
             two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K)
         plan = binding.ss2d_plan(two_d, cfg.B, cfg.D, cfg.H, cfg.W, cfg.N, cfg.K, variant)
@@ -419,7 +424,7 @@ def run_backward(args, rank, world, local_rank):
     from selective_scan_ss2d_b200 import binding
     from selective_scan_ss2d_b200 import workloads as wl
 
-    cfg = workload_config(args.config, args.dtype)
+    cfg = workload_config(args.config, args.dtype, args.n_states)
     dev = torch.device(f"cuda:{local_rank}")
     torch.cuda.set_device(dev)
     binding.lib()
@@ -504,7 +509,7 @@ def run_e2e(args, cfg_name, local_rank, world=1):
     import torch
     from selective_scan_ss2d_b200 import binding
     from selective_scan_ss2d_b200 import workloads as wl
-    cfg = workload_config(cfg_name, args.dtype)
+    cfg = workload_config(cfg_name, args.dtype, args.n_states)
     dev = torch.device(f"cuda:{local_rank}")
     inp, t = build_arrays(cfg, seed=0, device=None, pin=True)
     y = torch.empty(inp.x.shape, dtype=torch.float32).pin_memory()
@@ -536,7 +541,7 @@ def run_reference(args):
     (whole channels of batch element 0) of the workload."""
     import oracle
     from selective_scan_ss2d_b200 import workloads as wl
-    cfg = workload_config(args.config, args.dtype)
+    cfg = workload_config(args.config, args.dtype, args.n_states)
     threads = oracle.max_threads()
     # size one step to ~ (budget / (steps + warmup)) seconds of host work
     budget_s = float(os.environ.get("SS2D_REFERENCE_BUDGET_S", "150"))
@@ -587,6 +592,8 @@ def main():
     ap.add_argument("--variant", type=int, default=-1)
     ap.add_argument("--dtype", choices=["f32", "bf16", "f16"], default=None,
                     help="storage dtype of x, delta, Bs, Cs (default: the workload's own)")
+    ap.add_argument("--n-states", type=int, default=None,
+                    help="state count N, 1..64 (default: the workload's own, 16)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -647,7 +654,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             from selective_scan_ss2d_b200 import workloads as wl
-            cfg = workload_config(args.config, args.dtype)
+            cfg = workload_config(args.config, args.dtype, args.n_states)
             threads = oracle.max_threads()
             v, desc, _ = cpu_baseline_parallel(cfg, args.cpu_seconds, threads)
             line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": threads,

@@ -287,9 +287,12 @@ __device__ __forceinline__ uint32_t raw_bits(const __half *p)
 // grid: x = k, y = channel tile, z = b * NCg + chunk, NCg = chunks launched
 // (NC - 1 in kModeState, NC in kModeOutput).
 // COLS: the column-major directions (SS2D with K = 4) are compiled in.
-template <typename Tin, int WC, int MODE, int MINB, bool COLS>
+// QN: groups of 4 states the lane runs (4: up to 16 states; 2: up to 8, half
+// the exp2 and FMA work of a step).
+template <typename Tin, int WC, int MODE, int MINB, bool COLS, int QN>
 __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
 {
+    static_assert(QN == 2 || QN == 4, "8 or 16 states per lane");
     using Sh = ChunkShape<WC>;
     constexpr int NT = Sh::NT, BCPT = Sh::BC_PER_THREAD;
 
@@ -529,7 +532,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
             const float4 *col = sb + t;   // slot q at col[q * kT]
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < QN; ++q) {
                 const float4 bv = col[q * kT];
                 const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
                 const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);

@@ -24,8 +24,14 @@ template <typename Tin, int WC, int MODE, int R>
 cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
     using Sh = ChunkShape<WC>;
-    auto kern = (p.two_d && p.K == 4) ? chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, true>
-                                      : chunk_scan_kernel<Tin, WC, MODE, MinBlocks<WC, R>::value, false>;
+    constexpr int MB = MinBlocks<WC, R>::value;
+    // the column-major path only where a direction is column-major; half the
+    // state work when this call (or state group) has at most 8 states
+    const bool cols = p.two_d && p.K == 4, eight = p.N <= 8;
+    auto kern = cols ? (eight ? chunk_scan_kernel<Tin, WC, MODE, MB, true, 2>
+                              : chunk_scan_kernel<Tin, WC, MODE, MB, true, 4>)
+                     : (eight ? chunk_scan_kernel<Tin, WC, MODE, MB, false, 2>
+                              : chunk_scan_kernel<Tin, WC, MODE, MB, false, 4>);
     const size_t smem = Sh::SMEM_BYTES;
     if (smem > 48 * 1024) {
         cudaError_t e =

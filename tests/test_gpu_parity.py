@@ -403,3 +403,15 @@ def test_backward_rejects_more_than_16_states():
         binding.ss2d_backward(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"],
                               t["delta_bias"], torch.zeros((1, 4, 4, 4), device="cuda"))
     assert ei.value.status == -5
+
+
+@pytest.mark.parametrize("name", ["vmamba_t_stage1", "vim_s_bidir"])
+def test_eight_states_full_size_sampled(name):
+    """d_state 8 ("VMamba架构解析", section 5) at full size: the 8-state
+    kernels against the oracle on sampled channels."""
+    cfg = wl.CONFIGS[name].with_(N=8)
+    inp = wl.make_inputs(cfg, seed=0)
+    y = _gpu.run_gpu(inp)
+    for (b, d) in [(0, 0), (cfg.B - 1, cfg.D - 1), (cfg.B // 2, 77)]:
+        sub = wl.channel_subproblem(inp, b, d)
+        _gpu.assert_close(y[b:b + 1, d:d + 1], _gpu.run_oracle(sub), cfg.dtype, f"N=8 ({b},{d})")
