@@ -172,6 +172,38 @@ __device__ __forceinline__ void store16(float *dst, const float *v)
         d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 
+// States in pairs (2j, 2j+1) for the sm_100 packed f32x2 instructions
+// (__ffma2_rn, __fmul2_rn: each lane rounds as fmaf / a float multiply).
+__device__ __forceinline__ float2 ex2_pair(float2 a)
+{
+    return make_float2(mufu_ex2(a.x), mufu_ex2(a.y));
+}
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+// pair j of a 16-float shared-memory row (16-byte aligned)
+__device__ __forceinline__ float2 row_pair(const float *row, int j)
+{
+    return reinterpret_cast<const float2 *>(row)[j];
+}
+__device__ __forceinline__ void load_a2(float2 *A2, const BwdParams &p, size_t kd)
+{
+#pragma unroll
+    for (int j = 0; j < kNP / 2; ++j) {
+        const int n0 = 2 * j, n1 = 2 * j + 1;
+        A2[j].x = n0 < p.N ? -expf(__ldg(p.A_log + kd * p.N + n0)) * kLog2e : 0.f;
+        A2[j].y = n1 < p.N ? -expf(__ldg(p.A_log + kd * p.N + n1)) * kLog2e : 0.f;
+    }
+}
+// one step of the state recurrence, h = exp(dt A) h + dt u B, for all pairs
+__device__ __forceinline__ void state_step(float2 *h, const float2 *A2, float dt, float dtu,
+                                           const float *brow)
+{
+    const float2 dt2 = dup2(dt), dtu2 = dup2(dtu);
+#pragma unroll
+    for (int j = 0; j < kNP / 2; ++j)
+        h[j] = __ffma2_rn(ex2_pair(__fmul2_rn(dt2, A2[j])), h[j],
+                          __fmul2_rn(dtu2, row_pair(brow, j)));
+}
+
 template <typename Tin>
 __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
 {
@@ -181,10 +213,8 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
     const int lane = threadIdx.x;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
-    float A2[kNP];
-#pragma unroll
-    for (int n = 0; n < kNP; ++n)
-        A2[n] = n < p.N ? -expf(__ldg(p.A_log + kd * p.N + n)) * kLog2e : 0.f;
+    float2 A2[kNP / 2];
+    load_a2(A2, p, kd);
     const float bias = __ldg(p.delta_bias + kd);
     const int nc1 = p.NC - 1;
     const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
@@ -201,38 +231,37 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
         for (int t = 0; t < kT; ++t)
             dts += st4[t * kBwdLanes + lane].x;
         if (c < nc1) {
-            float h[kNP];
+            float2 h[kNP / 2];
 #pragma unroll
-            for (int n = 0; n < kNP; ++n)
-                h[n] = 0.f;
+            for (int j = 0; j < kNP / 2; ++j)
+                h[j] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int t = 0; t < kT; ++t) {
                 const float4 v = st4[t * kBwdLanes + lane];
-                const float dtu = v.x * v.y;
-#pragma unroll
-                for (int n = 0; n < kNP; ++n)
-                    h[n] = fmaf(mufu_ex2(v.x * A2[n]), h[n], dtu * sB[t * kNP + n]);
+                state_step(h, A2, v.x, v.x * v.y, sB + t * kNP);
             }
             if (q.active) {
-                store16(p.hfwd + (q.bkd * nc1 + c) * kNP, h);
+                store16(p.hfwd + (q.bkd * nc1 + c) * kNP, reinterpret_cast<const float *>(h));
                 p.dtf[q.bkd * nc1 + c] = dts;
             }
         }
         if (c > 0) {
-            float g[kNP];
+            float2 g[kNP / 2];
 #pragma unroll
-            for (int n = 0; n < kNP; ++n)
-                g[n] = 0.f;
+            for (int j = 0; j < kNP / 2; ++j)
+                g[j] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int t = kT - 1; t >= 0; --t) {
                 const float4 v = st4[t * kBwdLanes + lane];
+                const float2 dt2 = dup2(v.x), gy2 = dup2(v.z);
 #pragma unroll
-                for (int n = 0; n < kNP; ++n)
-                    g[n] = mufu_ex2(v.x * A2[n]) * fmaf(v.z, sC[t * kNP + n], g[n]);
+                for (int j = 0; j < kNP / 2; ++j)
+                    g[j] = __fmul2_rn(ex2_pair(__fmul2_rn(dt2, A2[j])),
+                                      __ffma2_rn(gy2, row_pair(sC + t * kNP, j), g[j]));
             }
             if (q.active) {
                 const int r = nc1 - c;   // reversed chunk order
-                store16(p.hadj + (q.bkd * nc1 + r) * kNP, g);
+                store16(p.hadj + (q.bkd * nc1 + r) * kNP, reinterpret_cast<const float *>(g));
                 p.dta[q.bkd * nc1 + r] = dts;
             }
         }
@@ -277,10 +306,8 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
     const int swz = (lane >> 1) & 3;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
-    float A2[kNP];
-#pragma unroll
-    for (int n = 0; n < kNP; ++n)
-        A2[n] = n < p.N ? -expf(__ldg(p.A_log + kd * p.N + n)) * kLog2e : 0.f;
+    float2 A2[kNP / 2];
+    load_a2(A2, p, kd);
     const float bias = __ldg(p.delta_bias + kd);
     const float Dk = __ldg(p.Dskip + kd);
     const int L = p.L, nc1 = p.NC - 1;
@@ -290,10 +317,10 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
     float *bcrow = p.bc_part +
                    ((((size_t)q.bk * p.G + q.gi) * 2 + (lane >> 4)) * kNP + (lane & 15)) * L;
     const bool bc_ok = (lane & 15) < p.N;
-    float dA[kNP];
+    float2 dA[kNP / 2];
 #pragma unroll
-    for (int n = 0; n < kNP; ++n)
-        dA[n] = 0.f;
+    for (int j = 0; j < kNP / 2; ++j)
+        dA[j] = make_float2(0.f, 0.f);
     float dD = 0.f, db = 0.f;
     const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
     BwdRaw<Tin> raw;
@@ -309,59 +336,60 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
         // are parked at a time: the first recompute runs the whole chunk from
         // the entry state and parks steps 8..15 for the walk back over them;
         // the second recomputes steps 0..7 from the entry state again.
-        auto entry = [&](float *h) {
+        auto entry = [&](float2 *h) {
             if (c > 0)
-                load16(h, p.hfwd + (q.bkd * nc1 + (c - 1)) * kNP);
+                load16(reinterpret_cast<float *>(h), p.hfwd + (q.bkd * nc1 + (c - 1)) * kNP);
             else
 #pragma unroll
-                for (int n = 0; n < kNP; ++n)
-                    h[n] = 0.f;
+                for (int j = 0; j < kNP / 2; ++j)
+                    h[j] = make_float2(0.f, 0.f);
         };
-        auto recompute = [&](float *h, int t1, int park0) {
+        auto recompute = [&](float2 *h, int t1, int park0) {
 #pragma unroll 1
             for (int t = 0; t < t1; ++t) {
                 const float4 v = st4[t * kBwdLanes + lane];
-                const float dtu = v.x * v.y;
-#pragma unroll
-                for (int n = 0; n < kNP; ++n)
-                    h[n] = fmaf(mufu_ex2(v.x * A2[n]), h[n], dtu * sB[t * kNP + n]);
+                state_step(h, A2, v.x, v.x * v.y, sB + t * kNP);
                 if (t >= park0) {
                     float4 *row = hs4 + ((t - park0) * kBwdLanes + lane) * 4;
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        row[j ^ swz] = make_float4(h[4 * j], h[4 * j + 1], h[4 * j + 2],
-                                                   h[4 * j + 3]);
+                        row[j ^ swz] = make_float4(h[2 * j].x, h[2 * j].y, h[2 * j + 1].x,
+                                                   h[2 * j + 1].y);
                 }
             }
         };
-        float g[kNP];
+        float2 g[kNP / 2];
         auto walk_back = [&](int t_hi, int base) {
 #pragma unroll 2
             for (int t = t_hi; t >= base; --t) {
                 const float4 v4 = st4[t * kBwdLanes + lane];
                 const float dt = v4.x, u = v4.y, gy = v4.z;
                 const float dtu = dt * u;
+                const float2 dt2 = dup2(dt), dtu2 = dup2(dtu), ndtu2 = dup2(-dtu), gy2 = dup2(gy);
                 const float4 *row = hs4 + ((t - base) * kBwdLanes + lane) * 4;
                 float v[2 * kNP];
-                float s1 = 0.f, s2 = 0.f;   // sum g A2 (a h_prev), sum g B
+                // sum g A2 (a h_prev), sum g B: two-wide partial sums
+                float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 h4 = row[j ^ swz];
-                    const float hj[4] = {h4.x, h4.y, h4.z, h4.w};
+                for (int qd = 0; qd < 4; ++qd) {
+                    const float4 h4 = row[qd ^ swz];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int n = 4 * j + i;
-                        const float Bv = sB[t * kNP + n];
-                        const float hv = hj[i];
-                        g[n] = fmaf(gy, sC[t * kNP + n], g[n]);
-                        const float hp = fmaf(-dtu, Bv, hv);   // a_t h_{t-1}
-                        const float gdt = g[n] * dt;
-                        v[n] = g[n] * dtu;
-                        v[kNP + n] = gy * hv;
-                        s2 = fmaf(g[n], Bv, s2);
-                        s1 = fmaf(g[n] * A2[n], hp, s1);
-                        dA[n] = fmaf(gdt, hp, dA[n]);
-                        g[n] *= mufu_ex2(dt * A2[n]);
+                    for (int i = 0; i < 2; ++i) {
+                        const int j = 2 * qd + i;
+                        const float2 B2 = row_pair(sB + t * kNP, j);
+                        const float2 hv = i ? make_float2(h4.z, h4.w) : make_float2(h4.x, h4.y);
+                        g[j] = __ffma2_rn(gy2, row_pair(sC + t * kNP, j), g[j]);
+                        const float2 hp = __ffma2_rn(ndtu2, B2, hv);   // a_t h_{t-1}
+                        const float2 vb = __fmul2_rn(g[j], dtu2);
+                        const float2 vc = __fmul2_rn(gy2, hv);
+                        v[2 * j] = vb.x;
+                        v[2 * j + 1] = vb.y;
+                        v[kNP + 2 * j] = vc.x;
+                        v[kNP + 2 * j + 1] = vc.y;
+                        s2 = __ffma2_rn(g[j], B2, s2);
+                        s1 = __ffma2_rn(__fmul2_rn(g[j], A2[j]), hp, s1);
+                        dA[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), hp, dA[j]);
+                        g[j] = __fmul2_rn(g[j], ex2_pair(__fmul2_rn(dt2, A2[j])));
                     }
                 }
                 const float red = reduce_scatter32(v);
@@ -369,29 +397,30 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
                     bcrow[s + t] = red;
                 if (q.active && t < nt) {
                     const int l = s + t;
-                    const float ddl = fmaf(kLn2, s1, u * s2) * v4.w;
+                    const float S1 = s1.x + s1.y, S2 = s2.x + s2.y;
+                    const float ddl = fmaf(kLn2, S1, u * S2) * v4.w;
                     dD = fmaf(gy, u, dD);
                     db += ddl;
                     ddrow[l] = ddl;
-                    durow[flip ? L - 1 - l : l] = fmaf(Dk, gy, dt * s2);
+                    durow[flip ? L - 1 - l : l] = fmaf(Dk, gy, dt * S2);
                 }
             }
         };
         // the adjoint entering at the chunk end
         if (c < nc1)
-            load16(g, p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
+            load16(reinterpret_cast<float *>(g), p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
         else
 #pragma unroll
-            for (int n = 0; n < kNP; ++n)
-                g[n] = 0.f;
+            for (int j = 0; j < kNP / 2; ++j)
+                g[j] = make_float2(0.f, 0.f);
         {
-            float h[kNP];
+            float2 h[kNP / 2];
             entry(h);
             recompute(h, kT, kHalf);
         }
         walk_back(kT - 1, kHalf);
         {
-            float h[kNP];
+            float2 h[kNP / 2];
             entry(h);
             recompute(h, kHalf, 0);
         }
@@ -400,8 +429,10 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
     if (q.active) {
         float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * kPrm;
 #pragma unroll
-        for (int n = 0; n < kNP; ++n)
-            pr[n] = dA[n];
+        for (int j = 0; j < kNP / 2; ++j) {
+            pr[2 * j] = dA[j].x;
+            pr[2 * j + 1] = dA[j].y;
+        }
         pr[kNP] = dD;
         pr[kNP + 1] = db;
     }
