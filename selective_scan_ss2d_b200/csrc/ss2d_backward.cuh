@@ -317,6 +317,9 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
     float *bcrow = p.bc_part +
                    ((((size_t)q.bk * p.G + q.gi) * 2 + (lane >> 4)) * kNP + (lane & 15)) * L;
     const bool bc_ok = (lane & 15) < p.N;
+    // rows of L floats: 16-byte segments at 16-step chunk starts when L % 4 == 0
+    // (the scratch and gradient buffers are 16-byte aligned)
+    const bool vec_rows = (L & 3) == 0;
     float2 dA[kNP / 2];
 #pragma unroll
     for (int j = 0; j < kNP / 2; ++j)
@@ -393,16 +396,14 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
                     }
                 }
                 const float red = reduce_scatter32(v);
-                if (bc_ok && t < nt)
-                    bcrow[s + t] = red;
+                // this step's results replace its staged inputs in the lane's own
+                // slot (consumed by now); the rows are written once per chunk
+                const float S1 = s1.x + s1.y, S2 = s2.x + s2.y;
+                const float ddl = fmaf(kLn2, S1, u * S2) * v4.w;
+                st4[t * kBwdLanes + lane] = make_float4(ddl, fmaf(Dk, gy, dt * S2), red, 0.f);
                 if (q.active && t < nt) {
-                    const int l = s + t;
-                    const float S1 = s1.x + s1.y, S2 = s2.x + s2.y;
-                    const float ddl = fmaf(kLn2, S1, u * S2) * v4.w;
                     dD = fmaf(gy, u, dD);
                     db += ddl;
-                    ddrow[l] = ddl;
-                    durow[flip ? L - 1 - l : l] = fmaf(Dk, gy, dt * S2);
                 }
             }
         };
@@ -425,6 +426,48 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
             recompute(h, kHalf, 0);
         }
         walk_back(kHalf - 1, 0);
+        // the chunk's rows: ddelta and du of this lane's channel, and the
+        // reduced dB | dC row this lane holds (16-byte segments when whole)
+        const bool whole = nt == kT && vec_rows;
+        if (q.active) {
+            if (whole) {
+                float4 *dd4 = reinterpret_cast<float4 *>(ddrow + s);
+                float4 *du4 = reinterpret_cast<float4 *>(durow + (flip ? L - kT - s : s));
+#pragma unroll
+                for (int i = 0; i < kT / 4; ++i) {
+                    const float4 a = st4[(4 * i) * kBwdLanes + lane];
+                    const float4 b = st4[(4 * i + 1) * kBwdLanes + lane];
+                    const float4 c4 = st4[(4 * i + 2) * kBwdLanes + lane];
+                    const float4 d4 = st4[(4 * i + 3) * kBwdLanes + lane];
+                    dd4[i] = make_float4(a.x, b.x, c4.x, d4.x);
+                    if (flip)
+                        du4[kT / 4 - 1 - i] = make_float4(d4.y, c4.y, b.y, a.y);
+                    else
+                        du4[i] = make_float4(a.y, b.y, c4.y, d4.y);
+                }
+            } else {
+                for (int t = 0; t < nt; ++t) {
+                    const float4 r = st4[t * kBwdLanes + lane];
+                    const int l = s + t;
+                    ddrow[l] = r.x;
+                    durow[flip ? L - 1 - l : l] = r.y;
+                }
+            }
+        }
+        if (bc_ok) {
+            if (whole) {
+                float4 *bc4 = reinterpret_cast<float4 *>(bcrow + s);
+#pragma unroll
+                for (int i = 0; i < kT / 4; ++i)
+                    bc4[i] = make_float4(st4[(4 * i) * kBwdLanes + lane].z,
+                                         st4[(4 * i + 1) * kBwdLanes + lane].z,
+                                         st4[(4 * i + 2) * kBwdLanes + lane].z,
+                                         st4[(4 * i + 3) * kBwdLanes + lane].z);
+            } else {
+                for (int t = 0; t < nt; ++t)
+                    bcrow[s + t] = st4[t * kBwdLanes + lane].z;
+            }
+        }
     }
     if (q.active) {
         float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * kPrm;

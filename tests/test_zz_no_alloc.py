@@ -76,6 +76,7 @@ SHAPES = [
     cfg(1, 32, 40, 40, 4, 16, wl.BF16),   # chunked: L = 1600, few sequences
     cfg(1, 24, 30, 33, 2, 16, wl.F32),    # K = 2, chunked
     cfg(1, 16, 36, 36, 1, 8, wl.F32),     # K = 1: chunk states only
+    cfg(1, 24, 30, 33, 4, 40, wl.BF16),   # N = 40: three state groups, chunked
 ]
 
 
