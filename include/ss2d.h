@@ -82,8 +82,7 @@ typedef enum {
     SS2D_ERR_SHAPE = -2,  /* a size is negative, or a product overflows     */
     SS2D_ERR_DTYPE = -3,  /* dtype is not one of ss2d_dtype                  */
     SS2D_ERR_K = -4,      /* K not in {1,2,4} (2D) or {1,2} (1D)             */
-    SS2D_ERR_N = -5,      /* N not in 1..64 (forward) or 1..16 (backward and
-                             ss2d_forward_timed)                         */
+    SS2D_ERR_N = -5,      /* N not in 1..64 (1..16 for ss2d_forward_timed) */
     SS2D_ERR_ALIGN = -6,  /* a pointer is not 16-byte aligned                */
     SS2D_ERR_ALLOC = -7,  /* device memory for scratch or staging ran out    */
     SS2D_ERR_CUDA = -8,   /* a CUDA call failed; see ss2d_last_error()       */

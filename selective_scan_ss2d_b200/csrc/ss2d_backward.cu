@@ -29,7 +29,9 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
         c.B = p.B;
         c.D = p.D;
         c.K = p.K;
-        c.N = p.N;
+        c.N = p.N;      // this state group's states, rows n0.. of A_log
+        c.n0 = p.n0;
+        c.NS = p.NS;
         c.L = p.L;
         c.NC = p.NC;
         const long long total = (long long)p.B * p.K * p.D * kNP;
@@ -73,31 +75,45 @@ BwdShape backward_shape(int B, int D, int L, int K)
 
 cudaError_t launch_backward(const BwdParams &p, int dtype, cudaStream_t st)
 {
-    switch (dtype) {
-    case 1:
-        return launch_bwd_t<__nv_bfloat16>(p, st);
-    case 2:
-        return launch_bwd_t<__half>(p, st);
-    default:
-        return launch_bwd_t<float>(p, st);
+    // more than 16 states: the passes once per group of at most 16, in order
+    // on the stream, later groups adding to the first group's rows
+    const int ns = p.NS;
+    cudaError_t e = cudaSuccess;
+    for (int n0 = 0; n0 < ns && e == cudaSuccess; n0 += kNP) {
+        BwdParams q = p;
+        q.n0 = n0;
+        q.N = ns - n0 < kNP ? ns - n0 : kNP;
+        q.accum = n0 > 0 ? 1 : 0;
+        switch (dtype) {
+        case 1:
+            e = launch_bwd_t<__nv_bfloat16>(q, st);
+            break;
+        case 2:
+            e = launch_bwd_t<__half>(q, st);
+            break;
+        default:
+            e = launch_bwd_t<float>(q, st);
+            break;
+        }
     }
+    return e;
 }
 
 cudaError_t launch_backward_reduce(const BwdParams &p, float *dBs, float *dCs, float *dA_log,
                                    float *dDskip, float *ddelta_bias, cudaStream_t st)
 {
-    const long long nbc = (long long)p.B * p.K * 2 * p.N * p.L;
+    const long long nbc = (long long)p.B * p.K * 2 * p.NS * p.L;
     long long blocks = (nbc + 255) / 256;
     if (blocks > 148LL * 64)
         blocks = 148LL * 64;
     bwd_reduce_bc_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.bc_part, dBs, dCs, p.B * p.K, p.G,
-                                                          p.N, p.L);
-    const long long npr = (long long)p.K * p.D * (p.N + 2);
+                                                          p.NS, p.L);
+    const long long npr = (long long)p.K * p.D * (p.NS + 2);
     blocks = (npr + 127) / 128;
     if (blocks > 148LL * 64)
         blocks = 148LL * 64;
     bwd_reduce_param_kernel<<<(unsigned)blocks, 128, 0, st>>>(p.prm_part, p.A_log, dA_log, dDskip,
-                                                             ddelta_bias, p.B, p.K, p.D, p.N,
+                                                             ddelta_bias, p.B, p.K, p.D, p.NS,
                                                              p.CGN);
     return cudaGetLastError();
 }

@@ -97,7 +97,8 @@ struct BwdRaw {
         const int lane = threadIdx.x;
         const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
         const bool nok = n < p.N;
-        const size_t row = (((size_t)q.b * p.K + q.k) * p.N + (nok ? n : 0)) * p.L + s + t0;
+        const size_t row =
+            (((size_t)q.b * p.K + q.k) * p.NS + p.n0 + (nok ? n : 0)) * p.L + s + t0;
         const RawT *Bp = static_cast<const RawT *>(p.Bs) + row;
         const RawT *Cp = static_cast<const RawT *>(p.Cs) + row;
 #pragma unroll
@@ -189,8 +190,9 @@ __device__ __forceinline__ void load_a2(float2 *A2, const BwdParams &p, size_t k
 #pragma unroll
     for (int j = 0; j < kNP / 2; ++j) {
         const int n0 = 2 * j, n1 = 2 * j + 1;
-        A2[j].x = n0 < p.N ? -expf(__ldg(p.A_log + kd * p.N + n0)) * kLog2e : 0.f;
-        A2[j].y = n1 < p.N ? -expf(__ldg(p.A_log + kd * p.N + n1)) * kLog2e : 0.f;
+        const float *al = p.A_log + kd * p.NS + p.n0;
+        A2[j].x = n0 < p.N ? -expf(__ldg(al + n0)) * kLog2e : 0.f;
+        A2[j].y = n1 < p.N ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
     }
 }
 // one step of the state recurrence, h = exp(dt A) h + dt u B, for all pairs
@@ -309,13 +311,14 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
     float2 A2[kNP / 2];
     load_a2(A2, p, kd);
     const float bias = __ldg(p.delta_bias + kd);
-    const float Dk = __ldg(p.Dskip + kd);
+    const bool accum = p.accum != 0;   // a later state group: add to the rows
+    const float Dk = accum ? 0.f : __ldg(p.Dskip + kd);
     const int L = p.L, nc1 = p.NC - 1;
     const bool flip = p.flip1 && q.k == 1;
     float *durow = p.du + q.bkd * L;
     float *ddrow = p.ddelta + q.bkd * L;
-    float *bcrow = p.bc_part +
-                   ((((size_t)q.bk * p.G + q.gi) * 2 + (lane >> 4)) * kNP + (lane & 15)) * L;
+    float *bcrow = p.bc_part + ((((size_t)q.bk * p.G + q.gi) * 2 + (lane >> 4)) * p.NS + p.n0 +
+                                (lane & 15)) * L;
     const bool bc_ok = (lane & 15) < p.N;
     // rows of L floats: 16-byte segments at 16-step chunk starts when L % 4 == 0
     // (the scratch and gradient buffers are 16-byte aligned)
@@ -430,6 +433,13 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
         // reduced dB | dC row this lane holds (16-byte segments when whole)
         const bool whole = nt == kT && vec_rows;
         if (q.active) {
+            auto put4 = [&](float4 *dst, float4 v) {
+                if (accum) {
+                    const float4 e = *dst;
+                    v = make_float4(e.x + v.x, e.y + v.y, e.z + v.z, e.w + v.w);
+                }
+                *dst = v;
+            };
             if (whole) {
                 float4 *dd4 = reinterpret_cast<float4 *>(ddrow + s);
                 float4 *du4 = reinterpret_cast<float4 *>(durow + (flip ? L - kT - s : s));
@@ -439,18 +449,19 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
                     const float4 b = st4[(4 * i + 1) * kBwdLanes + lane];
                     const float4 c4 = st4[(4 * i + 2) * kBwdLanes + lane];
                     const float4 d4 = st4[(4 * i + 3) * kBwdLanes + lane];
-                    dd4[i] = make_float4(a.x, b.x, c4.x, d4.x);
+                    put4(dd4 + i, make_float4(a.x, b.x, c4.x, d4.x));
                     if (flip)
-                        du4[kT / 4 - 1 - i] = make_float4(d4.y, c4.y, b.y, a.y);
+                        put4(du4 + (kT / 4 - 1 - i), make_float4(d4.y, c4.y, b.y, a.y));
                     else
-                        du4[i] = make_float4(a.y, b.y, c4.y, d4.y);
+                        put4(du4 + i, make_float4(a.y, b.y, c4.y, d4.y));
                 }
             } else {
                 for (int t = 0; t < nt; ++t) {
                     const float4 r = st4[t * kBwdLanes + lane];
                     const int l = s + t;
-                    ddrow[l] = r.x;
-                    durow[flip ? L - 1 - l : l] = r.y;
+                    float *o = durow + (flip ? L - 1 - l : l);
+                    ddrow[l] = accum ? ddrow[l] + r.x : r.x;
+                    *o = accum ? *o + r.y : r.y;
                 }
             }
         }
@@ -470,18 +481,27 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
         }
     }
     if (q.active) {
-        float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * kPrm;
+        // slots: dA of the call's NS states, dDskip, dbias; a later state group
+        // writes its own dA and adds its share of dbias (same thread, later launch)
+        float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * (p.NS + 2);
 #pragma unroll
         for (int j = 0; j < kNP / 2; ++j) {
-            pr[2 * j] = dA[j].x;
-            pr[2 * j + 1] = dA[j].y;
+            if (2 * j < p.N)
+                pr[p.n0 + 2 * j] = dA[j].x;
+            if (2 * j + 1 < p.N)
+                pr[p.n0 + 2 * j + 1] = dA[j].y;
         }
-        pr[kNP] = dD;
-        pr[kNP + 1] = db;
+        if (!accum) {
+            pr[p.NS] = dD;
+            pr[p.NS + 1] = db;
+        } else {
+            pr[p.NS + 1] += db;
+        }
     }
 }
 
-// dBs, dCs (B,K,N,L) = the sum over the channel groups, in group order
+// dBs, dCs (B,K,N,L) = the sum over the channel groups, in group order (the
+// partial holds N rows per (b, k, group, B|C))
 __global__ void bwd_reduce_bc_kernel(const float *__restrict__ part, float *__restrict__ dBs,
                                      float *__restrict__ dCs, int BK, int G, int N, int L)
 {
@@ -494,8 +514,8 @@ __global__ void bwd_reduce_bc_kernel(const float *__restrict__ part, float *__re
         r /= N;
         const int which = (int)(r & 1);
         const long long bk = r >> 1;
-        const float *src = part + (((size_t)bk * G * 2 + which) * kNP + n) * L + l;
-        const size_t gstride = (size_t)2 * kNP * L;
+        const float *src = part + (((size_t)bk * G * 2 + which) * N + n) * L + l;
+        const size_t gstride = (size_t)2 * N * L;
         float s = 0.f;
         for (int g = 0; g < G; ++g)
             s += __ldg(src + g * gstride);
@@ -516,12 +536,11 @@ __global__ void bwd_reduce_param_kernel(const float *__restrict__ prm,
         const int j = (int)(i % (N + 2));
         const long long kd = i / (N + 2);
         const int k = (int)(kd / D), d = (int)(kd % D);
-        const int jj = j < N ? j : (j == N ? kNP : kNP + 1);
         float s = 0.f;
         for (int b = 0; b < B; ++b) {
-            const float *src = prm + ((((size_t)b * K + k) * D + d) * CGN) * kPrm + jj;
+            const float *src = prm + ((((size_t)b * K + k) * D + d) * CGN) * (N + 2) + j;
             for (int cg = 0; cg < CGN; ++cg)
-                s += __ldg(src + (size_t)cg * kPrm);
+                s += __ldg(src + (size_t)cg * (N + 2));
         }
         if (j < N)
             dA_log[kd * N + j] = s * -expf(__ldg(A_log + kd * N + j));

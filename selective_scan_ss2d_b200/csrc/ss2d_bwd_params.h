@@ -16,16 +16,19 @@ struct BwdParams {
     float *dta;        // (B,K,D,NC-1): sum of dt of chunks NC-1..1
     float *du;         // du rows (direction 1 in pixel order when flip1); dx itself when K = 1
     float *ddelta;     // (B,K,D,L) float32, scan order
-    float *bc_part;    // (B,K,G,2,16,L): dB | dC summed over one group of 32 channels
-    float *prm_part;   // (B,K,D,CGN,kPrm): dA (natural A), dDskip, dbias per chunk group
+    float *bc_part;    // (B,K,G,2,NS,L): dB | dC summed over one group of 32 channels
+    float *prm_part;   // (B,K,D,CGN,NS+2): dA (natural A), dDskip, dbias per chunk group
     int B, D, H, W, L, N, K, two_d;
     int NC;            // chunks of kT steps
     int G;             // channel groups of 32
     int CPB;           // chunks per CTA
     int CGN;           // chunk groups (gridDim.y)
     int flip1;         // store direction 1's du in pixel order (the merge's layout)
+    // state groups (more than 16 states): N is this group's count
+    int n0;            // first state of this group
+    int NS;            // states per row of A_log, Bs, Cs (the call's N)
+    int accum;         // 1: add ddelta, du to the rows (no skip term, no dDskip)
 };
 
 constexpr int kBwdLanes = 32;
-constexpr int kPrm = kNP + 2;
 }  // namespace ss2d

@@ -346,8 +346,6 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     int rc = validate(pr);
     if (rc != SS2D_OK)
         return rc;
-    if (pr.N > ss2d::kNP)
-        return SS2D_ERR_N;   // the backward keeps all states of a channel in one lane
     if (pr.K * (long long)pr.D == 0)
         return SS2D_OK;
     // an empty batch or sequence reads nothing and writes only the parameter
@@ -399,8 +397,8 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     const size_t ds_bytes = align256(sizeof(float) * rows * nc1);
     const size_t du_bytes = pr.K > 1 ? align256(sizeof(float) * rows * L) : 0;
     const size_t bc_bytes =
-        align256(sizeof(float) * pr.B * pr.K * (size_t)sh.G * 2 * ss2d::kNP * L);
-    const size_t pr_bytes = align256(sizeof(float) * rows * sh.CGN * ss2d::kPrm);
+        align256(sizeof(float) * pr.B * pr.K * (size_t)sh.G * 2 * pr.N * L);
+    const size_t pr_bytes = align256(sizeof(float) * rows * sh.CGN * (pr.N + 2));
     const size_t total = 2 * hs_bytes + 2 * ds_bytes + du_bytes + bc_bytes + pr_bytes;
     void *scratch = nullptr;
     rc = pool_alloc(&scratch, total, st);
@@ -443,6 +441,7 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     p.CPB = sh.CPB;
     p.CGN = sh.CGN;
     p.flip1 = pr.K > 1 ? 1 : 0;
+    p.NS = pr.N;
     e = ss2d::launch_backward(p, pr.dtype, st);
     if (e == cudaSuccess && pr.K > 1)
         e = ss2d::launch_merge(p.du, gr.dx, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d, 1, st);

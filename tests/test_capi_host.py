@@ -148,7 +148,6 @@ def test_backward_argument_errors_are_reported_without_cuda(lib):
     assert _bwd_call(lib, aligned, dtype=9) == -3
     assert _bwd_call(lib, aligned, K=3) == -4
     assert _bwd_call(lib, aligned, K=4, two_d=False) == -4
-    assert _bwd_call(lib, aligned, N=17) == -5   # the backward keeps N <= 16
     assert _bwd_call(lib, aligned, N=65) == -5
     for i in (0, 7, 8, 14):   # x, dy, dx, ddelta_bias
         assert _bwd_call(lib, aligned, nulls=(i,)) == -1

@@ -82,6 +82,19 @@ def test_backward_matches_oracle(cfg, dtype):
     assert_grads_close(gpu_backward(inp, dy), oracle_backward(inp, dy), cfg.name)
 
 
+@pytest.mark.parametrize("cfg", SHAPES + [small(B=2, D=12, H=7, W=9, N=20),
+                                          small(B=1, D=40, H=14, W=14, N=40),
+                                          small(B=2, D=9, H=6, W=5, K=2, N=64),
+                                          small("1d", B=3, D=20, W=197, K=2, N=33)],
+                         ids=lambda c: c.name)
+def test_backward_row_parameters_and_state_groups(cfg):
+    """A_log and Dskip different in every row (k, d), and state counts above
+    16 (groups of 16 states run one after the other)."""
+    inp = _gpu.vary_params(wl.make_inputs(cfg, seed=13), seed=13)
+    dy = wl.make_cotangent(cfg, seed=13)
+    assert_grads_close(gpu_backward(inp, dy), oracle_backward(inp, dy), cfg.name + " varied")
+
+
 def test_backward_large_dt():
     """dt of order one (delta_bias = 0), where every term of the gradient,
     the decay terms included, carries weight."""

@@ -396,13 +396,26 @@ def test_more_than_16_states_full_size_sampled():
         _gpu.assert_close(y[b:b + 1, d:d + 1], _gpu.run_oracle(sub), cfg.dtype, f"N=32 ({b},{d})")
 
 
-def test_backward_rejects_more_than_16_states():
-    inp = wl.make_inputs(small(B=1, D=4, H=4, W=4, N=20), seed=0)
+VARIED = [small(B=2, D=40, H=7, W=9), small(B=1, D=24, H=14, W=14, K=2),
+          small(B=1, D=8, H=33, W=31, N=24), small(B=2, D=9, H=6, W=5, K=1, N=8),
+          small("1d", B=3, D=20, W=197, K=2), small("1d", B=2, D=7, W=50, K=1, N=40)]
+
+
+@pytest.mark.parametrize("cfg", VARIED, ids=lambda c: c.name)
+def test_row_parameters_are_read_per_row(cfg):
+    """A_log and Dskip different in every row (k, d): every variant, final
+    states included, against the oracle."""
+    inp = _gpu.vary_params(wl.make_inputs(cfg, seed=12), seed=12)
+    ref = _gpu.run_oracle(inp)
+    href = _final_oracle(inp)
     t = _gpu.tensors(inp)
-    with pytest.raises(binding.SS2DError) as ei:
-        binding.ss2d_backward(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"],
-                              t["delta_bias"], torch.zeros((1, 4, 4, 4), device="cuda"))
-    assert ei.value.status == -5
+    args = [t[n] for n in ("x", "delta", "A_log", "Bs", "Cs", "Dskip", "delta_bias")]
+    for v in [-1] + list(range(nvariants())):
+        _gpu.assert_close(_gpu.run_gpu(inp, variant=v, t=t), ref, cfg.dtype, f"{cfg.name} v{v}")
+        _, h = binding.forward_final_state(*args, variant=v)
+        torch.cuda.synchronize()
+        _gpu.assert_close(h.cpu().numpy().astype(np.float64), href, cfg.dtype,
+                          f"{cfg.name} v{v} final state")
 
 
 @pytest.mark.parametrize("name", ["vmamba_t_stage1", "vim_s_bidir"])
