@@ -39,9 +39,11 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
         c.hstate = p.hfwd;
         c.dtsum = p.dtf;
         carry_kernel<<<cgrid, 256, 0, st>>>(c);
-        c.hstate = p.hadj;
-        c.dtsum = p.dta;
-        carry_kernel<<<cgrid, 256, 0, st>>>(c);
+        if (p.adj_chunks) {
+            c.hstate = p.hadj;
+            c.dtsum = p.dta;
+            carry_kernel<<<cgrid, 256, 0, st>>>(c);
+        }
         e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;

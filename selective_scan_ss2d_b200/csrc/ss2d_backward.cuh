@@ -22,7 +22,10 @@
 //   2. carry_kernel (the forward's) run twice gives the entry state of every
 //      chunk and, over the reversed order, the adjoint G[c] = a_{e+1} g_{e+1}
 //      entering every chunk from its end: G[c-1] = exp(A sum_c dt) G[c] + Q[c].
-//   3. bwd_final_kernel: per chunk, h recomputed from its entry state (the
+//      The final pass needs G only at the top of each CTA's range of chunks;
+//      when one range covers a whole sequence, Q and its carry are skipped.
+//   3. bwd_final_kernel: per chunk, in descending order, h recomputed from
+//      its entry state (the
 //      16 states of 8 steps of every lane parked in shared memory at a time:
 //      the chunk is walked back in two halves), then the reverse walk from
 //      G[c] writes ddelta and du, reduces dB and dC over
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
                 p.dtf[q.bkd * nc1 + c] = dts;
             }
         }
-        if (c > 0) {
+        if (c > 0 && p.adj_chunks) {
             float2 g[kNP / 2];
 #pragma unroll
             for (int j = 0; j < kNP / 2; ++j)
@@ -329,15 +332,19 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
         dA[j] = make_float2(0.f, 0.f);
     float dD = 0.f, db = 0.f;
     const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
+    // The chunks of the range in descending order: the walk back over chunk c
+    // ends with g = a_s g_s, the adjoint entering chunk c - 1 at its end, so
+    // only the range's top chunk takes its adjoint from the carry.
+    float2 g[kNP / 2];
     BwdRaw<Tin> raw;
-    raw.fetch(p, q, c0 * kT);
-    for (int c = c0; c < c1; ++c) {
+    raw.fetch(p, q, (c1 - 1) * kT);
+    for (int c = c1 - 1; c >= c0; --c) {
         const int s = c * kT, nt = min(kT, L - s);
         __syncwarp();
         raw.commit(sB, sC, st4, bias, q.active);
         __syncwarp();
-        if (c + 1 < c1)
-            raw.fetch(p, q, (c + 1) * kT);   // in flight during this chunk's work
+        if (c - 1 >= c0)
+            raw.fetch(p, q, (c - 1) * kT);   // in flight during this chunk's work
         // The chunk in two halves of 8 steps, so that only half of its states
         // are parked at a time: the first recompute runs the whole chunk from
         // the entry state and parks steps 8..15 for the walk back over them;
@@ -364,7 +371,6 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
                 }
             }
         };
-        float2 g[kNP / 2];
         auto walk_back = [&](int t_hi, int base) {
 #pragma unroll 2
             for (int t = t_hi; t >= base; --t) {
@@ -410,13 +416,17 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
                 }
             }
         };
-        // the adjoint entering at the chunk end
-        if (c < nc1)
-            load16(reinterpret_cast<float *>(g), p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
-        else
+        // the adjoint entering the range's top chunk at its end (zero for the
+        // sequence's last chunk)
+        if (c == c1 - 1) {
+            if (c < nc1)
+                load16(reinterpret_cast<float *>(g),
+                       p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
+            else
 #pragma unroll
-            for (int j = 0; j < kNP / 2; ++j)
-                g[j] = make_float2(0.f, 0.f);
+                for (int j = 0; j < kNP / 2; ++j)
+                    g[j] = make_float2(0.f, 0.f);
+        }
         {
             float2 h[kNP / 2];
             entry(h);

@@ -28,6 +28,7 @@ struct BwdParams {
     int n0;            // first state of this group
     int NS;            // states per row of A_log, Bs, Cs (the call's N)
     int accum;         // 1: add ddelta, du to the rows (no skip term, no dDskip)
+    int adj_chunks;    // 1: local adjoints and their carry are needed (CGN > 1)
 };
 
 constexpr int kBwdLanes = 32;

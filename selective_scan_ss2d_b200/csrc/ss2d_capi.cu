@@ -442,6 +442,7 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     p.CGN = sh.CGN;
     p.flip1 = pr.K > 1 ? 1 : 0;
     p.NS = pr.N;
+    p.adj_chunks = sh.CGN > 1 ? 1 : 0;
     e = ss2d::launch_backward(p, pr.dtype, st);
     if (e == cudaSuccess && pr.K > 1)
         e = ss2d::launch_merge(p.du, gr.dx, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d, 1, st);

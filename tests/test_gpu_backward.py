@@ -95,6 +95,19 @@ def test_backward_row_parameters_and_state_groups(cfg):
     assert_grads_close(gpu_backward(inp, dy), oracle_backward(inp, dy), cfg.name + " varied")
 
 
+@pytest.mark.parametrize("cfg", [small(B=8, D=1024, H=16, W=16, K=4, N=16),
+                                 small(B=24, D=1024, H=6, W=8, K=4, N=16)],
+                         ids=["ranges_of_6_chunks", "one_range_per_sequence"])
+def test_backward_chunk_ranges(cfg):
+    """Enough channels that a CTA walks several chunks (the adjoint carried
+    from chunk to chunk inside the kernel, G from the carry only at the top
+    of each range), and so many that one range covers a whole sequence (no
+    local adjoints, no adjoint carry)."""
+    inp = _gpu.vary_params(wl.make_inputs(cfg, seed=14), seed=14)
+    dy = wl.make_cotangent(cfg, seed=14)
+    assert_grads_close(gpu_backward(inp, dy), oracle_backward(inp, dy), cfg.name)
+
+
 def test_backward_large_dt():
     """dt of order one (delta_bias = 0), where every term of the gradient,
     the decay terms included, carries weight."""
