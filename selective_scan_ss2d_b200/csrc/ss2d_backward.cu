@@ -48,7 +48,13 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
         if (e != cudaSuccess)
             return e;
     }
-    bwd_final_kernel<Tin><<<grid, kBwdLanes, kBwdFinalSmem, st>>>(p);
+    // the final pass: 4 warps per channel group, 4 states each
+    auto kern = bwd_final4_kernel<Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kBwd4Smem);
+    if (e != cudaSuccess)
+        return e;
+    kern<<<grid, kBwd4Threads, kBwd4Smem, st>>>(p);
     return cudaGetLastError();
 }
 }  // namespace

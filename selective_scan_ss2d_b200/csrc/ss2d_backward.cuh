@@ -13,8 +13,9 @@
 // dDskip the sums over (b, t), and dx gathers du of every direction back to
 // its pixel (the adjoint of cross_scan is cross_merge).
 //
-// Work decomposition: chunks of kT = 16 steps; a CTA is one warp holding 32
-// channels of one (b, k) and walks a range of chunks.
+// Work decomposition: chunks of kT = 16 steps; a CTA holds 32 channels of one
+// (b, k) (one warp for the local pass, four for the final pass) and walks a
+// range of chunks.
 //   1. bwd_local_kernel: per chunk, from zero, the forward end state h_end[c]
 //      and the local adjoint Q[c] = a_s g_s (g from zero at the chunk end),
 //      each with the chunk's sum of dt.  Q is stored in reversed chunk
@@ -24,13 +25,14 @@
 //      entering every chunk from its end: G[c-1] = exp(A sum_c dt) G[c] + Q[c].
 //      The final pass needs G only at the top of each CTA's range of chunks;
 //      when one range covers a whole sequence, Q and its carry are skipped.
-//   3. bwd_final_kernel: per chunk, in descending order, h recomputed from
-//      its entry state (the
-//      16 states of 8 steps of every lane parked in shared memory at a time:
-//      the chunk is walked back in two halves), then the reverse walk from
-//      G[c] writes ddelta and du, reduces dB and dC over
-//      the warp's channels (one reduce-scatter of 32 values per step) into a
-//      per-channel-group partial, and accumulates the parameter gradients.
+//   3. bwd_final4_kernel (4 warps per CTA, warp w holding states 4w..4w+3 of
+//      the same 32 channels): per chunk of its range, in descending order
+//      (the walk back over a chunk ends with the adjoint entering the chunk
+//      below), each warp recomputes its states from the entry state and
+//      parks them in shared memory, then walks back from G[c] reducing
+//      dB | dC of its states over the channels (9 shuffles per step) and
+//      accumulating dA; the per-step sums over all 16 states that du and
+//      ddelta need are combined through shared memory once per chunk.
 //   4. merge2_kernel (K > 1) sums du of the directions into dx; two fixed-order
 //      reductions finish dBs, dCs and dA_log, dDskip, ddelta_bias.
 // Every reduction runs in a fixed order: the result is reproducible.
@@ -43,15 +45,9 @@ namespace ss2d {
 
 constexpr float kLn2 = 0.6931471805599453f;
 
-// shared memory of both kernels (floats): B and C of the chunk [t][n], and the
-// lanes' staged (dt, u, dy, sigmoid(delta + bias)) as float4 [t][lane]
+// shared memory of the local pass (floats): B and C of the chunk [t][n], and
+// the lanes' staged (dt, u, dy, sigmoid(delta + bias)) as float4 [t][lane]
 constexpr int kBwdStage = 2 * kT * kNP + 4 * kT * kBwdLanes;
-// the final kernel adds the recomputed states of half a chunk, float4
-// [t][lane][4] with the float4 index XOR-swizzled by (lane >> 1) & 3 (no bank
-// conflicts for the lanes' 16-byte accesses)
-constexpr int kHalf = kT / 2;
-constexpr int kBwdStates = kHalf * kNP * kBwdLanes;
-constexpr size_t kBwdFinalSmem = sizeof(float) * (kBwdStage + kBwdStates);
 
 struct BwdLane {
     int b, k, gi, d, bk;
@@ -62,7 +58,7 @@ struct BwdLane {
 __device__ __forceinline__ BwdLane bwd_lane(const BwdParams &p)
 {
     BwdLane r;
-    const int lane = threadIdx.x;
+    const int lane = threadIdx.x & 31;
     r.gi = (int)(blockIdx.x % (unsigned)p.G);
     r.bk = (int)(blockIdx.x / (unsigned)p.G);
     r.b = r.bk / p.K;
@@ -154,19 +150,6 @@ struct BwdRaw {
         }
     }
 };
-
-__device__ __forceinline__ void load16(float *v, const float *src)
-{
-    const float4 *s4 = reinterpret_cast<const float4 *>(src);
-#pragma unroll
-    for (int i = 0; i < kNP / 4; ++i) {
-        const float4 a = s4[i];
-        v[4 * i] = a.x;
-        v[4 * i + 1] = a.y;
-        v[4 * i + 2] = a.z;
-        v[4 * i + 3] = a.w;
-    }
-}
 
 __device__ __forceinline__ void store16(float *dst, const float *v)
 {
@@ -273,239 +256,327 @@ __global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
     }
 }
 
-// One halving exchange: lanes with bit M set keep v[M..2M) (moved to v[0..M)),
-// the others v[0..M); each adds the half its partner sends.
-template <int M>
-__device__ __forceinline__ void halve(float *v)
+// ---------------------------------------------------------------------------
+// The final pass with the 16 states of a channel group split over 4 warps
+// (warp w: states 4w .. 4w+3 of the same 32 channels).  A warp parks the
+// states of a whole chunk (8 KB), so a chunk is recomputed once; dB | dC of
+// its 4 states reduce over the channels with 9 shuffles per step; the sums
+// over all 16 states that du and ddelta need are combined through shared
+// memory once per chunk, each warp finishing 4 of the 16 steps.
+constexpr int kQuadWarps = 4;
+constexpr int kBwd4Threads = kQuadWarps * kBwdLanes;
+constexpr int kBwd4Stage = 2 * kT * kNP + 4 * kT * kBwdLanes;   // B|C tiles, st4
+constexpr int kBwd4Hs = kQuadWarps * kT * kBwdLanes * 4;         // per warp [t][lane] float4
+constexpr int kBwd4Sums = kQuadWarps * kT * kBwdLanes * 2;       // per warp [t][lane] (s1, s2)
+constexpr int kBwd4Red = kQuadWarps * kT * 8;                    // per warp [t][8] reduced dB|dC
+constexpr size_t kBwd4Smem = sizeof(float) * (kBwd4Stage + kBwd4Hs + kBwd4Sums + kBwd4Red);
+
+// lanes with bit OFF set keep v[H..2H) (moved to v[0..H)), the others v[0..H)
+template <int H, int OFF>
+__device__ __forceinline__ void halve_at(float *v)
 {
-    const bool hi = (threadIdx.x & M) != 0;
+    const bool hi = (threadIdx.x & OFF) != 0;
 #pragma unroll
-    for (int i = 0; i < M; ++i) {
-        const float lo = v[i], up = v[i + M];
+    for (int i = 0; i < H; ++i) {
+        const float lo = v[i], up = v[i + H];
         const float send = hi ? lo : up;
         const float keep = hi ? up : lo;
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
     }
 }
 
-// Sum over the 32 lanes of v[j] for j = lane (v[0..15]: dB of the 16 states,
-// v[16..31]: dC): five halving exchanges, 31 shuffles.
-__device__ __forceinline__ float reduce_scatter32(float *v)
+// Sum over the 32 lanes of v[j], j = (lane >> 2) (v[0..3]: dB, v[4..7]: dC of
+// the warp's 4 states): three halvings over lane bits 4, 3, 2, then a
+// butterfly over bits 1, 0; 9 shuffles.
+__device__ __forceinline__ float reduce_scatter8(float *v)
 {
-    halve<16>(v);
-    halve<8>(v);
-    halve<4>(v);
-    halve<2>(v);
-    halve<1>(v);
-    return v[0];
+    halve_at<4, 16>(v);
+    halve_at<2, 8>(v);
+    halve_at<1, 4>(v);
+    float r = v[0];
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    return r;
 }
 
+// The raw inputs of one chunk, the staging split over the CTA's 128 threads:
+// 4 of the 512 B|C values, and 4 steps (4w .. 4w+3) of the lane's channel.
 template <typename Tin>
-__global__ void __launch_bounds__(kBwdLanes) bwd_final_kernel(const BwdParams p)
+struct BwdRaw4 {
+    using RawT = std::conditional_t<sizeof(Tin) == 2, unsigned short, float>;
+    RawT bc[4], dl[4], x[4];
+    float gy[4];
+    int nt;
+
+    __device__ __forceinline__ static float f32(RawT v)
+    {
+        if constexpr (sizeof(Tin) == 2)
+            return half_bits_to_f32<Tin>(v);
+        else
+            return v;
+    }
+
+    __device__ __forceinline__ void fetch(const BwdParams &p, const BwdLane &q, int s)
+    {
+        nt = min(kT, p.L - s);
+        const int tid = threadIdx.x, w = tid >> 5;
+        const size_t bkrow = ((size_t)q.b * p.K + q.k) * p.NS + p.n0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int item = tid + i * kBwd4Threads;   // 0..511: (B|C, n, t)
+            const int which = item >> 8, n = (item >> 4) & 15, t = item & 15;
+            const bool ok = n < p.N && t < nt;
+            const RawT *src = static_cast<const RawT *>(which ? p.Cs : p.Bs);
+            bc[i] = ok ? __ldg(src + (bkrow + n) * p.L + s + t) : RawT(0);
+        }
+        const RawT *dp = static_cast<const RawT *>(p.delta) + q.bkd * p.L + s;
+        const size_t xrow = ((size_t)q.b * p.D + q.d) * p.L;
+        const RawT *xp = static_cast<const RawT *>(p.x) + xrow;
+        const float *gp = p.dy + xrow;
+        PixWalk pw;
+        pw.init(p.two_d, q.k, min(s + 4 * w, p.L - 1), p.H, p.W, p.L);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * w + i;
+            const bool ok = t < nt && q.active;   // idle lanes add nothing to dB, dC
+            dl[i] = ok ? __ldg(dp + t) : RawT(0);
+            x[i] = ok ? __ldg(xp + pw.p) : RawT(0);
+            gy[i] = ok ? __ldg(gp + pw.p) : 0.f;
+            if (t + 1 < nt)
+                pw.next(p.H, p.W);
+        }
+    }
+
+    __device__ __forceinline__ void commit(float *sB, float *sC, float4 *st4, float bias,
+                                           bool active) const
+    {
+        const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int item = tid + i * kBwd4Threads;
+            const int which = item >> 8, n = (item >> 4) & 15, t = item & 15;
+            (which ? sC : sB)[t * kNP + n] = f32(bc[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * w + i;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < nt && active) {
+                const float z = f32(dl[i]) + bias;
+                v.x = softplus_f(z);
+                v.y = f32(x[i]);
+                v.z = gy[i];
+                v.w = __fdividef(1.f, 1.f + mufu_ex2(-z * kLog2e));   // sigmoid(z)
+            }
+            st4[t * kBwdLanes + lane] = v;
+        }
+    }
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParams p)
 {
-    extern __shared__ float4 smem_bwd4[];
-    float *sB = reinterpret_cast<float *>(smem_bwd4), *sC = sB + kT * kNP;
-    float4 *st4 = smem_bwd4 + 2 * kT * kNP / 4;
-    float4 *hs4 = st4 + kT * kBwdLanes;   // [t][lane][4 float4], half a chunk
-    const int lane = threadIdx.x;
-    const int swz = (lane >> 1) & 3;
+    extern __shared__ float4 smem_b4[];
+    float *sB = reinterpret_cast<float *>(smem_b4), *sC = sB + kT * kNP;
+    float4 *st4 = smem_b4 + 2 * kT * kNP / 4;                       // [t][lane]
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    float4 *hs = st4 + kT * kBwdLanes + w * kT * kBwdLanes;           // this warp's [t][lane]
+    float2 *sums = reinterpret_cast<float2 *>(st4 + kT * kBwdLanes + kQuadWarps * kT * kBwdLanes);
+    float *red = reinterpret_cast<float *>(sums + kQuadWarps * kT * kBwdLanes) + w * kT * 8;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
-    float2 A2[kNP / 2];
-    load_a2(A2, p, kd);
+    const int nw = 4 * w;   // this warp's first state within the group
+    float2 A2[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float *al = p.A_log + kd * p.NS + p.n0 + nw;
+        A2[j].x = nw + 2 * j < p.N ? -expf(__ldg(al + 2 * j)) * kLog2e : 0.f;
+        A2[j].y = nw + 2 * j + 1 < p.N ? -expf(__ldg(al + 2 * j + 1)) * kLog2e : 0.f;
+    }
     const float bias = __ldg(p.delta_bias + kd);
-    const bool accum = p.accum != 0;   // a later state group: add to the rows
+    const bool accum = p.accum != 0;
     const float Dk = accum ? 0.f : __ldg(p.Dskip + kd);
     const int L = p.L, nc1 = p.NC - 1;
     const bool flip = p.flip1 && q.k == 1;
     float *durow = p.du + q.bkd * L;
     float *ddrow = p.ddelta + q.bkd * L;
-    float *bcrow = p.bc_part + ((((size_t)q.bk * p.G + q.gi) * 2 + (lane >> 4)) * p.NS + p.n0 +
-                                (lane & 15)) * L;
-    const bool bc_ok = (lane & 15) < p.N;
-    // rows of L floats: 16-byte segments at 16-step chunk starts when L % 4 == 0
-    // (the scratch and gradient buffers are 16-byte aligned)
     const bool vec_rows = (L & 3) == 0;
-    float2 dA[kNP / 2];
-#pragma unroll
-    for (int j = 0; j < kNP / 2; ++j)
-        dA[j] = make_float2(0.f, 0.f);
+    // the reduced row this lane writes (lanes 0..7 of each warp: j = lane)
+    const int rj = lane & 7;
+    const bool bc_ok = lane < 8 && nw + (rj & 3) < p.N;
+    float *bcrow = p.bc_part + ((((size_t)q.bk * p.G + q.gi) * 2 + (rj >> 2)) * p.NS + p.n0 +
+                                nw + (rj & 3)) * L;
+    float2 dA[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float dD = 0.f, db = 0.f;
     const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
-    // The chunks of the range in descending order: the walk back over chunk c
-    // ends with g = a_s g_s, the adjoint entering chunk c - 1 at its end, so
-    // only the range's top chunk takes its adjoint from the carry.
-    float2 g[kNP / 2];
-    BwdRaw<Tin> raw;
+    // chunks in descending order: the adjoint flows from chunk to chunk
+    float2 g[2];
+    BwdRaw4<Tin> raw;
     raw.fetch(p, q, (c1 - 1) * kT);
     for (int c = c1 - 1; c >= c0; --c) {
         const int s = c * kT, nt = min(kT, L - s);
-        __syncwarp();
+        __syncthreads();   // every warp is done with the previous chunk's tiles
         raw.commit(sB, sC, st4, bias, q.active);
-        __syncwarp();
+        __syncthreads();
         if (c - 1 >= c0)
             raw.fetch(p, q, (c - 1) * kT);   // in flight during this chunk's work
-        // The chunk in two halves of 8 steps, so that only half of its states
-        // are parked at a time: the first recompute runs the whole chunk from
-        // the entry state and parks steps 8..15 for the walk back over them;
-        // the second recomputes steps 0..7 from the entry state again.
-        auto entry = [&](float2 *h) {
-            if (c > 0)
-                load16(reinterpret_cast<float *>(h), p.hfwd + (q.bkd * nc1 + (c - 1)) * kNP);
-            else
-#pragma unroll
-                for (int j = 0; j < kNP / 2; ++j)
-                    h[j] = make_float2(0.f, 0.f);
-        };
-        auto recompute = [&](float2 *h, int t1, int park0) {
-#pragma unroll 1
-            for (int t = 0; t < t1; ++t) {
-                const float4 v = st4[t * kBwdLanes + lane];
-                state_step(h, A2, v.x, v.x * v.y, sB + t * kNP);
-                if (t >= park0) {
-                    float4 *row = hs4 + ((t - park0) * kBwdLanes + lane) * 4;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        row[j ^ swz] = make_float4(h[2 * j].x, h[2 * j].y, h[2 * j + 1].x,
-                                                   h[2 * j + 1].y);
-                }
+        // this warp's 4 states over the chunk, from the entry state
+        {
+            float2 h[2];
+            if (c > 0) {
+                const float4 e = *reinterpret_cast<const float4 *>(
+                    p.hfwd + (q.bkd * nc1 + (c - 1)) * kNP + nw);
+                h[0] = make_float2(e.x, e.y);
+                h[1] = make_float2(e.z, e.w);
+            } else {
+                h[0] = h[1] = make_float2(0.f, 0.f);
             }
-        };
-        auto walk_back = [&](int t_hi, int base) {
+#pragma unroll 4
+            for (int t = 0; t < kT; ++t) {
+                const float4 v = st4[t * kBwdLanes + lane];
+                const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kNP + nw);
+                const float2 dt2 = dup2(v.x), dtu2 = dup2(v.x * v.y);
+                h[0] = __ffma2_rn(ex2_pair(__fmul2_rn(dt2, A2[0])), h[0],
+                                  __fmul2_rn(dtu2, make_float2(b4.x, b4.y)));
+                h[1] = __ffma2_rn(ex2_pair(__fmul2_rn(dt2, A2[1])), h[1],
+                                  __fmul2_rn(dtu2, make_float2(b4.z, b4.w)));
+                hs[t * kBwdLanes + lane] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+            }
+        }
+        if (c == c1 - 1) {   // the adjoint entering the range's top chunk at its end
+            if (c < nc1) {
+                const float4 e = *reinterpret_cast<const float4 *>(
+                    p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP + nw);
+                g[0] = make_float2(e.x, e.y);
+                g[1] = make_float2(e.z, e.w);
+            } else {
+                g[0] = g[1] = make_float2(0.f, 0.f);
+            }
+        }
 #pragma unroll 2
-            for (int t = t_hi; t >= base; --t) {
-                const float4 v4 = st4[t * kBwdLanes + lane];
-                const float dt = v4.x, u = v4.y, gy = v4.z;
-                const float dtu = dt * u;
-                const float2 dt2 = dup2(dt), dtu2 = dup2(dtu), ndtu2 = dup2(-dtu), gy2 = dup2(gy);
-                const float4 *row = hs4 + ((t - base) * kBwdLanes + lane) * 4;
-                float v[2 * kNP];
-                // sum g A2 (a h_prev), sum g B: two-wide partial sums
-                float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+        for (int t = kT - 1; t >= 0; --t) {
+            const float4 v4 = st4[t * kBwdLanes + lane];
+            const float dt = v4.x, u = v4.y, gy = v4.z;
+            const float2 dt2 = dup2(dt), dtu2 = dup2(dt * u), ndtu2 = dup2(-dt * u);
+            const float2 gy2 = dup2(gy);
+            const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kNP + nw);
+            const float4 c4 = *reinterpret_cast<const float4 *>(sC + t * kNP + nw);
+            const float4 h4 = hs[t * kBwdLanes + lane];
+            const float2 B2[2] = {make_float2(b4.x, b4.y), make_float2(b4.z, b4.w)};
+            const float2 C2[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
+            const float2 H2[2] = {make_float2(h4.x, h4.y), make_float2(h4.z, h4.w)};
+            float v[8];
+            float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int qd = 0; qd < 4; ++qd) {
-                    const float4 h4 = row[qd ^ swz];
+            for (int j = 0; j < 2; ++j) {
+                g[j] = __ffma2_rn(gy2, C2[j], g[j]);
+                const float2 hp = __ffma2_rn(ndtu2, B2[j], H2[j]);   // a_t h_{t-1}
+                const float2 vb = __fmul2_rn(g[j], dtu2);
+                const float2 vc = __fmul2_rn(gy2, H2[j]);
+                v[2 * j] = vb.x;
+                v[2 * j + 1] = vb.y;
+                v[4 + 2 * j] = vc.x;
+                v[4 + 2 * j + 1] = vc.y;
+                s2 = __ffma2_rn(g[j], B2[j], s2);
+                s1 = __ffma2_rn(__fmul2_rn(g[j], A2[j]), hp, s1);
+                dA[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), hp, dA[j]);
+                g[j] = __fmul2_rn(g[j], ex2_pair(__fmul2_rn(dt2, A2[j])));
+            }
+            const float r = reduce_scatter8(v);
+            if ((lane & 3) == 0)
+                red[t * 8 + (lane >> 2)] = r;
+            sums[(w * kT + t) * kBwdLanes + lane] = make_float2(s1.x + s1.y, s2.x + s2.y);
+        }
+        __syncthreads();   // every warp's (s1, s2) of the chunk
+        // warp w finishes steps 4w .. 4w+3 of its lanes' channels
+        float ddv[4], duv[4];
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const int j = 2 * qd + i;
-                        const float2 B2 = row_pair(sB + t * kNP, j);
-                        const float2 hv = i ? make_float2(h4.z, h4.w) : make_float2(h4.x, h4.y);
-                        g[j] = __ffma2_rn(gy2, row_pair(sC + t * kNP, j), g[j]);
-                        const float2 hp = __ffma2_rn(ndtu2, B2, hv);   // a_t h_{t-1}
-                        const float2 vb = __fmul2_rn(g[j], dtu2);
-                        const float2 vc = __fmul2_rn(gy2, hv);
-                        v[2 * j] = vb.x;
-                        v[2 * j + 1] = vb.y;
-                        v[kNP + 2 * j] = vc.x;
-                        v[kNP + 2 * j + 1] = vc.y;
-                        s2 = __ffma2_rn(g[j], B2, s2);
-                        s1 = __ffma2_rn(__fmul2_rn(g[j], A2[j]), hp, s1);
-                        dA[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), hp, dA[j]);
-                        g[j] = __fmul2_rn(g[j], ex2_pair(__fmul2_rn(dt2, A2[j])));
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * w + i;
+            float S1 = 0.f, S2 = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < kQuadWarps; ++ww) {
+                const float2 e = sums[(ww * kT + t) * kBwdLanes + lane];
+                S1 += e.x;
+                S2 += e.y;
+            }
+            const float4 v4 = st4[t * kBwdLanes + lane];
+            ddv[i] = fmaf(kLn2, S1, v4.y * S2) * v4.w;
+            duv[i] = fmaf(Dk, v4.z, v4.x * S2);
+            if (q.active && t < nt) {
+                dD = fmaf(v4.z, v4.y, dD);
+                db += ddv[i];
+            }
+        }
+        if (q.active) {
+            const int l0 = s + 4 * w;
+            if (vec_rows && 4 * w + 4 <= nt) {
+                float4 *dd4 = reinterpret_cast<float4 *>(ddrow + l0);
+                float4 *du4 = reinterpret_cast<float4 *>(durow + (flip ? L - 4 - l0 : l0));
+                float4 a = make_float4(ddv[0], ddv[1], ddv[2], ddv[3]);
+                float4 b = flip ? make_float4(duv[3], duv[2], duv[1], duv[0])
+                                : make_float4(duv[0], duv[1], duv[2], duv[3]);
+                if (accum) {
+                    const float4 ea = *dd4, eb = *du4;
+                    a = make_float4(ea.x + a.x, ea.y + a.y, ea.z + a.z, ea.w + a.w);
+                    b = make_float4(eb.x + b.x, eb.y + b.y, eb.z + b.z, eb.w + b.w);
+                }
+                *dd4 = a;
+                *du4 = b;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = 4 * w + i;
+                    if (t < nt) {
+                        const int l = s + t;
+                        float *o = durow + (flip ? L - 1 - l : l);
+                        ddrow[l] = accum ? ddrow[l] + ddv[i] : ddv[i];
+                        *o = accum ? *o + duv[i] : duv[i];
                     }
                 }
-                const float red = reduce_scatter32(v);
-                // this step's results replace its staged inputs in the lane's own
-                // slot (consumed by now); the rows are written once per chunk
-                const float S1 = s1.x + s1.y, S2 = s2.x + s2.y;
-                const float ddl = fmaf(kLn2, S1, u * S2) * v4.w;
-                st4[t * kBwdLanes + lane] = make_float4(ddl, fmaf(Dk, gy, dt * S2), red, 0.f);
-                if (q.active && t < nt) {
-                    dD = fmaf(gy, u, dD);
-                    db += ddl;
-                }
-            }
-        };
-        // the adjoint entering the range's top chunk at its end (zero for the
-        // sequence's last chunk)
-        if (c == c1 - 1) {
-            if (c < nc1)
-                load16(reinterpret_cast<float *>(g),
-                       p.hadj + (q.bkd * nc1 + (nc1 - 1 - c)) * kNP);
-            else
-#pragma unroll
-                for (int j = 0; j < kNP / 2; ++j)
-                    g[j] = make_float2(0.f, 0.f);
-        }
-        {
-            float2 h[kNP / 2];
-            entry(h);
-            recompute(h, kT, kHalf);
-        }
-        walk_back(kT - 1, kHalf);
-        {
-            float2 h[kNP / 2];
-            entry(h);
-            recompute(h, kHalf, 0);
-        }
-        walk_back(kHalf - 1, 0);
-        // the chunk's rows: ddelta and du of this lane's channel, and the
-        // reduced dB | dC row this lane holds (16-byte segments when whole)
-        const bool whole = nt == kT && vec_rows;
-        if (q.active) {
-            auto put4 = [&](float4 *dst, float4 v) {
-                if (accum) {
-                    const float4 e = *dst;
-                    v = make_float4(e.x + v.x, e.y + v.y, e.z + v.z, e.w + v.w);
-                }
-                *dst = v;
-            };
-            if (whole) {
-                float4 *dd4 = reinterpret_cast<float4 *>(ddrow + s);
-                float4 *du4 = reinterpret_cast<float4 *>(durow + (flip ? L - kT - s : s));
-#pragma unroll
-                for (int i = 0; i < kT / 4; ++i) {
-                    const float4 a = st4[(4 * i) * kBwdLanes + lane];
-                    const float4 b = st4[(4 * i + 1) * kBwdLanes + lane];
-                    const float4 c4 = st4[(4 * i + 2) * kBwdLanes + lane];
-                    const float4 d4 = st4[(4 * i + 3) * kBwdLanes + lane];
-                    put4(dd4 + i, make_float4(a.x, b.x, c4.x, d4.x));
-                    if (flip)
-                        put4(du4 + (kT / 4 - 1 - i), make_float4(d4.y, c4.y, b.y, a.y));
-                    else
-                        put4(du4 + i, make_float4(a.y, b.y, c4.y, d4.y));
-                }
-            } else {
-                for (int t = 0; t < nt; ++t) {
-                    const float4 r = st4[t * kBwdLanes + lane];
-                    const int l = s + t;
-                    float *o = durow + (flip ? L - 1 - l : l);
-                    ddrow[l] = accum ? ddrow[l] + r.x : r.x;
-                    *o = accum ? *o + r.y : r.y;
-                }
             }
         }
+        // the warp's reduced dB | dC rows of the chunk (lanes 0..7: one row each)
+        __syncwarp();
         if (bc_ok) {
-            if (whole) {
-                float4 *bc4 = reinterpret_cast<float4 *>(bcrow + s);
+            if (vec_rows && nt == kT) {
+                float4 *r4 = reinterpret_cast<float4 *>(bcrow + s);
 #pragma unroll
                 for (int i = 0; i < kT / 4; ++i)
-                    bc4[i] = make_float4(st4[(4 * i) * kBwdLanes + lane].z,
-                                         st4[(4 * i + 1) * kBwdLanes + lane].z,
-                                         st4[(4 * i + 2) * kBwdLanes + lane].z,
-                                         st4[(4 * i + 3) * kBwdLanes + lane].z);
+                    r4[i] = make_float4(red[(4 * i) * 8 + rj], red[(4 * i + 1) * 8 + rj],
+                                        red[(4 * i + 2) * 8 + rj], red[(4 * i + 3) * 8 + rj]);
             } else {
                 for (int t = 0; t < nt; ++t)
-                    bcrow[s + t] = st4[t * kBwdLanes + lane].z;
+                    bcrow[s + t] = red[t * 8 + rj];
             }
         }
     }
+    // parameter partials: this warp's dA; dDskip and dbias summed over the warps
+    __syncthreads();
+    float2 *acc = sums;   // reused: [warp][lane]
+    acc[w * kBwdLanes + lane] = make_float2(dD, db);
+    __syncthreads();
     if (q.active) {
-        // slots: dA of the call's NS states, dDskip, dbias; a later state group
-        // writes its own dA and adds its share of dbias (same thread, later launch)
         float *pr = p.prm_part + (q.bkd * p.CGN + blockIdx.y) * (p.NS + 2);
+        const float dav[4] = {dA[0].x, dA[0].y, dA[1].x, dA[1].y};
 #pragma unroll
-        for (int j = 0; j < kNP / 2; ++j) {
-            if (2 * j < p.N)
-                pr[p.n0 + 2 * j] = dA[j].x;
-            if (2 * j + 1 < p.N)
-                pr[p.n0 + 2 * j + 1] = dA[j].y;
-        }
-        if (!accum) {
-            pr[p.NS] = dD;
-            pr[p.NS + 1] = db;
-        } else {
-            pr[p.NS + 1] += db;
+        for (int i = 0; i < 4; ++i)
+            if (nw + i < p.N)
+                pr[p.n0 + nw + i] = dav[i];
+        if (w == 0) {
+            float sD = 0.f, sb = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < kQuadWarps; ++ww) {
+                const float2 e = acc[ww * kBwdLanes + lane];
+                sD += e.x;
+                sb += e.y;
+            }
+            if (!accum) {
+                pr[p.NS] = sD;
+                pr[p.NS + 1] = sb;
+            } else {
+                pr[p.NS + 1] += sb;
+            }
         }
     }
 }
