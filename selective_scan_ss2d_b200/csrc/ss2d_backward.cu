@@ -9,8 +9,10 @@
 namespace ss2d {
 
 namespace {
-// CTAs (one warp each) wanted in flight: about five resident per SM (the
-// final kernel's 42 KB of shared memory) times four waves
+// CTAs (one per channel group and chunk range) wanted per launch: 2960 = 148
+// SMs x 20, about 1.7 waves of the local pass (12 one-warp CTAs per SM) and
+// 6.7 of the final pass (3 four-warp CTAs per SM); fewer ranges would leave
+// SMs idle on the small-batch shapes, more would add carry work
 constexpr long long kBwdWantCtas = 148LL * 5 * 4;
 
 template <typename Tin>
