@@ -12,6 +12,9 @@ seeded synthetic arrays already resident in HBM; the L2 cache is flushed
   python bench.py --impl reference ...   # the float64 CPU oracle, rank 0
   python bench.py --report               # one line per workload (not the
                                          # contract line; for the notes)
+  python bench.py --backward [--config NAME]   # the gradient pass instead
+  python bench.py --gate                 # the gated entry point (y * SiLU(z))
+  python bench.py --dtype f16 --n-states 8     # another input dtype or N
 
 Multi-GPU (torchrun): the path has no exchange step, so every rank runs an
 independent replica of the workload (weak scaling, no collective on the data
