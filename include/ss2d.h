@@ -1,9 +1,10 @@
 /*
- * ss2d.h -- C ABI of the B200 (sm_100a) SS2D forward library.
+ * ss2d.h -- C ABI of the B200 (sm_100a) SS2D library.
  *
  * The library computes the forward pass of the 2D selective scan (SS2D) used
  * by VMamba, and the 1D selective scan with one or two directions used by
- * Vision Mamba (Vim):
+ * Vision Mamba (Vim), and the backward pass of both (ss2d_backward,
+ * selective_scan_bwd, below):
  *
  *   cross_scan   "Vision Mamba" (dileepadev tutorial), section "The 2D
  *                Challenge: Adapting SSMs to Images", CrossScanModule; and
@@ -224,7 +225,8 @@ int selective_scan_fwd_ex(const void *u, const void *delta, const float *A_log,
 /* How a call with this shape and variant (-1 = the library's choice) is
  * executed: steps per chunk, chunks per sequence, and kernel launches per
  * call (1 scan pass, or state pass + carry + scan pass when the sequence is
- * chunked; plus one cross_merge launch when K > 1).  Host only. */
+ * chunked, once per group of 16 states; plus one cross_merge launch when
+ * K > 1).  Host only. */
 int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
               int *chunk_len, int *num_chunks, int *launches);
 
