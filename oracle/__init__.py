@@ -18,7 +18,10 @@ What they compute and which page passage each step follows is stated in the
 header of ``ss2d_oracle.c``.  ``ss2d_backward_np.py`` (:func:`ss2d_backward`,
 :func:`selective_scan_bwd`) is the float64 reverse-mode gradient of the same
 forward definition, pinned against finite differences of the C forward;
-:func:`final_states` gives the state after each direction's last step.  Every part is pinned by ``tests/test_oracle_pins.py``
+:func:`final_states` gives the state after each direction's last step.
+``ss2d_front_np.py`` writes out the front that feeds the scan in the
+tutorial's SelectiveSSM (causal depthwise conv1d, SiLU, x_proj, dt_proj),
+pinned in ``tests/test_oracle_front.py``.  Every part is pinned by ``tests/test_oracle_pins.py``
 against closed forms, a matrix-exponential discretisation, an O(L^2) brute
 force and exact index-map invariants; parity is pinned for every function
 (no function here is "parity unpinned").
