@@ -169,3 +169,26 @@ def test_backward_binding_validates_tensors(lib):
         binding.ss2d_backward(x, delta, A_log, Bs, Bs, Dk, Dk, x.clone())
     with pytest.raises(ValueError, match="inconsistent"):
         binding.selective_scan_bwd(x[:, :, 0], delta, A_log, Bs, Bs, Dk, Dk, x[:, :, 0].clone())
+
+
+def test_final_state_argument_errors_are_reported_without_cuda(lib):
+    buf = (ctypes.c_float * 64)()
+    addr = ctypes.addressof(buf)
+    p = ctypes.c_void_p(addr + (-addr) % 16)
+    args = [p] * 8
+    # h_last missing: SS2D_ERR_NULL before anything else
+    assert lib.ss2d_forward_final_state(*args, None, 1, 1, 2, 2, 4, 4, 0, None, -1) == -1
+    assert lib.selective_scan_fwd_final_state(*args, None, 1, 1, 4, 4, 2, 0, None, -1) == -1
+    # then the forward's own rules
+    assert lib.ss2d_forward_final_state(*args, p, 1, 1, 2, 2, 65, 4, 0, None, -1) == -5
+    assert lib.ss2d_forward_final_state(*args, p, 1, 1, 2, 2, 4, 3, 0, None, -1) == -4
+    assert lib.selective_scan_fwd_final_state(*args, p, 1, 1, 4, 4, 4, 0, None, -1) == -4
+    assert lib.ss2d_forward_final_state(*args, p, 1, 1, 2, 2, 4, 4, 0, None, 10_000) == -10
+
+
+def test_plan_counts_launches_per_state_group(lib):
+    one = binding.ss2d_plan(True, 8, 192, 56, 56, 16, 4)
+    three = binding.ss2d_plan(True, 8, 192, 56, 56, 40, 4)
+    assert one["num_chunks"] == three["num_chunks"] > 1
+    # three groups of states: three (state pass, carry, output pass), one merge
+    assert one["launches"] == 3 + 1 and three["launches"] == 3 * 3 + 1
