@@ -1,5 +1,7 @@
-"""B200-native (sm_100a) SS2D forward path: cross_scan -> selective scan ->
-cross_merge, and the 1D one- or two-direction selective scan of Vision Mamba.
+"""B200-native (sm_100a) SS2D path: cross_scan -> selective scan ->
+cross_merge, and the 1D one- or two-direction selective scan of Vision Mamba;
+forward (plain, gated by SiLU(z), or returning the final states) and backward
+(every input's gradient).
 
 The computation lives in the CUDA library built from ``csrc/`` (C ABI in
 ``include/ss2d.h``); :mod:`.binding` marshals torch tensors into it.
