@@ -55,20 +55,20 @@ def test_scan_orders_are_permutations_and_agree(H, W):
         assert got == list(onp.scan_orders_1d(L)[k])
 
 
-@pytest.mark.parametrize("K", [1, 2, 4])
-def test_c_and_numpy_writeups_agree_2d(K):
-    rng = np.random.default_rng(100 + K)
-    p = _pins.rand_problem(rng, 2, 3, 5, 3, K, 6)
+@pytest.mark.parametrize("K,N", [(1, 6), (2, 6), (4, 6), (4, 40)])
+def test_c_and_numpy_writeups_agree_2d(K, N):
+    rng = np.random.default_rng(100 + K + N)
+    p = _pins.rand_problem(rng, 2, 3, 5, 3, K, N)
     yc, dc = _pins.call2d(IMPLS["c"], p, K=K, return_dirs=True)
     yn, dn = _pins.call2d(IMPLS["numpy"], p, K=K, return_dirs=True)
     np.testing.assert_allclose(yc, yn, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(dc, dn, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("K", [1, 2])
-def test_c_and_numpy_writeups_agree_1d(K):
-    rng = np.random.default_rng(200 + K)
-    p = _pins.rand_problem(rng, 2, 3, 1, 37, K, 16, one_d=True)
+@pytest.mark.parametrize("K,N", [(1, 16), (2, 16), (2, 64)])
+def test_c_and_numpy_writeups_agree_1d(K, N):
+    rng = np.random.default_rng(200 + K + N)
+    p = _pins.rand_problem(rng, 2, 3, 1, 37, K, N, one_d=True)
     yc = _pins.call1d(IMPLS["c"], p, K=K)
     yn = _pins.call1d(IMPLS["numpy"], p, K=K)
     np.testing.assert_allclose(yc, yn, rtol=1e-12, atol=1e-12)
