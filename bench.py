@@ -290,6 +290,7 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev)
 
     gate = getattr(args, "gate", False)
+    label = f"ss2d forward{' gated' if gate else ''} {cfg.name}"
     if gate:
         # the SiLU output gate: a seeded z in x's layout, the gated entry point
         # (the library's own variant choice)
@@ -323,12 +324,14 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push(f"{label} timed steps")   # marks the region for a trace
     for i in range(args.steps):
         flush.fill_(float(i))
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -340,11 +343,13 @@ def run_ours(args, rank, world, local_rank):
     # CUDA events recorded by the library on this stream around each launch
     two_d = cfg.kind == "2d"
     per = []
+    torch.cuda.nvtx.range_push(f"{label} per-launch timing")
     for i in range(args.steps):
         flush.fill_(float(i))
         per.append(binding.ss2d_forward_timed(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"],
                                               t["Dskip"], t["delta_bias"], y, two_d=two_d,
                                               stream=stream.cuda_stream, variant=args.variant))
+    torch.cuda.nvtx.range_pop()
     names = ["chunk_state_pass", "carry", "scan_pass", "cross_merge"]
     launch_ms = {}
     for j, nm in enumerate(names):
@@ -439,6 +444,8 @@ def run_backward(args, rank, world, local_rank):
     l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
     flush = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev)
 
+    label = f"ss2d backward {cfg.name}"
+
     def step():
         return fn(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"], t["Dskip"], t["delta_bias"],
                   dy, stream=stream.cuda_stream)
@@ -458,12 +465,14 @@ def run_backward(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push(f"{label} timed steps")   # marks the region for a trace
     for i in range(args.steps):
         flush.fill_(float(i))
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -523,6 +532,7 @@ def run_e2e(args, cfg_name, local_rank, world=1):
            stream=stream.cuda_stream, variant=args.variant)
     n = max(3, min(args.steps, 20))
     evs = []
+    torch.cuda.nvtx.range_push(f"ss2d forward end to end {cfg.name}")
     for _ in range(n):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -531,6 +541,7 @@ def run_e2e(args, cfg_name, local_rank, world=1):
         b.record(stream)
         evs.append((a, b))
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     total = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dev)
     h2d = sum(getattr(inp, nm).nbytes for nm in wl.Inputs.STREAMED + wl.Inputs.PARAMS)
     d2h = y.numel() * 4
