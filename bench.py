@@ -623,6 +623,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    if args.n_states is not None and not 1 <= args.n_states <= 64:
+        ap.error("--n-states must be in 1..64")
+    if args.n_states and args.n_states > 16 and not args.backward and args.impl == "ours":
+        # the per-launch timing of the forward line covers one group of 16 states
+        ap.error("the forward bench takes --n-states up to 16 (--backward takes up to 64)")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -43,3 +43,11 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
                                       "--steps", "1", "--warmup", "1"])
     assert bench.main() == 0
     assert capsys.readouterr().out == ""
+
+
+def test_bench_rejects_unsupported_state_counts(monkeypatch):
+    for argv in (["bench.py", "--n-states", "32"], ["bench.py", "--n-states", "65", "--backward"]):
+        monkeypatch.setattr(sys, "argv", argv)
+        with pytest.raises(SystemExit) as ei:
+            bench.main()
+        assert ei.value.code == 2
