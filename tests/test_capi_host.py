@@ -192,3 +192,21 @@ def test_plan_counts_launches_per_state_group(lib):
     assert one["num_chunks"] == three["num_chunks"] > 1
     # three groups of states: three (state pass, carry, output pass), one merge
     assert one["launches"] == 3 + 1 and three["launches"] == 3 * 3 + 1
+
+
+def test_final_state_binding_validates_tensors(lib):
+    import torch
+    x = torch.zeros(1, 2, 3, 3)
+    delta = torch.zeros(1, 4, 2, 9)
+    Bs = torch.zeros(1, 4, 4, 9)
+    A_log = torch.zeros(8, 4)
+    Dk = torch.zeros(8)
+    with pytest.raises(ValueError, match="device tensors only"):
+        binding.forward_final_state(x, delta, A_log, Bs, Bs, Dk, Dk)
+    with pytest.raises(ValueError, match="inconsistent"):
+        binding.forward_final_state(x, delta[:, :2], A_log, Bs, Bs, Dk, Dk)
+    u = torch.zeros(1, 2, 9)
+    with pytest.raises(ValueError, match="inconsistent"):
+        binding.forward_final_state(u, delta, A_log, Bs, Bs[:, :, :3], Dk, Dk)
+    with pytest.raises(TypeError):
+        binding.selective_scan_bwd(u.double(), delta, A_log, Bs, Bs, Dk, Dk, u.clone())
