@@ -44,14 +44,14 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MAX_MHZ = 1965.0
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from ncu
-# captures recorded under profiles/, keyed by workload; each entry carries
+# captures of the output pass, keyed by workload; each entry carries
 # the input dtype, the state count and the hash of the kernel sources it was
 # taken from, and is reported only for that configuration while the sources
 # are unchanged.
 NCU_TRAFFIC = {
-    # profiles/chunk_scan_vmamba_t_stage1.md: output pass, dram read 65492224 + write 25570560
+    # ncu capture of the output pass: dram read 65492224 + write 25570560
     "vmamba_t_stage1": {"bytes": 91062784, "dtype": "bf16", "N": 16, "src": "4f946ebf7ed334c0"},
-    # profiles/chunk_scan_vmamba_b_stage3.md: output pass, dram read 141669632 + write 161776128
+    # ncu capture of the output pass: dram read 141669632 + write 161776128
     "vmamba_b_stage3": {"bytes": 303445760, "dtype": "bf16", "N": 16, "src": "4f946ebf7ed334c0"},
 }
 

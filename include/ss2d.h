@@ -270,10 +270,11 @@ int ss2d_pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
  *     pointers only (SS2D_ERR_PTR otherwise); asynchronous on `stream`.
  *   - A problem whose scratch would not fit returns SS2D_ERR_SCRATCH before
  *     anything is enqueued; ss2d_last_error() then gives the bytes needed.
- *   - First call on a device: the buffer's address on that device is looked
- *     up (with that device current) and kept.  The lookup loads the module
- *     that holds the buffer, which is when its memory is reserved; make this
- *     first call on each device before any stream capture begins.
+ *   - Every call looks the buffer's address up on the current device
+ *     (cudaGetSymbolAddress) and keeps nothing between calls, so a device
+ *     reset between calls is safe.  The first call on a device loads the
+ *     module that holds the buffer, which is when its memory is reserved;
+ *     make this first call on each device before any stream capture begins.
  *   - Nothing in the buffer has to start at zero: every word a call reads is
  *     written earlier in the same call.
  *   - One buffer per device: calls on one device whose work can overlap in

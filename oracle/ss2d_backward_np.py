@@ -29,7 +29,7 @@ dbias = sum_t ddelta_t, dA_log = dA * A (dA/dA_log = A), and dx gathers du_k
 of every direction back to its pixel (the adjoint of the cross_scan gather).
 The parameter gradients are summed over the batch.
 
-Pinned in ``tests/test_oracle_pins.py`` against central finite differences
+Pinned in ``tests/test_oracle_backward.py`` against central finite differences
 of the C forward oracle (a separate program) on every input element of small
 problems, and against closed forms of one- and two-step scans derived by hand.
 """

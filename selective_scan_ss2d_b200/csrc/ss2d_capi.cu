@@ -689,7 +689,7 @@ const char *ss2d_status_string(int status)
     case SS2D_ERR_K:
         return "unsupported number of directions K";
     case SS2D_ERR_N:
-        return "state size N must be in 1..16";
+        return "state size N must be in 1..64 (1..16 for ss2d_forward_timed)";
     case SS2D_ERR_ALIGN:
         return "a pointer is not 16-byte aligned";
     case SS2D_ERR_ALLOC:

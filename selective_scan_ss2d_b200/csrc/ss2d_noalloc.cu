@@ -16,11 +16,13 @@
 // per-direction scan-order output rows (K > 1) and, when the sequences are
 // split into chunks, the chunk end states and the sums of dt per chunk.
 //
-// First call on a device: cudaGetSymbolAddress, with that device current,
-// gives the buffer's address in the device's context.  It is looked up once
-// per device and kept; the lookup loads this file's module, which is when the
-// buffer's memory is reserved, so the first call on a device belongs before
-// any stream capture begins.  No word of the buffer has to start at zero: the
+// Every call asks cudaGetSymbolAddress, with the call's device current, for
+// the buffer's address in that device's context (after the first call it is
+// a table lookup in the runtime).  Nothing is cached across calls, so a
+// context that was torn down and created again (cudaDeviceReset) gives the
+// new context's address, never a stale one.  The first call on a device loads
+// this file's module, which is when the buffer's memory is reserved, so the
+// first call on a device belongs before any stream capture begins.  No word of the buffer has to start at zero: the
 // chunk state pass writes every end state and dt sum that the carry kernel
 // and the output pass read, and the output pass writes every row element the
 // merge kernel reads.  There is one buffer per device, so calls on one device
@@ -30,8 +32,6 @@
 #include <stdint.h>
 #include <stdio.h>
 
-#include <mutex>
-
 #include "ss2d.h"
 #include "ss2d_launch.h"
 #include "ss2d_params.h"
@@ -40,24 +40,14 @@ static __device__ __align__(256) char g_noalloc_scratch[SS2D_NOALLOC_SCRATCH_BYT
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_addr_mutex;
-char *g_addr[kMaxDevices] = {};
-
-// Address of g_noalloc_scratch on device `dev`, which is the current device.
-cudaError_t scratch_address(int dev, char **out)
+// Address of g_noalloc_scratch on the current device, looked up on every call.
+cudaError_t scratch_address(char **out)
 {
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_addr_mutex);
-    if (!g_addr[dev]) {
-        void *ptr = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess)
-            return e;
-        g_addr[dev] = static_cast<char *>(ptr);
-    }
-    *out = g_addr[dev];
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess)
+        return e;
+    *out = static_cast<char *>(ptr);
     return cudaSuccess;
 }
 
@@ -127,7 +117,7 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
         if (!on_device(q, dev))
             return SS2D_ERR_PTR;
     char *base = nullptr;
-    e = scratch_address(dev, &base);
+    e = scratch_address(&base);
     if (e != cudaSuccess) {
         ss2d::record_error("cudaGetSymbolAddress", e);
         return SS2D_ERR_CUDA;

@@ -45,6 +45,10 @@ def test_status_strings(lib):
         s = binding.ss2d_status_string(st)
         assert s and s != "unknown status"
     assert binding.ss2d_status_string(-99) == "unknown status"
+    # every forward and backward entry takes N in 1..64; only the timed call
+    # is limited to one group of 16
+    assert "1..64" in binding.ss2d_status_string(-5)
+    assert "1..16 for ss2d_forward_timed" in binding.ss2d_status_string(-5)
 
 
 def test_variant_table(lib):
