@@ -16,7 +16,8 @@ section 4.1: the recurrence).  The cases:
   dt = 1e-1 (softplus^-1 of them as the bias, small delta), with the
   recipe's A_log = ln(n + 1) up to ln 16;
 * the kernel's softplus itself, observed through a one-step scan, against
-  float64 log1p(exp(z)) over z in [-40, 40].
+  float64 log1p(exp(z)) over z in [-40, 40], under the error bound its
+  float32 evaluation allows (derived below).
 """
 from __future__ import annotations
 
@@ -75,10 +76,18 @@ def test_highres_full_shape_fp32_sampled(extreme):
         _gpu.assert_close(y[0:1, d:d + 1], _gpu.run_oracle(sub), wl.F32, f"highres fp32 d={d}")
 
 
-# The kernel's softplus: degree-7 polynomial (relative error below 4e-7 in
-# float32, tests/test_softplus_fit.py) times e = exp(-|z|) from the exp2 of
-# the multi-function unit (relative error about 2^-22); together below 7e-7.
-SOFTPLUS_REL = 7e-7
+# The kernel's softplus, max(z, 0) + e * q(e) with e = 2^(-|z| * log2(e)):
+#   * q, the degree-7 polynomial, relative error below 4e-7 in float32
+#     (tests/test_softplus_fit.py);
+#   * the exp2 of the multi-function unit, relative error about 2^-22;
+#   * the float32 argument -|z| * log2(e): its rounding and that of the
+#     constant log2(e) shift it by at most 2^-23 * |z| * log2(e), which
+#     changes e by a factor 2^(2^-23 |z| log2 e) ~ 1 + 1.2e-7 * |z|.
+# The relative error of the result is therefore below 6.5e-7 + 1.2e-7 * |z|
+# (3 ulp of float32 at z = 0, growing to about 5e-6 at |z| = 40, where
+# softplus(z) is e^-40 and the step is far below any that matters).
+def softplus_bound(z):
+    return 6.5e-7 + 1.2e-7 * np.abs(z)
 
 
 def test_softplus_through_one_step_scan():
@@ -98,5 +107,8 @@ def test_softplus_through_one_step_scan():
     zz = z.astype(np.float64)
     want = np.maximum(zz, 0) + np.log1p(np.exp(-np.abs(zz)))
     rel = np.abs(got - want) / want
-    assert rel.max() <= SOFTPLUS_REL, (
-        f"softplus relative error {rel.max():.3e} at z = {zz[rel.argmax()]}")
+    ratio = rel / softplus_bound(zz)
+    worst = int(ratio.argmax())
+    assert ratio[worst] <= 1.0, (
+        f"softplus relative error {rel[worst]:.3e} at z = {zz[worst]} "
+        f"(bound {softplus_bound(zz[worst]):.3e})")
