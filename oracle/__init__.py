@@ -20,8 +20,9 @@ header of ``ss2d_oracle.c``.  ``ss2d_backward_np.py`` (:func:`ss2d_backward`,
 forward definition, pinned against finite differences of the C forward;
 :func:`final_states` gives the state after each direction's last step.
 ``ss2d_front_np.py`` writes out the front that feeds the scan in the
-tutorial's SelectiveSSM (causal depthwise conv1d, SiLU, x_proj, dt_proj),
-pinned in ``tests/test_oracle_front.py``.  Every part is pinned by ``tests/test_oracle_pins.py``
+tutorial's SelectiveSSM (causal depthwise conv1d, SiLU, x_proj, dt_proj) and
+its per-direction form of the Vim block; :func:`front_scan` runs it and then
+the scan of every direction, pinned in ``tests/test_oracle_front.py``.  Every part is pinned by ``tests/test_oracle_pins.py``
 against closed forms, a matrix-exponential discretisation, an O(L^2) brute
 force and exact index-map invariants; parity is pinned for every function
 (no function here is "parity unpinned").
@@ -36,6 +37,7 @@ import threading
 import numpy as np
 
 from .ss2d_backward_np import selective_scan_bwd, ss2d_backward  # noqa: F401
+from .ss2d_front_np import front_directions  # noqa: F401
 from .ss2d_oracle_np import final_states  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -203,3 +205,28 @@ def scan_pixel(mode: int, k: int, l: int, H: int, W: int) -> int:
 
 def max_threads() -> int:
     return lib().oracle_max_threads()
+
+
+def front_scan(x, conv_w, conv_b, W_x, w_dt, A_log, Dskip, delta_bias, *, storage=None,
+               operand="f64", threads=1):
+    """The front of every direction (:func:`front_directions`) followed by
+    that direction's selective scan over its own u, delta, B and C, each
+    direction's output turned back to the sequence order (direction 1 is
+    reversed) and the K outputs summed: y (B, D, L) float64.  A_log (K*D, N),
+    Dskip and delta_bias (K*D,) as in :func:`selective_scan_fwd`."""
+    u, delta, Bs, Cs = front_directions(x, conv_w, conv_b, W_x, w_dt, storage=storage,
+                                        operand=operand)
+    K, D = u.shape[1], u.shape[2]
+    A_log = np.asarray(A_log, dtype=np.float64)
+    Dskip = np.asarray(Dskip, dtype=np.float64)
+    delta_bias = np.asarray(delta_bias, dtype=np.float64)
+    y = None
+    for k in range(K):
+        rows = slice(k * D, (k + 1) * D)
+        yk = selective_scan_fwd(u[:, k], delta[:, k:k + 1], A_log[rows], Bs[:, k:k + 1],
+                                Cs[:, k:k + 1], Dskip[rows], delta_bias[rows], K=1,
+                                threads=threads)
+        if k == 1:
+            yk = yk[:, :, ::-1]
+        y = yk if y is None else y + yk
+    return np.ascontiguousarray(y)

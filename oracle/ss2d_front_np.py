@@ -23,6 +23,20 @@ out step by step.
 Pinned in ``tests/test_oracle_front.py``: the conv against NumPy's own
 ``convolve`` per channel, its impulse response and causality, x_proj against
 selector weights and linearity, and planted mistakes.
+
+``front_directions`` is the bidirectional form of the Vim block ("Vision
+Mamba ..." summary, section 4.3): each of the K directions runs its own conv1d
+and projections on its own sequence, the input itself (k = 0) or the input
+reversed along L (k = 1), and the results come out in that direction's scan
+order.  It states two readings the pages leave open, about precision:
+
+* ``operand="bf16"``: x_proj multiplies bfloat16 operands -- u and W_x each
+  rounded to bfloat16 (nearest, ties to even) from their exact values -- and
+  sums the products exactly (the tensor-core form of the product, with a
+  float32 accumulator on the GPU); ``operand="f64"`` keeps them exact;
+* ``storage``: u, which the scan reads, is stored in the input's dtype
+  ("f32", "bf16" or "f16", rounded to nearest even from the exact value), or
+  kept exact (None).
 """
 from __future__ import annotations
 
@@ -65,3 +79,54 @@ def front(x, conv_w, conv_b, W_x, w_dt):
             np.ascontiguousarray(delta[:, None]),
             np.ascontiguousarray(Bm.transpose(0, 2, 1)[:, None]),
             np.ascontiguousarray(Cm.transpose(0, 2, 1)[:, None]))
+
+
+def round_storage(a, storage):
+    """a (float64) rounded to a storage dtype, returned as float64 values:
+    "f32" and "f16" by NumPy's casts (nearest, ties to even), "bf16" by
+    keeping the upper 16 bits of the float32 value after rounding to nearest
+    with ties to even; None returns a unchanged."""
+    a = np.asarray(a, dtype=np.float64)
+    if storage is None:
+        return a
+    if storage == "f32":
+        return a.astype(np.float32).astype(np.float64)
+    if storage == "f16":
+        return a.astype(np.float16).astype(np.float64)
+    if storage == "bf16":
+        u = np.ascontiguousarray(a.astype(np.float32)).view(np.uint32).astype(np.uint64)
+        lsb = (u >> 16) & 1
+        r = (((u + 0x7FFF + lsb) >> 16) << 16).astype(np.uint32)
+        return r.view(np.float32).astype(np.float64)
+    raise ValueError(f"unknown storage {storage!r}")
+
+
+def front_directions(x, conv_w, conv_b, W_x, w_dt, *, storage=None, operand="f64"):
+    """x (B, L, D) input branch; conv_w (K, D, d_conv), conv_b (K, D), W_x
+    (K, 1 + 2N, D), w_dt (K, D): direction k's conv, x_proj and dt_proj
+    weights.  Direction 0 reads the sequence as it is, direction 1 reversed.
+    Returns, in each direction's scan order: u (B, K, D, L) as stored (see
+    ``storage``), delta (B, K, D, L) = w_dt[k, d] * dt_raw[b, k, l], Bs and Cs
+    (B, K, N, L), all float64."""
+    x = np.asarray(x, dtype=np.float64)
+    conv_w = np.asarray(conv_w, dtype=np.float64)
+    K = conv_w.shape[0]
+    outs = []
+    for k in range(K):
+        seq = x if k == 0 else x[:, ::-1, :]
+        u_exact = silu(causal_depthwise_conv(seq, conv_w[k], conv_b[k]))   # (B, L, D)
+        Wk = np.asarray(W_x[k], dtype=np.float64)
+        if operand == "bf16":
+            x_dbl = round_storage(u_exact, "bf16") @ round_storage(Wk, "bf16").T
+        elif operand == "f64":
+            x_dbl = u_exact @ Wk.T
+        else:
+            raise ValueError(f"unknown operand {operand!r}")
+        N = (Wk.shape[0] - 1) // 2
+        dt_raw = x_dbl[:, :, 0]                                      # (B, L)
+        delta = np.asarray(w_dt[k], dtype=np.float64)[None, :, None] * dt_raw[:, None, :]
+        outs.append((round_storage(u_exact, storage).transpose(0, 2, 1), delta,
+                     x_dbl[:, :, 1:1 + N].transpose(0, 2, 1),
+                     x_dbl[:, :, 1 + N:1 + 2 * N].transpose(0, 2, 1)))
+    return tuple(np.ascontiguousarray(np.stack([o[i] for o in outs], axis=1))
+                 for i in range(4))
