@@ -14,7 +14,12 @@ seeded synthetic arrays already resident in HBM; the L2 cache is flushed
                                          # contract line; for the notes)
   python bench.py --backward [--config NAME]   # the gradient pass instead
   python bench.py --gate                 # the gated entry point (y * SiLU(z))
+  python bench.py --front                # the fused front + scan of the Vim-S block
   python bench.py --dtype f16 --n-states 8     # another input dtype or N
+
+At one GPU the default line also carries `per_config`: every other workload
+of the set (tiny fp32, VMamba-B stage 3, the 256x256 map, Vim-S) timed the
+same way with fewer steps, with its rooflines and a short oracle sample.
 
 Multi-GPU (torchrun): the path has no exchange step, so every rank runs an
 independent replica of the workload (weak scaling, no collective on the data
@@ -42,6 +47,7 @@ MUFU_EX2_PER_CLK_PER_SM = 16       # exp2 results per clock per SM (MUFU)
 NUM_SMS = 148
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MAX_MHZ = 1965.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from ncu
 # captures of the output pass, keyed by workload; each entry carries
@@ -78,9 +84,14 @@ def measured_peaks() -> dict:
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", FALLBACK_SM_MAX_MHZ)),
+        bf16 = d.get("bf16_tflops")
+        return {"hbm_gbs": float(d["hbm_gbs"]),
+                "sm_max_mhz": float(d.get("sm_max_mhz", FALLBACK_SM_MAX_MHZ)),
+                "bf16_tflops": float(bf16) if bf16 else FALLBACK_BF16_TFLOPS,
+                "bf16_source": "measured (bf16_tflops, burst)" if bf16 else "fallback",
                 "source": "measured"}
-    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MAX_MHZ, "source": "fallback"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MAX_MHZ,
+            "bf16_tflops": FALLBACK_BF16_TFLOPS, "bf16_source": "fallback", "source": "fallback"}
 
 
 # ---------------------------------------------------------------------------
@@ -421,6 +432,187 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def run_per_config(args, rank, world, local_rank):
+    """The other workloads of the benchmark set, each timed like the
+    headline (inputs resident, L2 flushed before every timed step, CUDA
+    events) with fewer steps, and the float64 oracle on a bounded sample of
+    each (about args.per_config_cpu_seconds of host time).  Returns
+    {workload: summary} on rank 0."""
+    from selective_scan_ss2d_b200 import workloads as wl
+    out = {}
+    for name in wl.CONFIG_ORDER:
+        if name == args.config:
+            continue
+        a = argparse.Namespace(**vars(args))
+        a.config = name
+        a.steps = max(3, min(args.steps, args.per_config_steps))
+        a.dtype = None
+        a.n_states = None
+        a.gate = False
+        r = run_ours(a, rank, world, local_rank)
+        if rank != 0:
+            continue
+        ln = r["line"]
+        rf, rh = ln["roofline"], ln["roofline_hbm"]
+        summary = {
+            "config": ln["config"],
+            "ms_per_step": ln["ms_per_step"],
+            "value": ln["value"],
+            "unit": ln["unit"],
+            "steps": a.steps,
+            "roofline": {"bound": rf["bound"], "unit": rf["unit"], "peak": rf["peak"],
+                         "kernel_frac": rf["frac"], "step_frac": rf["step"]["frac"],
+                         "traffic": rf["traffic"], "kernel_ms": rf["kernel_ms"]},
+            "roofline_hbm": {"unit": rh["unit"], "peak": rh["peak"], "kernel_frac": rh["frac"],
+                             "step_frac": rh["step"]["frac"],
+                             "step_achieved": rh["step"]["achieved"]},
+            "launch_ms": ln["launch_ms"],
+            "plan": ln["plan"],
+            "gpu_launches": ln["gpu_launches"],
+            "clocks": r.get("clocks"),
+        }
+        if not args.no_cpu_baseline:
+            import oracle
+            threads = oracle.max_threads()
+            cfg = workload_config(name)
+            v, desc, _ = cpu_baseline_parallel(cfg, args.per_config_cpu_seconds, threads)
+            summary["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": threads,
+                                       "kind": "oracle", "sample": desc}
+        out[name] = summary
+    return out if rank == 0 else None
+
+
+def run_front(args, rank, world, local_rank):
+    """The fused front + scan (selective_scan_fwd_front) of the Vim-S block:
+    one step = conv1d + SiLU + x_proj (tensor cores) + dt_proj of both
+    directions, their scans and the sum, inputs resident in HBM, L2 flushed
+    before every timed step.  Returns the JSON line (rank 0)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from selective_scan_ss2d_b200 import binding
+    from selective_scan_ss2d_b200 import workloads as wl
+
+    cfg = wl.FRONT_CONFIGS[args.front_config]
+    if args.dtype:
+        cfg = cfg.with_(dtype=args.dtype)
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    binding.lib()
+    inp = wl.make_front_inputs(cfg, seed=rank)
+    tdt = {wl.F32: torch.float32, wl.BF16: torch.bfloat16, wl.F16: torch.float16}[cfg.dtype]
+    x = (torch.from_numpy(inp.x.view(np.int16)).view(torch.bfloat16) if inp.x.dtype == np.uint16
+         else torch.from_numpy(inp.x)).to(dev)
+    assert x.dtype == tdt
+    wts = {n: torch.from_numpy(getattr(inp, n)).to(dev) for n in wl.FrontInputs.WEIGHTS}
+    y = torch.empty((cfg.B, cfg.D, cfg.L), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
+    flush = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev)
+    args_f = [x] + [wts[n] for n in wl.FrontInputs.WEIGHTS]
+
+    def step():
+        binding.selective_scan_fwd_front(*args_f, y)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    gpu_id = str(getattr(props, "uuid", local_rank))
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.2)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push(f"front {cfg.name} timed steps")
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
+    value = whole_job_rate(cfg.updates, args.steps, world, total_ms)
+    per = []
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        per.append(binding.selective_scan_fwd_front_timed(*args_f, y, stream=stream.cuda_stream))
+    front_ms = statistics.mean(r[0] for r in per)
+    scan_ms = statistics.mean(r[1] for r in per)
+    merge_ms = statistics.mean(r[2] for r in per if r[2] >= 0) if cfg.K > 1 else None
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    esz = 4 if cfg.dtype == wl.F32 else 2
+    R = 1 + 2 * cfg.N
+    # x_proj on the tensor cores: useful flops (M = steps, N = 1 + 2N, K = D)
+    flops = 2.0 * cfg.B * cfg.K * cfg.L * cfg.D * R
+    # the front kernel's algorithmic bytes: x read once per direction, u
+    # written once (input dtype), dt_raw, B, C written once (float32), weights
+    front_bytes = (cfg.K * cfg.B * cfg.L * cfg.D * esz + cfg.B * cfg.K * cfg.D * cfg.L * esz +
+                   cfg.B * cfg.K * cfg.L * R * 4 + cfg.K * cfg.D * (4 + 1 + R + 1) * 4)
+    # the whole call's algorithmic bytes: x read once, y written once, weights
+    step_bytes = (cfg.B * cfg.L * cfg.D * esz + cfg.B * cfg.D * cfg.L * 4 +
+                  cfg.K * cfg.D * (4 + 1 + R + 1 + cfg.N + 2) * 4)
+    step_s = total_ms / args.steps / 1e3
+    exps = cfg.updates + cfg.B * cfg.K * cfg.D * cfg.L
+    mufu_peak = NUM_SMS * MUFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e9
+    tflops = flops / (front_ms / 1e3) / 1e12
+    front_gbs = front_bytes / (front_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "updates/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) input branch and unit-scale weights)",
+        "config": {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "D": cfg.D, "N": cfg.N,
+                   "K": cfg.K, "input_dtype": cfg.dtype, "entry": "selective_scan_fwd_front",
+                   "l2": "flushed before every timed step (2x L2 write, outside events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline_front_tensor": {"bound": "tensor", "achieved": tflops,
+                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                  "frac": tflops / peaks["bf16_tflops"],
+                                  "kernel": "front_kernel (x_proj on tcgen05, bf16 operands)",
+                                  "kernel_ms": front_ms, "flops_per_launch": flops,
+                                  "peak_source": peaks["bf16_source"]},
+        "roofline_front_hbm": {"bound": "hbm", "achieved": front_gbs, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": front_gbs / peaks["hbm_gbs"],
+                               "bytes_per_launch": front_bytes, "kernel_ms": front_ms,
+                               "peak_source": f"{peaks['source']} (hbm_gbs)"},
+        "roofline": {"bound": "alu", "unit": "Gexp2/s", "peak": mufu_peak,
+                     "achieved": exps / (scan_ms / 1e3) / 1e9,
+                     "frac": exps / (scan_ms / 1e3) / 1e9 / mufu_peak,
+                     "kernel": "lane_scan_kernel passes on the front's outputs",
+                     "kernel_ms": scan_ms,
+                     "step": {"achieved": exps / step_s / 1e9,
+                              "frac": exps / step_s / 1e9 / mufu_peak}},
+        "roofline_hbm": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                         "step": {"achieved": step_bytes / step_s / 1e9,
+                                  "frac": step_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
+                         "algorithmic_bytes_per_step": step_bytes},
+        "launch_ms": {"front": front_ms, "scan_passes": scan_ms, "cross_merge": merge_ms},
+        "clocks": clocks,
+    }
+    return line
+
+
 def run_backward(args, rank, world, local_rank):
     """The backward pass (ss2d_backward / selective_scan_bwd) of the workload:
     one step = the gradients of every input for one seeded cotangent, inputs
@@ -618,6 +810,15 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (gradients of every input) instead; "
                          "device buffers only, no e2e or CPU leg")
+    ap.add_argument("--front", action="store_true",
+                    help="time the fused front + scan (selective_scan_fwd_front) instead")
+    ap.add_argument("--front-config", default="vim_s_front")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="leave out the per_config summaries of the other workloads")
+    ap.add_argument("--per-config-steps", type=int, default=10,
+                    help="timed steps of each per_config workload")
+    ap.add_argument("--per-config-cpu-seconds", type=float, default=3.0,
+                    help="host seconds for each per_config oracle sample")
     ap.add_argument("--report", action="store_true",
                     help="one JSON line per workload (device-resident only)")
     args = ap.parse_args()
@@ -640,6 +841,16 @@ def main():
         return 0
 
     init_distributed(world, local_rank)
+
+    if args.front:
+        line = run_front(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     if args.backward:
         line = run_backward(args, rank, world, local_rank)
@@ -665,6 +876,9 @@ def main():
 
     r = run_ours(args, rank, world, local_rank)
     e2e = None if (args.no_e2e or args.gate) else run_e2e(args, args.config, local_rank, world)
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = run_per_config(args, rank, world, local_rank)
     if rank == 0:
         line = r["line"]
         line["clocks"] = r.get("clocks")
@@ -678,6 +892,8 @@ def main():
             v, desc, _ = cpu_baseline_parallel(cfg, args.cpu_seconds, threads)
             line["cpu_baseline"] = {"value": v, "unit": "updates/s", "cores": threads,
                                     "kind": "oracle", "sample": desc}
+        if per_config is not None:
+            line["per_config"] = per_config
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

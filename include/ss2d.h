@@ -286,6 +286,83 @@ int ss2d_forward_noalloc(const void *x, const void *delta, const float *A_log,
                          int B, int D, int H, int W, int N, int K, int dtype,
                          void *stream);
 
+/* ---- the fused front (conv1d + SiLU + x_proj + dt_proj) -----------------
+ *
+ * "Vision Mamba" (dileepadev tutorial), section "Background: State Space
+ * Models and Mamba", SelectiveSSM.forward; "Vision Mamba ..." summary,
+ * section 4.3 (the Vim block: every direction its own conv1d and
+ * projections, direction 1 on the sequence reversed).  For direction k
+ * (K = 1: forward only; K = 2: forward and reversed), batch element b and
+ * step l of the direction's own order s (s[l] = x[b, l] for k = 0,
+ * x[b, L-1-l] for k = 1):
+ *   c[l, d]   = conv_b[k, d] + sum_{j<4} conv_w[k, d, j] * s[l-3+j, d]
+ *               (causal depthwise conv1d of width 4, zeros before l = 0)
+ *   u[l, d]   = SiLU(c[l, d]) = c / (1 + exp(-c))
+ *   x_dbl[l]  = W_x[k] u[l]     (x_proj, D -> 1 + 2N, no bias) =
+ *               (dt_raw[l], B[0..N-1, l], C[0..N-1, l])
+ *   delta     = w_dt[k, d] * dt_raw[l]   (dt_proj, a Linear from 1 to D;
+ *               its bias is the scan's delta_bias)
+ * then the selective scan of every direction over its own u, delta, B, C
+ * (as selective_scan_fwd, with A_log, Dskip, delta_bias rows k*D + d) and
+ * y = Y_0 + Y_1 flipped back.  x_proj runs on the tensor cores (tcgen05)
+ * with bfloat16 operands -- u and W_x rounded to nearest even -- and a
+ * float32 accumulator; u is kept for the scan in the input dtype, dt_raw,
+ * B and C in float32; no (D, L) delta array is ever written.
+ *
+ * Layouts (contiguous, C order; all pointers DEVICE memory of the current
+ * device, 16-byte aligned):
+ *   x       (B, L, D)  dtype    the input branch, channels last
+ *   conv_w  (K, D, 4)  float32  taps, oldest step first
+ *   conv_b  (K, D)     float32
+ *   W_x     (K, 1 + 2N, D) float32   x_proj weight (row 0: dt, then B, then C)
+ *   w_dt    (K, D)     float32  dt_proj weight
+ *   A_log   (K*D, N), Dskip (K*D), delta_bias (K*D)  float32, as selective_scan_fwd
+ *   y       (B, D, L)  float32, overwritten
+ * K in {1, 2}, N in 1..64, dtype any ss2d_dtype.  Scratch (u, dt_raw, B, C
+ * with rows padded to a multiple of 8 steps, and the scan's scratch) comes
+ * from the stream-ordered pool on `stream`; asynchronous.  A tensor-core
+ * completion wait that runs out of time (2 s) is recorded for
+ * ss2d_check_waits(); the call's y is then not valid. */
+int selective_scan_fwd_front(const void *x, const float *conv_w, const float *conv_b,
+                             const float *W_x, const float *w_dt, const float *A_log,
+                             const float *Dskip, const float *delta_bias, float *y,
+                             int B, int D, int L, int N, int K, int dtype, void *stream);
+
+/* selective_scan_fwd_front that also synchronises `stream` and returns the
+ * device time of its launches in launch_ms[0..2] (milliseconds, CUDA events
+ * on `stream`): the front kernel, the scan passes, cross_merge (-1 when not
+ * launched, K = 1).  For benchmarks. */
+int selective_scan_fwd_front_timed(const void *x, const float *conv_w, const float *conv_b,
+                                   const float *W_x, const float *w_dt, const float *A_log,
+                                   const float *Dskip, const float *delta_bias, float *y,
+                                   int B, int D, int L, int N, int K, int dtype, void *stream,
+                                   float *launch_ms);
+
+/* The front alone (same definition and layouts as selective_scan_fwd_front),
+ * for callers that run their own scan: writes u (B, K, D, L) in the input
+ * dtype and dt_raw (B, K, L), Bs, Cs (B, K, N, L) float32, each in its
+ * direction's scan order.  L must be a multiple of 8 (SS2D_ERR_SHAPE
+ * otherwise).  Device pointers only; asynchronous. */
+int ss2d_front_project(const void *x, const float *conv_w, const float *conv_b,
+                       const float *W_x, void *u, float *dt_raw, float *Bs, float *Cs,
+                       int B, int D, int L, int N, int K, int dtype, void *stream);
+
+/* Bounded waits.  The kernels that wait on an mbarrier (the front's
+ * tensor-core completion) give up after a time limit instead of spinning
+ * forever; they then record the fault in a device word and finish without
+ * writing their outputs, so the CUDA context stays usable.  This call reads
+ * that word on the current device (a blocking copy: call it after the
+ * stream work it is meant to check), clears it, and returns SS2D_ERR_CUDA
+ * with a description in ss2d_last_error() if a wait ran out, SS2D_OK
+ * otherwise. */
+int ss2d_check_waits(void);
+
+/* Enqueue a kernel whose one wait can never complete (an mbarrier that
+ * nothing arrives on), with a limit of limit_us microseconds (1..10^6): it
+ * gives up, records the fault and returns; ss2d_check_waits() then reports
+ * it.  A check of the time-out path itself. */
+int ss2d_wait_selftest(int limit_us, void *stream);
+
 /* Static text for a status code. */
 const char *ss2d_status_string(int status);
 

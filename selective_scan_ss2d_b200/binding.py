@@ -88,6 +88,17 @@ def lib() -> ctypes.CDLL:
             L.ss2d_variant_name.restype = ctypes.c_char_p
             L.ss2d_pick_variant.argtypes = [i] * 7
             L.ss2d_pick_variant.restype = i
+            L.selective_scan_fwd_front.argtypes = [vp] + [fp] * 8 + [i] * 6 + [vp]
+            L.selective_scan_fwd_front.restype = i
+            L.selective_scan_fwd_front_timed.argtypes = ([vp] + [fp] * 8 + [i] * 6 +
+                                                         [vp, ctypes.POINTER(ctypes.c_float)])
+            L.selective_scan_fwd_front_timed.restype = i
+            L.ss2d_front_project.argtypes = [vp, fp, fp, fp, vp, fp, fp, fp] + [i] * 6 + [vp]
+            L.ss2d_front_project.restype = i
+            L.ss2d_check_waits.argtypes = []
+            L.ss2d_check_waits.restype = i
+            L.ss2d_wait_selftest.argtypes = [i, vp]
+            L.ss2d_wait_selftest.restype = i
             L.ss2d_status_string.argtypes = [i]
             L.ss2d_status_string.restype = ctypes.c_char_p
             L.ss2d_last_error.argtypes = []
@@ -402,3 +413,100 @@ def forward_final_state(x, delta, A_log, Bs, Cs, Dskip, delta_bias, *, stream=No
         rc = lib().selective_scan_fwd_final_state(*args, B, D, L, N, K, dt, st, int(variant))
     _check(rc)
     return y, h_last
+
+
+def _front_checks(x, conv_w, conv_b, W_x, w_dt, K, what):
+    if x.dtype not in _DTYPES:
+        raise TypeError(f"x must be float32, bfloat16 or float16, got {x.dtype}")
+    B, L, D = x.shape
+    R = W_x.shape[1] if W_x.dim() == 3 else -1
+    N = (R - 1) // 2
+    if tuple(conv_w.shape) != (K, D, 4) or tuple(conv_b.shape) != (K, D) \
+            or W_x.dim() != 3 or tuple(W_x.shape) != (K, 1 + 2 * N, D) or N < 1 \
+            or (w_dt is not None and tuple(w_dt.shape) != (K, D)):
+        raise ValueError(f"inconsistent shapes for {what}")
+    for t in (conv_w, conv_b, W_x) + ((w_dt,) if w_dt is not None else ()):
+        if t.dtype != torch.float32:
+            raise TypeError("conv_w, conv_b, W_x and w_dt must be float32")
+    for t in (x, conv_w, conv_b, W_x) + ((w_dt,) if w_dt is not None else ()):
+        if not t.is_cuda or t.device != x.device:
+            raise ValueError(f"{what} takes device tensors on one device")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+    return B, L, D, N
+
+
+def selective_scan_fwd_front(x, conv_w, conv_b, W_x, w_dt, A_log, Dskip, delta_bias, y=None,
+                             *, stream=None):
+    """The fused front (causal depthwise conv1d + SiLU + x_proj on the tensor
+    cores + dt_proj) of every direction, then its selective scan, directions
+    summed.  x (B, L, D) input branch; conv_w (K, D, 4), conv_b (K, D), W_x
+    (K, 1 + 2N, D), w_dt (K, D); A_log (K*D, N), Dskip, delta_bias (K*D,)
+    float32.  Returns y (B, D, L) float32.  Device tensors only."""
+    K = conv_w.shape[0]
+    B, L, D, N = _front_checks(x, conv_w, conv_b, W_x, w_dt, K, "selective_scan_fwd_front")
+    for t in (A_log, Dskip, delta_bias):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("A_log, Dskip and delta_bias must be contiguous float32 device tensors")
+    if tuple(A_log.shape) != (K * D, N) or tuple(Dskip.shape) != (K * D,) \
+            or tuple(delta_bias.shape) != (K * D,):
+        raise ValueError("inconsistent shapes for selective_scan_fwd_front")
+    if y is None:
+        y = torch.empty((B, D, L), dtype=torch.float32, device=x.device)
+    if y.dtype != torch.float32 or tuple(y.shape) != (B, D, L) or not y.is_contiguous() \
+            or not y.is_cuda:
+        raise ValueError(f"y must be a contiguous float32 device tensor of shape {(B, D, L)}")
+    st = _stream(True, x.device, stream)
+    rc = lib().selective_scan_fwd_front(_ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(W_x),
+                                        _ptr(w_dt), _ptr(A_log), _ptr(Dskip), _ptr(delta_bias),
+                                        _ptr(y), B, D, L, N, K, _DTYPES[x.dtype], st)
+    _check(rc)
+    return y
+
+
+def selective_scan_fwd_front_timed(x, conv_w, conv_b, W_x, w_dt, A_log, Dskip, delta_bias, y,
+                                   *, stream=None):
+    """selective_scan_fwd_front into y, synchronised; returns the device
+    milliseconds of [front kernel, scan passes, cross_merge] (-1: not run)."""
+    K = conv_w.shape[0]
+    B, L, D, N = _front_checks(x, conv_w, conv_b, W_x, w_dt, K, "selective_scan_fwd_front")
+    if y.dtype != torch.float32 or tuple(y.shape) != (B, D, L) or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous float32 device tensor of shape {(B, D, L)}")
+    ms = (ctypes.c_float * 3)()
+    st = _stream(True, x.device, stream)
+    rc = lib().selective_scan_fwd_front_timed(_ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(W_x),
+                                              _ptr(w_dt), _ptr(A_log), _ptr(Dskip),
+                                              _ptr(delta_bias), _ptr(y), B, D, L, N, K,
+                                              _DTYPES[x.dtype], st, ms)
+    _check(rc)
+    return [ms[0], ms[1], ms[2]]
+
+
+def ss2d_front_project(x, conv_w, conv_b, W_x, *, stream=None):
+    """The front alone: returns (u (B, K, D, L) in x's dtype, dt_raw (B, K, L),
+    Bs, Cs (B, K, N, L) float32), each in its direction's scan order.  L must
+    be a multiple of 8.  Device tensors only."""
+    K = conv_w.shape[0]
+    B, L, D, N = _front_checks(x, conv_w, conv_b, W_x, None, K, "ss2d_front_project")
+    dev = x.device
+    u = torch.empty((B, K, D, L), dtype=x.dtype, device=dev)
+    dt_raw = torch.empty((B, K, L), dtype=torch.float32, device=dev)
+    Bs = torch.empty((B, K, N, L), dtype=torch.float32, device=dev)
+    Cs = torch.empty((B, K, N, L), dtype=torch.float32, device=dev)
+    st = _stream(True, dev, stream)
+    rc = lib().ss2d_front_project(_ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(W_x), _ptr(u),
+                                  _ptr(dt_raw), _ptr(Bs), _ptr(Cs), B, D, L, N, K,
+                                  _DTYPES[x.dtype], st)
+    _check(rc)
+    return u, dt_raw, Bs, Cs
+
+
+def ss2d_check_waits() -> int:
+    """Status of the library's bounded waits on the current device since the
+    last check (0, or -8 if one ran out); clears the record."""
+    return lib().ss2d_check_waits()
+
+
+def ss2d_wait_selftest(limit_us: int, *, stream=None) -> None:
+    """Enqueue the wait that cannot complete, limited to limit_us."""
+    _check(lib().ss2d_wait_selftest(int(limit_us), _stream(True, None, stream)))

@@ -4,6 +4,7 @@
 #include <cuda_fp16.h>
 
 #include "ss2d_backward.cuh"
+#include "ss2d_scan.cuh"
 #include "ss2d_launch.h"
 
 namespace ss2d {
@@ -24,7 +25,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
-        // the forward's carry over the chunk end states, then over the
+        // the forward's carry scan over the chunk end states, then over the
         // reversed local adjoints
         ScanParams c{};
         c.A_log = p.A_log;
@@ -36,17 +37,14 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
         c.NS = p.NS;
         c.L = p.L;
         c.NC = p.NC;
-        const long long total = (long long)p.B * p.K * p.D * kNP;
-        const dim3 cgrid((unsigned)((total + 255) / 256));
         c.hstate = p.hfwd;
         c.dtsum = p.dtf;
-        carry_kernel<<<cgrid, 256, 0, st>>>(c);
-        if (p.adj_chunks) {
+        e = launch_carry_scan(c, st, false);
+        if (e == cudaSuccess && p.adj_chunks) {
             c.hstate = p.hadj;
             c.dtsum = p.dta;
-            carry_kernel<<<cgrid, 256, 0, st>>>(c);
+            e = launch_carry_scan(c, st, false);
         }
-        e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
     }

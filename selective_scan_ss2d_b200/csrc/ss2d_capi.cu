@@ -167,6 +167,7 @@ ss2d::ScanParams make_params(const Problem &pr)
     p.two_d = pr.two_d;
     p.hlast = pr.hlast;
     p.NS = pr.N;
+    p.LP = pr.H * pr.W;
     return p;
 }
 
@@ -464,6 +465,7 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
 }  // namespace
 
 namespace ss2d {
+int scratch_alloc(void **ptr, size_t bytes, cudaStream_t st) { return pool_alloc(ptr, bytes, st); }
 void record_error(const char *what, cudaError_t e) { set_error(what, e); }
 void record_message(const char *text) { snprintf(g_last_error, sizeof(g_last_error), "%s", text); }
 }  // namespace ss2d
@@ -591,7 +593,8 @@ int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
     if (num_chunks)
         *num_chunks = pl.NC;
     if (launches)
-        *launches = pl.launches + (pl.NC > 1 ? 3 : 1) * ((N + ss2d::kNP - 1) / ss2d::kNP - 1);
+        *launches = pl.launches + (pl.NC > 2 ? 3 : pl.NC > 1 ? 2 : 1) *
+                                      ((N + ss2d::kNP - 1) / ss2d::kNP - 1);
     return SS2D_OK;
 }
 

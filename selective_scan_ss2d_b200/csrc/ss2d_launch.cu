@@ -1,8 +1,11 @@
 // ss2d_launch.cu -- kernel variants, the execution plan of a call, launchers.
 #include "ss2d_launch.h"
 
+#include <cuda_bf16.h>
+
 #include "ss2d_kernels.cuh"
 #include "ss2d_quad.cuh"
+#include "ss2d_scan.cuh"
 
 namespace ss2d {
 
@@ -22,6 +25,9 @@ const VariantInfo kVariants[] = {
     {"quad4_lc512", 4, 512, 128, 1},
     {"wc2_lc256_r168", 2, 256, 168}, {"wc2_lc512_r168", 2, 512, 168},
     {"wc2_lcfit_r168", 2, -2, 168},
+    {"lane2_wave", 2, -3, 128, 2},   {"lane2_nochunk", 2, -1, 128, 2},
+    {"lane2_lc128", 2, 128, 128, 2}, {"lane2_lc16", 2, 16, 128, 2},
+    {"lane2_wave_r168", 2, -3, 168, 2}, {"lane2_lc112_r168", 2, 112, 168, 2},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
@@ -37,6 +43,21 @@ const VariantInfo *variant(int i)
 }
 
 namespace {
+// CTAs of lane_scan_kernel resident on one SM (2-byte inputs, aligned rows,
+// 128 registers per thread): limited by registers and by the 228 KB of shared
+// memory per SM (1 KB of it reserved per CTA)
+int lane_ctas_per_sm(int wc, bool cols)
+{
+    const size_t smem = wc == 2 ? (cols ? LaneShape<__nv_bfloat16, 2, true, true>::SMEM_BYTES
+                                        : LaneShape<__nv_bfloat16, 2, false, true>::SMEM_BYTES)
+                                : (cols ? LaneShape<__nv_bfloat16, 4, true, true>::SMEM_BYTES
+                                        : LaneShape<__nv_bfloat16, 4, false, true>::SMEM_BYTES);
+    const int by_regs = 65536 / (32 * wc * 128);
+    const int by_smem = (int)((228u * 1024u) / (smem + 1024u));
+    int n = by_regs < by_smem ? by_regs : by_smem;
+    return n < 1 ? 1 : (n > 32 ? 32 : n);
+}
+
 // Sequences of a call are split into chunks when there are too few of them
 // to give every SM sub-partition about four resident warps.
 constexpr long long kWantLanes = 148LL * 16 * 32;
@@ -92,6 +113,20 @@ Plan make_plan(int v, int B, int D, int L, int K)
         }
         if (lc > L)
             lc = L;
+    } else if (vi->chunk == -3) {
+        // about one wave of CTAs: the chunks that fill the CTAs resident on
+        // 148 SMs (2-byte inputs, 128 registers per thread), at least 64 steps each
+        const long long seqs = (long long)B * K * D;
+        long long nc = 1;
+        if (wants_chunks(seqs, L)) {
+            const long long ctas_per_chunk = (long long)((D + 32 * vi->wc - 1) / (32 * vi->wc)) * K * B;
+            nc = (148LL * lane_ctas_per_sm(vi->wc, K == 4)) / (ctas_per_chunk > 0 ? ctas_per_chunk : 1);
+            if (nc < 2)
+                nc = 2;
+        }
+        lc = (int)((L + nc - 1) / nc);
+        if (lc < 64)
+            lc = L < 64 ? L : 64;
     } else if (vi->chunk < 0) {
         lc = L;
     } else {
@@ -115,13 +150,16 @@ Plan make_plan(int v, int B, int D, int L, int K)
         lc = kT;
     pl.LC = lc;
     pl.NC = (L + lc - 1) / lc;
-    pl.launches = (pl.NC > 1 ? 3 : 1) + (K > 1 ? 1 : 0);
+    // chunked: state pass, carry (none with two chunks), output pass
+    pl.launches = (pl.NC > 2 ? 3 : pl.NC > 1 ? 2 : 1) + (K > 1 ? 1 : 0);
     return pl;
 }
 
 cudaError_t launch_scan(const Plan &plan, int dtype, ScanParams &p, cudaStream_t st,
                         cudaEvent_t *ev)
 {
+    if (p.front && plan.layout != 2)
+        return cudaErrorInvalidValue;   // only the lane kernel reads the front's rows
     p.LC = plan.LC;
     p.NC = plan.NC;
     // more than 16 states: the passes once per group of at most 16 states, in

@@ -35,14 +35,15 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 
 // A kernel variant: layout, CTA width (wc warps) and chunking policy
 // (chunk = 0: chosen from the shape; chunk > 0: that many steps per chunk;
-// chunk = -2: about 128 steps, fitted to the sequence length; chunk = -1:
-// never chunk).
+// chunk = -2: about 128 steps, fitted to the sequence length; chunk = -3:
+// chunks for about one wave of CTAs; chunk = -1: never chunk).
 struct VariantInfo {
     const char *name;
     int wc;
     int chunk;
     int regs;   // register cap per thread the kernels are compiled for
-    int layout; // 0: one lane per channel (chunk_scan_kernel); 1: four (quad_scan_kernel)
+    int layout; // 0: one lane per channel (chunk_scan_kernel); 1: four (quad_scan_kernel);
+                // 2: one lane per channel, cp.async staging (lane_scan_kernel)
 };
 
 // How one call is executed.
@@ -94,6 +95,9 @@ cudaError_t launch_backward(const BwdParams &p, int dtype, cudaStream_t st);
 // the per-chunk-group partials
 cudaError_t launch_backward_reduce(const BwdParams &p, float *dBs, float *dCs, float *dA_log,
                                    float *dDskip, float *ddelta_bias, cudaStream_t st);
+
+// Scratch from the device's stream-ordered pool (ss2d_capi.cu), on st.
+int scratch_alloc(void **ptr, size_t bytes, cudaStream_t st);
 
 // Text that ss2d_last_error() returns on the calling thread.
 void record_error(const char *what, cudaError_t e);

@@ -136,6 +136,7 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     p.H = H;
     p.W = W;
     p.L = (int)L;
+    p.LP = (int)L;
     p.N = N;
     p.NS = N;
     p.K = K;

@@ -32,6 +32,14 @@ struct ScanParams {
     int n0;                   // first state of this group
     int NS;                   // states per row of A_log, Bs, Cs, hlast (N is this group's count)
     int accum;                // 1: add this group's output to `out` (skip term left out)
+    // row pitch (elements) of the rows of x / u, delta, Bs and Cs: L for the
+    // caller's arrays, L rounded up to 8 for the fused front's scratch
+    int LP;
+    // fused front: u per direction (B,K,D,LP) in scan order in x, no delta;
+    // delta = w_dt[k*D+d] * dt_raw[b,k,l]; Bs, Cs float32 (B,K,N,LP)
+    int front;
+    const float *dt_raw;      // (B,K,LP)
+    const float *w_dt;        // (K*D)
 };
 
 }  // namespace ss2d

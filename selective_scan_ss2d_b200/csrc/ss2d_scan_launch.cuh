@@ -8,6 +8,7 @@
 #include "ss2d_kernels.cuh"
 #include "ss2d_launch.h"
 #include "ss2d_quad.cuh"
+#include "ss2d_scan.cuh"
 
 namespace ss2d {
 namespace {
@@ -53,13 +54,62 @@ cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st, bool depe
                          dependent, p);
 }
 
+// lane_scan_kernel with a cap of R registers per thread (128: 16 warps per
+// SM; 168: 12)
+template <typename Tin, int WC, int R, int MODE, bool C, int Q, bool A, bool F = false>
+cudaError_t launch_lane_k(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
+{
+    using Sh = LaneShape<Tin, WC, C, A, F>;
+    constexpr int MB = 65536 / (32 * WC * R);
+    auto kern = lane_scan_kernel<Tin, WC, MODE, MB, C, Q, A, F>;
+    const size_t smem = Sh::SMEM_BYTES;
+    // the largest shared-memory carveout, so that 16 warps per SM fit
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    const long long blocks = (long long)((p.D + Sh::NT - 1) / Sh::NT) * p.K * p.B * ncg;
+    if (blocks > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    return launch_kernel(kern, dim3((unsigned)blocks), dim3(Sh::NT), smem, st, dependent, p);
+}
+
+template <typename Tin, int WC, int R, int MODE>
+cudaError_t launch_lane(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
+{
+    // the column-major path only where a direction is column-major; half the
+    // state work when this call (or state group) has at most 8 states; packed
+    // row copies when every row starts on an 8-byte boundary
+    const bool cols = p.two_d && p.K == 4, eight = p.N <= 8, aligned = p.vec >= 8;
+    if (p.front)   // the fused front's scratch rows: 1D, aligned
+        return eight ? launch_lane_k<Tin, WC, R, MODE, false, 2, true, true>(p, ncg, st, dependent)
+                     : launch_lane_k<Tin, WC, R, MODE, false, 4, true, true>(p, ncg, st, dependent);
+    if (cols) {
+        if (eight)
+            return aligned ? launch_lane_k<Tin, WC, R, MODE, true, 2, true>(p, ncg, st, dependent)
+                           : launch_lane_k<Tin, WC, R, MODE, true, 2, false>(p, ncg, st, dependent);
+        return aligned ? launch_lane_k<Tin, WC, R, MODE, true, 4, true>(p, ncg, st, dependent)
+                       : launch_lane_k<Tin, WC, R, MODE, true, 4, false>(p, ncg, st, dependent);
+    }
+    if (eight)
+        return aligned ? launch_lane_k<Tin, WC, R, MODE, false, 2, true>(p, ncg, st, dependent)
+                       : launch_lane_k<Tin, WC, R, MODE, false, 2, false>(p, ncg, st, dependent);
+    return aligned ? launch_lane_k<Tin, WC, R, MODE, false, 4, true>(p, ncg, st, dependent)
+                   : launch_lane_k<Tin, WC, R, MODE, false, 4, false>(p, ncg, st, dependent);
+}
+
 template <typename Tin, int LAYOUT, int WC, int R, int MODE>
 cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
     if constexpr (LAYOUT == 0)
         return launch_chunk<Tin, WC, MODE, R>(p, ncg, st, dependent);
-    else
+    else if constexpr (LAYOUT == 1)
         return launch_quad<Tin, MODE, WC, R>(p, ncg, st, dependent);
+    else
+        return launch_lane<Tin, WC, R, MODE>(p, ncg, st, dependent);
 }
 
 template <typename Tin, int LAYOUT, int WC, int R>
@@ -74,10 +124,10 @@ cudaError_t launch_passes(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
             return e;
         if (ev)
             cudaEventRecord(ev[1], st);
-        const long long total = (long long)p.B * p.K * p.D * kNP;
-        const int threads = 256;
-        e = launch_kernel(carry_kernel, dim3((unsigned)((total + threads - 1) / threads)),
-                          dim3(threads), 0, st, ev == nullptr, p);
+        // with two chunks the end state of the first is already the entry
+        // state of the second: no carry to combine
+        if (plan.NC > 2)
+            e = launch_carry_scan(p, st, ev == nullptr);
         if (e != cudaSuccess)
             return e;
     }
@@ -104,6 +154,8 @@ cudaError_t launch_scan_t(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
     SS2D_DISPATCH(0, 2, 168)
     SS2D_DISPATCH(0, 4, 168)
     SS2D_DISPATCH(1, 4, 128)
+    SS2D_DISPATCH(2, 2, 128)
+    SS2D_DISPATCH(2, 2, 168)
 #undef SS2D_DISPATCH
     return cudaErrorInvalidValue;
 }

@@ -214,3 +214,77 @@ def batch_subproblem(inp: Inputs, b: int) -> Inputs:
     sub = inp.cfg.with_(name=f"{inp.cfg.name}[b={b}]", B=1)
     return Inputs(sub, *[np.ascontiguousarray(getattr(inp, n)[b:b + 1]) for n in Inputs.STREAMED],
                   inp.A_log, inp.Dskip, inp.delta_bias)
+
+
+# ---------------------------------------------------------------------------
+# the fused front's inputs
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class FrontConfig:
+    name: str
+    B: int
+    L: int
+    D: int
+    N: int
+    K: int
+    dtype: str
+    description: str = ""
+
+    @property
+    def updates(self) -> int:
+        return self.B * self.K * self.D * self.L * self.N
+
+    def with_(self, **kw) -> "FrontConfig":
+        return dataclasses.replace(self, **kw)
+
+
+FRONT_CONFIGS = {
+    "vim_s_front": FrontConfig(
+        "vim_s_front", 128, 197, 768, 16, 2, BF16,
+        "Vim-S bidirectional block, front + scan: B=128, L=197 tokens, D=768, K=2, N=16"),
+}
+
+
+@dataclasses.dataclass
+class FrontInputs:
+    """One front workload: x (B, L, D) in storage form (float32, uint16
+    bfloat16 patterns or float16), the float32 weights of every direction and
+    the scan parameters."""
+    cfg: FrontConfig
+    x: np.ndarray
+    conv_w: np.ndarray      # (K, D, 4)
+    conv_b: np.ndarray      # (K, D)
+    W_x: np.ndarray         # (K, 1 + 2N, D)
+    w_dt: np.ndarray        # (K, D)
+    A_log: np.ndarray       # (K*D, N)
+    Dskip: np.ndarray       # (K*D,)
+    delta_bias: np.ndarray  # (K*D,)
+
+    WEIGHTS = ("conv_w", "conv_b", "W_x", "w_dt", "A_log", "Dskip", "delta_bias")
+
+    def x_f64(self) -> np.ndarray:
+        a = bf16_bits_to_f32(self.x) if self.cfg.dtype == BF16 else self.x
+        return a.astype(np.float64)
+
+
+def make_front_inputs(cfg: FrontConfig | str, seed: int = 0) -> FrontInputs:
+    """Seeded front inputs (PCG64, draws in this order): x ~ N(0, 1), conv
+    taps ~ N(0, 1/2), conv bias ~ N(0, 0.1^2), W_x ~ N(0, 1/D) (unit-scale
+    projections), w_dt ~ U(0.5, 1.5), then dt log-uniform in [1e-3, 1e-1] per
+    row k*D+d with delta_bias = ln(expm1(dt)); A_log = ln(n + 1), Dskip = 1 as
+    in the forward's recipe.  x is rounded to the storage dtype."""
+    if isinstance(cfg, str):
+        cfg = FRONT_CONFIGS[cfg]
+    rng = np.random.default_rng(seed)
+    B, L, D, N, K = cfg.B, cfg.L, cfg.D, cfg.N, cfg.K
+    x = _normal(rng, (B, L, D), cfg.dtype)
+    conv_w = (rng.standard_normal((K, D, 4)) * math.sqrt(0.5)).astype(np.float32)
+    conv_b = (rng.standard_normal((K, D)) * 0.1).astype(np.float32)
+    W_x = (rng.standard_normal((K, 1 + 2 * N, D)) / math.sqrt(D)).astype(np.float32)
+    w_dt = rng.uniform(0.5, 1.5, (K, D)).astype(np.float32)
+    dt = np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), size=K * D))
+    delta_bias = np.log(np.expm1(dt)).astype(np.float32)
+    A_log = np.repeat(np.log(np.arange(1, N + 1, dtype=np.float64))[None, :],
+                      K * D, axis=0).astype(np.float32)
+    Dskip = np.ones(K * D, dtype=np.float32)
+    return FrontInputs(cfg, x, conv_w, conv_b, W_x, w_dt, A_log, Dskip, delta_bias)
