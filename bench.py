@@ -65,7 +65,7 @@ NCU_TRAFFIC = {
 # the files that define the forward scan kernels and their launch (the
 # kernels the traffic figures above were taken from)
 FORWARD_KERNEL_SOURCES = ("ss2d_kernels.cuh", "ss2d_launch.cu", "ss2d_launch.h", "ss2d_params.h",
-                          "ss2d_quad.cuh", "ss2d_scan_bf16.cu", "ss2d_scan_f16.cu",
+                          "ss2d_scan.cuh", "ss2d_scan_bf16.cu", "ss2d_scan_f16.cu",
                           "ss2d_scan_f32.cu", "ss2d_scan_launch.cuh")
 
 

@@ -57,7 +57,7 @@
  *   delta_bias (K*D)          float32
  *   y          (B, D, H, W) / (B, D, L)  float32, pixel order, overwritten
  * where L = H*W.  Every pointer must be 16-byte aligned.  Limits: B <= 65535,
- * L < 2^31, and for ss2d_forward with K = 4 an image width W <= 512.
+ * L < 2^31.
  *
  * Precision: dtype is the storage type of x, delta, Bs and Cs; all
  * arithmetic and the state are float32.

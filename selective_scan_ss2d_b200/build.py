@@ -19,7 +19,7 @@ LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libss2d_b200.so")
 SOURCES = ["ss2d_capi.cu", "ss2d_launch.cu", "ss2d_noalloc.cu", "ss2d_scan_bf16.cu",
            "ss2d_scan_f32.cu", "ss2d_scan_f16.cu", "ss2d_backward.cu", "ss2d_front.cu"]
-HEADERS = ["ss2d_kernels.cuh", "ss2d_scan.cuh", "ss2d_front.cuh", "ss2d_quad.cuh", "ss2d_scan_launch.cuh", "ss2d_launch.h",
+HEADERS = ["ss2d_kernels.cuh", "ss2d_scan.cuh", "ss2d_front.cuh", "ss2d_scan_launch.cuh", "ss2d_launch.h",
            "ss2d_params.h", "ss2d_backward.cuh", "ss2d_bwd_params.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

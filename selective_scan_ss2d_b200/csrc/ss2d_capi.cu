@@ -124,8 +124,6 @@ int validate(const Problem &pr)
     const long long L = (long long)pr.H * pr.W;
     if (L > INT_MAX || pr.B > 65535 || (long long)pr.K * pr.D > INT_MAX)
         return SS2D_ERR_SHAPE;
-    if (pr.two_d && pr.K == 4 && pr.W > 512)
-        return SS2D_ERR_SHAPE;
     return SS2D_OK;
 }
 
@@ -189,10 +187,6 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     const size_t in_esz = pr.dtype == SS2D_F32 ? 4 : 2;   // bytes per stored input value
     const long long L = p.L;
     const ss2d::Plan pl = ss2d::make_plan(variant, pr.B, pr.D, (int)L, pr.K);
-    if ((long long)pr.B * pl.NC > 65535)
-        return SS2D_ERR_SHAPE;
-    if (ss2d::merge_smem_bytes(pr.H, pr.W, pr.K, pr.two_d) > 200 * 1024)
-        return SS2D_ERR_SHAPE;
     const bool need_part = pr.K > 1 || pr.z;   // gated calls always merge (the gate runs there)
     const size_t rows = (size_t)pr.B * pr.K * pr.D;
     const size_t part_bytes = need_part ? align256(sizeof(float) * rows * L) : 0;
@@ -387,8 +381,6 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
         }
         return SS2D_OK;
     }
-    if (pr.K > 1 && ss2d::merge_smem_bytes(pr.H, pr.W, pr.K, pr.two_d) > 200 * 1024)
-        return SS2D_ERR_SHAPE;
     const ss2d::BwdShape sh = ss2d::backward_shape(pr.B, pr.D, (int)L, pr.K);
     if ((long long)sh.G * pr.B * pr.K > INT_MAX)
         return SS2D_ERR_SHAPE;

@@ -15,8 +15,8 @@
 // enough lanes exist; the chunks are independent given their entry state:
 //   1. chunk_scan_kernel<..., kModeState>: every chunk but the last runs
 //      from a zero state and stores its end state and its sum of dt;
-//   2. carry_kernel: per (b,k,d,n), sequentially over the chunks,
-//      h_in[c+1] = exp(A_n * sum_c(dt)) * h_in[c] + h_end[c];
+//   2. carry_scan_kernel (ss2d_scan.cuh): the entry state of every chunk,
+//      an associative scan over the chunks of (exp(A_n * sum_c(dt)), h_end[c]);
 //   3. chunk_scan_kernel<..., kModeOutput>: every chunk from its true entry
 //      state, writing y_k in scan order (per-direction scratch, or y when
 //      K = 1);
@@ -285,13 +285,13 @@ __device__ __forceinline__ uint32_t raw_bits(const __half *p)
 }
 
 // One chunk of LC steps of 32*WC channels of one (b, k); see the header.
-// grid: x = k, y = channel tile, z = b * NCg + chunk, NCg = chunks launched
-// (NC - 1 in kModeState, NC in kModeOutput).
+// grid: x = k, y = channel tile, z = b * NCg + chunk (looped past 65535),
+// NCg = chunks launched (NC - 1 in kModeState, NC in kModeOutput).
 // COLS: the column-major directions (SS2D with K = 4) are compiled in.
 // QN: groups of 4 states the lane runs (4: up to 16 states; 2: up to 8, half
 // the exp2 and FMA work of a step).
-template <typename Tin, int WC, int MODE, int MINB, bool COLS, int QN>
-__global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
+template <typename Tin, int WC, int MODE, bool COLS, int QN>
+__device__ __forceinline__ void chunk_scan_body(const ScanParams &p, int zz)
 {
     static_assert(QN == 2 || QN == 4, "8 or 16 states per lane");
     using Sh = ChunkShape<WC>;
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W, K = p.K;
     const int k = blockIdx.x, tile = blockIdx.y;
     const int ncg = (MODE == kModeState) ? p.NC - 1 : p.NC;
-    const int b = blockIdx.z / ncg, chunk = blockIdx.z % ncg;
+    const int b = zz / ncg, chunk = zz % ncg;
     const int d0 = tile * NT;
     const int d = d0 + tid;
     const bool cvalid = d < D;
@@ -619,60 +619,15 @@ __global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanPar
     }
 }
 
-// Entry states of every chunk after the first, in place over the chunk end
-// states: slot c of (b,k,d) holds h_end of chunk c on entry and h_in of chunk
-// c+1 on exit.  One thread per (b, k, d, n).
-static __global__ void carry_kernel(const ScanParams p)
+// The kernel: grid z runs over (b, chunk) pairs, more than 65535 of them by
+// looping (z, z + gridDim.z, ...); every iteration ends on a CTA barrier.
+template <typename Tin, int WC, int MODE, int MINB, bool COLS, int QN>
+__global__ void __launch_bounds__(32 * WC, MINB) chunk_scan_kernel(const ScanParams p)
 {
-    grid_dependency_wait();   // the chunk end states of the state pass
-    allow_dependents();
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long total = (long long)p.B * p.K * p.D * kNP;
-    if (idx >= total)
-        return;
-    const int n = (int)(idx % kNP);
-    const long long bkd = idx / kNP;
-    const int d = (int)(bkd % p.D);
-    const int k = (int)((bkd / p.D) % p.K);
-    const float a2 =
-        n < p.N ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0 + n)) * kLog2e
-                : 0.f;
-    float *hs = p.hstate + (size_t)bkd * (p.NC - 1) * kNP + n;
-    const float *ds = p.dtsum + (size_t)bkd * (p.NC - 1);
-    const int nc1 = p.NC - 1;
-    // the loads do not depend on h: groups of G chunks, the next group in
-    // flight while the current one is applied
-    constexpr int G = 16;
-    float heA[G], dcA[G], heB[G], dcB[G];
-    auto load = [&](float *he, float *dc, int c0) {
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-            const bool ok = c0 + i < nc1;
-            he[i] = ok ? hs[(size_t)(c0 + i) * kNP] : 0.f;
-            dc[i] = ok ? ds[c0 + i] : 0.f;
-        }
-    };
-    float h = 0.f;
-    auto apply = [&](const float *he, const float *dc, int c0) {
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-            if (c0 + i < nc1) {
-                h = fmaf(mufu_ex2(a2 * dc[i]), h, he[i]);
-                hs[(size_t)(c0 + i) * kNP] = h;
-            }
-        }
-    };
-    load(heA, dcA, 0);
-    for (int c0 = 0; c0 < nc1; c0 += 2 * G) {
-        if (c0 + G < nc1)
-            load(heB, dcB, c0 + G);
-        apply(heA, dcA, c0);
-        if (c0 + G >= nc1)
-            break;
-        if (c0 + 2 * G < nc1)
-            load(heA, dcA, c0 + 2 * G);
-        apply(heB, dcB, c0 + G);
-    }
+    const int ncg = (MODE == kModeState) ? p.NC - 1 : p.NC;
+    const int nz = p.B * ncg;
+    for (int zz = blockIdx.z; zz < nz; zz += gridDim.z)
+        chunk_scan_body<Tin, WC, MODE, COLS, QN>(p, zz);
 }
 
 // cross_merge, band form: a CTA covers `rows` full image rows (the band
@@ -951,4 +906,38 @@ __global__ void __launch_bounds__(kMerge2Threads)
     }
 }
 
+// cross_merge, one pixel per thread: the plain form, for maps too wide for the
+// band form's shared-memory tiles.  Pixel p = h*W + w of channel (b, d):
+// direction 0's row is in pixel order, direction 1's too (the output pass
+// stores it flipped), direction 2 visits p at scan step w*H + h, direction 3
+// at L-1-(w*H + h).  sum = 1: y = ((Y_0 + Y_1) + Y_2) + Y_3 (first K terms),
+// times SiLU(z) when z is given; sum = 0: y[b,k,d,p] = Y_k.
+static __global__ void merge1_kernel(const float *__restrict__ part, float *__restrict__ y, int B,
+                                     int D, int H, int W, int K, int cols, int sum,
+                                     const void *__restrict__ z, int zt)
+{
+    grid_dependency_wait();   // the output pass's rows
+    const long long L = (long long)H * W;
+    const long long total = (long long)B * D * L;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long pix = i % L, bd = i / L;
+        const long long b = bd / D, d = bd % D;
+        const long long h = pix / W, w = pix % W;
+        const long long s2 = w * H + h;
+        float acc = 0.f;
+        for (int k = 0; k < K; ++k) {
+            const long long idx = (cols && k >= 2) ? (k == 2 ? s2 : L - 1 - s2) : pix;
+            const float v = part[((b * K + k) * D + d) * L + idx];
+            if (sum)
+                acc = k == 0 ? v : acc + v;
+            else
+                y[((b * K + k) * D + d) * L + pix] = v;
+        }
+        if (sum)
+            y[i] = z ? acc * gate1(z, zt, (size_t)i) : acc;
+    }
+}
+
 }  // namespace ss2d
+

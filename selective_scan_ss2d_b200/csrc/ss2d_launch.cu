@@ -4,7 +4,6 @@
 #include <cuda_bf16.h>
 
 #include "ss2d_kernels.cuh"
-#include "ss2d_quad.cuh"
 #include "ss2d_scan.cuh"
 
 namespace ss2d {
@@ -14,26 +13,37 @@ namespace {
 // name: wc<W>_<chunking>: one lane per channel, wc = 32-channel warps per CTA;
 // chunking: auto (from the shape), lc<N> (N steps), nochunk, lcfit (the
 // multiple of 16 in 96..160 that pads the sequence least, ties toward 128);
-// quad<W>_<chunking>: four lanes per channel, W warps of 8 channels per CTA.
+// lane<W>_<chunking>: the cp.async lane kernel (wave: chunks for about one wave).
 const VariantInfo kVariants[] = {
     {"wc2_auto", 2, 0, 128},       {"wc4_auto", 4, 0, 128},       {"wc1_auto", 1, 0, 128},
     {"wc2_lc16", 2, 16, 128},      {"wc4_lc64", 4, 64, 128},      {"wc2_nochunk", 2, -1, 128},
     {"wc2_lc256", 2, 256, 128},    {"wc4_lc512", 4, 512, 128},    {"wc1_lc128", 1, 128, 128},
     {"wc2_auto_r168", 2, 0, 168},  {"wc4_auto_r168", 4, 0, 168},  {"wc4_lc64_r168", 4, 64, 168},
     {"wc2_lc128_r168", 2, 128, 168},
-    {"quad4_auto", 4, 0, 128, 1},  {"quad4_nochunk", 4, -1, 128, 1},
-    {"quad4_lc512", 4, 512, 128, 1},
     {"wc2_lc256_r168", 2, 256, 168}, {"wc2_lc512_r168", 2, 512, 168},
     {"wc2_lcfit_r168", 2, -2, 168},
     {"lane2_wave", 2, -3, 128, 2},   {"lane2_nochunk", 2, -1, 128, 2},
     {"lane2_lc128", 2, 128, 128, 2}, {"lane2_lc16", 2, 16, 128, 2},
-    {"lane2_wave_r168", 2, -3, 168, 2}, {"lane2_lc112_r168", 2, 112, 168, 2},
 };
 constexpr int kNumVariants = sizeof(kVariants) / sizeof(kVariants[0]);
 
 }  // namespace
 
 int num_variants() { return kNumVariants; }
+
+int variant_index(const char *name)
+{
+    for (int i = 0; i < kNumVariants; ++i) {
+        const char *a = kVariants[i].name, *b = name;
+        while (*a && *a == *b) {
+            ++a;
+            ++b;
+        }
+        if (*a == 0 && *b == 0)
+            return i;
+    }
+    return -1;
+}
 
 const VariantInfo *variant(int i)
 {
@@ -43,16 +53,14 @@ const VariantInfo *variant(int i)
 }
 
 namespace {
-// CTAs of lane_scan_kernel resident on one SM (2-byte inputs, aligned rows,
-// 128 registers per thread): limited by registers and by the 228 KB of shared
-// memory per SM (1 KB of it reserved per CTA)
-int lane_ctas_per_sm(int wc, bool cols)
+// CTAs of lane_scan_kernel (two warps, 2-byte inputs, aligned rows, 128
+// registers per thread) resident on one SM: limited by registers and by the
+// 228 KB of shared memory per SM (1 KB of it reserved per CTA)
+int lane_ctas_per_sm(bool cols)
 {
-    const size_t smem = wc == 2 ? (cols ? LaneShape<__nv_bfloat16, 2, true, true>::SMEM_BYTES
-                                        : LaneShape<__nv_bfloat16, 2, false, true>::SMEM_BYTES)
-                                : (cols ? LaneShape<__nv_bfloat16, 4, true, true>::SMEM_BYTES
-                                        : LaneShape<__nv_bfloat16, 4, false, true>::SMEM_BYTES);
-    const int by_regs = 65536 / (32 * wc * 128);
+    const size_t smem = cols ? LaneShape<__nv_bfloat16, 2, true, true>::SMEM_BYTES
+                             : LaneShape<__nv_bfloat16, 2, false, true>::SMEM_BYTES;
+    const int by_regs = 65536 / (32 * 2 * 128);
     const int by_smem = (int)((228u * 1024u) / (smem + 1024u));
     int n = by_regs < by_smem ? by_regs : by_smem;
     return n < 1 ? 1 : (n > 32 ? 32 : n);
@@ -75,17 +83,17 @@ int pick_variant(int two_d, int B, int D, int H, int W, int N, int K)
     // chunked shapes: 128-step chunks with the 168-register kernels (fewer,
     // fuller warps hide the longer per-chunk dependency chains better)
     if (wants_chunks((long long)B * K * D, L))
-        return 18;  // wc2_lcfit_r168
+        return variant_index("wc2_lcfit_r168");
     // SS2D (four directions, two column-major) unchunked: 64-channel CTAs at
     // 168 registers
     if (two_d && K == 4 && D % 64 == 0)
-        return 9;   // wc2_auto_r168
+        return variant_index("wc2_auto_r168");
     // otherwise the widest CTA that leaves no channel tile mostly empty
     if (D % 128 == 0)
-        return 1;   // wc4_auto
+        return variant_index("wc4_auto");
     if (D % 64 == 0 || D > 64)
-        return 0;   // wc2_auto
-    return 2;       // wc1_auto
+        return variant_index("wc2_auto");
+    return variant_index("wc1_auto");
 }
 
 Plan make_plan(int v, int B, int D, int L, int K)
@@ -119,8 +127,9 @@ Plan make_plan(int v, int B, int D, int L, int K)
         const long long seqs = (long long)B * K * D;
         long long nc = 1;
         if (wants_chunks(seqs, L)) {
-            const long long ctas_per_chunk = (long long)((D + 32 * vi->wc - 1) / (32 * vi->wc)) * K * B;
-            nc = (148LL * lane_ctas_per_sm(vi->wc, K == 4)) / (ctas_per_chunk > 0 ? ctas_per_chunk : 1);
+            const int ch = 32 * vi->wc;   // channels per CTA
+            const long long ctas_per_chunk = (long long)((D + ch - 1) / ch) * K * B;
+            nc = (148LL * lane_ctas_per_sm(K == 4)) / (ctas_per_chunk > 0 ? ctas_per_chunk : 1);
             if (nc < 2)
                 nc = 2;
         }
@@ -133,14 +142,7 @@ Plan make_plan(int v, int B, int D, int L, int K)
         // enough lanes for about four resident warps per SM sub-partition on
         // 148 SMs; short sequences are never split
         const long long seqs = (long long)B * K * D;
-        long long nc;
-        if (vi->layout == 1) {
-            // quad: about eight resident warps per SM are enough
-            const long long lanes = seqs * kQLanes, want = kWantLanes / 2;
-            nc = (lanes < want && L > 512) ? (want + lanes - 1) / lanes : 1;
-        } else {
-            nc = wants_chunks(seqs, L) ? (kWantLanes + seqs - 1) / seqs : 1;
-        }
+        long long nc = wants_chunks(seqs, L) ? (kWantLanes + seqs - 1) / seqs : 1;
         if (nc < 1)
             nc = 1;
         lc = (int)((L + nc - 1) / nc);
@@ -250,19 +252,20 @@ cudaError_t launch_merge2(const MergeShape &m, const float *part, float *y, int 
 }
 }  // namespace
 
-size_t merge_smem_bytes(int H, int W, int K, int two_d)
-{
-    return merge_shape(1, H, W, K, two_d).smem;
-}
 
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st, const void *z, int zt)
 {
     const MergeShape m = merge_shape(D, H, W, K, two_d);
-    if (m.smem > kMergeSmemMax)
-        return cudaErrorInvalidValue;
-    if ((long long)B * D > 0x7fffffffLL * m.CG || m.nbands > 65535)
-        return cudaErrorInvalidConfiguration;
+    if (m.smem > kMergeSmemMax || m.nbands > 65535 || (long long)B * D > 0x7fffffffLL) {
+        // too wide (or too many bands) for the band form: one pixel per thread
+        const long long total = (long long)B * D * H * W;
+        long long blocks = (total + 255) / 256;
+        if (blocks > 148LL * 64)
+            blocks = 148LL * 64;
+        return launch_kernel(merge1_kernel, dim3((unsigned)blocks), dim3(256), 0, st, true, part,
+                             y, B, D, H, W, K, m.cols, sum, z, zt);
+    }
 #define SS2D_MERGE(V, C)                                                             \
     if (m.vec == V && m.CG == C)                                                     \
         return launch_merge2<V, C>(m, part, y, B, D, H, W, K, sum, st, z, zt);

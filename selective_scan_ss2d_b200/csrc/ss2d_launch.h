@@ -42,7 +42,7 @@ struct VariantInfo {
     int wc;
     int chunk;
     int regs;   // register cap per thread the kernels are compiled for
-    int layout; // 0: one lane per channel (chunk_scan_kernel); 1: four (quad_scan_kernel);
+    int layout; // 0: one lane per channel (chunk_scan_kernel);
                 // 2: one lane per channel, cp.async staging (lane_scan_kernel)
 };
 
@@ -58,6 +58,7 @@ struct Plan {
 };
 
 int num_variants();
+int variant_index(const char *name);   // -1 if there is no variant of that name
 const VariantInfo *variant(int i);
 int pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
 Plan make_plan(int variant, int B, int D, int L, int K);
@@ -79,7 +80,6 @@ cudaError_t launch_scan_f16(const Plan &plan, ScanParams &p, cudaStream_t st, cu
 cudaError_t launch_merge(const float *part, float *y, int B, int D, int H, int W, int K,
                          int two_d, int sum, cudaStream_t st, const void *z = nullptr,
                          int zt = 0);
-size_t merge_smem_bytes(int H, int W, int K, int two_d);
 
 // Backward pass (ss2d_backward.cu): chunks of 16 steps, NC per sequence; G
 // groups of 32 channels; CPB chunks per CTA in CGN groups.

@@ -91,8 +91,6 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     const int variant = ss2d::pick_variant(1, B, D, H, W, N, K);
     const long long L = (long long)H * W;
     const ss2d::Plan pl = ss2d::make_plan(variant, B, D, (int)L, K);
-    if ((long long)B * pl.NC > 65535 || ss2d::merge_smem_bytes(H, W, K, 1) > 200 * 1024)
-        return SS2D_ERR_SHAPE;
     const size_t rows = (size_t)B * K * D;
     const size_t part_bytes = K > 1 ? round256(sizeof(float) * rows * (size_t)L) : 0;
     const size_t hs_bytes =

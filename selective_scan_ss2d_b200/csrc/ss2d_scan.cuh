@@ -111,65 +111,71 @@ __device__ __forceinline__ uint32_t neg_inf_word()
 // Shared-memory plan of lane_scan_kernel (bytes; every offset a multiple of 16).
 // FRONT: the fused front's inputs -- no delta rows (a dt_raw row of the
 // direction is staged with B and C instead), float32 B and C.
-template <typename Tin, int WC, bool COLS, bool ALIGNED, bool FRONT = false>
+// CPL: channels per lane.
+template <typename Tin, int WC, bool COLS, bool ALIGNED, bool FRONT = false, int CPL = 1>
 struct LaneShape {
-    static constexpr int NT = 32 * WC;                  // threads = channels per CTA
+    static constexpr int NT = 32 * WC;                  // threads per CTA
+    static constexpr int CH = CPL * NT;                 // channels per CTA
     static constexpr int ESZ = (int)sizeof(Tin);
     static constexpr int EBC = FRONT ? 4 : ESZ;         // bytes of a B|C value
     // delta of 2-byte types from aligned rows: 16 values packed in 2 units of
     // 16 bytes; otherwise one word per step (4 units)
     static constexpr bool DPACK2 = ALIGNED && ESZ == 2;
-    static constexpr int UD = FRONT ? 0 : (DPACK2 ? 2 : 4);   // units per lane and stage
+    static constexpr int UD = FRONT ? 0 : (DPACK2 ? 2 : 4);   // units per channel and stage
     static constexpr int UX = (DPACK2 && !COLS) ? 2 : 4;
     static constexpr int RW = ALIGNED ? 4 * EBC : 16;   // words of a raw B|C row segment
     static constexpr int RS = RW;                       // their row stride
     static constexpr int BCS = 3;                       // raw B|C stages
     static constexpr int BCR = FRONT ? 33 : 32;         // raw rows: B, C (and dt_raw)
-    static constexpr size_t OFF_X = sizeof(uint4) * 2 * UD * NT;
-    static constexpr size_t OFF_BC = OFF_X + sizeof(uint4) * 2 * UX * NT;
+    static constexpr size_t OFF_X = sizeof(uint4) * 2 * CPL * UD * NT;
+    static constexpr size_t OFF_BC = OFF_X + sizeof(uint4) * 2 * CPL * UX * NT;
     static constexpr size_t OFF_BCF = OFF_BC + sizeof(uint32_t) * BCS * BCR * RS;
     static constexpr size_t OFF_DT = OFF_BCF + sizeof(float4) * 2 * 8 * kT;
     static constexpr size_t OFF_DU = OFF_DT + (FRONT ? sizeof(float) * 2 * kT : 0);
-    // per warp [kT][32] (dt, u) of the sub-chunk being computed; dt is
+    // per warp [kT][CPL][32] (dt, u) of the sub-chunk being computed; dt is
     // overwritten by the step's output
-    static constexpr size_t SMEM_BYTES = OFF_DU + sizeof(float2) * WC * kT * 32;
+    static constexpr size_t SMEM_BYTES = OFF_DU + sizeof(float2) * WC * kT * CPL * 32;
 };
 
-// One chunk of LC steps of 32*WC channels of one (b, k); see the header.
+// One chunk of LC steps of CPL*32*WC channels of one (b, k); see the header.
 // grid: x = ((b * NCg + chunk) * K + k) * tiles + tile, NCg = chunks
 // launched (NC - 1 in kModeState, NC in kModeOutput).
 // COLS: the column-major directions (SS2D with K = 4) are compiled in.
-// QN: groups of 4 states per lane (4: up to 16 states; 2: up to 8).
+// QN: groups of 4 states per channel (4: up to 16 states; 2: up to 8).
 // ALIGNED: delta, x and B|C rows start on 8-byte boundaries (p.vec = 8 or
 // 16): packed row copies; otherwise one word per step.
 // FRONT: the inputs of the fused front (p.front): u of every direction in
 // its scan order (B,K,D,LP), delta = w_dt * dt_raw, float32 B|C.
+// CPL: channels per lane (channel c of thread t: tile * CPL*NT + c*NT + t);
+// the B|C values of a step, read from shared memory once, serve all of them.
 template <typename Tin, int WC, int MODE, int MINB, bool COLS, int QN, bool ALIGNED,
-          bool FRONT = false>
+          bool FRONT = false, int CPL = 1>
 __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanParams p)
 {
-    static_assert(QN == 2 || QN == 4, "8 or 16 states per lane");
+    static_assert(QN == 2 || QN == 4, "8 or 16 states per channel");
     static_assert(kT == 16, "16-step sub-chunks");
+    static_assert(CPL == 1 || CPL == 2, "one or two channels per lane");
     static_assert(!FRONT || (ALIGNED && !COLS), "front inputs: aligned 1D rows");
-    using Sh = LaneShape<Tin, WC, COLS, ALIGNED, FRONT>;
+    using Sh = LaneShape<Tin, WC, COLS, ALIGNED, FRONT, CPL>;
     using Tbc = std::conditional_t<FRONT, float, Tin>;   // type of the B|C rows
-    constexpr int NT = Sh::NT, UD = Sh::UD, UX = Sh::UX, ESZ = Sh::ESZ, RS = Sh::RS;
-    constexpr int EBC = Sh::EBC, BCR = Sh::BCR;
+    constexpr int NT = Sh::NT, CH = Sh::CH, UD = Sh::UD, UX = Sh::UX, ESZ = Sh::ESZ;
+    constexpr int RS = Sh::RS, EBC = Sh::EBC, BCR = Sh::BCR;
     constexpr bool DPACK2 = Sh::DPACK2;
 
     extern __shared__ __align__(16) unsigned char lane_smem[];
-    uint4 *rawD = reinterpret_cast<uint4 *>(lane_smem);                   // [2][UD][NT]
-    uint4 *rawX = reinterpret_cast<uint4 *>(lane_smem + Sh::OFF_X);       // [2][UX][NT]
+    uint4 *rawD = reinterpret_cast<uint4 *>(lane_smem);                   // [2][CPL][UD][NT]
+    uint4 *rawX = reinterpret_cast<uint4 *>(lane_smem + Sh::OFF_X);       // [2][CPL][UX][NT]
     uint32_t *rawBC = reinterpret_cast<uint32_t *>(lane_smem + Sh::OFF_BC);   // [3][BCR][RS]
     float4 *BCf = reinterpret_cast<float4 *>(lane_smem + Sh::OFF_BCF);    // [2][8][kT]
     float *sDT = reinterpret_cast<float *>(lane_smem + Sh::OFF_DT);       // FRONT: [2][kT] dt_raw
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
-    float2 *sDU = reinterpret_cast<float2 *>(lane_smem + Sh::OFF_DU) + warp * (kT * 32) + lane;
+    // this lane's (dt, u) of step t, channel c at sDU[(t * CPL + c) * 32]
+    float2 *sDU = reinterpret_cast<float2 *>(lane_smem + Sh::OFF_DU) + warp * (kT * CPL * 32) + lane;
 
     const int D = p.D, L = p.L, N = p.N, H = p.H, W = p.W, K = p.K;
     const int ncg = (MODE == kModeState) ? p.NC - 1 : p.NC;
-    const int ntiles = (D + NT - 1) / NT;
+    const int ntiles = (D + CH - 1) / CH;
     int rest = blockIdx.x;
     const int tile = rest % ntiles;
     rest /= ntiles;
@@ -177,54 +183,61 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     rest /= K;
     const int chunk = rest % ncg;
     const int b = rest / ncg;
-    const int d = tile * NT + tid;
-    const bool cvalid = d < D;
-    const int dc = cvalid ? d : D - 1;       // clamped channel for addressing
-    const int kd = k * D + dc;
     const int l_begin = chunk * p.LC;
     const int l_end = min(l_begin + p.LC, L);
     const int nsub = (l_end - l_begin + kT - 1) / kT;
-
-    float2 A2[8];   // A[n] * log2(e) for states (2j, 2j+1)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int n0 = 2 * j, n1 = 2 * j + 1;
-        const float *al = p.A_log + (size_t)kd * p.NS + p.n0;
-        A2[j].x = (n0 < N) ? -expf(__ldg(al + n0)) * kLog2e : 0.f;
-        A2[j].y = (n1 < N) ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
-    }
     const bool accum = p.accum != 0;   // a later state group: add to out, no skip term
-    const float dsk = accum ? 0.f : __ldg(p.Dskip + kd);
-    const float bias = __ldg(p.delta_bias + kd);
-
     const size_t row_bk = ((size_t)b * K + k) * D;   // row index of (b, k, d = 0)
     const size_t LP = (size_t)p.LP;                  // row pitch of the input rows
-    const Tin *drow = FRONT ? nullptr : static_cast<const Tin *>(p.delta) + (row_bk + dc) * LP;
-    // x rows: the caller's (b, d) map, or the front's u row of (b, k, d)
-    const Tin *xrow = static_cast<const Tin *>(p.x) +
-                      (FRONT ? (row_bk + dc) : ((size_t)b * D + dc)) * LP;
+
+    // the lane's channels
+    int dch[CPL];           // channel
+    bool cvalid[CPL];
+    float2 A2[CPL][8];      // A[n] * log2(e) for states (2j, 2j+1)
+    float dsk[CPL], bias[CPL], wdt[CPL];
+    const Tin *drow[CPL], *xrow[CPL];
+    float2 h2[CPL][8];
+    float dtsum[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        dch[c] = tile * CH + c * NT + tid;
+        cvalid[c] = dch[c] < D;
+        const int dc = cvalid[c] ? dch[c] : D - 1;   // clamped channel for addressing
+        const int kd = k * D + dc;
+        const float *al = p.A_log + (size_t)kd * p.NS + p.n0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            A2[c][j].x = (2 * j < N) ? -expf(__ldg(al + 2 * j)) * kLog2e : 0.f;
+            A2[c][j].y = (2 * j + 1 < N) ? -expf(__ldg(al + 2 * j + 1)) * kLog2e : 0.f;
+            h2[c][j] = make_float2(0.f, 0.f);
+        }
+        dsk[c] = accum ? 0.f : __ldg(p.Dskip + kd);
+        bias[c] = __ldg(p.delta_bias + kd);
+        wdt[c] = FRONT ? __ldg(p.w_dt + kd) : 0.f;
+        drow[c] = FRONT ? nullptr : static_cast<const Tin *>(p.delta) + (row_bk + dc) * LP;
+        // x rows: the caller's (b, d) map, or the front's u row of (b, k, d)
+        xrow[c] = static_cast<const Tin *>(p.x) + (FRONT ? (row_bk + dc) : ((size_t)b * D + dc)) * LP;
+        dtsum[c] = 0.f;
+    }
     const size_t bc_row0 = ((size_t)b * K + k) * p.NS + p.n0;   // row of this group's state 0
     const Tbc *Bg = static_cast<const Tbc *>(p.Bs) + bc_row0 * LP;
     const Tbc *Cg = static_cast<const Tbc *>(p.Cs) + bc_row0 * LP;
     const float *dtg = FRONT ? p.dt_raw + ((size_t)b * K + k) * LP : nullptr;
-    const float wdt = FRONT ? __ldg(p.w_dt + kd) : 0.f;
     // x order of this direction: 0 forward, 1 reversed (both contiguous),
     // 2 column-major (one word per step); the front's u rows are in scan order
     const int xmode = FRONT ? 0 : ((COLS && k >= 2) ? 2 : (k & 1));
     const int vec = p.vec;
 
-    float2 h2[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        h2[j] = make_float2(0.f, 0.f);
-    float dtsum = 0.f;
-
     // ---- staging ---------------------------------------------------------
-    const uint32_t sD0 = smem_u32(rawD) + tid * 16;   // unit u of stage s: + (s*UD + u)*NT*16
+    // unit u of channel c, stage s: + ((s*CPL + c)*U + u)*NT*16
+    const uint32_t sD0 = smem_u32(rawD) + tid * 16;
     const uint32_t sX0 = smem_u32(rawX) + tid * 16;
     // word halves of the staged values (2-byte types, one word per step):
-    // bit i = half of step i, per stage
-    uint32_t dpar0 = 0u, dpar1 = 0u, xpar0 = 0u, xpar1 = 0u;
+    // bit i = half of step i, per stage and channel
+    uint32_t dpar[2][CPL], xpar[2][CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c)
+        dpar[0][c] = dpar[1][c] = xpar[0][c] = xpar[1][c] = 0u;
     PixWalk xw;   // column-major directions: pixel of the next step to copy
     xw.init(p.two_d, k, l_begin, H, W, L);
     const int adv_q = kT / H, adv_r = kT % H;
@@ -250,86 +263,102 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                           row + max(min(e0 + u * PE, lastp), 0));
         }
     };
+    auto set_par = [&](uint32_t (&par)[2][CPL], int s, int c, uint32_t m) {
+        if (s)
+            par[1][c] = m;
+        else
+            par[0][c] = m;
+    };
     auto issue_dx = [&](int s, int ls) {
-        const uint32_t dD = sD0 + s * UD * NT * 16, dX = sX0 + s * UX * NT * 16;
-        (void)dD;
-        // delta: steps ls.. of this lane's row
-        if constexpr (FRONT) {
-            // delta comes from the dt_raw row staged with B and C
-        } else if constexpr (ALIGNED) {
-            copy_packed(dD, drow, ls);   // 4-byte types: one word per step as well
-        } else {
-            uint32_t m = 0;
 #pragma unroll
-            for (int i = 0; i < kT; ++i)
-                m |= cp_async_word(dD + (i >> 2) * NT * 16 + (i & 3) * 4, drow + min(ls + i, L - 1), i);
-            if (s)
-                dpar1 = m;
-            else
-                dpar0 = m;
+        for (int c = 0; c < CPL; ++c) {
+            const uint32_t dD = sD0 + (s * CPL + c) * UD * NT * 16;
+            const uint32_t dX = sX0 + (s * CPL + c) * UX * NT * 16;
+            (void)dD;
+            // delta: steps ls.. of the channel's row
+            if constexpr (FRONT) {
+                // delta comes from the dt_raw row staged with B and C
+            } else if constexpr (ALIGNED) {
+                copy_packed(dD, drow[c], ls);   // 4-byte types: one word per step as well
+            } else {
+                uint32_t m = 0;
+#pragma unroll
+                for (int i = 0; i < kT; ++i)
+                    m |= cp_async_word(dD + (i >> 2) * NT * 16 + (i & 3) * 4,
+                                       drow[c] + min(ls + i, L - 1), i);
+                set_par(dpar, s, c, m);
+            }
+            // x of the row-major directions
+            if (xmode == 0) {
+                if constexpr (ALIGNED) {
+                    copy_packed(dX, xrow[c], ls);
+                } else {
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int i = 0; i < kT; ++i)
+                        m |= cp_async_word(dX + (i >> 2) * NT * 16 + (i & 3) * 4,
+                                           xrow[c] + min(ls + i, L - 1), i);
+                    set_par(xpar, s, c, m);
+                }
+            } else if (xmode == 1) {   // pixels L-1-ls-i
+                if constexpr (ALIGNED) {
+                    copy_packed(dX, xrow[c], L - kT - ls);   // ascending; step i reads index 15 - i
+                } else {
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int i = 0; i < kT; ++i)
+                        m |= cp_async_word(dX + (i >> 2) * NT * 16 + (i & 3) * 4,
+                                           xrow[c] + max(L - 1 - ls - i, 0), i);
+                    set_par(xpar, s, c, m);
+                }
+            }
         }
-        // x
-        if (xmode == 0) {
-            if constexpr (ALIGNED) {
-                copy_packed(dX, xrow, ls);
-            } else {
-                uint32_t m = 0;
+        // x of the column-major directions: one word per step and channel
+        // (the same pixel for every channel of the lane)
+        if constexpr (COLS) {
+            if (xmode == 2) {
+                uint32_t m[CPL];
 #pragma unroll
-                for (int i = 0; i < kT; ++i)
-                    m |= cp_async_word(dX + (i >> 2) * NT * 16 + (i & 3) * 4, xrow + min(ls + i, L - 1), i);
-                if (s)
-                    xpar1 = m;
-                else
-                    xpar0 = m;
-            }
-        } else if (xmode == 1) {   // pixels L-1-ls-i
-            if constexpr (ALIGNED) {
-                copy_packed(dX, xrow, L - kT - ls);   // ascending; step i reads index 15 - i
-            } else {
-                uint32_t m = 0;
+                for (int c = 0; c < CPL; ++c)
+                    m[c] = 0u;
+                auto copy_step = [&](int i, int pix) {
 #pragma unroll
-                for (int i = 0; i < kT; ++i)
-                    m |= cp_async_word(dX + (i >> 2) * NT * 16 + (i & 3) * 4,
-                                       xrow + max(L - 1 - ls - i, 0), i);
-                if (s)
-                    xpar1 = m;
-                else
-                    xpar0 = m;
-            }
-        } else if constexpr (COLS) {
-            uint32_t m = 0;
-            if (ls + kT <= L && H >= 8) {
-                // pixel of step ls + i without walking: each column wrap moves
-                // the pixel by L - 1 against the row stride; with H >= 8 at most
-                // two wraps fall in 16 steps (one when H >= 16)
-                const int p0 = xw.p, h0 = xw.h, Lm1 = L - 1;
+                    for (int c = 0; c < CPL; ++c)
+                        m[c] |= cp_async_word(sX0 + (s * CPL + c) * UX * NT * 16 + (i >> 2) * NT * 16 +
+                                                  (i & 3) * 4,
+                                              xrow[c] + pix, i);
+                };
+                if (ls + kT <= L && H >= 8) {
+                    // pixel of step ls + i without walking: each column wrap moves
+                    // the pixel by L - 1 against the row stride; with H >= 8 at most
+                    // two wraps fall in 16 steps (one when H >= 16)
+                    const int p0 = xw.p, h0 = xw.h, Lm1 = L - 1;
 #pragma unroll
-                for (int i = 0; i < kT; ++i) {
-                    int pix;
-                    if (k == 2) {
-                        const int hh = h0 + i;
-                        const int c = (hh >= H) + (H < kT && hh >= 2 * H);
-                        pix = p0 + i * W - c * Lm1;
-                    } else {
-                        const int hh = h0 - i;
-                        const int c = (hh < 0) + (H < kT && hh < -H);
-                        pix = p0 - i * W + c * Lm1;
+                    for (int i = 0; i < kT; ++i) {
+                        int pix;
+                        if (k == 2) {
+                            const int hh = h0 + i;
+                            const int cw = (hh >= H) + (H < kT && hh >= 2 * H);
+                            pix = p0 + i * W - cw * Lm1;
+                        } else {
+                            const int hh = h0 - i;
+                            const int cw = (hh < 0) + (H < kT && hh < -H);
+                            pix = p0 - i * W + cw * Lm1;
+                        }
+                        copy_step(i, pix);
                     }
-                    m |= cp_async_word(dX + (i >> 2) * NT * 16 + (i & 3) * 4, xrow + pix, i);
-                }
-                xw.advance(kT, adv_q, adv_r, H, W);
-            } else {
+                    xw.advance(kT, adv_q, adv_r, H, W);
+                } else {
 #pragma unroll
-                for (int i = 0; i < kT; ++i) {
-                    const int pix = (ls + i < L) ? xw.p : 0;
-                    m |= cp_async_word(dX + (i >> 2) * NT * 16 + (i & 3) * 4, xrow + pix, i);
-                    xw.next(H, W);
+                    for (int i = 0; i < kT; ++i) {
+                        copy_step(i, (ls + i < L) ? xw.p : 0);
+                        xw.next(H, W);
+                    }
                 }
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    set_par(xpar, s, c, m[c]);
             }
-            if (s)
-                xpar1 = m;
-            else
-                xpar0 = m;
         }
     };
     // B|C rows of sub-chunk ls into raw stage s: row r < 16 is B of state r,
@@ -410,107 +439,132 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     auto mask_tail = [&](int s, int valid) {
         if constexpr (FRONT)
             return;   // no final states here: steps past L are computed and never stored
-        uint32_t *dw = reinterpret_cast<uint32_t *>(rawD + (s * UD) * NT + tid);
-        for (int i = valid; i < kT; ++i) {
-            if constexpr (DPACK2) {
-                // step i: unit i / 8, word (i % 8) / 2, half i % 2
-                uint32_t *w = dw + (i >> 3) * NT * 4 + ((i & 7) >> 1);
-                const uint32_t ninf = neg_inf_word<Tin>();
-                *w = (i & 1) ? ((*w & 0xffffu) | (ninf & 0xffff0000u))
-                             : ((*w & 0xffff0000u) | (ninf & 0xffffu));
-            } else {
-                dw[(i >> 2) * NT * 4 + (i & 3)] = neg_inf_word<Tin>();
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            uint32_t *dw = reinterpret_cast<uint32_t *>(rawD + ((s * CPL + c) * UD) * NT + tid);
+            for (int i = valid; i < kT; ++i) {
+                if constexpr (DPACK2) {
+                    // step i: unit i / 8, word (i % 8) / 2, half i % 2
+                    uint32_t *w = dw + (i >> 3) * NT * 4 + ((i & 7) >> 1);
+                    const uint32_t ninf = neg_inf_word<Tin>();
+                    *w = (i & 1) ? ((*w & 0xffffu) | (ninf & 0xffff0000u))
+                                 : ((*w & 0xffff0000u) | (ninf & 0xffffu));
+                } else {
+                    dw[(i >> 2) * NT * 4 + (i & 3)] = neg_inf_word<Tin>();
+                }
             }
         }
     };
 
-    // ---- the 16 steps of one sub-chunk ------------------------------------
     // ---- the 16 steps of one sub-chunk --------------------------------------
-    // (dt, u) of every step from the raw tiles of stage s into this lane's
-    // column of the du tile: softplus of 16 independent steps at a time
+    // (dt, u) of every step and channel from the raw tiles of stage s into
+    // this lane's column of the du tile: softplus of 16 independent steps
     auto stage_du = [&](auto xm_c, int s, int buf) {
         constexpr int XM = decltype(xm_c)::value;
-        const uint4 *dU = rawD + (s * UD) * NT + tid;
-        const uint4 *xU = rawX + (s * UX) * NT + tid;
-        const uint32_t dp = s ? dpar1 : dpar0, xp = s ? xpar1 : xpar0;
-        (void)dp;
-        (void)xp;
         (void)buf;
-        uint4 dv = make_uint4(0, 0, 0, 0), xv = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int t = 0; t < kT; ++t) {
-            // delta of step t
-            float draw;
-            if constexpr (FRONT) {
-                draw = wdt * sDT[buf * kT + t];
-            } else if constexpr (DPACK2) {
-                if ((t & 7) == 0)
-                    dv = dU[(t >> 3) * NT];
-                draw = raw_value<Tin>(u4c(dv, (t >> 1) & 3), t & 1);
-            } else {
-                if ((t & 3) == 0)
-                    dv = dU[(t >> 2) * NT];
-                draw = raw_value<Tin>(u4c(dv, t & 3), ESZ == 2 ? (dp >> t) & 1u : 0u);
-            }
-            // x of step t
-            float u;
-            if constexpr (XM == 2 || !DPACK2) {
-                // one word per step (column-major, unaligned rows, 4-byte types);
-                // reversed rows of 4-byte types are packed ascending: index 15 - t
-                if constexpr (XM == 1 && ESZ == 4 && ALIGNED) {
-                    const int ti = kT - 1 - t;
-                    if ((t & 3) == 0)
-                        xv = xU[(ti >> 2) * NT];
-                    u = raw_value<Tin>(u4c(xv, ti & 3), 0u);
+        for (int c = 0; c < CPL; ++c) {
+            const uint4 *dU = rawD + ((s * CPL + c) * UD) * NT + tid;
+            const uint4 *xU = rawX + ((s * CPL + c) * UX) * NT + tid;
+            const uint32_t dp = s ? dpar[1][c] : dpar[0][c];
+            const uint32_t xp = s ? xpar[1][c] : xpar[0][c];
+            (void)dp;
+            (void)xp;
+            (void)dU;
+            uint4 dv = make_uint4(0, 0, 0, 0), xv = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int t = 0; t < kT; ++t) {
+                // delta of step t
+                float draw;
+                if constexpr (FRONT) {
+                    draw = wdt[c] * sDT[buf * kT + t];
+                } else if constexpr (DPACK2) {
+                    if ((t & 7) == 0)
+                        dv = dU[(t >> 3) * NT];
+                    draw = raw_value<Tin>(u4c(dv, (t >> 1) & 3), t & 1);
                 } else {
                     if ((t & 3) == 0)
-                        xv = xU[(t >> 2) * NT];
-                    u = raw_value<Tin>(u4c(xv, t & 3), ESZ == 2 ? (xp >> t) & 1u : 0u);
+                        dv = dU[(t >> 2) * NT];
+                    draw = raw_value<Tin>(u4c(dv, t & 3), ESZ == 2 ? (dp >> t) & 1u : 0u);
                 }
-            } else {
-                // packed 2-byte row: forward index t, reversed index 15 - t
-                const int ti = (XM == 1) ? kT - 1 - t : t;
-                if ((t & 7) == 0)
-                    xv = xU[(ti >> 3) * NT];
-                u = raw_value<Tin>(u4c(xv, (ti >> 1) & 3), ti & 1);
+                // x of step t
+                float u;
+                if constexpr (XM == 2 || !DPACK2) {
+                    // one word per step (column-major, unaligned rows, 4-byte
+                    // types); reversed rows of 4-byte types are packed
+                    // ascending: index 15 - t
+                    if constexpr (XM == 1 && ESZ == 4 && ALIGNED) {
+                        const int ti = kT - 1 - t;
+                        if ((t & 3) == 0)
+                            xv = xU[(ti >> 2) * NT];
+                        u = raw_value<Tin>(u4c(xv, ti & 3), 0u);
+                    } else {
+                        if ((t & 3) == 0)
+                            xv = xU[(t >> 2) * NT];
+                        u = raw_value<Tin>(u4c(xv, t & 3), ESZ == 2 ? (xp >> t) & 1u : 0u);
+                    }
+                } else {
+                    // packed 2-byte row: forward index t, reversed index 15 - t
+                    const int ti = (XM == 1) ? kT - 1 - t : t;
+                    if ((t & 7) == 0)
+                        xv = xU[(ti >> 3) * NT];
+                    u = raw_value<Tin>(u4c(xv, (ti >> 1) & 3), ti & 1);
+                }
+                const float dt = softplus_f(draw + bias[c]);
+                if (MODE == kModeState)
+                    dtsum[c] += dt;
+                sDU[(t * CPL + c) * 32] = make_float2(dt, u);
             }
-            const float dt = softplus_f(draw + bias);
-            if (MODE == kModeState)
-                dtsum += dt;
-            sDU[t * 32] = make_float2(dt, u);
         }
     };
-    // the recurrence over the staged steps, B|C from tile buf; the outputs
-    // replace dt in the du tile
+    // the recurrence over the staged steps, B|C from tile buf (each value
+    // read once for all channels of the lane); the outputs replace dt in the
+    // du tile
     auto steps = [&](int buf) {
         const float4 *sb = BCf + buf * 8 * kT;
-#pragma unroll 4
+#pragma unroll(CPL == 1 ? 4 : 1)
         for (int t = 0; t < kT; ++t) {
-            const float2 dtu = sDU[t * 32];
-            const float dt = dtu.x, u = dtu.y;
-            const float du = dt * u;
-            const float2 dt2 = make_float2(dt, dt);
-            const float2 du2 = make_float2(du, du);
+            float2 dt2[CPL], du2[CPL], acc0[CPL], acc1[CPL];
+            float uu[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const float2 dtu = sDU[(t * CPL + c) * 32];
+                uu[c] = dtu.y;
+                const float du = dtu.x * dtu.y;
+                dt2[c] = make_float2(dtu.x, dtu.x);
+                du2[c] = make_float2(du, du);
+                acc0[c] = make_float2(0.f, 0.f);
+                acc1[c] = make_float2(0.f, 0.f);
+            }
             const float4 *col = sb + t;   // slot q at col[q * kT]
-            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < QN; ++q) {
                 const float4 bv = col[q * kT];
-                const float2 arg0 = __fmul2_rn(dt2, A2[2 * q]);
-                const float2 arg1 = __fmul2_rn(dt2, A2[2 * q + 1]);
-                const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
-                const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
-                h2[2 * q] = __ffma2_rn(a0, h2[2 * q], __fmul2_rn(du2, make_float2(bv.x, bv.y)));
-                h2[2 * q + 1] =
-                    __ffma2_rn(a1, h2[2 * q + 1], __fmul2_rn(du2, make_float2(bv.z, bv.w)));
-                if (MODE == kModeOutput) {
-                    const float4 cv = col[(4 + q) * kT];
-                    acc0 = __ffma2_rn(make_float2(cv.x, cv.y), h2[2 * q], acc0);
-                    acc1 = __ffma2_rn(make_float2(cv.z, cv.w), h2[2 * q + 1], acc1);
+                float4 cv = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (MODE == kModeOutput)
+                    cv = col[(4 + q) * kT];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    const float2 arg0 = __fmul2_rn(dt2[c], A2[c][2 * q]);
+                    const float2 arg1 = __fmul2_rn(dt2[c], A2[c][2 * q + 1]);
+                    const float2 a0 = make_float2(mufu_ex2(arg0.x), mufu_ex2(arg0.y));
+                    const float2 a1 = make_float2(mufu_ex2(arg1.x), mufu_ex2(arg1.y));
+                    h2[c][2 * q] =
+                        __ffma2_rn(a0, h2[c][2 * q], __fmul2_rn(du2[c], make_float2(bv.x, bv.y)));
+                    h2[c][2 * q + 1] = __ffma2_rn(a1, h2[c][2 * q + 1],
+                                                  __fmul2_rn(du2[c], make_float2(bv.z, bv.w)));
+                    if (MODE == kModeOutput) {
+                        acc0[c] = __ffma2_rn(make_float2(cv.x, cv.y), h2[c][2 * q], acc0[c]);
+                        acc1[c] = __ffma2_rn(make_float2(cv.z, cv.w), h2[c][2 * q + 1], acc1[c]);
+                    }
                 }
             }
-            if (MODE == kModeOutput)
-                sDU[t * 32].x = fmaf(dsk, u, (acc0.x + acc0.y) + (acc1.x + acc1.y));
+            if (MODE == kModeOutput) {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    sDU[(t * CPL + c) * 32].x =
+                        fmaf(dsk[c], uu[c], (acc0[c].x + acc0[c].y) + (acc1[c].x + acc1[c].y));
+            }
         }
     };
 
@@ -524,13 +578,17 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     // stream wrote (entry states, the output rows)
     grid_dependency_wait();
     if (MODE == kModeOutput && chunk > 0) {
-        const float4 *hs = reinterpret_cast<const float4 *>(
-            p.hstate + ((row_bk + dc) * (p.NC - 1) + (chunk - 1)) * kNP);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = hs[q];
-            h2[2 * q] = make_float2(v.x, v.y);
-            h2[2 * q + 1] = make_float2(v.z, v.w);
+        for (int c = 0; c < CPL; ++c) {
+            const int dc = cvalid[c] ? dch[c] : D - 1;
+            const float4 *hs = reinterpret_cast<const float4 *>(
+                p.hstate + ((row_bk + dc) * (p.NC - 1) + (chunk - 1)) * kNP);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = hs[q];
+                h2[c][2 * q] = make_float2(v.x, v.y);
+                h2[c][2 * q + 1] = make_float2(v.z, v.w);
+            }
         }
     }
     cp_async_wait_all();
@@ -562,37 +620,44 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
             stage_du(std::integral_constant<int, 2>{}, s, s);
         steps(s);
 
-        if (MODE == kModeOutput && cvalid) {
-            // this lane's 16 outputs, one segment of its output row: in scan
-            // order, except direction 1 of a multi-direction call (the reversed
-            // row-major order), which is stored flipped, in pixel order
-            const bool flip = k == 1 && K > 1;
-            float *rowp = p.out + (row_bk + d) * (size_t)L;
-            if (p.ovec && l0 + kT <= l_end) {
-                float4 *orow = reinterpret_cast<float4 *>(rowp + (flip ? L - kT - l0 : l0));
+        if (MODE == kModeOutput) {
 #pragma unroll
-                for (int q = 0; q < kT / 4; ++q) {
-                    float4 v = flip ? make_float4(sDU[(15 - 4 * q) * 32].x,
-                                                  sDU[(14 - 4 * q) * 32].x,
-                                                  sDU[(13 - 4 * q) * 32].x,
-                                                  sDU[(12 - 4 * q) * 32].x)
-                                    : make_float4(sDU[(4 * q) * 32].x,
-                                                  sDU[(4 * q + 1) * 32].x,
-                                                  sDU[(4 * q + 2) * 32].x,
-                                                  sDU[(4 * q + 3) * 32].x);
-                    if (accum) {
-                        const float4 o = orow[q];
-                        v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+            for (int c = 0; c < CPL; ++c) {
+                if (!cvalid[c])
+                    continue;
+                // this channel's 16 outputs, one segment of its output row: in
+                // scan order, except direction 1 of a multi-direction call (the
+                // reversed row-major order), which is stored flipped, in pixel order
+                const bool flip = k == 1 && K > 1;
+                float *rowp = p.out + (row_bk + dch[c]) * (size_t)L;
+                const float2 *yc = sDU + c * 32;   // step t at yc[t * CPL * 32]
+                if (p.ovec && l0 + kT <= l_end) {
+                    float4 *orow = reinterpret_cast<float4 *>(rowp + (flip ? L - kT - l0 : l0));
+#pragma unroll
+                    for (int q = 0; q < kT / 4; ++q) {
+                        float4 v = flip ? make_float4(yc[(15 - 4 * q) * CPL * 32].x,
+                                                      yc[(14 - 4 * q) * CPL * 32].x,
+                                                      yc[(13 - 4 * q) * CPL * 32].x,
+                                                      yc[(12 - 4 * q) * CPL * 32].x)
+                                        : make_float4(yc[(4 * q) * CPL * 32].x,
+                                                      yc[(4 * q + 1) * CPL * 32].x,
+                                                      yc[(4 * q + 2) * CPL * 32].x,
+                                                      yc[(4 * q + 3) * CPL * 32].x);
+                        if (accum) {
+                            const float4 o = orow[q];
+                            v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+                        }
+                        orow[q] = v;
                     }
-                    orow[q] = v;
+                } else {
+#pragma unroll
+                    for (int t = 0; t < kT; ++t)
+                        if (l0 + t < l_end) {
+                            float *o = rowp + (flip ? L - 1 - l0 - t : l0 + t);
+                            const float y = yc[t * CPL * 32].x;
+                            *o = accum ? *o + y : y;
+                        }
                 }
-            } else {
-#pragma unroll
-                for (int t = 0; t < kT; ++t)
-                    if (l0 + t < l_end) {
-                        float *o = rowp + (flip ? L - 1 - l0 - t : l0 + t);
-                        *o = accum ? *o + sDU[t * 32].x : sDU[t * 32].x;
-                    }
             }
         }
         cp_async_wait_all();
@@ -602,23 +667,29 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     }
     allow_dependents();
 
-    if (MODE == kModeState && cvalid) {
-        float4 *hs = reinterpret_cast<float4 *>(
-            p.hstate + ((row_bk + d) * (p.NC - 1) + chunk) * kNP);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            hs[q] = make_float4(h2[2 * q].x, h2[2 * q].y, h2[2 * q + 1].x, h2[2 * q + 1].y);
-        p.dtsum[(row_bk + d) * (p.NC - 1) + chunk] = dtsum;
-    }
-    // the state after the last step (steps past L have dt = 0: identity)
-    if (MODE == kModeOutput && p.hlast && cvalid && chunk == p.NC - 1) {
-        float *hl = p.hlast + (row_bk + d) * p.NS + p.n0;
+    for (int c = 0; c < CPL; ++c) {
+        if (!cvalid[c])
+            continue;
+        if (MODE == kModeState) {
+            float4 *hs = reinterpret_cast<float4 *>(
+                p.hstate + ((row_bk + dch[c]) * (p.NC - 1) + chunk) * kNP);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (2 * j < N)
-                hl[2 * j] = h2[j].x;
-            if (2 * j + 1 < N)
-                hl[2 * j + 1] = h2[j].y;
+            for (int q = 0; q < 4; ++q)
+                hs[q] = make_float4(h2[c][2 * q].x, h2[c][2 * q].y, h2[c][2 * q + 1].x,
+                                    h2[c][2 * q + 1].y);
+            p.dtsum[(row_bk + dch[c]) * (p.NC - 1) + chunk] = dtsum[c];
+        }
+        // the state after the last step (steps past L have dt = 0: identity)
+        if (MODE == kModeOutput && p.hlast && chunk == p.NC - 1) {
+            float *hl = p.hlast + (row_bk + dch[c]) * p.NS + p.n0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (2 * j < N)
+                    hl[2 * j] = h2[c][j].x;
+                if (2 * j + 1 < N)
+                    hl[2 * j + 1] = h2[c][j].y;
+            }
         }
     }
 }
@@ -633,8 +704,13 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
 // [(32w + l) * per, (32w + l + 1) * per).
 constexpr int kCarryWarps = 4;
 
+template <int PMAX>
 static __global__ void __launch_bounds__(32 * kCarryWarps) carry_scan_kernel(const ScanParams p, int SW)
 {
+    // PMAX > 0: a lane owns at most PMAX chunks, whose end states and dt sums
+    // it loads once, all at the same time, and keeps in registers for both
+    // runs over them; PMAX = 0: any number, loaded in each run
+    constexpr int PR = PMAX > 0 ? PMAX : 1;
     __shared__ float s_tot[kCarryWarps][2][kNP];   // per warp: (a, e) of its whole range
     grid_dependency_wait();   // the chunk end states of the state pass
     allow_dependents();
@@ -667,12 +743,31 @@ static __global__ void __launch_bounds__(32 * kCarryWarps) carry_scan_kernel(con
     float *hs = p.hstate + rr * (long long)nc1 * kNP;
     const float *ds = p.dtsum + rr * (long long)nc1;
     const float *al = p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0;
+    if (!live)
+        c0 = c1 = 0;
+    // the lane's chunks in registers (PMAX > 0), loads in flight together
+    float hv[PR][kNP], dv[PR];
+    if constexpr (PMAX > 0) {
+#pragma unroll
+        for (int j = 0; j < PMAX; ++j) {
+            const int c = c0 + j;
+            const bool in = c < c1;
+            dv[j] = in ? ds[c] : 0.f;
+            const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)(in ? c : 0) * kNP);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = in ? he[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                hv[j][4 * q] = v.x;
+                hv[j][4 * q + 1] = v.y;
+                hv[j][4 * q + 2] = v.z;
+                hv[j][4 * q + 3] = v.w;
+            }
+        }
+    }
     float A[kNP];
 #pragma unroll
     for (int n = 0; n < kNP; ++n)
         A[n] = (live && n < p.N) ? -expf(__ldg(al + n)) * kLog2e : 0.f;
-    if (!live)
-        c0 = c1 = 0;
 
     // the map of this lane's chunks, composed in order
     float a[kNP], e[kNP];
@@ -681,19 +776,32 @@ static __global__ void __launch_bounds__(32 * kCarryWarps) carry_scan_kernel(con
         a[n] = 1.f;
         e[n] = 0.f;
     }
-    for (int c = c0; c < c1; ++c) {
-        const float dsum = ds[c];
-        const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)c * kNP);
+    auto compose = [&](float dsum, const float (&h)[kNP]) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = he[q];
-            const float hv[4] = {v.x, v.y, v.z, v.w};
+        for (int n = 0; n < kNP; ++n) {
+            const float ai = mufu_ex2(A[n] * dsum);
+            e[n] = fmaf(ai, e[n], h[n]);
+            a[n] *= ai;
+        }
+    };
+    if constexpr (PMAX > 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float ai = mufu_ex2(A[4 * q + i] * dsum);
-                e[4 * q + i] = fmaf(ai, e[4 * q + i], hv[i]);
-                a[4 * q + i] *= ai;
+        for (int j = 0; j < PMAX; ++j)
+            if (c0 + j < c1)
+                compose(dv[j], hv[j]);
+    } else {
+        for (int c = c0; c < c1; ++c) {
+            float h[kNP];
+            const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)c * kNP);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = he[q];
+                h[4 * q] = v.x;
+                h[4 * q + 1] = v.y;
+                h[4 * q + 2] = v.z;
+                h[4 * q + 3] = v.w;
             }
+            compose(ds[c], h);
         }
     }
     // inclusive scan across the lanes of the segment: earlier lanes' maps first
@@ -744,20 +852,33 @@ static __global__ void __launch_bounds__(32 * kCarryWarps) carry_scan_kernel(con
             pe[n] = fmaf(pa[n], we[n], pe[n]);
     }
     // the state entering each chunk of the segment, over its end state
-    for (int c = c0; c < c1; ++c) {
-        const float dsum = ds[c];
+    auto advance = [&](int c, float dsum, const float (&h)[kNP]) {
+#pragma unroll
+        for (int n = 0; n < kNP; ++n)
+            pe[n] = fmaf(mufu_ex2(A[n] * dsum), pe[n], h[n]);
         float4 *slot = reinterpret_cast<float4 *>(hs + (size_t)c * kNP);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = slot[q];
-            const float hv[4] = {v.x, v.y, v.z, v.w};
-            float o[4];
+        for (int q = 0; q < 4; ++q)
+            slot[q] = make_float4(pe[4 * q], pe[4 * q + 1], pe[4 * q + 2], pe[4 * q + 3]);
+    };
+    if constexpr (PMAX > 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                pe[4 * q + i] = fmaf(mufu_ex2(A[4 * q + i] * dsum), pe[4 * q + i], hv[i]);
-                o[i] = pe[4 * q + i];
+        for (int j = 0; j < PMAX; ++j)
+            if (c0 + j < c1)
+                advance(c0 + j, dv[j], hv[j]);
+    } else {
+        for (int c = c0; c < c1; ++c) {
+            float h[kNP];
+            const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)c * kNP);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = he[q];
+                h[4 * q] = v.x;
+                h[4 * q + 1] = v.y;
+                h[4 * q + 2] = v.z;
+                h[4 * q + 3] = v.w;
             }
-            slot[q] = make_float4(o[0], o[1], o[2], o[3]);
+            advance(c, ds[c], h);
         }
     }
 }
@@ -794,7 +915,12 @@ inline cudaError_t launch_carry_scan(const ScanParams &p, cudaStream_t st, bool 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, carry_scan_kernel, p, SW);
+    const int per = nc1 <= 32 ? 1 : (nc1 + 32 * nw - 1) / (32 * nw);   // chunks per lane
+    if (per <= 1)
+        return cudaLaunchKernelEx(&cfg, carry_scan_kernel<1>, p, SW);
+    if (per <= 4)
+        return cudaLaunchKernelEx(&cfg, carry_scan_kernel<4>, p, SW);
+    return cudaLaunchKernelEx(&cfg, carry_scan_kernel<0>, p, SW);
 }
 
 }  // namespace ss2d

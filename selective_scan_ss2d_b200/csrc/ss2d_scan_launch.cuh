@@ -7,7 +7,6 @@
 
 #include "ss2d_kernels.cuh"
 #include "ss2d_launch.h"
-#include "ss2d_quad.cuh"
 #include "ss2d_scan.cuh"
 
 namespace ss2d {
@@ -40,28 +39,19 @@ cudaError_t launch_chunk(const ScanParams &p, int ncg, cudaStream_t st, bool dep
         if (e != cudaSuccess)
             return e;
     }
-    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT), (unsigned)(p.B * ncg));
+    const long long nz = (long long)p.B * ncg;   // (b, chunk) pairs, looped past 65535
+    dim3 grid((unsigned)p.K, (unsigned)((p.D + Sh::NT - 1) / Sh::NT),
+              (unsigned)(nz < 65535 ? nz : 65535));
     return launch_kernel(kern, grid, dim3(Sh::NT), smem, st, dependent, p);
 }
 
-template <typename Tin, int MODE, int NW, int R>
-cudaError_t launch_quad(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
-{
-    constexpr int MINB = 65536 / (32 * NW * R);
-    constexpr int CH = kQCh * NW;
-    dim3 grid((unsigned)p.K, (unsigned)((p.D + CH - 1) / CH), (unsigned)(p.B * ncg));
-    return launch_kernel(quad_scan_kernel<Tin, MODE, NW, MINB>, grid, dim3(32 * NW), 0, st,
-                         dependent, p);
-}
-
-// lane_scan_kernel with a cap of R registers per thread (128: 16 warps per
-// SM; 168: 12)
-template <typename Tin, int WC, int R, int MODE, bool C, int Q, bool A, bool F = false>
+// lane_scan_kernel with a cap of R registers per thread (128: 16 warps per SM)
+template <typename Tin, int WC, int R, int MODE, int CPL, bool C, int Q, bool A, bool F = false>
 cudaError_t launch_lane_k(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
-    using Sh = LaneShape<Tin, WC, C, A, F>;
+    using Sh = LaneShape<Tin, WC, C, A, F, CPL>;
     constexpr int MB = 65536 / (32 * WC * R);
-    auto kern = lane_scan_kernel<Tin, WC, MODE, MB, C, Q, A, F>;
+    auto kern = lane_scan_kernel<Tin, WC, MODE, MB, C, Q, A, F, CPL>;
     const size_t smem = Sh::SMEM_BYTES;
     // the largest shared-memory carveout, so that 16 warps per SM fit
     cudaError_t e =
@@ -71,13 +61,13 @@ cudaError_t launch_lane_k(const ScanParams &p, int ncg, cudaStream_t st, bool de
                                  (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess)
         return e;
-    const long long blocks = (long long)((p.D + Sh::NT - 1) / Sh::NT) * p.K * p.B * ncg;
+    const long long blocks = (long long)((p.D + Sh::CH - 1) / Sh::CH) * p.K * p.B * ncg;
     if (blocks > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
     return launch_kernel(kern, dim3((unsigned)blocks), dim3(Sh::NT), smem, st, dependent, p);
 }
 
-template <typename Tin, int WC, int R, int MODE>
+template <typename Tin, int WC, int R, int MODE, int CPL>
 cudaError_t launch_lane(const ScanParams &p, int ncg, cudaStream_t st, bool dependent)
 {
     // the column-major path only where a direction is column-major; half the
@@ -85,20 +75,20 @@ cudaError_t launch_lane(const ScanParams &p, int ncg, cudaStream_t st, bool depe
     // row copies when every row starts on an 8-byte boundary
     const bool cols = p.two_d && p.K == 4, eight = p.N <= 8, aligned = p.vec >= 8;
     if (p.front)   // the fused front's scratch rows: 1D, aligned
-        return eight ? launch_lane_k<Tin, WC, R, MODE, false, 2, true, true>(p, ncg, st, dependent)
-                     : launch_lane_k<Tin, WC, R, MODE, false, 4, true, true>(p, ncg, st, dependent);
+        return eight ? launch_lane_k<Tin, WC, R, MODE, CPL, false, 2, true, true>(p, ncg, st, dependent)
+                     : launch_lane_k<Tin, WC, R, MODE, CPL, false, 4, true, true>(p, ncg, st, dependent);
     if (cols) {
         if (eight)
-            return aligned ? launch_lane_k<Tin, WC, R, MODE, true, 2, true>(p, ncg, st, dependent)
-                           : launch_lane_k<Tin, WC, R, MODE, true, 2, false>(p, ncg, st, dependent);
-        return aligned ? launch_lane_k<Tin, WC, R, MODE, true, 4, true>(p, ncg, st, dependent)
-                       : launch_lane_k<Tin, WC, R, MODE, true, 4, false>(p, ncg, st, dependent);
+            return aligned ? launch_lane_k<Tin, WC, R, MODE, CPL, true, 2, true>(p, ncg, st, dependent)
+                           : launch_lane_k<Tin, WC, R, MODE, CPL, true, 2, false>(p, ncg, st, dependent);
+        return aligned ? launch_lane_k<Tin, WC, R, MODE, CPL, true, 4, true>(p, ncg, st, dependent)
+                       : launch_lane_k<Tin, WC, R, MODE, CPL, true, 4, false>(p, ncg, st, dependent);
     }
     if (eight)
-        return aligned ? launch_lane_k<Tin, WC, R, MODE, false, 2, true>(p, ncg, st, dependent)
-                       : launch_lane_k<Tin, WC, R, MODE, false, 2, false>(p, ncg, st, dependent);
-    return aligned ? launch_lane_k<Tin, WC, R, MODE, false, 4, true>(p, ncg, st, dependent)
-                   : launch_lane_k<Tin, WC, R, MODE, false, 4, false>(p, ncg, st, dependent);
+        return aligned ? launch_lane_k<Tin, WC, R, MODE, CPL, false, 2, true>(p, ncg, st, dependent)
+                       : launch_lane_k<Tin, WC, R, MODE, CPL, false, 2, false>(p, ncg, st, dependent);
+    return aligned ? launch_lane_k<Tin, WC, R, MODE, CPL, false, 4, true>(p, ncg, st, dependent)
+                   : launch_lane_k<Tin, WC, R, MODE, CPL, false, 4, false>(p, ncg, st, dependent);
 }
 
 template <typename Tin, int LAYOUT, int WC, int R, int MODE>
@@ -106,10 +96,8 @@ cudaError_t launch_pass(const ScanParams &p, int ncg, cudaStream_t st, bool depe
 {
     if constexpr (LAYOUT == 0)
         return launch_chunk<Tin, WC, MODE, R>(p, ncg, st, dependent);
-    else if constexpr (LAYOUT == 1)
-        return launch_quad<Tin, MODE, WC, R>(p, ncg, st, dependent);
     else
-        return launch_lane<Tin, WC, R, MODE>(p, ncg, st, dependent);
+        return launch_lane<Tin, WC, R, MODE, 1>(p, ncg, st, dependent);
 }
 
 template <typename Tin, int LAYOUT, int WC, int R>
@@ -153,9 +141,7 @@ cudaError_t launch_scan_t(const Plan &plan, ScanParams &p, cudaStream_t st, cuda
     SS2D_DISPATCH(0, 4, 128)
     SS2D_DISPATCH(0, 2, 168)
     SS2D_DISPATCH(0, 4, 168)
-    SS2D_DISPATCH(1, 4, 128)
     SS2D_DISPATCH(2, 2, 128)
-    SS2D_DISPATCH(2, 2, 168)
 #undef SS2D_DISPATCH
     return cudaErrorInvalidValue;
 }

@@ -428,3 +428,37 @@ def test_eight_states_full_size_sampled(name):
     for (b, d) in [(0, 0), (cfg.B - 1, cfg.D - 1), (cfg.B // 2, 77)]:
         sub = wl.channel_subproblem(inp, b, d)
         _gpu.assert_close(y[b:b + 1, d:d + 1], _gpu.run_oracle(sub), cfg.dtype, f"N=8 ({b},{d})")
+
+
+# ---------------------------------------------------------------------------
+# shapes past the launch limits of a single grid: more (b, chunk) pairs than
+# a grid dimension holds, and maps too wide for the band-form merge
+# ---------------------------------------------------------------------------
+def test_more_chunk_launches_than_one_grid_dimension():
+    """1D, B = 300, L = 4096 with 16-step chunks: 300 * 256 (b, chunk) pairs,
+    more than 65535, run by looping over grid z."""
+    cfg = small("1d", B=300, D=1, W=4096, K=1, N=4)
+    inp = wl.make_inputs(cfg, seed=13)
+    v = [i for i in range(nvariants()) if binding.ss2d_variant_name(i) == "wc2_lc16"][0]
+    plan = binding.ss2d_plan(False, cfg.B, cfg.D, 1, cfg.L, cfg.N, cfg.K, v)
+    assert cfg.B * plan["num_chunks"] > 65535
+    _gpu.assert_close(_gpu.run_gpu(inp, variant=v), _gpu.run_oracle(inp), wl.F32, cfg.name)
+
+
+def test_wide_map_plain_merge():
+    """An 8 x 1600 map (K = 4): too wide for the band merge's tiles, merged
+    one pixel per thread; every element against the oracle."""
+    cfg = small(B=1, D=4, H=8, W=1600, K=4, N=16)
+    inp = wl.make_inputs(cfg, seed=14)
+    _gpu.assert_close(_gpu.run_gpu(inp), _gpu.run_oracle(inp), wl.F32, cfg.name)
+
+
+def test_map_1024x1024_sampled_channels():
+    """A 1024 x 1024 map, D = 8, bf16 (L = 2^20): sampled channels against the
+    oracle."""
+    cfg = small(B=1, D=8, H=1024, W=1024, K=4, N=16, dtype=wl.BF16)
+    inp = wl.make_inputs(cfg, seed=15)
+    y = _gpu.run_gpu(inp)
+    for d in (0, 5):
+        sub = wl.channel_subproblem(inp, 0, d)
+        _gpu.assert_close(y[0:1, d:d + 1], _gpu.run_oracle(sub), wl.BF16, f"1024^2 d={d}")
