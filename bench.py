@@ -589,7 +589,8 @@ def run_front(args, rank, world, local_rank):
         "roofline_front_tensor": {"bound": "tensor", "achieved": tflops,
                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": tflops / peaks["bf16_tflops"],
-                                  "kernel": "front_kernel (x_proj on tcgen05, bf16 operands)",
+                                  "kernel": "front_wprep_kernel + front_conv_kernel + "
+                                            "front_proj_kernel (x_proj on tcgen05, bf16 operands)",
                                   "kernel_ms": front_ms, "flops_per_launch": flops,
                                   "peak_source": peaks["bf16_source"]},
         "roofline_front_hbm": {"bound": "hbm", "achieved": front_gbs, "peak": peaks["hbm_gbs"],
@@ -608,9 +609,23 @@ def run_front(args, rank, world, local_rank):
                                   "frac": step_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
                          "algorithmic_bytes_per_step": step_bytes},
         "launch_ms": {"front": front_ms, "scan_passes": scan_ms, "cross_merge": merge_ms},
+        # three front kernels, then the front-mode scan's own launches (its
+        # passes and the merge) under the lane kernel's plan
+        "gpu_launches": args.steps * (3 + front_scan_launches(cfg)),
         "clocks": clocks,
     }
     return line
+
+
+def front_scan_launches(cfg) -> int:
+    """Kernel launches of the scan + merge half of one selective_scan_fwd_front
+    call: the plan of the lane kernel's wave-chunked variant, which that call
+    always uses."""
+    from selective_scan_ss2d_b200 import binding
+    names = [binding.ss2d_variant_name(i) for i in range(binding.ss2d_num_variants())]
+    plan = binding.ss2d_plan(False, cfg.B, cfg.D, 1, cfg.L, cfg.N, cfg.K,
+                             variant=names.index("lane2_wave"))
+    return plan["launches"]
 
 
 def run_backward(args, rank, world, local_rank):

@@ -54,11 +54,46 @@ int front_validate(const FrontCall &c)
     return SS2D_OK;
 }
 
-// the front kernel for one call; scratch rows of pitch LP
-cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, float *Bs,
-                         float *Cs, cudaStream_t st)
+int front_nm(int N) { return ((1 + 2 * N) + 15) / 16 * 16; }
+
+// bytes of the bf16 B operands of every direction and channel block, and of
+// the A operands of every (b, k, tile, channel block)
+size_t front_wb_bytes(int K, int D, int N)
 {
+    const int nblk = (D + ss2d::kFrontCh - 1) / ss2d::kFrontCh;
+    return (size_t)K * nblk * ss2d::front_bbytes(front_nm(N));
+}
+size_t front_ab_bytes(int B, int K, int D, int L)
+{
+    const long long nblk = (D + ss2d::kFrontCh - 1) / ss2d::kFrontCh;
+    const long long ntiles = (L + ss2d::kFrontTile - 1) / ss2d::kFrontTile;
+    return (size_t)B * K * ntiles * nblk * ss2d::kFrontABytes;
+}
+size_t up256_(size_t v) { return (v + 255) & ~(size_t)255; }
+// scratch of the front kernels: Wb then Ab
+size_t front_op_bytes(const FrontCall &c)
+{
+    return up256_(front_wb_bytes(c.K, c.D, c.N)) + up256_(front_ab_bytes(c.B, c.K, c.D, c.L));
+}
+
+// the front kernels for one call (W_x conversion, conv, x_proj); scratch
+// rows of pitch LP, ops of front_op_bytes
+cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, float *Bs,
+                         float *Cs, void *ops, cudaStream_t st)
+{
+    void *Wb = ops;
+    void *Ab = static_cast<char *>(ops) + up256_(front_wb_bytes(c.K, c.D, c.N));
+    {
+        const int nblk = (c.D + ss2d::kFrontCh - 1) / ss2d::kFrontCh;
+        ss2d::front_wprep_kernel<<<(unsigned)(c.K * nblk), 256, 0, st>>>(
+            c.W_x, static_cast<__nv_bfloat16 *>(Wb), c.D, 1 + 2 * c.N, front_nm(c.N), nblk);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
     ss2d::FrontParams fp{};
+    fp.Wb = Wb;
+    fp.Ab = Ab;
     fp.x = c.x;
     fp.conv_w = c.conv_w;
     fp.conv_b = c.conv_b;
@@ -78,29 +113,37 @@ cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, flo
     fp.LP = LP;
     fp.N = c.N;
     fp.K = c.K;
-    fp.NM = ((1 + 2 * c.N) + 15) / 16 * 16;
+    fp.NM = front_nm(c.N);
     int tc = 32;
     while (tc < fp.NM)
         tc <<= 1;
     fp.tcols = tc;
-    const int smem = ss2d::front_smem_bytes(fp.NM);
-    const dim3 grid((unsigned)((c.L + ss2d::kFrontTile - 1) / ss2d::kFrontTile), (unsigned)c.K,
-                    (unsigned)c.B);
-    auto launch = [&](auto kern) {
-        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (r != cudaSuccess)
-            return r;
-        return ss2d::launch_kernel(kern, grid, dim3(ss2d::kFrontThreads), (size_t)smem, st, false,
-                                   fp);
-    };
-    switch (c.dtype) {
-    case SS2D_BF16:
-        return launch(ss2d::front_kernel<__nv_bfloat16>);
-    case SS2D_F16:
-        return launch(ss2d::front_kernel<__half>);
-    default:
-        return launch(ss2d::front_kernel<float>);
+    const unsigned ntiles = (unsigned)((c.L + ss2d::kFrontTile - 1) / ss2d::kFrontTile);
+    const unsigned nblk = (unsigned)((c.D + ss2d::kFrontCh - 1) / ss2d::kFrontCh);
+    {
+        const dim3 grid(ntiles, nblk, (unsigned)(c.B * c.K));
+        switch (c.dtype) {
+        case SS2D_BF16:
+            ss2d::front_conv_kernel<__nv_bfloat16><<<grid, ss2d::kFrontConvThreads, 0, st>>>(fp);
+            break;
+        case SS2D_F16:
+            ss2d::front_conv_kernel<__half><<<grid, ss2d::kFrontConvThreads, 0, st>>>(fp);
+            break;
+        default:
+            ss2d::front_conv_kernel<float><<<grid, ss2d::kFrontConvThreads, 0, st>>>(fp);
+            break;
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
     }
+    const int smem = ss2d::front_smem_bytes(fp.NM);
+    cudaError_t r = cudaFuncSetAttribute(ss2d::front_proj_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (r != cudaSuccess)
+        return r;
+    return ss2d::launch_kernel(ss2d::front_proj_kernel, dim3(ntiles, (unsigned)c.K, (unsigned)c.B),
+                               dim3(ss2d::kFrontProjThreads), (size_t)smem, st, false, fp);
 }
 
 int check_front_pointers(const FrontCall &c, const void *const *extra, int nextra, int dev)
@@ -152,7 +195,8 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
 
     const int LP = (L + 7) / 8 * 8;
     const size_t esz = dtype == SS2D_F32 ? 4 : 2;
-    const int variant = 19;   // lane2_wave: the lane kernel reads the front's scratch rows
+    // the lane kernel reads the front's scratch rows
+    const int variant = ss2d::variant_index("lane2_wave");
     const ss2d::Plan pl = ss2d::make_plan(variant, B, D, L, K);
     const size_t rows = (size_t)B * K * D;
     const size_t u_bytes = up256(esz * rows * LP);
@@ -161,7 +205,9 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
     const size_t part_bytes = K > 1 ? up256(sizeof(float) * rows * L) : 0;
     const size_t hs_bytes = pl.NC > 1 ? up256(sizeof(float) * rows * (pl.NC - 1) * ss2d::kNP) : 0;
     const size_t ds_bytes = pl.NC > 1 ? up256(sizeof(float) * rows * (pl.NC - 1)) : 0;
-    const size_t total = u_bytes + dt_bytes + 2 * bc_bytes + part_bytes + hs_bytes + ds_bytes;
+    const size_t wb_bytes = up256(front_op_bytes(c));
+    const size_t total = u_bytes + dt_bytes + 2 * bc_bytes + part_bytes + hs_bytes + ds_bytes +
+                         wb_bytes;
     void *scratch = nullptr;
     rc = ss2d::scratch_alloc(&scratch, total, st);
     if (rc != SS2D_OK)
@@ -175,7 +221,8 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
 
     if (ev)
         cudaEventRecord(ev[0], st);
-    e = launch_front(c, LP, u, dt_raw, Bs, Cs, st);
+    void *Wb = rest + part_bytes + hs_bytes + ds_bytes;
+    e = launch_front(c, LP, u, dt_raw, Bs, Cs, Wb, st);
     if (ev)
         cudaEventRecord(ev[1], st);
     if (e == cudaSuccess) {
@@ -301,9 +348,19 @@ int ss2d_front_project(const void *x, const float *conv_w, const float *conv_b, 
     rc = check_front_pointers(c, extra, 4, dev);
     if (rc != SS2D_OK)
         return rc;
-    e = launch_front(c, L, u, dt_raw, Bs, Cs, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *Wb = nullptr;
+    rc = ss2d::scratch_alloc(&Wb, front_op_bytes(c), st);
+    if (rc != SS2D_OK)
+        return rc;
+    e = launch_front(c, L, u, dt_raw, Bs, Cs, Wb, st);
+    const cudaError_t ef = cudaFreeAsync(Wb, st);
     if (e != cudaSuccess) {
         ss2d::record_error("kernel launch", e);
+        return SS2D_ERR_CUDA;
+    }
+    if (ef != cudaSuccess) {
+        ss2d::record_error("cudaFreeAsync", ef);
         return SS2D_ERR_CUDA;
     }
     return SS2D_OK;

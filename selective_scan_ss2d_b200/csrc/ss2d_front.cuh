@@ -14,25 +14,33 @@
 // w_dt[k, d] * dt_raw[l], its bias the scan's delta bias, so no (D, L) delta
 // array is ever written.
 //
-// front_kernel: one CTA of 128 threads per (128-step tile, k, b).  Channels
-// are taken 64 at a time: the CTA convolves its tile (3-step halo, taps in
-// registers), applies SiLU, stores u for the scan (in the input dtype) and
-// writes u, rounded to bf16, as the A operand of x_proj into shared memory;
-// the matching 64 columns of W_x go in as the B operand.  One thread issues
-// the tcgen05.mma instructions (M = 128 steps, N = 1 + 2N rounded up to 16,
-// K = 16 per instruction) that accumulate x_dbl in tensor memory, and a
-// tcgen05.commit tells an mbarrier when the buffers may be refilled (two
-// buffers: the conv of the next 64 channels overlaps the MMAs of these).
+// Two kernels:
+//   front_conv_kernel: one CTA of 256 threads per (128-step tile, 64-channel
+//     block, b * K + k); the tile's input steps (3-step halo) are staged in
+//     shared memory with cp.async, then a thread holds a channel pair over 16
+//     steps, convolves, applies SiLU and writes u twice: for the scan, in the
+//     input dtype, (B, K, D, LP) rows; and, rounded to bf16, as the tile's
+//     x_proj A operand, already in the tensor-core operand layout (one 16 KB
+//     block per tile and channel block).
+//   front_proj_kernel: one CTA of 128 threads per (128-step tile, k, b).  One
+//     thread streams the tile's A blocks and the matching bf16 blocks of W_x
+//     (the B operand, converted once per call by front_wprep_kernel) into a
+//     ring of shared-memory stages with cp.async.bulk, each stage completing
+//     an mbarrier (expected bytes), and issues the tcgen05.mma instructions
+//     (M = 128 steps, N = 1 + 2N rounded up to 16, K = 16 per instruction)
+//     that accumulate x_dbl in tensor memory; a tcgen05.commit frees each
+//     stage for the next copy.  The epilogue reads the accumulator back with
+//     tcgen05.ld (warp w: steps 32w..32w+31, one step per lane) and stores
+//     dt_raw, B and C.
 // Every mbarrier wait gives up after a time limit, records the fault in a
 // device word that ss2d_check_waits() reports, and lets the kernel finish.
-// The epilogue reads the accumulator back with tcgen05.ld (warp w: steps
-// 32w..32w+31, one step per lane) and stores dt_raw, B and C.
 //
 // Operand layout (K-major, no swizzle): core matrices of 8 rows x 16 bytes;
 // element (row r, channel c) of a 64-channel block at byte
-//     (r / 8) * kSBO + (c / 8) * kLBO + (r % 8) * 16 + (c % 8) * 2,
-// kLBO = 144 (the 8 core matrices of a row group 144 bytes apart, which
-// spreads a warp's stores of one row over 16 banks) and kSBO = 8 * kLBO.
+//     (r / 8) * 1024 + (c / 8) * 128 + (r % 8) * 16 + (c % 8) * 2
+// (LBO = 128 between the core matrices of a row group, SBO = 1024 between
+// row groups): the layout both operand blocks have in global memory, so a
+// block is one contiguous copy.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -48,6 +56,8 @@ struct FrontParams {
     const float *conv_w;    // (K, D, 4)
     const float *conv_b;    // (K, D)
     const float *W_x;       // (K, 1 + 2N, D)
+    const void *Wb;         // W_x in bf16, per direction and 64-channel block, in the B layout
+    void *Ab;               // u in bf16, per (b, k, tile, 64-channel block), in the A layout
     void *u;                // (B, K, D, LP) u of every direction in its scan order, dtype
     float *dt_raw;          // (B, K, LP)
     float *Bs, *Cs;         // (B, K, N, LP)
@@ -57,19 +67,21 @@ struct FrontParams {
     int tcols;              // tensor-memory columns held (power of 2, >= 32, >= NM)
 };
 
-constexpr int kFrontThreads = 128;
-constexpr int kFrontTile = 128;       // steps per CTA (MMA M)
+constexpr int kFrontConvThreads = 256;
+constexpr int kFrontProjThreads = 128;
+constexpr int kFrontTile = 128;       // steps per tile (MMA M)
 constexpr int kFrontCh = 64;          // channels per block (4 MMAs of K = 16)
-constexpr int kFrontLBO = 144;
-constexpr int kFrontSBO = 8 * kFrontLBO;
-constexpr int kFrontABytes = (kFrontTile / 8) * kFrontSBO;   // one A buffer
+constexpr int kFrontLBO = 128;
+constexpr int kFrontSBO = 1024;
+constexpr int kFrontABytes = (kFrontTile / 8) * kFrontSBO;   // one A block (16 KB)
+constexpr int kFrontStages = 2;                              // shared-memory ring
 
 __host__ __device__ constexpr int front_bbytes(int NM) { return (NM / 8) * kFrontSBO; }
-// dynamic shared memory: two A buffers, two B buffers, three mbarriers, the
-// tensor-memory address
+// dynamic shared memory of front_proj_kernel: the ring of (A, B) stages,
+// 2 * stages + 1 mbarriers, the tensor-memory address
 __host__ __device__ constexpr int front_smem_bytes(int NM)
 {
-    return 2 * kFrontABytes + 2 * front_bbytes(NM) + 64;
+    return kFrontStages * (kFrontABytes + front_bbytes(NM)) + 8 * (2 * kFrontStages + 1) + 16;
 }
 
 // codes written to the fault word
@@ -123,12 +135,12 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // shared-memory matrix descriptor: K-major, no swizzle, version 1 (sm_100)
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr)
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3fffu);
-    d |= (uint64_t)((kFrontLBO >> 4) & 0x3fffu) << 16;
-    d |= (uint64_t)((kFrontSBO >> 4) & 0x3fffu) << 32;
+    d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3fffu) << 32;
     d |= (uint64_t)1 << 46;
     return d;   // base offset 0, layout type 0 (no swizzle)
 }
@@ -174,6 +186,28 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
         v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void cp_async_16b(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+
+// W_x (K, R, D) float32 -> Wb: for direction k and 64-channel block cb, the
+// NM x 64 bf16 B operand (rows >= R and channels >= D zero) in the layout
+// (r / 8) * 1024 + (c / 8) * 128 + (r % 8) * 16 + (c % 8) * 2.
+// grid: K * nblk CTAs.
+static __global__ void front_wprep_kernel(const float *W_x, __nv_bfloat16 *Wb, int D, int R,
+                                          int NM, int nblk)
+{
+    const int k = blockIdx.x / nblk, cb = blockIdx.x % nblk;
+    __nv_bfloat16 *dst = Wb + (size_t)blockIdx.x * NM * kFrontCh;
+    for (int i = threadIdx.x; i < NM * kFrontCh; i += blockDim.x) {
+        const int r = i / kFrontCh, cc = i % kFrontCh, dd = cb * kFrontCh + cc;
+        const float v = (r < R && dd < D) ? W_x[((size_t)k * R + r) * D + dd] : 0.f;
+        dst[((r >> 3) * kFrontSBO + (cc >> 3) * kFrontLBO + (r & 7) * 16 + (cc & 7) * 2) / 2] =
+            __float2bfloat16_rn(v);
+    }
+}
+
 template <typename Tin>
 __device__ __forceinline__ float front_load(const Tin *p)
 {
@@ -191,28 +225,199 @@ __device__ __forceinline__ uint32_t store_bits(float v, __half *)
     return (uint32_t)__half_as_ushort(__float2half_rn(v));
 }
 
+// cp.async of 16 bytes that reads `bytes` (0 or 16) and zero-fills the rest
+__device__ __forceinline__ void cp_async_16b_zfill(uint32_t dst, const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
+
+constexpr int kFrontRows = kFrontTile + 3;   // input steps of a tile with the 3-step halo
+
+// conv + SiLU of one (128-step tile, 64-channel block, b * K + k): u for the
+// scan and the bf16 A operand block.  grid (tiles, channel blocks, B * K).
+// The CTA first copies the tile's 131 input steps (3-step halo) of its 64
+// channels into shared memory (cp.async, 16-byte pieces, zeros outside the
+// sequence and past channel D - 1), so that all its loads are in flight at
+// once.  Thread t then owns the channel pair 2 * (t % 32), + 1 over steps
+// 16 * (t / 32) .. + 15 of the tile: it writes per step one 4-byte word of
+// the A operand (two channels in bf16) and per channel the 16 steps of u.
+// Warps whose steps all lie past the end of the sequence do nothing (the A
+// rows of those steps only feed accumulator rows that are never stored).
 template <typename Tin>
-__global__ void __launch_bounds__(kFrontThreads) front_kernel(const FrontParams p)
+__global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const FrontParams p)
+{
+    constexpr int CP = 2, SG = 16;   // channels and steps per thread
+    static_assert(kFrontCh / CP * (kFrontTile / SG) == kFrontConvThreads, "thread layout");
+    constexpr int ROWB = kFrontCh * (int)sizeof(Tin);   // bytes of a staged row
+    __shared__ __align__(16) unsigned char sx[kFrontRows * ROWB];
+    const int tid = threadIdx.x;
+    const int tile = blockIdx.x, cb = blockIdx.y, bk = blockIdx.z;
+    const int b = bk / p.K, k = bk % p.K;
+    const int D = p.D, L = p.L, LP = p.LP;
+    const int lt = tile * kFrontTile;            // first step of the tile
+    const int dblk = cb * kFrontCh;              // first channel of the block
+    const Tin *xb = static_cast<const Tin *>(p.x) + (size_t)b * L * D;
+
+    // ---- stage: row r holds step lt - 3 + r, which reads input position
+    // l (k = 0) or L-1-l (k = 1)
+    constexpr int EPV = 16 / (int)sizeof(Tin);   // elements per 16-byte piece
+    const bool vec = D % EPV == 0 && (reinterpret_cast<uintptr_t>(p.x) & 15) == 0;
+    if (vec) {
+        constexpr int PPR = kFrontCh / EPV;      // pieces per row
+        const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(sx));
+        for (int i = tid; i < kFrontRows * PPR; i += kFrontConvThreads) {
+            const int r = i / PPR, pc = i % PPR;
+            const int l = lt - 3 + r, d = dblk + pc * EPV;
+            const bool in = l >= 0 && l < L && d < D;
+            const int pos = in ? (k == 0 ? l : L - 1 - l) : 0;
+            cp_async_16b_zfill(s0 + r * ROWB + pc * 16, xb + (size_t)pos * D + (in ? d : 0),
+                               in ? 16u : 0u);
+        }
+        asm volatile("cp.async.wait_all;\n" ::: "memory");
+    } else {
+        Tin *st = reinterpret_cast<Tin *>(sx);
+        for (int i = tid; i < kFrontRows * kFrontCh; i += kFrontConvThreads) {
+            const int r = i / kFrontCh, c = i % kFrontCh;
+            const int l = lt - 3 + r, d = dblk + c;
+            const bool in = l >= 0 && l < L && d < D;
+            st[i] = in ? xb[(size_t)(k == 0 ? l : L - 1 - l) * D + d] : Tin(0.f);
+        }
+    }
+    __syncthreads();
+
+    const int pr = tid % (kFrontCh / CP), sg = tid / (kFrontCh / CP);
+    const int c0 = pr * CP;                      // first channel of the pair in the block
+    const int m0 = sg * SG;                      // first step of the thread in the tile
+    const int l0 = lt + m0;
+    if (l0 >= L)
+        return;                                  // the whole warp: no step of it is stored
+    const int d0 = dblk + c0;
+    float w[CP][4], bias[CP];
+#pragma unroll
+    for (int j = 0; j < CP; ++j) {
+        const int d = d0 + j;
+        if (d < D) {
+            const float4 wv = *reinterpret_cast<const float4 *>(p.conv_w + ((size_t)k * D + d) * 4);
+            w[j][0] = wv.x;
+            w[j][1] = wv.y;
+            w[j][2] = wv.z;
+            w[j][3] = wv.w;
+            bias[j] = p.conv_b[(size_t)k * D + d];
+        } else {
+            w[j][0] = w[j][1] = w[j][2] = w[j][3] = bias[j] = 0.f;
+        }
+    }
+    // the pair's value at staged row r
+    auto xrow = [&](int r, float (&v)[CP]) {
+        if constexpr (sizeof(Tin) == 2) {
+            const uint32_t wd = *reinterpret_cast<const uint32_t *>(sx + r * ROWB + c0 * 2);
+            v[0] = half_bits_to_f32<Tin>(wd & 0xffffu);
+            v[1] = half_bits_to_f32<Tin>(wd >> 16);
+        } else {
+            const float2 f = *reinterpret_cast<const float2 *>(sx + r * ROWB + c0 * 4);
+            v[0] = f.x;
+            v[1] = f.y;
+        }
+    };
+    float win[4][CP];   // steps m - 3 .. m of the pair
+    xrow(m0, win[0]);
+    xrow(m0 + 1, win[1]);
+    xrow(m0 + 2, win[2]);
+    unsigned char *ab = static_cast<unsigned char *>(p.Ab) +
+                        (((size_t)bk * gridDim.x + tile) * gridDim.y + cb) * kFrontABytes +
+                        (c0 >> 3) * kFrontLBO + (c0 & 7) * 2;
+    float uu[CP][SG];
+#pragma unroll
+    for (int i = 0; i < SG; ++i) {
+        xrow(m0 + i + 3, win[(i + 3) & 3]);
+#pragma unroll
+        for (int j = 0; j < CP; ++j) {
+            const float cv = fmaf(w[j][3], win[(i + 3) & 3][j],
+                                  fmaf(w[j][2], win[(i + 2) & 3][j],
+                                       fmaf(w[j][1], win[(i + 1) & 3][j], fmaf(w[j][0], win[i & 3][j], bias[j]))));
+            uu[j][i] = silu_f(cv);   // channels past D: zero inputs and taps give SiLU(0) = 0
+        }
+        const int mt = m0 + i;
+        const uint32_t wv = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(uu[0][i])) |
+                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(uu[1][i])) << 16);
+        *reinterpret_cast<uint32_t *>(ab + (mt >> 3) * kFrontSBO + (mt & 7) * 16) = wv;
+    }
+    // u for the scan, in the input dtype: 16-byte stores of 8 (2-byte) or 4
+    // (float) steps; every store starts before L (LP is a multiple of 8)
+    Tin *ub = static_cast<Tin *>(p.u) + (size_t)bk * D * LP;
+    constexpr int PER = sizeof(Tin) == 2 ? 8 : 4;
+#pragma unroll
+    for (int j = 0; j < CP; ++j) {
+        const int d = d0 + j;
+        if (d >= D)
+            continue;
+#pragma unroll
+        for (int q = 0; q < SG / PER; ++q) {
+            const int lv = l0 + q * PER;
+            if (lv >= L)
+                continue;
+            uint4 v;
+            if constexpr (sizeof(Tin) == 2) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    w4[e] = store_bits(uu[j][q * PER + 2 * e], static_cast<Tin *>(nullptr)) |
+                            (store_bits(uu[j][q * PER + 2 * e + 1], static_cast<Tin *>(nullptr)) << 16);
+                v = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            } else {
+                v = make_uint4(__float_as_uint(uu[j][q * PER]), __float_as_uint(uu[j][q * PER + 1]),
+                               __float_as_uint(uu[j][q * PER + 2]), __float_as_uint(uu[j][q * PER + 3]));
+            }
+            *reinterpret_cast<uint4 *>(ub + (size_t)d * LP + lv) = v;
+        }
+    }
+}
+
+// bulk copy global -> shared completing `bytes` on the mbarrier (TMA, no
+// tensor map, no multicast); src, dst 16-byte aligned, bytes a multiple of 16
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// x_proj of one (128-step tile, k, b) on the tensor cores; see the header.
+// grid (tiles, K, B).
+__global__ void __launch_bounds__(kFrontProjThreads) front_proj_kernel(const FrontParams p)
 {
     extern __shared__ __align__(1024) unsigned char fsm[];
     const int NM = p.NM;
-    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(fsm));
-    const uint32_t sA = sbase, sB = sbase + 2 * kFrontABytes;
     const uint32_t bbytes = (uint32_t)front_bbytes(NM);
-    unsigned char *bars_g = fsm + 2 * kFrontABytes + 2 * bbytes;
-    const uint32_t bar0 = sB + 2 * bbytes;              // buffer 0 free, buffer 1 free, done
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars_g + 32);
-
+    const uint32_t stage_bytes = kFrontABytes + bbytes;
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(fsm));
+    // stage s: A at sbase + s * stage_bytes, B right after it
+    const uint32_t bars = sbase + kFrontStages * stage_bytes;   // full[s], empty[s], done
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(fsm + kFrontStages * stage_bytes +
+                                                   8 * (2 * kFrontStages + 1));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int l0 = blockIdx.x * kFrontTile;
-    const int k = blockIdx.y, b = blockIdx.z;
-    const int D = p.D, L = p.L, LP = p.LP, N = p.N, K = p.K;
+    const int tile = blockIdx.x, k = blockIdx.y, b = blockIdx.z;
+    const int N = p.N, K = p.K, L = p.L, LP = p.LP;
     const int R = 1 + 2 * N;
+    const int l0 = tile * kFrontTile;
+    const int nblk = (p.D + kFrontCh - 1) / kFrontCh, ntiles = gridDim.x;
+    const size_t bk = (size_t)b * K + k;
+    const unsigned char *ag = static_cast<const unsigned char *>(p.Ab) +
+                              ((bk * ntiles + tile) * nblk) * kFrontABytes;
+    const unsigned char *wg = static_cast<const unsigned char *>(p.Wb) + (size_t)k * nblk * bbytes;
+    constexpr uint64_t kLimitNs = 2000000000ull;   // 2 s
 
     if (tid == 0) {
-        mbar_init(bar0, 1);
-        mbar_init(bar0 + 8, 1);
-        mbar_init(bar0 + 16, 1);
+        for (int i = 0; i < 2 * kFrontStages + 1; ++i)
+            mbar_init(bars + 8 * i, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -226,110 +431,47 @@ __global__ void __launch_bounds__(kFrontThreads) front_kernel(const FrontParams 
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    const Tin *xb = static_cast<const Tin *>(p.x) + (size_t)b * L * D;
-    Tin *ub = static_cast<Tin *>(p.u) + ((size_t)b * K + k) * (size_t)D * LP;
-    const uint32_t idesc = umma_idesc_bf16(NM);
-    const int c = tid & 63, half = tid >> 6;          // this thread's channel and 64-step half
-    const int nblk = (D + kFrontCh - 1) / kFrontCh;
-    constexpr uint64_t kLimitNs = 2000000000ull;       // 2 s
     bool ok = true;
-
-    for (int cb = 0; cb < nblk; ++cb) {
-        const int buf = cb & 1;
-        // the MMAs of block cb - 2 read this buffer
-        if (cb >= 2)
-            ok = ok && mbar_wait_bounded(bar0 + 8 * buf, ((cb >> 1) - 1) & 1, kLimitNs, p.fault,
-                                         kFaultFrontMma);
-        const uint32_t aBuf = sA + buf * kFrontABytes, bBuf = sB + buf * bbytes;
-        unsigned char *aPtr = fsm + buf * kFrontABytes;
-        unsigned char *bPtr = fsm + 2 * kFrontABytes + buf * bbytes;
-
-        // ---- conv + SiLU of channel d over steps half*64 .. half*64 + 63 ----
-        const int d = cb * kFrontCh + c;
-        const bool dv = d < D;
-        float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, bias = 0.f;
-        if (dv) {
-            const float4 wv = *reinterpret_cast<const float4 *>(p.conv_w + ((size_t)k * D + d) * 4);
-            w0 = wv.x;
-            w1 = wv.y;
-            w2 = wv.z;
-            w3 = wv.w;
-            bias = p.conv_b[(size_t)k * D + d];
-        }
-        // the direction's step l reads input position l (k = 0) or L-1-l (k = 1)
-        auto xat = [&](int l) -> float {
-            if (!dv || l < 0 || l >= L)
-                return 0.f;
-            const int pos = k == 0 ? l : L - 1 - l;
-            return front_load(xb + (size_t)pos * D + d);
+    if (tid == 0) {
+        const uint32_t idesc = umma_idesc_bf16(NM);
+        auto load = [&](int cb) {   // block cb into stage cb % S
+            const int st = cb % kFrontStages;
+            const uint32_t full = bars + 8 * st, dA = sbase + st * stage_bytes;
+            mbar_expect_tx(full, stage_bytes);
+            bulk_copy(dA, ag + (size_t)cb * kFrontABytes, kFrontABytes, full);
+            bulk_copy(dA + kFrontABytes, wg + (size_t)cb * bbytes, bbytes, full);
         };
-        const int m0 = half * 64;
-        float s0 = xat(l0 + m0 - 3), s1 = xat(l0 + m0 - 2), s2 = xat(l0 + m0 - 1);
-        constexpr int PER = sizeof(Tin) == 2 ? 8 : 4;   // steps per 16-byte store of u
-        for (int mb = 0; mb < 64; mb += PER) {
-            float xs[PER];
-#pragma unroll
-            for (int j = 0; j < PER; ++j)   // the group's inputs, loads in flight together
-                xs[j] = xat(l0 + m0 + mb + j);
-            uint32_t pack[PER];
-#pragma unroll
-            for (int j = 0; j < PER; ++j) {
-                const int mt = m0 + mb + j;
-                const float s3 = xs[j];
-                const float cv = fmaf(w3, s3, fmaf(w2, s2, fmaf(w1, s1, fmaf(w0, s0, bias))));
-                const float uu = dv ? silu_f(cv) : 0.f;
-                s0 = s1;
-                s1 = s2;
-                s2 = s3;
-                // A operand (bf16, nearest even)
-                *reinterpret_cast<__nv_bfloat16 *>(aPtr + (mt >> 3) * kFrontSBO +
-                                                   (c >> 3) * kFrontLBO + (mt & 7) * 16 +
-                                                   (c & 7) * 2) = __float2bfloat16_rn(uu);
-                pack[j] = store_bits(uu, static_cast<Tin *>(nullptr));
-            }
-            // u for the scan, in the input dtype: one 16-byte store of PER steps
-            const int lv = l0 + m0 + mb;
-            if (dv && lv < L) {
-                uint4 v;
-                if constexpr (sizeof(Tin) == 2)
-                    v = make_uint4(pack[0] | (pack[1] << 16), pack[2] | (pack[3] << 16),
-                                   pack[4] | (pack[5] << 16), pack[6] | (pack[7] << 16));
-                else
-                    v = make_uint4(pack[0], pack[1], pack[2], pack[3]);
-                *reinterpret_cast<uint4 *>(ub + (size_t)d * LP + lv) = v;
-            }
-        }
-        // ---- B operand: rows 0..NM-1 of W_x (zero beyond 1 + 2N and D) ----
-        for (int i = tid; i < NM * kFrontCh; i += kFrontThreads) {
-            const int r = i / kFrontCh, cc = i % kFrontCh, dd = cb * kFrontCh + cc;
-            const float wv = (r < R && dd < D) ? p.W_x[((size_t)k * R + r) * D + dd] : 0.f;
-            *reinterpret_cast<__nv_bfloat16 *>(bPtr + (r >> 3) * kFrontSBO + (cc >> 3) * kFrontLBO +
-                                               (r & 7) * 16 + (cc & 7) * 2) = __float2bfloat16_rn(wv);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+        for (int cb = 0; cb < kFrontStages && cb < nblk; ++cb)
+            load(cb);
+        for (int cb = 0; cb < nblk; ++cb) {
+            const int st = cb % kFrontStages, use = cb / kFrontStages;
+            const uint32_t full = bars + 8 * st, empty = bars + 8 * (kFrontStages + st);
+            ok = ok && mbar_wait_bounded(full, use & 1, kLimitNs, p.fault, kFaultFrontMma);
             tc_fence_after();
             if (ok) {
+                const uint32_t aS = sbase + st * stage_bytes, bS = aS + kFrontABytes;
 #pragma unroll
                 for (int kk = 0; kk < kFrontCh / 16; ++kk)
-                    umma_bf16(tmem, umma_desc(aBuf + kk * 2 * kFrontLBO),
-                              umma_desc(bBuf + kk * 2 * kFrontLBO), idesc,
+                    umma_bf16(tmem, umma_desc(aS + kk * 2 * kFrontLBO, kFrontLBO, kFrontSBO),
+                              umma_desc(bS + kk * 2 * kFrontLBO, kFrontLBO, kFrontSBO), idesc,
                               (cb > 0 || kk > 0) ? 1u : 0u);
             }
-            umma_commit(bar0 + 8 * buf);
+            umma_commit(empty);
+            if (cb + kFrontStages < nblk) {
+                // the stage is refilled once its MMAs have read it
+                ok = ok && mbar_wait_bounded(empty, use & 1, kLimitNs, p.fault, kFaultFrontMma);
+                if (ok)
+                    load(cb + kFrontStages);
+            }
         }
+        umma_commit(bars + 8 * (2 * kFrontStages));   // every MMA of the tile done
     }
-    // every MMA of the tile done
-    if (tid == 0)
-        umma_commit(bar0 + 16);
-    ok = mbar_wait_bounded(bar0 + 16, 0, kLimitNs, p.fault, kFaultFrontMma) && ok;
+    ok = mbar_wait_bounded(bars + 8 * (2 * kFrontStages), 0, kLimitNs, p.fault, kFaultFrontMma) &&
+         ok;
     tc_fence_after();
 
-    // ---- epilogue: x_dbl rows from tensor memory ----
+    // ---- epilogue: x_dbl rows from tensor memory (warp w: lanes 32w..) ----
     const int l = l0 + warp * 32 + lane;
-    const size_t row_bk = (size_t)b * K + k;
     for (int c0 = 0; c0 < NM; c0 += 16) {
         float v[16];
         tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
@@ -338,11 +480,11 @@ __global__ void __launch_bounds__(kFrontThreads) front_kernel(const FrontParams 
             for (int i = 0; i < 16; ++i) {
                 const int col = c0 + i;
                 if (col == 0)
-                    p.dt_raw[row_bk * LP + l] = v[i];
+                    p.dt_raw[bk * LP + l] = v[i];
                 else if (col <= N)
-                    p.Bs[(row_bk * N + (col - 1)) * LP + l] = v[i];
+                    p.Bs[(bk * N + (col - 1)) * LP + l] = v[i];
                 else if (col < R)
-                    p.Cs[(row_bk * N + (col - 1 - N)) * LP + l] = v[i];
+                    p.Cs[(bk * N + (col - 1 - N)) * LP + l] = v[i];
             }
         }
     }
