@@ -55,18 +55,23 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # taken from, and is reported only for that configuration while the sources
 # are unchanged.
 NCU_TRAFFIC = {
-    # ncu capture of the output pass: dram read 65492224 + write 25570560
-    "vmamba_t_stage1": {"bytes": 91062784, "dtype": "bf16", "N": 16, "src": "4f946ebf7ed334c0"},
-    # ncu capture of the output pass: dram read 141669632 + write 161776128
-    "vmamba_b_stage3": {"bytes": 303445760, "dtype": "bf16", "N": 16, "src": "4f946ebf7ed334c0"},
+    # ncu captures of the output pass (L2 flushed before the kernel by ncu):
+    # dram read 65392128 + write 25670144
+    "vmamba_t_stage1": {"bytes": 91062272, "dtype": "bf16", "N": 16, "src": "891b7f4e50017c33"},
+    # dram read 141739520 + write 161474816
+    "vmamba_b_stage3": {"bytes": 303214336, "dtype": "bf16", "N": 16, "src": "891b7f4e50017c33"},
+    # dram read 184824832 + write 156676096
+    "highres_256": {"bytes": 341500928, "dtype": "bf16", "N": 16, "src": "891b7f4e50017c33"},
+    # dram read 156436992 + write 134876928
+    "vim_s_bidir": {"bytes": 291313920, "dtype": "bf16", "N": 16, "src": "891b7f4e50017c33"},
 }
 
 
-# the files that define the forward scan kernels and their launch (the
-# kernels the traffic figures above were taken from)
+# the files that define the output pass (chunk_scan_kernel), its variant
+# choice and its launch: the kernel the traffic figures above were taken from
 FORWARD_KERNEL_SOURCES = ("ss2d_kernels.cuh", "ss2d_launch.cu", "ss2d_launch.h", "ss2d_params.h",
-                          "ss2d_scan.cuh", "ss2d_scan_bf16.cu", "ss2d_scan_f16.cu",
-                          "ss2d_scan_f32.cu", "ss2d_scan_launch.cuh")
+                          "ss2d_scan_bf16.cu", "ss2d_scan_f16.cu", "ss2d_scan_f32.cu",
+                          "ss2d_scan_launch.cuh")
 
 
 def kernel_source_hash() -> str:

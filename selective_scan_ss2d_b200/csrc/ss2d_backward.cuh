@@ -20,8 +20,8 @@
 //      and the local adjoint Q[c] = a_s g_s (g from zero at the chunk end),
 //      each with the chunk's sum of dt.  Q is stored in reversed chunk
 //      order, so that
-//   2. carry_scan_kernel (the forward's) run twice gives the entry state of every
-//      chunk and, over the reversed order, the adjoint G[c] = a_{e+1} g_{e+1}
+//   2. the forward's carry scan (launch_carry_scan) run twice gives the entry
+//      state of every chunk and, over the reversed order, the adjoint G[c] = a_{e+1} g_{e+1}
 //      entering every chunk from its end: G[c-1] = exp(A sum_c dt) G[c] + Q[c].
 //      The final pass needs G only at the top of each CTA's range of chunks;
 //      when one range covers a whole sequence, Q and its carry are skipped.

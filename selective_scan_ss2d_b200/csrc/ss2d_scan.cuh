@@ -695,218 +695,207 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
 }
 
 // Entry states of every chunk after the first, in place over the chunk end
-// states (slot c of a (b,k,d) row holds h_end of chunk c on entry and the
-// state entering chunk c+1 on exit); see the header.  All 16 states of a
-// chunk are handled by one lane.  Rows of at most 32 chunk end states: one
-// warp holds 32 / SW rows, a segment of SW lanes (SW = the power of two at or
-// above NC - 1) per row, one chunk per lane.  Longer rows: one CTA of
-// kCarryWarps warps per row, lane l of warp w owning the chunks
-// [(32w + l) * per, (32w + l + 1) * per).
-constexpr int kCarryWarps = 4;
+// states: slot c of a (b,k,d) row holds h_end of chunk c (from a zero entry
+// state) on entry and the state entering chunk c + 1 on exit.
+//
+// With a_c = exp(A * sum of dt over chunk c), chunk c maps an entry state h
+// to a_c h + h_end(c); maps compose associatively,
+//     (a1, e1) then (a2, e2) = (a1 a2, a2 e1 + e2),
+// and the entry state of chunk c is the composition of chunks 0 .. c-1
+// applied to zero.  The scan is reduce-then-scan over segments:
+//   1. thread (row, segment, state n) composes the chunks of its segment in
+//      order (16 neighbouring threads read one chunk's 16 states, one
+//      64-byte piece);
+//   2. a Kogge-Stone scan over the G segments of each (row, n), G lanes of
+//      one warp (shuffles of width G), gives each segment its entry state;
+//   3. each thread walks its segment again, writing the entry states.
+// Two forms: carry_scan_staged_kernel (below) copies a CTA's rows into
+// shared memory first, for rows of up to about 960 chunks; this one reads
+// them from global memory twice, for longer rows (32 segments, a CTA of
+// kCarryThreads threads per row).
+constexpr int kCarryThreads = 512;
 
-template <int PMAX>
-static __global__ void __launch_bounds__(32 * kCarryWarps) carry_scan_kernel(const ScanParams p, int SW)
+static __global__ void __launch_bounds__(kCarryThreads, 2)
+    carry_scan_kernel(const ScanParams p, int G, int seg_len)
 {
-    // PMAX > 0: a lane owns at most PMAX chunks, whose end states and dt sums
-    // it loads once, all at the same time, and keeps in registers for both
-    // runs over them; PMAX = 0: any number, loaded in each run
-    constexpr int PR = PMAX > 0 ? PMAX : 1;
-    __shared__ float s_tot[kCarryWarps][2][kNP];   // per warp: (a, e) of its whole range
+    __shared__ float s_a[32][kNP], s_e[32][kNP];   // per (row, segment) slot and state
     grid_dependency_wait();   // the chunk end states of the state pass
-    allow_dependents();
-    const int nw = blockDim.x >> 5;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
     const int nc1 = p.NC - 1;
     const long long rows = (long long)p.B * p.K * p.D;
-    // this lane's row, its chunks [c0, c1), its position in the row's scan
-    long long row;
-    int c0, c1, pos, seg;
-    if (nc1 <= 32) {
-        const int rpw = 32 / SW;   // rows per warp
-        row = ((long long)blockIdx.x * nw + warp) * rpw + lane / SW;
-        pos = lane & (SW - 1);
-        seg = SW;
-        c0 = min(pos, nc1);
-        c1 = min(pos + 1, nc1);
-    } else {
-        row = blockIdx.x;
-        const int per = (nc1 + 32 * nw - 1) / (32 * nw);
-        pos = lane;
-        seg = 32;
-        c0 = min((warp * 32 + lane) * per, nc1);
-        c1 = min(c0 + per, nc1);
-    }
-    const bool live = row < rows;
-    const long long rr = live ? row : 0;
-    const int d = (int)(rr % p.D);
-    const int k = (int)((rr / p.D) % p.K);
-    float *hs = p.hstate + rr * (long long)nc1 * kNP;
-    const float *ds = p.dtsum + rr * (long long)nc1;
-    const float *al = p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0;
-    if (!live)
-        c0 = c1 = 0;
-    // the lane's chunks in registers (PMAX > 0), loads in flight together
-    float hv[PR][kNP], dv[PR];
-    if constexpr (PMAX > 0) {
-#pragma unroll
-        for (int j = 0; j < PMAX; ++j) {
-            const int c = c0 + j;
-            const bool in = c < c1;
-            dv[j] = in ? ds[c] : 0.f;
-            const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)(in ? c : 0) * kNP);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = in ? he[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                hv[j][4 * q] = v.x;
-                hv[j][4 * q + 1] = v.y;
-                hv[j][4 * q + 2] = v.z;
-                hv[j][4 * q + 3] = v.w;
-            }
-        }
-    }
-    float A[kNP];
-#pragma unroll
-    for (int n = 0; n < kNP; ++n)
-        A[n] = (live && n < p.N) ? -expf(__ldg(al + n)) * kLog2e : 0.f;
+    const int rpc = 32 / G;   // rows per CTA
 
-    // the map of this lane's chunks, composed in order
-    float a[kNP], e[kNP];
-#pragma unroll
-    for (int n = 0; n < kNP; ++n) {
-        a[n] = 1.f;
-        e[n] = 0.f;
+    // ---- 1. compose the segment's chunks
+    const int slot = tid / kNP, n = tid % kNP;
+    const int rl = slot / G, sg = slot % G;
+    const long long row = (long long)blockIdx.x * rpc + rl;
+    const bool live = row < rows && n < p.N;
+    const long long rr = live ? row : 0;
+    const unsigned ur = (unsigned)rr;   // rows < 2^31 (checked at launch)
+    const int d = (int)(ur % (unsigned)p.D), k = (int)((ur / (unsigned)p.D) % (unsigned)p.K);
+    float *hs = p.hstate + rr * (long long)nc1 * kNP + n;   // slot c at hs[c * kNP]
+    const float *ds = p.dtsum + rr * (long long)nc1;
+    const int c0 = min(sg * seg_len, nc1);
+    const int cnt = live ? min(seg_len, nc1 - c0) : 0;
+    const float A2 = live ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0 + n)) * kLog2e
+                          : 0.f;
+    float a = 1.f, e = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+        const float ai = mufu_ex2(A2 * ds[c0 + j]);
+        e = fmaf(ai, e, hs[(size_t)(c0 + j) * kNP]);
+        a *= ai;
     }
-    auto compose = [&](float dsum, const float (&h)[kNP]) {
-#pragma unroll
-        for (int n = 0; n < kNP; ++n) {
-            const float ai = mufu_ex2(A[n] * dsum);
-            e[n] = fmaf(ai, e[n], h[n]);
-            a[n] *= ai;
-        }
-    };
-    if constexpr (PMAX > 0) {
-#pragma unroll
-        for (int j = 0; j < PMAX; ++j)
-            if (c0 + j < c1)
-                compose(dv[j], hv[j]);
-    } else {
-        for (int c = c0; c < c1; ++c) {
-            float h[kNP];
-            const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)c * kNP);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = he[q];
-                h[4 * q] = v.x;
-                h[4 * q + 1] = v.y;
-                h[4 * q + 2] = v.z;
-                h[4 * q + 3] = v.w;
-            }
-            compose(ds[c], h);
-        }
-    }
-    // inclusive scan across the lanes of the segment: earlier lanes' maps first
-    for (int off = 1; off < seg; off <<= 1) {
-#pragma unroll
-        for (int n = 0; n < kNP; ++n) {
-            const float au = __shfl_up_sync(0xffffffffu, a[n], off);
-            const float eu = __shfl_up_sync(0xffffffffu, e[n], off);
-            if (pos >= off) {
-                e[n] = fmaf(a[n], eu, e[n]);
-                a[n] *= au;
+    s_a[slot][n] = a;
+    s_e[slot][n] = e;
+    __syncthreads();
+
+    // ---- 2. scan over the segments of each (row, n): lane group of G lanes
+    {
+        const int pair = tid / G, q = tid % G;   // pair = (row, n)
+        const int cs = (pair / kNP) * G + q, cn = pair % kNP;
+        float ca = s_a[cs][cn], ce = s_e[cs][cn];
+        for (int off = 1; off < G; off <<= 1) {
+            const float au = __shfl_up_sync(0xffffffffu, ca, off, G);
+            const float eu = __shfl_up_sync(0xffffffffu, ce, off, G);
+            if (q >= off) {
+                ce = fmaf(ca, eu, ce);
+                ca *= au;
             }
         }
+        // entry state of segment q: the inclusive result of segment q - 1
+        const float pe = __shfl_up_sync(0xffffffffu, ce, 1, G);
+        __syncthreads();   // every slot read before any is overwritten
+        s_e[cs][cn] = q == 0 ? 0.f : pe;
     }
-    // the state entering this lane's first chunk: the inclusive result of the
-    // lane before (zero for the segment's first lane) ...
-    float pa[kNP], pe[kNP];
-#pragma unroll
-    for (int n = 0; n < kNP; ++n) {
-        pa[n] = __shfl_up_sync(0xffffffffu, a[n], 1);
-        pe[n] = __shfl_up_sync(0xffffffffu, e[n], 1);
-        if (pos == 0) {
-            pa[n] = 1.f;
-            pe[n] = 0.f;
-        }
+    __syncthreads();
+
+    // ---- 3. the entry state of each chunk after this one
+    float h = s_e[slot][n];
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+        const size_t c = (size_t)(c0 + j);
+        h = fmaf(mufu_ex2(A2 * ds[c]), h, hs[c * kNP]);
+        hs[c * kNP] = h;
     }
-    // ... after the maps of the earlier warps (one row per CTA)
-    if (nc1 > 32 && nw > 1) {
-        if (lane == 31) {
-#pragma unroll
-            for (int n = 0; n < kNP; ++n) {
-                s_tot[warp][0][n] = a[n];
-                s_tot[warp][1][n] = e[n];
+    allow_dependents();   // after the stores (see carry_scan_staged_kernel)
+}
+
+// The same scan with the CTA's rows staged in shared memory: R rows of nc1
+// chunk end states (R * nc1 * 64 bytes, contiguous in p.hstate) and their
+// dt sums are copied in with cp.async, all in flight at once; threads
+// (row, segment of seg_len chunks, state n), R * G * 16 = kCarryStagedThreads
+// of them, compose, scan over the G segments (shuffles of width G), walk
+// their segments writing entry states into the staged rows, and the CTA
+// copies the rows back with 16-byte stores.  One wave of CTAs covers the
+// rows of every shape this is used for.
+constexpr int kCarryStagedThreads = 256;
+constexpr size_t kCarryStagedSmemMax = 64 * 1024;
+
+static __global__ void __launch_bounds__(kCarryStagedThreads)
+    carry_scan_staged_kernel(const ScanParams p, int R, int G, int seg_len)
+{
+    extern __shared__ float4 carry_smem[];
+    __shared__ float s_a[kCarryStagedThreads / kNP][kNP], s_e[kCarryStagedThreads / kNP][kNP];
+    const int tid = threadIdx.x;
+    const int nc1 = p.NC - 1;
+    const long long rows = (long long)p.B * p.K * p.D;
+    const long long row0 = (long long)blockIdx.x * R;
+    const int nrows = (int)min((long long)R, rows - row0);
+    float *sh = reinterpret_cast<float *>(carry_smem);   // [R][nc1][kNP]
+    float *sd = sh + (size_t)R * nc1 * kNP;               // [R][nc1]
+    float *gh = p.hstate + row0 * nc1 * kNP;
+    const float *gd = p.dtsum + row0 * nc1;
+    const int pieces = nrows * nc1 * (kNP / 4);
+    const int nds = nrows * nc1;
+
+    // the chunk end states of the state pass.  The output pass is let in
+    // only after the last store below: triggered earlier, its CTAs take the
+    // SMs while they wait and the 256x256 step ran about 9 % longer.
+    grid_dependency_wait();
+    {
+        const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(sh));
+        const uint32_t d0 = static_cast<uint32_t>(__cvta_generic_to_shared(sd));
+        for (int i = tid; i < pieces; i += kCarryStagedThreads)
+            cp_async16(s0 + 16u * i, gh + 4 * (size_t)i);
+        for (int i = tid; i < nds; i += kCarryStagedThreads)
+            cp_async4(d0 + 4u * i, gd + i);
+        cp_async_commit();
+        cp_async_wait_all();
+    }
+    __syncthreads();
+
+    // ---- compose the segment's chunks
+    const int slot = tid / kNP, n = tid % kNP;   // slot = (row, segment)
+    const int rl = slot / G, sg = slot % G;
+    const bool live = rl < nrows && n < p.N;
+    const long long rr = live ? row0 + rl : 0;
+    const unsigned ur = (unsigned)rr;   // rows < 2^31 (checked at launch)
+    const int d = (int)(ur % (unsigned)p.D), k = (int)((ur / (unsigned)p.D) % (unsigned)p.K);
+    const float A2 = live ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0 + n)) * kLog2e
+                          : 0.f;
+    const int c0 = min(sg * seg_len, nc1);
+    const int cnt = live ? min(seg_len, nc1 - c0) : 0;
+    float *hrow = sh + ((size_t)(live ? rl : 0) * nc1 + c0) * kNP + n;   // chunk c0 + j at [j * kNP]
+    const float *drow = sd + (size_t)(live ? rl : 0) * nc1 + c0;
+    float a = 1.f, e = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+        const float ai = mufu_ex2(A2 * drow[j]);
+        e = fmaf(ai, e, hrow[j * kNP]);
+        a *= ai;
+    }
+    s_a[slot][n] = a;
+    s_e[slot][n] = e;
+    __syncthreads();
+
+    // ---- scan over the segments of each (row, n)
+    {
+        const int pair = tid / G, q = tid % G;
+        const int cs = (pair / kNP) * G + q, cn = pair % kNP;
+        float ca = s_a[cs][cn], ce = s_e[cs][cn];
+        for (int off = 1; off < G; off <<= 1) {
+            const float au = __shfl_up_sync(0xffffffffu, ca, off, G);
+            const float eu = __shfl_up_sync(0xffffffffu, ce, off, G);
+            if (q >= off) {
+                ce = fmaf(ca, eu, ce);
+                ca *= au;
             }
         }
+        const float pe = __shfl_up_sync(0xffffffffu, ce, 1, G);
         __syncthreads();
-        float we[kNP];
-#pragma unroll
-        for (int n = 0; n < kNP; ++n)
-            we[n] = 0.f;
-        for (int w = 0; w < warp; ++w) {
-#pragma unroll
-            for (int n = 0; n < kNP; ++n)
-                we[n] = fmaf(s_tot[w][0][n], we[n], s_tot[w][1][n]);
-        }
-#pragma unroll
-        for (int n = 0; n < kNP; ++n)
-            pe[n] = fmaf(pa[n], we[n], pe[n]);
+        s_e[cs][cn] = q == 0 ? 0.f : pe;
     }
-    // the state entering each chunk of the segment, over its end state
-    auto advance = [&](int c, float dsum, const float (&h)[kNP]) {
-#pragma unroll
-        for (int n = 0; n < kNP; ++n)
-            pe[n] = fmaf(mufu_ex2(A[n] * dsum), pe[n], h[n]);
-        float4 *slot = reinterpret_cast<float4 *>(hs + (size_t)c * kNP);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            slot[q] = make_float4(pe[4 * q], pe[4 * q + 1], pe[4 * q + 2], pe[4 * q + 3]);
-    };
-    if constexpr (PMAX > 0) {
-#pragma unroll
-        for (int j = 0; j < PMAX; ++j)
-            if (c0 + j < c1)
-                advance(c0 + j, dv[j], hv[j]);
-    } else {
-        for (int c = c0; c < c1; ++c) {
-            float h[kNP];
-            const float4 *he = reinterpret_cast<const float4 *>(hs + (size_t)c * kNP);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = he[q];
-                h[4 * q] = v.x;
-                h[4 * q + 1] = v.y;
-                h[4 * q + 2] = v.z;
-                h[4 * q + 3] = v.w;
-            }
-            advance(c, ds[c], h);
-        }
+    __syncthreads();
+
+    // ---- entry states into the staged rows, then back to global memory
+    float h = s_e[slot][n];
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+        h = fmaf(mufu_ex2(A2 * drow[j]), h, hrow[j * kNP]);
+        hrow[j * kNP] = h;
     }
+    __syncthreads();
+    const float4 *s4 = reinterpret_cast<const float4 *>(sh);
+    float4 *g4 = reinterpret_cast<float4 *>(gh);
+    for (int i = tid; i < pieces; i += kCarryStagedThreads)
+        g4[i] = s4[i];
+    allow_dependents();
 }
 
 // The carry scan of a plan's chunk end states (p.hstate, p.dtsum, p.NC),
 // launched on st (as a programmatic dependent of the previous kernel when
-// dependent is true).
+// dependent is true).  G: the power of two of segments (at most 32) that
+// leaves at most 16 chunks per segment where it can.
 inline cudaError_t launch_carry_scan(const ScanParams &p, cudaStream_t st, bool dependent)
 {
     const int nc1 = p.NC - 1;
+    if (nc1 < 1)
+        return cudaSuccess;
     const long long rows = (long long)p.B * p.K * p.D;
-    int SW = 1, nw = kCarryWarps;
-    long long blocks;
-    if (nc1 <= 32) {
-        while (SW < nc1)
-            SW <<= 1;
-        const long long rows_per_cta = (long long)nw * (32 / SW);
-        blocks = (rows + rows_per_cta - 1) / rows_per_cta;
-    } else {
-        nw = (nc1 + 31) / 32;
-        nw = nw > kCarryWarps ? kCarryWarps : nw;
-        blocks = rows;
-    }
-    if (blocks > 0x7fffffffLL)
+    if (rows > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(32 * nw);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     if (dependent) {
@@ -915,12 +904,33 @@ inline cudaError_t launch_carry_scan(const ScanParams &p, cudaStream_t st, bool 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    const int per = nc1 <= 32 ? 1 : (nc1 + 32 * nw - 1) / (32 * nw);   // chunks per lane
-    if (per <= 1)
-        return cudaLaunchKernelEx(&cfg, carry_scan_kernel<1>, p, SW);
-    if (per <= 4)
-        return cudaLaunchKernelEx(&cfg, carry_scan_kernel<4>, p, SW);
-    return cudaLaunchKernelEx(&cfg, carry_scan_kernel<0>, p, SW);
+    // staged: G segments of at most 16 chunks (at most 16 segments), R =
+    // 16 / G rows per CTA, while the rows fit the shared-memory budget
+    {
+        int G = 1;
+        while (G < 16 && (long long)G * 16 < nc1)
+            G <<= 1;
+        const int R = 16 / G;
+        const int seg_len = (nc1 + G - 1) / G;
+        const size_t smem = (size_t)R * nc1 * (kNP + 1) * sizeof(float);
+        const long long blocks = (rows + R - 1) / R;
+        if (smem <= kCarryStagedSmemMax) {
+            cudaError_t e = cudaFuncSetAttribute(carry_scan_staged_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess)
+                return e;
+            cfg.gridDim = dim3((unsigned)blocks);
+            cfg.blockDim = dim3(kCarryStagedThreads);
+            cfg.dynamicSmemBytes = smem;
+            return cudaLaunchKernelEx(&cfg, carry_scan_staged_kernel, p, R, G, seg_len);
+        }
+    }
+    // longer rows: 32 segments, one row per CTA
+    const int G = 32, seg_len = (nc1 + G - 1) / G;
+    cfg.gridDim = dim3((unsigned)rows);
+    cfg.blockDim = dim3(kCarryThreads);
+    return cudaLaunchKernelEx(&cfg, carry_scan_kernel, p, G, seg_len);
 }
 
 }  // namespace ss2d

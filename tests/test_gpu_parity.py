@@ -462,3 +462,19 @@ def test_map_1024x1024_sampled_channels():
     for d in (0, 5):
         sub = wl.channel_subproblem(inp, 0, d)
         _gpu.assert_close(y[0:1, d:d + 1], _gpu.run_oracle(sub), wl.BF16, f"1024^2 d={d}")
+
+
+@pytest.mark.parametrize("chunks", [4, 21, 101, 601, 1001])
+def test_carry_segments(chunks):
+    """The carry scan's segment plans, 16-step chunks (1D, K = 2, N = 5 so
+    that threads of states past N idle): 3 chunk boundaries (16 rows per CTA,
+    one segment each), 20 (two segments), 100 (eight), 600 (16 segments of
+    38 chunks, one row per CTA), all staged in shared memory; 1000 (too long
+    to stage: 32 segments read from global memory); every element against
+    the oracle at the float32 bar."""
+    cfg = small("1d", B=2, D=3, W=16 * chunks - 5, K=2, N=5)
+    inp = wl.make_inputs(cfg, seed=16)
+    v = [i for i in range(nvariants()) if binding.ss2d_variant_name(i) == "wc2_lc16"][0]
+    plan = binding.ss2d_plan(False, cfg.B, cfg.D, 1, cfg.L, cfg.N, cfg.K, v)
+    assert plan["num_chunks"] == chunks
+    _gpu.assert_close(_gpu.run_gpu(inp, variant=v), _gpu.run_oracle(inp), wl.F32, cfg.name)
