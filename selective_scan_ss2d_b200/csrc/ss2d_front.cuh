@@ -327,21 +327,35 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
     unsigned char *ab = static_cast<unsigned char *>(p.Ab) +
                         (((size_t)bk * gridDim.x + tile) * gridDim.y + cb) * kFrontABytes +
                         (c0 >> 3) * kFrontLBO + (c0 & 7) * 2;
-    float uu[CP][SG];
+    // per step: the A operand word (the pair in bf16, one packed conversion);
+    // 2-byte inputs: the pair in the input dtype, whose halves are u's values
+    // (for bf16 the A word itself); float inputs: the float values
+    uint32_t aw[SG], hw[sizeof(Tin) == 2 ? SG : 1];
+    float uu[sizeof(Tin) == 4 ? CP : 1][sizeof(Tin) == 4 ? SG : 1];
 #pragma unroll
     for (int i = 0; i < SG; ++i) {
         xrow(m0 + i + 3, win[(i + 3) & 3]);
+        float v[CP];
 #pragma unroll
         for (int j = 0; j < CP; ++j) {
             const float cv = fmaf(w[j][3], win[(i + 3) & 3][j],
                                   fmaf(w[j][2], win[(i + 2) & 3][j],
                                        fmaf(w[j][1], win[(i + 1) & 3][j], fmaf(w[j][0], win[i & 3][j], bias[j]))));
-            uu[j][i] = silu_f(cv);   // channels past D: zero inputs and taps give SiLU(0) = 0
+            v[j] = silu_f(cv);   // channels past D: zero inputs and taps give SiLU(0) = 0
         }
+        const __nv_bfloat162 a2 = __floats2bfloat162_rn(v[0], v[1]);
+        aw[i] = *reinterpret_cast<const uint32_t *>(&a2);
         const int mt = m0 + i;
-        const uint32_t wv = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(uu[0][i])) |
-                            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(uu[1][i])) << 16);
-        *reinterpret_cast<uint32_t *>(ab + (mt >> 3) * kFrontSBO + (mt & 7) * 16) = wv;
+        *reinterpret_cast<uint32_t *>(ab + (mt >> 3) * kFrontSBO + (mt & 7) * 16) = aw[i];
+        if constexpr (std::is_same_v<Tin, __half>) {
+            const __half2 h2 = __floats2half2_rn(v[0], v[1]);
+            hw[i] = *reinterpret_cast<const uint32_t *>(&h2);
+        } else if constexpr (sizeof(Tin) == 2) {
+            hw[i] = aw[i];
+        } else {
+            uu[0][i] = v[0];
+            uu[1][i] = v[1];
+        }
     }
     // u for the scan, in the input dtype: 16-byte stores of 8 (2-byte) or 4
     // (float) steps; every store starts before L (LP is a multiple of 8)
@@ -359,11 +373,13 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
                 continue;
             uint4 v;
             if constexpr (sizeof(Tin) == 2) {
+                // channel j's values of steps 2e, 2e + 1: the low (j = 0) or
+                // high (j = 1) halves of two pair words
+                const uint32_t sel = j == 0 ? 0x5410u : 0x7632u;
                 uint32_t w4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    w4[e] = store_bits(uu[j][q * PER + 2 * e], static_cast<Tin *>(nullptr)) |
-                            (store_bits(uu[j][q * PER + 2 * e + 1], static_cast<Tin *>(nullptr)) << 16);
+                    w4[e] = __byte_perm(hw[q * PER + 2 * e], hw[q * PER + 2 * e + 1], sel);
                 v = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             } else {
                 v = make_uint4(__float_as_uint(uu[j][q * PER]), __float_as_uint(uu[j][q * PER + 1]),
