@@ -11,9 +11,9 @@ namespace ss2d {
 
 namespace {
 // CTAs (one per channel group and chunk range) wanted per launch: 2960 = 148
-// SMs x 20, about 1.7 waves of the local pass (12 one-warp CTAs per SM) and
-// 6.7 of the final pass (3 four-warp CTAs per SM); fewer ranges would leave
-// SMs idle on the small-batch shapes, more would add carry work
+// SMs x 20, about 6.7 waves of the final pass (3 four-warp CTAs per SM);
+// fewer ranges would leave SMs idle on the small-batch shapes, more would
+// add carry work
 constexpr long long kBwdWantCtas = 148LL * 5 * 4;
 
 template <typename Tin>
@@ -21,7 +21,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st)
 {
     const dim3 grid((unsigned)((long long)p.G * p.B * p.K), (unsigned)p.CGN);
     if (p.NC > 1) {
-        bwd_local_kernel<Tin><<<grid, kBwdLanes, 0, st>>>(p);
+        bwd_local4_kernel<Tin><<<grid, kBwd4Threads, 0, st>>>(p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;

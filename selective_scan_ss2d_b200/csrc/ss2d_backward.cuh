@@ -14,12 +14,13 @@
 // its pixel (the adjoint of cross_scan is cross_merge).
 //
 // Work decomposition: chunks of kT = 16 steps; a CTA holds 32 channels of one
-// (b, k) (one warp for the local pass, four for the final pass) and walks a
-// range of chunks.
-//   1. bwd_local_kernel: per chunk, from zero, the forward end state h_end[c]
+// (b, k) in four warps (warp w: states 4w .. 4w+3) and walks a range of
+// chunks.
+//   1. bwd_local4_kernel: per chunk, from zero, the forward end state h_end[c]
 //      and the local adjoint Q[c] = a_s g_s (g from zero at the chunk end),
-//      each with the chunk's sum of dt.  Q is stored in reversed chunk
-//      order, so that
+//      each with the chunk's sum of dt, in one forward walk with one exp2 per
+//      state and step (Q as the sum of dy_t C_t weighted by the running
+//      product of the a's).  Q is stored in reversed chunk order, so that
 //   2. the forward's carry scan (launch_carry_scan) run twice gives the entry
 //      state of every chunk and, over the reversed order, the adjoint G[c] = a_{e+1} g_{e+1}
 //      entering every chunk from its end: G[c-1] = exp(A sum_c dt) G[c] + Q[c].
@@ -71,86 +72,6 @@ __device__ __forceinline__ BwdLane bwd_lane(const BwdParams &p)
     return r;
 }
 
-// The raw inputs of one chunk (steps s .. s+nt-1) that a lane stages: its
-// channel's delta, x and dy, and its share of the chunk's B and C (state
-// n = lane >> 1, 8 steps), loaded one chunk ahead into registers and turned
-// into the shared-memory tiles after the current chunk's work.
-template <typename Tin>
-struct BwdRaw {
-    using RawT = std::conditional_t<sizeof(Tin) == 2, unsigned short, float>;
-    RawT dl[kT], x[kT], b[kT / 2], c[kT / 2];
-    float gy[kT];
-    int nt;
-
-    __device__ __forceinline__ static float f32(RawT v)
-    {
-        if constexpr (sizeof(Tin) == 2)
-            return half_bits_to_f32<Tin>(v);
-        else
-            return v;
-    }
-
-    __device__ __forceinline__ void fetch(const BwdParams &p, const BwdLane &q, int s)
-    {
-        nt = min(kT, p.L - s);
-        const int lane = threadIdx.x;
-        const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
-        const bool nok = n < p.N;
-        const size_t row =
-            (((size_t)q.b * p.K + q.k) * p.NS + p.n0 + (nok ? n : 0)) * p.L + s + t0;
-        const RawT *Bp = static_cast<const RawT *>(p.Bs) + row;
-        const RawT *Cp = static_cast<const RawT *>(p.Cs) + row;
-#pragma unroll
-        for (int i = 0; i < kT / 2; ++i) {
-            const bool ok = nok && t0 + i < nt;
-            b[i] = ok ? __ldg(Bp + i) : RawT(0);
-            c[i] = ok ? __ldg(Cp + i) : RawT(0);
-        }
-        const RawT *dp = static_cast<const RawT *>(p.delta) + q.bkd * p.L + s;
-        const size_t xrow = ((size_t)q.b * p.D + q.d) * p.L;
-        const RawT *xp = static_cast<const RawT *>(p.x) + xrow;
-        const float *gp = p.dy + xrow;
-        PixWalk w;
-        w.init(p.two_d, q.k, s, p.H, p.W, p.L);
-#pragma unroll
-        for (int t = 0; t < kT; ++t) {
-            const bool ok = t < nt && q.active;   // idle lanes add nothing to dB, dC
-            dl[t] = ok ? __ldg(dp + t) : RawT(0);
-            x[t] = ok ? __ldg(xp + w.p) : RawT(0);
-            gy[t] = ok ? __ldg(gp + w.p) : 0.f;
-            if (t + 1 < nt)
-                w.next(p.H, p.W);
-        }
-    }
-
-    // sB, sC [t][n] and st4 [t][lane] = (dt, u, dy, sigmoid(z)), z = delta + bias;
-    // steps past nt (and idle lanes) stage zeros: dt = 0 makes a step the identity
-    __device__ __forceinline__ void commit(float *sB, float *sC, float4 *st4, float bias,
-                                           bool active) const
-    {
-        const int lane = threadIdx.x;
-        const int n = lane >> 1, t0 = (lane & 1) * (kT / 2);
-#pragma unroll
-        for (int i = 0; i < kT / 2; ++i) {
-            sB[(t0 + i) * kNP + n] = f32(b[i]);
-            sC[(t0 + i) * kNP + n] = f32(c[i]);
-        }
-#pragma unroll
-        for (int t = 0; t < kT; ++t) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t < nt && active) {
-                const float z = f32(dl[t]) + bias;
-                v.x = softplus_f(z);
-                v.y = f32(x[t]);
-                v.z = gy[t];
-                // sigmoid(z) = 1 / (1 + e^-z); e^-z = inf gives 0
-                v.w = __fdividef(1.f, 1.f + mufu_ex2(-z * kLog2e));
-            }
-            st4[t * kBwdLanes + lane] = v;
-        }
-    }
-};
-
 __device__ __forceinline__ void store16(float *dst, const float *v)
 {
     float4 *d4 = reinterpret_cast<float4 *>(dst);
@@ -179,80 +100,6 @@ __device__ __forceinline__ void load_a2(float2 *A2, const BwdParams &p, size_t k
         const float *al = p.A_log + kd * p.NS + p.n0;
         A2[j].x = n0 < p.N ? -expf(__ldg(al + n0)) * kLog2e : 0.f;
         A2[j].y = n1 < p.N ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
-    }
-}
-// one step of the state recurrence, h = exp(dt A) h + dt u B, for all pairs
-__device__ __forceinline__ void state_step(float2 *h, const float2 *A2, float dt, float dtu,
-                                           const float *brow)
-{
-    const float2 dt2 = dup2(dt), dtu2 = dup2(dtu);
-#pragma unroll
-    for (int j = 0; j < kNP / 2; ++j)
-        h[j] = __ffma2_rn(ex2_pair(__fmul2_rn(dt2, A2[j])), h[j],
-                          __fmul2_rn(dtu2, row_pair(brow, j)));
-}
-
-template <typename Tin>
-__global__ void __launch_bounds__(kBwdLanes) bwd_local_kernel(const BwdParams p)
-{
-    __shared__ float4 sm4[kBwdStage / 4];
-    float *sB = reinterpret_cast<float *>(sm4), *sC = sB + kT * kNP;
-    float4 *st4 = sm4 + 2 * kT * kNP / 4;
-    const int lane = threadIdx.x;
-    const BwdLane q = bwd_lane(p);
-    const size_t kd = (size_t)q.k * p.D + q.d;
-    float2 A2[kNP / 2];
-    load_a2(A2, p, kd);
-    const float bias = __ldg(p.delta_bias + kd);
-    const int nc1 = p.NC - 1;
-    const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
-    BwdRaw<Tin> raw;
-    raw.fetch(p, q, c0 * kT);
-    for (int c = c0; c < c1; ++c) {
-        __syncwarp();
-        raw.commit(sB, sC, st4, bias, q.active);
-        __syncwarp();
-        if (c + 1 < c1)
-            raw.fetch(p, q, (c + 1) * kT);   // in flight during this chunk's work
-        float dts = 0.f;
-#pragma unroll
-        for (int t = 0; t < kT; ++t)
-            dts += st4[t * kBwdLanes + lane].x;
-        if (c < nc1) {
-            float2 h[kNP / 2];
-#pragma unroll
-            for (int j = 0; j < kNP / 2; ++j)
-                h[j] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int t = 0; t < kT; ++t) {
-                const float4 v = st4[t * kBwdLanes + lane];
-                state_step(h, A2, v.x, v.x * v.y, sB + t * kNP);
-            }
-            if (q.active) {
-                store16(p.hfwd + (q.bkd * nc1 + c) * kNP, reinterpret_cast<const float *>(h));
-                p.dtf[q.bkd * nc1 + c] = dts;
-            }
-        }
-        if (c > 0 && p.adj_chunks) {
-            float2 g[kNP / 2];
-#pragma unroll
-            for (int j = 0; j < kNP / 2; ++j)
-                g[j] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int t = kT - 1; t >= 0; --t) {
-                const float4 v = st4[t * kBwdLanes + lane];
-                const float2 dt2 = dup2(v.x), gy2 = dup2(v.z);
-#pragma unroll
-                for (int j = 0; j < kNP / 2; ++j)
-                    g[j] = __fmul2_rn(ex2_pair(__fmul2_rn(dt2, A2[j])),
-                                      __ffma2_rn(gy2, row_pair(sC + t * kNP, j), g[j]));
-            }
-            if (q.active) {
-                const int r = nc1 - c;   // reversed chunk order
-                store16(p.hadj + (q.bkd * nc1 + r) * kNP, reinterpret_cast<const float *>(g));
-                p.dta[q.bkd * nc1 + r] = dts;
-            }
-        }
     }
 }
 
@@ -372,6 +219,104 @@ struct BwdRaw4 {
         }
     }
 };
+
+// One forward walk over a staged chunk from zero for the warp's 4 states
+// (4w .. 4w+3: pairs A2[0], A2[1]), one exp2 per state and step serving both
+// results:
+//   HS: the end state h (h = a_t h + dt_t u_t B_t);
+//   QS: the local adjoint Q = a_0 g_0 with g from zero at the chunk end,
+//       g_t = a_t (dy_t C_t + g_{t+1}); unrolled, Q = sum_t P_t dy_t C_t with
+//       P_t = a_0 a_1 ... a_t, which the walk accumulates forwards.
+template <bool HS, bool QS>
+__device__ __forceinline__ void local_walk4(const float4 *st4, const float *sB, const float *sC,
+                                            const float2 (&A2)[2], int nw, float2 (&h)[2],
+                                            float2 (&Q)[2])
+{
+    const int lane = threadIdx.x & 31;
+    float2 P[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        h[j] = make_float2(0.f, 0.f);
+        Q[j] = make_float2(0.f, 0.f);
+        P[j] = make_float2(1.f, 1.f);
+    }
+#pragma unroll 4
+    for (int t = 0; t < kT; ++t) {
+        const float4 v = st4[t * kBwdLanes + lane];
+        const float2 dt2 = dup2(v.x), dtu2 = dup2(v.x * v.y), gy2 = dup2(v.z);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const float2 a = ex2_pair(__fmul2_rn(dt2, A2[j]));
+            if constexpr (HS)
+                h[j] = __ffma2_rn(a, h[j], __fmul2_rn(dtu2, row_pair(sB + t * kNP + nw, j)));
+            if constexpr (QS) {
+                P[j] = __fmul2_rn(P[j], a);
+                Q[j] = __ffma2_rn(P[j], __fmul2_rn(gy2, row_pair(sC + t * kNP + nw, j)), Q[j]);
+            }
+        }
+    }
+}
+
+// The local pass with the 16 states of a channel group split over 4 warps
+// (warp w: states 4w .. 4w+3 of the same 32 channels), the chunk's inputs
+// staged once for the CTA (BwdRaw4): per chunk of its range, from zero, the
+// forward end state h_end[c] and the local adjoint Q[c], each with the
+// chunk's sum of dt, in one forward walk.
+template <typename Tin>
+__global__ void __launch_bounds__(kBwd4Threads, 4) bwd_local4_kernel(const BwdParams p)
+{
+    __shared__ float4 sm4[kBwdStage / 4];
+    float *sB = reinterpret_cast<float *>(sm4), *sC = sB + kT * kNP;
+    float4 *st4 = sm4 + 2 * kT * kNP / 4;   // [t][lane]
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const BwdLane q = bwd_lane(p);
+    const size_t kd = (size_t)q.k * p.D + q.d;
+    const int nw = 4 * w;   // this warp's first state within the group
+    float2 A2[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float *al = p.A_log + kd * p.NS + p.n0 + nw;
+        A2[j].x = nw + 2 * j < p.N ? -expf(__ldg(al + 2 * j)) * kLog2e : 0.f;
+        A2[j].y = nw + 2 * j + 1 < p.N ? -expf(__ldg(al + 2 * j + 1)) * kLog2e : 0.f;
+    }
+    const float bias = __ldg(p.delta_bias + kd);
+    const int nc1 = p.NC - 1;
+    const int c0 = blockIdx.y * p.CPB, c1 = min(p.NC, c0 + p.CPB);
+    BwdRaw4<Tin> raw;
+    raw.fetch(p, q, c0 * kT);
+    for (int c = c0; c < c1; ++c) {
+        __syncthreads();   // the previous chunk's tiles are read
+        raw.commit(sB, sC, st4, bias, q.active);
+        __syncthreads();
+        if (c + 1 < c1)
+            raw.fetch(p, q, (c + 1) * kT);   // in flight during this chunk's work
+        float dts = 0.f;
+#pragma unroll
+        for (int t = 0; t < kT; ++t)
+            dts += st4[t * kBwdLanes + lane].x;
+        const bool hs = c < nc1, qs = c > 0 && p.adj_chunks;
+        float2 h[2], g[2];
+        if (hs && qs)
+            local_walk4<true, true>(st4, sB, sC, A2, nw, h, g);
+        else if (hs)
+            local_walk4<true, false>(st4, sB, sC, A2, nw, h, g);
+        else if (qs)
+            local_walk4<false, true>(st4, sB, sC, A2, nw, h, g);
+        if (hs && q.active) {
+            *reinterpret_cast<float4 *>(p.hfwd + (q.bkd * nc1 + c) * kNP + nw) =
+                make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+            if (w == 0)
+                p.dtf[q.bkd * nc1 + c] = dts;
+        }
+        if (qs && q.active) {
+            const int r = nc1 - c;   // reversed chunk order
+            *reinterpret_cast<float4 *>(p.hadj + (q.bkd * nc1 + r) * kNP + nw) =
+                make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
+            if (w == 0)
+                p.dta[q.bkd * nc1 + r] = dts;
+        }
+    }
+}
 
 template <typename Tin>
 __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParams p)

@@ -702,191 +702,123 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
 // to a_c h + h_end(c); maps compose associatively,
 //     (a1, e1) then (a2, e2) = (a1 a2, a2 e1 + e2),
 // and the entry state of chunk c is the composition of chunks 0 .. c-1
-// applied to zero.  The scan is reduce-then-scan over segments:
-//   1. thread (row, segment, state n) composes the chunks of its segment in
-//      order (16 neighbouring threads read one chunk's 16 states, one
-//      64-byte piece);
-//   2. a Kogge-Stone scan over the G segments of each (row, n), G lanes of
-//      one warp (shuffles of width G), gives each segment its entry state;
-//   3. each thread walks its segment again, writing the entry states.
-// Two forms: carry_scan_staged_kernel (below) copies a CTA's rows into
-// shared memory first, for rows of up to about 960 chunks; this one reads
-// them from global memory twice, for longer rows (32 segments, a CTA of
-// kCarryThreads threads per row).
-constexpr int kCarryThreads = 512;
+// applied to zero.  Thread (row, segment, state n) owns a segment of
+// seg_len chunks of one row (16 neighbouring threads read one chunk's 16
+// states, one 64-byte piece; chunks stream through two register groups of
+// 16, the next group's loads in flight while the current one is applied):
+//   1. it composes its segment's maps in order;
+//   2. a Kogge-Stone scan over the G segments of each (row, n) -- G lanes of
+//      one warp, shuffles of width G -- gives every segment its entry state;
+//   3. it walks its segment again, writing the entry states.
+// G (a power of two <= 16) is chosen for parallelism: with rows * 16 threads
+// already filling the GPU, G = 1 and steps 1-2 vanish (one sequential walk
+// per (row, n)); small batches and long rows (the 256x256 map: 768 rows of
+// 511 chunks) get up to 16 segments.  A CTA of kCarryThreads threads holds
+// 16 / G rows.
+constexpr int kCarryThreads = 256;
+constexpr int kCarryGroup = 16;   // chunks per register group
 
-static __global__ void __launch_bounds__(kCarryThreads, 2)
+static __global__ void __launch_bounds__(kCarryThreads)
     carry_scan_kernel(const ScanParams p, int G, int seg_len)
 {
-    __shared__ float s_a[32][kNP], s_e[32][kNP];   // per (row, segment) slot and state
-    grid_dependency_wait();   // the chunk end states of the state pass
+    constexpr int GB = kCarryGroup;
+    __shared__ float s_a[kCarryThreads / kNP][kNP], s_e[kCarryThreads / kNP][kNP];
+    // the chunk end states of the state pass (the output pass is let in only
+    // after the last store: triggered earlier, its waiting CTAs held the SMs
+    // and the 256x256 step ran about 9 % longer)
+    grid_dependency_wait();
     const int tid = threadIdx.x;
     const int nc1 = p.NC - 1;
     const long long rows = (long long)p.B * p.K * p.D;
-    const int rpc = 32 / G;   // rows per CTA
-
-    // ---- 1. compose the segment's chunks
-    const int slot = tid / kNP, n = tid % kNP;
+    const int rpc = (kCarryThreads / kNP) / G;   // rows per CTA
+    const int slot = tid / kNP, n = tid % kNP;   // slot = (row, segment)
     const int rl = slot / G, sg = slot % G;
     const long long row = (long long)blockIdx.x * rpc + rl;
     const bool live = row < rows && n < p.N;
     const long long rr = live ? row : 0;
     const unsigned ur = (unsigned)rr;   // rows < 2^31 (checked at launch)
     const int d = (int)(ur % (unsigned)p.D), k = (int)((ur / (unsigned)p.D) % (unsigned)p.K);
-    float *hs = p.hstate + rr * (long long)nc1 * kNP + n;   // slot c at hs[c * kNP]
-    const float *ds = p.dtsum + rr * (long long)nc1;
     const int c0 = min(sg * seg_len, nc1);
     const int cnt = live ? min(seg_len, nc1 - c0) : 0;
+    float *hs = p.hstate + (rr * (long long)nc1 + c0) * kNP + n;   // chunk c0 + j at [j * kNP]
+    const float *ds = p.dtsum + rr * (long long)nc1 + c0;
     const float A2 = live ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0 + n)) * kLog2e
                           : 0.f;
-    float a = 1.f, e = 0.f;
-#pragma unroll 4
-    for (int j = 0; j < cnt; ++j) {
-        const float ai = mufu_ex2(A2 * ds[c0 + j]);
-        e = fmaf(ai, e, hs[(size_t)(c0 + j) * kNP]);
-        a *= ai;
-    }
-    s_a[slot][n] = a;
-    s_e[slot][n] = e;
-    __syncthreads();
 
-    // ---- 2. scan over the segments of each (row, n): lane group of G lanes
-    {
-        const int pair = tid / G, q = tid % G;   // pair = (row, n)
-        const int cs = (pair / kNP) * G + q, cn = pair % kNP;
-        float ca = s_a[cs][cn], ce = s_e[cs][cn];
-        for (int off = 1; off < G; off <<= 1) {
-            const float au = __shfl_up_sync(0xffffffffu, ca, off, G);
-            const float eu = __shfl_up_sync(0xffffffffu, ce, off, G);
-            if (q >= off) {
-                ce = fmaf(ca, eu, ce);
-                ca *= au;
-            }
+    float hA[GB], dA[GB], hB[GB], dB[GB];
+    auto load = [&](float *hv, float *dv, int j0) {
+#pragma unroll
+        for (int i = 0; i < GB; ++i) {
+            const bool ok = j0 + i < cnt;
+            hv[i] = ok ? hs[(size_t)(j0 + i) * kNP] : 0.f;
+            dv[i] = ok ? ds[j0 + i] : 0.f;
         }
-        // entry state of segment q: the inclusive result of segment q - 1
-        const float pe = __shfl_up_sync(0xffffffffu, ce, 1, G);
-        __syncthreads();   // every slot read before any is overwritten
-        s_e[cs][cn] = q == 0 ? 0.f : pe;
-    }
-    __syncthreads();
-
-    // ---- 3. the entry state of each chunk after this one
-    float h = s_e[slot][n];
-#pragma unroll 4
-    for (int j = 0; j < cnt; ++j) {
-        const size_t c = (size_t)(c0 + j);
-        h = fmaf(mufu_ex2(A2 * ds[c]), h, hs[c * kNP]);
-        hs[c * kNP] = h;
-    }
-    allow_dependents();   // after the stores (see carry_scan_staged_kernel)
-}
-
-// The same scan with the CTA's rows staged in shared memory: R rows of nc1
-// chunk end states (R * nc1 * 64 bytes, contiguous in p.hstate) and their
-// dt sums are copied in with cp.async, all in flight at once; threads
-// (row, segment of seg_len chunks, state n), R * G * 16 = kCarryStagedThreads
-// of them, compose, scan over the G segments (shuffles of width G), walk
-// their segments writing entry states into the staged rows, and the CTA
-// copies the rows back with 16-byte stores.  One wave of CTAs covers the
-// rows of every shape this is used for.
-constexpr int kCarryStagedThreads = 256;
-constexpr size_t kCarryStagedSmemMax = 64 * 1024;
-
-static __global__ void __launch_bounds__(kCarryStagedThreads)
-    carry_scan_staged_kernel(const ScanParams p, int R, int G, int seg_len)
-{
-    extern __shared__ float4 carry_smem[];
-    __shared__ float s_a[kCarryStagedThreads / kNP][kNP], s_e[kCarryStagedThreads / kNP][kNP];
-    const int tid = threadIdx.x;
-    const int nc1 = p.NC - 1;
-    const long long rows = (long long)p.B * p.K * p.D;
-    const long long row0 = (long long)blockIdx.x * R;
-    const int nrows = (int)min((long long)R, rows - row0);
-    float *sh = reinterpret_cast<float *>(carry_smem);   // [R][nc1][kNP]
-    float *sd = sh + (size_t)R * nc1 * kNP;               // [R][nc1]
-    float *gh = p.hstate + row0 * nc1 * kNP;
-    const float *gd = p.dtsum + row0 * nc1;
-    const int pieces = nrows * nc1 * (kNP / 4);
-    const int nds = nrows * nc1;
-
-    // the chunk end states of the state pass.  The output pass is let in
-    // only after the last store below: triggered earlier, its CTAs take the
-    // SMs while they wait and the 256x256 step ran about 9 % longer.
-    grid_dependency_wait();
-    {
-        const uint32_t s0 = static_cast<uint32_t>(__cvta_generic_to_shared(sh));
-        const uint32_t d0 = static_cast<uint32_t>(__cvta_generic_to_shared(sd));
-        for (int i = tid; i < pieces; i += kCarryStagedThreads)
-            cp_async16(s0 + 16u * i, gh + 4 * (size_t)i);
-        for (int i = tid; i < nds; i += kCarryStagedThreads)
-            cp_async4(d0 + 4u * i, gd + i);
-        cp_async_commit();
-        cp_async_wait_all();
-    }
-    __syncthreads();
-
-    // ---- compose the segment's chunks
-    const int slot = tid / kNP, n = tid % kNP;   // slot = (row, segment)
-    const int rl = slot / G, sg = slot % G;
-    const bool live = rl < nrows && n < p.N;
-    const long long rr = live ? row0 + rl : 0;
-    const unsigned ur = (unsigned)rr;   // rows < 2^31 (checked at launch)
-    const int d = (int)(ur % (unsigned)p.D), k = (int)((ur / (unsigned)p.D) % (unsigned)p.K);
-    const float A2 = live ? -expf(__ldg(p.A_log + ((size_t)k * p.D + d) * p.NS + p.n0 + n)) * kLog2e
-                          : 0.f;
-    const int c0 = min(sg * seg_len, nc1);
-    const int cnt = live ? min(seg_len, nc1 - c0) : 0;
-    float *hrow = sh + ((size_t)(live ? rl : 0) * nc1 + c0) * kNP + n;   // chunk c0 + j at [j * kNP]
-    const float *drow = sd + (size_t)(live ? rl : 0) * nc1 + c0;
-    float a = 1.f, e = 0.f;
-#pragma unroll 4
-    for (int j = 0; j < cnt; ++j) {
-        const float ai = mufu_ex2(A2 * drow[j]);
-        e = fmaf(ai, e, hrow[j * kNP]);
-        a *= ai;
-    }
-    s_a[slot][n] = a;
-    s_e[slot][n] = e;
-    __syncthreads();
-
-    // ---- scan over the segments of each (row, n)
-    {
-        const int pair = tid / G, q = tid % G;
-        const int cs = (pair / kNP) * G + q, cn = pair % kNP;
-        float ca = s_a[cs][cn], ce = s_e[cs][cn];
-        for (int off = 1; off < G; off <<= 1) {
-            const float au = __shfl_up_sync(0xffffffffu, ca, off, G);
-            const float eu = __shfl_up_sync(0xffffffffu, ce, off, G);
-            if (q >= off) {
-                ce = fmaf(ca, eu, ce);
-                ca *= au;
-            }
+    };
+    // the segment's chunks in order, group by group, f applied to each
+    auto stream = [&](auto &&f) {
+        load(hA, dA, 0);
+        for (int j0 = 0; j0 < cnt; j0 += 2 * GB) {
+            if (j0 + GB < cnt)
+                load(hB, dB, j0 + GB);
+#pragma unroll
+            for (int i = 0; i < GB; ++i)
+                if (j0 + i < cnt)
+                    f(j0 + i, hA[i], dA[i]);
+            if (j0 + GB >= cnt)
+                break;
+            if (j0 + 2 * GB < cnt)
+                load(hA, dA, j0 + 2 * GB);
+#pragma unroll
+            for (int i = 0; i < GB; ++i)
+                if (j0 + GB + i < cnt)
+                    f(j0 + GB + i, hB[i], dB[i]);
         }
-        const float pe = __shfl_up_sync(0xffffffffu, ce, 1, G);
+    };
+
+    float h = 0.f;   // the state entering the segment
+    if (G > 1) {
+        // ---- 1. compose the segment's maps
+        float a = 1.f, e = 0.f;
+        stream([&](int, float he, float dsum) {
+            const float ai = mufu_ex2(A2 * dsum);
+            e = fmaf(ai, e, he);
+            a *= ai;
+        });
+        s_a[slot][n] = a;
+        s_e[slot][n] = e;
         __syncthreads();
-        s_e[cs][cn] = q == 0 ? 0.f : pe;
+        // ---- 2. scan over the segments of each (row, n): lane group of G lanes
+        {
+            const int pair = tid / G, q = tid % G;   // pair = (row, n)
+            const int cs = (pair / kNP) * G + q, cn = pair % kNP;
+            float ca = s_a[cs][cn], ce = s_e[cs][cn];
+            for (int off = 1; off < G; off <<= 1) {
+                const float au = __shfl_up_sync(0xffffffffu, ca, off, G);
+                const float eu = __shfl_up_sync(0xffffffffu, ce, off, G);
+                if (q >= off) {
+                    ce = fmaf(ca, eu, ce);
+                    ca *= au;
+                }
+            }
+            // entry state of segment q: the inclusive result of segment q - 1
+            const float pe = __shfl_up_sync(0xffffffffu, ce, 1, G);
+            __syncthreads();   // every slot read before any is overwritten
+            s_e[cs][cn] = q == 0 ? 0.f : pe;
+        }
+        __syncthreads();
+        h = s_e[slot][n];
     }
-    __syncthreads();
-
-    // ---- entry states into the staged rows, then back to global memory
-    float h = s_e[slot][n];
-#pragma unroll 4
-    for (int j = 0; j < cnt; ++j) {
-        h = fmaf(mufu_ex2(A2 * drow[j]), h, hrow[j * kNP]);
-        hrow[j * kNP] = h;
-    }
-    __syncthreads();
-    const float4 *s4 = reinterpret_cast<const float4 *>(sh);
-    float4 *g4 = reinterpret_cast<float4 *>(gh);
-    for (int i = tid; i < pieces; i += kCarryStagedThreads)
-        g4[i] = s4[i];
+    // ---- 3. the entry state of each chunk after this one
+    stream([&](int j, float he, float dsum) {
+        h = fmaf(mufu_ex2(A2 * dsum), h, he);
+        hs[(size_t)j * kNP] = h;
+    });
     allow_dependents();
 }
 
 // The carry scan of a plan's chunk end states (p.hstate, p.dtsum, p.NC),
 // launched on st (as a programmatic dependent of the previous kernel when
-// dependent is true).  G: the power of two of segments (at most 32) that
-// leaves at most 16 chunks per segment where it can.
+// dependent is true).
 inline cudaError_t launch_carry_scan(const ScanParams &p, cudaStream_t st, bool dependent)
 {
     const int nc1 = p.NC - 1;
@@ -895,7 +827,19 @@ inline cudaError_t launch_carry_scan(const ScanParams &p, cudaStream_t st, bool 
     const long long rows = (long long)p.B * p.K * p.D;
     if (rows > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
+    // segments: double them while the threads number under 64K (about 3
+    // resident CTAs of 256 on each of 148 SMs, twice) and segments keep at
+    // least 8 chunks
+    constexpr long long kWantThreads = 65536;
+    int G = 1;
+    while (G < 16 && rows * kNP * G < kWantThreads && nc1 >= 16 * G)
+        G <<= 1;
+    const int seg_len = (nc1 + G - 1) / G;
+    const long long rpc = (kCarryThreads / kNP) / G;
+    const long long blocks = (rows + rpc - 1) / rpc;
     cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kCarryThreads);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     if (dependent) {
@@ -904,32 +848,6 @@ inline cudaError_t launch_carry_scan(const ScanParams &p, cudaStream_t st, bool 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    // staged: G segments of at most 16 chunks (at most 16 segments), R =
-    // 16 / G rows per CTA, while the rows fit the shared-memory budget
-    {
-        int G = 1;
-        while (G < 16 && (long long)G * 16 < nc1)
-            G <<= 1;
-        const int R = 16 / G;
-        const int seg_len = (nc1 + G - 1) / G;
-        const size_t smem = (size_t)R * nc1 * (kNP + 1) * sizeof(float);
-        const long long blocks = (rows + R - 1) / R;
-        if (smem <= kCarryStagedSmemMax) {
-            cudaError_t e = cudaFuncSetAttribute(carry_scan_staged_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem);
-            if (e != cudaSuccess)
-                return e;
-            cfg.gridDim = dim3((unsigned)blocks);
-            cfg.blockDim = dim3(kCarryStagedThreads);
-            cfg.dynamicSmemBytes = smem;
-            return cudaLaunchKernelEx(&cfg, carry_scan_staged_kernel, p, R, G, seg_len);
-        }
-    }
-    // longer rows: 32 segments, one row per CTA
-    const int G = 32, seg_len = (nc1 + G - 1) / G;
-    cfg.gridDim = dim3((unsigned)rows);
-    cfg.blockDim = dim3(kCarryThreads);
     return cudaLaunchKernelEx(&cfg, carry_scan_kernel, p, G, seg_len);
 }
 
