@@ -180,17 +180,64 @@ struct BwdRaw4 {
         const size_t xrow = ((size_t)q.b * p.D + q.d) * p.L;
         const RawT *xp = static_cast<const RawT *>(p.x) + xrow;
         const float *gp = p.dy + xrow;
-        PixWalk pw;
-        pw.init(p.two_d, q.k, min(s + 4 * w, p.L - 1), p.H, p.W, p.L);
+        const int t0 = 4 * w;
+        // the 4 steps whole and L % 4 == 0: the delta row segment is one
+        // 8-byte (2-byte types) or 16-byte load, and so are x and dy of the
+        // row-major directions (pixels s+t0.. ascending, or descending from
+        // L-1-s-t0: loaded ascending from L-4-s-t0 and reversed); every such
+        // segment starts on a multiple of 4 elements
+        const bool vec = (p.L & 3) == 0 && t0 + 4 <= nt && q.active;
+        const int xmode = (!p.two_d || q.k < 2) ? (q.k & 1) : 2;
+        if (vec) {
+            load4(dp + t0, dl);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = 4 * w + i;
-            const bool ok = t < nt && q.active;   // idle lanes add nothing to dB, dC
-            dl[i] = ok ? __ldg(dp + t) : RawT(0);
-            x[i] = ok ? __ldg(xp + pw.p) : RawT(0);
-            gy[i] = ok ? __ldg(gp + pw.p) : 0.f;
-            if (t + 1 < nt)
-                pw.next(p.H, p.W);
+            for (int i = 0; i < 4; ++i) {
+                const bool ok = t0 + i < nt && q.active;   // idle lanes add nothing to dB, dC
+                dl[i] = ok ? __ldg(dp + t0 + i) : RawT(0);
+            }
+        }
+        if (vec && xmode != 2) {
+            const int base = xmode == 0 ? s + t0 : p.L - 4 - s - t0;
+            RawT xv[4];
+            load4(xp + base, xv);
+            const float4 g4 = __ldg(reinterpret_cast<const float4 *>(gp + base));
+            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[i] = xmode == 0 ? xv[i] : xv[3 - i];
+                gy[i] = xmode == 0 ? gv[i] : gv[3 - i];
+            }
+        } else {
+            PixWalk pw;
+            pw.init(p.two_d, q.k, min(s + t0, p.L - 1), p.H, p.W, p.L);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = t0 + i;
+                const bool ok = t < nt && q.active;
+                x[i] = ok ? __ldg(xp + pw.p) : RawT(0);
+                gy[i] = ok ? __ldg(gp + pw.p) : 0.f;
+                if (t + 1 < nt)
+                    pw.next(p.H, p.W);
+            }
+        }
+    }
+    // 4 consecutive values from a 4-element-aligned address: one 8-byte
+    // (2-byte types) or 16-byte load
+    __device__ __forceinline__ static void load4(const RawT *src, RawT (&v)[4])
+    {
+        if constexpr (sizeof(RawT) == 2) {
+            const uint2 r = __ldg(reinterpret_cast<const uint2 *>(src));
+            v[0] = (RawT)(r.x & 0xffffu);
+            v[1] = (RawT)(r.x >> 16);
+            v[2] = (RawT)(r.y & 0xffffu);
+            v[3] = (RawT)(r.y >> 16);
+        } else {
+            const float4 r = __ldg(reinterpret_cast<const float4 *>(src));
+            v[0] = r.x;
+            v[1] = r.y;
+            v[2] = r.z;
+            v[3] = r.w;
         }
     }
 
