@@ -48,7 +48,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 // shared memory of the local pass (floats): B and C of the chunk [t][n], and
 // the lanes' staged (dt, u, dy, sigmoid(delta + bias)) as float4 [t][lane]
-constexpr int kBwdStage = 2 * kT * kNP + 4 * kT * kBwdLanes;
+// B and C tiles [t][kBCS]: rows of 16 states padded to 20 floats, so that
+// the staging stores (16 consecutive steps of a state per half warp) fall
+// into 16 different banks pairwise instead of two, and rows stay 16-byte
+// aligned for the walks' float4 reads
+constexpr int kBCS = 20;
+constexpr int kBwdStage = 2 * kT * kBCS + 4 * kT * kBwdLanes;
 
 struct BwdLane {
     int b, k, gi, d, bk;
@@ -72,14 +77,6 @@ __device__ __forceinline__ BwdLane bwd_lane(const BwdParams &p)
     return r;
 }
 
-__device__ __forceinline__ void store16(float *dst, const float *v)
-{
-    float4 *d4 = reinterpret_cast<float4 *>(dst);
-#pragma unroll
-    for (int i = 0; i < kNP / 4; ++i)
-        d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-}
-
 // States in pairs (2j, 2j+1) for the sm_100 packed f32x2 instructions
 // (__ffma2_rn, __fmul2_rn: each lane rounds as fmaf / a float multiply).
 __device__ __forceinline__ float2 ex2_pair(float2 a)
@@ -87,20 +84,10 @@ __device__ __forceinline__ float2 ex2_pair(float2 a)
     return make_float2(mufu_ex2(a.x), mufu_ex2(a.y));
 }
 __device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
-// pair j of a 16-float shared-memory row (16-byte aligned)
+// pair j of a shared-memory row of states (16-byte aligned)
 __device__ __forceinline__ float2 row_pair(const float *row, int j)
 {
     return reinterpret_cast<const float2 *>(row)[j];
-}
-__device__ __forceinline__ void load_a2(float2 *A2, const BwdParams &p, size_t kd)
-{
-#pragma unroll
-    for (int j = 0; j < kNP / 2; ++j) {
-        const int n0 = 2 * j, n1 = 2 * j + 1;
-        const float *al = p.A_log + kd * p.NS + p.n0;
-        A2[j].x = n0 < p.N ? -expf(__ldg(al + n0)) * kLog2e : 0.f;
-        A2[j].y = n1 < p.N ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -112,7 +99,7 @@ __device__ __forceinline__ void load_a2(float2 *A2, const BwdParams &p, size_t k
 // memory once per chunk, each warp finishing 4 of the 16 steps.
 constexpr int kQuadWarps = 4;
 constexpr int kBwd4Threads = kQuadWarps * kBwdLanes;
-constexpr int kBwd4Stage = 2 * kT * kNP + 4 * kT * kBwdLanes;   // B|C tiles, st4
+constexpr int kBwd4Stage = 2 * kT * kBCS + 4 * kT * kBwdLanes;   // B|C tiles, st4
 constexpr int kBwd4Hs = kQuadWarps * kT * kBwdLanes * 4;         // per warp [t][lane] float4
 constexpr int kBwd4Sums = kQuadWarps * kT * kBwdLanes * 2;       // per warp [t][lane] (s1, s2)
 constexpr int kBwd4Red = kQuadWarps * kT * 8;                    // per warp [t][8] reduced dB|dC
@@ -249,7 +236,7 @@ struct BwdRaw4 {
         for (int i = 0; i < 4; ++i) {
             const int item = tid + i * kBwd4Threads;
             const int which = item >> 8, n = (item >> 4) & 15, t = item & 15;
-            (which ? sC : sB)[t * kNP + n] = f32(bc[i]);
+            (which ? sC : sB)[t * kBCS + n] = f32(bc[i]);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -295,10 +282,10 @@ __device__ __forceinline__ void local_walk4(const float4 *st4, const float *sB, 
         for (int j = 0; j < 2; ++j) {
             const float2 a = ex2_pair(__fmul2_rn(dt2, A2[j]));
             if constexpr (HS)
-                h[j] = __ffma2_rn(a, h[j], __fmul2_rn(dtu2, row_pair(sB + t * kNP + nw, j)));
+                h[j] = __ffma2_rn(a, h[j], __fmul2_rn(dtu2, row_pair(sB + t * kBCS + nw, j)));
             if constexpr (QS) {
                 P[j] = __fmul2_rn(P[j], a);
-                Q[j] = __ffma2_rn(P[j], __fmul2_rn(gy2, row_pair(sC + t * kNP + nw, j)), Q[j]);
+                Q[j] = __ffma2_rn(P[j], __fmul2_rn(gy2, row_pair(sC + t * kBCS + nw, j)), Q[j]);
             }
         }
     }
@@ -313,8 +300,8 @@ template <typename Tin>
 __global__ void __launch_bounds__(kBwd4Threads, 4) bwd_local4_kernel(const BwdParams p)
 {
     __shared__ float4 sm4[kBwdStage / 4];
-    float *sB = reinterpret_cast<float *>(sm4), *sC = sB + kT * kNP;
-    float4 *st4 = sm4 + 2 * kT * kNP / 4;   // [t][lane]
+    float *sB = reinterpret_cast<float *>(sm4), *sC = sB + kT * kBCS;
+    float4 *st4 = sm4 + 2 * kT * kBCS / 4;   // [t][lane]
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
@@ -369,8 +356,8 @@ template <typename Tin>
 __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParams p)
 {
     extern __shared__ float4 smem_b4[];
-    float *sB = reinterpret_cast<float *>(smem_b4), *sC = sB + kT * kNP;
-    float4 *st4 = smem_b4 + 2 * kT * kNP / 4;                       // [t][lane]
+    float *sB = reinterpret_cast<float *>(smem_b4), *sC = sB + kT * kBCS;
+    float4 *st4 = smem_b4 + 2 * kT * kBCS / 4;                      // [t][lane]
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     float4 *hs = st4 + kT * kBwdLanes + w * kT * kBwdLanes;           // this warp's [t][lane]
     float2 *sums = reinterpret_cast<float2 *>(st4 + kT * kBwdLanes + kQuadWarps * kT * kBwdLanes);
@@ -426,7 +413,7 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
 #pragma unroll 4
             for (int t = 0; t < kT; ++t) {
                 const float4 v = st4[t * kBwdLanes + lane];
-                const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kNP + nw);
+                const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kBCS + nw);
                 const float2 dt2 = dup2(v.x), dtu2 = dup2(v.x * v.y);
                 h[0] = __ffma2_rn(ex2_pair(__fmul2_rn(dt2, A2[0])), h[0],
                                   __fmul2_rn(dtu2, make_float2(b4.x, b4.y)));
@@ -451,8 +438,8 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
             const float dt = v4.x, u = v4.y, gy = v4.z;
             const float2 dt2 = dup2(dt), dtu2 = dup2(dt * u), ndtu2 = dup2(-dt * u);
             const float2 gy2 = dup2(gy);
-            const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kNP + nw);
-            const float4 c4 = *reinterpret_cast<const float4 *>(sC + t * kNP + nw);
+            const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kBCS + nw);
+            const float4 c4 = *reinterpret_cast<const float4 *>(sC + t * kBCS + nw);
             const float4 h4 = hs[t * kBwdLanes + lane];
             const float2 B2[2] = {make_float2(b4.x, b4.y), make_float2(b4.z, b4.w)};
             const float2 C2[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
