@@ -45,6 +45,9 @@ SMALL_2D = [
     small(B=1, D=8, H=33, W=31, K=4, N=16),         # L = 1023, long ragged chunks
     small(B=2, D=9, H=6, W=5, K=2, N=5),            # K = 2, odd N
     small(B=2, D=9, H=6, W=5, K=1, N=1),            # K = 1, N = 1
+    small(B=1, D=40, H=24, W=16, K=4, N=16),        # D = 32 + 8, 384 steps
+    small(B=2, D=8, H=56, W=16, K=4, N=5),          # VMamba-T's image height, odd N
+    small(B=1, D=33, H=32, W=8, K=4, N=16),         # tall and narrow
 ]
 SMALL_1D = [
     small("1d", B=3, D=20, W=197, K=2, N=16),
