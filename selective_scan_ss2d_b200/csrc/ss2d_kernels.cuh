@@ -100,6 +100,23 @@ __device__ __forceinline__ float softplus_f(float z)
     q = fmaf(q, e, 9.999998102e-01f);
     return fmaf(e, q, fmaxf(z, 0.f));
 }
+// softplus_f of two values on the packed f32x2 instructions (each lane
+// rounds as fmaf / a float multiply: the results equal softplus_f's)
+__device__ __forceinline__ float2 softplus2_f(float2 z)
+{
+    const float2 a = __fmul2_rn(make_float2(fabsf(z.x), fabsf(z.y)), make_float2(-kLog2e, -kLog2e));
+    const float2 e = make_float2(mufu_ex2(a.x), mufu_ex2(a.y));
+    auto c2 = [](float v) { return make_float2(v, v); };
+    float2 q = c2(-8.574676204e-03f);
+    q = __ffma2_rn(q, e, c2(4.421419234e-02f));
+    q = __ffma2_rn(q, e, c2(-1.078536792e-01f));
+    q = __ffma2_rn(q, e, c2(1.775702399e-01f));
+    q = __ffma2_rn(q, e, c2(-2.449961172e-01f));
+    q = __ffma2_rn(q, e, c2(3.327617657e-01f));
+    q = __ffma2_rn(q, e, c2(-4.999744938e-01f));
+    q = __ffma2_rn(q, e, c2(9.999998102e-01f));
+    return __ffma2_rn(e, q, make_float2(fmaxf(z.x, 0.f), fmaxf(z.y, 0.f)));
+}
 
 // Walks direction k's scan -> pixel map (see include/ss2d.h) a fixed stride
 // of steps at a time, without divisions.
@@ -443,14 +460,21 @@ __device__ __forceinline__ void chunk_scan_body(const ScanParams &p, int zz)
     auto unpack_store = [&](int buf, int ls) {
         float2 *du = sDU + buf * (kT * 32) + lane;
         if (ls + kT <= l_end) {   // whole sub-chunk inside the chunk
+            // softplus of two steps at a time on the packed pair instructions
             if (xmode == 1) {
 #pragma unroll
-                for (int i = 0; i < kT; ++i)
-                    du[i * 32] = make_float2(softplus_f(pd.get(i) + bias), px.get(kT - 1 - i));
+                for (int i = 0; i < kT; i += 2) {
+                    const float2 sp = softplus2_f(make_float2(pd.get(i) + bias, pd.get(i + 1) + bias));
+                    du[i * 32] = make_float2(sp.x, px.get(kT - 1 - i));
+                    du[(i + 1) * 32] = make_float2(sp.y, px.get(kT - 2 - i));
+                }
             } else {
 #pragma unroll
-                for (int i = 0; i < kT; ++i)
-                    du[i * 32] = make_float2(softplus_f(pd.get(i) + bias), px.get(i));
+                for (int i = 0; i < kT; i += 2) {
+                    const float2 sp = softplus2_f(make_float2(pd.get(i) + bias, pd.get(i + 1) + bias));
+                    du[i * 32] = make_float2(sp.x, px.get(i));
+                    du[(i + 1) * 32] = make_float2(sp.y, px.get(i + 1));
+                }
             }
         } else {
 #pragma unroll
