@@ -437,20 +437,23 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     };
     // steps valid.. of raw delta stage s read -inf (dt = 0: identity steps)
     auto mask_tail = [&](int s, int valid) {
-        if constexpr (FRONT)
-            return;   // no final states here: steps past L are computed and never stored
+        if constexpr (FRONT) {
+            (void)s;   // no final states here: steps past L are computed and never stored
+            (void)valid;
+        } else {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            uint32_t *dw = reinterpret_cast<uint32_t *>(rawD + ((s * CPL + c) * UD) * NT + tid);
-            for (int i = valid; i < kT; ++i) {
-                if constexpr (DPACK2) {
-                    // step i: unit i / 8, word (i % 8) / 2, half i % 2
-                    uint32_t *w = dw + (i >> 3) * NT * 4 + ((i & 7) >> 1);
-                    const uint32_t ninf = neg_inf_word<Tin>();
-                    *w = (i & 1) ? ((*w & 0xffffu) | (ninf & 0xffff0000u))
-                                 : ((*w & 0xffff0000u) | (ninf & 0xffffu));
-                } else {
-                    dw[(i >> 2) * NT * 4 + (i & 3)] = neg_inf_word<Tin>();
+            for (int c = 0; c < CPL; ++c) {
+                uint32_t *dw = reinterpret_cast<uint32_t *>(rawD + ((s * CPL + c) * UD) * NT + tid);
+                for (int i = valid; i < kT; ++i) {
+                    if constexpr (DPACK2) {
+                        // step i: unit i / 8, word (i % 8) / 2, half i % 2
+                        uint32_t *w = dw + (i >> 3) * NT * 4 + ((i & 7) >> 1);
+                        const uint32_t ninf = neg_inf_word<Tin>();
+                        *w = (i & 1) ? ((*w & 0xffffu) | (ninf & 0xffff0000u))
+                                     : ((*w & 0xffff0000u) | (ninf & 0xffffu));
+                    } else {
+                        dw[(i >> 2) * NT * 4 + (i & 3)] = neg_inf_word<Tin>();
+                    }
                 }
             }
         }
@@ -472,10 +475,9 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
             (void)xp;
             (void)dU;
             uint4 dv = make_uint4(0, 0, 0, 0), xv = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int t = 0; t < kT; ++t) {
-                // delta of step t
-                float draw;
+            // raw delta and x of step t (t ascending: the vector registers
+            // dv, xv are refilled at their first step)
+            auto fetch = [&](int t, float &draw, float &u) {
                 if constexpr (FRONT) {
                     draw = wdt[c] * sDT[buf * kT + t];
                 } else if constexpr (DPACK2) {
@@ -488,7 +490,6 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                     draw = raw_value<Tin>(u4c(dv, t & 3), ESZ == 2 ? (dp >> t) & 1u : 0u);
                 }
                 // x of step t
-                float u;
                 if constexpr (XM == 2 || !DPACK2) {
                     // one word per step (column-major, unaligned rows, 4-byte
                     // types); reversed rows of 4-byte types are packed
@@ -510,10 +511,20 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                         xv = xU[(ti >> 3) * NT];
                     u = raw_value<Tin>(u4c(xv, (ti >> 1) & 3), ti & 1);
                 }
-                const float dt = softplus_f(draw + bias[c]);
-                if (MODE == kModeState)
-                    dtsum[c] += dt;
-                sDU[(t * CPL + c) * 32] = make_float2(dt, u);
+            };
+            // softplus of two steps at a time on the packed pair instructions
+#pragma unroll
+            for (int t = 0; t < kT; t += 2) {
+                float d0, u0, d1, u1;
+                fetch(t, d0, u0);
+                fetch(t + 1, d1, u1);
+                const float2 dt = softplus2_f(make_float2(d0 + bias[c], d1 + bias[c]));
+                if (MODE == kModeState) {
+                    dtsum[c] += dt.x;
+                    dtsum[c] += dt.y;
+                }
+                sDU[(t * CPL + c) * 32] = make_float2(dt.x, u0);
+                sDU[((t + 1) * CPL + c) * 32] = make_float2(dt.y, u1);
             }
         }
     };
