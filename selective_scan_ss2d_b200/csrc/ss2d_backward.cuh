@@ -261,12 +261,14 @@ struct BwdRaw4 {
 //   QS: the local adjoint Q = a_0 g_0 with g from zero at the chunk end,
 //       g_t = a_t (dy_t C_t + g_{t+1}); unrolled, Q = sum_t P_t dy_t C_t with
 //       P_t = a_0 a_1 ... a_t, which the walk accumulates forwards.
+// Also returns the chunk's sum of dt in dts (the walk reads every step's dt).
 template <bool HS, bool QS>
 __device__ __forceinline__ void local_walk4(const float4 *st4, const float *sB, const float *sC,
                                             const float2 (&A2)[2], int nw, float2 (&h)[2],
-                                            float2 (&Q)[2])
+                                            float2 (&Q)[2], float &dts)
 {
     const int lane = threadIdx.x & 31;
+    dts = 0.f;
     float2 P[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -277,6 +279,7 @@ __device__ __forceinline__ void local_walk4(const float4 *st4, const float *sB, 
 #pragma unroll 4
     for (int t = 0; t < kT; ++t) {
         const float4 v = st4[t * kBwdLanes + lane];
+        dts += v.x;
         const float2 dt2 = dup2(v.x), dtu2 = dup2(v.x * v.y), gy2 = dup2(v.z);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -324,18 +327,15 @@ __global__ void __launch_bounds__(kBwd4Threads, 4) bwd_local4_kernel(const BwdPa
         __syncthreads();
         if (c + 1 < c1)
             raw.fetch(p, q, (c + 1) * kT);   // in flight during this chunk's work
-        float dts = 0.f;
-#pragma unroll
-        for (int t = 0; t < kT; ++t)
-            dts += st4[t * kBwdLanes + lane].x;
         const bool hs = c < nc1, qs = c > 0 && p.adj_chunks;
         float2 h[2], g[2];
+        float dts = 0.f;   // the chunk's sum of dt (summed in step order by the walk)
         if (hs && qs)
-            local_walk4<true, true>(st4, sB, sC, A2, nw, h, g);
+            local_walk4<true, true>(st4, sB, sC, A2, nw, h, g, dts);
         else if (hs)
-            local_walk4<true, false>(st4, sB, sC, A2, nw, h, g);
+            local_walk4<true, false>(st4, sB, sC, A2, nw, h, g, dts);
         else if (qs)
-            local_walk4<false, true>(st4, sB, sC, A2, nw, h, g);
+            local_walk4<false, true>(st4, sB, sC, A2, nw, h, g, dts);
         if (hs && q.active) {
             *reinterpret_cast<float4 *>(p.hfwd + (q.bkd * nc1 + c) * kNP + nw) =
                 make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
