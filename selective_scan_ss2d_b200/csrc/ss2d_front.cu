@@ -76,13 +76,19 @@ size_t front_op_bytes(const FrontCall &c)
     return up256_(front_wb_bytes(c.K, c.D, c.N)) + up256_(front_ab_bytes(c.B, c.K, c.D, c.L));
 }
 
+// the A blocks within the scratch of front_op_bytes (after the B blocks)
+void *front_ab(void *ops, const FrontCall &c)
+{
+    return static_cast<char *>(ops) + up256_(front_wb_bytes(c.K, c.D, c.N));
+}
+
 // the front kernels for one call (W_x conversion, conv, x_proj); scratch
-// rows of pitch LP, ops of front_op_bytes
+// rows of pitch LP, ops of front_op_bytes; utile: u only as the A blocks
 cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, float *Bs,
-                         float *Cs, void *ops, cudaStream_t st)
+                         float *Cs, void *ops, cudaStream_t st, bool utile)
 {
     void *Wb = ops;
-    void *Ab = static_cast<char *>(ops) + up256_(front_wb_bytes(c.K, c.D, c.N));
+    void *Ab = front_ab(ops, c);
     {
         const int nblk = (c.D + ss2d::kFrontCh - 1) / ss2d::kFrontCh;
         ss2d::front_wprep_kernel<<<(unsigned)(c.K * nblk), 256, 0, st>>>(
@@ -94,6 +100,7 @@ cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, flo
     ss2d::FrontParams fp{};
     fp.Wb = Wb;
     fp.Ab = Ab;
+    fp.utile = utile ? 1 : 0;
     fp.x = c.x;
     fp.conv_w = c.conv_w;
     fp.conv_b = c.conv_b;
@@ -195,11 +202,13 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
 
     const int LP = (L + 7) / 8 * 8;
     const size_t esz = dtype == SS2D_F32 ? 4 : 2;
+    // bf16 input: the x_proj A blocks are u itself (no rows of u)
+    const bool utile = dtype == SS2D_BF16;
     // the lane kernel reads the front's scratch rows
     const int variant = ss2d::variant_index("lane2_wave");
     const ss2d::Plan pl = ss2d::make_plan(variant, B, D, L, K);
     const size_t rows = (size_t)B * K * D;
-    const size_t u_bytes = up256(esz * rows * LP);
+    const size_t u_bytes = utile ? 0 : up256(esz * rows * LP);
     const size_t dt_bytes = up256(sizeof(float) * (size_t)B * K * LP);
     const size_t bc_bytes = up256(sizeof(float) * (size_t)B * K * N * LP);
     const size_t part_bytes = K > 1 ? up256(sizeof(float) * rows * L) : 0;
@@ -213,7 +222,7 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
     if (rc != SS2D_OK)
         return rc;
     char *base = static_cast<char *>(scratch);
-    void *u = base;
+    void *u = utile ? nullptr : static_cast<void *>(base);
     float *dt_raw = reinterpret_cast<float *>(base + u_bytes);
     float *Bs = reinterpret_cast<float *>(base + u_bytes + dt_bytes);
     float *Cs = reinterpret_cast<float *>(base + u_bytes + dt_bytes + bc_bytes);
@@ -222,12 +231,13 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
     if (ev)
         cudaEventRecord(ev[0], st);
     void *Wb = rest + part_bytes + hs_bytes + ds_bytes;
-    e = launch_front(c, LP, u, dt_raw, Bs, Cs, Wb, st);
+    e = launch_front(c, LP, u, dt_raw, Bs, Cs, Wb, st, utile);
     if (ev)
         cudaEventRecord(ev[1], st);
     if (e == cudaSuccess) {
         ss2d::ScanParams p{};
-        p.x = u;
+        p.x = utile ? front_ab(Wb, c) : u;
+        p.utile = utile ? 1 : 0;
         p.delta = nullptr;
         p.A_log = A_log;
         p.Bs = Bs;
@@ -353,7 +363,7 @@ int ss2d_front_project(const void *x, const float *conv_w, const float *conv_b, 
     rc = ss2d::scratch_alloc(&Wb, front_op_bytes(c), st);
     if (rc != SS2D_OK)
         return rc;
-    e = launch_front(c, L, u, dt_raw, Bs, Cs, Wb, st);
+    e = launch_front(c, L, u, dt_raw, Bs, Cs, Wb, st, false);
     const cudaError_t ef = cudaFreeAsync(Wb, st);
     if (e != cudaSuccess) {
         ss2d::record_error("kernel launch", e);

@@ -18,10 +18,12 @@
 //   front_conv_kernel: one CTA of 256 threads per (128-step tile, 64-channel
 //     block, b * K + k); the tile's input steps (3-step halo) are staged in
 //     shared memory with cp.async, then a thread holds a channel pair over 16
-//     steps, convolves, applies SiLU and writes u twice: for the scan, in the
-//     input dtype, (B, K, D, LP) rows; and, rounded to bf16, as the tile's
-//     x_proj A operand, already in the tensor-core operand layout (one 16 KB
-//     block per tile and channel block).
+//     steps, convolves, applies SiLU and writes u rounded to bf16 as the
+//     tile's x_proj A operand block, already in the tensor-core operand
+//     layout (one 16 KB block per tile and channel block).  For bf16 inputs
+//     of the fused call those blocks are the only copy of u: the scan reads
+//     its rows from them (p.utile).  Otherwise it also writes u for the scan,
+//     in the input dtype, as (B, K, D, LP) rows.
 //   front_proj_kernel: one CTA of 128 threads per (128-step tile, k, b).  One
 //     thread streams the tile's A blocks and the matching bf16 blocks of W_x
 //     (the B operand, converted once per call by front_wprep_kernel) into a
@@ -35,12 +37,16 @@
 // Every mbarrier wait gives up after a time limit, records the fault in a
 // device word that ss2d_check_waits() reports, and lets the kernel finish.
 //
-// Operand layout (K-major, no swizzle): core matrices of 8 rows x 16 bytes;
-// element (row r, channel c) of a 64-channel block at byte
+// Operand layouts, no swizzle, core matrices of 8 rows x 16 bytes:
+// A, MN-major (steps contiguous): element (step r, channel c) of a block at
+//     (r / 8) * 1024 + c * 16 + (r % 8) * 2,
+// core matrices 1024 bytes apart along the steps (SBO) and 128 bytes apart
+// along the channels (LBO): each 16-byte run of 8 steps of one channel is one
+// core-matrix row, which the conv kernel stores whole and the scan can read
+// as a piece of its row.  B, K-major: element (row r, channel c) at
 //     (r / 8) * 1024 + (c / 8) * 128 + (r % 8) * 16 + (c % 8) * 2
-// (LBO = 128 between the core matrices of a row group, SBO = 1024 between
-// row groups): the layout both operand blocks have in global memory, so a
-// block is one contiguous copy.
+// (LBO = 128 along the channels, SBO = 1024 along the rows).  Both blocks
+// are contiguous in global memory, so a block is one bulk copy.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -58,6 +64,7 @@ struct FrontParams {
     const float *W_x;       // (K, 1 + 2N, D)
     const void *Wb;         // W_x in bf16, per direction and 64-channel block, in the B layout
     void *Ab;               // u in bf16, per (b, k, tile, 64-channel block), in the A layout
+    int utile;              // 1: Ab is the only copy of u (bf16 inputs of the fused call)
     void *u;                // (B, K, D, LP) u of every direction in its scan order, dtype
     float *dt_raw;          // (B, K, LP)
     float *Bs, *Cs;         // (B, K, N, LP)
@@ -71,8 +78,8 @@ constexpr int kFrontConvThreads = 256;
 constexpr int kFrontProjThreads = 128;
 constexpr int kFrontTile = 128;       // steps per tile (MMA M)
 constexpr int kFrontCh = 64;          // channels per block (4 MMAs of K = 16)
-constexpr int kFrontLBO = 128;
-constexpr int kFrontSBO = 1024;
+constexpr int kFrontLBO = 128;                               // B: channel stride; A: channel stride
+constexpr int kFrontSBO = 1024;                              // B: row stride; A: step stride
 constexpr int kFrontABytes = (kFrontTile / 8) * kFrontSBO;   // one A block (16 KB)
 constexpr int kFrontStages = 2;                              // shared-memory ring
 
@@ -145,7 +152,8 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
     return d;   // base offset 0, layout type 0 (no swizzle)
 }
 // instruction descriptor of kind::f16: bf16 A and B, f32 accumulator,
-// both K-major, M = 128, N = nm
+// M = 128, N = nm, both operands K-major (the caller sets bit 15 for an
+// MN-major A)
 __device__ __forceinline__ uint32_t umma_idesc_bf16(int nm)
 {
     return (1u << 4)                     // accumulator f32
@@ -234,16 +242,18 @@ __device__ __forceinline__ void cp_async_16b_zfill(uint32_t dst, const void *src
 
 constexpr int kFrontRows = kFrontTile + 3;   // input steps of a tile with the 3-step halo
 
-// conv + SiLU of one (128-step tile, 64-channel block, b * K + k): u for the
-// scan and the bf16 A operand block.  grid (tiles, channel blocks, B * K).
+// conv + SiLU of one (128-step tile, 64-channel block, b * K + k): the bf16
+// A operand block and, unless p.utile, u for the scan.  grid (tiles,
+// channel blocks, B * K).
 // The CTA first copies the tile's 131 input steps (3-step halo) of its 64
 // channels into shared memory (cp.async, 16-byte pieces, zeros outside the
 // sequence and past channel D - 1), so that all its loads are in flight at
 // once.  Thread t then owns the channel pair 2 * (t % 32), + 1 over steps
-// 16 * (t / 32) .. + 15 of the tile: it writes per step one 4-byte word of
-// the A operand (two channels in bf16) and per channel the 16 steps of u.
-// Warps whose steps all lie past the end of the sequence do nothing (the A
-// rows of those steps only feed accumulator rows that are never stored).
+// 16 * (t / 32) .. + 15 of the tile: it writes per channel its 16 steps as
+// two 16-byte A rows (and as u row segments).  Warps whose steps all lie
+// past the end of the sequence do nothing (the A rows of those steps only
+// feed accumulator rows that are never stored, and the scan never reads
+// them).
 template <typename Tin>
 __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const FrontParams p)
 {
@@ -326,7 +336,7 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
     xrow(m0 + 2, win[2]);
     unsigned char *ab = static_cast<unsigned char *>(p.Ab) +
                         (((size_t)bk * gridDim.x + tile) * gridDim.y + cb) * kFrontABytes +
-                        (c0 >> 3) * kFrontLBO + (c0 & 7) * 2;
+                        (m0 >> 3) * kFrontSBO + c0 * 16;   // channel c0, steps m0..m0+7
     // per step: the A operand word (the pair in bf16, one packed conversion);
     // 2-byte inputs: the pair in the input dtype, whose halves are u's values
     // (for bf16 the A word itself); float inputs: the float values
@@ -345,8 +355,6 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
         }
         const __nv_bfloat162 a2 = __floats2bfloat162_rn(v[0], v[1]);
         aw[i] = *reinterpret_cast<const uint32_t *>(&a2);
-        const int mt = m0 + i;
-        *reinterpret_cast<uint32_t *>(ab + (mt >> 3) * kFrontSBO + (mt & 7) * 16) = aw[i];
         if constexpr (std::is_same_v<Tin, __half>) {
             const __half2 h2 = __floats2half2_rn(v[0], v[1]);
             hw[i] = *reinterpret_cast<const uint32_t *>(&h2);
@@ -357,6 +365,23 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
             uu[1][i] = v[1];
         }
     }
+    // the A rows: per channel j and 8-step group q, the 8 bf16 values, the
+    // low (j = 0) or high (j = 1) halves of the pair words
+#pragma unroll
+    for (int j = 0; j < CP; ++j) {
+        const uint32_t sel = j == 0 ? 0x5410u : 0x7632u;
+#pragma unroll
+        for (int q = 0; q < SG / 8; ++q) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                w4[e] = __byte_perm(aw[q * 8 + 2 * e], aw[q * 8 + 2 * e + 1], sel);
+            *reinterpret_cast<uint4 *>(ab + q * kFrontSBO + j * 16) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+    }
+    if (p.utile)
+        return;   // the A rows are u
     // u for the scan, in the input dtype: 16-byte stores of 8 (2-byte) or 4
     // (float) steps; every store starts before L (LP is a multiple of 8)
     Tin *ub = static_cast<Tin *>(p.u) + (size_t)bk * D * LP;
@@ -449,12 +474,15 @@ __global__ void __launch_bounds__(kFrontProjThreads) front_proj_kernel(const Fro
 
     bool ok = true;
     if (tid == 0) {
-        const uint32_t idesc = umma_idesc_bf16(NM);
+        const uint32_t idesc = umma_idesc_bf16(NM) | (1u << 15);   // A MN-major
+        // the 8-step groups of A that hold steps before L (the last tile's
+        // later rows only feed accumulator rows that are never stored)
+        const uint32_t a_bytes = (uint32_t)min(kFrontTile / 8, (L - l0 + 7) / 8) * kFrontSBO;
         auto load = [&](int cb) {   // block cb into stage cb % S
             const int st = cb % kFrontStages;
             const uint32_t full = bars + 8 * st, dA = sbase + st * stage_bytes;
-            mbar_expect_tx(full, stage_bytes);
-            bulk_copy(dA, ag + (size_t)cb * kFrontABytes, kFrontABytes, full);
+            mbar_expect_tx(full, a_bytes + bbytes);
+            bulk_copy(dA, ag + (size_t)cb * kFrontABytes, a_bytes, full);
             bulk_copy(dA + kFrontABytes, wg + (size_t)cb * bbytes, bbytes, full);
         };
         for (int cb = 0; cb < kFrontStages && cb < nblk; ++cb)
@@ -468,7 +496,7 @@ __global__ void __launch_bounds__(kFrontProjThreads) front_proj_kernel(const Fro
                 const uint32_t aS = sbase + st * stage_bytes, bS = aS + kFrontABytes;
 #pragma unroll
                 for (int kk = 0; kk < kFrontCh / 16; ++kk)
-                    umma_bf16(tmem, umma_desc(aS + kk * 2 * kFrontLBO, kFrontLBO, kFrontSBO),
+                    umma_bf16(tmem, umma_desc(aS + kk * 16 * 16, kFrontLBO, kFrontSBO),
                               umma_desc(bS + kk * 2 * kFrontLBO, kFrontLBO, kFrontSBO), idesc,
                               (cb > 0 || kk > 0) ? 1u : 0u);
             }

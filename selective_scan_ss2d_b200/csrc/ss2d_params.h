@@ -38,6 +38,10 @@ struct ScanParams {
     // fused front: u per direction (B,K,D,LP) in scan order in x, no delta;
     // delta = w_dt[k*D+d] * dt_raw[b,k,l]; Bs, Cs float32 (B,K,N,LP)
     int front;
+    // fused front with bf16 input: u only as the x_proj A blocks, x of
+    // ((b*K+k)*tiles + l/128)*blocks + d/64 blocks of 16 KB, element (l, d)
+    // at (l%128/8)*1024 + (d%64)*16 + (l%8)*2 bytes (blocks of 64 channels)
+    int utile;
     const float *dt_raw;      // (B,K,LP)
     const float *w_dt;        // (K*D)
 };

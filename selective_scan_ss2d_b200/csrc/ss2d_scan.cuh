@@ -196,8 +196,10 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     float2 A2[CPL][8];      // A[n] * log2(e) for states (2j, 2j+1)
     float dsk[CPL], bias[CPL], wdt[CPL];
     const Tin *drow[CPL], *xrow[CPL];
+    size_t utb[CPL];        // p.utile: byte offset of the channel's rows in the A blocks
     float2 h2[CPL][8];
     float dtsum[CPL];
+    const int ublk = (D + 63) / 64, utiles = (L + 127) / 128;   // A blocks: channel blocks, tiles
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
         dch[c] = tile * CH + c * NT + tid;
@@ -217,6 +219,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
         drow[c] = FRONT ? nullptr : static_cast<const Tin *>(p.delta) + (row_bk + dc) * LP;
         // x rows: the caller's (b, d) map, or the front's u row of (b, k, d)
         xrow[c] = static_cast<const Tin *>(p.x) + (FRONT ? (row_bk + dc) : ((size_t)b * D + dc)) * LP;
+        // u as the x_proj A blocks: block (b * K + k, tile 0, dc / 64), row dc % 64
+        utb[c] = (((size_t)b * K + k) * utiles * ublk + (dc >> 6)) * 16384u + (size_t)(dc & 63) * 16u;
         dtsum[c] = 0.f;
     }
     const size_t bc_row0 = ((size_t)b * K + k) * p.NS + p.n0;   // row of this group's state 0
@@ -263,6 +267,19 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                           row + max(min(e0 + u * PE, lastp), 0));
         }
     };
+    // the same 16 elements from the A blocks (p.utile, 2-byte u): 8 steps of
+    // a channel are one 16-byte row, steps 128 apart are ublk blocks apart;
+    // a row past the sequence end reads the last one inside
+    auto copy_tile = [&](uint32_t dst, int c, int e0) {
+        const unsigned char *base = static_cast<const unsigned char *>(p.x) + utb[c];
+        const int lastu = ((L - 1) >> 3) << 3;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = max(min(e0 + u * 8, lastu), 0);
+            cp_async16(dst + u * NT * 16,
+                       base + ((size_t)(e >> 7) * ublk * 16384u + ((e >> 3) & 15) * 1024u));
+        }
+    };
     auto set_par = [&](uint32_t (&par)[2][CPL], int s, int c, uint32_t m) {
         if (s)
             par[1][c] = m;
@@ -290,7 +307,12 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
             }
             // x of the row-major directions
             if (xmode == 0) {
-                if constexpr (ALIGNED) {
+                if constexpr (FRONT && ESZ == 2) {
+                    if (p.utile)
+                        copy_tile(dX, c, ls);
+                    else
+                        copy_packed(dX, xrow[c], ls);
+                } else if constexpr (ALIGNED) {
                     copy_packed(dX, xrow[c], ls);
                 } else {
                     uint32_t m = 0;

@@ -58,6 +58,8 @@ SHAPES = [  # B, L, D, N, K
     (1, 300, 40, 8, 2),      # d_state 8, fewer channels than a block
     (2, 64, 70, 5, 1),       # odd N, a partial tile
     (1, 1100, 64, 16, 2),    # long enough to be chunked
+    (2, 150, 130, 24, 2),    # two state groups, a 2-channel last tile
+    (2, 199, 70, 16, 2),     # a last tile whose rows are not a whole number of float4
 ]
 
 
