@@ -106,6 +106,10 @@ typedef enum {
  * never interact, so more than 16 run as groups of 16 states one after the
  * other, each adding its C.h terms to the output (the skip term once); the
  * pages use N = 16 and mention d_state 8 ("VMamba架构解析", section 5).
+ * K = 2 with N <= 16: the scan pass does the cross_merge itself -- y is
+ * zeroed on `stream`, then both directions add their outputs into it with
+ * float atomic adds; two terms give the same bits in either order, so y is
+ * exactly y_0 + y_1 as the merge kernel would sum it.
  * `stream` is a cudaStream_t (NULL = the legacy default stream). */
 int ss2d_forward(const void *x, const void *delta, const float *A_log,
                  const void *Bs, const void *Cs, const float *Dskip,
@@ -226,7 +230,8 @@ int selective_scan_fwd_ex(const void *u, const void *delta, const float *A_log,
  * executed: steps per chunk, chunks per sequence, and kernel launches per
  * call (1 scan pass, or state pass + carry + scan pass when the sequence is
  * chunked, once per group of 16 states; plus one cross_merge launch when
- * K > 1).  Host only. */
+ * K = 4, or K = 2 with N > 16; K = 2 with N <= 16 merges in the scan pass
+ * after a memset of y, which is not counted).  Host only. */
 int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
               int *chunk_len, int *num_chunks, int *launches);
 
@@ -235,7 +240,9 @@ int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
  * events on `stream` around each of its kernel launches, synchronises the
  * stream and writes the device time of each launch in milliseconds to
  * launch_ms[0..3] in the order [chunk state pass, carry, scan pass,
- * cross_merge]; a launch the call does not make gets -1.  Blocking. */
+ * cross_merge]; a launch the call does not make gets -1 (K = 2 with
+ * N <= 16: cross_merge is the empty interval after the scan pass, which
+ * merges itself).  Blocking. */
 int ss2d_forward_timed(const void *x, const void *delta, const float *A_log,
                        const void *Bs, const void *Cs, const float *Dskip,
                        const float *delta_bias, float *y,
@@ -262,7 +269,8 @@ int ss2d_pick_variant(int two_d, int B, int D, int H, int W, int N, int K);
  * allocator has reserved (nearly) all device memory, latency-bound loops in
  * which a growing pool would call into the driver, processes held to a fixed
  * device footprint.  Its scratch (the per-direction rows and chunk states
- * ss2d_forward takes from its pool: 4*B*K*D*H*W bytes when K > 1, plus
+ * ss2d_forward takes from its pool: 4*B*K*D*H*W bytes when K = 4 or
+ * K = 2 with N > 16 (K = 2 with N <= 16 adds into y instead), plus
  * 68*B*K*D*(chunks-1) bytes when ss2d_plan reports chunks > 1, each rounded
  * up to 256) lives in one statically sized device buffer of
  * SS2D_NOALLOC_SCRATCH_BYTES per device, part of the library's device image.
@@ -331,7 +339,9 @@ int selective_scan_fwd_front(const void *x, const float *conv_w, const float *co
 /* selective_scan_fwd_front that also synchronises `stream` and returns the
  * device time of its launches in launch_ms[0..2] (milliseconds, CUDA events
  * on `stream`): the front kernel, the scan passes, cross_merge (-1 when not
- * launched, K = 1).  For benchmarks. */
+ * launched, K = 1; K = 2 with N <= 16 merges inside the scan pass, after a
+ * memset of y that the second figure includes, and the third is the empty
+ * interval after it).  For benchmarks. */
 int selective_scan_fwd_front_timed(const void *x, const float *conv_w, const float *conv_b,
                                    const float *W_x, const float *w_dt, const float *A_log,
                                    const float *Dskip, const float *delta_bias, float *y,

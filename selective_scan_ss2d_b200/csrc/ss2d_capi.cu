@@ -176,7 +176,9 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 //   K = 1: the output pass writes y (scan order of direction 0 = pixel order);
 //   K > 1: the output pass writes per-direction scan-order rows to scratch
 //   and the merge kernel sums them into y in fixed order (directions = true:
-//   copies them to y as per-direction pixel-order outputs instead).
+//   copies them to y as per-direction pixel-order outputs instead);
+//   K = 2 without a gate, at most 16 states: y is zeroed and both
+//   directions add into it in the output pass (no rows, no merge kernel).
 // Scratch comes from the pool on the stream and goes back to it on the stream.
 int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
                cudaEvent_t *ev = nullptr)
@@ -187,7 +189,9 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     const size_t in_esz = pr.dtype == SS2D_F32 ? 4 : 2;   // bytes per stored input value
     const long long L = p.L;
     const ss2d::Plan pl = ss2d::make_plan(variant, pr.B, pr.D, (int)L, pr.K);
-    const bool need_part = pr.K > 1 || pr.z;   // gated calls always merge (the gate runs there)
+    // two directions, one state group, no gate: the output pass adds both into y
+    const bool add_merge = pr.K == 2 && !pr.z && !directions && pr.N <= ss2d::kNP;
+    const bool need_part = (pr.K > 1 || pr.z) && !add_merge;   // gated calls merge (the gate runs there)
     const size_t rows = (size_t)pr.B * pr.K * pr.D;
     const size_t part_bytes = need_part ? align256(sizeof(float) * rows * L) : 0;
     const size_t hs_bytes = pl.NC > 1 ? align256(sizeof(float) * rows * (pl.NC - 1) * ss2d::kNP) : 0;
@@ -212,7 +216,14 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     }
     p.hstate = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes) : nullptr;
     p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes + hs_bytes) : nullptr;
-    cudaError_t e = ss2d::launch_scan(pl, pr.dtype, p, st, ev);
+    p.ymerge = add_merge ? pr.y : nullptr;
+    cudaError_t e = cudaSuccess;
+    if (add_merge)
+        e = cudaMemsetAsync(pr.y, 0, sizeof(float) * (size_t)pr.B * pr.D * L, st);
+    if (e == cudaSuccess)
+        e = ss2d::launch_scan(pl, pr.dtype, p, st, ev);
+    if (e == cudaSuccess && add_merge && ev)
+        cudaEventRecord(ev[4], st);   // no merge launch
     if (e == cudaSuccess && need_part) {
         e = ss2d::launch_merge(p.out, pr.y, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d,
                                directions ? 0 : 1, st, pr.z, pr.dtype);
@@ -586,7 +597,8 @@ int ss2d_plan(int two_d, int B, int D, int H, int W, int N, int K, int variant,
         *num_chunks = pl.NC;
     if (launches)
         *launches = pl.launches + (pl.NC > 2 ? 3 : pl.NC > 1 ? 2 : 1) *
-                                      ((N + ss2d::kNP - 1) / ss2d::kNP - 1);
+                                      ((N + ss2d::kNP - 1) / ss2d::kNP - 1) -
+                    (K == 2 && N <= ss2d::kNP ? 1 : 0);   // merged in the scan pass
     return SS2D_OK;
 }
 

@@ -211,7 +211,10 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
     const size_t u_bytes = utile ? 0 : up256(esz * rows * LP);
     const size_t dt_bytes = up256(sizeof(float) * (size_t)B * K * LP);
     const size_t bc_bytes = up256(sizeof(float) * (size_t)B * K * N * LP);
-    const size_t part_bytes = K > 1 ? up256(sizeof(float) * rows * L) : 0;
+    // two directions, one state group: both add into y (zeroed first)
+    // instead of writing rows for a merge kernel
+    const bool pair_merge = K == 2 && N <= ss2d::kNP;
+    const size_t part_bytes = K > 1 && !pair_merge ? up256(sizeof(float) * rows * L) : 0;
     const size_t hs_bytes = pl.NC > 1 ? up256(sizeof(float) * rows * (pl.NC - 1) * ss2d::kNP) : 0;
     const size_t ds_bytes = pl.NC > 1 ? up256(sizeof(float) * rows * (pl.NC - 1)) : 0;
     const size_t wb_bytes = up256(front_op_bytes(c));
@@ -257,15 +260,19 @@ int front_forward(const FrontCall &c, float *y, cudaStream_t st, cudaEvent_t *ev
         p.front = 1;
         p.dt_raw = dt_raw;
         p.w_dt = w_dt;
-        p.out = K > 1 ? reinterpret_cast<float *>(rest) : y;
+        p.out = K > 1 && !pair_merge ? reinterpret_cast<float *>(rest) : y;
+        p.ymerge = pair_merge ? y : nullptr;
         p.hstate = pl.NC > 1 ? reinterpret_cast<float *>(rest + part_bytes) : nullptr;
         p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(rest + part_bytes + hs_bytes) : nullptr;
         p.vec = 16;   // scratch rows of pitch LP (a multiple of 8) start on 16-byte boundaries
         p.ovec = ((((uintptr_t)p.out) & 15) == 0 && ((size_t)L * 4) % 16 == 0) ? 1 : 0;
-        e = ss2d::launch_scan(pl, dtype, p, st, nullptr);
+        if (pair_merge)
+            e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)B * D * L, st);
+        if (e == cudaSuccess)
+            e = ss2d::launch_scan(pl, dtype, p, st, nullptr);
         if (ev)
             cudaEventRecord(ev[2], st);
-        if (e == cudaSuccess && K > 1)
+        if (e == cudaSuccess && K > 1 && !pair_merge)
             e = ss2d::launch_merge(p.out, y, B, D, 1, L, K, 0, 1, st);
         if (ev)
             cudaEventRecord(ev[3], st);

@@ -343,6 +343,7 @@ __device__ __forceinline__ void chunk_scan_body(const ScanParams &p, int zz)
         A2[j].y = (n1 < N) ? -expf(__ldg(al + n1)) * kLog2e : 0.f;
     }
     const bool accum = p.accum != 0;   // a later state group: add to out, no skip term
+    const bool ymode = MODE == kModeOutput && p.ymerge != nullptr;   // both directions add into y
     const float dsk = accum ? 0.f : __ldg(p.Dskip + kd);
     const float bias = __ldg(p.delta_bias + kd);
 
@@ -580,7 +581,7 @@ __device__ __forceinline__ void chunk_scan_body(const ScanParams &p, int zz)
             // order, except direction 1 of a multi-direction call (the reversed
             // row-major order), which is stored flipped, in pixel order
             const bool flip = k == 1 && K > 1;
-            float *rowp = p.out + (row_bk + d) * L;
+            float *rowp = ymode ? p.ymerge + ((size_t)b * D + d) * L : p.out + (row_bk + d) * L;
             if (ovec && l0 + kT <= l_end) {
                 float4 *orow = reinterpret_cast<float4 *>(rowp + (flip ? L - kT - l0 : l0));
 #pragma unroll
@@ -593,6 +594,10 @@ __device__ __forceinline__ void chunk_scan_body(const ScanParams &p, int zz)
                                                   sY[(4 * q + 1) * 33 + lane],
                                                   sY[(4 * q + 2) * 33 + lane],
                                                   sY[(4 * q + 3) * 33 + lane]);
+                    if (ymode) {
+                        atomicAdd(orow + q, v);
+                        continue;
+                    }
                     if (accum) {
                         const float4 o = orow[q];
                         v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
@@ -604,7 +609,10 @@ __device__ __forceinline__ void chunk_scan_body(const ScanParams &p, int zz)
                 for (int t = 0; t < kT; ++t)
                     if (l0 + t < l_end) {
                         float *o = rowp + (flip ? L - 1 - l0 - t : l0 + t);
-                        *o = accum ? *o + sY[t * 33 + lane] : sY[t * 33 + lane];
+                        if (ymode)
+                            atomicAdd(o, sY[t * 33 + lane]);
+                        else
+                            *o = accum ? *o + sY[t * 33 + lane] : sY[t * 33 + lane];
                     }
             }
         }

@@ -162,6 +162,8 @@ cudaError_t launch_scan(const Plan &plan, int dtype, ScanParams &p, cudaStream_t
 {
     if (p.front && plan.layout != 2)
         return cudaErrorInvalidValue;   // only the lane kernel reads the front's rows
+    if (p.ymerge && (p.K != 2 || p.N > kNP))
+        return cudaErrorInvalidValue;   // the merge by adds: two directions, one state group
     p.LC = plan.LC;
     p.NC = plan.NC;
     // more than 16 states: the passes once per group of at most 16 states, in

@@ -92,7 +92,9 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     const long long L = (long long)H * W;
     const ss2d::Plan pl = ss2d::make_plan(variant, B, D, (int)L, K);
     const size_t rows = (size_t)B * K * D;
-    const size_t part_bytes = K > 1 ? round256(sizeof(float) * rows * (size_t)L) : 0;
+    // K = 2, one state group: both directions add into y (zeroed first)
+    const bool add_merge = K == 2 && N <= ss2d::kNP;
+    const size_t part_bytes = K > 1 && !add_merge ? round256(sizeof(float) * rows * (size_t)L) : 0;
     const size_t hs_bytes =
         pl.NC > 1 ? round256(sizeof(float) * rows * (size_t)(pl.NC - 1) * ss2d::kNP) : 0;
     const size_t ds_bytes = pl.NC > 1 ? round256(sizeof(float) * rows * (size_t)(pl.NC - 1)) : 0;
@@ -139,7 +141,8 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
     p.NS = N;
     p.K = K;
     p.two_d = 1;
-    p.out = K > 1 ? reinterpret_cast<float *>(base) : y;
+    p.out = K > 1 && !add_merge ? reinterpret_cast<float *>(base) : y;
+    p.ymerge = add_merge ? y : nullptr;
     p.hstate = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes) : nullptr;
     p.dtsum = pl.NC > 1 ? reinterpret_cast<float *>(base + part_bytes + hs_bytes) : nullptr;
     {
@@ -151,8 +154,11 @@ extern "C" int ss2d_forward_noalloc(const void *x, const void *delta, const floa
         p.ovec = (ptr_ok && ((size_t)L * 4) % 16 == 0) ? 1 : 0;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    e = ss2d::launch_scan(pl, dtype, p, st, nullptr);
-    if (e == cudaSuccess && K > 1)
+    if (add_merge)
+        e = cudaMemsetAsync(y, 0, sizeof(float) * (size_t)B * D * L, st);
+    if (e == cudaSuccess)
+        e = ss2d::launch_scan(pl, dtype, p, st, nullptr);
+    if (e == cudaSuccess && K > 1 && !add_merge)
         e = ss2d::launch_merge(p.out, y, B, D, H, W, K, 1, 1, st);
     if (e != cudaSuccess) {
         ss2d::record_error("kernel launch", e);

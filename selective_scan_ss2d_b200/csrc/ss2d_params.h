@@ -44,6 +44,12 @@ struct ScanParams {
     int utile;
     const float *dt_raw;      // (B,K,LP)
     const float *w_dt;        // (K*D)
+    // K = 2 (no column-major direction), one state group: both directions
+    // add their outputs into ymerge (B,D,L), zero on entry, with float
+    // atomic adds; the two terms meet in either order and a + b = b + a
+    // exactly, so ymerge ends as y_0 + y_1 bit for bit, cross_merge's sum.
+    // Null: the output pass writes out and a merge kernel sums.
+    float *ymerge;
 };
 
 }  // namespace ss2d

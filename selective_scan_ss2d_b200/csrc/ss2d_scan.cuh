@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
     const int l_end = min(l_begin + p.LC, L);
     const int nsub = (l_end - l_begin + kT - 1) / kT;
     const bool accum = p.accum != 0;   // a later state group: add to out, no skip term
+    const bool ymode = MODE == kModeOutput && p.ymerge != nullptr;   // both directions add into y
     const size_t row_bk = ((size_t)b * K + k) * D;   // row index of (b, k, d = 0)
     const size_t LP = (size_t)p.LP;                  // row pitch of the input rows
 
@@ -662,7 +663,8 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                 // scan order, except direction 1 of a multi-direction call (the
                 // reversed row-major order), which is stored flipped, in pixel order
                 const bool flip = k == 1 && K > 1;
-                float *rowp = p.out + (row_bk + dch[c]) * (size_t)L;
+                float *rowp = ymode ? p.ymerge + ((size_t)b * D + dch[c]) * (size_t)L
+                                    : p.out + (row_bk + dch[c]) * (size_t)L;
                 const float2 *yc = sDU + c * 32;   // step t at yc[t * CPL * 32]
                 if (p.ovec && l0 + kT <= l_end) {
                     float4 *orow = reinterpret_cast<float4 *>(rowp + (flip ? L - kT - l0 : l0));
@@ -676,6 +678,10 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                                                       yc[(4 * q + 1) * CPL * 32].x,
                                                       yc[(4 * q + 2) * CPL * 32].x,
                                                       yc[(4 * q + 3) * CPL * 32].x);
+                        if (ymode) {
+                            atomicAdd(orow + q, v);
+                            continue;
+                        }
                         if (accum) {
                             const float4 o = orow[q];
                             v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
@@ -688,7 +694,10 @@ __global__ void __launch_bounds__(32 * WC, MINB) lane_scan_kernel(const ScanPara
                         if (l0 + t < l_end) {
                             float *o = rowp + (flip ? L - 1 - l0 - t : l0 + t);
                             const float y = yc[t * CPL * 32].x;
-                            *o = accum ? *o + y : y;
+                            if (ymode)
+                                atomicAdd(o, y);
+                            else
+                                *o = accum ? *o + y : y;
                         }
                 }
             }

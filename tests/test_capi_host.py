@@ -128,7 +128,9 @@ def test_plans_for_the_workloads(lib):
         assert pl["num_chunks"] == -(-cfg.L // pl["chunk_len"])
         nc = pl["num_chunks"]
         # state pass, carry (not needed with two chunks), output pass; merge
-        want = (3 if nc > 2 else 2 if nc > 1 else 1) + (1 if cfg.K > 1 else 0)
+        # (K = 2 with at most 16 states merges in the output pass)
+        merge = 1 if cfg.K == 4 or (cfg.K == 2 and cfg.N > 16) else 0
+        want = (3 if nc > 2 else 2 if nc > 1 else 1) + merge
         assert pl["launches"] == want
     # long sequences with few channels are chunked, short ones are not
     t = wl.CONFIGS["vmamba_t_stage1"]
@@ -198,6 +200,9 @@ def test_plan_counts_launches_per_state_group(lib):
     assert one["num_chunks"] == three["num_chunks"] > 1
     # three groups of states: three (state pass, carry, output pass), one merge
     assert one["launches"] == 3 + 1 and three["launches"] == 3 * 3 + 1
+    # K = 2: merged in the output pass with one state group, a merge launch with more
+    assert binding.ss2d_plan(False, 128, 768, 1, 197, 16, 2)["launches"] == 1
+    assert binding.ss2d_plan(False, 128, 768, 1, 197, 24, 2)["launches"] == 2 + 1
 
 
 def test_final_state_binding_validates_tensors(lib):

@@ -26,7 +26,7 @@ def scratch_bytes(B, D, H, W, N, K):
     """Scratch the call needs, as the header states it."""
     nc = binding.ss2d_plan(True, B, D, H, W, N, K)["num_chunks"]
     r = lambda v: (v + 255) // 256 * 256
-    part = r(4 * B * K * D * H * W) if K > 1 else 0
+    part = r(4 * B * K * D * H * W) if (K == 4 or (K == 2 and N > 16)) else 0
     states = r(64 * B * K * D * (nc - 1)) + r(4 * B * K * D * (nc - 1)) if nc > 1 else 0
     return part + states
 
