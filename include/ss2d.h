@@ -195,6 +195,9 @@ int selective_scan_fwd_final_state(const void *u, const void *delta, const float
  * Asynchronous on `stream`; scratch comes from the library's stream-ordered
  * pool.  The parameter gradients are summed over the batch and the
  * sequence in a fixed order, so repeated calls give identical results.
+ * dx sums the directions' du as the forward's cross_merge sums y (K = 2
+ * with N <= 16: dx zeroed, then both directions added into it with float
+ * atomic adds, the same bits in either order).
  * With B, H*W or L zero the parameter gradients are set to zero. */
 int ss2d_backward(const void *x, const void *delta, const float *A_log,
                   const void *Bs, const void *Cs, const float *Dskip,

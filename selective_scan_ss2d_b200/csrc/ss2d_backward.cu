@@ -86,6 +86,8 @@ cudaError_t launch_backward(const BwdParams &p, int dtype, cudaStream_t st)
     // more than 16 states: the passes once per group of at most 16, in order
     // on the stream, later groups adding to the first group's rows
     const int ns = p.NS;
+    if (p.dxmerge && (p.K != 2 || ns > kNP))
+        return cudaErrorInvalidValue;   // the dx merge by adds: two directions, one group
     cudaError_t e = cudaSuccess;
     for (int n0 = 0; n0 < ns && e == cudaSuccess; n0 += kNP) {
         BwdParams q = p;

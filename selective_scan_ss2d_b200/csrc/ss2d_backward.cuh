@@ -377,7 +377,8 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
     const float Dk = accum ? 0.f : __ldg(p.Dskip + kd);
     const int L = p.L, nc1 = p.NC - 1;
     const bool flip = p.flip1 && q.k == 1;
-    float *durow = p.du + q.bkd * L;
+    const bool xmerge = p.dxmerge != nullptr;   // both directions add into dx
+    float *durow = xmerge ? p.dxmerge + ((size_t)q.b * p.D + q.d) * L : p.du + q.bkd * L;
     float *ddrow = p.ddelta + q.bkd * L;
     const bool vec_rows = (L & 3) == 0;
     // the reduced row this lane writes (lanes 0..7 of each warp: j = lane)
@@ -496,12 +497,19 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
                 float4 b = flip ? make_float4(duv[3], duv[2], duv[1], duv[0])
                                 : make_float4(duv[0], duv[1], duv[2], duv[3]);
                 if (accum) {
-                    const float4 ea = *dd4, eb = *du4;
+                    const float4 ea = *dd4;
                     a = make_float4(ea.x + a.x, ea.y + a.y, ea.z + a.z, ea.w + a.w);
-                    b = make_float4(eb.x + b.x, eb.y + b.y, eb.z + b.z, eb.w + b.w);
                 }
                 *dd4 = a;
-                *du4 = b;
+                if (xmerge) {
+                    atomicAdd(du4, b);
+                } else {
+                    if (accum) {
+                        const float4 eb = *du4;
+                        b = make_float4(eb.x + b.x, eb.y + b.y, eb.z + b.z, eb.w + b.w);
+                    }
+                    *du4 = b;
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -510,7 +518,10 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
                         const int l = s + t;
                         float *o = durow + (flip ? L - 1 - l : l);
                         ddrow[l] = accum ? ddrow[l] + ddv[i] : ddv[i];
-                        *o = accum ? *o + duv[i] : duv[i];
+                        if (xmerge)
+                            atomicAdd(o, duv[i]);
+                        else
+                            *o = accum ? *o + duv[i] : duv[i];
                     }
                 }
             }

@@ -29,6 +29,11 @@ struct BwdParams {
     int NS;            // states per row of A_log, Bs, Cs (the call's N)
     int accum;         // 1: add ddelta, du to the rows (no skip term, no dDskip)
     int adj_chunks;    // 1: local adjoints and their carry are needed (CGN > 1)
+    // K = 2, one state group: both directions add their du into dxmerge
+    // (B,D,H,W) / (B,D,L), zero on entry, with float atomic adds (two terms:
+    // the same bits in either order, the merge kernel's sum); du unused.
+    // Null: du rows and a merge kernel.
+    float *dxmerge;
 };
 
 constexpr int kBwdLanes = 32;

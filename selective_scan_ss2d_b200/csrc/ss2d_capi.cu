@@ -399,7 +399,9 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     const size_t nc1 = (size_t)sh.NC - 1;
     const size_t hs_bytes = align256(sizeof(float) * rows * nc1 * ss2d::kNP);
     const size_t ds_bytes = align256(sizeof(float) * rows * nc1);
-    const size_t du_bytes = pr.K > 1 ? align256(sizeof(float) * rows * L) : 0;
+    // two directions, one state group: both add their du into dx (zeroed first)
+    const bool add_merge = pr.K == 2 && pr.N <= ss2d::kNP;
+    const size_t du_bytes = pr.K > 1 && !add_merge ? align256(sizeof(float) * rows * L) : 0;
     const size_t bc_bytes =
         align256(sizeof(float) * pr.B * pr.K * (size_t)sh.G * 2 * pr.N * L);
     const size_t pr_bytes = align256(sizeof(float) * rows * sh.CGN * (pr.N + 2));
@@ -428,7 +430,8 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     p.hadj = take(hs_bytes);
     p.dtf = take(ds_bytes);
     p.dta = take(ds_bytes);
-    p.du = pr.K > 1 ? take(du_bytes) : gr.dx;
+    p.du = pr.K > 1 && !add_merge ? take(du_bytes) : gr.dx;
+    p.dxmerge = add_merge ? gr.dx : nullptr;
     p.bc_part = take(bc_bytes);
     p.prm_part = take(pr_bytes);
     p.ddelta = gr.ddelta;
@@ -447,8 +450,12 @@ int backward(const Problem &pr, const Grads &gr, void *stream)
     p.flip1 = pr.K > 1 ? 1 : 0;
     p.NS = pr.N;
     p.adj_chunks = sh.CGN > 1 ? 1 : 0;
-    e = ss2d::launch_backward(p, pr.dtype, st);
-    if (e == cudaSuccess && pr.K > 1)
+    e = cudaSuccess;
+    if (add_merge)
+        e = cudaMemsetAsync(gr.dx, 0, sizeof(float) * (size_t)pr.B * pr.D * L, st);
+    if (e == cudaSuccess)
+        e = ss2d::launch_backward(p, pr.dtype, st);
+    if (e == cudaSuccess && pr.K > 1 && !add_merge)
         e = ss2d::launch_merge(p.du, gr.dx, pr.B, pr.D, pr.H, pr.W, pr.K, pr.two_d, 1, st);
     if (e == cudaSuccess)
         e = ss2d::launch_backward_reduce(p, gr.dBs, gr.dCs, gr.dA_log, gr.dDskip,

@@ -128,6 +128,17 @@ def test_backward_deterministic():
         assert np.array_equal(a[n], b[n]), n
 
 
+def test_backward_deterministic_two_directions():
+    # K = 2: both directions add their du into dx (atomic adds of two terms)
+    cfg = small("1d", B=2, D=70, W=203, K=2, dtype=wl.BF16)
+    inp = wl.make_inputs(cfg, seed=4)
+    dy = wl.make_cotangent(cfg, seed=4)
+    t = _gpu.tensors(inp)
+    a, b = gpu_backward(inp, dy, t), gpu_backward(inp, dy, t)
+    for n in GRADS:
+        assert np.array_equal(a[n], b[n]), n
+
+
 def test_zero_cotangent_gives_zero_gradients():
     cfg = small(B=2, D=12, H=9, W=9)
     inp = wl.make_inputs(cfg, seed=1)
