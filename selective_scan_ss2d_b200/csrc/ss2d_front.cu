@@ -48,8 +48,12 @@ int front_validate(const FrontCall &c)
         return SS2D_ERR_K;
     if (c.N < 1 || c.N > ss2d::kMaxN)
         return SS2D_ERR_N;
+    // the conv kernel's CTAs (tiles x channel blocks x B x K) fit one grid dimension
+    const long long conv_ctas = ((long long)c.L + ss2d::kFrontTile - 1) / ss2d::kFrontTile *
+                                (((long long)c.D + ss2d::kFrontCh - 1) / ss2d::kFrontCh) * c.B *
+                                c.K;
     if ((long long)c.L + 7 > INT_MAX || c.B > 65535 || (long long)c.K * c.D > INT_MAX ||
-        (long long)(c.L + ss2d::kFrontTile - 1) / ss2d::kFrontTile > 0x7fffffffLL)
+        conv_ctas > 0x7fffffffLL)
         return SS2D_ERR_SHAPE;
     return SS2D_OK;
 }
@@ -128,7 +132,7 @@ cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, flo
     const unsigned ntiles = (unsigned)((c.L + ss2d::kFrontTile - 1) / ss2d::kFrontTile);
     const unsigned nblk = (unsigned)((c.D + ss2d::kFrontCh - 1) / ss2d::kFrontCh);
     {
-        const dim3 grid(ntiles, nblk, (unsigned)(c.B * c.K));
+        const dim3 grid((unsigned)((long long)ntiles * nblk * c.B * c.K));
         switch (c.dtype) {
         case SS2D_BF16:
             ss2d::front_conv_kernel<__nv_bfloat16><<<grid, ss2d::kFrontConvThreads, 0, st>>>(fp);

@@ -243,8 +243,8 @@ __device__ __forceinline__ void cp_async_16b_zfill(uint32_t dst, const void *src
 constexpr int kFrontRows = kFrontTile + 3;   // input steps of a tile with the 3-step halo
 
 // conv + SiLU of one (128-step tile, 64-channel block, b * K + k): the bf16
-// A operand block and, unless p.utile, u for the scan.  grid (tiles,
-// channel blocks, B * K).
+// A operand block and, unless p.utile, u for the scan.  grid: tiles *
+// channel blocks * B * K CTAs in one dimension, the tile fastest.
 // The CTA first copies the tile's 131 input steps (3-step halo) of its 64
 // channels into shared memory (cp.async, 16-byte pieces, zeros outside the
 // sequence and past channel D - 1), so that all its loads are in flight at
@@ -262,7 +262,11 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
     constexpr int ROWB = kFrontCh * (int)sizeof(Tin);   // bytes of a staged row
     __shared__ __align__(16) unsigned char sx[kFrontRows * ROWB];
     const int tid = threadIdx.x;
-    const int tile = blockIdx.x, cb = blockIdx.y, bk = blockIdx.z;
+    const int ntiles = (p.L + kFrontTile - 1) / kFrontTile;
+    const int nblk = (p.D + kFrontCh - 1) / kFrontCh;
+    const int tile = (int)(blockIdx.x % (unsigned)ntiles);
+    const unsigned rest = blockIdx.x / (unsigned)ntiles;
+    const int cb = (int)(rest % (unsigned)nblk), bk = (int)(rest / (unsigned)nblk);
     const int b = bk / p.K, k = bk % p.K;
     const int D = p.D, L = p.L, LP = p.LP;
     const int lt = tile * kFrontTile;            // first step of the tile
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
     xrow(m0 + 1, win[1]);
     xrow(m0 + 2, win[2]);
     unsigned char *ab = static_cast<unsigned char *>(p.Ab) +
-                        (((size_t)bk * gridDim.x + tile) * gridDim.y + cb) * kFrontABytes +
+                        (((size_t)bk * ntiles + tile) * nblk + cb) * kFrontABytes +
                         (m0 >> 3) * kFrontSBO + c0 * 16;   // channel c0, steps m0..m0+7
     // per step: the A operand word (the pair in bf16, one packed conversion);
     // 2-byte inputs: the pair in the input dtype, whose halves are u's values

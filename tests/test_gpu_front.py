@@ -128,6 +128,21 @@ def test_front_deterministic():
     assert torch.equal(y1, y2)
 
 
+def test_front_more_sequences_than_one_grid_dimension():
+    # B * K = 66000 (b, direction) pairs: more than a grid's y or z dimension holds
+    B, L, D, N, K = 33000, 3, 2, 2, 2
+    a = make_front(B, L, D, N, K, wl.BF16, seed=36)
+    ref = oracle.front_scan(a["x"], a["conv_w"], a["conv_b"], a["W_x"], a["w_dt"], a["A_log"],
+                            a["Dskip"], a["delta_bias"], storage=STORAGE[wl.BF16],
+                            operand="bf16", threads=oracle.max_threads())
+    t = to_dev(a, wl.BF16)
+    y = binding.selective_scan_fwd_front(t["x"], t["conv_w"], t["conv_b"], t["W_x"], t["w_dt"],
+                                         t["A_log"], t["Dskip"], t["delta_bias"])
+    torch.cuda.synchronize()
+    assert binding.ss2d_check_waits() == 0
+    _gpu.assert_close(y.cpu().numpy().astype(np.float64), ref, wl.BF16, "front B*K > 65535")
+
+
 def test_front_rejects_bad_arguments():
     a = make_front(1, 64, 64, 4, 2, wl.F32, seed=34)
     t = to_dev(a, wl.F32)
