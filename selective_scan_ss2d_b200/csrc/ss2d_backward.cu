@@ -112,19 +112,22 @@ cudaError_t launch_backward(const BwdParams &p, int dtype, cudaStream_t st)
 cudaError_t launch_backward_reduce(const BwdParams &p, float *dBs, float *dCs, float *dA_log,
                                    float *dDskip, float *ddelta_bias, cudaStream_t st)
 {
-    const long long nbc = (long long)p.B * p.K * 2 * p.NS * p.L;
-    long long blocks = (nbc + 255) / 256;
+    const long long rows = (long long)p.B * p.K * 2 * p.NS;   // one CTA per dBs | dCs row
+    if (rows > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    const int vec = ((p.L & 3) == 0 && ((reinterpret_cast<uintptr_t>(dBs) |
+                                         reinterpret_cast<uintptr_t>(dCs) |
+                                         reinterpret_cast<uintptr_t>(p.bc_part)) & 15) == 0)
+                        ? 1
+                        : 0;
+    bwd_reduce_bc_kernel<<<(unsigned)rows, kReduceBcThreads, 0, st>>>(p.bc_part, dBs, dCs, p.G,
+                                                                     p.NS, p.L, vec);
+    const long long npr = (long long)p.K * p.D * (p.NS + 2);   // one warp each
+    long long blocks = (npr + kReduceParamThreads / 32 - 1) / (kReduceParamThreads / 32);
     if (blocks > 148LL * 64)
         blocks = 148LL * 64;
-    bwd_reduce_bc_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.bc_part, dBs, dCs, p.B * p.K, p.G,
-                                                          p.NS, p.L);
-    const long long npr = (long long)p.K * p.D * (p.NS + 2);
-    blocks = (npr + 127) / 128;
-    if (blocks > 148LL * 64)
-        blocks = 148LL * 64;
-    bwd_reduce_param_kernel<<<(unsigned)blocks, 128, 0, st>>>(p.prm_part, p.A_log, dA_log, dDskip,
-                                                             ddelta_bias, p.B, p.K, p.D, p.NS,
-                                                             p.CGN);
+    bwd_reduce_param_kernel<<<(unsigned)blocks, kReduceParamThreads, 0, st>>>(
+        p.prm_part, p.A_log, dA_log, dDskip, ddelta_bias, p.B, p.K, p.D, p.NS, p.CGN);
     return cudaGetLastError();
 }
 

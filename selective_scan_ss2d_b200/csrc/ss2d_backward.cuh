@@ -572,53 +572,77 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
 }
 
 // dBs, dCs (B,K,N,L) = the sum over the channel groups, in group order (the
-// partial holds N rows per (b, k, group, B|C))
-__global__ void bwd_reduce_bc_kernel(const float *__restrict__ part, float *__restrict__ dBs,
-                                     float *__restrict__ dCs, int BK, int G, int N, int L)
+// partial holds N rows per (b, k, group, B|C)).  One CTA per output row
+// r = (b * K + k) * 2N + which * N + n; vec: 16-byte pieces (L % 4 = 0).
+constexpr int kReduceBcThreads = 256;
+__global__ void __launch_bounds__(kReduceBcThreads)
+    bwd_reduce_bc_kernel(const float *__restrict__ part, float *__restrict__ dBs,
+                         float *__restrict__ dCs, int G, int N, int L, int vec)
 {
-    const long long total = (long long)BK * 2 * N * L;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int l = (int)(i % L);
-        long long r = i / L;
-        const int n = (int)(r % N);
-        r /= N;
-        const int which = (int)(r & 1);
-        const long long bk = r >> 1;
-        const float *src = part + (((size_t)bk * G * 2 + which) * N + n) * L + l;
-        const size_t gstride = (size_t)2 * N * L;
-        float s = 0.f;
-        for (int g = 0; g < G; ++g)
-            s += __ldg(src + g * gstride);
-        (which ? dCs : dBs)[((size_t)bk * N + n) * L + l] = s;
+    const unsigned r = blockIdx.x;
+    const int n = (int)(r % (unsigned)N);
+    const unsigned q = r / (unsigned)N;
+    const int which = (int)(q & 1u);
+    const size_t bk = q >> 1;
+    const float *src = part + ((bk * G * 2 + which) * N + n) * (size_t)L;
+    const size_t gstride = (size_t)2 * N * L;
+    float *dst = (which ? dCs : dBs) + (bk * N + n) * (size_t)L;
+    if (vec) {
+        const int n4 = L / 4;
+        for (int i = threadIdx.x; i < n4; i += kReduceBcThreads) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int g = 0; g < G; ++g) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(src + g * gstride) + i);
+                a = make_float4(a.x + v.x, a.y + v.y, a.z + v.z, a.w + v.w);
+            }
+            reinterpret_cast<float4 *>(dst)[i] = a;
+        }
+    } else {
+        for (int l = threadIdx.x; l < L; l += kReduceBcThreads) {
+            float a = 0.f;
+            for (int g = 0; g < G; ++g)
+                a += __ldg(src + g * gstride + l);
+            dst[l] = a;
+        }
     }
 }
 
-// dA_log = A * sum dA, dDskip, ddelta_bias: per (k, d), the sum over b and
-// the chunk groups, in that order
-__global__ void bwd_reduce_param_kernel(const float *__restrict__ prm,
-                                        const float *__restrict__ A_log, float *__restrict__ dA_log,
-                                        float *__restrict__ dDskip, float *__restrict__ dbias,
-                                        int B, int K, int D, int N, int CGN)
+// dA_log = A * sum dA, dDskip, ddelta_bias: per (k, d, j) one warp; lane t
+// sums b = t, t + 32, ... (each over the chunk groups in order), then the
+// lanes' sums meet in a fixed butterfly, so every call adds in the same order
+constexpr int kReduceParamThreads = 128;
+__global__ void __launch_bounds__(kReduceParamThreads)
+    bwd_reduce_param_kernel(const float *__restrict__ prm, const float *__restrict__ A_log,
+                            float *__restrict__ dA_log, float *__restrict__ dDskip,
+                            float *__restrict__ dbias, int B, int K, int D, int N, int CGN)
 {
     const long long total = (long long)K * D * (N + 2);
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (kReduceParamThreads / 32);
+    for (long long i = (long long)blockIdx.x * (kReduceParamThreads / 32) + (threadIdx.x >> 5);
+         i < total; i += warps) {
         const int j = (int)(i % (N + 2));
         const long long kd = i / (N + 2);
         const int k = (int)(kd / D), d = (int)(kd % D);
         float s = 0.f;
-        for (int b = 0; b < B; ++b) {
+        for (int b = lane; b < B; b += 32) {
             const float *src = prm + ((((size_t)b * K + k) * D + d) * CGN) * (N + 2) + j;
+            float t = 0.f;
             for (int cg = 0; cg < CGN; ++cg)
-                s += __ldg(src + (size_t)cg * (N + 2));
+                t += __ldg(src + (size_t)cg * (N + 2));
+            s += t;
         }
-        if (j < N)
-            dA_log[kd * N + j] = s * -expf(__ldg(A_log + kd * N + j));
-        else if (j == N)
-            dDskip[kd] = s;
-        else
-            dbias[kd] = s;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) {
+            if (j < N)
+                dA_log[kd * N + j] = s * -expf(__ldg(A_log + kd * N + j));
+            else if (j == N)
+                dDskip[kd] = s;
+            else
+                dbias[kd] = s;
+        }
     }
 }
 
