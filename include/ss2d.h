@@ -38,13 +38,19 @@
  * CUDA device, or managed memory) or a HOST pointer; all pointers of one call
  * must be of the same kind.
  *   - device pointers: the call is asynchronous on `stream` and returns after
- *     enqueueing.  Scratch for the per-direction partial outputs (K > 1,
- *     4*B*K*D*L bytes) and, when sequences are split into chunks, for the
+ *     enqueueing.  Scratch for the per-direction partial outputs (K = 4, or
+ *     K = 2 with N > 16: 4*B*K*D*L bytes) and, when sequences are split into chunks, for the
  *     chunk states (68*B*K*D*(chunks-1) bytes) is taken from a stream-ordered
  *     pool on `stream` and returned on `stream`.  Nothing is synchronised.
  *   - host pointers (pageable or pinned): the call copies the inputs to the
  *     current device, runs the device path, copies y back and synchronises
  *     `stream` before returning.  Device buffers come from the same pool.
+ *     With more than 16 MB of input the batch goes in slices of whole
+ *     elements (up to 8) through two copy streams of the library's own, so
+ *     that copies in, kernels and copies out overlap (pinned buffers are
+ *     needed for the overlap); every slice keeps the whole call's chunk
+ *     plan, so y is bit for bit the device path's.  The extra streams are
+ *     ordered after `stream`'s earlier work and joined back into it.
  * The caller owns every buffer; the library keeps no pointer after a call.
  * Inputs are never written.  y must not overlap any input.
  *

@@ -180,15 +180,17 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 //   K = 2 without a gate, at most 16 states: y is zeroed and both
 //   directions add into it in the output pass (no rows, no merge kernel).
 // Scratch comes from the pool on the stream and goes back to it on the stream.
+// plan_B: the batch size the chunk plan is made for (0: pr.B); a slice of a
+// larger call keeps the whole call's plan, so that it computes the same bits.
 int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
-               cudaEvent_t *ev = nullptr)
+               cudaEvent_t *ev = nullptr, int plan_B = 0)
 {
     if (ev && pr.N > ss2d::kNP)
         return SS2D_ERR_N;   // per-launch timing covers one state group
     ss2d::ScanParams p = make_params(pr);
     const size_t in_esz = pr.dtype == SS2D_F32 ? 4 : 2;   // bytes per stored input value
     const long long L = p.L;
-    const ss2d::Plan pl = ss2d::make_plan(variant, pr.B, pr.D, (int)L, pr.K);
+    const ss2d::Plan pl = ss2d::make_plan(variant, plan_B > 0 ? plan_B : pr.B, pr.D, (int)L, pr.K);
     // two directions, one state group, no gate: the output pass adds both into y
     const bool add_merge = pr.K == 2 && !pr.z && !directions && pr.N <= ss2d::kNP;
     const bool need_part = (pr.K > 1 || pr.z) && !add_merge;   // gated calls merge (the gate runs there)
@@ -244,23 +246,46 @@ int run_device(const Problem &pr, cudaStream_t st, int variant, bool directions,
     return SS2D_OK;
 }
 
-// Host path: copy in, run, copy out, synchronise.
-int run_host(const Problem &pr, cudaStream_t st, int variant)
-{
-    const size_t L = (size_t)pr.H * pr.W;
-    const size_t esz = pr.dtype == SS2D_F32 ? 4 : 2;
-    const size_t n_x = (size_t)pr.B * pr.D * L;
-    const size_t n_dl = (size_t)pr.B * pr.K * pr.D * L;
-    const size_t n_bc = (size_t)pr.B * pr.K * pr.N * L;
-    const size_t n_kd = (size_t)pr.K * pr.D;
-    auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
-    const size_t sz[8] = {n_x * esz, n_dl * esz, n_bc * esz, n_bc * esz,
-                          n_kd * pr.N * 4, n_kd * 4, n_kd * 4, n_x * 4};
-    size_t off[8], total = 0;
-    for (int i = 0; i < 8; ++i) {
-        off[i] = total;
-        total += up(sz[i]);
+// Host path: copy in, run, copy out, synchronise.  A batch of more than one
+// element is cut into slices of about kHostSliceBytes of input (at most
+// kHostSlices, whole batch elements) that flow through three streams: the
+// inputs of
+// slice s + 1 are copied in (one copy stream) while slice s is computed on
+// the caller's stream and slice s - 1 is copied out (a second copy stream),
+// so that the two copy directions and the kernels overlap.  Every slice runs
+// with the whole call's chunk plan: the result is bit for bit the device
+// path's.
+constexpr int kHostSlices = 8;
+constexpr size_t kHostSliceBytes = 16u << 20;   // smaller slices scan too few sequences
+
+struct HostStreams {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t ev[2 * kHostSlices + 2] = {};
+    int nev = 0;
+    cudaError_t create(int n)
+    {
+        cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
+        if (e == cudaSuccess)
+            e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
+        for (; nev < n && e == cudaSuccess; ++nev)
+            e = cudaEventCreateWithFlags(&ev[nev], cudaEventDisableTiming);
+        return e;
     }
+    ~HostStreams()
+    {
+        for (int i = 0; i < nev; ++i)
+            cudaEventDestroy(ev[i]);
+        if (in)
+            cudaStreamDestroy(in);
+        if (out)
+            cudaStreamDestroy(out);
+    }
+};
+
+// one element: copy in, run, copy out on the caller's stream
+int run_host_whole(const Problem &pr, cudaStream_t st, int variant, const size_t *sz,
+                   const size_t *off, size_t total)
+{
     void *buf = nullptr;
     int rc = pool_alloc(&buf, total, st);
     if (rc != SS2D_OK)
@@ -300,6 +325,112 @@ int run_host(const Problem &pr, cudaStream_t st, int variant)
         rc = SS2D_ERR_CUDA;
     }
     return rc;
+}
+
+int run_host(const Problem &pr, cudaStream_t st, int variant)
+{
+    const size_t L = (size_t)pr.H * pr.W;
+    const size_t esz = pr.dtype == SS2D_F32 ? 4 : 2;
+    // per batch element: x, delta, Bs, Cs, y
+    const size_t e_x = (size_t)pr.D * L, e_dl = (size_t)pr.K * pr.D * L;
+    const size_t e_bc = (size_t)pr.K * pr.N * L;
+    const size_t n_kd = (size_t)pr.K * pr.D;
+    auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    const size_t sz[8] = {pr.B * e_x * esz, pr.B * e_dl * esz, pr.B * e_bc * esz,
+                          pr.B * e_bc * esz, n_kd * pr.N * 4, n_kd * 4, n_kd * 4,
+                          pr.B * e_x * 4};
+    const size_t per_b[8] = {e_x * esz, e_dl * esz, e_bc * esz, e_bc * esz, 0, 0, 0, e_x * 4};
+    size_t off[8], total = 0;
+    for (int i = 0; i < 8; ++i) {
+        off[i] = total;
+        total += up(sz[i]);
+    }
+    const size_t in_bytes = sz[0] + sz[1] + sz[2] + sz[3];
+    long long want = (long long)((in_bytes + kHostSliceBytes - 1) / kHostSliceBytes);
+    want = want < 1 ? 1 : (want > kHostSlices ? kHostSlices : want);
+    const int nsl = pr.B < want ? pr.B : (int)want;
+    if (nsl == 1)
+        return run_host_whole(pr, st, variant, sz, off, total);
+    HostStreams hs;
+    cudaError_t e = hs.create(2 * nsl + 2);
+    if (e != cudaSuccess) {
+        set_error("cudaStreamCreate / cudaEventCreate", e);
+        return SS2D_ERR_CUDA;
+    }
+    cudaEvent_t ready = hs.ev[0], copied_out = hs.ev[1];
+    cudaEvent_t *in_done = hs.ev + 2, *computed = hs.ev + 2 + nsl;
+    void *buf = nullptr;
+    int rc = pool_alloc(&buf, total, st);
+    if (rc != SS2D_OK)
+        return rc;
+    char *base = static_cast<char *>(buf);
+    const void *src[7] = {pr.x, pr.delta, pr.Bs, pr.Cs, pr.A_log, pr.Dskip, pr.delta_bias};
+    // the copy streams start after everything before this call on `st` (the
+    // buffer's allocation included)
+    e = cudaEventRecord(ready, st);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(hs.in, ready, 0);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(hs.out, ready, 0);
+    for (int i = 4; i < 7 && e == cudaSuccess; ++i)   // the parameters, once
+        e = cudaMemcpyAsync(base + off[i], src[i], sz[i], cudaMemcpyHostToDevice, hs.in);
+    for (int s = 0; s < nsl && e == cudaSuccess && rc == SS2D_OK; ++s) {
+        const int b0 = (int)((long long)pr.B * s / nsl), b1 = (int)((long long)pr.B * (s + 1) / nsl);
+        for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+            e = cudaMemcpyAsync(base + off[i] + b0 * per_b[i],
+                                static_cast<const char *>(src[i]) + b0 * per_b[i],
+                                (size_t)(b1 - b0) * per_b[i], cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(in_done[s], hs.in);
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(st, in_done[s], 0);
+        if (e != cudaSuccess)
+            break;
+        Problem dp = pr;
+        dp.B = b1 - b0;
+        dp.x = base + off[0] + b0 * per_b[0];
+        dp.delta = base + off[1] + b0 * per_b[1];
+        dp.Bs = base + off[2] + b0 * per_b[2];
+        dp.Cs = base + off[3] + b0 * per_b[3];
+        dp.A_log = reinterpret_cast<const float *>(base + off[4]);
+        dp.Dskip = reinterpret_cast<const float *>(base + off[5]);
+        dp.delta_bias = reinterpret_cast<const float *>(base + off[6]);
+        dp.y = reinterpret_cast<float *>(base + off[7] + b0 * per_b[7]);
+        rc = run_device(dp, st, variant, false, nullptr, pr.B);
+        if (rc != SS2D_OK)
+            break;
+        e = cudaEventRecord(computed[s], st);
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(hs.out, computed[s], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<char *>(static_cast<void *>(pr.y)) + b0 * per_b[7],
+                                dp.y, (size_t)(b1 - b0) * per_b[7], cudaMemcpyDeviceToHost,
+                                hs.out);
+    }
+    // `st` waits for both copy streams before the buffer goes back to the pool
+    cudaError_t e2 = cudaEventRecord(copied_out, hs.out);
+    if (e2 == cudaSuccess)
+        e2 = cudaStreamWaitEvent(st, copied_out, 0);
+    cudaError_t e3 = cudaEventRecord(ready, hs.in);
+    if (e3 == cudaSuccess)
+        e3 = cudaStreamWaitEvent(st, ready, 0);
+    if (e2 == cudaSuccess && e3 == cudaSuccess)
+        cudaFreeAsync(buf, st);
+    const cudaError_t es = cudaStreamSynchronize(st);
+    if (e2 != cudaSuccess || e3 != cudaSuccess) {
+        // the streams could not be joined: wait for them before the buffer is freed
+        cudaStreamSynchronize(hs.in);
+        cudaStreamSynchronize(hs.out);
+        cudaFree(buf);
+    }
+    if (rc != SS2D_OK)
+        return rc;
+    const cudaError_t ef = e != cudaSuccess ? e : e2 != cudaSuccess ? e2 : e3 != cudaSuccess ? e3 : es;
+    if (ef != cudaSuccess) {
+        set_error("host-buffer call (copies, stream order)", ef);
+        return SS2D_ERR_CUDA;
+    }
+    return SS2D_OK;
 }
 
 int forward(const Problem &pr, void *stream, int variant, bool directions_only = false,

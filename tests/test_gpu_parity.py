@@ -162,6 +162,31 @@ def test_host_buffers_match_device(pin):
     assert np.array_equal(yh.numpy().astype(np.float64), yd)
 
 
+# the host path cuts a batch with more than 16 MB of input into slices
+# whose copies overlap the scans of the others; each slice keeps the whole
+# call's chunk plan, so the bits are the device path's: uneven slices,
+# chunked and unchunked, K = 4, K = 2 (added into y) and the 1D call
+@pytest.mark.parametrize("case", [
+    ("2d", 5, 128, 64, 64, 4, 16, wl.BF16),   # 30 MB: slices of 2 and 3 elements
+    ("2d", 3, 64, 96, 96, 4, 16, wl.F32),     # chunked rows, 3 slices of one
+    ("2d", 7, 256, 48, 48, 2, 8, wl.F16),     # K = 2: slices of 3 and 4
+    ("1d", 40, 768, 1, 197, 2, 16, wl.BF16),  # the 1D bidirectional call, 3 slices
+    ("1d", 6, 512, 1, 1100, 2, 33, wl.BF16),  # two state groups, chunked, 2 slices
+    ("2d", 3, 16, 10, 12, 4, 16, wl.BF16),    # under 16 MB: one piece
+], ids=lambda c: "{}_B{}_D{}_{}x{}_K{}_N{}_{}".format(*c))
+def test_host_slices_match_device(case):
+    kind, B, D, H, W, K, N, dt = case
+    cfg = (wl.Config(f"hs_{B}_{D}_{W}_{K}_{N}_{dt}", "1d", B, D, 1, W, K, N, dt) if kind == "1d"
+           else wl.Config(f"hs_{B}_{D}_{H}x{W}_{K}_{N}_{dt}", "2d", B, D, H, W, K, N, dt))
+    inp = wl.make_inputs(cfg, seed=11)
+    yd = _gpu.run_gpu(inp)
+    th = _gpu.tensors(inp, device=None, pin=True)
+    fn = binding.ss2d_forward if kind == "2d" else binding.selective_scan_fwd
+    yh = fn(th["x"], th["delta"], th["A_log"], th["Bs"], th["Cs"], th["Dskip"], th["delta_bias"])
+    assert not yh.is_cuda
+    assert np.array_equal(yh.numpy().astype(np.float64), yd)
+
+
 def test_mixed_pointers_rejected():
     inp = wl.make_inputs(small(B=1, D=4, H=4, W=4), seed=0)
     t = _gpu.tensors(inp)
