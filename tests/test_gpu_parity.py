@@ -263,6 +263,28 @@ def test_scan_directions_match_oracle(cfg):
         _gpu.assert_close(got, yd_ref, wl.F32, f"directions variant {v}")
 
 
+@pytest.mark.parametrize("cfg", [small(B=2, D=40, H=20, W=12, K=2, dtype=wl.BF16),
+                                 small("1d", B=3, D=70, W=197, K=2),
+                                 small("1d", B=1, D=33, W=1100, K=2, dtype=wl.BF16)],
+                         ids=lambda c: c.name)
+def test_two_directions_added_in_the_scan_equal_their_sum(cfg):
+    # K = 2 with N <= 16: the output pass adds both directions into y; two
+    # float32 terms meet in either order with the same bits, so y is exactly
+    # the float32 sum of the per-direction outputs
+    inp = wl.make_inputs(cfg, seed=12)
+    t = _gpu.tensors(inp)
+    lane = [i for i in range(nvariants()) if binding.ss2d_variant_name(i) == "lane2_wave"]
+    for v in [-1, 3, 5] + lane:
+        y = _gpu.run_gpu(inp, variant=v, t=t)
+        yd = binding.ss2d_scan_directions(t["x"], t["delta"], t["A_log"], t["Bs"], t["Cs"],
+                                          t["Dskip"], t["delta_bias"], two_d=cfg.kind == "2d",
+                                          variant=v)
+        torch.cuda.synchronize()
+        d = yd.cpu().numpy().reshape(cfg.B, cfg.K, cfg.D, cfg.L)
+        want = (d[:, 0] + d[:, 1]).astype(np.float32).reshape(inp.x.shape)
+        assert np.array_equal(y.astype(np.float32), want), f"variant {v}"
+
+
 def test_timed_call_matches_forward():
     cfg = small(B=2, D=70, H=24, W=40, K=4, dtype=wl.BF16)
     inp = wl.make_inputs(cfg, seed=9)
