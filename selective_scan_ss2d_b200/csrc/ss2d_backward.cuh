@@ -30,11 +30,14 @@
 //      the same 32 channels): per chunk of its range, in descending order
 //      (the walk back over a chunk ends with the adjoint entering the chunk
 //      below), each warp recomputes its states from the entry state and
-//      parks them in shared memory, then walks back from G[c] reducing
-//      dB | dC of its states over the channels (9 shuffles per step) and
-//      accumulating dA; the per-step sums over all 16 states that du and
-//      ddelta need are combined through shared memory once per chunk.
-//   4. merge2_kernel (K > 1) sums du of the directions into dx; two fixed-order
+//      parks them in shared memory, sums dC = dy h of its states over the
+//      channels from there, then walks back from G[c] accumulating dA and
+//      parking g dt u in the place of h, whose channel sums are dB; the
+//      per-step sums over all 16 states that du and ddelta need are
+//      combined through shared memory once per chunk.
+//   4. merge2_kernel (K = 4, or K = 2 with N > 16) sums du of the
+//      directions into dx (K = 2 otherwise: the final pass adds both into
+//      dx); two fixed-order
 //      reductions finish dBs, dCs and dA_log, dDskip, ddelta_bias.
 // Every reduction runs in a fixed order: the result is reproducible.
 #pragma once
@@ -93,8 +96,9 @@ __device__ __forceinline__ float2 row_pair(const float *row, int j)
 // ---------------------------------------------------------------------------
 // The final pass with the 16 states of a channel group split over 4 warps
 // (warp w: states 4w .. 4w+3 of the same 32 channels).  A warp parks the
-// states of a whole chunk (8 KB), so a chunk is recomputed once; dB | dC of
-// its 4 states reduce over the channels with 9 shuffles per step; the sums
+// states of a whole chunk (8 KB), so a chunk is recomputed once; dC and dB
+// of its 4 states are summed over the channels from that tile (lane_sums,
+// before and after the walk back); the sums
 // over all 16 states that du and ddelta need are combined through shared
 // memory once per chunk, each warp finishing 4 of the 16 steps.
 constexpr int kQuadWarps = 4;
@@ -105,32 +109,33 @@ constexpr int kBwd4Sums = kQuadWarps * kT * kBwdLanes * 2;       // per warp [t]
 constexpr int kBwd4Red = kQuadWarps * kT * 8;                    // per warp [t][8] reduced dB|dC
 constexpr size_t kBwd4Smem = sizeof(float) * (kBwd4Stage + kBwd4Hs + kBwd4Sums + kBwd4Red);
 
-// lanes with bit OFF set keep v[H..2H) (moved to v[0..H)), the others v[0..H)
-template <int H, int OFF>
-__device__ __forceinline__ void halve_at(float *v)
+// Sums over the warp's 32 channels of a [t][lane] float4 tile of 4 states
+// (hs): lane = 2 t + p sums states 2p, 2p + 1 of step t, times dy of the
+// channel (st4[.].z) when weighted, into red[t * 8 + base + 2p + {0, 1}].  The
+// lane starts at channel t and wraps around, so that the 16 steps read
+// different banks (8 distinct 16-byte bank groups, 2-way at most); the order
+// is fixed, so every call gives the same sums.
+__device__ __forceinline__ void lane_sums(const float4 *hs, const float4 *st4, float *red,
+                                          int lane, int base, bool weighted)
 {
-    const bool hi = (threadIdx.x & OFF) != 0;
-#pragma unroll
-    for (int i = 0; i < H; ++i) {
-        const float lo = v[i], up = v[i + H];
-        const float send = hi ? lo : up;
-        const float keep = hi ? up : lo;
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+    const int t = lane >> 1, p = lane & 1;
+    const float2 *row = reinterpret_cast<const float2 *>(hs + t * kBwdLanes) + p;
+    const float4 *dyrow = st4 + t * kBwdLanes;
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 8
+    for (int i = 0; i < kBwdLanes; ++i) {
+        const int l = (i + t) & (kBwdLanes - 1);
+        const float2 v = row[2 * l];
+        if (weighted) {
+            const float gy = dyrow[l].z;
+            acc.x = fmaf(gy, v.x, acc.x);
+            acc.y = fmaf(gy, v.y, acc.y);
+        } else {
+            acc.x += v.x;
+            acc.y += v.y;
+        }
     }
-}
-
-// Sum over the 32 lanes of v[j], j = (lane >> 2) (v[0..3]: dB, v[4..7]: dC of
-// the warp's 4 states): three halvings over lane bits 4, 3, 2, then a
-// butterfly over bits 1, 0; 9 shuffles.
-__device__ __forceinline__ float reduce_scatter8(float *v)
-{
-    halve_at<4, 16>(v);
-    halve_at<2, 8>(v);
-    halve_at<1, 4>(v);
-    float r = v[0];
-    r += __shfl_xor_sync(0xffffffffu, r, 2);
-    r += __shfl_xor_sync(0xffffffffu, r, 1);
-    return r;
+    *reinterpret_cast<float2 *>(red + t * 8 + base + 2 * p) = acc;
 }
 
 // The raw inputs of one chunk, the staging split over the CTA's 128 threads:
@@ -423,6 +428,11 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
                 hs[t * kBwdLanes + lane] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
             }
         }
+        // dC of the warp's 4 states at every step of the chunk: lane (t, pair)
+        // sums dy * h over the 32 channels
+        __syncwarp();
+        lane_sums(hs, st4, red, lane, 4, true);
+        __syncwarp();   // every lane is done with h before the walk back overwrites it
         if (c == c1 - 1) {   // the adjoint entering the range's top chunk at its end
             if (c < nc1) {
                 const float4 e = *reinterpret_cast<const float4 *>(
@@ -445,28 +455,26 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
             const float2 B2[2] = {make_float2(b4.x, b4.y), make_float2(b4.z, b4.w)};
             const float2 C2[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
             const float2 H2[2] = {make_float2(h4.x, h4.y), make_float2(h4.z, h4.w)};
-            float v[8];
+            float2 vb[2];
             float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 g[j] = __ffma2_rn(gy2, C2[j], g[j]);
                 const float2 hp = __ffma2_rn(ndtu2, B2[j], H2[j]);   // a_t h_{t-1}
-                const float2 vb = __fmul2_rn(g[j], dtu2);
-                const float2 vc = __fmul2_rn(gy2, H2[j]);
-                v[2 * j] = vb.x;
-                v[2 * j + 1] = vb.y;
-                v[4 + 2 * j] = vc.x;
-                v[4 + 2 * j + 1] = vc.y;
+                vb[j] = __fmul2_rn(g[j], dtu2);
                 s2 = __ffma2_rn(g[j], B2[j], s2);
                 s1 = __ffma2_rn(__fmul2_rn(g[j], A2[j]), hp, s1);
                 dA[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), hp, dA[j]);
                 g[j] = __fmul2_rn(g[j], ex2_pair(__fmul2_rn(dt2, A2[j])));
             }
-            const float r = reduce_scatter8(v);
-            if ((lane & 3) == 0)
-                red[t * 8 + (lane >> 2)] = r;
+            // g dt u of the 4 states, in the place of h_t (read above)
+            hs[t * kBwdLanes + lane] = make_float4(vb[0].x, vb[0].y, vb[1].x, vb[1].y);
             sums[(w * kT + t) * kBwdLanes + lane] = make_float2(s1.x + s1.y, s2.x + s2.y);
         }
+        // dB of the warp's 4 states at every step: lane (t, pair) sums g dt u
+        // over the 32 channels
+        __syncwarp();
+        lane_sums(hs, st4, red, lane, 0, false);
         __syncthreads();   // every warp's (s1, s2) of the chunk
         // warp w finishes steps 4w .. 4w+3 of its lanes' channels
         float ddv[4], duv[4];
