@@ -107,35 +107,46 @@ constexpr int kBwd4Stage = 2 * kT * kBCS + 4 * kT * kBwdLanes;   // B|C tiles, s
 constexpr int kBwd4Hs = kQuadWarps * kT * kBwdLanes * 4;         // per warp [t][lane] float4
 constexpr int kBwd4Sums = kQuadWarps * kT * kBwdLanes * 2;       // per warp [t][lane] (s1, s2)
 constexpr int kBwd4Red = kQuadWarps * kT * 8;                    // per warp [t][8] reduced dB|dC
-constexpr size_t kBwd4Smem = sizeof(float) * (kBwd4Stage + kBwd4Hs + kBwd4Sums + kBwd4Red);
+constexpr int kBwd4Dy = kT * kBwdLanes;                          // [t][lane] dy, 4-byte stride
+constexpr size_t kBwd4Smem =
+    sizeof(float) * (kBwd4Stage + kBwd4Hs + kBwd4Sums + kBwd4Red + kBwd4Dy);
 
-// Sums over the warp's 32 channels of a [t][lane] float4 tile of 4 states
-// (hs): lane = 2 t + p sums states 2p, 2p + 1 of step t, times dy of the
-// channel (st4[.].z) when weighted, into red[t * 8 + base + 2p + {0, 1}].  The
-// lane starts at channel t and wraps around, so that the 16 steps read
-// different banks (8 distinct 16-byte bank groups, 2-way at most); the order
-// is fixed, so every call gives the same sums.
-__device__ __forceinline__ void lane_sums(const float4 *hs, const float4 *st4, float *red,
+// Sums over the warp's 32 channels of a [t][lane] float4 tile of its 4
+// states (hs), times dy of the channel (sdy[t][lane]) when weighted: lane
+// 16 h + t sums channels 16 h .. 16 h + 15 of step t (16-byte loads, the
+// channel order rotated by t so that each quarter-warp reads 8 different
+// bank groups), then the two halves meet in one exchange: half h keeps
+// states 2h, 2h + 1 and writes them to red[t * 8 + base + 2h + {0, 1}].
+// The order is fixed, so every call gives the same sums.
+__device__ __forceinline__ void lane_sums(const float4 *hs, const float *sdy, float *red,
                                           int lane, int base, bool weighted)
 {
-    const int t = lane >> 1, p = lane & 1;
-    const float2 *row = reinterpret_cast<const float2 *>(hs + t * kBwdLanes) + p;
-    const float4 *dyrow = st4 + t * kBwdLanes;
-    float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-    for (int i = 0; i < kBwdLanes; ++i) {
-        const int l = (i + t) & (kBwdLanes - 1);
-        const float2 v = row[2 * l];
+    const int t = lane & 15, hf = lane >> 4;
+    const float4 *row = hs + t * kBwdLanes + 16 * hf;
+    const float *dyrow = sdy + t * kBwdLanes + 16 * hf;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int l = (i + t) & 15;
+        const float4 v = row[l];
         if (weighted) {
-            const float gy = dyrow[l].z;
+            const float gy = dyrow[l];
             acc.x = fmaf(gy, v.x, acc.x);
             acc.y = fmaf(gy, v.y, acc.y);
+            acc.z = fmaf(gy, v.z, acc.z);
+            acc.w = fmaf(gy, v.w, acc.w);
         } else {
             acc.x += v.x;
             acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
         }
     }
-    *reinterpret_cast<float2 *>(red + t * 8 + base + 2 * p) = acc;
+    const float s0 = hf ? acc.x : acc.z, s1 = hf ? acc.y : acc.w;   // the other half's states
+    const float k0 = hf ? acc.z : acc.x, k1 = hf ? acc.w : acc.y;   // this half's states
+    const float r0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 16);
+    const float r1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 16);
+    *reinterpret_cast<float2 *>(red + t * 8 + base + 2 * hf) = make_float2(r0, r1);
 }
 
 // The raw inputs of one chunk, the staging split over the CTA's 128 threads:
@@ -233,8 +244,9 @@ struct BwdRaw4 {
         }
     }
 
+    // sdy (optional): dy again as a [t][lane] row of floats
     __device__ __forceinline__ void commit(float *sB, float *sC, float4 *st4, float bias,
-                                           bool active) const
+                                           bool active, float *sdy = nullptr) const
     {
         const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
 #pragma unroll
@@ -255,6 +267,8 @@ struct BwdRaw4 {
                 v.w = __fdividef(1.f, 1.f + mufu_ex2(-z * kLog2e));   // sigmoid(z)
             }
             st4[t * kBwdLanes + lane] = v;
+            if (sdy)
+                sdy[t * kBwdLanes + lane] = v.z;
         }
     }
 };
@@ -367,6 +381,7 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
     float4 *hs = st4 + kT * kBwdLanes + w * kT * kBwdLanes;           // this warp's [t][lane]
     float2 *sums = reinterpret_cast<float2 *>(st4 + kT * kBwdLanes + kQuadWarps * kT * kBwdLanes);
     float *red = reinterpret_cast<float *>(sums + kQuadWarps * kT * kBwdLanes) + w * kT * 8;
+    float *sdy = reinterpret_cast<float *>(sums + kQuadWarps * kT * kBwdLanes) + kBwd4Red;
     const BwdLane q = bwd_lane(p);
     const size_t kd = (size_t)q.k * p.D + q.d;
     const int nw = 4 * w;   // this warp's first state within the group
@@ -401,7 +416,7 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
     for (int c = c1 - 1; c >= c0; --c) {
         const int s = c * kT, nt = min(kT, L - s);
         __syncthreads();   // every warp is done with the previous chunk's tiles
-        raw.commit(sB, sC, st4, bias, q.active);
+        raw.commit(sB, sC, st4, bias, q.active, sdy);
         __syncthreads();
         if (c - 1 >= c0)
             raw.fetch(p, q, (c - 1) * kT);   // in flight during this chunk's work
@@ -431,7 +446,7 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
         // dC of the warp's 4 states at every step of the chunk: lane (t, pair)
         // sums dy * h over the 32 channels
         __syncwarp();
-        lane_sums(hs, st4, red, lane, 4, true);
+        lane_sums(hs, sdy, red, lane, 4, true);
         __syncwarp();   // every lane is done with h before the walk back overwrites it
         if (c == c1 - 1) {   // the adjoint entering the range's top chunk at its end
             if (c < nc1) {
@@ -474,7 +489,7 @@ __global__ void __launch_bounds__(kBwd4Threads) bwd_final4_kernel(const BwdParam
         // dB of the warp's 4 states at every step: lane (t, pair) sums g dt u
         // over the 32 channels
         __syncwarp();
-        lane_sums(hs, st4, red, lane, 0, false);
+        lane_sums(hs, sdy, red, lane, 0, false);
         __syncthreads();   // every warp's (s1, s2) of the chunk
         // warp w finishes steps 4w .. 4w+3 of its lanes' channels
         float ddv[4], duv[4];
