@@ -323,8 +323,11 @@ int ss2d_forward_noalloc(const void *x, const void *delta, const float *A_log,
  * (as selective_scan_fwd, with A_log, Dskip, delta_bias rows k*D + d) and
  * y = Y_0 + Y_1 flipped back.  x_proj runs on the tensor cores (tcgen05)
  * with bfloat16 operands -- u and W_x rounded to nearest even -- and a
- * float32 accumulator; u is kept for the scan in the input dtype, dt_raw,
- * B and C in float32; no (D, L) delta array is ever written.
+ * float32 accumulator; u is kept for the scan in the input dtype (for
+ * bfloat16 input the x_proj operand blocks are that copy), dt_raw, B and C
+ * in float32; no (D, L) delta array is ever written.  K = 2 with N <= 16:
+ * y is zeroed and both directions add into it (two terms, the same bits in
+ * either order) instead of a merge launch.
  *
  * Layouts (contiguous, C order; all pointers DEVICE memory of the current
  * device, 16-byte aligned):
@@ -335,9 +338,11 @@ int ss2d_forward_noalloc(const void *x, const void *delta, const float *A_log,
  *   w_dt    (K, D)     float32  dt_proj weight
  *   A_log   (K*D, N), Dskip (K*D), delta_bias (K*D)  float32, as selective_scan_fwd
  *   y       (B, D, L)  float32, overwritten
- * K in {1, 2}, N in 1..64, dtype any ss2d_dtype.  Scratch (u, dt_raw, B, C
- * with rows padded to a multiple of 8 steps, and the scan's scratch) comes
- * from the stream-ordered pool on `stream`; asynchronous.  A tensor-core
+ * K in {1, 2}, N in 1..64, dtype any ss2d_dtype; B * K * ceil(L / 128) *
+ * ceil(D / 64) at most 2^31 - 1 (SS2D_ERR_SHAPE otherwise).  Scratch (u,
+ * dt_raw, B, C with rows padded to a multiple of 8 steps, the x_proj
+ * operand blocks, and the scan's scratch) comes from the stream-ordered
+ * pool on `stream`; asynchronous.  A tensor-core
  * completion wait that runs out of time (2 s) is recorded for
  * ss2d_check_waits(); the call's y is then not valid. */
 int selective_scan_fwd_front(const void *x, const float *conv_w, const float *conv_b,
