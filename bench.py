@@ -593,7 +593,7 @@ def run_front(args, rank, world, local_rank):
         "roofline_front_tensor": {"bound": "tensor", "achieved": tflops,
                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": tflops / peaks["bf16_tflops"],
-                                  "kernel": "front_wprep_kernel + front_conv_kernel + "
+                                  "kernel": "front_conv_kernel (with the W_x conversion) + "
                                             "front_proj_kernel (x_proj on tcgen05, bf16 operands)",
                                   "kernel_ms": front_ms, "flops_per_launch": flops,
                                   "peak_source": peaks["bf16_source"]},
@@ -613,9 +613,9 @@ def run_front(args, rank, world, local_rank):
                                   "frac": step_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
                          "algorithmic_bytes_per_step": step_bytes},
         "launch_ms": {"front": front_ms, "scan_passes": scan_ms, "cross_merge": merge_ms},
-        # three front kernels, then the front-mode scan's own launches (its
+        # two front kernels, then the front-mode scan's own launches (its
         # passes and the merge) under the lane kernel's plan
-        "gpu_launches": args.steps * (3 + front_scan_launches(cfg)),
+        "gpu_launches": args.steps * (2 + front_scan_launches(cfg)),
         "clocks": clocks,
     }
     return line

@@ -86,21 +86,13 @@ void *front_ab(void *ops, const FrontCall &c)
     return static_cast<char *>(ops) + up256_(front_wb_bytes(c.K, c.D, c.N));
 }
 
-// the front kernels for one call (W_x conversion, conv, x_proj); scratch
+// the front kernels for one call (conv with the W_x conversion, x_proj); scratch
 // rows of pitch LP, ops of front_op_bytes; utile: u only as the A blocks
 cudaError_t launch_front(const FrontCall &c, int LP, void *u, float *dt_raw, float *Bs,
                          float *Cs, void *ops, cudaStream_t st, bool utile)
 {
     void *Wb = ops;
     void *Ab = front_ab(ops, c);
-    {
-        const int nblk = (c.D + ss2d::kFrontCh - 1) / ss2d::kFrontCh;
-        ss2d::front_wprep_kernel<<<(unsigned)(c.K * nblk), 256, 0, st>>>(
-            c.W_x, static_cast<__nv_bfloat16 *>(Wb), c.D, 1 + 2 * c.N, front_nm(c.N), nblk);
-        const cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess)
-            return e;
-    }
     ss2d::FrontParams fp{};
     fp.Wb = Wb;
     fp.Ab = Ab;

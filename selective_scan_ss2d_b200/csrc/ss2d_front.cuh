@@ -23,11 +23,11 @@
 //     layout (one 16 KB block per tile and channel block).  For bf16 inputs
 //     of the fused call those blocks are the only copy of u: the scan reads
 //     its rows from them (p.utile).  Otherwise it also writes u for the scan,
-//     in the input dtype, as (B, K, D, LP) rows.
+//     in the input dtype, as (B, K, D, LP) rows.  The CTAs of the first tile
+//     of batch element 0 also convert W_x to the bf16 B operand blocks.
 //   front_proj_kernel: one CTA of 128 threads per (128-step tile, k, b).  One
 //     thread streams the tile's A blocks and the matching bf16 blocks of W_x
-//     (the B operand, converted once per call by front_wprep_kernel) into a
-//     ring of shared-memory stages with cp.async.bulk, each stage completing
+//     into a ring of shared-memory stages with cp.async.bulk, each stage completing
 //     an mbarrier (expected bytes), and issues the tcgen05.mma instructions
 //     (M = 128 steps, N = 1 + 2N rounded up to 16, K = 16 per instruction)
 //     that accumulate x_dbl in tensor memory; a tcgen05.commit frees each
@@ -199,15 +199,14 @@ __device__ __forceinline__ void cp_async_16b(uint32_t dst, const void *src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
 }
 
-// W_x (K, R, D) float32 -> Wb: for direction k and 64-channel block cb, the
-// NM x 64 bf16 B operand (rows >= R and channels >= D zero) in the layout
-// (r / 8) * 1024 + (c / 8) * 128 + (r % 8) * 16 + (c % 8) * 2.
-// grid: K * nblk CTAs.
-static __global__ void front_wprep_kernel(const float *W_x, __nv_bfloat16 *Wb, int D, int R,
-                                          int NM, int nblk)
+// W_x (K, R, D) float32 -> Wb, one block: for direction k and 64-channel
+// block cb, the NM x 64 bf16 B operand (rows >= R and channels >= D zero) in
+// the layout (r / 8) * 1024 + (c / 8) * 128 + (r % 8) * 16 + (c % 8) * 2, by
+// the calling CTA's threads.
+__device__ __forceinline__ void front_wprep_block(const float *W_x, __nv_bfloat16 *Wb, int D,
+                                                  int R, int NM, int k, int cb, int nblk)
 {
-    const int k = blockIdx.x / nblk, cb = blockIdx.x % nblk;
-    __nv_bfloat16 *dst = Wb + (size_t)blockIdx.x * NM * kFrontCh;
+    __nv_bfloat16 *dst = Wb + ((size_t)k * nblk + cb) * NM * kFrontCh;
     for (int i = threadIdx.x; i < NM * kFrontCh; i += blockDim.x) {
         const int r = i / kFrontCh, cc = i % kFrontCh, dd = cb * kFrontCh + cc;
         const float v = (r < R && dd < D) ? W_x[((size_t)k * R + r) * D + dd] : 0.f;
@@ -269,6 +268,11 @@ __global__ void __launch_bounds__(kFrontConvThreads) front_conv_kernel(const Fro
     const int cb = (int)(rest % (unsigned)nblk), bk = (int)(rest / (unsigned)nblk);
     const int b = bk / p.K, k = bk % p.K;
     const int D = p.D, L = p.L, LP = p.LP;
+    // the CTAs of the first tile of b = 0 also convert W_x's block (k, cb)
+    // for x_proj (which runs after this kernel on the stream)
+    if (tile == 0 && bk < p.K)
+        front_wprep_block(p.W_x, static_cast<__nv_bfloat16 *>(const_cast<void *>(p.Wb)), D,
+                          1 + 2 * p.N, p.NM, k, cb, nblk);
     const int lt = tile * kFrontTile;            // first step of the tile
     const int dblk = cb * kFrontCh;              // first channel of the block
     const Tin *xb = static_cast<const Tin *>(p.x) + (size_t)b * L * D;
