@@ -19,8 +19,10 @@
 //      an associative scan over the chunks of (exp(A_n * sum_c(dt)), h_end[c]);
 //   3. chunk_scan_kernel<..., kModeOutput>: every chunk from its true entry
 //      state, writing y_k in scan order (per-direction scratch, or y when
-//      K = 1);
-//   4. merge2_kernel (K > 1): y[p] = ((Y_0[s_0(p)] + Y_1[s_1(p)]) +
+//      K = 1; with K = 2 and one state group both directions add into a
+//      zeroed y with float atomic adds, and no merge runs: two terms give
+//      the same bits in either order);
+//   4. merge2_kernel (K > 1 otherwise): y[p] = ((Y_0[s_0(p)] + Y_1[s_1(p)]) +
 //      Y_2[s_2(p)]) + Y_3[s_3(p)], s_k the pixel -> scan-step map of
 //      direction k (cross_merge), always in that order.
 // Chunking costs one extra exp per update on the chunked workloads only,

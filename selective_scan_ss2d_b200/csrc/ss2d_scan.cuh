@@ -18,7 +18,8 @@
 //   * each lane copies its own delta row segment and its own x values: as
 //     packed 16- or 8-byte pieces of the row (rows whose start is aligned),
 //     or as one 4-byte word per step (the column-major directions, whose
-//     pixels are W apart, and rows that are only 2-byte aligned);
+//     pixels are W apart, and rows that are only 2-byte aligned); the fused
+//     front's bf16 u comes as 16-byte rows of its x_proj operand blocks;
 //   * B and C of the sub-chunk (shared by every channel of the CTA) are
 //     copied by the whole CTA two sub-chunks ahead, converted once to a
 //     float32 [slot][step] tile one sub-chunk ahead, and read with broadcast
@@ -145,7 +146,8 @@ struct LaneShape {
 // ALIGNED: delta, x and B|C rows start on 8-byte boundaries (p.vec = 8 or
 // 16): packed row copies; otherwise one word per step.
 // FRONT: the inputs of the fused front (p.front): u of every direction in
-// its scan order (B,K,D,LP), delta = w_dt * dt_raw, float32 B|C.
+// its scan order (B,K,D,LP) rows, or (p.utile) the x_proj A blocks, delta =
+// w_dt * dt_raw, float32 B|C.
 // CPL: channels per lane (channel c of thread t: tile * CPL*NT + c*NT + t);
 // the B|C values of a step, read from shared memory once, serve all of them.
 template <typename Tin, int WC, int MODE, int MINB, bool COLS, int QN, bool ALIGNED,
