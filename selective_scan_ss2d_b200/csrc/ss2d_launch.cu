@@ -84,6 +84,12 @@ int pick_variant(int two_d, int B, int D, int H, int W, int N, int K)
     // fuller warps hide the longer per-chunk dependency chains better)
     if (wants_chunks((long long)B * K * D, L))
         return variant_index("wc2_lcfit_r168");
+    // a handful of sequences of 64..512 steps (at most 1024 channels in all:
+    // a few warps on the whole GPU): 16-step chunks, so that the scan's
+    // latency is a chunk's and not a sequence's (B = 1, D = 8, 8 x 8, K = 4:
+    // 28.9 -> 23.2 us per call with the extra carry launch)
+    if ((long long)B * K * D <= 1024 && L >= 64 && L <= 512)
+        return variant_index("wc2_lc16");
     // SS2D (four directions, two column-major) unchunked: 64-channel CTAs at
     // 168 registers
     if (two_d && K == 4 && D % 64 == 0)
